@@ -1,0 +1,271 @@
+"""The oracle: a plain, slow CPU statement of MoE dispatch / combine.
+
+TEST INFRASTRUCTURE.  Only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg may import this package.  The product path
+(``combine_ep_dispatch_04_b200``) never imports it, and it never imports the
+product.  The arithmetic lives in ``ep_oracle.c``; this module only builds and
+loads it and marshals numpy arrays.
+
+Modes and layouts use the names of the product's enums, mapped here by value:
+bf16=0, e4m3_b128=1, int8_token=2, mxfp8=3, mxfp4=4; padded=0, packed=1.
+"""
+import ctypes as C
+
+import numpy as np
+
+from . import build as _build
+
+MODES = {"bf16": 0, "e4m3_b128": 1, "int8_token": 2, "mxfp8": 3, "mxfp4": 4}
+LAYOUTS = {"padded": 0, "packed": 1}
+ST_BAD_INDEX = 0x1
+ST_CAPACITY = 0x2
+
+_lib = C.CDLL(_build.build())
+
+_p = C.c_void_p
+_i = C.c_int
+_f = C.c_float
+_l = C.c_long
+
+_lib.orc_bf16_to_f32.restype = C.c_float
+_lib.orc_bf16_to_f32.argtypes = [C.c_uint16]
+_lib.orc_f32_to_bf16.restype = C.c_uint16
+_lib.orc_f32_to_bf16.argtypes = [C.c_float]
+_lib.orc_e4m3_encode.restype = C.c_uint8
+_lib.orc_e4m3_encode.argtypes = [C.c_float]
+_lib.orc_e2m1_encode.restype = C.c_uint8
+_lib.orc_e2m1_encode.argtypes = [C.c_float]
+_lib.orc_e4m3_decode.restype = C.c_float
+_lib.orc_e4m3_decode.argtypes = [C.c_uint8]
+_lib.orc_e2m1_decode.restype = C.c_float
+_lib.orc_e2m1_decode.argtypes = [C.c_uint8]
+_lib.orc_mx_exponent.restype = C.c_int
+_lib.orc_mx_exponent.argtypes = [C.c_float, C.c_float]
+_lib.orc_row_data_bytes.restype = C.c_long
+_lib.orc_row_data_bytes.argtypes = [_i, _i]
+_lib.orc_row_scale_bytes.restype = C.c_long
+_lib.orc_row_scale_bytes.argtypes = [_i, _i]
+_lib.orc_quant_row_f32.restype = None
+_lib.orc_quant_row_f32.argtypes = [_i, _i, _f, _p, _p, _p]
+_lib.orc_quant_row_bf16.restype = None
+_lib.orc_quant_row_bf16.argtypes = [_i, _i, _f, _p, _p, _p]
+_lib.orc_layout.restype = C.c_uint32
+_lib.orc_layout.argtypes = [_i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]
+_lib.orc_dispatch.restype = C.c_uint32
+_lib.orc_dispatch.argtypes = [_i, _i, _i, _i, _i, _i, _i, _f, _i, _p, _p, _p, _p, _p, _p, _p, _p, _p]
+_lib.orc_combine_row.restype = None
+_lib.orc_combine_row.argtypes = [_i, _i, _p, _p, _p, _p]
+_lib.orc_combine.restype = C.c_uint32
+_lib.orc_combine.argtypes = [_i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p]
+_lib.orc_combine_bwd.restype = C.c_uint32
+_lib.orc_combine_bwd.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]
+for _n in ("orc_e4m3_encode_array", "orc_e2m1_encode_array"):
+    getattr(_lib, _n).restype = None
+    getattr(_lib, _n).argtypes = [_p, _p, _l]
+for _n in ("orc_e4m3_encode_bits", "orc_e2m1_encode_bits"):
+    getattr(_lib, _n).restype = None
+    getattr(_lib, _n).argtypes = [C.c_uint32, _p, _l]
+_lib.orc_mx_exponent_array.restype = None
+_lib.orc_mx_exponent_array.argtypes = [_p, _f, _p, _l]
+_lib.orc_f32_to_bf16_array.restype = None
+_lib.orc_f32_to_bf16_array.argtypes = [_p, _p, _l]
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def _mode(m):
+    return MODES[m] if isinstance(m, str) else int(m)
+
+
+def _layout(l):
+    return LAYOUTS[l] if isinstance(l, str) else int(l)
+
+
+# ---- scalar formats -------------------------------------------------------
+
+def e4m3_encode(x):
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint8)
+    _lib.orc_e4m3_encode_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def e2m1_encode(x):
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint8)
+    _lib.orc_e2m1_encode_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def e4m3_encode_bits(start, n):
+    """Codes of the binary32 values whose bit patterns are start .. start+n-1."""
+    out = np.empty(n, np.uint8)
+    _lib.orc_e4m3_encode_bits(start, _ptr(out), n)
+    return out
+
+
+def e2m1_encode_bits(start, n):
+    out = np.empty(n, np.uint8)
+    _lib.orc_e2m1_encode_bits(start, _ptr(out), n)
+    return out
+
+
+def e4m3_decode(c):
+    return np.array([_lib.orc_e4m3_decode(int(v)) for v in np.ravel(c)], np.float32).reshape(np.shape(c))
+
+
+def e2m1_decode(c):
+    return np.array([_lib.orc_e2m1_decode(int(v)) for v in np.ravel(c)], np.float32).reshape(np.shape(c))
+
+
+def mx_exponent(amax, qmax):
+    a = _c(amax, np.float32)
+    out = np.empty(a.shape, np.int32)
+    _lib.orc_mx_exponent_array(_ptr(a), float(qmax), _ptr(out), a.size)
+    return out
+
+
+def f32_to_bf16(x):
+    x = _c(x, np.float32)
+    out = np.empty(x.shape, np.uint16)
+    _lib.orc_f32_to_bf16_array(_ptr(x), _ptr(out), x.size)
+    return out
+
+
+def bf16_to_f32(b):
+    return (_c(b, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+# ---- rows -----------------------------------------------------------------
+
+def row_bytes(mode, H):
+    """(data bytes, scale bytes) of one quantised row."""
+    m = _mode(mode)
+    return int(_lib.orc_row_data_bytes(m, H)), int(_lib.orc_row_scale_bytes(m, H))
+
+
+def quant_row(mode, x, e4m3_qmax=0.0):
+    """Quantise one row: bf16 bits (uint16) or fp32 values.  Returns (data, scale) bytes."""
+    m = _mode(mode)
+    H = int(np.size(x))
+    D, S = row_bytes(m, H)
+    data = np.zeros(D, np.uint8)
+    scale = np.zeros(max(S, 1), np.uint8)
+    if np.asarray(x).dtype == np.uint16:
+        xb = _c(x, np.uint16)
+        _lib.orc_quant_row_bf16(m, H, float(e4m3_qmax), _ptr(xb), _ptr(data), _ptr(scale))
+    else:
+        xf = _c(x, np.float32)
+        _lib.orc_quant_row_f32(m, H, float(e4m3_qmax), _ptr(xf), _ptr(data), _ptr(scale))
+    return data, scale[:S]
+
+
+def rows_max(R, T, K, E, M, layout, align=1):
+    """Rows a receive buffer must hold (padded: E*R*M; packed: every entry valid)."""
+    if _layout(layout) == 0:
+        return E * R * M
+    return R * T * K + E * (align - 1)
+
+
+def row_index(layout, R, M, e, slot, expert_offset=None):
+    """Row of (expert e, slot) in the receive layout (no validity check)."""
+    if _layout(layout) == 0:
+        return np.asarray(e, np.int64) * (R * M) + np.asarray(slot, np.int64)
+    return np.asarray(expert_offset, np.int64)[np.asarray(e, np.int64)] + np.asarray(slot, np.int64)
+
+
+# ---- the path -------------------------------------------------------------
+
+def layout(R, T, K, E, M, topk_idx, layout="padded", align=1):
+    idx = _c(topk_idx, np.int64).reshape(R * T, K)
+    N = R * T
+    out = dict(
+        tokens_per_rank=np.zeros((R, R), np.int32),
+        tokens_per_expert=np.zeros((R, E), np.int32),
+        is_token_in_rank=np.zeros((N, R), np.uint8),
+        token_slot=np.zeros((N, K), np.int32),
+        recv_count=np.zeros(E, np.int64),
+        expert_offset=np.zeros(E + 1, np.int64) if _layout(layout) == 1 else None,
+    )
+    st = _lib.orc_layout(R, T, K, E, M, _layout(layout), align, _ptr(idx),
+                         _ptr(out["tokens_per_rank"]), _ptr(out["tokens_per_expert"]),
+                         _ptr(out["is_token_in_rank"]), _ptr(out["token_slot"]),
+                         _ptr(out["recv_count"]), _ptr(out["expert_offset"]))
+    out["status"] = int(st)
+    return out
+
+
+def dispatch(R, T, K, E, M, H, mode, x, topk_idx, token_slot, expert_offset=None,
+             topk_weights=None, layout="padded", align=1, e4m3_qmax=0.0):
+    """Returns dict(recv_data [rows, D] u8, recv_scale [rows, S] u8, src_info, recv_weights, status).
+
+    Rows without an entry keep the fill value (0xAB bytes / -7 / nan) so that
+    tests can see that they were not written."""
+    m = _mode(mode)
+    rows = rows_max(R, T, K, E, M, layout, align)
+    D, S = row_bytes(m, H)
+    x = _c(x, np.uint16).reshape(R * T, H)
+    idx = _c(topk_idx, np.int64)
+    slot = _c(token_slot, np.int32)
+    eo = None if expert_offset is None else _c(expert_offset, np.int64)
+    w = None if topk_weights is None else _c(topk_weights, np.float32)
+    out = dict(
+        recv_data=np.full((rows, D), 0xAB, np.uint8),
+        recv_scale=np.full((rows, max(S, 1)), 0xAB, np.uint8),
+        src_info=np.full(rows, -7, np.int32),
+        recv_weights=np.full(rows, np.nan, np.float32) if w is not None else None,
+    )
+    st = _lib.orc_dispatch(R, T, K, E, M, H, m, float(e4m3_qmax), _layout(layout), _ptr(x),
+                           _ptr(idx), _ptr(w), _ptr(slot), _ptr(eo), _ptr(out["recv_data"]),
+                           _ptr(out["recv_scale"]), _ptr(out["src_info"]), _ptr(out["recv_weights"]))
+    out["recv_scale"] = out["recv_scale"][:, :S]
+    out["status"] = int(st)
+    return out
+
+
+def combine(R, T, K, E, M, H, y, topk_idx, topk_weights, token_slot, expert_offset=None,
+            layout="padded"):
+    """y: expert outputs, bf16 bits [rows, H] in the receive layout.  Returns (out [N, H] u16, status)."""
+    y = _c(y, np.uint16)
+    idx = _c(topk_idx, np.int64)
+    w = _c(topk_weights, np.float32)
+    slot = _c(token_slot, np.int32)
+    eo = None if expert_offset is None else _c(expert_offset, np.int64)
+    out = np.zeros((R * T, H), np.uint16)
+    st = _lib.orc_combine(R, T, K, E, M, H, _layout(layout), _ptr(y), _ptr(idx), _ptr(w),
+                          _ptr(slot), _ptr(eo), _ptr(out))
+    return out, int(st)
+
+
+def combine_row(yrows, w, valid):
+    """One token: yrows [K, H] bf16 bits, w [K] f32, valid [K] bool -> [H] bf16 bits."""
+    yrows = _c(yrows, np.uint16)
+    K, H = yrows.shape
+    ptrs = (C.c_void_p * K)(*[yrows.ctypes.data + k * H * 2 for k in range(K)])
+    w = _c(w, np.float32)
+    v = _c(valid, np.uint8)
+    out = np.zeros(H, np.uint16)
+    _lib.orc_combine_row(H, K, C.cast(ptrs, C.c_void_p), _ptr(w), _ptr(v), _ptr(out))
+    return out
+
+
+def combine_bwd(R, T, K, E, M, H, g, topk_idx, topk_weights, token_slot, expert_offset=None,
+                layout="padded", align=1, unweighted=False):
+    """Returns dict(grad_data [rows, H] u8, grad_scale [rows, H/32] u8, status)."""
+    rows = rows_max(R, T, K, E, M, layout, align)
+    g = _c(g, np.uint16).reshape(R * T, H)
+    idx = _c(topk_idx, np.int64)
+    w = _c(topk_weights, np.float32)
+    slot = _c(token_slot, np.int32)
+    eo = None if expert_offset is None else _c(expert_offset, np.int64)
+    gd = np.full((rows, H), 0xAB, np.uint8)
+    gs = np.full((rows, H // 32), 0xAB, np.uint8)
+    st = _lib.orc_combine_bwd(R, T, K, E, M, H, _layout(layout), int(bool(unweighted)), _ptr(g),
+                              _ptr(idx), _ptr(w), _ptr(slot), _ptr(eo), _ptr(gd), _ptr(gs))
+    return dict(grad_data=gd, grad_scale=gs, status=int(st))

@@ -1,0 +1,512 @@
+"""Pins for the oracle: each test checks the oracle against something other
+than itself -- brute force over tiny code tables and tiny routings, closed
+forms, library conversions (torch's float8 / bfloat16 casts), exact error
+bounds, and the routing table printed on "[feat] A5 deep fused moe
+supported" (Testing).  CPU only."""
+import itertools
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(12345)
+
+
+# ---------------------------------------------------------------------------
+# small-float encoders: brute force over the code tables written from the
+# OCP format definitions (independent of the oracle's rounding arithmetic)
+# ---------------------------------------------------------------------------
+
+def _e4m3_table():
+    vals = []
+    for c in range(0x7F):  # 0x7F is NaN
+        e, m = c >> 3, c & 7
+        vals.append(m * 2.0 ** -9 if e == 0 else (1 + m / 8) * 2.0 ** (e - 7))
+    return np.array(vals)
+
+
+def _e2m1_table():
+    return np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+
+
+def _brute_encode(x, table, sign_bit):
+    """Nearest table value, ties to the even code, beyond the top -> top."""
+    x = np.asarray(x, np.float64)
+    a = np.abs(x)
+    hi = np.clip(np.searchsorted(table, a), 1, len(table) - 1)
+    lo = hi - 1
+    dlo, dhi = a - table[lo], table[hi] - a
+    pick = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
+    pick = np.where(a >= table[-1], len(table) - 1, pick)
+    return (pick | np.where(np.signbit(x), sign_bit, 0)).astype(np.uint8)
+
+
+def _all_bf16_finite_f32():
+    b = np.arange(1 << 16, dtype=np.uint32) << 16
+    f = b.view(np.float32)
+    return f[np.isfinite(f)]
+
+
+def _midpoint_probe(table):
+    """Every midpoint between neighbouring codes, and its fp32 neighbours."""
+    mids = ((table[1:] + table[:-1]) / 2).astype(np.float32)
+    mids = np.concatenate([mids, np.float32([table[-1] * 1.0625, table[-1] * 1.5, 1e30])])
+    out = [mids]
+    for d in (1, 2):
+        out.append(np.nextafter(mids, np.float32(np.inf)))
+        out.append(np.nextafter(mids, np.float32(0)))
+        mids = out[-2]
+    v = np.concatenate(out)
+    return np.concatenate([v, -v])
+
+
+def _random_f32(n, lo_exp, hi_exp):
+    mag = 2.0 ** RNG.uniform(lo_exp, hi_exp, n)
+    sign = np.where(RNG.random(n) < 0.5, -1.0, 1.0)
+    return (mag * sign).astype(np.float32)
+
+
+@pytest.mark.parametrize("probe", ["bf16", "midpoints", "random"])
+def test_e4m3_encoder_matches_brute_force(probe):
+    table = _e4m3_table()
+    x = {"bf16": _all_bf16_finite_f32, "midpoints": lambda: _midpoint_probe(table),
+         "random": lambda: _random_f32(2_000_000, -14, 10)}[probe]()
+    got = oracle.e4m3_encode(x)
+    want = _brute_encode(x, table, 0x80)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (x[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def test_e4m3_encoder_matches_torch_float8_in_range():
+    # torch's float8_e4m3fn cast rounds to nearest even but does not saturate:
+    # compare where no saturation is involved (|x| < 464 rounds to <= 448).
+    x = np.concatenate([_all_bf16_finite_f32(), _random_f32(1_000_000, -12, 8.85)])
+    x = x[np.abs(x) < 464]
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = oracle.e4m3_encode(x)
+    assert np.array_equal(got, ref)
+
+
+def test_e4m3_nan_and_saturation():
+    got = oracle.e4m3_encode(np.float32([np.nan, 448, 449, 1e38, -1e38, np.inf, -np.inf, 0.0, -0.0]))
+    assert list(got) == [0x7F, 0x7E, 0x7E, 0x7E, 0xFE, 0x7E, 0xFE, 0x00, 0x80]
+
+
+@pytest.mark.parametrize("probe", ["bf16", "midpoints", "random"])
+def test_e2m1_encoder_matches_brute_force(probe):
+    table = _e2m1_table()
+    x = {"bf16": _all_bf16_finite_f32, "midpoints": lambda: _midpoint_probe(table),
+         "random": lambda: _random_f32(2_000_000, -4, 4)}[probe]()
+    got = oracle.e2m1_encode(x)
+    want = _brute_encode(x, table, 0x8)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (x[bad[:5]], got[bad[:5]], want[bad[:5]])
+
+
+def test_decoders_invert_encoders_on_every_code():
+    for c in range(256):
+        if c & 0x7F == 0x7F:
+            continue
+        v = oracle.e4m3_decode(np.uint8([c]))[0]
+        assert oracle.e4m3_encode(np.float32([v]))[0] == c
+    for c in range(16):
+        v = oracle.e2m1_decode(np.uint8([c]))[0]
+        assert oracle.e2m1_encode(np.float32([v]))[0] == c
+
+
+def test_bf16_rounding_matches_torch():
+    x = np.concatenate([_random_f32(1_000_000, -130, 127),
+                        # exact ties: low half 0x8000 with even and odd kept bit
+                        (np.arange(0, 1 << 16, 7, dtype=np.uint32) << 16 | 0x8000).view(np.float32)])
+    x = x[np.isfinite(x)]
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.f32_to_bf16(x), ref)
+
+
+# ---------------------------------------------------------------------------
+# e8m0 exponent: closed form 2^(X-1) < amax/qmax <= 2^X (exact in float64)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("qmax", [448.0, 6.0])
+def test_mx_exponent_is_ceil_log2(qmax):
+    amax = np.concatenate([
+        _random_f32(500_000, -140, 127), _all_bf16_finite_f32(),
+        (2.0 ** np.arange(-149, 120) * qmax).astype(np.float32)])
+    amax = np.abs(amax[np.isfinite(amax) & (amax != 0)]).astype(np.float32)
+    X = oracle.mx_exponent(amax, qmax).astype(np.int64)
+    v = (amax / np.float32(qmax)).astype(np.float64)  # the IEEE fp32 division, widened exactly
+    inside = (X > -127) & (X < 127) & (v > 0)
+    Xi = X[inside]
+    assert np.all(v[inside] <= np.ldexp(1.0, Xi))
+    assert np.all(v[inside] > np.ldexp(1.0, Xi - 1))
+    low = ~inside & (X == -127)
+    assert np.all((v[low] <= 2.0 ** -127))
+    assert oracle.mx_exponent(np.float32([0.0]), qmax)[0] == 0
+
+
+# ---------------------------------------------------------------------------
+# row quantisation: exact error bounds and the codes that must appear
+# ---------------------------------------------------------------------------
+
+def _bf16_row(n, scale=1.0, seed=0):
+    r = np.random.default_rng(seed)
+    return synth.to_bf16_bits((r.standard_normal(n) * scale).astype(np.float32))
+
+
+def _f(bits):
+    return oracle.bf16_to_f32(bits).astype(np.float64)
+
+
+def test_quant_bf16_is_a_copy():
+    x = _bf16_row(1024)
+    d, s = oracle.quant_row("bf16", x)
+    assert s.size == 0 and np.array_equal(d.view(np.uint16), x)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_quant_int8_token_bounds(seed):
+    H = 4096
+    x = _bf16_row(H, scale=10.0 ** (seed - 3), seed=seed)
+    if seed == 5:  # outlier channels, as in the skewed workload
+        f = oracle.bf16_to_f32(x).copy()
+        f[::97] *= 50
+        x = synth.to_bf16_bits(f)
+    d, s = oracle.quant_row("int8_token", x)
+    q = d.view(np.int8).astype(np.float64)
+    sinv = float(s.view(np.float32)[0])
+    xf = _f(x)
+    amax = np.abs(xf).max()
+    assert sinv == pytest.approx(amax / 127, rel=2 ** -23)
+    assert np.abs(q).max() == 127 and np.all(np.abs(q) <= 127)
+    # q = rint(fl(x * fl(127/amax))): within half a step plus two fp32 roundings
+    err = np.abs(xf - q * sinv)
+    assert np.all(err <= 0.5 * sinv * (1 + 2 ** -20) + np.abs(xf) * 2 ** -21)
+    # the element of largest magnitude maps to +-127 with its sign
+    i = int(np.argmax(np.abs(xf)))
+    assert q[i] == np.sign(xf[i]) * 127
+
+
+def _e4m3_elem_bound(v):
+    """|v - e4m3(v)| for |v| <= 448: half a code step (2^-4 relative in the
+    normal range, 2^-10 absolute among subnormals)."""
+    return np.maximum(np.abs(v) * 2.0 ** -4, 2.0 ** -10)
+
+
+@pytest.mark.parametrize("qmax", [448.0, 127.0])
+@pytest.mark.parametrize("seed", range(4))
+def test_quant_e4m3_b128_bounds(qmax, seed):
+    H = 7168
+    x = _bf16_row(H, scale=10.0 ** (seed - 2), seed=seed)
+    d, s = oracle.quant_row("e4m3_b128", x, e4m3_qmax=qmax)
+    sinv = s.view(np.float32).astype(np.float64)
+    dec = oracle.e4m3_decode(d).astype(np.float64).reshape(-1, 128)
+    xf = _f(x).reshape(-1, 128)
+    amax = np.abs(xf).max(axis=1)
+    assert np.allclose(sinv, amax / qmax, rtol=2 ** -23, atol=0)
+    v = xf * (qmax / amax)[:, None]          # the scaled values, exact in float64
+    assert np.all(np.abs(v - dec) <= _e4m3_elem_bound(v) * (1 + 2 ** -18) + np.abs(v) * 2 ** -22)
+    top = oracle.e4m3_encode(np.float32([qmax]))[0]
+    assert np.all(np.abs(d.reshape(-1, 128).view(np.int8) & 0x7F).max(axis=1) == top)
+
+
+@pytest.mark.parametrize("mode,qmax", [("mxfp8", 448.0), ("mxfp4", 6.0)])
+@pytest.mark.parametrize("seed", range(4))
+def test_quant_mx_bounds(mode, qmax, seed):
+    H = 7168
+    r = np.random.default_rng(seed)
+    f = (r.standard_t(3, H) * 0.5 * 10.0 ** (seed - 1)).astype(np.float32)
+    x = synth.to_bf16_bits(f)
+    d, s = oracle.quant_row(mode, x)
+    X = s.astype(np.int64) - 127
+    assert np.all((s != 255))
+    xf = _f(x).reshape(-1, 32)
+    amax = np.abs(xf).max(axis=1)
+    # ceil rule: amax * 2^-X lies in (qmax/2, qmax]
+    scaled_amax = amax * np.ldexp(1.0, -X)
+    assert np.all(scaled_amax <= qmax) and np.all(scaled_amax > qmax / 2)
+    if mode == "mxfp8":
+        dec = oracle.e4m3_decode(d).astype(np.float64).reshape(-1, 32)
+        v = xf * np.ldexp(1.0, -X)[:, None]
+        assert np.all(np.abs(v - dec) <= _e4m3_elem_bound(v))
+    else:
+        codes = np.stack([d & 0xF, d >> 4], axis=1).reshape(-1)  # element 2i = low nibble
+        dec = oracle.e2m1_decode(codes).astype(np.float64).reshape(-1, 32)
+        v = xf * np.ldexp(1.0, -X)[:, None]
+        step = np.where(np.abs(v) < 2, 0.5, np.where(np.abs(v) < 4, 1.0, 2.0))
+        assert np.all(np.abs(v - dec) <= step / 2)
+
+
+def test_mxfp4_block_worked_by_hand():
+    # A block whose amax is 6 has X = ceil(log2(6/6)) = 0, so the codes are the
+    # e2m1 grid itself: 0,.5,1,1.5,2,3,4,6 -> codes 0..7, negatives add 8.
+    vals = [0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.5, -1, -1.5, -2, -3, -4, -6, 0] * 2
+    x = synth.to_bf16_bits(np.float32(vals))
+    d, s = oracle.quant_row("mxfp4", x)
+    assert list(s) == [127]
+    codes = [0, 1, 2, 3, 4, 5, 6, 7, 9, 10, 11, 12, 13, 14, 15, 0] * 2
+    want = [codes[2 * i] | (codes[2 * i + 1] << 4) for i in range(16)]
+    assert list(d) == want
+    # doubling every value doubles the scale (X = 1) and keeps the codes
+    d2, s2 = oracle.quant_row("mxfp4", synth.to_bf16_bits(np.float32(vals) * 2))
+    assert list(s2) == [128] and np.array_equal(d2, d)
+
+
+def test_mxfp8_block_worked_by_hand():
+    # amax 448 -> X = 0: codes are the e4m3 encodings of the values themselves;
+    # amax 1 -> X = ceil(log2(1/448)) = -8, every value is scaled by 256.
+    vals = np.float32([448, -448, 1, -1, 0.5, 2 ** -9, 0, 3] + [0] * 24)
+    d, s = oracle.quant_row("mxfp8", synth.to_bf16_bits(vals))
+    assert list(s) == [127]
+    assert list(d[:8]) == [0x7E, 0xFE, 0x38, 0xB8, 0x30, 0x01, 0x00, 0x44]
+    d, s = oracle.quant_row("mxfp8", synth.to_bf16_bits(np.float32([1, -0.25] + [0] * 30)))
+    assert list(s) == [127 - 8]
+    assert list(d[:2]) == list(oracle.e4m3_encode(np.float32([256, -64])))
+
+
+def test_zero_rows_use_unit_scale():
+    x = np.zeros(256, np.uint16)
+    d, s = oracle.quant_row("int8_token", x)
+    assert not d.any() and s.view(np.float32)[0] == 1.0
+    d, s = oracle.quant_row("e4m3_b128", x)
+    assert not d.any() and np.all(s.view(np.float32) == 1.0)
+    for m in ("mxfp8", "mxfp4"):
+        d, s = oracle.quant_row(m, x)
+        assert not d.any() and np.all(s == 127)
+
+
+# ---------------------------------------------------------------------------
+# layout: brute force over every routing of tiny shapes, closed forms
+# ---------------------------------------------------------------------------
+
+def _layout_by_definition(R, T, K, E, M, idx, align):
+    """Counts straight from the definitions, one question per output."""
+    N, L = R * T, E // R
+    flat = [(n, k, int(idx[n][k])) for n in range(N) for k in range(K)]
+    valid = lambda e: 0 <= e < E
+    slot = np.full((N, K), -1, np.int64)
+    for i, (n, k, e) in enumerate(flat):
+        if valid(e):
+            slot[n, k] = sum(1 for (_, _, e2) in flat[:i] if e2 == e)
+    recv = np.array([sum(1 for (_, _, e2) in flat if e2 == e) for e in range(E)], dtype=np.int64)
+    itr = np.array([[int(any(valid(e) and e // L == d for e in idx[n])) for d in range(R)]
+                    for n in range(N)], dtype=np.int64).reshape(N, R)
+    tpe = np.array([[sum(1 for t in range(T) for e in idx[r * T + t] if e == x) for x in range(E)]
+                    for r in range(R)], dtype=np.int64).reshape(R, E)
+    tpr = np.array([[itr[r * T:(r + 1) * T, d].sum() for d in range(R)] for r in range(R)])
+    rounded = (recv + align - 1) // align * align
+    eo = np.concatenate([[0], np.cumsum(rounded)])
+    return slot, recv, itr, tpe, tpr, eo
+
+
+def _check_layout(R, T, K, E, M, idx, align=1):
+    idx = np.asarray(idx, np.int64).reshape(R * T, K)
+    got = oracle.layout(R, T, K, E, M, idx, layout="packed", align=align)
+    slot, recv, itr, tpe, tpr, eo = _layout_by_definition(R, T, K, E, M, idx, align)
+    assert np.array_equal(got["token_slot"], slot)
+    assert np.array_equal(got["recv_count"], recv)
+    assert np.array_equal(got["is_token_in_rank"], itr)
+    assert np.array_equal(got["tokens_per_expert"], tpe)
+    assert np.array_equal(got["tokens_per_rank"], tpr)
+    assert np.array_equal(got["expert_offset"], eo)
+    bad = bool(((idx < -1) | (idx >= E)).any())
+    assert bool(got["status"] & oracle.ST_BAD_INDEX) == bad
+
+
+@pytest.mark.parametrize("R,T,K,E", [(1, 2, 2, 2), (2, 1, 2, 2), (2, 2, 1, 4), (1, 3, 2, 2),
+                                     (2, 1, 3, 2)])
+def test_layout_every_routing_of_tiny_shapes(R, T, K, E):
+    values = list(range(-1, E))
+    for combo in itertools.product(values, repeat=R * T * K):
+        _check_layout(R, T, K, E, T, combo, align=1 + (sum(combo) % 3))
+
+
+def test_layout_random_small_routings_with_bad_indices():
+    r = np.random.default_rng(7)
+    for _ in range(300):
+        R = int(r.integers(1, 4))
+        L = int(r.integers(1, 4))
+        E, T, K = R * L, int(r.integers(0, 5)), int(r.integers(1, 4))
+        idx = r.integers(-3, E + 2, size=(R * T, K))
+        _check_layout(R, T, K, E, max(T, 1), idx, align=int(r.integers(1, 5)))
+
+
+def test_layout_a5_worked_example():
+    """The Ascend 950 table: 8 ranks x 8 local experts, 24 rows each, 192 per rank."""
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "a5_950_fused_counts.txt"))
+            if l.strip() and not l.startswith("#")]
+    want = np.array([[int(c) for c in r[2].split(",")] for r in rows])
+    sums = np.array([int(r[3]) for r in rows])
+    R, T, K, E = 8, 32, 6, 64
+    n = np.arange(R * T)[:, None]
+    idx = (n * K + np.arange(K)[None, :]) % E
+    got = oracle.layout(R, T, K, E, T, idx)
+    per_rank = got["recv_count"].reshape(R, E // R)
+    assert np.array_equal(per_rank, want)
+    assert np.array_equal(per_rank.sum(axis=1), sums)
+    assert got["status"] == 0
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_layout_invariants_on_workload_routing(name):
+    w = synth.workload(name)
+    if w["N"] > 20000:
+        w = synth.workload(name, T=max(1, 20000 // w["R"]))
+    idx, _ = synth.make_routing(w)
+    got = oracle.layout(w["R"], w["T"], w["K"], w["E"], w["M"], idx, layout=w["layout"])
+    valid = (idx >= 0) & (idx < w["E"])
+    assert got["recv_count"].sum() == valid.sum()
+    assert np.array_equal(got["tokens_per_expert"].sum(axis=0), got["recv_count"])
+    # each expert's slots are exactly 0 .. count-1, in (token, k) order
+    s = got["token_slot"]
+    for e in range(w["E"]):
+        sel = np.nonzero(idx.reshape(-1) == e)[0]
+        assert np.array_equal(s.reshape(-1)[sel], np.arange(sel.size))
+    # a token with at least one expert is in at least one rank
+    assert np.array_equal(got["is_token_in_rank"].any(axis=1), valid.any(axis=1))
+
+
+def test_layout_capacity_overflow_flag():
+    # duplicates inside a token can exceed cap = R*M in the padded layout
+    R, T, K, E, M = 1, 2, 3, 2, 2
+    idx = np.zeros((2, 3), np.int64)
+    got = oracle.layout(R, T, K, E, M, idx, layout="padded")
+    assert got["status"] & oracle.ST_CAPACITY
+    assert list(got["token_slot"].reshape(-1)) == [0, 1, 2, 3, 4, 5]
+
+
+# ---------------------------------------------------------------------------
+# dispatch / combine / combine-backward
+# ---------------------------------------------------------------------------
+
+def _small(name, **kw):
+    w = synth.workload(name, **kw)
+    idx, wt = synth.make_routing(w)
+    x = synth.make_x(w)
+    return w, idx, wt, x
+
+
+def _run_layout(w, idx, layout, align=1):
+    return oracle.layout(w["R"], w["T"], w["K"], w["E"], w["M"], idx, layout=layout, align=align)
+
+
+@pytest.mark.parametrize("layout,align", [("padded", 1), ("packed", 1), ("packed", 8)])
+def test_dispatch_bf16_is_an_exact_scatter(layout, align):
+    w, idx, wt, x = _small("tiny")
+    lay = _run_layout(w, idx, layout, align)
+    out = oracle.dispatch(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], "bf16", x, idx,
+                          lay["token_slot"], lay["expert_offset"], topk_weights=wt,
+                          layout=layout, align=align)
+    rows_seen = np.zeros(out["recv_data"].shape[0], bool)
+    for n in range(w["N"]):
+        for k in range(w["K"]):
+            e = idx[n, k]
+            if e < 0:
+                continue
+            row = int(oracle.row_index(layout, w["R"], w["M"], e, lay["token_slot"][n, k],
+                                       lay["expert_offset"]))
+            rows_seen[row] = True
+            assert np.array_equal(out["recv_data"][row].view(np.uint16), x[n])
+            assert out["src_info"][row] == (n // w["T"]) * w["M"] + n % w["T"]
+            assert out["recv_weights"][row] == wt[n, k]
+    assert np.all(out["recv_data"][~rows_seen] == 0xAB)
+    assert rows_seen.sum() == (idx >= 0).sum()
+
+
+def test_combine_one_hot_identity_reproduces_x():
+    w, idx, wt, x = _small("tiny")
+    lay = _run_layout(w, idx, "padded")
+    d = oracle.dispatch(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], "bf16", x, idx,
+                        lay["token_slot"])
+    y = d["recv_data"].view(np.uint16)  # identity experts
+    valid = idx >= 0
+    first = np.argmax(valid, axis=1)
+    onehot = np.zeros_like(wt)
+    onehot[np.arange(w["N"]), first] = 1.0
+    out, st = oracle.combine(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], y, idx, onehot,
+                             lay["token_slot"])
+    has = valid.any(axis=1)
+    assert st == 0
+    assert np.array_equal(out[has], x[has])
+    assert not out[~has].any()  # all-masked tokens give +0
+
+
+def test_combine_equal_weights_identical_rows_is_exact():
+    # K = 8 rows all equal to x, weights 1/8: every fma is exact, so the sum is x.
+    H, K = 256, 8
+    x = _bf16_row(H, seed=3)
+    yrows = np.tile(x, (K, 1))
+    out = oracle.combine_row(yrows, np.full(K, 0.125, np.float32), np.ones(K, np.uint8))
+    assert np.array_equal(out, x)
+    # and with weights 0.5 on two valid rows out of 8
+    v = np.zeros(K, np.uint8)
+    v[[2, 5]] = 1
+    out = oracle.combine_row(yrows, np.full(K, 0.5, np.float32), v)
+    assert np.array_equal(out, x)
+
+
+def _bf16_ulp_distance(a, b):
+    """Distance in bf16 ulps between two arrays of bf16 bits (monotone integer map)."""
+    def key(u):
+        u = u.astype(np.int64)
+        return np.where(u & 0x8000, -(u & 0x7FFF), u)
+    return np.abs(key(a) - key(b))
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_combine_within_one_ulp_of_float64_sum(seed):
+    r = np.random.default_rng(seed)
+    H, K = 2048, 8
+    yrows = synth.to_bf16_bits(r.standard_normal((K, H)).astype(np.float32))
+    wts = r.random(K).astype(np.float32)
+    valid = (r.random(K) < 0.8).astype(np.uint8)
+    out = oracle.combine_row(yrows, wts, valid)
+    exact = (wts.astype(np.float64)[:, None] * oracle.bf16_to_f32(yrows) * valid[:, None]).sum(0)
+    want = synth.to_bf16_bits(exact.astype(np.float32))  # float64 -> nearest fp32 -> bf16
+    assert _bf16_ulp_distance(out, want).max() <= 1
+
+
+def test_combine_backward_unweighted_equals_mxfp8_dispatch():
+    w = synth.workload("prefill", R=4, T=24, E=32)
+    idx, wt = synth.make_routing(w)
+    pool, off = synth.g_source(w)
+    g = synth.windows(pool, off, w["H"])
+    lay = _run_layout(w, idx, "packed")
+    args = (w["R"], w["T"], w["K"], w["E"], w["M"], w["H"])
+    bwd = oracle.combine_bwd(*args, g, idx, wt, lay["token_slot"], lay["expert_offset"],
+                             layout="packed", unweighted=True)
+    dis = oracle.dispatch(*args, "mxfp8", g, idx, lay["token_slot"], lay["expert_offset"],
+                          layout="packed")
+    rows = lay["expert_offset"][-1]
+    assert np.array_equal(bwd["grad_data"][:rows], dis["recv_data"][:rows])
+    assert np.array_equal(bwd["grad_scale"][:rows], dis["recv_scale"][:rows])
+
+
+def test_combine_backward_weighted_rows():
+    w = synth.workload("prefill", R=2, T=16, E=16, H=256)
+    idx, wt = synth.make_routing(w)
+    pool, off = synth.g_source(w)
+    g = synth.windows(pool, off, w["H"])
+    lay = _run_layout(w, idx, "packed")
+    bwd = oracle.combine_bwd(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], g, idx, wt,
+                             lay["token_slot"], lay["expert_offset"], layout="packed")
+    gf = oracle.bf16_to_f32(g)
+    for n in range(w["N"]):
+        for k in range(w["K"]):
+            if idx[n, k] < 0:
+                continue
+            row = lay["expert_offset"][idx[n, k]] + lay["token_slot"][n, k]
+            p = (np.float32(wt[n, k]) * gf[n]).astype(np.float32)  # one fp32 multiply each
+            d, s = oracle.quant_row("mxfp8", p)
+            assert np.array_equal(bwd["grad_data"][row], d)
+            assert np.array_equal(bwd["grad_scale"][row], s)
+            # dequantised grad is w * g within the e4m3 step
+            X = s.astype(np.int64) - 127
+            dec = oracle.e4m3_decode(d).astype(np.float64).reshape(-1, 32) * np.ldexp(1.0, X)[:, None]
+            ref = p.astype(np.float64).reshape(-1, 32)
+            assert np.all(np.abs(dec - ref) <= np.maximum(np.abs(ref) * 2 ** -4,
+                                                          np.ldexp(2.0 ** -10, X)[:, None]))
