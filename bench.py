@@ -1,0 +1,533 @@
+#!/usr/bin/env python
+"""Benchmark of MoE expert-parallel dispatch + combine on B200.
+
+One step = the whole hot path over one batch: routing layout, quantise +
+scatter (dispatch), weighted combine (and combine-backward for the prefill
+workload).  Default workload: decode (R=8 logical ranks x T=128 tokens,
+H=7168, top-8 of 256 experts, M=128, per-128-channel e4m3 dispatch, padded
+receive layout), on one GPU.
+
+Timing: CUDA events on the stream the kernels run on, one pair per kernel per
+step; a 512 MiB write flushes L2 between steps, outside the step's events.
+The K timed steps are bracketed by a barrier and a synchronize on both sides;
+the reported time is the max over ranks.  With --gpus N > 1 (torchrun), each
+rank runs an independent replica of the workload (different seed): the path
+has no exchange step on one GPU, so no collective is added ("weak" scaling).
+
+  python bench.py [--steps K] [--warmup W] [--workload decode] [--impl reference]
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
+FALLBACK_HBM_GBS = 6650.0
+WORKLOAD_MODE = {"tiny": "int8_token", "decode": "e4m3_b128", "skewed": "int8_token",
+                 "prefill": "mxfp8", "large": "mxfp4"}
+KERNEL_SOURCES = ["combine_ep_dispatch_04_b200/csrc/" + f for f in
+                  ("ep_api.cu", "ep_device.cuh", "ep_layout.cuh", "ep_dispatch.cuh", "ep_combine.cuh")]
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=300)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--workload", default="decode", choices=sorted(synth.WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--flush-mib", type=int, default=512)
+    p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes (what the method must move; unwritten capacity not counted)
+# ---------------------------------------------------------------------------
+def algorithmic_bytes(w, mode, idx):
+    """Bytes per launch of each kernel, from the per-token counts."""
+    import oracle
+
+    N, K, H, R = w["N"], w["K"], w["H"], w["R"]
+    D, S = oracle.row_bytes(mode, H)
+    v = int(((idx >= 0) & (idx < w["E"])).sum())
+    out = {
+        "layout": N * (8 * K + 4 * K + R),
+        "dispatch": N * (2 * H + 8 * K + 4 * K) + v * (D + S + 4),
+        "combine": v * 2 * H + N * (8 * K + 4 * K + 4 * K + 2 * H),
+    }
+    if w.get("backward"):
+        out["combine_bwd"] = N * (2 * H + 4 * K + 4 * K + 8 * K) + v * (H + H // 32)
+    return out, v
+
+
+def source_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return json.load(f)
+    except (OSError, ValueError):
+        return None
+
+
+def ncu_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    e = t.get(workload, {}).get(kernel)
+    if not e or e.get("source_hash") != source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ---------------------------------------------------------------------------
+REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+           0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+           0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+           0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, device_index):
+        self.samples, self.reasons, self.ok = [], 0, False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(device_index)
+            h = None
+            uuid = getattr(props, "uuid", None)
+            if uuid is not None:
+                try:
+                    h = pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(uuid))
+                except Exception:
+                    h = None
+            if h is None:
+                h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.nv, self.h = pynvml, h
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as exc:  # no NVML: report what is known
+            self.err = str(exc)
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(0.005)
+
+    def sample(self):
+        try:
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            self.samples.append(mhz)
+            self.reasons |= int(r)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self.ok:
+            self.sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self.sample()
+
+    def report(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvml unavailable"]}
+        names = [n for b, n in REASONS.items() if self.reasons & b and b != 0x1]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (replicas; no data-path collective)
+# ---------------------------------------------------------------------------
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(value, world):
+    """Max of a float over ranks (the timed duration)."""
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_done(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# the oracle as the CPU baseline / reference arm
+# ---------------------------------------------------------------------------
+class OracleStep:
+    """The oracle (plain single-threaded C) running one step of the workload --
+    layout, dispatch and combine -- on a bounded sample: the first `sub_t`
+    tokens of every source rank (same ranks, experts, capacity and hidden
+    size).  Inputs and output arrays are built before timing; only rows that
+    hold entries are ever touched."""
+
+    def __init__(self, w, mode, idx, wts, x, sub_t, replica=0):
+        import oracle
+        self.o, self.mode = oracle, mode
+        R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
+        sub_t = max(1, min(sub_t, T))
+        take = (np.arange(R)[:, None] * T + np.arange(sub_t)[None, :]).reshape(-1)
+        self.w = synth.workload(w["name"], T=sub_t)
+        self.idx, self.wts, self.x = idx[take], wts[take], x[take]
+        self.n = take.size
+        lay = oracle.layout(R, sub_t, K, E, M, self.idx, layout=w["layout"])
+        rows = oracle.rows_max(R, sub_t, K, E, M, w["layout"])
+        self.bufs = oracle.dispatch_buffers(R, sub_t, K, E, M, H, mode, w["layout"], fill=False)
+        self.y = np.zeros((rows, H), np.uint16)   # pages of rows never read stay unmapped
+        pool, off = synth.y_source(w, rows, replica)
+        used = (self.idx >= 0) & (self.idx < E)
+        r_used = oracle.row_index(w["layout"], R, M, self.idx[used], lay["token_slot"][used],
+                                  lay["expert_offset"])
+        for r in np.asarray(r_used).tolist():
+            self.y[r] = pool[off[r]: off[r] + H]
+        self.out = np.empty((self.n, H), np.uint16)
+        self.sample = (f"first {sub_t} of {T} tokens of each of the {R} ranks "
+                       f"({self.n} tokens): layout, dispatch and combine per step")
+
+    def step(self):
+        o, w = self.o, self.w
+        R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
+        lay = o.layout(R, T, K, E, M, self.idx, layout=w["layout"])
+        o.dispatch(R, T, K, E, M, H, self.mode, self.x, self.idx, lay["token_slot"],
+                   lay["expert_offset"], layout=w["layout"], out=self.bufs)
+        o.combine(R, T, K, E, M, H, self.y, self.idx, self.wts, lay["token_slot"],
+                  lay["expert_offset"], layout=w["layout"], out=self.out)
+        return self.n
+
+
+def cpu_baseline(w, mode, idx, wts, x, seconds, replica=0):
+    st = OracleStep(w, mode, idx, wts, x, sub_t=w["T"], replica=replica)
+    st.step()
+    t0 = time.perf_counter()
+    done, reps = 0, 0
+    while True:
+        done += st.step()
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": done / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{st.sample}; {reps} steps in {el:.1f} s, single thread"}
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    world, rank, local = dist_init()
+    wname = args.workload
+    w = synth.workload(wname)
+    mode = WORKLOAD_MODE[wname]
+    replica = rank
+
+    if args.impl == "reference":
+        run_reference(args, w, mode, world, rank)
+        return
+
+    import combine_ep_dispatch_04_b200 as ep
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
+    N = w["N"]
+    idx, wts = synth.make_routing(w, replica)
+    x = synth.make_x(w, replica)
+    cfg = ep.make_config(R, T, M, K, E, H, mode, w["layout"])
+    b = ep.Buffers(cfg, device=dev, grad=bool(w.get("backward")))
+    rows = b.sizes["rows"]
+    idx_d = torch.from_numpy(idx).to(dev)
+    wts_d = torch.from_numpy(wts).to(dev)
+    x_d = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    ypool, yoff = synth.y_source(w, rows, replica)
+    pool_d = torch.from_numpy(ypool.view(np.int16)).to(dev)
+    torch.index_select(pool_d.as_strided((synth.POOL, H), (1, 1)), 0,
+                       torch.from_numpy(yoff).to(dev), out=b.y.view(torch.int16))
+    del pool_d
+    g_d = None
+    if w.get("backward"):
+        gp, go = synth.g_source(w, replica)
+        g_d = torch.from_numpy(synth.windows(gp, go, H).view(np.int16)).to(dev).view(torch.bfloat16)
+    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    kernels = ["layout", "dispatch", "combine"] + (["combine_bwd"] if g_d is not None else [])
+
+    def step(evs=None):
+        if evs:
+            evs[0].record(stream)
+        ep.ep_dispatch_layout(cfg, idx_d, b.token_slot, b.recv_count, b.workspace, b.dev_status,
+                              expert_offset=b.expert_offset, stream=stream)
+        if evs:
+            evs[1].record(stream)
+        ep.ep_dispatch(cfg, x_d, idx_d, b.token_slot, b.recv_buf, b.src_info, b.dev_status,
+                       expert_offset=b.expert_offset, stream=stream)
+        if evs:
+            evs[2].record(stream)
+        ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
+                      expert_offset=b.expert_offset, stream=stream)
+        if evs:
+            evs[3].record(stream)
+        if g_d is not None:
+            ep.ep_combine_backward(cfg, g_d, idx_d, wts_d, b.token_slot, b.grad_buf, b.dev_status,
+                                   expert_offset=b.expert_offset, stream=stream)
+            if evs:
+                evs[4].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.fill_(1)
+        step()
+    torch.cuda.synchronize(dev)
+    if ep.ep_get_status(b.dev_status) != 0:
+        raise SystemExit("device status reported errors during warm-up")
+
+    nev = len(kernels) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    launches0 = ep.ep_kernel_launches()
+    with clocks:
+        for s in range(args.steps):
+            flush.fill_(s & 0xFF)
+            step(evs[s])
+        torch.cuda.synchronize(dev)
+    launches = ep.ep_kernel_launches() - launches0
+    barrier(world)
+    per_kernel = {k: [] for k in kernels}
+    step_ms = []
+    for e in evs:
+        for i, k in enumerate(kernels):
+            per_kernel[k].append(e[i].elapsed_time(e[i + 1]))
+        step_ms.append(e[0].elapsed_time(e[-1]))
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    value = world * N * args.steps / (total_ms / 1e3)
+
+    alg, v = algorithmic_bytes(w, mode, idx)
+    peaks = measured_peaks()
+    peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else FALLBACK_HBM_GBS
+    peak_src = "measured" if peaks and peaks.get("hbm_gbs") else "fallback"
+    kstats = {}
+    for k in kernels:
+        mean_ms = statistics.mean(per_kernel[k])
+        gbs = alg[k] / (mean_ms * 1e-3) / 1e9
+        kstats[k] = {"us_mean": round(mean_ms * 1e3, 2),
+                     "us_p10": round(float(np.percentile(per_kernel[k], 10)) * 1e3, 2),
+                     "us_p90": round(float(np.percentile(per_kernel[k], 90)) * 1e3, 2),
+                     "alg_bytes": alg[k], "gbs": round(gbs, 1),
+                     "frac_of_" + peak_src: round(gbs / peak, 4)}
+    dom = max(kernels, key=lambda k: alg[k])
+    dmean = statistics.mean(per_kernel[dom]) * 1e-3
+    achieved = alg[dom] / dmean / 1e9
+    step_bytes = sum(alg.values())
+
+    # same-run copy bandwidth (reference for the fractions above)
+    copy_gbs = None
+    try:
+        src = torch.empty(2 << 30, dtype=torch.uint8, device=dev)
+        dst = torch.empty_like(src)
+        for _ in range(3):
+            ep.ep_copy(dst, src, stream=stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        best = None
+        for _ in range(10):
+            e0.record(stream)
+            ep.ep_copy(dst, src, stream=stream)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+            t = e0.elapsed_time(e1)
+            best = t if best is None or t < best else best
+        copy_gbs = round(2 * src.numel() / (best * 1e-3) / 1e9, 1)
+        del src, dst
+    except Exception:
+        pass
+
+    e2e = None if args.no_e2e else run_e2e(ep, cfg, b, w, idx, wts, x, g_d, flush, stream, dev,
+                                          args, world)
+
+    out = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{wname}: R={R} T={T} H={H} K={K} E={E} M={M} {mode} {w['layout']}",
+            "tokens_per_step": N, "valid_entries": v,
+            "l2": f"flushed between steps ({args.flush_mib} MiB write outside the step events)",
+            "parallelism": "replicas" if world > 1 else "single",
+        },
+        "hbm_gbs": round(step_bytes / (ms_per_step * 1e-3) / 1e9, 1),
+        "hbm_frac_of_" + peak_src: round(step_bytes / (ms_per_step * 1e-3) / 1e9 / peak, 4),
+        "clocks": clocks.report(),
+        "gpu_launches": launches,
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": peak, "peak_source": peak_src, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "traffic": ncu_traffic(dom, wname)},
+        "kernels": kstats,
+        "copy_gbs_same_run": copy_gbs,
+        "e2e": e2e,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(w, mode, idx, wts, x, args.cpu_seconds, replica)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    dist_done(world)
+
+
+def run_e2e(ep, cfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, world):
+    """The same step through the public API with host buffers: pinned host
+    inputs copied in, the combined output and the counts copied back, inside
+    the timed region of every step.  Expert outputs (and the gradient) stay on
+    the device: in a MoE layer the experts produce them there."""
+    N, H = w["N"], w["H"]
+    x_h = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    idx_h = torch.from_numpy(idx).pin_memory()
+    wts_h = torch.from_numpy(wts).pin_memory()
+    out_h = torch.empty((N, H), dtype=torch.bfloat16).pin_memory()
+    cnt_h = torch.empty(w["E"], dtype=torch.int64).pin_memory()
+    x_d = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+    idx_d = torch.empty_like(idx_h, device=dev)
+    wts_d = torch.empty_like(wts_h, device=dev)
+    h2d = x_h.numel() * 2 + idx_h.numel() * 8 + wts_h.numel() * 4
+    d2h = out_h.numel() * 2 + cnt_h.numel() * 8
+
+    def one():
+        x_d.copy_(x_h, non_blocking=True)
+        idx_d.copy_(idx_h, non_blocking=True)
+        wts_d.copy_(wts_h, non_blocking=True)
+        ep.ep_dispatch_layout(cfg, idx_d, b.token_slot, b.recv_count, b.workspace, b.dev_status,
+                              expert_offset=b.expert_offset, stream=stream)
+        ep.ep_dispatch(cfg, x_d, idx_d, b.token_slot, b.recv_buf, b.src_info, b.dev_status,
+                       expert_offset=b.expert_offset, stream=stream)
+        ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
+                      expert_offset=b.expert_offset, stream=stream)
+        if g_d is not None:
+            ep.ep_combine_backward(cfg, g_d, idx_d, wts_d, b.token_slot, b.grad_buf,
+                                   b.dev_status, expert_offset=b.expert_offset, stream=stream)
+        out_h.copy_(b.out, non_blocking=True)
+        cnt_h.copy_(b.recv_count, non_blocking=True)
+
+    for _ in range(3):
+        flush.fill_(1)
+        one()
+    steps = max(10, min(args.steps, 100))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for s in range(steps):
+        flush.fill_(s & 0xFF)
+        evs[s][0].record(stream)
+        one()
+        evs[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    total_ms = max_over_ranks(sum(a.elapsed_time(c) for a, c in evs), world)
+    return {"value": round(world * N * steps / (total_ms / 1e3), 1), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def run_reference(args, w, mode, world, rank):
+    """The reference arm: the oracle on the host cores, rank 0 only."""
+    if rank != 0:
+        dist_done(world)
+        return
+    idx, wts = synth.make_routing(w, 0)
+    x = synth.make_x(w, 0)
+    st = OracleStep(w, mode, idx, wts, x, sub_t=max(1, w["T"] // 8))
+    for _ in range(args.warmup):
+        st.step()
+    t0 = time.perf_counter()
+    done = 0
+    for _ in range(args.steps):
+        done += st.step()
+    el = time.perf_counter() - t0
+    value = done / el
+    R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
+    out = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": f"{w['name']}: R={R} T={T} H={H} K={K} E={E} M={M} {mode} "
+                               f"{w['layout']}", "tokens_per_step": st.n},
+        "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": 1,
+                         "kind": "oracle", "sample": st.sample},
+        "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out), flush=True)
+    dist_done(world)
+
+
+if __name__ == "__main__":
+    main()

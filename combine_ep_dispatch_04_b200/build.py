@@ -1,0 +1,42 @@
+"""Build libep.so (the C ABI of include/ep.h) in-tree for sm_100a.
+
+The library is compiled with IEEE semantics (no fast-math: divisions and
+square roots correctly rounded, subnormals kept); the kernels spell out every
+rounding they need with __fmul_rn / __fdiv_rn / __fmaf_rn.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+CSRC = os.path.join(HERE, "csrc")
+LIB = os.path.join(HERE, "libep.so")
+SOURCES = [os.path.join(CSRC, "ep_api.cu")]
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + \
+    [os.path.join(ROOT, "include", "ep.h")]
+
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+FLAGS = [
+    "-gencode", "arch=compute_100a,code=sm_100a",
+    "-O3", "-lineinfo", "-std=c++17",
+    "-Xcompiler", "-fPIC", "-shared",
+    "-I", os.path.join(ROOT, "include"),
+]
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    """Compile the library when it is missing or older than its sources."""
+    if not force and os.path.exists(LIB):
+        newest = max(os.path.getmtime(p) for p in DEPS)
+        if os.path.getmtime(LIB) >= newest:
+            return LIB
+    tmp = LIB + ".tmp%d" % os.getpid()
+    cmd = [NVCC, *FLAGS, *(["-Xptxas", "-v"] if verbose else []), *SOURCES, "-o", tmp]
+    subprocess.check_call(cmd)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force=True, verbose="-v" in sys.argv))

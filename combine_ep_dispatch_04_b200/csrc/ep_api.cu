@@ -1,0 +1,410 @@
+// ep_api.cu -- the C ABI of libep (declared in include/ep.h): argument
+// validation, buffer sizing and kernel selection.  Every hot step runs in the
+// kernels of ep_layout.cuh, ep_dispatch.cuh and ep_combine.cuh.
+#include <atomic>
+#include <cmath>
+#include <cstring>
+
+#include "ep.h"
+#include "ep_combine.cuh"
+#include "ep_device.cuh"
+#include "ep_dispatch.cuh"
+#include "ep_layout.cuh"
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+constexpr int kMaxExperts = 1024;
+constexpr int kMaxHidden = 8192;
+constexpr int64_t kIntLimit = (int64_t(1) << 31) - 1;
+// one-block layout when the routing is small (its per-warp counters fit in
+// the default 48 KB of shared memory)
+constexpr int64_t kSingleMaxEntries = 32768;
+constexpr int kSingleMaxExperts = 384;
+
+cudaStream_t cs(ep_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+ep_status_t launched() {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
+// Derived quantities of a validated configuration.
+struct Plan {
+    int R, T, M, K, E, H, L;
+    int64_t N, cap, rows, D, S, scale_off, recv_bytes, grad_scale_off, grad_bytes;
+    int TC, CR, C;
+    int64_t ws_bytes;
+};
+
+int64_t data_row_bytes(int quant, int H) {
+    return quant == EP_Q_BF16 ? 2LL * H : (quant == EP_Q_MXFP4 ? H / 2 : H);
+}
+int64_t scale_row_bytes(int quant, int H) {
+    switch (quant) {
+    case EP_Q_BF16: return 0;
+    case EP_Q_INT8_TOKEN: return 4;
+    case EP_Q_E4M3_B128: return 4LL * (H / 128);
+    default: return H / 32;
+    }
+}
+
+// Every check happens before any arithmetic that uses the values.
+ep_status_t make_plan(const ep_config_t *c, Plan &p) {
+    if (!c) return EP_ERR_INVALID_ARG;
+    if (c->num_ranks <= 0 || c->max_tokens_per_rank <= 0 || c->num_tokens < 0 ||
+        c->num_tokens > c->max_tokens_per_rank)
+        return EP_ERR_INVALID_ARG;
+    if (c->num_topk < 1 || c->num_topk > ep::kMaxTopk) return EP_ERR_INVALID_ARG;
+    if (c->num_experts < 1 || c->num_experts > kMaxExperts) return EP_ERR_INVALID_ARG;
+    if (c->num_experts % c->num_ranks != 0) return EP_ERR_INVALID_ARG;
+    if (c->hidden < 32 || c->hidden > kMaxHidden || c->hidden % 32 != 0) return EP_ERR_INVALID_ARG;
+    if (c->quant < EP_Q_BF16 || c->quant > EP_Q_MXFP4) return EP_ERR_INVALID_ARG;
+    if (c->quant == EP_Q_E4M3_B128 && c->hidden % 128 != 0) return EP_ERR_INVALID_ARG;
+    if (c->layout != EP_LAYOUT_PADDED && c->layout != EP_LAYOUT_PACKED) return EP_ERR_INVALID_ARG;
+    if (c->expert_align < 1) return EP_ERR_INVALID_ARG;
+    if (!(c->e4m3_qmax >= 0.0f && c->e4m3_qmax <= 448.0f)) return EP_ERR_INVALID_ARG;  // NaN fails
+    const uint32_t known = EP_F_BWD_UNWEIGHTED | EP_F_LAYOUT_SINGLE_CTA | EP_F_LAYOUT_MULTI_CTA;
+    if (c->flags & ~known) return EP_ERR_INVALID_ARG;
+    if ((c->flags & EP_F_LAYOUT_SINGLE_CTA) && (c->flags & EP_F_LAYOUT_MULTI_CTA))
+        return EP_ERR_INVALID_ARG;
+
+    p.R = c->num_ranks;
+    p.T = c->num_tokens;
+    p.M = c->max_tokens_per_rank;
+    p.K = c->num_topk;
+    p.E = c->num_experts;
+    p.H = c->hidden;
+    p.L = p.E / p.R;
+    p.N = (int64_t)p.R * p.T;
+    if (p.N * p.K > kIntLimit) return EP_ERR_INVALID_ARG;
+    p.cap = (int64_t)p.R * p.M;
+    if (c->layout == EP_LAYOUT_PADDED) {
+        if (p.cap > kIntLimit) return EP_ERR_INVALID_ARG;  // slots are int32
+        p.rows = (int64_t)p.E * p.cap;
+    } else {
+        if ((int64_t)c->expert_align > kIntLimit / p.E) return EP_ERR_INVALID_ARG;
+        p.rows = p.N * p.K + (int64_t)p.E * (c->expert_align - 1);
+        if (p.rows > kIntLimit) return EP_ERR_INVALID_ARG;  // expert_offset scan is int32 per tile
+    }
+    p.D = data_row_bytes(c->quant, p.H);
+    p.S = scale_row_bytes(c->quant, p.H);
+    p.scale_off = round_up(p.rows * p.D, 256);
+    p.recv_bytes = p.scale_off + p.rows * p.S;
+    p.grad_scale_off = round_up(p.rows * p.H, 256);
+    p.grad_bytes = p.grad_scale_off + p.rows * (p.H / 32);
+    // layout chunks: whole tokens of one source rank, about 2048 entries each
+    p.TC = (2048 + p.K - 1) / p.K;
+    if (p.TC > p.T) p.TC = p.T > 0 ? p.T : 1;
+    p.CR = (p.T + p.TC - 1) / p.TC;
+    p.C = p.R * p.CR;
+    p.ws_bytes = round_up((int64_t)(p.E + p.R) * p.C * 4, 256);
+    if (p.ws_bytes == 0) p.ws_bytes = 256;
+    return EP_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *ep_status_string(ep_status_t s) {
+    switch (s) {
+    case EP_OK: return "ok";
+    case EP_ERR_INVALID_ARG: return "invalid argument";
+    case EP_ERR_UNSUPPORTED: return "unsupported";
+    case EP_ERR_MISALIGNED: return "buffer not 16-byte aligned";
+    case EP_ERR_CUDA: return "CUDA runtime error";
+    case EP_ERR_DEVICE_STATUS: return "device reported bad indices or capacity overflow";
+    case EP_ERR_TIMEOUT: return "timed out";
+    }
+    return "unknown status";
+}
+
+uint64_t ep_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
+
+ep_status_t ep_buffer_sizes(const ep_config_t *cfg, ep_sizes_t *out) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (!out) return EP_ERR_INVALID_ARG;
+    std::memset(out, 0, sizeof(*out));
+    out->rows = p.rows;
+    out->data_row_bytes = p.D;
+    out->scale_row_bytes = p.S;
+    out->recv_scale_offset = p.scale_off;
+    out->recv_bytes = p.recv_bytes;
+    out->src_info_bytes = p.rows * 4;
+    out->recv_weights_bytes = p.rows * 4;
+    out->expert_out_bytes = p.rows * p.H * 2;
+    out->grad_scale_offset = p.grad_scale_off;
+    out->grad_bytes = p.grad_bytes;
+    out->workspace_bytes = p.ws_bytes;
+    out->token_slot_bytes = p.N * p.K * 4;
+    out->is_token_in_rank_bytes = p.N * p.R;
+    return EP_OK;
+}
+
+ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const int64_t *topk_idx,
+                               int32_t *tokens_per_rank, int32_t *tokens_per_expert,
+                               uint8_t *is_token_in_rank, int32_t *token_slot,
+                               int64_t *recv_count, int64_t *expert_offset,
+                               int64_t *cumulative_recv_stats, void *workspace,
+                               uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (!recv_count || !workspace || !dev_status) return EP_ERR_INVALID_ARG;
+    if (p.N > 0 && (!topk_idx || !token_slot)) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+
+    ep::LayoutArgs a;
+    a.R = p.R; a.T = p.T; a.K = p.K; a.E = p.E; a.M = p.M; a.L = p.L;
+    a.TC = p.TC; a.CR = p.CR; a.C = p.C;
+    a.packed = cfg->layout == EP_LAYOUT_PACKED;
+    a.align = cfg->expert_align;
+    a.cap = p.cap;
+    a.idx = topk_idx;
+    a.tpr = tokens_per_rank;
+    a.tpe = tokens_per_expert;
+    a.itr = is_token_in_rank;
+    a.slot = token_slot;
+    a.recv_count = recv_count;
+    a.eo = expert_offset;
+    a.stats = cumulative_recv_stats;
+    a.ws_hist = static_cast<int32_t *>(workspace);
+    a.ws_rk = a.ws_hist + (int64_t)p.E * p.C;
+    a.status = dev_status;
+
+    cudaStream_t s = cs(stream);
+    const bool single = (cfg->flags & EP_F_LAYOUT_SINGLE_CTA) ||
+                        (!(cfg->flags & EP_F_LAYOUT_MULTI_CTA) && p.N * p.K <= kSingleMaxEntries &&
+                         p.E <= kSingleMaxExperts);
+    if (single) {
+        const size_t smem1 = (size_t)(ep::kLayoutSingleThreads / 32) * p.E * sizeof(int);
+        if (smem1 > 48 * 1024 &&
+            cudaFuncSetAttribute(ep::layout_single_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem1) != cudaSuccess)
+            return EP_ERR_CUDA;
+        ep::layout_single_kernel<<<1, ep::kLayoutSingleThreads, smem1, s>>>(a);
+        return launched();
+    }
+    if (p.C > 0) {
+        ep::layout_count_kernel<<<p.C, ep::kLayoutThreads, (p.E + p.R) * sizeof(int), s>>>(a);
+        if ((st = launched()) != EP_OK) return st;
+    }
+    ep::layout_scan_kernel<<<p.E + p.R, ep::kLayoutThreads, 0, s>>>(a);
+    if ((st = launched()) != EP_OK) return st;
+    const size_t smem = (size_t)(ep::kLayoutThreads / 32) * p.E * sizeof(int);
+    ep::layout_assign_kernel<<<p.C > 0 ? p.C : 1, ep::kLayoutThreads, smem, s>>>(a);
+    return launched();
+}
+
+}  // extern "C"
+
+namespace {
+
+// granules of 16 elements -> (threads per token, granules per thread)
+template <int MODE>
+ep_status_t launch_dispatch(const ep::DispatchArgs &a, cudaStream_t s) {
+    const int ng = a.H / 16;
+    auto grid = [&](int tpt) { return (unsigned)((a.N + (ep::kDispatchThreads / tpt) - 1) /
+                                                 (ep::kDispatchThreads / tpt)); };
+    if (ng <= 32) ep::dispatch_kernel<MODE, 32, 1><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
+    else if (ng <= 64) ep::dispatch_kernel<MODE, 32, 2><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
+    else if (ng <= 128) ep::dispatch_kernel<MODE, 32, 4><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
+    else if (ng <= 256) ep::dispatch_kernel<MODE, 32, 8><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
+    else ep::dispatch_kernel<MODE, 64, 8><<<grid(64), ep::kDispatchThreads, 0, s>>>(a);
+    return launched();
+}
+
+ep_status_t launch_combine_bwd(const ep::DispatchArgs &a, cudaStream_t s) {
+    const int ng = a.H / 16;
+    auto grid = [&](int tpt) { return (unsigned)((a.N + (ep::kDispatchThreads / tpt) - 1) /
+                                                 (ep::kDispatchThreads / tpt)); };
+    if (ng <= 32) ep::combine_bwd_kernel<32, 1><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
+    else if (ng <= 64) ep::combine_bwd_kernel<32, 2><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
+    else if (ng <= 128) ep::combine_bwd_kernel<32, 4><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
+    else if (ng <= 256) ep::combine_bwd_kernel<32, 8><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
+    else ep::combine_bwd_kernel<64, 8><<<grid(64), ep::kDispatchThreads, 0, s>>>(a);
+    return launched();
+}
+
+ep::DispatchArgs dispatch_args(const ep_config_t *cfg, const Plan &p) {
+    ep::DispatchArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.N = p.N; a.T = p.T; a.K = p.K; a.E = p.E; a.M = p.M; a.H = p.H;
+    a.packed = cfg->layout == EP_LAYOUT_PACKED;
+    a.cap = p.cap;
+    a.rows = p.rows;
+    a.qmax = cfg->e4m3_qmax > 0.0f ? cfg->e4m3_qmax : 448.0f;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const int64_t *topk_idx,
+                        const float *topk_weights, const int32_t *token_slot,
+                        const int64_t *expert_offset, void *recv_buf, int32_t *src_info,
+                        float *recv_weights, uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (!dev_status) return EP_ERR_INVALID_ARG;
+    if (p.N == 0) return EP_OK;
+    if (!x || !topk_idx || !token_slot || !recv_buf || !src_info) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    if (recv_weights && !topk_weights) return EP_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(recv_buf)) return EP_ERR_MISALIGNED;
+
+    ep::DispatchArgs a = dispatch_args(cfg, p);
+    a.D = p.D; a.S = p.S; a.scale_off = p.scale_off;
+    a.x = x; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
+    a.out = static_cast<uint8_t *>(recv_buf);
+    a.src_info = src_info;
+    a.recv_w = recv_weights;
+    a.status = dev_status;
+    cudaStream_t s = cs(stream);
+    switch (cfg->quant) {
+    case EP_Q_BF16: return launch_dispatch<ep::Q_BF16>(a, s);
+    case EP_Q_E4M3_B128: return launch_dispatch<ep::Q_E4M3_B128>(a, s);
+    case EP_Q_INT8_TOKEN: return launch_dispatch<ep::Q_INT8>(a, s);
+    case EP_Q_MXFP8: return launch_dispatch<ep::Q_MXFP8>(a, s);
+    default: return launch_dispatch<ep::Q_MXFP4>(a, s);
+    }
+}
+
+ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t *topk_idx,
+                       const float *topk_weights, const int32_t *token_slot,
+                       const int64_t *expert_offset, uint16_t *out, uint32_t *dev_status,
+                       ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (!dev_status) return EP_ERR_INVALID_ARG;
+    if (p.N == 0) return EP_OK;
+    if (!y || !topk_idx || !topk_weights || !token_slot || !out) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    if (!aligned16(y) || !aligned16(out)) return EP_ERR_MISALIGNED;
+
+    ep::CombineArgs a;
+    a.N = p.N; a.K = p.K; a.E = p.E; a.H = p.H;
+    a.packed = cfg->layout == EP_LAYOUT_PACKED;
+    a.cap = p.cap; a.rows = p.rows;
+    a.y = y; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
+    a.out = out; a.status = dev_status;
+    constexpr int TPT = 128, TOKS = ep::kCombineThreads / TPT;
+    const unsigned grid = (unsigned)((p.N + TOKS - 1) / TOKS);
+    const int ng = p.H / 8;
+    cudaStream_t s = cs(stream);
+    if (ng <= TPT) ep::combine_kernel<TPT, 1, 8><<<grid, ep::kCombineThreads, 0, s>>>(a);
+    else if (ng <= 2 * TPT) ep::combine_kernel<TPT, 2, 8><<<grid, ep::kCombineThreads, 0, s>>>(a);
+    else if (ng <= 4 * TPT) ep::combine_kernel<TPT, 4, 8><<<grid, ep::kCombineThreads, 0, s>>>(a);
+    else ep::combine_kernel<TPT, 8, 8><<<grid, ep::kCombineThreads, 0, s>>>(a);
+    return launched();
+}
+
+ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
+                                const int64_t *topk_idx, const float *topk_weights,
+                                const int32_t *token_slot, const int64_t *expert_offset,
+                                void *grad_buf, uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (!dev_status) return EP_ERR_INVALID_ARG;
+    if (p.N == 0) return EP_OK;
+    const bool unweighted = (cfg->flags & EP_F_BWD_UNWEIGHTED) != 0;
+    if (!g || !topk_idx || !token_slot || !grad_buf) return EP_ERR_INVALID_ARG;
+    if (!unweighted && !topk_weights) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    if (!aligned16(g) || !aligned16(grad_buf)) return EP_ERR_MISALIGNED;
+
+    ep::DispatchArgs a = dispatch_args(cfg, p);
+    a.D = p.H; a.S = p.H / 32; a.scale_off = p.grad_scale_off;
+    a.unweighted = unweighted;
+    a.x = g; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
+    a.out = static_cast<uint8_t *>(grad_buf);
+    a.status = dev_status;
+    return launch_combine_bwd(a, cs(stream));
+}
+
+ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream) {
+    if (!dev_status || !host_flags) return EP_ERR_INVALID_ARG;
+    cudaStream_t s = cs(stream);
+    uint32_t h = 0;
+    if (cudaMemcpyAsync(&h, dev_status, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return EP_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return EP_ERR_CUDA;
+    if (cudaMemsetAsync(dev_status, 0, sizeof(uint32_t), s) != cudaSuccess) return EP_ERR_CUDA;
+    *host_flags = h;
+    return h ? EP_ERR_DEVICE_STATUS : EP_OK;
+}
+
+}  // extern "C"
+
+// ---- diagnostics -------------------------------------------------------------
+namespace ep {
+
+__global__ void __launch_bounds__(512) copy_kernel(uint4 *__restrict__ dst,
+                                                   const uint4 *__restrict__ src, int64_t n) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    for (; i + 3 * stride < n; i += 4 * stride) {
+        const uint4 a = ld_stream(src + i), b = ld_stream(src + i + stride);
+        const uint4 c = ld_stream(src + i + 2 * stride), d = ld_stream(src + i + 3 * stride);
+        dst[i] = a; dst[i + stride] = b; dst[i + 2 * stride] = c; dst[i + 3 * stride] = d;
+    }
+    for (; i < n; i += stride) dst[i] = ld_stream(src + i);
+}
+
+__global__ void cvt_sweep_kernel(int format, uint32_t start, int64_t n, uint8_t *out) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const float v = __uint_as_float(start + (uint32_t)i);
+        out[i] = format == 0 ? (uint8_t)(cvt_e4m3x2(v, 0.0f) & 0xFFu)
+                             : (uint8_t)(cvt_e2m1x2(v, 0.0f) & 0xFu);
+    }
+}
+
+}  // namespace ep
+
+namespace {
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n > 0 ? n : 148;
+}
+}  // namespace
+
+extern "C" ep_status_t ep_copy(void *dst, const void *src, size_t bytes, ep_stream_t stream) {
+    if (!dst || !src || bytes % 16 != 0) return EP_ERR_INVALID_ARG;
+    if (!aligned16(dst) || !aligned16(src)) return EP_ERR_MISALIGNED;
+    if (bytes == 0) return EP_OK;
+    const int64_t n = (int64_t)(bytes / 16);
+    int64_t blocks = (n + 511) / 512;
+    const int64_t cap = (int64_t)sm_count() * 4;
+    if (blocks > cap) blocks = cap;
+    ep::copy_kernel<<<(unsigned)blocks, 512, 0, cs(stream)>>>(
+        static_cast<uint4 *>(dst), static_cast<const uint4 *>(src), n);
+    return launched();
+}
+
+extern "C" ep_status_t ep_cvt_sweep(int32_t format, uint32_t start, int64_t n, uint8_t *out,
+                                    ep_stream_t stream) {
+    if ((format != 0 && format != 1) || n < 0 || !out) return EP_ERR_INVALID_ARG;
+    if (n > (int64_t(1) << 32) - (int64_t)start) return EP_ERR_INVALID_ARG;
+    if (n == 0) return EP_OK;
+    int64_t blocks = (n + 255) / 256;
+    const int64_t cap = (int64_t)sm_count() * 16;
+    if (blocks > cap) blocks = cap;
+    ep::cvt_sweep_kernel<<<(unsigned)blocks, 256, 0, cs(stream)>>>(format, start, n, out);
+    return launched();
+}

@@ -1,0 +1,101 @@
+// ep_device.cuh -- device helpers shared by the dispatch / combine kernels:
+// bf16 unpacking, the native sm_100a format conversions (cvt ... satfinite to
+// e4m3 / e2m1), the e8m0 exponent of an MX block, and streaming memory access.
+//
+// Arithmetic contract (matches the quantisation rules of the header): every
+// scale is one IEEE division (__fdiv_rn), every scaled value one rounded
+// multiply (__fmul_rn, never contracted into an FMA), conversions round to
+// nearest even.  The library is built without fast-math, so subnormals are kept.
+#pragma once
+
+#include <cfloat>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace ep {
+
+constexpr uint32_t kFull = 0xFFFFFFFFu;
+constexpr uint32_t kDevBadIndex = 0x1u;
+constexpr uint32_t kDevCapacity = 0x2u;
+
+// ---- bf16 ------------------------------------------------------------------
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// |x| of the two bf16 halves compared as integers: for finite values the
+// magnitude order of bf16 bit patterns (sign cleared) is the numeric order.
+__device__ __forceinline__ uint32_t bf2_absmax(uint32_t acc, uint32_t w) {
+    return __vmaxu2(acc, w & 0x7FFF7FFFu);
+}
+__device__ __forceinline__ float bf2_fold(uint32_t m) {  // max of the two halves as fp32
+    uint32_t lo = m & 0xFFFFu, hi = m >> 16;
+    return __uint_as_float((lo > hi ? lo : hi) << 16);
+}
+
+// Two fp32 -> bf16x2 (round to nearest even); `lo` lands in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ---- native format conversions (sm_100a) ----------------------------------
+// cvt ... e4m3x2 / e2m1x2 put their first source operand in the upper part of
+// the result, so `lo` is passed second to land at the lower address / nibble.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(hi), "f"(lo));
+    return r;
+}
+
+// ---- scales ------------------------------------------------------------------
+// ceil(log2 v) for a positive finite fp32 v, exactly, from its bits.
+__device__ __forceinline__ int ceil_log2_pos(float v) {
+    uint32_t b = __float_as_uint(v);
+    int ex = (int)(b >> 23);
+    uint32_t m = b & 0x7FFFFFu;
+    if (ex != 0) return ex - 127 + (m != 0u);
+    return (32 - __clz((int)(m - 1u))) - 149;  // subnormal: v = m * 2^-149
+}
+
+// e8m0 exponent X of an MX block: the smallest power of two with
+// amax / qmax <= 2^X, i.e. ceil(log2(amax / qmax)) with one IEEE division,
+// clamped to [-127, 127]; amax == 0 gives 0.
+__device__ __forceinline__ int mx_exponent(float amax, float qmax) {
+    if (amax == 0.0f) return 0;
+    float v = __fdiv_rn(amax, qmax);
+    if (v == 0.0f) return -127;
+    int X = ceil_log2_pos(v);
+    return X < -127 ? -127 : (X > 127 ? 127 : X);
+}
+
+// 2^-X as an fp32 for X in [-127, 127] (2^-127 is the subnormal 0x00400000).
+__device__ __forceinline__ float exp2_neg(int X) {
+    int e = 127 - X;
+    return e > 0 ? __uint_as_float((uint32_t)e << 23) : __uint_as_float(0x00400000u);
+}
+
+// ---- streaming memory access --------------------------------------------------
+__device__ __forceinline__ uint4 ld_stream(const void *p) {
+    return __ldcs(reinterpret_cast<const uint4 *>(p));
+}
+__device__ __forceinline__ uint4 ld_ro(const void *p) {
+    return __ldg(reinterpret_cast<const uint4 *>(p));
+}
+__device__ __forceinline__ void st_v4(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+__device__ __forceinline__ void st_v2(void *p, uint2 v) { *reinterpret_cast<uint2 *>(p) = v; }
+
+__device__ __forceinline__ uint32_t lanemask_lt() {
+    uint32_t m;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));
+    return m;
+}
+
+}  // namespace ep

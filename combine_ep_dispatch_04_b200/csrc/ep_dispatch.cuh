@@ -1,0 +1,333 @@
+// ep_dispatch.cuh -- fused quantise + scatter (dispatch) and the reverse
+// dispatch of the combine backward.
+//
+// Dispatch ("Low-Latency Mode API", low_latency_dispatch Return Values;
+// "DeepEP FP8 Dispatch and Combine Operations", The Dispatch Stage;
+// "EP dispatch with unfused MXFP8 quantization", Changes): every source token
+// is read once, quantised once, and its row is stored to each of its <= K
+// receive rows (data region) with its scales (scale region), src_info and the
+// optional weight.
+//
+// Work split: a group of TPT threads (1 or 2 warps) owns one token.  The row
+// is cut into 16-element granules (32 bytes of bf16 input); thread lt of the
+// group holds granules g = i*TPT + lt, i < GMAX, as two 16-byte loads.  A
+// quantisation block of 128 elements is 8 consecutive threads and one of 32
+// elements is 2, so block maxima are warp shuffles; the per-row int8 maximum
+// crosses warps through shared memory.  Codes are computed once, then the
+// group stores them to every destination row with 16-byte (8 for e2m1)
+// coalesced stores: per warp instruction 512 (256) contiguous bytes.
+#pragma once
+
+#include "ep_device.cuh"
+
+namespace ep {
+
+enum { Q_BF16 = 0, Q_E4M3_B128 = 1, Q_INT8 = 2, Q_MXFP8 = 3, Q_MXFP4 = 4 };
+
+struct DispatchArgs {
+    int64_t N;
+    int T, K, E, M, H;
+    int packed;
+    int64_t cap, rows;       // padded rows per expert, buffer row capacity
+    int64_t D, S, scale_off; // row data bytes, row scale bytes, scale region offset
+    float qmax;              // e4m3_b128 target max
+    int unweighted;          // combine backward only
+    const uint16_t *x;       // [N][H] bf16 (the gradient g for the backward)
+    const int64_t *idx;
+    const float *wts;
+    const int32_t *slot;
+    const int64_t *eo;
+    uint8_t *out;            // recv_buf / grad_buf
+    int32_t *src_info;
+    float *recv_w;
+    uint32_t *status;
+};
+
+constexpr int kDispatchThreads = 256;
+
+// Row of entry (n, k) in the receive layout, or -1 (masked, or no row).
+__device__ __forceinline__ int64_t entry_row(const DispatchArgs &a, int64_t n, int k,
+                                             uint32_t &flags) {
+    const int64_t e = a.idx[n * a.K + k];
+    if (e < -1 || e >= a.E) flags |= kDevBadIndex;
+    if (e < 0 || e >= a.E) return -1;
+    const int32_t s = a.slot[n * a.K + k];
+    if (s < 0) return -1;
+    int64_t row;
+    if (!a.packed) {
+        if (s >= a.cap) { flags |= kDevCapacity; return -1; }
+        row = e * a.cap + s;
+    } else {
+        row = a.eo[e] + s;
+        if (row >= a.eo[e + 1] || row >= a.rows) { flags |= kDevCapacity; return -1; }
+    }
+    return row;
+}
+
+template <int MODE>
+struct GranOut;  // bytes a 16-element granule becomes
+template <> struct GranOut<Q_BF16> { static constexpr int bytes = 32; };
+template <> struct GranOut<Q_E4M3_B128> { static constexpr int bytes = 16; };
+template <> struct GranOut<Q_INT8> { static constexpr int bytes = 16; };
+template <> struct GranOut<Q_MXFP8> { static constexpr int bytes = 16; };
+template <> struct GranOut<Q_MXFP4> { static constexpr int bytes = 8; };
+
+__device__ __forceinline__ uint32_t q_i8(float v, float s) {
+    int q = __float2int_rn(__fmul_rn(v, s));
+    q = q > 127 ? 127 : (q < -127 ? -127 : q);
+    return (uint32_t)q & 0xFFu;
+}
+
+template <int MODE, int TPT, int GMAX>
+__global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs a) {
+    constexpr int TOKS = kDispatchThreads / TPT;
+    constexpr int WPG = TPT / 32;  // warps per token group
+    constexpr int OB = GranOut<MODE>::bytes;
+    __shared__ int64_t s_row[TOKS][16];
+    __shared__ float s_red[TOKS][WPG];
+
+    const int grp = threadIdx.x / TPT, lt = threadIdx.x % TPT;
+    const int64_t n = (int64_t)blockIdx.x * TOKS + grp;
+    const bool active = n < a.N;
+    const int ngran = a.H >> 4;
+
+    if (active && lt < a.K) {
+        uint32_t flags = 0;
+        const int64_t row = entry_row(a, n, lt, flags);
+        if (flags) atomicOr(a.status, flags);
+        s_row[grp][lt] = row;
+        if (row >= 0) {
+            a.src_info[row] = (int32_t)((n / a.T) * a.M + n % a.T);
+            if (a.recv_w) a.recv_w[row] = a.wts[n * a.K + lt];
+        }
+    }
+
+    // load the token's granules (two 16-byte loads each)
+    uint32_t v[GMAX][8];
+#pragma unroll
+    for (int i = 0; i < GMAX; i++) {
+        const int g = i * TPT + lt;
+        if (active && g < ngran) {
+            const uint16_t *p = a.x + n * a.H + (int64_t)g * 16;
+            const uint4 u0 = ld_stream(p), u1 = ld_stream(p + 8);
+            v[i][0] = u0.x; v[i][1] = u0.y; v[i][2] = u0.z; v[i][3] = u0.w;
+            v[i][4] = u1.x; v[i][5] = u1.y; v[i][6] = u1.z; v[i][7] = u1.w;
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; q++) v[i][q] = 0u;
+        }
+    }
+
+    // per-granule block maxima (bf16 magnitudes, exact)
+    float gmax[GMAX];
+#pragma unroll
+    for (int i = 0; i < GMAX; i++) {
+        uint32_t m = 0u;
+#pragma unroll
+        for (int q = 0; q < 8; q++) m = bf2_absmax(m, v[i][q]);
+        gmax[i] = bf2_fold(m);
+    }
+
+    // scales
+    float rs = 1.0f, rsinv = 1.0f;  // int8: per row
+    float bs[GMAX];                 // e4m3_b128: per 128-block multiplier; mx: 2^-X
+    float bsinv[GMAX];              // e4m3_b128: stored scale_inv
+    uint32_t bx[GMAX];              // mx: e8m0 byte
+    if constexpr (MODE == Q_INT8) {
+        float m = 0.0f;
+#pragma unroll
+        for (int i = 0; i < GMAX; i++) m = fmaxf(m, gmax[i]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(kFull, m, o));
+        if constexpr (WPG > 1) {
+            if ((lt & 31) == 0) s_red[grp][lt >> 5] = m;
+        }
+        __syncthreads();
+        if constexpr (WPG > 1) {
+#pragma unroll
+            for (int q = 0; q < WPG; q++) m = fmaxf(m, s_red[grp][q]);
+        }
+        if (m != 0.0f) {
+            rs = fminf(__fdiv_rn(127.0f, m), FLT_MAX);
+            rsinv = __fdiv_rn(m, 127.0f);
+        }
+    } else {
+        __syncthreads();  // s_row visible to the whole group
+    }
+    if constexpr (MODE == Q_E4M3_B128) {
+#pragma unroll
+        for (int i = 0; i < GMAX; i++) {
+            float m = gmax[i];
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 2));
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
+            bs[i] = 1.0f;
+            bsinv[i] = 1.0f;
+            if (m != 0.0f) {
+                bs[i] = fminf(__fdiv_rn(a.qmax, m), FLT_MAX);
+                bsinv[i] = __fdiv_rn(m, a.qmax);
+            }
+        }
+    }
+    if constexpr (MODE == Q_MXFP8 || MODE == Q_MXFP4) {
+        constexpr float QM = MODE == Q_MXFP8 ? 448.0f : 6.0f;
+#pragma unroll
+        for (int i = 0; i < GMAX; i++) {
+            float m = gmax[i];
+            m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+            const int X = mx_exponent(m, QM);
+            bs[i] = exp2_neg(X);
+            bx[i] = (uint32_t)(X + 127);
+        }
+    }
+
+    // codes
+    uint32_t c[GMAX][OB / 4];
+#pragma unroll
+    for (int i = 0; i < GMAX; i++) {
+        if constexpr (MODE == Q_BF16) {
+#pragma unroll
+            for (int q = 0; q < 8; q++) c[i][q] = v[i][q];
+        } else if constexpr (MODE == Q_INT8) {
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const uint32_t w0 = v[i][2 * q], w1 = v[i][2 * q + 1];
+                c[i][q] = q_i8(bf_lo(w0), rs) | (q_i8(bf_hi(w0), rs) << 8) |
+                          (q_i8(bf_lo(w1), rs) << 16) | (q_i8(bf_hi(w1), rs) << 24);
+            }
+        } else if constexpr (MODE == Q_E4M3_B128 || MODE == Q_MXFP8) {
+            const float s = bs[i];
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const uint32_t w0 = v[i][2 * q], w1 = v[i][2 * q + 1];
+                c[i][q] = cvt_e4m3x2(__fmul_rn(bf_lo(w0), s), __fmul_rn(bf_hi(w0), s)) |
+                          (cvt_e4m3x2(__fmul_rn(bf_lo(w1), s), __fmul_rn(bf_hi(w1), s)) << 16);
+            }
+        } else {  // MXFP4: element 2i in the low nibble
+            const float s = bs[i];
+#pragma unroll
+            for (int q = 0; q < 2; q++) {
+                uint32_t word = 0u;
+#pragma unroll
+                for (int h = 0; h < 4; h++) {
+                    const uint32_t wv = v[i][4 * q + h];
+                    word |= cvt_e2m1x2(__fmul_rn(bf_lo(wv), s), __fmul_rn(bf_hi(wv), s)) << (8 * h);
+                }
+                c[i][q] = word;
+            }
+        }
+    }
+
+    if (!active) return;
+    // scatter to every destination row
+    for (int k = 0; k < a.K; k++) {
+        const int64_t row = s_row[grp][k];
+        if (row < 0) continue;
+        uint8_t *dst = a.out + row * a.D;
+        uint8_t *sdst = a.out + a.scale_off + row * a.S;
+#pragma unroll
+        for (int i = 0; i < GMAX; i++) {
+            const int g = i * TPT + lt;
+            if (g >= ngran) continue;
+            uint8_t *p = dst + (int64_t)g * OB;
+            if constexpr (OB == 32) {
+                st_v4(p, make_uint4(c[i][0], c[i][1], c[i][2], c[i][3]));
+                st_v4(p + 16, make_uint4(c[i][4], c[i][5], c[i][6], c[i][7]));
+            } else if constexpr (OB == 16) {
+                st_v4(p, make_uint4(c[i][0], c[i][1], c[i][2], c[i][3]));
+            } else {
+                st_v2(p, make_uint2(c[i][0], c[i][1]));
+            }
+            if constexpr (MODE == Q_E4M3_B128) {
+                if ((g & 7) == 0) reinterpret_cast<float *>(sdst)[g >> 3] = bsinv[i];
+            }
+            if constexpr (MODE == Q_MXFP8 || MODE == Q_MXFP4) {
+                if ((g & 1) == 0) sdst[g >> 1] = (uint8_t)bx[i];
+            }
+        }
+        if constexpr (MODE == Q_INT8) {
+            if (lt == 0) *reinterpret_cast<float *>(sdst) = rsinv;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Combine backward ("EP dispatch with unfused MXFP8 quantization",
+// Description): row(n,k) <- MXFP8(w[n,k] * g[n,:]).  The block maximum of
+// |fl(w*g_h)| equals fl(|w| * max|g_h|) because rounding is monotone and sign
+// symmetric, so it is taken once per token and scaled per entry.
+template <int TPT, int GMAX>
+__global__ void __launch_bounds__(kDispatchThreads) combine_bwd_kernel(DispatchArgs a) {
+    constexpr int TOKS = kDispatchThreads / TPT;
+    __shared__ int64_t s_row[TOKS][16];
+    __shared__ float s_w[TOKS][16];
+
+    const int grp = threadIdx.x / TPT, lt = threadIdx.x % TPT;
+    const int64_t n = (int64_t)blockIdx.x * TOKS + grp;
+    const bool active = n < a.N;
+    const int ngran = a.H >> 4;
+
+    if (active && lt < a.K) {
+        uint32_t flags = 0;
+        const int64_t row = entry_row(a, n, lt, flags);
+        if (flags) atomicOr(a.status, flags);
+        s_row[grp][lt] = row;
+        s_w[grp][lt] = a.unweighted ? 1.0f : a.wts[n * a.K + lt];
+    }
+
+    uint32_t v[GMAX][8];
+    float gmax[GMAX];
+#pragma unroll
+    for (int i = 0; i < GMAX; i++) {
+        const int g = i * TPT + lt;
+        if (active && g < ngran) {
+            const uint16_t *p = a.x + n * a.H + (int64_t)g * 16;
+            const uint4 u0 = ld_stream(p), u1 = ld_stream(p + 8);
+            v[i][0] = u0.x; v[i][1] = u0.y; v[i][2] = u0.z; v[i][3] = u0.w;
+            v[i][4] = u1.x; v[i][5] = u1.y; v[i][6] = u1.z; v[i][7] = u1.w;
+        } else {
+#pragma unroll
+            for (int q = 0; q < 8; q++) v[i][q] = 0u;
+        }
+        uint32_t m = 0u;
+#pragma unroll
+        for (int q = 0; q < 8; q++) m = bf2_absmax(m, v[i][q]);
+        float f = bf2_fold(m);
+        gmax[i] = fmaxf(f, __shfl_xor_sync(kFull, f, 1));
+    }
+    __syncthreads();
+    if (!active) return;
+
+    for (int k = 0; k < a.K; k++) {
+        const int64_t row = s_row[grp][k];
+        if (row < 0) continue;
+        const float w = s_w[grp][k];
+        const float aw = fabsf(w);
+        uint8_t *dst = a.out + row * (int64_t)a.H;
+        uint8_t *sdst = a.out + a.scale_off + row * (int64_t)(a.H >> 5);
+#pragma unroll
+        for (int i = 0; i < GMAX; i++) {
+            const int g = i * TPT + lt;
+            if (g >= ngran) continue;
+            const float amax = a.unweighted ? gmax[i] : __fmul_rn(aw, gmax[i]);
+            const int X = mx_exponent(amax, 448.0f);
+            const float s = exp2_neg(X);
+            uint32_t cw[4];
+#pragma unroll
+            for (int q = 0; q < 4; q++) {
+                const uint32_t w0 = v[i][2 * q], w1 = v[i][2 * q + 1];
+                float p0 = bf_lo(w0), p1 = bf_hi(w0), p2 = bf_lo(w1), p3 = bf_hi(w1);
+                if (!a.unweighted) {
+                    p0 = __fmul_rn(w, p0); p1 = __fmul_rn(w, p1);
+                    p2 = __fmul_rn(w, p2); p3 = __fmul_rn(w, p3);
+                }
+                cw[q] = cvt_e4m3x2(__fmul_rn(p0, s), __fmul_rn(p1, s)) |
+                        (cvt_e4m3x2(__fmul_rn(p2, s), __fmul_rn(p3, s)) << 16);
+            }
+            st_v4(dst + (int64_t)g * 16, make_uint4(cw[0], cw[1], cw[2], cw[3]));
+            if ((g & 1) == 0) sdst[g >> 1] = (uint8_t)(X + 127);
+        }
+    }
+}
+
+}  // namespace ep

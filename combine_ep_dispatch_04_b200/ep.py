@@ -1,0 +1,288 @@
+"""Thin Python binding of libep (include/ep.h): argument checks and marshalling.
+
+Every step of the path runs in libep's CUDA kernels; this module only turns
+torch tensors into device pointers and the caller's stream into a
+cudaStream_t.  Tensor checks follow "DeepEP topk_idx_t Custom Dtype
+Requirements" (Tensor Requirements and Constraints: exact dtype, 2-D,
+contiguous, matching top-k, checked before any GPU work) and "EP dispatch
+with unfused MXFP8 quantization" (Changes: a pre-quantised input is
+rejected -- x must be bfloat16).  If libep.so is missing the import fails:
+there is no fallback path.
+"""
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libep.so")
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libep.so not built at {LIB_PATH}: run combine_ep_dispatch_04_b200/build.py")
+lib = C.CDLL(LIB_PATH)
+
+QUANT = {"bf16": 0, "e4m3_b128": 1, "int8_token": 2, "mxfp8": 3, "mxfp4": 4}
+LAYOUT = {"padded": 0, "packed": 1}
+DEV_BAD_INDEX = 0x1
+DEV_CAPACITY_OVERFLOW = 0x2
+F_BWD_UNWEIGHTED = 0x1
+F_LAYOUT_SINGLE_CTA = 0x100
+F_LAYOUT_MULTI_CTA = 0x200
+
+STATUS = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_UNSUPPORTED", 3: "EP_ERR_MISALIGNED",
+          4: "EP_ERR_CUDA", 5: "EP_ERR_DEVICE_STATUS", 6: "EP_ERR_TIMEOUT"}
+
+
+class EpError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        msg = lib.ep_status_string(status).decode()
+        super().__init__(f"{where}: {STATUS.get(status, status)} ({msg})")
+
+
+class EpConfig(C.Structure):
+    _fields_ = [("num_ranks", C.c_int32), ("num_tokens", C.c_int32),
+                ("max_tokens_per_rank", C.c_int32), ("num_topk", C.c_int32),
+                ("num_experts", C.c_int32), ("hidden", C.c_int32), ("quant", C.c_int32),
+                ("layout", C.c_int32), ("expert_align", C.c_int32), ("e4m3_qmax", C.c_float),
+                ("flags", C.c_uint32)]
+
+
+class EpSizes(C.Structure):
+    _fields_ = [(n, C.c_int64) for n in (
+        "rows", "data_row_bytes", "scale_row_bytes", "recv_scale_offset", "recv_bytes",
+        "src_info_bytes", "recv_weights_bytes", "expert_out_bytes", "grad_scale_offset",
+        "grad_bytes", "workspace_bytes", "token_slot_bytes", "is_token_in_rank_bytes")]
+
+
+_P = C.c_void_p
+_CFG = C.POINTER(EpConfig)
+lib.ep_status_string.restype = C.c_char_p
+lib.ep_status_string.argtypes = [C.c_int]
+lib.ep_buffer_sizes.restype = C.c_int
+lib.ep_buffer_sizes.argtypes = [_CFG, C.POINTER(EpSizes)]
+lib.ep_dispatch_layout.restype = C.c_int
+lib.ep_dispatch_layout.argtypes = [_CFG] + [_P] * 11
+lib.ep_dispatch.restype = C.c_int
+lib.ep_dispatch.argtypes = [_CFG] + [_P] * 10
+lib.ep_combine.restype = C.c_int
+lib.ep_combine.argtypes = [_CFG] + [_P] * 8
+lib.ep_combine_backward.restype = C.c_int
+lib.ep_combine_backward.argtypes = [_CFG] + [_P] * 8
+lib.ep_get_status.restype = C.c_int
+lib.ep_get_status.argtypes = [_P, C.POINTER(C.c_uint32), _P]
+lib.ep_copy.restype = C.c_int
+lib.ep_copy.argtypes = [_P, _P, C.c_size_t, _P]
+lib.ep_cvt_sweep.restype = C.c_int
+lib.ep_cvt_sweep.argtypes = [C.c_int32, C.c_uint32, C.c_int64, _P, _P]
+lib.ep_kernel_launches.restype = C.c_uint64
+lib.ep_kernel_launches.argtypes = []
+
+
+def make_config(R, T, M, K, E, H, quant="bf16", layout="padded", expert_align=1, e4m3_qmax=0.0,
+                flags=0):
+    q = QUANT[quant] if isinstance(quant, str) else int(quant)
+    lay = LAYOUT[layout] if isinstance(layout, str) else int(layout)
+    return EpConfig(R, T, M, K, E, H, q, lay, expert_align, float(e4m3_qmax), flags)
+
+
+def _check(st, where):
+    if st != 0:
+        raise EpError(st, where)
+
+
+def ep_buffer_sizes(cfg):
+    s = EpSizes()
+    _check(lib.ep_buffer_sizes(C.byref(cfg), C.byref(s)), "ep_buffer_sizes")
+    return {n: getattr(s, n) for n, _ in EpSizes._fields_}
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, name, dtype, shape=None, optional=False):
+    """Device pointer of a contiguous CUDA tensor of the given dtype (and shape)."""
+    if t is None:
+        if optional:
+            return None
+        raise ValueError(f"{name} is required")
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return C.c_void_p(t.data_ptr())
+
+
+def _bytes(t, name, nbytes, optional=False):
+    """Device pointer of a contiguous CUDA byte buffer of at least nbytes."""
+    if t is None and optional:
+        return None
+    if t is None or not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if t.numel() * t.element_size() < nbytes:
+        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, needs {nbytes}")
+    return C.c_void_p(t.data_ptr())
+
+
+def _nk(cfg):
+    return cfg.num_ranks * cfg.num_tokens, cfg.num_topk
+
+
+def ep_dispatch_layout(cfg, topk_idx, token_slot, recv_count, workspace, dev_status,
+                       tokens_per_rank=None, tokens_per_expert=None, is_token_in_rank=None,
+                       expert_offset=None, cumulative_recv_stats=None, stream=None):
+    N, K = _nk(cfg)
+    R, E = cfg.num_ranks, cfg.num_experts
+    sz = ep_buffer_sizes(cfg)
+    args = [
+        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(tokens_per_rank, "tokens_per_rank", torch.int32, (R, R), optional=True),
+        _dev(tokens_per_expert, "tokens_per_expert", torch.int32, (R, E), optional=True),
+        _dev(is_token_in_rank, "is_token_in_rank", torch.uint8, (N, R), optional=True),
+        _dev(token_slot, "token_slot", torch.int32, (N, K)),
+        _dev(recv_count, "recv_count", torch.int64, (E,)),
+        _dev(expert_offset, "expert_offset", torch.int64, (E + 1,),
+             optional=cfg.layout == LAYOUT["padded"]),
+        _dev(cumulative_recv_stats, "cumulative_recv_stats", torch.int64, (E,), optional=True),
+        _bytes(workspace, "workspace", sz["workspace_bytes"]),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    _check(lib.ep_dispatch_layout(C.byref(cfg), *args), "ep_dispatch_layout")
+
+
+def ep_dispatch(cfg, x, topk_idx, token_slot, recv_buf, src_info, dev_status, topk_weights=None,
+                expert_offset=None, recv_weights=None, stream=None):
+    N, K = _nk(cfg)
+    sz = ep_buffer_sizes(cfg)
+    args = [
+        _dev(x, "x", torch.bfloat16, (N, cfg.hidden)),
+        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(topk_weights, "topk_weights", torch.float32, (N, K), optional=True),
+        _dev(token_slot, "token_slot", torch.int32, (N, K)),
+        _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
+             optional=cfg.layout == LAYOUT["padded"]),
+        _bytes(recv_buf, "recv_buf", sz["recv_bytes"]),
+        _bytes(src_info, "src_info", sz["src_info_bytes"]),
+        _bytes(recv_weights, "recv_weights", sz["recv_weights_bytes"], optional=True),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    _check(lib.ep_dispatch(C.byref(cfg), *args), "ep_dispatch")
+
+
+def ep_combine(cfg, y, topk_idx, topk_weights, token_slot, out, dev_status, expert_offset=None,
+               stream=None):
+    N, K = _nk(cfg)
+    sz = ep_buffer_sizes(cfg)
+    if y is None or y.dtype != torch.bfloat16:
+        raise TypeError("y (expert outputs) must be bfloat16")
+    args = [
+        _bytes(y, "y", sz["expert_out_bytes"]),
+        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(topk_weights, "topk_weights", torch.float32, (N, K)),
+        _dev(token_slot, "token_slot", torch.int32, (N, K)),
+        _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
+             optional=cfg.layout == LAYOUT["padded"]),
+        _dev(out, "out", torch.bfloat16, (N, cfg.hidden)),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    _check(lib.ep_combine(C.byref(cfg), *args), "ep_combine")
+
+
+def ep_combine_backward(cfg, g, topk_idx, topk_weights, token_slot, grad_buf, dev_status,
+                        expert_offset=None, stream=None):
+    N, K = _nk(cfg)
+    sz = ep_buffer_sizes(cfg)
+    args = [
+        _dev(g, "g", torch.bfloat16, (N, cfg.hidden)),
+        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(topk_weights, "topk_weights", torch.float32, (N, K),
+             optional=bool(cfg.flags & F_BWD_UNWEIGHTED)),
+        _dev(token_slot, "token_slot", torch.int32, (N, K)),
+        _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
+             optional=cfg.layout == LAYOUT["padded"]),
+        _bytes(grad_buf, "grad_buf", sz["grad_bytes"]),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    _check(lib.ep_combine_backward(C.byref(cfg), *args), "ep_combine_backward")
+
+
+def ep_get_status(dev_status, stream=None):
+    """Synchronise, read and clear the device status word; returns its bits."""
+    flags = C.c_uint32(0)
+    st = lib.ep_get_status(_dev(dev_status, "dev_status", torch.int32, (1,)), C.byref(flags),
+                           _stream(stream))
+    if st not in (0, 5):
+        raise EpError(st, "ep_get_status")
+    return flags.value
+
+
+def ep_copy(dst, src, stream=None):
+    n = src.numel() * src.element_size()
+    _check(lib.ep_copy(_bytes(dst, "dst", n), _bytes(src, "src", n), n, _stream(stream)),
+           "ep_copy")
+
+
+def ep_cvt_sweep(fmt, start, out, stream=None):
+    _check(lib.ep_cvt_sweep(fmt, start, out.numel(), _dev(out, "out", torch.uint8), _stream(stream)),
+           "ep_cvt_sweep")
+
+
+def ep_kernel_launches():
+    return int(lib.ep_kernel_launches())
+
+
+class Buffers:
+    """Caller-owned device buffers for one configuration (plain torch allocations)."""
+
+    def __init__(self, cfg, device="cuda", recv_weights=False, expert_out=True, grad=False):
+        sz = ep_buffer_sizes(cfg)
+        self.sizes = sz
+        N, K = _nk(cfg)
+        R, E, H = cfg.num_ranks, cfg.num_experts, cfg.hidden
+        u8 = dict(dtype=torch.uint8, device=device)
+        self.tokens_per_rank = torch.empty((R, R), dtype=torch.int32, device=device)
+        self.tokens_per_expert = torch.empty((R, E), dtype=torch.int32, device=device)
+        self.is_token_in_rank = torch.empty((N, R), **u8)
+        self.token_slot = torch.empty((N, K), dtype=torch.int32, device=device)
+        self.recv_count = torch.empty(E, dtype=torch.int64, device=device)
+        self.expert_offset = torch.empty(E + 1, dtype=torch.int64, device=device) \
+            if cfg.layout == LAYOUT["packed"] else None
+        self.workspace = torch.empty(sz["workspace_bytes"], **u8)
+        self.recv_buf = torch.empty(sz["recv_bytes"], **u8)
+        self.src_info = torch.empty(sz["rows"], dtype=torch.int32, device=device)
+        self.recv_weights = torch.empty(sz["rows"], dtype=torch.float32, device=device) \
+            if recv_weights else None
+        self.y = torch.empty((sz["rows"], H), dtype=torch.bfloat16, device=device) \
+            if expert_out else None
+        self.out = torch.empty((N, H), dtype=torch.bfloat16, device=device)
+        self.grad_buf = torch.empty(sz["grad_bytes"], **u8) if grad else None
+        self.dev_status = torch.zeros(1, dtype=torch.int32, device=device)
+
+    def recv_data(self):
+        """View of the data region: [rows, D] bytes."""
+        s = self.sizes
+        return self.recv_buf[: s["rows"] * s["data_row_bytes"]].view(s["rows"], s["data_row_bytes"])
+
+    def recv_scale(self):
+        s = self.sizes
+        a = s["recv_scale_offset"]
+        return self.recv_buf[a: a + s["rows"] * s["scale_row_bytes"]].view(s["rows"], s["scale_row_bytes"])
+
+    def grad_data(self, H):
+        s = self.sizes
+        return self.grad_buf[: s["rows"] * H].view(s["rows"], H)
+
+    def grad_scale(self, H):
+        s = self.sizes
+        a = s["grad_scale_offset"]
+        return self.grad_buf[a: a + s["rows"] * (H // 32)].view(s["rows"], H // 32)

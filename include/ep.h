@@ -1,0 +1,218 @@
+/*
+ * ep.h -- C ABI of libep: MoE expert-parallel token dispatch and combine on
+ * one NVIDIA B200 (sm_100a).
+ *
+ * On one GPU the R "ranks" of expert parallelism are logical partitions of
+ * buffers that all sit in this GPU's memory: no inter-GPU traffic exists.
+ * Token n = r*T + t is token t of source rank r.  Expert e (of E) lives on
+ * rank e / L, L = E / R, as local expert e % L.
+ *
+ * Page citations (title, section):
+ *   [LL]  "Low-Latency Mode API" (DeepEP-Ascend docs): low_latency_dispatch
+ *         and low_latency_combine -- Parameters, Return Values, Constraints.
+ *   [FP8] "DeepEP FP8 Dispatch and Combine Operations: Low-Precision
+ *         All-to-All for MoE": The Dispatch Stage, The FP8 Combine Operation.
+ *   [TE]  "[Common][PyTorch] EP dispatch with unfused MXFP8 quantization"
+ *         (TransformerEngine PR): Description, Changes.
+ *   [IDX] "DeepEP topk_idx_t Custom Dtype Requirements": Tensor Requirements
+ *         and Constraints, Runtime Validation.
+ *   [A5]  "[feat] A5 deep fused moe supported" (sgl-kernel-npu PR): review
+ *         comments on tiling validation.
+ *
+ * Conventions for every entry point:
+ *   - Pointers are DEVICE pointers unless stated; every buffer is allocated
+ *     and owned by the caller.  The library allocates no device memory and
+ *     keeps no per-call state.
+ *   - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) and is asynchronous; outputs are valid in stream order.
+ *   - Host-side checks run before any launch and before any division by a
+ *     caller value ([A5] review: validate before dividing); a failed check
+ *     returns an error and launches nothing.  Vector buffers (x, y, out,
+ *     recv_buf, grad_buf) must be 16-byte aligned (EP_ERR_MISALIGNED).
+ *   - Conditions found on the device (an expert index outside [-1, E), a
+ *     slot beyond the receive capacity) never trap: the offending entry is
+ *     skipped and a bit is OR-ed into *dev_status (a caller-owned uint32_t in
+ *     device memory, zero before first use).  ep_get_status reads it.
+ *   - Combine and combine-backward must be given the configuration and the
+ *     layout outputs (token_slot, expert_offset) of the dispatch whose rows
+ *     they read ([LL] low_latency_combine: indices must match dispatch; the
+ *     handle is passed unchanged).
+ */
+#ifndef EP_H
+#define EP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *ep_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    EP_OK = 0,
+    EP_ERR_INVALID_ARG = 1,   /* a size, enum or pointer argument is out of range */
+    EP_ERR_UNSUPPORTED = 2,   /* valid request outside what this build implements */
+    EP_ERR_MISALIGNED = 3,    /* a vector buffer is not 16-byte aligned */
+    EP_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, copy, sync) */
+    EP_ERR_DEVICE_STATUS = 5, /* ep_get_status found device-side error bits */
+    EP_ERR_TIMEOUT = 6        /* reserved for bounded waits (multi-GPU); not produced */
+} ep_status_t;
+
+/* Quantisation of dispatched rows.  Values 2..4 equal the DeepEP-Ascend
+ * quant_mode numbers ([LL] use_fp8 / use_ue8m0 / use_mxfp4). */
+typedef enum {
+    EP_Q_BF16 = 0,       /* plain bf16 rows ([LL] use_fp8=False) */
+    EP_Q_E4M3_B128 = 1,  /* e4m3 + one fp32 scale_inv per 128 elements ([FP8] Dispatch Stage) */
+    EP_Q_INT8_TOKEN = 2, /* int8 + one fp32 scale per row ([LL] use_fp8, quant_mode 2) */
+    EP_Q_MXFP8 = 3,      /* e4m3 + one e8m0 byte per 32 elements ([LL] use_ue8m0; [TE]) */
+    EP_Q_MXFP4 = 4       /* e2m1 x2 per byte + one e8m0 byte per 32 ([LL] use_mxfp4) */
+} ep_quant_t;
+
+/* Receive-buffer layouts. */
+typedef enum {
+    EP_LAYOUT_PADDED = 0, /* [R][L][R*M] rows: per rank [L, R*M, H] ([LL] combine x) */
+    EP_LAYOUT_PACKED = 1  /* rows of expert e at expert_offset[e] .. ([TE] grouped tensor) */
+} ep_layout_t;
+
+/* Bits of *dev_status. */
+#define EP_DEV_BAD_INDEX 0x1u         /* topk_idx value < -1 or >= E (entry skipped) */
+#define EP_DEV_CAPACITY_OVERFLOW 0x2u /* slot >= R*M in the padded layout (row skipped) */
+
+/* ep_config_t.flags */
+#define EP_F_BWD_UNWEIGHTED 0x1u    /* combine-backward re-dispatches g without w */
+#define EP_F_LAYOUT_SINGLE_CTA 0x100u /* force the one-block layout path */
+#define EP_F_LAYOUT_MULTI_CTA 0x200u  /* force the multi-block layout path */
+
+typedef struct {
+    int32_t num_ranks;           /* R > 0 */
+    int32_t num_tokens;          /* T tokens per rank, 0 <= T <= M */
+    int32_t max_tokens_per_rank; /* M > 0 ([LL] num_max_dispatch_tokens_per_rank) */
+    int32_t num_topk;            /* K in [1, 16] ([LL] Constraints) */
+    int32_t num_experts;         /* E in [1, 1024], E % R == 0 */
+    int32_t hidden;              /* H in [32, 8192], H % 32 == 0; % 128 for E4M3_B128 */
+    int32_t quant;               /* ep_quant_t */
+    int32_t layout;              /* ep_layout_t */
+    int32_t expert_align;        /* packed layout: rows per expert rounded up to this (>= 1) */
+    float e4m3_qmax;             /* E4M3_B128 target max, (0, 448]; 0 selects 448 */
+    uint32_t flags;              /* EP_F_* */
+} ep_config_t;
+
+/* Byte sizes of the caller-owned buffers for one configuration.  "rows" is
+ * the row capacity of every receive-layout buffer: E*R*M (padded) or
+ * R*T*K + E*(expert_align-1) (packed, enough for every entry). */
+typedef struct {
+    int64_t rows;
+    int64_t data_row_bytes;     /* D: 2H bf16, H int8/e4m3, H/2 e2m1 */
+    int64_t scale_row_bytes;    /* S: 0 bf16, 4 int8, 4*H/128 e4m3_b128, H/32 mx */
+    int64_t recv_scale_offset;  /* recv_buf: data region [rows][D] then, here, scales [rows][S] */
+    int64_t recv_bytes;
+    int64_t src_info_bytes;     /* int32 [rows] */
+    int64_t recv_weights_bytes; /* float [rows] */
+    int64_t expert_out_bytes;   /* y for ep_combine: bf16 [rows][H] */
+    int64_t grad_scale_offset;  /* grad_buf: e4m3 [rows][H] then e8m0 [rows][H/32] here */
+    int64_t grad_bytes;
+    int64_t workspace_bytes;    /* scratch for ep_dispatch_layout */
+    int64_t token_slot_bytes;   /* int32 [N][K] */
+    int64_t is_token_in_rank_bytes; /* uint8 [N][R] */
+} ep_sizes_t;
+
+/* Buffer sizes for `cfg` (validates it).  Host only; no device work. */
+ep_status_t ep_buffer_sizes(const ep_config_t *cfg, ep_sizes_t *out);
+
+/*
+ * Routing layout and slot assignment ([LL] low_latency_dispatch: topk_idx
+ * [num_tokens, num_topk] int64, -1 = no expert; recv_count [num_local_experts]
+ * int64; cumulative_local_expert_recv_stats).
+ *   topk_idx            int64 [N][K], N = R*T
+ *   tokens_per_rank     int32 [R][R]: tokens of src r with >= 1 expert on rank d (nullable)
+ *   tokens_per_expert   int32 [R][E]: entries of src r routed to e (nullable)
+ *   is_token_in_rank    uint8 [N][R]: 1 if token n has an expert on rank d (nullable)
+ *   token_slot          int32 [N][K]: rank of entry (n,k) among its expert's entries
+ *                       ordered by (source rank, token, k); -1 when masked
+ *   recv_count          int64 [E]
+ *   expert_offset       int64 [E+1]: exclusive scan of recv_count rounded up to
+ *                       expert_align (required for PACKED, nullable for PADDED)
+ *   cumulative_recv_stats int64 [E]: += recv_count (nullable; [LL] load-balance stats)
+ *   workspace           ep_sizes_t.workspace_bytes of scratch (contents undefined after)
+ * Deterministic: the result never depends on thread timing.
+ */
+ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const int64_t *topk_idx,
+                               int32_t *tokens_per_rank, int32_t *tokens_per_expert,
+                               uint8_t *is_token_in_rank, int32_t *token_slot,
+                               int64_t *recv_count, int64_t *expert_offset,
+                               int64_t *cumulative_recv_stats, void *workspace,
+                               uint32_t *dev_status, ep_stream_t stream);
+
+/*
+ * Quantise each token once and scatter it to its experts' receive rows
+ * ([LL] low_latency_dispatch Return Values; [FP8] The Dispatch Stage; [TE]
+ * Changes: data region then scale region in one caller buffer).
+ *   x              bf16 [N][H]
+ *   topk_idx       int64 [N][K]; token_slot/expert_offset from ep_dispatch_layout
+ *   topk_weights   float [N][K] (nullable; needed for recv_weights)
+ *   recv_buf       ep_sizes_t.recv_bytes: row (e, slot) holds the token's
+ *                  quantised row; padded row = e*R*M + slot, packed row =
+ *                  expert_offset[e] + slot.  Rows without an entry are not written.
+ *   src_info       int32 [rows]: r*M + t of the row's source token
+ *   recv_weights   float [rows] (nullable): the entry's top-k weight
+ */
+ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const int64_t *topk_idx,
+                        const float *topk_weights, const int32_t *token_slot,
+                        const int64_t *expert_offset, void *recv_buf, int32_t *src_info,
+                        float *recv_weights, uint32_t *dev_status, ep_stream_t stream);
+
+/*
+ * Weighted top-k combine ([LL] low_latency_combine: combined_x [T, H] bf16 is
+ * the weighted sum across experts; `out` written in place):
+ *   out[n,:] = bf16_rne( sum over valid k = 0..K-1, in order, of
+ *                        w[n,k] * y[row(n,k), :] )
+ * accumulated in fp32 with one fused multiply-add per term.  Masked entries
+ * add nothing; a token with no valid entry gets +0.  Weights are used as given.
+ *   y      bf16 [rows][H] expert outputs in the receive layout
+ *   out    bf16 [N][H]
+ */
+ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t *topk_idx,
+                       const float *topk_weights, const int32_t *token_slot,
+                       const int64_t *expert_offset, uint16_t *out, uint32_t *dev_status,
+                       ep_stream_t stream);
+
+/*
+ * Combine backward ([TE] Description: the result gradient goes back to the
+ * expert positions through the reverse dispatch, quantised to MXFP8): for
+ * each valid entry, row(n,k) of grad_buf receives MXFP8(w[n,k] * g[n,:])
+ * (MXFP8(g[n,:]) with EP_F_BWD_UNWEIGHTED).  cfg->quant is ignored: the
+ * gradient is always MXFP8.
+ *   g          bf16 [N][H]
+ *   grad_buf   ep_sizes_t.grad_bytes: e4m3 [rows][H] then e8m0 [rows][H/32]
+ */
+ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
+                                const int64_t *topk_idx, const float *topk_weights,
+                                const int32_t *token_slot, const int64_t *expert_offset,
+                                void *grad_buf, uint32_t *dev_status, ep_stream_t stream);
+
+/* Synchronise `stream`, read *dev_status into *host_flags (host pointer) and
+ * clear it.  Returns EP_ERR_DEVICE_STATUS when any bit was set. */
+ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream);
+
+/* Static description of a status code. */
+const char *ep_status_string(ep_status_t status);
+
+/* ---- diagnostics ---------------------------------------------------------
+ * ep_copy: a plain 16-byte-vector device copy, the same-run HBM bandwidth
+ * reference for the kernels above (bytes % 16 == 0, both pointers aligned).
+ * ep_cvt_sweep: out[i] = the kernels' conversion of the binary32 value with
+ * bit pattern start+i (format 0: e4m3 satfinite byte; 1: e2m1 satfinite code
+ * in the low nibble), for checking the hardware conversion against the
+ * format definition.
+ * ep_kernel_launches: kernels launched by this library in this process. */
+ep_status_t ep_copy(void *dst, const void *src, size_t bytes, ep_stream_t stream);
+ep_status_t ep_cvt_sweep(int32_t format, uint32_t start, int64_t n, uint8_t *out,
+                         ep_stream_t stream);
+uint64_t ep_kernel_launches(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* EP_H */

@@ -59,6 +59,10 @@ _lib.orc_combine.restype = C.c_uint32
 _lib.orc_combine.argtypes = [_i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p]
 _lib.orc_combine_bwd.restype = C.c_uint32
 _lib.orc_combine_bwd.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]
+_lib.orc_bwd_row.restype = None
+_lib.orc_bwd_row.argtypes = [_i, _f, _i, _p, _p, _p]
+_lib.orc_combine_gathered.restype = None
+_lib.orc_combine_gathered.argtypes = [_l, _i, _i, _p, _p, _p, _p]
 for _n in ("orc_e4m3_encode_array", "orc_e2m1_encode_array"):
     getattr(_lib, _n).restype = None
     getattr(_lib, _n).argtypes = [_p, _p, _l]
@@ -201,26 +205,35 @@ def layout(R, T, K, E, M, topk_idx, layout="padded", align=1):
     return out
 
 
+def dispatch_buffers(R, T, K, E, M, H, mode, layout="padded", align=1, weights=False, fill=True):
+    """Output arrays for dispatch().  With fill, rows keep 0xAB bytes / -7 / nan
+    until written, so tests can see which rows were written; without, the
+    arrays are left uninitialised (only written rows are touched)."""
+    rows = rows_max(R, T, K, E, M, layout, align)
+    D, S = row_bytes(_mode(mode), H)
+    mk = (lambda shape, dt, v: np.full(shape, v, dt)) if fill else \
+        (lambda shape, dt, v: np.empty(shape, dt))
+    return dict(recv_data=mk((rows, D), np.uint8, 0xAB),
+                recv_scale=mk((rows, max(S, 1)), np.uint8, 0xAB),
+                src_info=mk(rows, np.int32, -7),
+                recv_weights=mk(rows, np.float32, np.nan) if weights else None)
+
+
 def dispatch(R, T, K, E, M, H, mode, x, topk_idx, token_slot, expert_offset=None,
-             topk_weights=None, layout="padded", align=1, e4m3_qmax=0.0):
+             topk_weights=None, layout="padded", align=1, e4m3_qmax=0.0, out=None):
     """Returns dict(recv_data [rows, D] u8, recv_scale [rows, S] u8, src_info, recv_weights, status).
 
-    Rows without an entry keep the fill value (0xAB bytes / -7 / nan) so that
-    tests can see that they were not written."""
+    `out` may hold arrays from dispatch_buffers(); otherwise they are made here."""
     m = _mode(mode)
-    rows = rows_max(R, T, K, E, M, layout, align)
     D, S = row_bytes(m, H)
     x = _c(x, np.uint16).reshape(R * T, H)
     idx = _c(topk_idx, np.int64)
     slot = _c(token_slot, np.int32)
     eo = None if expert_offset is None else _c(expert_offset, np.int64)
     w = None if topk_weights is None else _c(topk_weights, np.float32)
-    out = dict(
-        recv_data=np.full((rows, D), 0xAB, np.uint8),
-        recv_scale=np.full((rows, max(S, 1)), 0xAB, np.uint8),
-        src_info=np.full(rows, -7, np.int32),
-        recv_weights=np.full(rows, np.nan, np.float32) if w is not None else None,
-    )
+    if out is None:
+        out = dispatch_buffers(R, T, K, E, M, H, m, layout, align, weights=w is not None)
+    out = dict(out)
     st = _lib.orc_dispatch(R, T, K, E, M, H, m, float(e4m3_qmax), _layout(layout), _ptr(x),
                            _ptr(idx), _ptr(w), _ptr(slot), _ptr(eo), _ptr(out["recv_data"]),
                            _ptr(out["recv_scale"]), _ptr(out["src_info"]), _ptr(out["recv_weights"]))
@@ -230,14 +243,15 @@ def dispatch(R, T, K, E, M, H, mode, x, topk_idx, token_slot, expert_offset=None
 
 
 def combine(R, T, K, E, M, H, y, topk_idx, topk_weights, token_slot, expert_offset=None,
-            layout="padded"):
+            layout="padded", out=None):
     """y: expert outputs, bf16 bits [rows, H] in the receive layout.  Returns (out [N, H] u16, status)."""
     y = _c(y, np.uint16)
     idx = _c(topk_idx, np.int64)
     w = _c(topk_weights, np.float32)
     slot = _c(token_slot, np.int32)
     eo = None if expert_offset is None else _c(expert_offset, np.int64)
-    out = np.zeros((R * T, H), np.uint16)
+    if out is None:
+        out = np.zeros((R * T, H), np.uint16)
     st = _lib.orc_combine(R, T, K, E, M, H, _layout(layout), _ptr(y), _ptr(idx), _ptr(w),
                           _ptr(slot), _ptr(eo), _ptr(out))
     return out, int(st)
@@ -269,3 +283,25 @@ def combine_bwd(R, T, K, E, M, H, g, topk_idx, topk_weights, token_slot, expert_
     st = _lib.orc_combine_bwd(R, T, K, E, M, H, _layout(layout), int(bool(unweighted)), _ptr(g),
                               _ptr(idx), _ptr(w), _ptr(slot), _ptr(eo), _ptr(gd), _ptr(gs))
     return dict(grad_data=gd, grad_scale=gs, status=int(st))
+
+
+def combine_gathered(yrows, w, valid):
+    """Tokens whose K expert rows are gathered: yrows [N, K, H] bf16 bits,
+    w [N, K] f32, valid [N, K] -> out [N, H] bf16 bits."""
+    yrows = _c(yrows, np.uint16)
+    N, K, H = yrows.shape
+    w = _c(w, np.float32)
+    v = _c(valid, np.uint8)
+    out = np.zeros((N, H), np.uint16)
+    _lib.orc_combine_gathered(N, K, H, _ptr(yrows), _ptr(w), _ptr(v), _ptr(out))
+    return out
+
+
+def bwd_row(g_row, w, unweighted=False):
+    """One entry of the combine backward: (e4m3 data [H], e8m0 scales [H/32])."""
+    g_row = _c(g_row, np.uint16)
+    H = g_row.size
+    d = np.zeros(H, np.uint8)
+    s = np.zeros(H // 32, np.uint8)
+    _lib.orc_bwd_row(H, float(w), int(bool(unweighted)), _ptr(g_row), _ptr(d), _ptr(s))
+    return d, s

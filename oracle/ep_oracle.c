@@ -432,6 +432,31 @@ uint32_t orc_combine(int R, int T, int K, int E, int M, int H, int layout, const
  * product one fp32 multiply); `unweighted` gives the plain re-dispatch of
  * g_n.  The row is MXFP8-quantised and written at the forward's slot.
  */
+/* One entry of the combine backward: MXFP8(w * g) (or MXFP8(g) unweighted). */
+void orc_bwd_row(int H, float w, int unweighted, const uint16_t *g, uint8_t *data, uint8_t *scale)
+{
+    float *p = (float *)malloc(sizeof(float) * (size_t)H);
+    for (int h = 0; h < H; h++) {
+        float gv = orc_bf16_to_f32(g[h]);
+        p[h] = unweighted ? gv : w * gv;
+    }
+    orc_quant_row_f32(ORC_MXFP8, H, 0.0f, p, data, scale);
+    free(p);
+}
+
+/* Combine of N tokens whose K expert rows are already gathered:
+ * yrows [N][K][H], w [N][K], valid [N][K] -> out [N][H]. */
+void orc_combine_gathered(long N, int K, int H, const uint16_t *yrows, const float *w,
+                          const uint8_t *valid, uint16_t *out)
+{
+    const uint16_t **rows = (const uint16_t **)malloc(sizeof(void *) * (size_t)K);
+    for (long n = 0; n < N; n++) {
+        for (int k = 0; k < K; k++) rows[k] = yrows + (n * K + k) * (long)H;
+        orc_combine_row(H, K, rows, w + n * K, valid + n * K, out + n * H);
+    }
+    free(rows);
+}
+
 uint32_t orc_combine_bwd(int R, int T, int K, int E, int M, int H, int layout, int unweighted,
                          const uint16_t *g, const int64_t *idx, const float *topk_weights,
                          const int32_t *token_slot, const int64_t *expert_offset,
@@ -440,7 +465,6 @@ uint32_t orc_combine_bwd(int R, int T, int K, int E, int M, int H, int layout, i
     uint32_t st = 0;
     long N = (long)R * T, cap = (long)R * M;
     long D = orc_row_data_bytes(ORC_MXFP8, H), S = orc_row_scale_bytes(ORC_MXFP8, H);
-    float *p = (float *)malloc(sizeof(float) * (size_t)H);
     for (long n = 0; n < N; n++) {
         for (int k = 0; k < K; k++) {
             int64_t e = idx[n * K + k];
@@ -448,15 +472,10 @@ uint32_t orc_combine_bwd(int R, int T, int K, int E, int M, int H, int layout, i
             if (e < 0 || e >= E || slot < 0) continue;
             long row = row_of(layout, cap, expert_offset, e, slot);
             if (row < 0) { st |= ORC_ST_CAPACITY; continue; }
-            float w = topk_weights[n * K + k];
-            for (int h = 0; h < H; h++) {
-                float gv = orc_bf16_to_f32(g[n * H + h]);
-                p[h] = unweighted ? gv : w * gv;
-            }
-            orc_quant_row_f32(ORC_MXFP8, H, 0.0f, p, grad_data + row * D, grad_scale + row * S);
+            float w = unweighted ? 1.0f : topk_weights[n * K + k];
+            orc_bwd_row(H, w, unweighted, g + n * H, grad_data + row * D, grad_scale + row * S);
         }
     }
-    free(p);
     return st;
 }
 

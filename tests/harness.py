@@ -1,0 +1,181 @@
+"""Shared helpers for the GPU parity tests: run the path on cuda:0 through the
+C ABI, and compare it with the oracle on the same seeded inputs.
+
+The oracle never sees a value produced on the device: its inputs are the host
+arrays the seeded recipes build, and expert outputs are rebuilt on the host
+from the same pool windows the device gathered."""
+import numpy as np
+import torch
+
+import combine_ep_dispatch_04_b200 as ep
+import oracle
+import synth
+
+
+def bf16_dev(a_u16):
+    return torch.from_numpy(np.ascontiguousarray(a_u16).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def to_np_u16(t):
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+class Run:
+    """One pass of layout -> dispatch -> combine (-> combine backward) on the GPU."""
+
+    def __init__(self, w, mode, layout="padded", align=1, qmax=0.0, flags=0, idx=None, wts=None,
+                 x=None, with_weights=True, backward=False, bwd_unweighted=False, stats=False,
+                 replica=0, fill=0xAB):
+        self.w, self.mode, self.layout, self.align, self.qmax = w, mode, layout, align, qmax
+        R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
+        if idx is None or wts is None:
+            i2, w2 = synth.make_routing(w, replica)
+            idx = i2 if idx is None else idx
+            wts = w2 if wts is None else wts
+        self.idx = np.ascontiguousarray(idx, np.int64)
+        self.wts = np.ascontiguousarray(wts, np.float32)
+        self.x = synth.make_x(w, replica) if x is None else np.ascontiguousarray(x, np.uint16)
+        self.cfg = ep.make_config(R, T, M, K, E, H, mode, layout, align, qmax,
+                                  flags | (ep.F_BWD_UNWEIGHTED if bwd_unweighted else 0))
+        self.bwd_unweighted = bwd_unweighted
+        b = ep.Buffers(self.cfg, recv_weights=with_weights, grad=backward)
+        self.b = b
+        b.recv_buf.fill_(fill)
+        if b.recv_weights is not None:
+            b.recv_weights.fill_(float("nan"))
+        b.src_info.fill_(-7)
+        self.sizes = b.sizes
+        N = R * T
+        self.idx_d = torch.from_numpy(self.idx).cuda()
+        self.wts_d = torch.from_numpy(self.wts).cuda()
+        self.x_d = bf16_dev(self.x)
+        self.stats_d = torch.zeros(E, dtype=torch.int64, device="cuda") if stats else None
+        ep.ep_dispatch_layout(self.cfg, self.idx_d, b.token_slot, b.recv_count, b.workspace,
+                              b.dev_status, b.tokens_per_rank, b.tokens_per_expert,
+                              b.is_token_in_rank, b.expert_offset, self.stats_d)
+        ep.ep_dispatch(self.cfg, self.x_d, self.idx_d, b.token_slot, b.recv_buf, b.src_info,
+                       b.dev_status, topk_weights=self.wts_d if with_weights else None,
+                       expert_offset=b.expert_offset, recv_weights=b.recv_weights)
+        # expert outputs: pool windows for every buffer row
+        rows = self.sizes["rows"]
+        self.y_pool, self.y_off = synth.y_source(w, rows, replica)
+        pool_d = torch.from_numpy(self.y_pool.view(np.int16)).cuda()
+        off_d = torch.from_numpy(self.y_off).cuda()
+        torch.index_select(pool_d.as_strided((synth.POOL, H), (1, 1)), 0, off_d,
+                           out=b.y.view(torch.int16))
+        del pool_d, off_d
+        b.out.fill_(1.0)
+        ep.ep_combine(self.cfg, b.y, self.idx_d, self.wts_d, b.token_slot, b.out, b.dev_status,
+                      expert_offset=b.expert_offset)
+        self.g = None
+        if backward:
+            gp, go = synth.g_source(w, replica)
+            self.g = synth.windows(gp, go, H)
+            self.g_d = bf16_dev(self.g)
+            b.grad_buf.fill_(fill)
+            ep.ep_combine_backward(self.cfg, self.g_d, self.idx_d, self.wts_d, b.token_slot,
+                                   b.grad_buf, b.dev_status, expert_offset=b.expert_offset)
+        self.status = ep.ep_get_status(b.dev_status)
+        self.lay = oracle.layout(R, T, K, E, M, self.idx, layout=layout, align=align)
+
+    # ---- comparisons ----------------------------------------------------------
+    def check_layout(self):
+        b, o = self.b, self.lay
+        assert np.array_equal(b.token_slot.cpu().numpy(), o["token_slot"])
+        assert np.array_equal(b.recv_count.cpu().numpy(), o["recv_count"])
+        assert np.array_equal(b.tokens_per_expert.cpu().numpy(), o["tokens_per_expert"])
+        assert np.array_equal(b.tokens_per_rank.cpu().numpy(), o["tokens_per_rank"])
+        assert np.array_equal(b.is_token_in_rank.cpu().numpy(), o["is_token_in_rank"])
+        if self.layout == "packed":
+            assert np.array_equal(b.expert_offset.cpu().numpy(), o["expert_offset"])
+        assert self.status == o["status"], (self.status, o["status"])
+        if self.stats_d is not None:
+            assert np.array_equal(self.stats_d.cpu().numpy(), o["recv_count"])
+
+    def entries(self, tokens=None):
+        """(n, k, row) of every valid entry of the given tokens, from the oracle layout."""
+        w, o = self.w, self.lay
+        idx = self.idx
+        n_all = np.arange(idx.shape[0]) if tokens is None else np.asarray(tokens)
+        ns, ks = np.nonzero((idx[n_all] >= 0) & (idx[n_all] < w["E"]))
+        ns = n_all[ns]
+        slots = o["token_slot"][ns, ks]
+        rows = oracle.row_index(self.layout, w["R"], w["M"], idx[ns, ks], slots, o["expert_offset"])
+        if self.layout == "padded":
+            ok = slots < w["R"] * w["M"]
+            ns, ks, rows = ns[ok], ks[ok], rows[ok]
+        return ns, ks, rows
+
+    def check_dispatch(self, tokens=None, check_unwritten=True):
+        w, b = self.w, self.b
+        ns, ks, rows = self.entries(tokens)
+        rows_d = torch.from_numpy(rows).cuda()
+        data = b.recv_data().index_select(0, rows_d).cpu().numpy()
+        S = self.sizes["scale_row_bytes"]
+        scale = b.recv_scale().index_select(0, rows_d).cpu().numpy() if S else None
+        src = b.src_info.index_select(0, rows_d).cpu().numpy()
+        expect_cache = {}
+        for i, (n, k, row) in enumerate(zip(ns, ks, rows)):
+            if n not in expect_cache:
+                expect_cache[n] = oracle.quant_row(self.mode, self.x[n], e4m3_qmax=self.qmax)
+            d, s = expect_cache[n]
+            assert np.array_equal(data[i], d), f"data row {row} (token {n}, k {k})"
+            if S:
+                assert np.array_equal(scale[i], s), f"scale row {row} (token {n}, k {k})"
+            assert src[i] == (n // w["T"]) * w["M"] + n % w["T"]
+        if b.recv_weights is not None:
+            rw = b.recv_weights.index_select(0, rows_d).cpu().numpy()
+            assert np.array_equal(rw, self.wts[ns, ks])
+        if check_unwritten and tokens is None:
+            written = (b.recv_data() != 0xAB).any(dim=1).cpu().numpy()
+            want = np.zeros(self.sizes["rows"], bool)
+            want[rows] = True
+            assert np.array_equal(written, want)
+        return len(rows)
+
+    def y_rows_host(self, rows):
+        return synth.windows(self.y_pool, self.y_off[np.asarray(rows, np.int64)], self.w["H"])
+
+    def check_combine(self, tokens=None, max_ulp=1):
+        w, b = self.w, self.b
+        K, H = w["K"], w["H"]
+        tokens = np.arange(self.idx.shape[0]) if tokens is None else np.asarray(tokens)
+        got = to_np_u16(b.out.index_select(0, torch.from_numpy(tokens).cuda()))
+        worst = 0
+        for a in range(0, len(tokens), 512):
+            tk = tokens[a:a + 512]
+            yr = np.zeros((len(tk), K, H), np.uint16)
+            valid = np.zeros((len(tk), K), np.uint8)
+            ns, ks, rows = self.entries(tk)
+            pos = {n: i for i, n in enumerate(tk)}
+            if len(rows):
+                ys = self.y_rows_host(rows)
+                for j, (n, k) in enumerate(zip(ns, ks)):
+                    yr[pos[n], k] = ys[j]
+                    valid[pos[n], k] = 1
+            want = oracle.combine_gathered(yr, self.wts[tk], valid)
+            d = ulp_distance(got[a:a + 512], want)
+            worst = max(worst, int(d.max()) if d.size else 0)
+        assert worst <= max_ulp, worst
+        return worst
+
+    def check_backward(self, tokens=None):
+        w, b = self.w, self.b
+        H = w["H"]
+        ns, ks, rows = self.entries(tokens)
+        rows_d = torch.from_numpy(rows).cuda()
+        gd = b.grad_data(H).index_select(0, rows_d).cpu().numpy()
+        gs = b.grad_scale(H).index_select(0, rows_d).cpu().numpy()
+        for i, (n, k) in enumerate(zip(ns, ks)):
+            d, s = oracle.bwd_row(self.g[n], self.wts[n, k], self.bwd_unweighted)
+            assert np.array_equal(gd[i], d), f"grad row {rows[i]} (token {n}, k {k})"
+            assert np.array_equal(gs[i], s), f"grad scale row {rows[i]}"
+        return len(rows)
+
+
+def ulp_distance(a, b):
+    """Distance in bf16 ulps between arrays of bf16 bit patterns."""
+    def key(u):
+        u = u.astype(np.int64)
+        return np.where(u & 0x8000, -(u & 0x7FFF), u)
+    return np.abs(key(a) - key(b))

@@ -1,0 +1,105 @@
+"""The C ABI without a GPU: libep.so loads, exports every function that
+include/ep.h declares, sizes buffers, and rejects invalid arguments on the
+host before any launch (no CUDA call is reached on these paths)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+import combine_ep_dispatch_04_b200 as ep
+from combine_ep_dispatch_04_b200.ep import lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(ep_[a-z0-9_]+)\s*\(", text))
+    return names
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared_functions()
+    assert {"ep_dispatch_layout", "ep_dispatch", "ep_combine", "ep_combine_backward",
+            "ep_buffer_sizes", "ep_get_status"} <= names
+    for n in sorted(names):
+        assert hasattr(lib, n), n
+
+
+def _cfg(**kw):
+    base = dict(R=8, T=128, M=128, K=8, E=256, H=7168, quant="e4m3_b128")
+    base.update(kw)
+    return ep.make_config(base["R"], base["T"], base["M"], base["K"], base["E"], base["H"],
+                          base["quant"], base.get("layout", "padded"), base.get("expert_align", 1),
+                          base.get("e4m3_qmax", 0.0), base.get("flags", 0))
+
+
+def test_sizes_padded_decode_shape():
+    s = ep.ep_buffer_sizes(_cfg())
+    assert s["rows"] == 256 * 8 * 128
+    assert s["data_row_bytes"] == 7168 and s["scale_row_bytes"] == 4 * 56
+    assert s["recv_scale_offset"] % 256 == 0
+    assert s["recv_bytes"] == s["recv_scale_offset"] + s["rows"] * 224
+    assert s["expert_out_bytes"] == s["rows"] * 7168 * 2
+    assert s["grad_bytes"] == s["grad_scale_offset"] + s["rows"] * 7168 // 32
+
+
+@pytest.mark.parametrize("quant,D,S", [("bf16", 2048, 0), ("int8_token", 1024, 4),
+                                        ("e4m3_b128", 1024, 32), ("mxfp8", 1024, 32),
+                                        ("mxfp4", 512, 32)])
+def test_sizes_packed_every_mode(quant, D, S):
+    s = ep.ep_buffer_sizes(_cfg(R=4, T=10, M=16, K=3, E=8, H=1024, quant=quant, layout="packed",
+                                expert_align=4))
+    assert s["rows"] == 4 * 10 * 3 + 8 * 3
+    assert (s["data_row_bytes"], s["scale_row_bytes"]) == (D, S)
+
+
+@pytest.mark.parametrize("bad", [
+    dict(R=0), dict(M=0), dict(T=-1), dict(T=129), dict(K=0), dict(K=17), dict(E=0),
+    dict(E=1025 * 8), dict(E=255), dict(H=0), dict(H=48), dict(H=8224), dict(H=7168 + 32),
+    dict(quant=7), dict(layout=2), dict(expert_align=0), dict(e4m3_qmax=449.0),
+    dict(e4m3_qmax=float("nan")), dict(e4m3_qmax=-1.0), dict(flags=0x8000),
+    dict(flags=ep.F_LAYOUT_MULTI_CTA | ep.F_LAYOUT_SINGLE_CTA),
+    dict(quant="e4m3_b128", H=96),
+])
+def test_invalid_configs_rejected(bad):
+    with pytest.raises(ep.EpError) as ei:
+        ep.ep_buffer_sizes(_cfg(**bad))
+    assert ei.value.status == 1
+
+
+def test_entry_points_reject_before_any_launch():
+    """Null buffers, a null config and a bad config are refused on the host:
+    these calls reach no CUDA API (there is no device here)."""
+    cfg = _cfg()
+    null = C.c_void_p(0)
+    n0 = ep.ep_kernel_launches()
+    assert lib.ep_dispatch_layout(None, *([null] * 11)) == 1
+    assert lib.ep_dispatch_layout(C.byref(cfg), *([null] * 11)) == 1
+    assert lib.ep_dispatch(C.byref(cfg), *([null] * 10)) == 1
+    assert lib.ep_combine(C.byref(cfg), *([null] * 8)) == 1
+    assert lib.ep_combine_backward(C.byref(cfg), *([null] * 8)) == 1
+    assert lib.ep_get_status(null, None, null) == 1
+    bad = _cfg(E=255)
+    fake = C.c_void_p(0x1000)
+    assert lib.ep_dispatch(C.byref(bad), *([fake] * 9), null) == 1
+    # misaligned vector buffers
+    odd = C.c_void_p(0x1008)
+    args = [odd, fake, fake, fake, fake, fake, fake, fake, fake, null]
+    assert lib.ep_dispatch(C.byref(cfg), *args) == 3
+    assert lib.ep_copy(fake, fake, 24, null) == 1
+    assert lib.ep_copy(odd, fake, 32, null) == 3
+    assert lib.ep_cvt_sweep(2, 0, 16, fake, null) == 1
+    assert lib.ep_cvt_sweep(0, 0xFFFFFFF0, 17, fake, null) == 1
+    assert ep.ep_kernel_launches() == n0
+
+
+def test_status_strings():
+    for s in range(7):
+        assert lib.ep_status_string(s)
+    assert b"unknown" in lib.ep_status_string(99)

@@ -1,0 +1,267 @@
+"""Parity of the CUDA path with the oracle, through the C ABI, on cuda:0.
+
+Bit-exact: layout outputs, slots, counts, src_info, recv weights, quantised
+codes and scales, combine-backward rows and the device status word.  Combine:
+within 1 bf16 ulp of the oracle (both accumulate in fp32 with one FMA per
+entry in k order, so the results are expected to be identical).
+
+Sizes: every named workload at full size where the oracle finishes in
+seconds (tiny, decode, skewed, large), reduced-T variants with a ragged tail
+for the others, and the full prefill workload checked on sampled tokens.
+"""
+import numpy as np
+import pytest
+import torch
+
+import combine_ep_dispatch_04_b200 as ep
+import oracle
+import synth
+from harness import Run, bf16_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("mode", ["bf16", "int8_token"])
+@pytest.mark.parametrize("layout", ["padded", "packed"])
+def test_tiny_workload(mode, layout):
+    w = synth.workload("tiny")
+    r = Run(w, mode, layout=layout, stats=True)
+    r.check_layout()
+    assert r.check_dispatch() == (r.idx >= 0).sum()
+    r.check_combine()
+
+
+@pytest.mark.parametrize("qmax", [0.0, 127.0])
+def test_decode_workload_full_size(qmax):
+    w = synth.workload("decode")
+    r = Run(w, "e4m3_b128", qmax=qmax)
+    r.check_layout()
+    assert r.check_dispatch() == w["N"] * w["K"]
+    r.check_combine()
+
+
+def test_skewed_workload_full_size():
+    w = synth.workload("skewed")
+    r = Run(w, "int8_token")
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+
+
+@pytest.mark.parametrize("align", [1, 16])
+@pytest.mark.parametrize("unweighted", [False, True])
+def test_prefill_workload_ragged(align, unweighted):
+    w = synth.workload("prefill", T=97)  # 3104 tokens: many layout chunks, ragged tail
+    r = Run(w, "mxfp8", layout="packed", align=align, backward=True, bwd_unweighted=unweighted)
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+    r.check_backward()
+
+
+def test_large_workload_full_size():
+    w = synth.workload("large")
+    r = Run(w, "mxfp4", layout="packed")
+    r.check_layout()
+    r.check_dispatch()
+    sample = np.random.default_rng(5).choice(w["N"], 2048, replace=False)
+    r.check_combine(tokens=np.sort(sample))
+
+
+def test_prefill_workload_full_size_sampled():
+    """The full prefill workload (131072 tokens, ~1M entries) in the launch
+    configuration the benchmark uses; outputs checked on sampled tokens and the
+    layout checked in full."""
+    w = synth.workload("prefill")
+    r = Run(w, "mxfp8", layout="packed", backward=True)
+    r.check_layout()
+    rng = np.random.default_rng(11)
+    sample = np.sort(np.concatenate([rng.choice(w["N"], 1500, replace=False),
+                                     [0, w["N"] - 1]]))
+    r.check_dispatch(tokens=sample)
+    r.check_combine(tokens=sample)
+    r.check_backward(tokens=sample[:300])
+
+
+# ---------------------------------------------------------------------------
+# both layout paths agree with the oracle (and so with each other)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name,override", [
+    ("decode", {}), ("skewed", dict(T=100)), ("large", dict(T=40)), ("tiny", {}),
+    ("prefill", dict(T=33, E=1024)),
+])
+@pytest.mark.parametrize("path", [ep.F_LAYOUT_SINGLE_CTA, ep.F_LAYOUT_MULTI_CTA])
+def test_layout_paths(name, override, path):
+    w = synth.workload(name, **override)
+    r = Run(w, "bf16", layout="packed", align=4, flags=path)
+    r.check_layout()
+
+
+# ---------------------------------------------------------------------------
+# edge cases
+# ---------------------------------------------------------------------------
+def _edge(R=2, T=8, M=8, K=3, E=8, H=256, x="normal"):
+    w = synth.workload("tiny", R=R, T=T, M=M, K=K, E=E, H=H)
+    w["x"] = x
+    return w
+
+
+@pytest.mark.parametrize("mode", ["bf16", "int8_token", "e4m3_b128", "mxfp8", "mxfp4"])
+@pytest.mark.parametrize("layout", ["padded", "packed"])
+def test_every_mode_small_ragged(mode, layout):
+    w = _edge(R=3, T=13, M=16, K=4, E=12, H=640)
+    r = Run(w, mode, layout=layout, backward=True)
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+    r.check_backward()
+
+
+@pytest.mark.parametrize("path", [ep.F_LAYOUT_SINGLE_CTA, ep.F_LAYOUT_MULTI_CTA])
+def test_zero_tokens(path):
+    w = _edge(T=0)
+    r = Run(w, "mxfp8", layout="packed", flags=path)
+    r.check_layout()
+    assert r.b.recv_count.sum().item() == 0
+    assert r.b.expert_offset.cpu().numpy().tolist() == [0] * (w["E"] + 1)
+
+
+def test_all_entries_masked():
+    w = _edge()
+    idx = np.full((w["N"], w["K"]), -1, np.int64)
+    r = Run(w, "int8_token", idx=idx)
+    r.check_layout()
+    r.check_dispatch()
+    assert not r.b.out.view(torch.int16).any().item()  # +0 everywhere
+
+
+@pytest.mark.parametrize("mode", ["bf16", "mxfp4"])
+def test_k1_r1_and_one_expert_per_rank(mode):
+    for (R, E, K) in [(1, 4, 1), (4, 4, 2), (1, 1, 1)]:
+        w = _edge(R=R, E=E, K=K, T=7, M=9, H=128)
+        r = Run(w, mode)
+        r.check_layout()
+        r.check_dispatch()
+        r.check_combine()
+
+
+@pytest.mark.parametrize("mode,H", [("bf16", 32), ("int8_token", 32), ("mxfp8", 32),
+                                    ("mxfp4", 32), ("e4m3_b128", 128), ("mxfp8", 8192),
+                                    ("int8_token", 8192)])
+def test_min_and_max_hidden(mode, H):
+    w = _edge(H=H, T=5, M=5)
+    r = Run(w, mode, layout="packed", backward=True)
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+    r.check_backward()
+
+
+def test_duplicates_overflow_padded_capacity():
+    # every entry of every token on expert 0: 2*6*3 entries > cap = 2*6
+    w = _edge(R=2, T=6, M=6, K=3, E=4)
+    idx = np.zeros((w["N"], w["K"]), np.int64)
+    r = Run(w, "bf16", idx=idx)
+    assert r.status & ep.DEV_CAPACITY_OVERFLOW
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()  # entries beyond the capacity contribute nothing
+
+
+def test_duplicates_fit_packed():
+    w = _edge(R=2, T=6, M=6, K=3, E=4)
+    idx = np.zeros((w["N"], w["K"]), np.int64)
+    idx[::2, 1] = 3
+    r = Run(w, "mxfp8", layout="packed", idx=idx, backward=True)
+    assert r.status == 0
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+    r.check_backward()
+
+
+def test_full_capacity_expert():
+    # T == M and every token of every rank picks expert 0 once: slot R*M-1 is used
+    w = _edge(R=4, T=8, M=8, K=2, E=8)
+    idx = np.stack([np.zeros(w["N"], np.int64), np.arange(w["N"]) % 7 + 1], axis=1)
+    r = Run(w, "int8_token", idx=idx)
+    assert r.status == 0
+    assert r.b.recv_count[0].item() == w["R"] * w["M"]
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+
+
+def test_bad_indices_flagged_and_skipped():
+    w = _edge()
+    idx, wts = synth.make_routing(w)
+    idx[1, 0] = w["E"]
+    idx[3, 2] = -5
+    idx[4, 1] = 1 << 40
+    r = Run(w, "e4m3_b128", idx=idx, wts=wts)
+    assert r.status & ep.DEV_BAD_INDEX
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+    assert ep.ep_get_status(r.b.dev_status) == 0  # read-and-clear
+
+
+def test_zero_and_signed_zero_rows():
+    w = _edge(H=256)
+    x = synth.make_x(w)
+    x[0] = 0
+    x[1] = 0x8000  # -0.0 everywhere
+    x[2, :128] = 0  # one zero 128-block, one normal block
+    x[3, 32:64] = 0x8000
+    for mode in ["int8_token", "e4m3_b128", "mxfp8", "mxfp4", "bf16"]:
+        r = Run(w, mode, layout="packed", x=x)
+        r.check_dispatch()
+
+
+def test_tiny_magnitudes_and_outliers():
+    w = _edge(H=512)
+    x = synth.make_x(w)
+    f = oracle.bf16_to_f32(x).copy()
+    f[0] *= np.float32(2.0 ** -120)    # subnormal block maxima after the scale division
+    f[1] *= np.float32(2.0 ** -126)
+    f[2] *= np.float32(2.0 ** 100)
+    f[3, ::7] *= 50
+    x = synth.to_bf16_bits(f)
+    for mode in ["int8_token", "e4m3_b128", "mxfp8", "mxfp4"]:
+        r = Run(w, mode, layout="packed", x=x, backward=True)
+        r.check_dispatch()
+        r.check_backward()
+
+
+def test_recv_weights_optional_and_deterministic():
+    w = synth.workload("skewed", T=64)
+    a = Run(w, "int8_token", with_weights=False)
+    b = Run(w, "int8_token", with_weights=False)
+    for name in ("token_slot", "recv_count", "recv_buf", "src_info", "out"):
+        assert torch.equal(getattr(a.b, name), getattr(b.b, name)), name
+
+
+def test_stats_accumulate():
+    w = synth.workload("decode", T=16)
+    r = Run(w, "bf16", stats=True)
+    cnt = r.b.recv_count.clone()
+    ep.ep_dispatch_layout(r.cfg, r.idx_d, r.b.token_slot, r.b.recv_count, r.b.workspace,
+                          r.b.dev_status, cumulative_recv_stats=r.stats_d)
+    torch.cuda.synchronize()
+    assert torch.equal(r.stats_d, 2 * cnt)
+
+
+def test_python_checks_reject_prequantised_input():
+    w = _edge()
+    cfg = ep.make_config(w["R"], w["T"], w["M"], w["K"], w["E"], w["H"], "mxfp8")
+    b = ep.Buffers(cfg)
+    x8 = torch.zeros((w["N"], w["H"]), dtype=torch.float8_e4m3fn, device="cuda")
+    idx = torch.zeros((w["N"], w["K"]), dtype=torch.int64, device="cuda")
+    with pytest.raises(TypeError):
+        ep.ep_dispatch(cfg, x8, idx, b.token_slot, b.recv_buf, b.src_info, b.dev_status)
+    with pytest.raises(TypeError):
+        ep.ep_dispatch_layout(cfg, idx.int(), b.token_slot, b.recv_count, b.workspace,
+                              b.dev_status)
+    with pytest.raises(ValueError):
+        ep.ep_dispatch_layout(cfg, idx.t().contiguous().t(), b.token_slot, b.recv_count,
+                              b.workspace, b.dev_status)
