@@ -312,26 +312,27 @@ def main():
 
     kernels = ["layout", "dispatch", "combine"] + (["combine_bwd"] if g_d is not None else [])
 
+    # each C-ABI call is checked and marshalled once, then replayed every step
+    calls = [
+        ep.ep_dispatch_layout(cfg, idx_d, b.token_slot, b.recv_count, b.workspace, b.dev_status,
+                              expert_offset=b.expert_offset, stream=stream, bind=True),
+        ep.ep_dispatch(cfg, x_d, idx_d, b.token_slot, b.recv_buf, b.src_info, b.dev_status,
+                       expert_offset=b.expert_offset, stream=stream, bind=True),
+        ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
+                      expert_offset=b.expert_offset, stream=stream, bind=True),
+    ]
+    if g_d is not None:
+        calls.append(ep.ep_combine_backward(cfg, g_d, idx_d, wts_d, b.token_slot, b.grad_buf,
+                                            b.dev_status, expert_offset=b.expert_offset,
+                                            stream=stream, bind=True))
+
     def step(evs=None):
         if evs:
             evs[0].record(stream)
-        ep.ep_dispatch_layout(cfg, idx_d, b.token_slot, b.recv_count, b.workspace, b.dev_status,
-                              expert_offset=b.expert_offset, stream=stream)
-        if evs:
-            evs[1].record(stream)
-        ep.ep_dispatch(cfg, x_d, idx_d, b.token_slot, b.recv_buf, b.src_info, b.dev_status,
-                       expert_offset=b.expert_offset, stream=stream)
-        if evs:
-            evs[2].record(stream)
-        ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
-                      expert_offset=b.expert_offset, stream=stream)
-        if evs:
-            evs[3].record(stream)
-        if g_d is not None:
-            ep.ep_combine_backward(cfg, g_d, idx_d, wts_d, b.token_slot, b.grad_buf, b.dev_status,
-                                   expert_offset=b.expert_offset, stream=stream)
+        for i, c in enumerate(calls):
+            c()
             if evs:
-                evs[4].record(stream)
+                evs[i + 1].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         flush.fill_(1)
@@ -460,19 +461,25 @@ def run_e2e(ep, cfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, world):
     h2d = x_h.numel() * 2 + idx_h.numel() * 8 + wts_h.numel() * 4
     d2h = out_h.numel() * 2 + cnt_h.numel() * 8
 
+    calls = [
+        ep.ep_dispatch_layout(cfg, idx_d, b.token_slot, b.recv_count, b.workspace, b.dev_status,
+                              expert_offset=b.expert_offset, stream=stream, bind=True),
+        ep.ep_dispatch(cfg, x_d, idx_d, b.token_slot, b.recv_buf, b.src_info, b.dev_status,
+                       expert_offset=b.expert_offset, stream=stream, bind=True),
+        ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
+                      expert_offset=b.expert_offset, stream=stream, bind=True),
+    ]
+    if g_d is not None:
+        calls.append(ep.ep_combine_backward(cfg, g_d, idx_d, wts_d, b.token_slot, b.grad_buf,
+                                            b.dev_status, expert_offset=b.expert_offset,
+                                            stream=stream, bind=True))
+
     def one():
         x_d.copy_(x_h, non_blocking=True)
         idx_d.copy_(idx_h, non_blocking=True)
         wts_d.copy_(wts_h, non_blocking=True)
-        ep.ep_dispatch_layout(cfg, idx_d, b.token_slot, b.recv_count, b.workspace, b.dev_status,
-                              expert_offset=b.expert_offset, stream=stream)
-        ep.ep_dispatch(cfg, x_d, idx_d, b.token_slot, b.recv_buf, b.src_info, b.dev_status,
-                       expert_offset=b.expert_offset, stream=stream)
-        ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
-                      expert_offset=b.expert_offset, stream=stream)
-        if g_d is not None:
-            ep.ep_combine_backward(cfg, g_d, idx_d, wts_d, b.token_slot, b.grad_buf,
-                                   b.dev_status, expert_offset=b.expert_offset, stream=stream)
+        for c in calls:
+            c()
         out_h.copy_(b.out, non_blocking=True)
         cnt_h.copy_(b.recv_count, non_blocking=True)
 

@@ -90,6 +90,28 @@ def _check(st, where):
         raise EpError(st, where)
 
 
+class Bound:
+    """One entry-point call with its arguments checked and marshalled once.
+    Calling it replays the C call with the same pointers and stream (for loops
+    that run the same step many times, e.g. a timing loop)."""
+
+    def __init__(self, fn, cfg, args, where):
+        self._fn, self._cfg, self._args, self._where = fn, cfg, tuple(args), where
+        self._ref = C.byref(cfg)
+
+    def __call__(self):
+        st = self._fn(self._ref, *self._args)
+        if st != 0:
+            raise EpError(st, self._where)
+
+
+def _call(fn, cfg, args, where, bind):
+    if bind:
+        return Bound(fn, cfg, args, where)
+    _check(fn(C.byref(cfg), *args), where)
+    return None
+
+
 def ep_buffer_sizes(cfg):
     s = EpSizes()
     _check(lib.ep_buffer_sizes(C.byref(cfg), C.byref(s)), "ep_buffer_sizes")
@@ -136,7 +158,7 @@ def _nk(cfg):
 
 def ep_dispatch_layout(cfg, topk_idx, token_slot, recv_count, workspace, dev_status,
                        tokens_per_rank=None, tokens_per_expert=None, is_token_in_rank=None,
-                       expert_offset=None, cumulative_recv_stats=None, stream=None):
+                       expert_offset=None, cumulative_recv_stats=None, stream=None, bind=False):
     N, K = _nk(cfg)
     R, E = cfg.num_ranks, cfg.num_experts
     sz = ep_buffer_sizes(cfg)
@@ -154,11 +176,11 @@ def ep_dispatch_layout(cfg, topk_idx, token_slot, recv_count, workspace, dev_sta
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
     ]
-    _check(lib.ep_dispatch_layout(C.byref(cfg), *args), "ep_dispatch_layout")
+    return _call(lib.ep_dispatch_layout, cfg, args, "ep_dispatch_layout", bind)
 
 
 def ep_dispatch(cfg, x, topk_idx, token_slot, recv_buf, src_info, dev_status, topk_weights=None,
-                expert_offset=None, recv_weights=None, stream=None):
+                expert_offset=None, recv_weights=None, stream=None, bind=False):
     N, K = _nk(cfg)
     sz = ep_buffer_sizes(cfg)
     args = [
@@ -174,11 +196,11 @@ def ep_dispatch(cfg, x, topk_idx, token_slot, recv_buf, src_info, dev_status, to
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
     ]
-    _check(lib.ep_dispatch(C.byref(cfg), *args), "ep_dispatch")
+    return _call(lib.ep_dispatch, cfg, args, "ep_dispatch", bind)
 
 
 def ep_combine(cfg, y, topk_idx, topk_weights, token_slot, out, dev_status, expert_offset=None,
-               stream=None):
+               stream=None, bind=False):
     N, K = _nk(cfg)
     sz = ep_buffer_sizes(cfg)
     if y is None or y.dtype != torch.bfloat16:
@@ -194,11 +216,11 @@ def ep_combine(cfg, y, topk_idx, topk_weights, token_slot, out, dev_status, expe
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
     ]
-    _check(lib.ep_combine(C.byref(cfg), *args), "ep_combine")
+    return _call(lib.ep_combine, cfg, args, "ep_combine", bind)
 
 
 def ep_combine_backward(cfg, g, topk_idx, topk_weights, token_slot, grad_buf, dev_status,
-                        expert_offset=None, stream=None):
+                        expert_offset=None, stream=None, bind=False):
     N, K = _nk(cfg)
     sz = ep_buffer_sizes(cfg)
     args = [
@@ -213,7 +235,7 @@ def ep_combine_backward(cfg, g, topk_idx, topk_weights, token_slot, grad_buf, de
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
     ]
-    _check(lib.ep_combine_backward(C.byref(cfg), *args), "ep_combine_backward")
+    return _call(lib.ep_combine_backward, cfg, args, "ep_combine_backward", bind)
 
 
 def ep_get_status(dev_status, stream=None):
