@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "ep.h"
 #include "ep_combine.cuh"
@@ -406,5 +407,78 @@ extern "C" ep_status_t ep_cvt_sweep(int32_t format, uint32_t start, int64_t n, u
     const int64_t cap = (int64_t)sm_count() * 16;
     if (blocks > cap) blocks = cap;
     ep::cvt_sweep_kernel<<<(unsigned)blocks, 256, 0, cs(stream)>>>(format, start, n, out);
+    return launched();
+}
+
+// ---- allocation-free layout ------------------------------------------------------
+// The multi-block layout path with its scratch in a static device array, for
+// callers that cannot allocate device memory (see ep_dispatch_layout_static in
+// ep.h).  The array's device address is looked up once per device, with that
+// device current, and cached.
+namespace {
+
+__device__ __align__(256) unsigned char g_static_scratch[EP_STATIC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void *g_static_ptr[kMaxDevices] = {};
+
+ep_status_t static_scratch(void **out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return EP_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return EP_ERR_CUDA;
+        g_static_ptr[dev] = p;
+    }
+    *out = g_static_ptr[dev];
+    return EP_OK;
+}
+
+}  // namespace
+
+extern "C" ep_status_t ep_dispatch_layout_static(
+    const ep_config_t *cfg, const int64_t *topk_idx, int32_t *tokens_per_rank,
+    int32_t *tokens_per_expert, uint8_t *is_token_in_rank, int32_t *token_slot,
+    int64_t *recv_count, int64_t *expert_offset, int64_t *cumulative_recv_stats,
+    uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (!recv_count || !dev_status) return EP_ERR_INVALID_ARG;
+    if (p.N > 0 && (!topk_idx || !token_slot)) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    if (p.ws_bytes > (int64_t)EP_STATIC_SCRATCH_BYTES) return EP_ERR_UNSUPPORTED;
+    void *scratch = nullptr;
+    if ((st = static_scratch(&scratch)) != EP_OK) return st;
+
+    ep::LayoutArgs a;
+    a.R = p.R; a.T = p.T; a.K = p.K; a.E = p.E; a.M = p.M; a.L = p.L;
+    a.TC = p.TC; a.CR = p.CR; a.C = p.C;
+    a.packed = cfg->layout == EP_LAYOUT_PACKED;
+    a.align = cfg->expert_align;
+    a.cap = p.cap;
+    a.idx = topk_idx;
+    a.tpr = tokens_per_rank;
+    a.tpe = tokens_per_expert;
+    a.itr = is_token_in_rank;
+    a.slot = token_slot;
+    a.recv_count = recv_count;
+    a.eo = expert_offset;
+    a.stats = cumulative_recv_stats;
+    a.ws_hist = static_cast<int32_t *>(scratch);
+    a.ws_rk = a.ws_hist + (int64_t)p.E * p.C;
+    a.status = dev_status;
+
+    cudaStream_t s = cs(stream);
+    if (p.C > 0) {
+        ep::layout_count_kernel<<<p.C, ep::kLayoutThreads, (p.E + p.R) * sizeof(int), s>>>(a);
+        if ((st = launched()) != EP_OK) return st;
+    }
+    ep::layout_scan_kernel<<<p.E + p.R, ep::kLayoutThreads, 0, s>>>(a);
+    if ((st = launched()) != EP_OK) return st;
+    const size_t smem = (size_t)(ep::kLayoutThreads / 32) * p.E * sizeof(int);
+    ep::layout_assign_kernel<<<p.C > 0 ? p.C : 1, ep::kLayoutThreads, smem, s>>>(a);
     return launched();
 }

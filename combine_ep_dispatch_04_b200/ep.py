@@ -28,6 +28,8 @@ F_BWD_UNWEIGHTED = 0x1
 F_LAYOUT_SINGLE_CTA = 0x100
 F_LAYOUT_MULTI_CTA = 0x200
 
+STATIC_SCRATCH_BYTES = 1 << 20  # EP_STATIC_SCRATCH_BYTES of include/ep.h
+
 STATUS = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_UNSUPPORTED", 3: "EP_ERR_MISALIGNED",
           4: "EP_ERR_CUDA", 5: "EP_ERR_DEVICE_STATUS", 6: "EP_ERR_TIMEOUT"}
 
@@ -62,6 +64,8 @@ lib.ep_buffer_sizes.restype = C.c_int
 lib.ep_buffer_sizes.argtypes = [_CFG, C.POINTER(EpSizes)]
 lib.ep_dispatch_layout.restype = C.c_int
 lib.ep_dispatch_layout.argtypes = [_CFG] + [_P] * 11
+lib.ep_dispatch_layout_static.restype = C.c_int
+lib.ep_dispatch_layout_static.argtypes = [_CFG] + [_P] * 10
 lib.ep_dispatch.restype = C.c_int
 lib.ep_dispatch.argtypes = [_CFG] + [_P] * 10
 lib.ep_combine.restype = C.c_int
@@ -177,6 +181,31 @@ def ep_dispatch_layout(cfg, topk_idx, token_slot, recv_count, workspace, dev_sta
         _stream(stream),
     ]
     return _call(lib.ep_dispatch_layout, cfg, args, "ep_dispatch_layout", bind)
+
+
+def ep_dispatch_layout_static(cfg, topk_idx, token_slot, recv_count, dev_status,
+                              tokens_per_rank=None, tokens_per_expert=None, is_token_in_rank=None,
+                              expert_offset=None, cumulative_recv_stats=None, stream=None,
+                              bind=False):
+    """ep_dispatch_layout without a workspace: for callers that cannot allocate
+    device memory.  Its scratch is a static array inside libep.so, shared by
+    every call on the device (serialise calls; see include/ep.h)."""
+    N, K = _nk(cfg)
+    R, E = cfg.num_ranks, cfg.num_experts
+    args = [
+        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(tokens_per_rank, "tokens_per_rank", torch.int32, (R, R), optional=True),
+        _dev(tokens_per_expert, "tokens_per_expert", torch.int32, (R, E), optional=True),
+        _dev(is_token_in_rank, "is_token_in_rank", torch.uint8, (N, R), optional=True),
+        _dev(token_slot, "token_slot", torch.int32, (N, K)),
+        _dev(recv_count, "recv_count", torch.int64, (E,)),
+        _dev(expert_offset, "expert_offset", torch.int64, (E + 1,),
+             optional=cfg.layout == LAYOUT["padded"]),
+        _dev(cumulative_recv_stats, "cumulative_recv_stats", torch.int64, (E,), optional=True),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    return _call(lib.ep_dispatch_layout_static, cfg, args, "ep_dispatch_layout_static", bind)
 
 
 def ep_dispatch(cfg, x, topk_idx, token_slot, recv_buf, src_info, dev_status, topk_weights=None,

@@ -192,6 +192,37 @@ ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
                                 const int32_t *token_slot, const int64_t *expert_offset,
                                 void *grad_buf, uint32_t *dev_status, ep_stream_t stream);
 
+/*
+ * Allocation-free variant of ep_dispatch_layout.  The pages have no
+ * counterpart to this call; it exists for callers that cannot allocate
+ * device memory when they route tokens -- for example a serving loop whose
+ * device memory is reserved in full up front, or a plugin running inside a
+ * host framework that owns every device allocation -- and so cannot provide
+ * the `workspace` buffer.  Arguments and results are those of
+ * ep_dispatch_layout without `workspace`; the multi-block layout kernels run
+ * with their scratch in a static device array of EP_STATIC_SCRATCH_BYTES
+ * inside this library (every GPU that loads the library holds it until the
+ * process exits).  The caller still owns and passes all inputs and outputs.
+ *   - A configuration whose ep_sizes_t.workspace_bytes exceeds
+ *     EP_STATIC_SCRATCH_BYTES is rejected with EP_ERR_UNSUPPORTED before any
+ *     launch.
+ *   - The first call on a device looks up the array's device address with
+ *     that device current (the device of `stream` must be the current
+ *     device); make that first call before any stream capture.
+ *   - Every call on a device shares the one array and leaves its contents
+ *     behind.  Each launch writes every scratch word it reads, so nothing has
+ *     to start at zero; but calls that overlap on the GPU (different streams,
+ *     or several host threads) race on the array: serialise them.
+ *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ */
+#define EP_STATIC_SCRATCH_BYTES (1u << 20)
+ep_status_t ep_dispatch_layout_static(const ep_config_t *cfg, const int64_t *topk_idx,
+                                      int32_t *tokens_per_rank, int32_t *tokens_per_expert,
+                                      uint8_t *is_token_in_rank, int32_t *token_slot,
+                                      int64_t *recv_count, int64_t *expert_offset,
+                                      int64_t *cumulative_recv_stats, uint32_t *dev_status,
+                                      ep_stream_t stream);
+
 /* Synchronise `stream`, read *dev_status into *host_flags (host pointer) and
  * clear it.  Returns EP_ERR_DEVICE_STATUS when any bit was set. */
 ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream);
