@@ -7,8 +7,14 @@ workload).  Default workload: decode (R=8 logical ranks x T=128 tokens,
 H=7168, top-8 of 256 experts, M=128, per-128-channel e4m3 dispatch, padded
 receive layout), on one GPU.
 
-Timing: CUDA events on the stream the kernels run on, one pair per kernel per
-step; a 512 MiB write flushes L2 between steps, outside the step's events.
+Timing: CUDA events on the stream the kernels run on.  The timed region
+brackets each step with one event pair (the reported value); a second pass
+over the same steps puts an event between consecutive kernels for the
+per-kernel durations behind the roofline figures.  Between steps, outside the step's events, L2 is flushed by writing one
+512 MiB buffer and then reading another: the read evicts the write's dirty
+lines, so every step starts from a cold L2 holding only clean lines (a
+write-only flush would leave ~126 MB of dirty lines whose write-back the next
+step's kernels would pay for).
 The K timed steps are bracketed by a barrier and a synchronize on both sides;
 the reported time is the max over ranks.  With --gpus N > 1 (torchrun), each
 rank runs an independent replica of the workload (different seed): the path
@@ -307,8 +313,13 @@ def main():
     if w.get("backward"):
         gp, go = synth.g_source(w, replica)
         g_d = torch.from_numpy(synth.windows(gp, go, H).view(np.int16)).to(dev).view(torch.bfloat16)
-    flush = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+    flush_w = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(args.flush_mib << 20, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    def flush(v):
+        flush_w.fill_(v)
+        flush_r.max()
 
     kernels = ["layout", "dispatch", "combine"] + (["combine_bwd"] if g_d is not None else [])
 
@@ -335,34 +346,47 @@ def main():
                 evs[i + 1].record(stream)
 
     for _ in range(max(args.warmup, 3)):
-        flush.fill_(1)
+        flush(1)
         step()
     torch.cuda.synchronize(dev)
     if ep.ep_get_status(b.dev_status) != 0:
         raise SystemExit("device status reported errors during warm-up")
 
-    nev = len(kernels) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    # timed region: K steps, one event pair per step (events between the
+    # kernels would add their own ~2 us each to the step)
+    steps_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize(dev)
     launches0 = ep.ep_kernel_launches()
     with clocks:
         for s in range(args.steps):
-            flush.fill_(s & 0xFF)
-            step(evs[s])
+            flush(s & 0xFF)
+            steps_ev[s][0].record(stream)
+            step()
+            steps_ev[s][1].record(stream)
         torch.cuda.synchronize(dev)
     launches = ep.ep_kernel_launches() - launches0
     barrier(world)
-    per_kernel = {k: [] for k in kernels}
-    step_ms = []
-    for e in evs:
-        for i, k in enumerate(kernels):
-            per_kernel[k].append(e[i].elapsed_time(e[i + 1]))
-        step_ms.append(e[0].elapsed_time(e[-1]))
+    step_ms = [a.elapsed_time(c) for a, c in steps_ev]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
     value = world * N * args.steps / (total_ms / 1e3)
+
+    # per-kernel durations (for the roofline): the same steps again, with an
+    # event between consecutive kernels
+    nev = len(kernels) + 1
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    torch.cuda.synchronize(dev)
+    for s in range(args.steps):
+        flush(s & 0xFF)
+        step(evs[s])
+    torch.cuda.synchronize(dev)
+    per_kernel = {k: [] for k in kernels}
+    for e in evs:
+        for i, k in enumerate(kernels):
+            per_kernel[k].append(e[i].elapsed_time(e[i + 1]))
 
     alg, v = algorithmic_bytes(w, mode, idx)
     peaks = measured_peaks()
@@ -422,7 +446,8 @@ def main():
         "config": {
             "workload": f"{wname}: R={R} T={T} H={H} K={K} E={E} M={M} {mode} {w['layout']}",
             "tokens_per_step": N, "valid_entries": v,
-            "l2": f"flushed between steps ({args.flush_mib} MiB write outside the step events)",
+            "l2": f"flushed between steps outside the step events ({args.flush_mib} MiB write, "
+                  f"then {args.flush_mib} MiB read)",
             "parallelism": "replicas" if world > 1 else "single",
         },
         "hbm_gbs": round(step_bytes / (ms_per_step * 1e-3) / 1e9, 1),
@@ -484,7 +509,7 @@ def run_e2e(ep, cfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, world):
         cnt_h.copy_(b.recv_count, non_blocking=True)
 
     for _ in range(3):
-        flush.fill_(1)
+        flush(1)
         one()
     steps = max(10, min(args.steps, 100))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -492,7 +517,7 @@ def run_e2e(ep, cfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, world):
     barrier(world)
     torch.cuda.synchronize(dev)
     for s in range(steps):
-        flush.fill_(s & 0xFF)
+        flush(s & 0xFF)
         evs[s][0].record(stream)
         one()
         evs[s][1].record(stream)

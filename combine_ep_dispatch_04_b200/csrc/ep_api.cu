@@ -19,10 +19,11 @@ std::atomic<uint64_t> g_launches{0};
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxHidden = 8192;
 constexpr int64_t kIntLimit = (int64_t(1) << 31) - 1;
-// one-block layout when the routing is small (its per-warp counters fit in
-// the default 48 KB of shared memory)
+// one-block layout when the routing is small and its counters fit in the
+// default 48 KB of shared memory
 constexpr int64_t kSingleMaxEntries = 32768;
-constexpr int kSingleMaxExperts = 384;
+constexpr size_t kDefaultSmem = 48 * 1024;
+constexpr size_t kMaxSmem = 200 * 1024;
 
 cudaStream_t cs(ep_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -109,6 +110,88 @@ ep_status_t make_plan(const ep_config_t *c, Plan &p) {
     return EP_OK;
 }
 
+
+// ---- layout launch helpers -------------------------------------------------------
+// The one-block layout cuts the N tokens into chunks of whole tokens of one
+// source rank, about one chunk per warp (ceil(W/R) per rank).  Its shared
+// memory holds the per-chunk counters (C*E ints), one mask word per warp and
+// expert (W*E), the expert-to-rank table (E) and the staged keys (N*K), each
+// part rounded up to a multiple of 4 ints.
+struct SinglePlan {
+    int warps, TC, CR, C;
+    size_t smem;
+    bool ok;
+};
+
+SinglePlan single_chunks(const Plan &p, int W) {
+    SinglePlan sp{};
+    sp.warps = W;
+    sp.CR = (W + p.R - 1) / p.R;
+    if (sp.CR > p.T) sp.CR = p.T > 0 ? p.T : 1;
+    sp.TC = p.T > 0 ? (p.T + sp.CR - 1) / sp.CR : 1;
+    sp.CR = p.T > 0 ? (p.T + sp.TC - 1) / sp.TC : 0;
+    sp.C = p.R * sp.CR;
+    auto r4 = [](int64_t v) { return (v + 3) & ~int64_t(3); };
+    const int64_t ints = r4((int64_t)sp.C * p.E) + r4((int64_t)W * p.E) + r4(p.E) + r4(p.N * p.K);
+    sp.smem = (size_t)ints * sizeof(int);
+    sp.ok = sp.smem <= kMaxSmem;
+    return sp;
+}
+
+SinglePlan plan_single(const Plan &p) {
+    for (int W : {32, 16, 8, 4}) {
+        const SinglePlan sp = single_chunks(p, W);
+        if (sp.ok) return sp;
+    }
+    SinglePlan none{};
+    return none;
+}
+
+// Kernels that may ask for more than the default 48 KB of shared memory get
+// the larger limit once per device (the attribute is per function and device).
+constexpr int kMaxDevices = 64;
+std::atomic<uint32_t> g_smem_done[kMaxDevices];
+
+template <typename Kernel>
+bool allow_smem(Kernel k, int which, size_t bytes) {
+    if (bytes <= kDefaultSmem) return true;
+    if (bytes > kMaxSmem) return false;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+    if (g_smem_done[dev].load() & (1u << which)) return true;
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem) !=
+        cudaSuccess)
+        return false;
+    g_smem_done[dev].fetch_or(1u << which);
+    return true;
+}
+
+ep_status_t launch_layout_single(ep::LayoutArgs a, const SinglePlan &sp, cudaStream_t s) {
+    if (!sp.ok) return EP_ERR_UNSUPPORTED;
+    a.TC = sp.TC;
+    a.CR = sp.CR;
+    a.C = sp.C;
+    if (!allow_smem(ep::layout_single_kernel, 0, sp.smem)) return EP_ERR_CUDA;
+    ep::layout_single_kernel<<<1, sp.warps * 32, sp.smem, s>>>(a);
+    return launched();
+}
+
+ep_status_t launch_layout_multi(const ep::LayoutArgs &a, const Plan &p, cudaStream_t s) {
+    ep_status_t st;
+    if (p.C > 0) {
+        const size_t smem = (size_t)(p.TC * p.K + p.E + p.R) * sizeof(int);
+        if (!allow_smem(ep::layout_count_kernel, 2, smem)) return EP_ERR_CUDA;
+        ep::layout_count_kernel<<<p.C, ep::kLayoutThreads, smem, s>>>(a);
+        if ((st = launched()) != EP_OK) return st;
+    }
+    ep::layout_scan_kernel<<<p.E + p.R, ep::kLayoutThreads, 0, s>>>(a);
+    if ((st = launched()) != EP_OK) return st;
+    const size_t smem = (size_t)(p.TC * p.K + 2 * (ep::kLayoutThreads / 32) * p.E) * sizeof(int);
+    if (!allow_smem(ep::layout_assign_kernel, 3, smem)) return EP_ERR_CUDA;
+    ep::layout_assign_kernel<<<p.C > 0 ? p.C : 1, ep::kLayoutThreads, smem, s>>>(a);
+    return launched();
+}
+
 }  // namespace
 
 extern "C" {
@@ -182,58 +265,76 @@ ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const int64_t *topk_idx,
     a.status = dev_status;
 
     cudaStream_t s = cs(stream);
+    const SinglePlan sp = plan_single(p);
     const bool single = (cfg->flags & EP_F_LAYOUT_SINGLE_CTA) ||
                         (!(cfg->flags & EP_F_LAYOUT_MULTI_CTA) && p.N * p.K <= kSingleMaxEntries &&
-                         p.E <= kSingleMaxExperts);
-    if (single) {
-        const size_t smem1 = (size_t)(ep::kLayoutSingleThreads / 32) * p.E * sizeof(int);
-        if (smem1 > 48 * 1024 &&
-            cudaFuncSetAttribute(ep::layout_single_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem1) != cudaSuccess)
-            return EP_ERR_CUDA;
-        ep::layout_single_kernel<<<1, ep::kLayoutSingleThreads, smem1, s>>>(a);
-        return launched();
-    }
-    if (p.C > 0) {
-        ep::layout_count_kernel<<<p.C, ep::kLayoutThreads, (p.E + p.R) * sizeof(int), s>>>(a);
-        if ((st = launched()) != EP_OK) return st;
-    }
-    ep::layout_scan_kernel<<<p.E + p.R, ep::kLayoutThreads, 0, s>>>(a);
-    if ((st = launched()) != EP_OK) return st;
-    const size_t smem = (size_t)(ep::kLayoutThreads / 32) * p.E * sizeof(int);
-    ep::layout_assign_kernel<<<p.C > 0 ? p.C : 1, ep::kLayoutThreads, smem, s>>>(a);
-    return launched();
+                         sp.ok);
+    if (single) return launch_layout_single(a, sp, s);
+    return launch_layout_multi(a, p, s);
 }
 
 }  // extern "C"
 
 namespace {
 
-// granules of 16 elements -> (threads per token, granules per thread)
-template <int MODE>
-ep_status_t launch_dispatch(const ep::DispatchArgs &a, cudaStream_t s) {
-    const int ng = a.H / 16;
-    auto grid = [&](int tpt) { return (unsigned)((a.N + (ep::kDispatchThreads / tpt) - 1) /
-                                                 (ep::kDispatchThreads / tpt)); };
-    if (ng <= 32) ep::dispatch_kernel<MODE, 32, 1><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
-    else if (ng <= 64) ep::dispatch_kernel<MODE, 32, 2><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
-    else if (ng <= 128) ep::dispatch_kernel<MODE, 32, 4><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
-    else if (ng <= 256) ep::dispatch_kernel<MODE, 32, 8><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
-    else ep::dispatch_kernel<MODE, 64, 8><<<grid(64), ep::kDispatchThreads, 0, s>>>(a);
-    return launched();
+// Threads per token (TPT) and granules per thread (G): the smallest TPT that
+// keeps G <= max_g (8 unless stated), doubled (up to 256, and up to one granule per thread) while
+// the grid has fewer than kTargetWarps warps -- few tokens (decode) then
+// spread each row over more warps instead of leaving SMs idle.
+constexpr int64_t kTargetWarps = 8192;
+
+struct Split {
+    int tpt, gmax;
+};
+
+Split split_rows(int64_t N, int ngran, int max_g = 8) {
+    int tpt = 32;
+    while (tpt < 256 && (ngran + tpt - 1) / tpt > max_g) tpt *= 2;
+    while (tpt < 256 && tpt < ngran && N * (tpt / 32) < kTargetWarps) tpt *= 2;
+    const int g = (ngran + tpt - 1) / tpt;
+    const int gmax = g <= 1 ? 1 : (g <= 2 ? 2 : (g <= 4 ? 4 : 8));
+    return {tpt, gmax};
 }
 
+unsigned grid_for(int64_t N, int threads, int tpt) {
+    const int toks = threads / tpt;
+    return (unsigned)((N + toks - 1) / toks);
+}
+
+// Instantiated (TPT, GMAX) pairs: every split_rows result for H <= 8192 with
+// 16-element granules (dispatch, backward: at most 512) and 8-element
+// granules (combine: at most 1024).
+#define EP_SPLITS(X) X(32, 1) X(32, 2) X(32, 4) X(32, 8) X(64, 1) X(64, 2) X(64, 4) X(64, 8) \
+    X(128, 1) X(128, 2) X(128, 4) X(128, 8) X(256, 1) X(256, 2) X(256, 4)
+
+template <int MODE>
+ep_status_t launch_dispatch(const ep::DispatchArgs &a, cudaStream_t s) {
+    const Split sp = split_rows(a.N, a.H / 16);
+    const unsigned grid = grid_for(a.N, ep::kDispatchThreads, sp.tpt);
+#define EP_CASE(T_, G_)                                                                     \
+    if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
+        ep::dispatch_kernel<MODE, T_, G_><<<grid, ep::kDispatchThreads, 0, s>>>(a);         \
+        return launched();                                                                  \
+    }
+    EP_SPLITS(EP_CASE)
+#undef EP_CASE
+    return EP_ERR_UNSUPPORTED;
+}
+
+// The backward quantises every entry separately (K scaled copies of the
+// row), so its per-thread state grows with G: keep G <= 2 (about 60
+// registers) for occupancy.
 ep_status_t launch_combine_bwd(const ep::DispatchArgs &a, cudaStream_t s) {
-    const int ng = a.H / 16;
-    auto grid = [&](int tpt) { return (unsigned)((a.N + (ep::kDispatchThreads / tpt) - 1) /
-                                                 (ep::kDispatchThreads / tpt)); };
-    if (ng <= 32) ep::combine_bwd_kernel<32, 1><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
-    else if (ng <= 64) ep::combine_bwd_kernel<32, 2><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
-    else if (ng <= 128) ep::combine_bwd_kernel<32, 4><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
-    else if (ng <= 256) ep::combine_bwd_kernel<32, 8><<<grid(32), ep::kDispatchThreads, 0, s>>>(a);
-    else ep::combine_bwd_kernel<64, 8><<<grid(64), ep::kDispatchThreads, 0, s>>>(a);
-    return launched();
+    const Split sp = split_rows(a.N, a.H / 16, 2);
+    const unsigned grid = grid_for(a.N, ep::kDispatchThreads, sp.tpt);
+#define EP_CASE(T_, G_)                                                                     \
+    if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
+        ep::combine_bwd_kernel<T_, G_><<<grid, ep::kDispatchThreads, 0, s>>>(a);            \
+        return launched();                                                                  \
+    }
+    EP_SPLITS(EP_CASE)
+#undef EP_CASE
+    return EP_ERR_UNSUPPORTED;
 }
 
 ep::DispatchArgs dispatch_args(const ep_config_t *cfg, const Plan &p) {
@@ -301,15 +402,17 @@ ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t 
     a.cap = p.cap; a.rows = p.rows;
     a.y = y; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
     a.out = out; a.status = dev_status;
-    constexpr int TPT = 128, TOKS = ep::kCombineThreads / TPT;
-    const unsigned grid = (unsigned)((p.N + TOKS - 1) / TOKS);
-    const int ng = p.H / 8;
     cudaStream_t s = cs(stream);
-    if (ng <= TPT) ep::combine_kernel<TPT, 1, 8><<<grid, ep::kCombineThreads, 0, s>>>(a);
-    else if (ng <= 2 * TPT) ep::combine_kernel<TPT, 2, 8><<<grid, ep::kCombineThreads, 0, s>>>(a);
-    else if (ng <= 4 * TPT) ep::combine_kernel<TPT, 4, 8><<<grid, ep::kCombineThreads, 0, s>>>(a);
-    else ep::combine_kernel<TPT, 8, 8><<<grid, ep::kCombineThreads, 0, s>>>(a);
-    return launched();
+    const Split sp = split_rows(p.N, p.H / 8);  // 8-element granules (16 bytes of bf16)
+    const unsigned grid = grid_for(p.N, ep::kCombineThreads, sp.tpt);
+#define EP_CASE(T_, G_)                                                                     \
+    if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
+        ep::combine_kernel<T_, G_, 8><<<grid, ep::kCombineThreads, 0, s>>>(a);              \
+        return launched();                                                                  \
+    }
+    EP_SPLITS(EP_CASE)
+#undef EP_CASE
+    return EP_ERR_UNSUPPORTED;
 }
 
 ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
@@ -419,7 +522,6 @@ namespace {
 
 __device__ __align__(256) unsigned char g_static_scratch[EP_STATIC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_static_mu;
 void *g_static_ptr[kMaxDevices] = {};
 
@@ -471,14 +573,5 @@ extern "C" ep_status_t ep_dispatch_layout_static(
     a.ws_rk = a.ws_hist + (int64_t)p.E * p.C;
     a.status = dev_status;
 
-    cudaStream_t s = cs(stream);
-    if (p.C > 0) {
-        ep::layout_count_kernel<<<p.C, ep::kLayoutThreads, (p.E + p.R) * sizeof(int), s>>>(a);
-        if ((st = launched()) != EP_OK) return st;
-    }
-    ep::layout_scan_kernel<<<p.E + p.R, ep::kLayoutThreads, 0, s>>>(a);
-    if ((st = launched()) != EP_OK) return st;
-    const size_t smem = (size_t)(ep::kLayoutThreads / 32) * p.E * sizeof(int);
-    ep::layout_assign_kernel<<<p.C > 0 ? p.C : 1, ep::kLayoutThreads, smem, s>>>(a);
-    return launched();
+    return launch_layout_multi(a, p, cs(stream));
 }
