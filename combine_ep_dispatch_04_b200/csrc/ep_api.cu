@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstring>
+#include <map>
 #include <mutex>
 
 #include "ep.h"
@@ -19,9 +20,11 @@ std::atomic<uint64_t> g_launches{0};
 constexpr int kMaxExperts = 1024;
 constexpr int kMaxHidden = 8192;
 constexpr int64_t kIntLimit = (int64_t(1) << 31) - 1;
-// one-block layout when the routing is small and its counters fit in the
-// default 48 KB of shared memory
-constexpr int64_t kSingleMaxEntries = 32768;
+// Layout paths by routing size: one block up to kSingleMaxEntries entries, one
+// thread-block cluster up to kClusterMaxEntries, three multi-block launches
+// beyond.
+constexpr int64_t kSingleMaxEntries = 2048;
+constexpr int64_t kClusterMaxEntries = 131072;
 constexpr size_t kDefaultSmem = 48 * 1024;
 constexpr size_t kMaxSmem = 200 * 1024;
 
@@ -30,6 +33,25 @@ cudaStream_t cs(ep_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int64_t round_up(int64_t v, int64_t a) { return (v + a - 1) / a * a; }
+
+// Launch with programmatic stream serialisation (see pdl_enter in
+// ep_device.cuh): the kernel may begin while the previous grid on the stream
+// drains, and waits for it before touching memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                   Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 
 ep_status_t launched() {
     g_launches.fetch_add(1, std::memory_order_relaxed);
@@ -71,10 +93,11 @@ ep_status_t make_plan(const ep_config_t *c, Plan &p) {
     if (c->layout != EP_LAYOUT_PADDED && c->layout != EP_LAYOUT_PACKED) return EP_ERR_INVALID_ARG;
     if (c->expert_align < 1) return EP_ERR_INVALID_ARG;
     if (!(c->e4m3_qmax >= 0.0f && c->e4m3_qmax <= 448.0f)) return EP_ERR_INVALID_ARG;  // NaN fails
-    const uint32_t known = EP_F_BWD_UNWEIGHTED | EP_F_LAYOUT_SINGLE_CTA | EP_F_LAYOUT_MULTI_CTA;
+    const uint32_t paths = EP_F_LAYOUT_SINGLE_CTA | EP_F_LAYOUT_MULTI_CTA | EP_F_LAYOUT_CLUSTER;
+    const uint32_t known = EP_F_BWD_UNWEIGHTED | paths;
     if (c->flags & ~known) return EP_ERR_INVALID_ARG;
-    if ((c->flags & EP_F_LAYOUT_SINGLE_CTA) && (c->flags & EP_F_LAYOUT_MULTI_CTA))
-        return EP_ERR_INVALID_ARG;
+    const uint32_t forced = c->flags & paths;
+    if (forced & (forced - 1)) return EP_ERR_INVALID_ARG;  // at most one path flag
 
     p.R = c->num_ranks;
     p.T = c->num_tokens;
@@ -172,7 +195,102 @@ ep_status_t launch_layout_single(ep::LayoutArgs a, const SinglePlan &sp, cudaStr
     a.CR = sp.CR;
     a.C = sp.C;
     if (!allow_smem(ep::layout_single_kernel, 0, sp.smem)) return EP_ERR_CUDA;
-    ep::layout_single_kernel<<<1, sp.warps * 32, sp.smem, s>>>(a);
+    launch(ep::layout_single_kernel, 1, sp.warps * 32, sp.smem, s, a);
+    return launched();
+}
+
+// One cluster of Q blocks of 512 threads: chunks of whole tokens of one
+// source rank, about one per warp of the cluster, contiguous per block.
+// Shared memory per block: [off: CPQ*E][tot: E][msk: W*E][rank_of: E][keys],
+// each part rounded up to a multiple of 4 ints.
+constexpr int kClusterThreads = 512;
+
+struct ClusterChoice {
+    bool ok;
+    ep::ClusterPlan cp;
+    size_t smem;
+};
+
+// Largest cluster size that can be resident (16 needs the non-portable
+// attribute), checked once per device.
+int cluster_size_limit() {
+    static std::mutex mu;
+    static int limit[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 8;
+    std::lock_guard<std::mutex> lock(mu);
+    if (limit[dev]) return limit[dev];
+    int q = 8;
+    if (cudaFuncSetAttribute(ep::layout_cluster_kernel,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
+        cudaFuncSetAttribute(ep::layout_cluster_kernel,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem) ==
+            cudaSuccess) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(16);
+        cfg.blockDim = dim3(kClusterThreads);
+        cfg.dynamicSmemBytes = kMaxSmem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 16;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, ep::layout_cluster_kernel, &cfg) == cudaSuccess &&
+            n >= 1)
+            q = 16;
+    }
+    cudaGetLastError();  // a refused query leaves no sticky error
+    limit[dev] = q;
+    return q;
+}
+
+ClusterChoice plan_cluster(const Plan &p) {
+    const int W = kClusterThreads / 32;
+    auto r4 = [](int64_t v) { return (v + 3) & ~int64_t(3); };
+    for (int Q = cluster_size_limit(); Q >= 2; Q /= 2) {
+        ep::ClusterPlan cp{};
+        cp.Q = Q;
+        int cr = (Q * W + p.R - 1) / p.R;
+        if (cr > p.T) cr = p.T > 0 ? p.T : 1;
+        cp.TC = p.T > 0 ? (p.T + cr - 1) / cr : 1;
+        cp.CR = p.T > 0 ? (p.T + cp.TC - 1) / cp.TC : 0;
+        cp.C = p.R * cp.CR;
+        cp.CPQ = (cp.C + Q - 1) / Q;
+        const int64_t ints = r4((int64_t)cp.CPQ * p.E) + r4(p.E) + r4((int64_t)W * p.E) + r4(p.E) +
+                             r4((int64_t)cp.CPQ * cp.TC * p.K);
+        const size_t smem = (size_t)ints * sizeof(int);
+        if (smem <= kMaxSmem) return {true, cp, smem};
+    }
+    ClusterChoice none{};
+    return none;
+}
+
+ep_status_t launch_layout_cluster(const ep::LayoutArgs &a, const ClusterChoice &cc,
+                                  cudaStream_t s) {
+    if (!cc.ok) return EP_ERR_UNSUPPORTED;
+    if (cc.cp.Q > 8 &&
+        cudaFuncSetAttribute(ep::layout_cluster_kernel,
+                             cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
+        return EP_ERR_CUDA;
+    if (!allow_smem(ep::layout_cluster_kernel, 4, cc.smem)) return EP_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cc.cp.Q);
+    cfg.blockDim = dim3(kClusterThreads);
+    cfg.dynamicSmemBytes = cc.smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cc.cp.Q;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cudaLaunchKernelEx(&cfg, ep::layout_cluster_kernel, a, cc.cp);
     return launched();
 }
 
@@ -181,14 +299,14 @@ ep_status_t launch_layout_multi(const ep::LayoutArgs &a, const Plan &p, cudaStre
     if (p.C > 0) {
         const size_t smem = (size_t)(p.TC * p.K + p.E + p.R) * sizeof(int);
         if (!allow_smem(ep::layout_count_kernel, 2, smem)) return EP_ERR_CUDA;
-        ep::layout_count_kernel<<<p.C, ep::kLayoutThreads, smem, s>>>(a);
+        launch(ep::layout_count_kernel, p.C, ep::kLayoutThreads, smem, s, a);
         if ((st = launched()) != EP_OK) return st;
     }
-    ep::layout_scan_kernel<<<p.E + p.R, ep::kLayoutThreads, 0, s>>>(a);
+    launch(ep::layout_scan_kernel, p.E + p.R, ep::kLayoutThreads, 0, s, a);
     if ((st = launched()) != EP_OK) return st;
     const size_t smem = (size_t)(p.TC * p.K + 2 * (ep::kLayoutThreads / 32) * p.E) * sizeof(int);
     if (!allow_smem(ep::layout_assign_kernel, 3, smem)) return EP_ERR_CUDA;
-    ep::layout_assign_kernel<<<p.C > 0 ? p.C : 1, ep::kLayoutThreads, smem, s>>>(a);
+    launch(ep::layout_assign_kernel, p.C > 0 ? p.C : 1, ep::kLayoutThreads, smem, s, a);
     return launched();
 }
 
@@ -265,11 +383,18 @@ ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const int64_t *topk_idx,
     a.status = dev_status;
 
     cudaStream_t s = cs(stream);
-    const SinglePlan sp = plan_single(p);
-    const bool single = (cfg->flags & EP_F_LAYOUT_SINGLE_CTA) ||
-                        (!(cfg->flags & EP_F_LAYOUT_MULTI_CTA) && p.N * p.K <= kSingleMaxEntries &&
-                         sp.ok);
-    if (single) return launch_layout_single(a, sp, s);
+    if (cfg->flags & EP_F_LAYOUT_SINGLE_CTA) return launch_layout_single(a, plan_single(p), s);
+    if (cfg->flags & EP_F_LAYOUT_MULTI_CTA) return launch_layout_multi(a, p, s);
+    if (cfg->flags & EP_F_LAYOUT_CLUSTER) return launch_layout_cluster(a, plan_cluster(p), s);
+    const int64_t entries = p.N * p.K;
+    if (entries <= kSingleMaxEntries) {
+        const SinglePlan sp = plan_single(p);
+        if (sp.ok) return launch_layout_single(a, sp, s);
+    }
+    if (entries <= kClusterMaxEntries) {
+        const ClusterChoice cc = plan_cluster(p);
+        if (cc.ok) return launch_layout_cluster(a, cc, s);
+    }
     return launch_layout_multi(a, p, s);
 }
 
@@ -277,23 +402,52 @@ ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const int64_t *topk_idx,
 
 namespace {
 
-// Threads per token (TPT) and granules per thread (G): the smallest TPT that
-// keeps G <= max_g (8 unless stated), doubled (up to 256, and up to one granule per thread) while
-// the grid has fewer than kTargetWarps warps -- few tokens (decode) then
-// spread each row over more warps instead of leaving SMs idle.
-constexpr int64_t kTargetWarps = 8192;
-
+// Threads per token (TPT) and granules per thread (G).  When the grid can
+// fit in one wave of resident blocks, take the largest TPT that does (few
+// tokens -- decode -- then spread each row over up to 8 warps, and no second,
+// partial wave doubles the tail); otherwise (many waves) the smallest TPT
+// with G <= max_g.  TPT never exceeds the granule count by more than a warp.
 struct Split {
     int tpt, gmax;
 };
 
-Split split_rows(int64_t N, int ngran, int max_g = 8) {
+int pow2_at_least(int g) { return g <= 1 ? 1 : (g <= 2 ? 2 : (g <= 4 ? 4 : 8)); }
+
+// Resident blocks per SM of a kernel, queried once per function and device.
+int blocks_per_sm(const void *fn, int threads) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, int> cache;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find({fn, dev});
+    if (it != cache.end()) return it->second;
+    int nb = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, fn, threads, 0) != cudaSuccess || nb < 1)
+        nb = 1;
+    cache[{fn, dev}] = nb;
+    return nb;
+}
+
+int sm_count();
+
+// `kernel_of(tpt, gmax)` returns the kernel instance (nullptr if none).
+template <typename KernelOf>
+Split split_rows(int64_t N, int ngran, int threads, int max_g, KernelOf kernel_of) {
+    const int64_t sms = sm_count();
+    for (int tpt = 256; tpt >= 32; tpt >>= 1) {
+        if (tpt > 32 && tpt / 2 >= ngran) continue;  // more than a warp of idle threads
+        const int g = (ngran + tpt - 1) / tpt;
+        if (g > max_g) break;
+        const int gmax = pow2_at_least(g);
+        const void *fn = kernel_of(tpt, gmax);
+        if (!fn) continue;
+        const int64_t ctas = (N + threads / tpt - 1) / (threads / tpt);
+        if (ctas <= sms * blocks_per_sm(fn, threads)) return {tpt, gmax};
+    }
     int tpt = 32;
     while (tpt < 256 && (ngran + tpt - 1) / tpt > max_g) tpt *= 2;
-    while (tpt < 256 && tpt < ngran && N * (tpt / 32) < kTargetWarps) tpt *= 2;
-    const int g = (ngran + tpt - 1) / tpt;
-    const int gmax = g <= 1 ? 1 : (g <= 2 ? 2 : (g <= 4 ? 4 : 8));
-    return {tpt, gmax};
+    return {tpt, pow2_at_least((ngran + tpt - 1) / tpt)};
 }
 
 unsigned grid_for(int64_t N, int threads, int tpt) {
@@ -309,11 +463,17 @@ unsigned grid_for(int64_t N, int threads, int tpt) {
 
 template <int MODE>
 ep_status_t launch_dispatch(const ep::DispatchArgs &a, cudaStream_t s) {
-    const Split sp = split_rows(a.N, a.H / 16);
+    auto kernel_of = [](int t, int g) -> const void * {
+#define EP_FN(T_, G_) if (t == T_ && g == G_) return (const void *)ep::dispatch_kernel<MODE, T_, G_>;
+        EP_SPLITS(EP_FN)
+#undef EP_FN
+        return nullptr;
+    };
+    const Split sp = split_rows(a.N, a.H / 16, ep::kDispatchThreads, 8, kernel_of);
     const unsigned grid = grid_for(a.N, ep::kDispatchThreads, sp.tpt);
 #define EP_CASE(T_, G_)                                                                     \
     if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
-        ep::dispatch_kernel<MODE, T_, G_><<<grid, ep::kDispatchThreads, 0, s>>>(a);         \
+        launch(ep::dispatch_kernel<MODE, T_, G_>, grid, ep::kDispatchThreads, 0, s, a);     \
         return launched();                                                                  \
     }
     EP_SPLITS(EP_CASE)
@@ -325,11 +485,17 @@ ep_status_t launch_dispatch(const ep::DispatchArgs &a, cudaStream_t s) {
 // row), so its per-thread state grows with G: keep G <= 2 (about 60
 // registers) for occupancy.
 ep_status_t launch_combine_bwd(const ep::DispatchArgs &a, cudaStream_t s) {
-    const Split sp = split_rows(a.N, a.H / 16, 2);
+    auto kernel_of = [](int t, int g) -> const void * {
+#define EP_FN(T_, G_) if (t == T_ && g == G_) return (const void *)ep::combine_bwd_kernel<T_, G_>;
+        EP_SPLITS(EP_FN)
+#undef EP_FN
+        return nullptr;
+    };
+    const Split sp = split_rows(a.N, a.H / 16, ep::kDispatchThreads, 2, kernel_of);
     const unsigned grid = grid_for(a.N, ep::kDispatchThreads, sp.tpt);
 #define EP_CASE(T_, G_)                                                                     \
     if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
-        ep::combine_bwd_kernel<T_, G_><<<grid, ep::kDispatchThreads, 0, s>>>(a);            \
+        launch(ep::combine_bwd_kernel<T_, G_>, grid, ep::kDispatchThreads, 0, s, a);        \
         return launched();                                                                  \
     }
     EP_SPLITS(EP_CASE)
@@ -403,11 +569,18 @@ ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t 
     a.y = y; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
     a.out = out; a.status = dev_status;
     cudaStream_t s = cs(stream);
-    const Split sp = split_rows(p.N, p.H / 8);  // 8-element granules (16 bytes of bf16)
+    auto kernel_of = [](int t, int g) -> const void * {
+#define EP_FN(T_, G_) if (t == T_ && g == G_) return (const void *)ep::combine_kernel<T_, G_, 8>;
+        EP_SPLITS(EP_FN)
+#undef EP_FN
+        return nullptr;
+    };
+    // 8-element granules (16 bytes of bf16)
+    const Split sp = split_rows(p.N, p.H / 8, ep::kCombineThreads, 8, kernel_of);
     const unsigned grid = grid_for(p.N, ep::kCombineThreads, sp.tpt);
 #define EP_CASE(T_, G_)                                                                     \
     if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
-        ep::combine_kernel<T_, G_, 8><<<grid, ep::kCombineThreads, 0, s>>>(a);              \
+        launch(ep::combine_kernel<T_, G_, 8>, grid, ep::kCombineThreads, 0, s, a);          \
         return launched();                                                                  \
     }
     EP_SPLITS(EP_CASE)
@@ -480,7 +653,7 @@ __global__ void cvt_sweep_kernel(int format, uint32_t start, int64_t n, uint8_t 
 }  // namespace ep
 
 namespace {
-int sm_count() {
+int sm_count() {  // declared above
     int dev = 0, n = 148;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);

@@ -37,6 +37,7 @@ constexpr int kCombineThreads = 256;
 
 template <int TPT, int GMAX, int KB>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
+    pdl_enter();
     constexpr int TOKS = kCombineThreads / TPT;
     __shared__ int64_t s_row[TOKS][16];
     __shared__ float s_w[TOKS][16];

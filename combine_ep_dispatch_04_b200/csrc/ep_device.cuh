@@ -92,6 +92,17 @@ __device__ __forceinline__ uint4 ld_ro(const void *p) {
 __device__ __forceinline__ void st_v4(void *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
 __device__ __forceinline__ void st_v2(void *p, uint2 v) { *reinterpret_cast<uint2 *>(p) = v; }
 
+// Programmatic dependent launch: every kernel of the library is launched so
+// that it may start while the previous grid on the stream finishes.  Before
+// touching global memory it waits until that grid has completed and its
+// writes are visible (a no-op when there is no such grid), then lets its own
+// dependents start launching.  Nothing is read before the wait, so this is
+// safe whatever kernel precedes.
+__device__ __forceinline__ void pdl_enter() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t lanemask_lt() {
     uint32_t m;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(m));

@@ -80,6 +80,7 @@ __device__ __forceinline__ uint32_t q_i8(float v, float s) {
 
 template <int MODE, int TPT, int GMAX>
 __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs a) {
+    pdl_enter();
     constexpr int TOKS = kDispatchThreads / TPT;
     constexpr int WPG = TPT / 32;  // warps per token group
     constexpr int OB = GranOut<MODE>::bytes;
@@ -258,6 +259,7 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
 // symmetric, so it is taken once per token and scaled per entry.
 template <int TPT, int GMAX>
 __global__ void __launch_bounds__(kDispatchThreads) combine_bwd_kernel(DispatchArgs a) {
+    pdl_enter();
     constexpr int TOKS = kDispatchThreads / TPT;
     __shared__ int64_t s_row[TOKS][16];
     __shared__ float s_w[TOKS][16];

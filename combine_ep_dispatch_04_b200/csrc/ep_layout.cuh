@@ -32,6 +32,8 @@
 // sum of order-free atomics, so the result never depends on thread timing.
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "ep_device.cuh"
 
 namespace ep {
@@ -207,6 +209,7 @@ __device__ __forceinline__ void write_expert_offset(const LayoutArgs &a, int *wa
 // ---- multi-block path ------------------------------------------------------------
 
 __global__ void __launch_bounds__(kLayoutThreads) layout_count_kernel(LayoutArgs a) {
+    pdl_enter();
     extern __shared__ int sm[];
     const int c = blockIdx.x, r = c / a.CR, j = c % a.CR;
     const int t0 = j * a.TC, t1 = min(a.T, t0 + a.TC);
@@ -231,6 +234,7 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_count_kernel(LayoutArgs
 }
 
 __global__ void __launch_bounds__(kLayoutThreads) layout_scan_kernel(LayoutArgs a) {
+    pdl_enter();
     __shared__ int warp_sums[kLayoutThreads / 32];
     const int b = blockIdx.x;
     if (b < a.E) {
@@ -272,6 +276,7 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_scan_kernel(LayoutArgs 
 }
 
 __global__ void __launch_bounds__(kLayoutThreads) layout_assign_kernel(LayoutArgs a) {
+    pdl_enter();
     extern __shared__ int sm[];
     __shared__ int warp_sums[kLayoutThreads / 32];
     constexpr int W = kLayoutThreads / 32;
@@ -331,6 +336,7 @@ __global__ void __launch_bounds__(kLayoutThreads) layout_assign_kernel(LayoutArg
 // gives each expert's rank (no integer division), and zeroing uses 16-byte
 // stores.  Same result as the multi-block path, bit for bit.
 __global__ void __launch_bounds__(1024, 1) layout_single_kernel(LayoutArgs a) {
+    pdl_enter();
     extern __shared__ __align__(16) int sm[];
     __shared__ int warp_sums[32];
     const int W = blockDim.x >> 5;
@@ -475,6 +481,199 @@ __global__ void __launch_bounds__(1024, 1) layout_single_kernel(LayoutArgs a) {
     }
     if (over) atomicOr(a.status, kDevCapacity);
     if (a.eo) {
+        __syncthreads();
+        write_expert_offset(a, warp_sums);
+    }
+}
+
+// ---- cluster path -------------------------------------------------------------------
+// One thread-block cluster of Q blocks (Q <= 16, all co-scheduled, hardware
+// cluster barriers) spreads the one-block design over Q SMs.  The N tokens
+// are cut into C chunks of whole tokens of one source rank; block q owns the
+// contiguous chunks [q*CPQ, (q+1)*CPQ) and warp w of a block owns its local
+// chunks w, w+W, ...
+//   0  every block stages its chunks' entries; block 0 zeroes the global
+//      per-rank counters.                                       cluster barrier
+//   1  per-chunk expert counts, is_token_in_rank rows, tokens_per_rank
+//      (ballots, global atomics).
+//   2a per expert: local exclusive scan over the block's chunks, the block
+//      total tot[e], and each rank's share added to tokens_per_expert.
+//                                                               cluster barrier
+//   2b per expert: the block's base is the sum of tot[e] of the lower blocks,
+//      read from their shared memory; block 0 sums all blocks for recv_count,
+//      the stats and expert_offset.                              cluster barrier
+//      (after it no block reads another block's shared memory)
+//   3  stable ranks of each chunk, 32 entries a step.
+// Counts are order-free integer sums, so the result is the one of the other
+// paths, bit for bit.
+struct ClusterPlan {
+    int Q, TC, CR, C, CPQ;
+};
+
+__global__ void __launch_bounds__(512, 1) layout_cluster_kernel(LayoutArgs a, ClusterPlan cp) {
+    pdl_enter();
+    namespace cg = cooperative_groups;
+    cg::cluster_group cluster = cg::this_cluster();
+    extern __shared__ __align__(16) int sm[];
+    __shared__ int warp_sums[32];
+    const int q = (int)cluster.block_rank();
+    const int W = blockDim.x >> 5;
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int E = a.E, R = a.R, K = a.K, T = a.T;
+    const int TC = cp.TC, CR = cp.CR, C = cp.C, CPQ = cp.CPQ;
+    const int c_lo = min(C, q * CPQ), c_hi = min(C, c_lo + CPQ), nloc = c_hi - c_lo;
+    // entries of this block: chunks are contiguous in entry order
+    auto chunk_first_entry = [&](int c) {
+        const int r = c / CR, j = c - r * CR;
+        return (r * T + min(T, j * TC)) * K;
+    };
+    const int f0 = nloc > 0 ? chunk_first_entry(c_lo) : 0;
+    const int f1 = nloc > 0 ? (c_hi % CR == 0 ? (c_hi / CR) * T * K : chunk_first_entry(c_hi)) : 0;
+    const int nent = f1 - f0;
+
+    // shared memory: [off: CPQ*E][tot: E][msk: W*E][rank_of: E][keys: nent]
+    const int off_n = (CPQ * E + 3) & ~3, e4 = (E + 3) & ~3, msk_n = (W * E + 3) & ~3;
+    int *off = sm;
+    int *tot = sm + off_n;
+    uint32_t *msk = reinterpret_cast<uint32_t *>(sm + off_n + e4);
+    int *rank_of = sm + off_n + e4 + msk_n;
+    int *keys = rank_of + e4;
+
+    {
+        int4 *z = reinterpret_cast<int4 *>(sm);
+        const int n4 = (off_n + e4 + msk_n) >> 2;
+        for (int i = threadIdx.x; i < n4; i += blockDim.x) z[i] = make_int4(0, 0, 0, 0);
+    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) rank_of[e] = e / a.L;
+    if (q == 0) {
+        if (a.tpr) for (int i = threadIdx.x; i < R * R; i += blockDim.x) a.tpr[i] = 0;
+        if (a.tpe) for (int i = threadIdx.x; i < R * E; i += blockDim.x) a.tpe[i] = 0;
+    }
+    if (stage_keys(a.idx, f0, nent, E, keys)) atomicOr(a.status, kDevBadIndex);
+    cluster.sync();
+
+    // phase 1
+    for (int lc = w; lc < nloc; lc += W) {
+        const int c = c_lo + lc;
+        const int r = c / CR, j = c - r * CR;
+        const int t0 = j * TC, t1 = min(T, t0 + TC);
+        int *coff = off + lc * E;
+        int rc0 = 0, rc1 = 0;
+        for (int tb = t0; tb < t1; tb += 32) {
+            const int t = tb + lane;
+            uint64_t mask = 0;
+            if (t < t1) {
+                const int n = r * T + t;
+                const int *tk = keys + (n * K - f0);
+                for (int k = 0; k < K; k++) {
+                    const int e = tk[k];
+                    if (e >= 0) {
+                        atomicAdd(&coff[e], 1);
+                        mask |= 1ull << (rank_of[e] & 63);
+                    }
+                }
+                if (R > 64) {
+                    token_ranks(tk, K, a.L, R, a.itr ? a.itr + (int64_t)n * R : nullptr,
+                                a.tpr ? a.tpr + (int64_t)r * R : nullptr);
+                } else if (a.itr) {
+                    uint8_t *row = a.itr + (int64_t)n * R;
+                    if ((R & 3) == 0) {
+                        for (int d = 0; d < R; d += 4) {
+                            const uint32_t bits = (uint32_t)(mask >> d);
+                            reinterpret_cast<uint32_t *>(row)[d >> 2] =
+                                (bits & 1u) | ((bits >> 1) & 1u) << 8 | ((bits >> 2) & 1u) << 16 |
+                                ((bits >> 3) & 1u) << 24;
+                        }
+                    } else {
+                        for (int d = 0; d < R; d++) row[d] = (uint8_t)((mask >> d) & 1u);
+                    }
+                }
+            }
+            if (R <= 64) {
+                for (int d = 0; d < R; d++) {
+                    const int cnt = __popc(__ballot_sync(kFull, (mask >> d) & 1ull));
+                    if (d == lane) rc0 += cnt;
+                    if (d == lane + 32) rc1 += cnt;
+                }
+            }
+        }
+        if (R <= 64 && a.tpr) {
+            if (lane < R && rc0) atomicAdd(&a.tpr[(int64_t)r * R + lane], rc0);
+            if (lane + 32 < R && rc1) atomicAdd(&a.tpr[(int64_t)r * R + lane + 32], rc1);
+        }
+    }
+    __syncthreads();
+
+    // phase 2a: local scan over the block's chunks; per-rank shares of tpe
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int run = 0, rank_run = 0;
+        int cur_r = nloc > 0 ? c_lo / CR : 0;
+        for (int lc = 0; lc < nloc; lc++) {
+            const int r = (c_lo + lc) / CR;
+            if (r != cur_r) {
+                if (a.tpe && rank_run) atomicAdd(&a.tpe[(int64_t)cur_r * E + e], rank_run);
+                cur_r = r;
+                rank_run = 0;
+            }
+            const int v = off[lc * E + e];
+            off[lc * E + e] = run;
+            run += v;
+            rank_run += v;
+        }
+        if (a.tpe && rank_run) atomicAdd(&a.tpe[(int64_t)cur_r * E + e], rank_run);
+        tot[e] = run;
+    }
+    cluster.sync();
+
+    // phase 2b: bases from the lower blocks' totals (distributed shared memory)
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int base = 0;
+        for (int q2 = 0; q2 < q; q2++) base += cluster.map_shared_rank(tot, q2)[e];
+        for (int lc = 0; lc < nloc; lc++) off[lc * E + e] += base;
+        if (q == 0) {
+            int all = 0;
+            for (int q2 = 0; q2 < cp.Q; q2++) all += cluster.map_shared_rank(tot, q2)[e];
+            a.recv_count[e] = all;
+            if (a.stats) a.stats[e] += all;
+        }
+    }
+    cluster.sync();  // no shared-memory reads across blocks after this point
+
+    // phase 3: stable ranks, each warp over its local chunks in order
+    uint32_t *wmsk = msk + w * E;
+    const uint32_t lt = lanemask_lt();
+    bool over = false;
+    for (int lc = w; lc < nloc; lc += W) {
+        const int c = c_lo + lc;
+        const int r = c / CR, j = c - r * CR;
+        const int t0 = j * TC, t1 = min(T, t0 + TC);
+        const int g_lo = (r * T + t0) * K, g_hi = (r * T + t1) * K;  // global entry range
+        int *coff = off + lc * E;
+        for (int b0 = g_lo; b0 < g_hi; b0 += 32) {
+            const int f = b0 + lane;
+            const int key = f < g_hi ? keys[f - f0] : -1;
+            if (key >= 0) atomicOr(&wmsk[key], 1u << lane);
+            __syncwarp();
+            uint32_t m = 0;
+            int base = 0;
+            if (key >= 0) {
+                m = wmsk[key];
+                base = coff[key];
+            }
+            __syncwarp();
+            const int rank = __popc(m & lt);
+            if (key >= 0 && rank == 0) {
+                coff[key] = base + __popc(m);
+                wmsk[key] = 0u;
+            }
+            __syncwarp();
+            const int sl = key >= 0 ? base + rank : -1;
+            if (f < g_hi) a.slot[f] = sl;
+            if (!a.packed && sl >= a.cap) over = true;
+        }
+    }
+    if (over) atomicOr(a.status, kDevCapacity);
+    if (q == 0 && a.eo) {
         __syncthreads();
         write_expert_offset(a, warp_sums);
     }

@@ -27,6 +27,7 @@ DEV_CAPACITY_OVERFLOW = 0x2
 F_BWD_UNWEIGHTED = 0x1
 F_LAYOUT_SINGLE_CTA = 0x100
 F_LAYOUT_MULTI_CTA = 0x200
+F_LAYOUT_CLUSTER = 0x400
 
 STATIC_SCRATCH_BYTES = 1 << 20  # EP_STATIC_SCRATCH_BYTES of include/ep.h
 

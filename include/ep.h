@@ -84,6 +84,7 @@ typedef enum {
 #define EP_F_BWD_UNWEIGHTED 0x1u    /* combine-backward re-dispatches g without w */
 #define EP_F_LAYOUT_SINGLE_CTA 0x100u /* force the one-block layout path */
 #define EP_F_LAYOUT_MULTI_CTA 0x200u  /* force the multi-block layout path */
+#define EP_F_LAYOUT_CLUSTER 0x400u    /* force the thread-block-cluster layout path */
 
 typedef struct {
     int32_t num_ranks;           /* R > 0 */

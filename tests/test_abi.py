@@ -65,6 +65,8 @@ def test_sizes_packed_every_mode(quant, D, S):
     dict(quant=7), dict(layout=2), dict(expert_align=0), dict(e4m3_qmax=449.0),
     dict(e4m3_qmax=float("nan")), dict(e4m3_qmax=-1.0), dict(flags=0x8000),
     dict(flags=ep.F_LAYOUT_MULTI_CTA | ep.F_LAYOUT_SINGLE_CTA),
+    dict(flags=ep.F_LAYOUT_CLUSTER | ep.F_LAYOUT_SINGLE_CTA),
+    dict(flags=ep.F_LAYOUT_CLUSTER | ep.F_LAYOUT_MULTI_CTA),
     dict(quant="e4m3_b128", H=96),
 ])
 def test_invalid_configs_rejected(bad):

@@ -88,9 +88,10 @@ def test_prefill_workload_full_size_sampled():
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("name,override", [
     ("decode", {}), ("skewed", dict(T=100)), ("large", dict(T=40)), ("tiny", {}),
-    ("prefill", dict(T=33, E=1024)),
+    ("prefill", dict(T=33, E=1024)), ("skewed", dict(R=3, E=6, K=4, T=1000, M=1000)),
 ])
-@pytest.mark.parametrize("path", [ep.F_LAYOUT_SINGLE_CTA, ep.F_LAYOUT_MULTI_CTA])
+@pytest.mark.parametrize("path", [ep.F_LAYOUT_SINGLE_CTA, ep.F_LAYOUT_MULTI_CTA,
+                                  ep.F_LAYOUT_CLUSTER])
 def test_layout_paths(name, override, path):
     w = synth.workload(name, **override)
     r = Run(w, "bf16", layout="packed", align=4, flags=path)
@@ -117,7 +118,8 @@ def test_every_mode_small_ragged(mode, layout):
     r.check_backward()
 
 
-@pytest.mark.parametrize("path", [ep.F_LAYOUT_SINGLE_CTA, ep.F_LAYOUT_MULTI_CTA])
+@pytest.mark.parametrize("path", [ep.F_LAYOUT_SINGLE_CTA, ep.F_LAYOUT_MULTI_CTA,
+                                  ep.F_LAYOUT_CLUSTER])
 def test_zero_tokens(path):
     w = _edge(T=0)
     r = Run(w, "mxfp8", layout="packed", flags=path)
@@ -265,3 +267,17 @@ def test_python_checks_reject_prequantised_input():
     with pytest.raises(ValueError):
         ep.ep_dispatch_layout(cfg, idx.t().contiguous().t(), b.token_slot, b.recv_count,
                               b.workspace, b.dev_status)
+
+
+@pytest.mark.parametrize("path", [ep.F_LAYOUT_SINGLE_CTA, ep.F_LAYOUT_MULTI_CTA,
+                                  ep.F_LAYOUT_CLUSTER])
+def test_layout_paths_bad_indices_and_duplicates(path):
+    w = _edge(R=4, T=37, M=40, K=5, E=8)
+    idx, wts = synth.make_routing(w)
+    idx[::3, 1] = idx[::3, 0]          # duplicates
+    idx[5, 2] = w["E"] + 3             # out of range
+    idx[7, 0] = -9
+    r = Run(w, "mxfp8", layout="packed", align=3, idx=idx, wts=wts, flags=path, stats=True)
+    assert r.status & ep.DEV_BAD_INDEX
+    r.check_layout()
+    r.check_dispatch()
