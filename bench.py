@@ -54,6 +54,8 @@ def parse():
     p.add_argument("--steps", type=int, default=300)
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--workload", default="decode", choices=sorted(synth.WORKLOADS))
+    p.add_argument("--tokens-per-rank", type=int, default=None,
+                   help="override T (profiling a reduced case; the reported workload says so)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--flush-mib", type=int, default=512)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -282,7 +284,8 @@ def main():
     args = parse()
     world, rank, local = dist_init()
     wname = args.workload
-    w = synth.workload(wname)
+    w = synth.workload(wname) if args.tokens_per_rank is None else \
+        synth.workload(wname, T=args.tokens_per_rank)
     mode = WORKLOAD_MODE[wname]
     replica = rank
 
@@ -323,7 +326,17 @@ def main():
 
     kernels = ["layout", "dispatch", "combine"] + (["combine_bwd"] if g_d is not None else [])
 
-    # each C-ABI call is checked and marshalled once, then replayed every step
+    # each C-ABI call is checked and marshalled once, then replayed every step.
+    # The timed step uses the one-call dispatch (layout + dispatch, the
+    # dispatch kernel overlapping the layout); the per-kernel pass uses the
+    # separate calls so that every kernel gets its own duration.
+    step_calls = [
+        ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
+                                   b.recv_buf, b.src_info, b.dev_status,
+                                   expert_offset=b.expert_offset, stream=stream, bind=True),
+        ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
+                      expert_offset=b.expert_offset, stream=stream, bind=True),
+    ]
     calls = [
         ep.ep_dispatch_layout(cfg, idx_d, b.token_slot, b.recv_count, b.workspace, b.dev_status,
                               expert_offset=b.expert_offset, stream=stream, bind=True),
@@ -336,14 +349,17 @@ def main():
         calls.append(ep.ep_combine_backward(cfg, g_d, idx_d, wts_d, b.token_slot, b.grad_buf,
                                             b.dev_status, expert_offset=b.expert_offset,
                                             stream=stream, bind=True))
+        step_calls.append(calls[-1])
 
     def step(evs=None):
-        if evs:
-            evs[0].record(stream)
+        if evs is None:
+            for c in step_calls:
+                c()
+            return
+        evs[0].record(stream)
         for i, c in enumerate(calls):
             c()
-            if evs:
-                evs[i + 1].record(stream)
+            evs[i + 1].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         flush(1)
@@ -487,10 +503,9 @@ def run_e2e(ep, cfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, world):
     d2h = out_h.numel() * 2 + cnt_h.numel() * 8
 
     calls = [
-        ep.ep_dispatch_layout(cfg, idx_d, b.token_slot, b.recv_count, b.workspace, b.dev_status,
-                              expert_offset=b.expert_offset, stream=stream, bind=True),
-        ep.ep_dispatch(cfg, x_d, idx_d, b.token_slot, b.recv_buf, b.src_info, b.dev_status,
-                       expert_offset=b.expert_offset, stream=stream, bind=True),
+        ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
+                                   b.recv_buf, b.src_info, b.dev_status,
+                                   expert_offset=b.expert_offset, stream=stream, bind=True),
         ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
                       expert_offset=b.expert_offset, stream=stream, bind=True),
     ]

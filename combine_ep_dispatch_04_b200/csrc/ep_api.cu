@@ -134,6 +134,14 @@ ep_status_t make_plan(const ep_config_t *c, Plan &p) {
 }
 
 
+struct ClusterChoice;
+ep_status_t check_layout_args(const ep_config_t *, const Plan &, const int64_t *, const int32_t *,
+                              const int64_t *, const int64_t *, const void *, const uint32_t *);
+ep::LayoutArgs layout_args(const ep_config_t *, const Plan &, const int64_t *, int32_t *, int32_t *,
+                           uint8_t *, int32_t *, int64_t *, int64_t *, int64_t *, void *,
+                           uint32_t *);
+ep_status_t run_layout(const ep_config_t *, const Plan &, const ep::LayoutArgs &, cudaStream_t);
+
 // ---- layout launch helpers -------------------------------------------------------
 // The one-block layout cuts the N tokens into chunks of whole tokens of one
 // source rank, about one chunk per warp (ceil(W/R) per rank).  Its shared
@@ -360,42 +368,13 @@ ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const int64_t *topk_idx,
     Plan p;
     ep_status_t st = make_plan(cfg, p);
     if (st != EP_OK) return st;
-    if (!recv_count || !workspace || !dev_status) return EP_ERR_INVALID_ARG;
-    if (p.N > 0 && (!topk_idx || !token_slot)) return EP_ERR_INVALID_ARG;
-    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
-
-    ep::LayoutArgs a;
-    a.R = p.R; a.T = p.T; a.K = p.K; a.E = p.E; a.M = p.M; a.L = p.L;
-    a.TC = p.TC; a.CR = p.CR; a.C = p.C;
-    a.packed = cfg->layout == EP_LAYOUT_PACKED;
-    a.align = cfg->expert_align;
-    a.cap = p.cap;
-    a.idx = topk_idx;
-    a.tpr = tokens_per_rank;
-    a.tpe = tokens_per_expert;
-    a.itr = is_token_in_rank;
-    a.slot = token_slot;
-    a.recv_count = recv_count;
-    a.eo = expert_offset;
-    a.stats = cumulative_recv_stats;
-    a.ws_hist = static_cast<int32_t *>(workspace);
-    a.ws_rk = a.ws_hist + (int64_t)p.E * p.C;
-    a.status = dev_status;
-
-    cudaStream_t s = cs(stream);
-    if (cfg->flags & EP_F_LAYOUT_SINGLE_CTA) return launch_layout_single(a, plan_single(p), s);
-    if (cfg->flags & EP_F_LAYOUT_MULTI_CTA) return launch_layout_multi(a, p, s);
-    if (cfg->flags & EP_F_LAYOUT_CLUSTER) return launch_layout_cluster(a, plan_cluster(p), s);
-    const int64_t entries = p.N * p.K;
-    if (entries <= kSingleMaxEntries) {
-        const SinglePlan sp = plan_single(p);
-        if (sp.ok) return launch_layout_single(a, sp, s);
-    }
-    if (entries <= kClusterMaxEntries) {
-        const ClusterChoice cc = plan_cluster(p);
-        if (cc.ok) return launch_layout_cluster(a, cc, s);
-    }
-    return launch_layout_multi(a, p, s);
+    if ((st = check_layout_args(cfg, p, topk_idx, token_slot, recv_count, expert_offset, workspace,
+                                dev_status)) != EP_OK)
+        return st;
+    const ep::LayoutArgs a =
+        layout_args(cfg, p, topk_idx, tokens_per_rank, tokens_per_expert, is_token_in_rank,
+                    token_slot, recv_count, expert_offset, cumulative_recv_stats, workspace, dev_status);
+    return run_layout(cfg, p, a, cs(stream));
 }
 
 }  // extern "C"
@@ -514,6 +493,97 @@ ep::DispatchArgs dispatch_args(const ep_config_t *cfg, const Plan &p) {
     return a;
 }
 
+
+// ---- argument checks and launch bodies shared by the entry points ----------------
+ep_status_t check_layout_args(const ep_config_t *cfg, const Plan &p, const int64_t *topk_idx,
+                              const int32_t *token_slot, const int64_t *recv_count,
+                              const int64_t *expert_offset, const void *workspace,
+                              const uint32_t *dev_status) {
+    if (!recv_count || !workspace || !dev_status) return EP_ERR_INVALID_ARG;
+    if (p.N > 0 && (!topk_idx || !token_slot)) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    return EP_OK;
+}
+
+ep::LayoutArgs layout_args(const ep_config_t *cfg, const Plan &p, const int64_t *topk_idx,
+                           int32_t *tokens_per_rank, int32_t *tokens_per_expert,
+                           uint8_t *is_token_in_rank, int32_t *token_slot, int64_t *recv_count,
+                           int64_t *expert_offset, int64_t *cumulative_recv_stats,
+                           void *workspace, uint32_t *dev_status) {
+    ep::LayoutArgs a;
+    a.R = p.R; a.T = p.T; a.K = p.K; a.E = p.E; a.M = p.M; a.L = p.L;
+    a.TC = p.TC; a.CR = p.CR; a.C = p.C;
+    a.packed = cfg->layout == EP_LAYOUT_PACKED;
+    a.align = cfg->expert_align;
+    a.cap = p.cap;
+    a.idx = topk_idx;
+    a.tpr = tokens_per_rank;
+    a.tpe = tokens_per_expert;
+    a.itr = is_token_in_rank;
+    a.slot = token_slot;
+    a.recv_count = recv_count;
+    a.eo = expert_offset;
+    a.stats = cumulative_recv_stats;
+    a.ws_hist = static_cast<int32_t *>(workspace);
+    a.ws_rk = a.ws_hist ? a.ws_hist + (int64_t)p.E * p.C : nullptr;
+    a.status = dev_status;
+    return a;
+}
+
+// Layout path by routing size (or the path a flag forces).
+ep_status_t run_layout(const ep_config_t *cfg, const Plan &p, const ep::LayoutArgs &a,
+                       cudaStream_t s) {
+    if (cfg->flags & EP_F_LAYOUT_SINGLE_CTA) return launch_layout_single(a, plan_single(p), s);
+    if (cfg->flags & EP_F_LAYOUT_MULTI_CTA) return launch_layout_multi(a, p, s);
+    if (cfg->flags & EP_F_LAYOUT_CLUSTER) return launch_layout_cluster(a, plan_cluster(p), s);
+    const int64_t entries = p.N * p.K;
+    if (entries <= kSingleMaxEntries) {
+        const SinglePlan sp = plan_single(p);
+        if (sp.ok) return launch_layout_single(a, sp, s);
+    }
+    if (entries <= kClusterMaxEntries) {
+        const ClusterChoice cc = plan_cluster(p);
+        if (cc.ok) return launch_layout_cluster(a, cc, s);
+    }
+    return launch_layout_multi(a, p, s);
+}
+
+ep_status_t check_dispatch_args(const ep_config_t *cfg, const uint16_t *x, const int64_t *topk_idx,
+                                const float *topk_weights, const int32_t *token_slot,
+                                const int64_t *expert_offset, const void *recv_buf,
+                                const int32_t *src_info, const float *recv_weights) {
+    if (!x || !topk_idx || !token_slot || !recv_buf || !src_info) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    if (recv_weights && !topk_weights) return EP_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(recv_buf)) return EP_ERR_MISALIGNED;
+    return EP_OK;
+}
+
+ep::DispatchArgs full_dispatch_args(const ep_config_t *cfg, const Plan &p, const uint16_t *x,
+                                    const int64_t *topk_idx, const float *topk_weights,
+                                    const int32_t *token_slot, const int64_t *expert_offset,
+                                    void *recv_buf, int32_t *src_info, float *recv_weights,
+                                    uint32_t *dev_status) {
+    ep::DispatchArgs a = dispatch_args(cfg, p);
+    a.D = p.D; a.S = p.S; a.scale_off = p.scale_off;
+    a.x = x; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
+    a.out = static_cast<uint8_t *>(recv_buf);
+    a.src_info = src_info;
+    a.recv_w = recv_weights;
+    a.status = dev_status;
+    return a;
+}
+
+ep_status_t run_dispatch(const ep_config_t *cfg, const ep::DispatchArgs &a, cudaStream_t s) {
+    switch (cfg->quant) {
+    case EP_Q_BF16: return launch_dispatch<ep::Q_BF16>(a, s);
+    case EP_Q_E4M3_B128: return launch_dispatch<ep::Q_E4M3_B128>(a, s);
+    case EP_Q_INT8_TOKEN: return launch_dispatch<ep::Q_INT8>(a, s);
+    case EP_Q_MXFP8: return launch_dispatch<ep::Q_MXFP8>(a, s);
+    default: return launch_dispatch<ep::Q_MXFP4>(a, s);
+    }
+}
+
 }  // namespace
 
 extern "C" {
@@ -527,26 +597,44 @@ ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const int64_t
     if (st != EP_OK) return st;
     if (!dev_status) return EP_ERR_INVALID_ARG;
     if (p.N == 0) return EP_OK;
-    if (!x || !topk_idx || !token_slot || !recv_buf || !src_info) return EP_ERR_INVALID_ARG;
-    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
-    if (recv_weights && !topk_weights) return EP_ERR_INVALID_ARG;
-    if (!aligned16(x) || !aligned16(recv_buf)) return EP_ERR_MISALIGNED;
+    if ((st = check_dispatch_args(cfg, x, topk_idx, topk_weights, token_slot, expert_offset,
+                                  recv_buf, src_info, recv_weights)) != EP_OK)
+        return st;
+    ep::DispatchArgs a = full_dispatch_args(cfg, p, x, topk_idx, topk_weights, token_slot,
+                                            expert_offset, recv_buf, src_info, recv_weights,
+                                            dev_status);
+    return run_dispatch(cfg, a, cs(stream));
+}
 
-    ep::DispatchArgs a = dispatch_args(cfg, p);
-    a.D = p.D; a.S = p.S; a.scale_off = p.scale_off;
-    a.x = x; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
-    a.out = static_cast<uint8_t *>(recv_buf);
-    a.src_info = src_info;
-    a.recv_w = recv_weights;
-    a.status = dev_status;
+ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
+                                    const int64_t *topk_idx, const float *topk_weights,
+                                    int32_t *tokens_per_rank, int32_t *tokens_per_expert,
+                                    uint8_t *is_token_in_rank, int32_t *token_slot,
+                                    int64_t *recv_count, int64_t *expert_offset,
+                                    int64_t *cumulative_recv_stats, void *workspace,
+                                    void *recv_buf, int32_t *src_info, float *recv_weights,
+                                    uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if ((st = check_layout_args(cfg, p, topk_idx, token_slot, recv_count, expert_offset, workspace,
+                                dev_status)) != EP_OK)
+        return st;
+    if (p.N > 0 && (st = check_dispatch_args(cfg, x, topk_idx, topk_weights, token_slot,
+                                             expert_offset, recv_buf, src_info, recv_weights)) !=
+                       EP_OK)
+        return st;
     cudaStream_t s = cs(stream);
-    switch (cfg->quant) {
-    case EP_Q_BF16: return launch_dispatch<ep::Q_BF16>(a, s);
-    case EP_Q_E4M3_B128: return launch_dispatch<ep::Q_E4M3_B128>(a, s);
-    case EP_Q_INT8_TOKEN: return launch_dispatch<ep::Q_INT8>(a, s);
-    case EP_Q_MXFP8: return launch_dispatch<ep::Q_MXFP8>(a, s);
-    default: return launch_dispatch<ep::Q_MXFP4>(a, s);
-    }
+    const ep::LayoutArgs la =
+        layout_args(cfg, p, topk_idx, tokens_per_rank, tokens_per_expert, is_token_in_rank,
+                    token_slot, recv_count, expert_offset, cumulative_recv_stats, workspace, dev_status);
+    if ((st = run_layout(cfg, p, la, s)) != EP_OK) return st;
+    if (p.N == 0) return EP_OK;
+    ep::DispatchArgs a = full_dispatch_args(cfg, p, x, topk_idx, topk_weights, token_slot,
+                                            expert_offset, recv_buf, src_info, recv_weights,
+                                            dev_status);
+    a.early = 1;  // the previous grid is the layout launched just above
+    return run_dispatch(cfg, a, s);
 }
 
 ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t *topk_idx,

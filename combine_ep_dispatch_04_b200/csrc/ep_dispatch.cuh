@@ -32,6 +32,7 @@ struct DispatchArgs {
     int64_t D, S, scale_off; // row data bytes, row scale bytes, scale region offset
     float qmax;              // e4m3_b128 target max
     int unweighted;          // combine backward only
+    int early;               // load and quantise x before waiting for the previous grid
     const uint16_t *x;       // [N][H] bf16 (the gradient g for the backward)
     const int64_t *idx;
     const float *wts;
@@ -64,6 +65,23 @@ __device__ __forceinline__ int64_t entry_row(const DispatchArgs &a, int64_t n, i
     return row;
 }
 
+// The same from an expert index and slot already loaded.
+__device__ __forceinline__ int64_t row_of_entry(const DispatchArgs &a, int64_t e, int32_t s,
+                                                uint32_t &flags) {
+    if (e < -1 || e >= a.E) flags |= kDevBadIndex;
+    if (e < 0 || e >= a.E) return -1;
+    if (s < 0) return -1;
+    int64_t row;
+    if (!a.packed) {
+        if (s >= a.cap) { flags |= kDevCapacity; return -1; }
+        row = e * a.cap + s;
+    } else {
+        row = a.eo[e] + s;
+        if (row >= a.eo[e + 1] || row >= a.rows) { flags |= kDevCapacity; return -1; }
+    }
+    return row;
+}
+
 template <int MODE>
 struct GranOut;  // bytes a 16-element granule becomes
 template <> struct GranOut<Q_BF16> { static constexpr int bytes = 32; };
@@ -78,9 +96,13 @@ __device__ __forceinline__ uint32_t q_i8(float v, float s) {
     return (uint32_t)q & 0xFFu;
 }
 
+// With a.early (only set by ep_dispatch_with_layout, whose previous grid is
+// the library's own layout kernel) the token is loaded and quantised before
+// the wait for the previous grid: x is not produced by the layout, and the
+// layout grid lets this grid launch only after its own wait for all earlier
+// work returned.  The slots are read after the wait.
 template <int MODE, int TPT, int GMAX>
 __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs a) {
-    pdl_enter();
     constexpr int TOKS = kDispatchThreads / TPT;
     constexpr int WPG = TPT / 32;  // warps per token group
     constexpr int OB = GranOut<MODE>::bytes;
@@ -90,17 +112,21 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
     const int grp = threadIdx.x / TPT, lt = threadIdx.x % TPT;
     const int64_t n = (int64_t)blockIdx.x * TOKS + grp;
     const bool active = n < a.N;
+    const bool router = active && lt < a.K;  // thread lt reads entry (n, lt)
     const int ngran = a.H >> 4;
 
-    if (active && lt < a.K) {
-        uint32_t flags = 0;
-        const int64_t row = entry_row(a, n, lt, flags);
-        if (flags) atomicOr(a.status, flags);
-        s_row[grp][lt] = row;
-        if (row >= 0) {
-            a.src_info[row] = (int32_t)((n / a.T) * a.M + n % a.T);
-            if (a.recv_w) a.recv_w[row] = a.wts[n * a.K + lt];
-        }
+    // The entry's expert, slot and weight are loaded here and used after the
+    // quantisation, so their latency overlaps the row loads.  topk_idx and the
+    // weights are inputs; the slot comes from the layout and, in early mode,
+    // is read only after the wait.
+    int64_t r_e = -1;
+    int32_t r_s = -1;
+    float r_w = 0.0f;
+    if (!a.early) pdl_enter();
+    if (router) {
+        r_e = a.idx[n * a.K + lt];
+        if (a.recv_w) r_w = a.wts[n * a.K + lt];
+        if (!a.early) r_s = a.slot[n * a.K + lt];
     }
 
     // load the token's granules (two 16-byte loads each)
@@ -152,8 +178,6 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
             rs = fminf(__fdiv_rn(127.0f, m), FLT_MAX);
             rsinv = __fdiv_rn(m, 127.0f);
         }
-    } else {
-        __syncthreads();  // s_row visible to the whole group
     }
     if constexpr (MODE == Q_E4M3_B128) {
 #pragma unroll
@@ -219,6 +243,22 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
         }
     }
 
+    if (a.early) {
+        pdl_enter();
+        if (router) r_s = a.slot[n * a.K + lt];
+    }
+    // destination rows of the token's entries
+    if (router) {
+        uint32_t flags = 0;
+        const int64_t row = row_of_entry(a, r_e, r_s, flags);
+        if (flags) atomicOr(a.status, flags);
+        s_row[grp][lt] = row;
+        if (row >= 0) {
+            a.src_info[row] = (int32_t)((n / a.T) * a.M + n % a.T);
+            if (a.recv_w) a.recv_w[row] = r_w;
+        }
+    }
+    __syncthreads();
     if (!active) return;
     // scatter to every destination row
     for (int k = 0; k < a.K; k++) {

@@ -67,6 +67,8 @@ lib.ep_dispatch_layout.restype = C.c_int
 lib.ep_dispatch_layout.argtypes = [_CFG] + [_P] * 11
 lib.ep_dispatch_layout_static.restype = C.c_int
 lib.ep_dispatch_layout_static.argtypes = [_CFG] + [_P] * 10
+lib.ep_dispatch_with_layout.restype = C.c_int
+lib.ep_dispatch_with_layout.argtypes = [_CFG] + [_P] * 16
 lib.ep_dispatch.restype = C.c_int
 lib.ep_dispatch.argtypes = [_CFG] + [_P] * 10
 lib.ep_combine.restype = C.c_int
@@ -227,6 +229,38 @@ def ep_dispatch(cfg, x, topk_idx, token_slot, recv_buf, src_info, dev_status, to
         _stream(stream),
     ]
     return _call(lib.ep_dispatch, cfg, args, "ep_dispatch", bind)
+
+
+def ep_dispatch_with_layout(cfg, x, topk_idx, token_slot, recv_count, workspace, recv_buf,
+                            src_info, dev_status, topk_weights=None, tokens_per_rank=None,
+                            tokens_per_expert=None, is_token_in_rank=None, expert_offset=None,
+                            cumulative_recv_stats=None, recv_weights=None, stream=None,
+                            bind=False):
+    """ep_dispatch_layout + ep_dispatch in one call (the dispatch kernel
+    overlaps the layout; see include/ep.h)."""
+    N, K = _nk(cfg)
+    R, E = cfg.num_ranks, cfg.num_experts
+    sz = ep_buffer_sizes(cfg)
+    args = [
+        _dev(x, "x", torch.bfloat16, (N, cfg.hidden)),
+        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(topk_weights, "topk_weights", torch.float32, (N, K), optional=True),
+        _dev(tokens_per_rank, "tokens_per_rank", torch.int32, (R, R), optional=True),
+        _dev(tokens_per_expert, "tokens_per_expert", torch.int32, (R, E), optional=True),
+        _dev(is_token_in_rank, "is_token_in_rank", torch.uint8, (N, R), optional=True),
+        _dev(token_slot, "token_slot", torch.int32, (N, K)),
+        _dev(recv_count, "recv_count", torch.int64, (E,)),
+        _dev(expert_offset, "expert_offset", torch.int64, (E + 1,),
+             optional=cfg.layout == LAYOUT["padded"]),
+        _dev(cumulative_recv_stats, "cumulative_recv_stats", torch.int64, (E,), optional=True),
+        _bytes(workspace, "workspace", sz["workspace_bytes"]),
+        _bytes(recv_buf, "recv_buf", sz["recv_bytes"]),
+        _bytes(src_info, "src_info", sz["src_info_bytes"]),
+        _bytes(recv_weights, "recv_weights", sz["recv_weights_bytes"], optional=True),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    return _call(lib.ep_dispatch_with_layout, cfg, args, "ep_dispatch_with_layout", bind)
 
 
 def ep_combine(cfg, y, topk_idx, topk_weights, token_slot, out, dev_status, expert_offset=None,

@@ -165,6 +165,23 @@ ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const int64_t
                         float *recv_weights, uint32_t *dev_status, ep_stream_t stream);
 
 /*
+ * ep_dispatch_layout followed by ep_dispatch in one call, with the same
+ * arguments and results as the two calls ([LL] low_latency_dispatch returns
+ * the received tokens and recv_count from one call).  Because the call
+ * launches the layout itself, the dispatch kernel may start while the layout
+ * runs: it loads and quantises its tokens first and waits for the layout only
+ * before reading token_slot / expert_offset.
+ */
+ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
+                                    const int64_t *topk_idx, const float *topk_weights,
+                                    int32_t *tokens_per_rank, int32_t *tokens_per_expert,
+                                    uint8_t *is_token_in_rank, int32_t *token_slot,
+                                    int64_t *recv_count, int64_t *expert_offset,
+                                    int64_t *cumulative_recv_stats, void *workspace,
+                                    void *recv_buf, int32_t *src_info, float *recv_weights,
+                                    uint32_t *dev_status, ep_stream_t stream);
+
+/*
  * Weighted top-k combine ([LL] low_latency_combine: combined_x [T, H] bf16 is
  * the weighted sum across experts; `out` written in place):
  *   out[n,:] = bf16_rne( sum over valid k = 0..K-1, in order, of

@@ -281,3 +281,35 @@ def test_layout_paths_bad_indices_and_duplicates(path):
     assert r.status & ep.DEV_BAD_INDEX
     r.check_layout()
     r.check_dispatch()
+
+
+@pytest.mark.parametrize("mode", ["bf16", "int8_token", "e4m3_b128", "mxfp8", "mxfp4"])
+@pytest.mark.parametrize("name,override,path", [
+    ("decode", {}, 0), ("tiny", {}, 0), ("skewed", dict(T=64), ep.F_LAYOUT_MULTI_CTA),
+    ("large", dict(T=40), ep.F_LAYOUT_SINGLE_CTA), ("prefill", dict(T=50), 0),
+])
+def test_dispatch_with_layout_equals_separate_calls(mode, name, override, path):
+    """The one-call dispatch (whose kernel overlaps the layout) gives the
+    bytes of ep_dispatch_layout + ep_dispatch, and so the oracle's."""
+    w = synth.workload(name, **override)
+    r = Run(w, mode, layout=w["layout"], flags=path, stats=True)
+    r.check_layout()
+    b = ep.Buffers(r.cfg, recv_weights=True, expert_out=False)
+    b.recv_buf.fill_(0xAB)
+    b.src_info.fill_(-7)
+    b.recv_weights.fill_(float("nan"))
+    stats = torch.zeros(w["E"], dtype=torch.int64, device="cuda")
+    ep.ep_dispatch_with_layout(r.cfg, r.x_d, r.idx_d, b.token_slot, b.recv_count, b.workspace,
+                               b.recv_buf, b.src_info, b.dev_status, topk_weights=r.wts_d,
+                               tokens_per_rank=b.tokens_per_rank,
+                               tokens_per_expert=b.tokens_per_expert,
+                               is_token_in_rank=b.is_token_in_rank, expert_offset=b.expert_offset,
+                               cumulative_recv_stats=stats, recv_weights=b.recv_weights)
+    assert ep.ep_get_status(b.dev_status) == r.status
+    for name_ in ("token_slot", "recv_count", "tokens_per_rank", "tokens_per_expert",
+                  "is_token_in_rank", "recv_buf", "src_info"):
+        assert torch.equal(getattr(b, name_), getattr(r.b, name_)), name_
+    assert torch.equal(b.recv_weights.nan_to_num(-1), r.b.recv_weights.nan_to_num(-1))
+    if b.expert_offset is not None:
+        assert torch.equal(b.expert_offset, r.b.expert_offset)
+    assert torch.equal(stats, r.stats_d)
