@@ -733,8 +733,15 @@ __global__ void cvt_sweep_kernel(int format, uint32_t start, int64_t n, uint8_t 
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
         const float v = __uint_as_float(start + (uint32_t)i);
-        out[i] = format == 0 ? (uint8_t)(cvt_e4m3x2(v, 0.0f) & 0xFFu)
-                             : (uint8_t)(cvt_e2m1x2(v, 0.0f) & 0xFu);
+        const float av = __uint_as_float((start + (uint32_t)i) & 0x7FFFFFFFu);
+        uint8_t r;
+        switch (format) {
+        case 0: r = (uint8_t)(cvt_e4m3x2(v, 0.0f) & 0xFFu); break;
+        case 1: r = (uint8_t)(cvt_e2m1x2(v, 0.0f) & 0xFu); break;
+        case 2: r = (uint8_t)(mx_exponent_fast<448>(av) + 127); break;
+        default: r = (uint8_t)(mx_exponent_fast<6>(av) + 127); break;
+        }
+        out[i] = r;
     }
 }
 
@@ -764,7 +771,7 @@ extern "C" ep_status_t ep_copy(void *dst, const void *src, size_t bytes, ep_stre
 
 extern "C" ep_status_t ep_cvt_sweep(int32_t format, uint32_t start, int64_t n, uint8_t *out,
                                     ep_stream_t stream) {
-    if ((format != 0 && format != 1) || n < 0 || !out) return EP_ERR_INVALID_ARG;
+    if (format < 0 || format > 3 || n < 0 || !out) return EP_ERR_INVALID_ARG;
     if (n > (int64_t(1) << 32) - (int64_t)start) return EP_ERR_INVALID_ARG;
     if (n == 0) return EP_OK;
     int64_t blocks = (n + 255) / 256;

@@ -76,6 +76,30 @@ __device__ __forceinline__ int mx_exponent(float amax, float qmax) {
     return X < -127 ? -127 : (X > 127 ? 127 : X);
 }
 
+// The same exponent without the division, for qmax = 448 (= 7 * 2^6) and
+// qmax = 6 (= 3 * 2^1).  For a normal amax = m * 2^e whose quotient is normal,
+// fl(amax / (q * 2^s)) = fl(amax / q) * 2^-s, and fl(m / q) is a power of two
+// only for m = 1.75 (q = 7) or m = 1.5 (q = 3) exactly -- the neighbouring
+// mantissas are more than half an ulp away -- so
+//   X = e - 8 + [m > 1.75]   (qmax 448),   X = e - 2 + [m > 1.5]   (qmax 6).
+// Zero, subnormal and tiny values (quotient below the normal range) and
+// non-finite values take the division.  Checked against the division-based
+// definition on every fp32 input (ep_cvt_sweep formats 2 and 3).
+template <int QMAX>
+__device__ __forceinline__ int mx_exponent_fast(float amax) {
+    static_assert(QMAX == 448 || QMAX == 6, "exponent shortcut is derived for 448 and 6");
+    const uint32_t b = __float_as_uint(amax);
+    const int ex = (int)(b >> 23);  // amax >= 0: no sign bit
+    const uint32_t mant = b & 0x7FFFFFu;
+    if (QMAX == 448) {
+        if (ex >= 10 && ex < 255) return ex - 127 - 8 + (mant > 0x600000u);
+        return mx_exponent(amax, 448.0f);
+    } else {
+        if (ex >= 4 && ex < 255) return ex - 127 - 2 + (mant > 0x400000u);
+        return mx_exponent(amax, 6.0f);
+    }
+}
+
 // 2^-X as an fp32 for X in [-127, 127] (2^-127 is the subnormal 0x00400000).
 __device__ __forceinline__ float exp2_neg(int X) {
     int e = 127 - X;

@@ -195,12 +195,11 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
         }
     }
     if constexpr (MODE == Q_MXFP8 || MODE == Q_MXFP4) {
-        constexpr float QM = MODE == Q_MXFP8 ? 448.0f : 6.0f;
 #pragma unroll
         for (int i = 0; i < GMAX; i++) {
             float m = gmax[i];
             m = fmaxf(m, __shfl_xor_sync(kFull, m, 1));
-            const int X = mx_exponent(m, QM);
+            const int X = mx_exponent_fast<MODE == Q_MXFP8 ? 448 : 6>(m);
             bs[i] = exp2_neg(X);
             bx[i] = (uint32_t)(X + 127);
         }
@@ -317,29 +316,36 @@ __global__ void __launch_bounds__(kDispatchThreads) combine_bwd_kernel(DispatchA
         s_w[grp][lt] = a.unweighted ? 1.0f : a.wts[n * a.K + lt];
     }
 
-    uint32_t v[GMAX][8];
+    // the token's gradient row, unpacked to fp32 once for all its entries
+    float f[GMAX][16];
     float gmax[GMAX];
 #pragma unroll
     for (int i = 0; i < GMAX; i++) {
         const int g = i * TPT + lt;
+        uint32_t v[8];
         if (active && g < ngran) {
             const uint16_t *p = a.x + n * a.H + (int64_t)g * 16;
             const uint4 u0 = ld_stream(p), u1 = ld_stream(p + 8);
-            v[i][0] = u0.x; v[i][1] = u0.y; v[i][2] = u0.z; v[i][3] = u0.w;
-            v[i][4] = u1.x; v[i][5] = u1.y; v[i][6] = u1.z; v[i][7] = u1.w;
+            v[0] = u0.x; v[1] = u0.y; v[2] = u0.z; v[3] = u0.w;
+            v[4] = u1.x; v[5] = u1.y; v[6] = u1.z; v[7] = u1.w;
         } else {
 #pragma unroll
-            for (int q = 0; q < 8; q++) v[i][q] = 0u;
+            for (int q = 0; q < 8; q++) v[q] = 0u;
         }
         uint32_t m = 0u;
 #pragma unroll
-        for (int q = 0; q < 8; q++) m = bf2_absmax(m, v[i][q]);
-        float f = bf2_fold(m);
-        gmax[i] = fmaxf(f, __shfl_xor_sync(kFull, f, 1));
+        for (int q = 0; q < 8; q++) {
+            m = bf2_absmax(m, v[q]);
+            f[i][2 * q] = bf_lo(v[q]);
+            f[i][2 * q + 1] = bf_hi(v[q]);
+        }
+        const float fm = bf2_fold(m);
+        gmax[i] = fmaxf(fm, __shfl_xor_sync(kFull, fm, 1));
     }
     __syncthreads();
     if (!active) return;
 
+    const bool weighted = !a.unweighted;
     for (int k = 0; k < a.K; k++) {
         const int64_t row = s_row[grp][k];
         if (row < 0) continue;
@@ -351,15 +357,14 @@ __global__ void __launch_bounds__(kDispatchThreads) combine_bwd_kernel(DispatchA
         for (int i = 0; i < GMAX; i++) {
             const int g = i * TPT + lt;
             if (g >= ngran) continue;
-            const float amax = a.unweighted ? gmax[i] : __fmul_rn(aw, gmax[i]);
-            const int X = mx_exponent(amax, 448.0f);
+            const float amax = weighted ? __fmul_rn(aw, gmax[i]) : gmax[i];
+            const int X = mx_exponent_fast<448>(amax);
             const float s = exp2_neg(X);
             uint32_t cw[4];
 #pragma unroll
             for (int q = 0; q < 4; q++) {
-                const uint32_t w0 = v[i][2 * q], w1 = v[i][2 * q + 1];
-                float p0 = bf_lo(w0), p1 = bf_hi(w0), p2 = bf_lo(w1), p3 = bf_hi(w1);
-                if (!a.unweighted) {
+                float p0 = f[i][4 * q], p1 = f[i][4 * q + 1], p2 = f[i][4 * q + 2], p3 = f[i][4 * q + 3];
+                if (weighted) {
                     p0 = __fmul_rn(w, p0); p1 = __fmul_rn(w, p1);
                     p2 = __fmul_rn(w, p2); p3 = __fmul_rn(w, p3);
                 }

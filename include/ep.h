@@ -253,8 +253,9 @@ const char *ep_status_string(ep_status_t status);
  * reference for the kernels above (bytes % 16 == 0, both pointers aligned).
  * ep_cvt_sweep: out[i] = the kernels' conversion of the binary32 value with
  * bit pattern start+i (format 0: e4m3 satfinite byte; 1: e2m1 satfinite code
- * in the low nibble), for checking the hardware conversion against the
- * format definition.
+ * in the low nibble; 2 and 3: the e8m0 byte X+127 of an MX block whose
+ * maximum is |value|, for qmax 448 and 6), for checking the hardware
+ * conversions and the exponent arithmetic against their definitions.
  * ep_kernel_launches: kernels launched by this library in this process. */
 ep_status_t ep_copy(void *dst, const void *src, size_t bytes, ep_stream_t stream);
 ep_status_t ep_cvt_sweep(int32_t format, uint32_t start, int64_t n, uint8_t *out,

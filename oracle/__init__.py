@@ -69,6 +69,8 @@ for _n in ("orc_e4m3_encode_array", "orc_e2m1_encode_array"):
 for _n in ("orc_e4m3_encode_bits", "orc_e2m1_encode_bits"):
     getattr(_lib, _n).restype = None
     getattr(_lib, _n).argtypes = [C.c_uint32, _p, _l]
+_lib.orc_mx_exponent_bits.restype = None
+_lib.orc_mx_exponent_bits.argtypes = [C.c_uint32, _f, _p, _l]
 _lib.orc_mx_exponent_array.restype = None
 _lib.orc_mx_exponent_array.argtypes = [_p, _f, _p, _l]
 _lib.orc_f32_to_bf16_array.restype = None
@@ -117,6 +119,13 @@ def e4m3_encode_bits(start, n):
 def e2m1_encode_bits(start, n):
     out = np.empty(n, np.uint8)
     _lib.orc_e2m1_encode_bits(start, _ptr(out), n)
+    return out
+
+
+def mx_exponent_bits(start, n, qmax):
+    """e8m0 bytes of blocks whose maxima are |bit patterns start .. start+n-1| (0xFF: not finite)."""
+    out = np.empty(n, np.uint8)
+    _lib.orc_mx_exponent_bits(start, float(qmax), _ptr(out), n)
     return out
 
 

@@ -501,6 +501,15 @@ void orc_e2m1_encode_bits(uint32_t start, uint8_t *out, long n)
         out[i] = isnan(f) ? 0xFF : orc_e2m1_encode(f);
     }
 }
+/* e8m0 byte (X + 127) of a block whose maximum is |value of bit pattern
+ * start+i|; 0xFF marks non-finite patterns (not an amax). */
+void orc_mx_exponent_bits(uint32_t start, float qmax, uint8_t *out, long n)
+{
+    for (long i = 0; i < n; i++) {
+        float a = fabsf(bits_to_f32(start + (uint32_t)i));
+        out[i] = isfinite(a) ? (uint8_t)(orc_mx_exponent(a, qmax) + 127) : 0xFF;
+    }
+}
 void orc_mx_exponent_array(const float *amax, float qmax, int32_t *out, long n)
 {
     for (long i = 0; i < n; i++) out[i] = orc_mx_exponent(amax[i], qmax);

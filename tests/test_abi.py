@@ -96,7 +96,7 @@ def test_entry_points_reject_before_any_launch():
     assert lib.ep_dispatch(C.byref(cfg), *args) == 3
     assert lib.ep_copy(fake, fake, 24, null) == 1
     assert lib.ep_copy(odd, fake, 32, null) == 3
-    assert lib.ep_cvt_sweep(2, 0, 16, fake, null) == 1
+    assert lib.ep_cvt_sweep(4, 0, 16, fake, null) == 1
     assert lib.ep_cvt_sweep(0, 0xFFFFFFF0, 17, fake, null) == 1
     assert ep.ep_kernel_launches() == n0
 

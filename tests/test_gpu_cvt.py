@@ -2,7 +2,9 @@
 written from the OCP format definitions, over EVERY binary32 bit pattern
 (2^32 inputs per format; NaN inputs excluded from the e2m1 comparison, where
 the format has no NaN).  This pins the hardware `cvt ... satfinite` used by
-the dispatch and combine-backward kernels to the oracle bit for bit."""
+the dispatch and combine-backward kernels to the oracle bit for bit.  Formats
+2 and 3 pin the kernels' division-free MX exponent (qmax 448 and 6) to the
+oracle's frexp-based definition on every finite block maximum."""
 from concurrent.futures import ThreadPoolExecutor
 
 import numpy as np
@@ -18,10 +20,14 @@ CHUNK = 1 << 28
 
 
 def _oracle_chunk(fmt, start, n):
-    return oracle.e4m3_encode_bits(start, n) if fmt == 0 else oracle.e2m1_encode_bits(start, n)
+    if fmt == 0:
+        return oracle.e4m3_encode_bits(start, n)
+    if fmt == 1:
+        return oracle.e2m1_encode_bits(start, n)
+    return oracle.mx_exponent_bits(start, n, 448.0 if fmt == 2 else 6.0)
 
 
-@pytest.mark.parametrize("fmt", [0, 1], ids=["e4m3", "e2m1"])
+@pytest.mark.parametrize("fmt", [0, 1, 2, 3], ids=["e4m3", "e2m1", "e8m0_448", "e8m0_6"])
 def test_cvt_exhaustive(fmt):
     out = torch.empty(CHUNK, dtype=torch.uint8, device="cuda")
     pieces = 16
@@ -37,5 +43,7 @@ def test_cvt_exhaustive(fmt):
                 nan = (bits & 0x7F800000) == 0x7F800000
                 nan &= (bits & 0x007FFFFF) != 0
                 got = np.where(nan, 0xFF, got)
+            if fmt >= 2:  # non-finite patterns are not block maxima
+                got = np.where(want == 0xFF, 0xFF, got)
             bad = np.nonzero(got != want)[0]
             assert bad.size == 0, [(hex(c + int(i)), int(got[i]), int(want[i])) for i in bad[:8]]
