@@ -94,7 +94,7 @@ ep_status_t make_plan(const ep_config_t *c, Plan &p) {
     if (c->expert_align < 1) return EP_ERR_INVALID_ARG;
     if (!(c->e4m3_qmax >= 0.0f && c->e4m3_qmax <= 448.0f)) return EP_ERR_INVALID_ARG;  // NaN fails
     const uint32_t paths = EP_F_LAYOUT_SINGLE_CTA | EP_F_LAYOUT_MULTI_CTA | EP_F_LAYOUT_CLUSTER;
-    const uint32_t known = EP_F_BWD_UNWEIGHTED | paths;
+    const uint32_t known = EP_F_BWD_UNWEIGHTED | EP_F_COMBINE_QUANTIZED | paths;
     if (c->flags & ~known) return EP_ERR_INVALID_ARG;
     const uint32_t forced = c->flags & paths;
     if (forced & (forced - 1)) return EP_ERR_INVALID_ARG;  // at most one path flag
@@ -574,6 +574,27 @@ ep::DispatchArgs full_dispatch_args(const ep_config_t *cfg, const Plan &p, const
     return a;
 }
 
+// 8-element granules: 16 bytes of bf16, 8 of int8 / e4m3, 4 of e2m1.
+template <int QIN>
+ep_status_t launch_combine(const ep::CombineArgs &a, cudaStream_t s) {
+    auto kernel_of = [](int t, int g) -> const void * {
+#define EP_FN(T_, G_) if (t == T_ && g == G_) return (const void *)ep::combine_kernel<T_, G_, 8, QIN>;
+        EP_SPLITS(EP_FN)
+#undef EP_FN
+        return nullptr;
+    };
+    const Split sp = split_rows(a.N, a.H / 8, ep::kCombineThreads, 8, kernel_of);
+    const unsigned grid = grid_for(a.N, ep::kCombineThreads, sp.tpt);
+#define EP_CASE(T_, G_)                                                                     \
+    if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
+        launch(ep::combine_kernel<T_, G_, 8, QIN>, grid, ep::kCombineThreads, 0, s, a);     \
+        return launched();                                                                  \
+    }
+    EP_SPLITS(EP_CASE)
+#undef EP_CASE
+    return EP_ERR_UNSUPPORTED;
+}
+
 ep_status_t run_dispatch(const ep_config_t *cfg, const ep::DispatchArgs &a, cudaStream_t s) {
     switch (cfg->quant) {
     case EP_Q_BF16: return launch_dispatch<ep::Q_BF16>(a, s);
@@ -650,30 +671,22 @@ ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t 
     if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
     if (!aligned16(y) || !aligned16(out)) return EP_ERR_MISALIGNED;
 
+    const int qin = (cfg->flags & EP_F_COMBINE_QUANTIZED) ? cfg->quant : EP_Q_BF16;
     ep::CombineArgs a;
     a.N = p.N; a.K = p.K; a.E = p.E; a.H = p.H;
     a.packed = cfg->layout == EP_LAYOUT_PACKED;
     a.cap = p.cap; a.rows = p.rows;
+    a.D = p.D; a.S = p.S; a.scale_off = p.scale_off;
     a.y = y; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
     a.out = out; a.status = dev_status;
     cudaStream_t s = cs(stream);
-    auto kernel_of = [](int t, int g) -> const void * {
-#define EP_FN(T_, G_) if (t == T_ && g == G_) return (const void *)ep::combine_kernel<T_, G_, 8>;
-        EP_SPLITS(EP_FN)
-#undef EP_FN
-        return nullptr;
-    };
-    // 8-element granules (16 bytes of bf16)
-    const Split sp = split_rows(p.N, p.H / 8, ep::kCombineThreads, 8, kernel_of);
-    const unsigned grid = grid_for(p.N, ep::kCombineThreads, sp.tpt);
-#define EP_CASE(T_, G_)                                                                     \
-    if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
-        launch(ep::combine_kernel<T_, G_, 8>, grid, ep::kCombineThreads, 0, s, a);          \
-        return launched();                                                                  \
+    switch (qin) {
+    case EP_Q_BF16: return launch_combine<ep::QIN_BF16>(a, s);
+    case EP_Q_E4M3_B128: return launch_combine<ep::QIN_E4M3_B128>(a, s);
+    case EP_Q_INT8_TOKEN: return launch_combine<ep::QIN_INT8>(a, s);
+    case EP_Q_MXFP8: return launch_combine<ep::QIN_MXFP8>(a, s);
+    default: return launch_combine<ep::QIN_MXFP4>(a, s);
     }
-    EP_SPLITS(EP_CASE)
-#undef EP_CASE
-    return EP_ERR_UNSUPPORTED;
 }
 
 ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,

@@ -1,4 +1,4 @@
-// ep_combine.cuh -- weighted top-k combine.
+// ep_combine.cuh -- weighted top-k combine (bf16 or quantised expert outputs).
 //
 // "Low-Latency Mode API", low_latency_combine (Return Values: combined_x is
 // the weighted sum across experts) and "DeepEP FP8 Dispatch and Combine
@@ -24,7 +24,8 @@ struct CombineArgs {
     int K, E, H;
     int packed;
     int64_t cap, rows;
-    const uint16_t *y;
+    int64_t D, S, scale_off;  // quantised expert outputs: row bytes, scale bytes, scale region
+    const uint16_t *y;        // bf16 rows, or the quantised buffer (data then scales)
     const int64_t *idx;
     const float *wts;
     const int32_t *slot;
@@ -35,7 +36,75 @@ struct CombineArgs {
 
 constexpr int kCombineThreads = 256;
 
-template <int TPT, int GMAX, int KB>
+enum { QIN_BF16 = 0, QIN_E4M3_B128 = 1, QIN_INT8 = 2, QIN_MXFP8 = 3, QIN_MXFP4 = 4 };
+
+// Eight expert-output values of granule g of `row`, as fp32: bf16 widened, or
+// quantised codes decoded and multiplied by their scale (one fp32 multiply --
+// "DeepEP FP8 Dispatch and Combine Operations", The FP8 Combine Operation).
+template <int QIN>
+struct Granule {
+    uint4 raw;   // bf16: 16 bytes; e4m3 / int8: 8 bytes in .x .y; e2m1: 4 bytes in .x
+    float scale;
+};
+
+template <int QIN>
+__device__ __forceinline__ Granule<QIN> load_granule(const CombineArgs &a, int64_t row, int g) {
+    Granule<QIN> r;
+    const uint8_t *base = reinterpret_cast<const uint8_t *>(a.y);
+    if constexpr (QIN == QIN_BF16) {
+        r.raw = ld_stream(a.y + row * a.H + (int64_t)g * 8);
+        r.scale = 1.0f;
+    } else {
+        const uint8_t *sc = base + a.scale_off + row * a.S;
+        if constexpr (QIN == QIN_MXFP4) {
+            r.raw.x = __ldcs(reinterpret_cast<const unsigned int *>(base + row * a.D + (int64_t)g * 4));
+            r.raw.y = r.raw.z = r.raw.w = 0u;
+        } else {
+            const uint2 d = __ldcs(reinterpret_cast<const uint2 *>(base + row * a.D + (int64_t)g * 8));
+            r.raw = make_uint4(d.x, d.y, 0u, 0u);
+        }
+        if constexpr (QIN == QIN_INT8) r.scale = __ldg(reinterpret_cast<const float *>(sc));
+        if constexpr (QIN == QIN_E4M3_B128)
+            r.scale = __ldg(reinterpret_cast<const float *>(sc) + (g >> 4));
+        if constexpr (QIN == QIN_MXFP8 || QIN == QIN_MXFP4)
+            r.scale = exp2_neg(127 - (int)__ldg(sc + (g >> 2)));
+    }
+    return r;
+}
+
+template <int QIN>
+__device__ __forceinline__ void decode_granule(const Granule<QIN> &r, float (&v)[8]) {
+    if constexpr (QIN == QIN_BF16) {
+        const uint32_t u[4] = {r.raw.x, r.raw.y, r.raw.z, r.raw.w};
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            v[2 * q] = bf_lo(u[q]);
+            v[2 * q + 1] = bf_hi(u[q]);
+        }
+    } else if constexpr (QIN == QIN_INT8) {
+        const uint32_t u[2] = {r.raw.x, r.raw.y};
+#pragma unroll
+        for (int q = 0; q < 8; q++)
+            v[q] = __fmul_rn((float)(int8_t)((u[q >> 2] >> (8 * (q & 3))) & 0xFFu), r.scale);
+    } else if constexpr (QIN == QIN_MXFP4) {
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const float2 f = e2m1x2_to_f32(r.raw.x >> (8 * q));
+            v[2 * q] = __fmul_rn(f.x, r.scale);
+            v[2 * q + 1] = __fmul_rn(f.y, r.scale);
+        }
+    } else {  // e4m3 codes
+        const uint32_t u[2] = {r.raw.x, r.raw.y};
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const float2 f = e4m3x2_to_f32(u[q >> 1] >> (16 * (q & 1)));
+            v[2 * q] = __fmul_rn(f.x, r.scale);
+            v[2 * q + 1] = __fmul_rn(f.y, r.scale);
+        }
+    }
+}
+
+template <int TPT, int GMAX, int KB, int QIN>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
     pdl_enter();
     constexpr int TOKS = kCombineThreads / TPT;
@@ -70,7 +139,6 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
     if (!active) return;
 
     const int ngran = a.H >> 3;
-    const uint16_t *ybase = a.y;
 #pragma unroll
     for (int i = 0; i < GMAX; i++) {
         const int g = i * TPT + lt;
@@ -79,24 +147,44 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
 #pragma unroll
         for (int q = 0; q < 8; q++) acc[q] = 0.0f;
         for (int k0 = 0; k0 < a.K; k0 += KB) {
-            uint4 buf[KB];
+            if constexpr (QIN == QIN_BF16) {
+                uint4 buf[KB];
 #pragma unroll
-            for (int kk = 0; kk < KB; kk++) {
-                const int k = k0 + kk;
-                const int64_t row = k < a.K ? s_row[grp][k] : -1;
-                buf[kk] = row >= 0 ? ld_stream(ybase + row * a.H + (int64_t)g * 8)
-                                   : make_uint4(0u, 0u, 0u, 0u);
-            }
+                for (int kk = 0; kk < KB; kk++) {
+                    const int k = k0 + kk;
+                    const int64_t row = k < a.K ? s_row[grp][k] : -1;
+                    buf[kk] = row >= 0 ? ld_stream(a.y + row * a.H + (int64_t)g * 8)
+                                       : make_uint4(0u, 0u, 0u, 0u);
+                }
 #pragma unroll
-            for (int kk = 0; kk < KB; kk++) {
-                const int k = k0 + kk;
-                if (k >= a.K || s_row[grp][k] < 0) continue;
-                const float w = s_w[grp][k];
-                const uint32_t u[4] = {buf[kk].x, buf[kk].y, buf[kk].z, buf[kk].w};
+                for (int kk = 0; kk < KB; kk++) {
+                    const int k = k0 + kk;
+                    if (k >= a.K || s_row[grp][k] < 0) continue;
+                    const float w = s_w[grp][k];
+                    const uint32_t u[4] = {buf[kk].x, buf[kk].y, buf[kk].z, buf[kk].w};
 #pragma unroll
-                for (int q = 0; q < 4; q++) {
-                    acc[2 * q] = __fmaf_rn(w, bf_lo(u[q]), acc[2 * q]);
-                    acc[2 * q + 1] = __fmaf_rn(w, bf_hi(u[q]), acc[2 * q + 1]);
+                    for (int q = 0; q < 4; q++) {
+                        acc[2 * q] = __fmaf_rn(w, bf_lo(u[q]), acc[2 * q]);
+                        acc[2 * q + 1] = __fmaf_rn(w, bf_hi(u[q]), acc[2 * q + 1]);
+                    }
+                }
+            } else {
+                Granule<QIN> buf[KB];
+#pragma unroll
+                for (int kk = 0; kk < KB; kk++) {
+                    const int k = k0 + kk;
+                    const int64_t row = k < a.K ? s_row[grp][k] : -1;
+                    if (row >= 0) buf[kk] = load_granule<QIN>(a, row, g);
+                }
+#pragma unroll
+                for (int kk = 0; kk < KB; kk++) {
+                    const int k = k0 + kk;
+                    if (k >= a.K || s_row[grp][k] < 0) continue;
+                    const float w = s_w[grp][k];
+                    float v[8];
+                    decode_granule<QIN>(buf[kk], v);
+#pragma unroll
+                    for (int q = 0; q < 8; q++) acc[q] = __fmaf_rn(w, v[q], acc[q]);
                 }
             }
         }

@@ -10,6 +10,7 @@
 
 #include <cfloat>
 #include <cstdint>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace ep {
@@ -53,6 +54,23 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
         : "=r"(r)
         : "f"(hi), "f"(lo));
     return r;
+}
+
+// Exact widening of two e4m3 / e2m1 codes (the low byte / nibble first) to
+// fp32, through f16 (every e4m3 and e2m1 value is an f16 value).
+__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two_codes) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}"
+        : "=r"(h2)
+        : "r"(two_codes & 0xFFFFu));
+    return __half22float2(*reinterpret_cast<__half2 *>(&h2));
+}
+__device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t two_codes) {
+    uint32_t h2;
+    asm("{\n\t.reg .b8 c;\n\tcvt.u8.u32 c, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+        : "=r"(h2)
+        : "r"(two_codes & 0xFFu));
+    return __half22float2(*reinterpret_cast<__half2 *>(&h2));
 }
 
 // ---- scales ------------------------------------------------------------------

@@ -25,6 +25,7 @@ LAYOUT = {"padded": 0, "packed": 1}
 DEV_BAD_INDEX = 0x1
 DEV_CAPACITY_OVERFLOW = 0x2
 F_BWD_UNWEIGHTED = 0x1
+F_COMBINE_QUANTIZED = 0x2
 F_LAYOUT_SINGLE_CTA = 0x100
 F_LAYOUT_MULTI_CTA = 0x200
 F_LAYOUT_CLUSTER = 0x400
@@ -267,10 +268,11 @@ def ep_combine(cfg, y, topk_idx, topk_weights, token_slot, out, dev_status, expe
                stream=None, bind=False):
     N, K = _nk(cfg)
     sz = ep_buffer_sizes(cfg)
-    if y is None or y.dtype != torch.bfloat16:
-        raise TypeError("y (expert outputs) must be bfloat16")
+    quantized = bool(cfg.flags & F_COMBINE_QUANTIZED) and cfg.quant != QUANT["bf16"]
+    if y is None or (not quantized and y.dtype != torch.bfloat16):
+        raise TypeError("y (expert outputs) must be bfloat16 unless F_COMBINE_QUANTIZED")
     args = [
-        _bytes(y, "y", sz["expert_out_bytes"]),
+        _bytes(y, "y", sz["recv_bytes"] if quantized else sz["expert_out_bytes"]),
         _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
         _dev(topk_weights, "topk_weights", torch.float32, (N, K)),
         _dev(token_slot, "token_slot", torch.int32, (N, K)),

@@ -82,6 +82,7 @@ typedef enum {
 
 /* ep_config_t.flags */
 #define EP_F_BWD_UNWEIGHTED 0x1u    /* combine-backward re-dispatches g without w */
+#define EP_F_COMBINE_QUANTIZED 0x2u /* ep_combine's y is in cfg->quant's format (recv_buf layout) */
 #define EP_F_LAYOUT_SINGLE_CTA 0x100u /* force the one-block layout path */
 #define EP_F_LAYOUT_MULTI_CTA 0x200u  /* force the multi-block layout path */
 #define EP_F_LAYOUT_CLUSTER 0x400u    /* force the thread-block-cluster layout path */
@@ -188,7 +189,13 @@ ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
  *                        w[n,k] * y[row(n,k), :] )
  * accumulated in fp32 with one fused multiply-add per term.  Masked entries
  * add nothing; a token with no valid entry gets +0.  Weights are used as given.
- *   y      bf16 [rows][H] expert outputs in the receive layout
+ *   y      bf16 [rows][H] expert outputs in the receive layout; with
+ *          EP_F_COMBINE_QUANTIZED (and cfg->quant != EP_Q_BF16) y is instead a
+ *          buffer of ep_sizes_t.recv_bytes in cfg->quant's format (data region
+ *          then scale region, as ep_dispatch writes it) and each expert value
+ *          is decode(code) * scale as one fp32 multiply before the FMA ([FP8]
+ *          The FP8 Combine Operation: FP8 values times scale_inv, cast through
+ *          fp32).  An e8m0 scale byte of 255 (NaN) is not a valid input.
  *   out    bf16 [N][H]
  */
 ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t *topk_idx,

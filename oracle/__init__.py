@@ -63,6 +63,10 @@ _lib.orc_bwd_row.restype = None
 _lib.orc_bwd_row.argtypes = [_i, _f, _i, _p, _p, _p]
 _lib.orc_combine_gathered.restype = None
 _lib.orc_combine_gathered.argtypes = [_l, _i, _i, _p, _p, _p, _p]
+_lib.orc_dequant_row.restype = None
+_lib.orc_dequant_row.argtypes = [_i, _i, _p, _p, _p]
+_lib.orc_combine_gathered_q.restype = None
+_lib.orc_combine_gathered_q.argtypes = [_i, _l, _i, _i, _p, _p, _p, _p, _p]
 for _n in ("orc_e4m3_encode_array", "orc_e2m1_encode_array"):
     getattr(_lib, _n).restype = None
     getattr(_lib, _n).argtypes = [_p, _p, _l]
@@ -314,3 +318,27 @@ def bwd_row(g_row, w, unweighted=False):
     s = np.zeros(H // 32, np.uint8)
     _lib.orc_bwd_row(H, float(w), int(bool(unweighted)), _ptr(g_row), _ptr(d), _ptr(s))
     return d, s
+
+
+def dequant_row(mode, data, scale, H):
+    """fp32 values of one quantised row (data bytes, scale bytes)."""
+    d = _c(data, np.uint8)
+    sc = _c(scale, np.uint8) if np.size(scale) else np.zeros(1, np.uint8)
+    out = np.zeros(H, np.float32)
+    _lib.orc_dequant_row(_mode(mode), H, _ptr(d), _ptr(sc), _ptr(out))
+    return out
+
+
+def combine_gathered_q(mode, data, scale, w, valid, H):
+    """Tokens whose K rows are quantised: data [N, K, D] u8, scale [N, K, S] u8,
+    w [N, K] f32, valid [N, K] -> out [N, H] bf16 bits."""
+    m = _mode(mode)
+    d = _c(data, np.uint8)
+    N, K = d.shape[0], d.shape[1]
+    D, S = row_bytes(m, H)
+    sc = _c(scale, np.uint8) if S else np.zeros((N, K, 1), np.uint8)
+    w = _c(w, np.float32)
+    v = _c(valid, np.uint8)
+    out = np.zeros((N, H), np.uint16)
+    _lib.orc_combine_gathered_q(m, N, K, H, _ptr(d), _ptr(sc), _ptr(w), _ptr(v), _ptr(out))
+    return out

@@ -479,6 +479,77 @@ uint32_t orc_combine_bwd(int R, int T, int K, int E, int M, int H, int layout, i
     return st;
 }
 
+/*
+ * Dequantisation of one row stored in a quantised format ([FP8] The FP8
+ * Combine Operation: the FP8 values are multiplied by the stored inverse
+ * scale, casting through fp32).  Each element is decode(code) * scale_inv as
+ * one fp32 multiply: int8 codes and e4m3 / e2m1 values times the row's or
+ * block's fp32 scale_inv, MX codes times 2^(byte-127).  BF16 rows widen
+ * exactly.
+ */
+void orc_dequant_row(int mode, int H, const uint8_t *data, const uint8_t *scale, float *out)
+{
+    for (int h = 0; h < H; h++) {
+        float v, s;
+        switch (mode) {
+        case ORC_BF16: {
+            uint16_t b;
+            memcpy(&b, data + 2L * h, 2);
+            out[h] = orc_bf16_to_f32(b);
+            continue;
+        }
+        case ORC_INT8_TOKEN:
+            v = (float)(int8_t)data[h];
+            memcpy(&s, scale, 4);
+            break;
+        case ORC_E4M3_B128:
+            v = orc_e4m3_decode(data[h]);
+            memcpy(&s, scale + 4L * (h / 128), 4);
+            break;
+        case ORC_MXFP8:
+            v = orc_e4m3_decode(data[h]);
+            s = ldexpf(1.0f, (int)scale[h / 32] - 127);
+            break;
+        default: /* MXFP4: element 2i in the low nibble */
+            v = orc_e2m1_decode((uint8_t)((h % 2 == 0) ? (data[h / 2] & 0xF) : (data[h / 2] >> 4)));
+            s = ldexpf(1.0f, (int)scale[h / 32] - 127);
+            break;
+        }
+        out[h] = v * s;
+    }
+}
+
+/*
+ * Weighted top-k combine of quantised expert outputs: as orc_combine_row, with
+ * each expert row dequantised first (rows: data [K][D], scales [K][S]).
+ */
+void orc_combine_row_q(int mode, int H, int K, const uint8_t *data, const uint8_t *scale,
+                       const float *w, const uint8_t *valid, uint16_t *out)
+{
+    long D = orc_row_data_bytes(mode, H), S = orc_row_scale_bytes(mode, H);
+    float *y = (float *)malloc(sizeof(float) * (size_t)H * (size_t)K);
+    for (int k = 0; k < K; k++)
+        if (valid[k]) orc_dequant_row(mode, H, data + k * D, scale + k * S, y + (long)k * H);
+    for (int h = 0; h < H; h++) {
+        float acc = 0.0f;
+        for (int k = 0; k < K; k++)
+            if (valid[k]) acc = fmaf(w[k], y[(long)k * H + h], acc);
+        out[h] = orc_f32_to_bf16(acc);
+    }
+    free(y);
+}
+
+/* Tokens whose K quantised rows are gathered: data [N][K][D], scale [N][K][S]. */
+void orc_combine_gathered_q(int mode, long N, int K, int H, const uint8_t *data,
+                            const uint8_t *scale, const float *w, const uint8_t *valid,
+                            uint16_t *out)
+{
+    long D = orc_row_data_bytes(mode, H), S = orc_row_scale_bytes(mode, H);
+    for (long n = 0; n < N; n++)
+        orc_combine_row_q(mode, H, K, data + n * K * D, scale + n * K * S, w + n * K,
+                          valid + n * K, out + n * H);
+}
+
 /* ---- array helpers for the tests (loops over the scalar functions) ------ */
 void orc_e4m3_encode_array(const float *x, uint8_t *out, long n)
 {

@@ -179,3 +179,58 @@ def ulp_distance(a, b):
         u = u.astype(np.int64)
         return np.where(u & 0x8000, -(u & 0x7FFF), u)
     return np.abs(key(a) - key(b))
+
+
+def quantized_rows(mode, H, nrows, seed):
+    """Random expert outputs stored in a quantised format: (data [n, D], scale [n, S])
+    bytes.  Every code value occurs; NaN codes and NaN scales do not."""
+    r = np.random.default_rng(seed)
+    D, S = oracle.row_bytes(mode, H)
+    data = r.integers(0, 256, (nrows, D), dtype=np.uint8)
+    if mode in ("e4m3_b128", "mxfp8"):
+        data[(data & 0x7F) == 0x7F] ^= 0x01          # 0x7F / 0xFF are NaN in e4m3
+    if mode == "int8_token":
+        scale = (r.random((nrows, 1)) * 0.05 + 1e-3).astype(np.float32).view(np.uint8)
+    elif mode == "e4m3_b128":
+        scale = (r.random((nrows, S // 4)) * 0.02 + 1e-4).astype(np.float32).view(np.uint8)
+    else:
+        scale = r.integers(112, 140, (nrows, S), dtype=np.uint8)
+    return data, scale.reshape(nrows, S)
+
+
+def combine_quantized_check(run, tokens=None, seed=0):
+    """Combine of quantised expert outputs on the GPU against the oracle."""
+    w, b = run.w, run.b
+    K, H = w["K"], w["H"]
+    mode = run.mode
+    cfg = ep.make_config(w["R"], w["T"], w["M"], K, w["E"], H, mode, run.layout, run.align,
+                         run.qmax, run.cfg.flags | ep.F_COMBINE_QUANTIZED)
+    ns, ks, rows = run.entries(None)
+    data, scale = quantized_rows(mode, H, len(rows), seed)
+    sz = run.sizes
+    yq = torch.zeros(sz["recv_bytes"], dtype=torch.uint8, device="cuda")
+    D, S = sz["data_row_bytes"], sz["scale_row_bytes"]
+    rows_d = torch.from_numpy(rows).cuda()
+    yq[: sz["rows"] * D].view(sz["rows"], D).index_copy_(0, rows_d, torch.from_numpy(data).cuda())
+    if S:
+        a = sz["recv_scale_offset"]
+        yq[a: a + sz["rows"] * S].view(sz["rows"], S).index_copy_(0, rows_d, torch.from_numpy(scale).cuda())
+    out = torch.full((w["N"], H), 1.0, dtype=torch.bfloat16, device="cuda")
+    ep.ep_combine(cfg, yq, run.idx_d, run.wts_d,
+                  b.token_slot, out, b.dev_status, expert_offset=b.expert_offset)
+    assert ep.ep_get_status(b.dev_status) == run.status
+    tokens = np.arange(w["N"]) if tokens is None else np.asarray(tokens)
+    got = to_np_u16(out)[tokens]
+    where = {(int(n), int(k)): i for i, (n, k) in enumerate(zip(ns, ks))}
+    qd = np.zeros((len(tokens), K, D), np.uint8)
+    qs = np.zeros((len(tokens), K, S), np.uint8)
+    valid = np.zeros((len(tokens), K), np.uint8)
+    for j, n in enumerate(tokens):
+        for k in range(K):
+            i = where.get((int(n), k))
+            if i is not None:
+                qd[j, k], qs[j, k], valid[j, k] = data[i], scale[i], 1
+    want = oracle.combine_gathered_q(mode, qd, qs, run.wts[tokens], valid, H)
+    d = ulp_distance(got, want)
+    assert d.max() <= 1, int(d.max())
+    return int(d.max())

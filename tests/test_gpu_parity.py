@@ -313,3 +313,15 @@ def test_dispatch_with_layout_equals_separate_calls(mode, name, override, path):
     if b.expert_offset is not None:
         assert torch.equal(b.expert_offset, r.b.expert_offset)
     assert torch.equal(stats, r.stats_d)
+
+
+@pytest.mark.parametrize("mode", ["int8_token", "e4m3_b128", "mxfp8", "mxfp4"])
+@pytest.mark.parametrize("name,override", [("decode", {}), ("tiny", {}), ("large", dict(T=40)),
+                                           ("skewed", dict(T=64))])
+def test_combine_of_quantized_expert_outputs(mode, name, override):
+    w = synth.workload(name, **override)
+    if mode == "e4m3_b128" and w["H"] % 128:
+        pytest.skip("H % 128")
+    from harness import combine_quantized_check
+    r = Run(w, mode, layout=w["layout"])
+    combine_quantized_check(r, seed=31 * len(mode) + len(name))

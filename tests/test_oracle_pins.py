@@ -510,3 +510,109 @@ def test_combine_backward_weighted_rows():
             ref = p.astype(np.float64).reshape(-1, 32)
             assert np.all(np.abs(dec - ref) <= np.maximum(np.abs(ref) * 2 ** -4,
                                                           np.ldexp(2.0 ** -10, X)[:, None]))
+
+
+# ---------------------------------------------------------------------------
+# dequantisation and the combine of quantised expert outputs
+# ---------------------------------------------------------------------------
+
+def test_dequant_rows_worked_by_hand():
+    # int8: codes times the row scale
+    d = np.array([1, 0xFE, 127, 0x81], np.uint8)           # 1, -2, 127, -127
+    s = np.float32([0.5]).view(np.uint8)
+    assert list(oracle.dequant_row("int8_token", d, s, 4)) == [0.5, -1.0, 63.5, -63.5]
+    # e4m3 per 128: 0x38 = 1.0, 0x40 = 2.0, 0xB8 = -1.0; scale_inv 2
+    d = np.zeros(128, np.uint8)
+    d[:3] = [0x38, 0x40, 0xB8]
+    s = np.float32([2.0]).view(np.uint8)
+    assert list(oracle.dequant_row("e4m3_b128", d, s, 128)[:3]) == [2.0, 4.0, -2.0]
+    # MXFP8: byte 128 -> 2^1
+    d = np.zeros(32, np.uint8)
+    d[:2] = [0x38, 0x7E]                                      # 1.0, 448
+    assert list(oracle.dequant_row("mxfp8", d, np.uint8([128]), 32)[:2]) == [2.0, 896.0]
+    # MXFP4: element 0 is the low nibble; byte 126 -> 2^-1
+    d = np.zeros(16, np.uint8)
+    d[0] = 0x72                                               # low 2 (1.0), high 7 (6.0)
+    assert list(oracle.dequant_row("mxfp4", d, np.uint8([126]), 32)[:2]) == [0.5, 3.0]
+
+
+@pytest.mark.parametrize("mode", ["int8_token", "e4m3_b128", "mxfp8", "mxfp4"])
+def test_dequant_of_quant_within_format_bounds(mode):
+    H = 1024
+    x = _bf16_row(H, seed=21)
+    d, s = oracle.quant_row(mode, x)
+    y = oracle.dequant_row(mode, d, s, H).astype(np.float64)
+    xf = _f(x)
+    if mode == "int8_token":
+        sinv = float(s.view(np.float32)[0])
+        assert np.all(np.abs(xf - y) <= 0.5 * sinv * (1 + 2 ** -20) + np.abs(xf) * 2 ** -21)
+    elif mode == "e4m3_b128":
+        sinv = np.repeat(s.view(np.float32).astype(np.float64), 128)
+        assert np.all(np.abs(xf - y) <= np.maximum(np.abs(xf) * 2 ** -4, sinv * 2 ** -10) * (1 + 2 ** -18)
+                      + np.abs(xf) * 2 ** -21)
+    else:
+        step = np.repeat(np.ldexp(1.0, s.astype(np.int64) - 127), 32)
+        rel = 2 ** -4 if mode == "mxfp8" else 2 ** -1
+        assert np.all(np.abs(xf - y) <= np.maximum(np.abs(xf) * rel, step * (2 ** -10 if mode == "mxfp8" else 0.25)))
+
+
+def _table_dequant(mode, d, s, H):
+    """Dequantisation written from the brute-force code tables of this file
+    (not the oracle's decoders): exact values in float64."""
+    if mode == "mxfp8":
+        t = _e4m3_table()
+        mag = t[d & 0x7F]
+        v = np.where(d & 0x80, -mag, mag)
+    else:
+        t = _e2m1_table()
+        codes = np.stack([d & 0xF, d >> 4], axis=1).reshape(-1)
+        mag = t[codes & 0x7]
+        v = np.where(codes & 0x8, -mag, mag)
+    return v * np.repeat(np.ldexp(1.0, s.astype(np.int64) - 127), 32)
+
+
+@pytest.mark.parametrize("mode", ["mxfp8", "mxfp4"])
+def test_combine_of_mx_rows_equals_bf16_combine_of_their_values(mode):
+    # An MX value (<= 4 significant bits times a power of two) is exact in
+    # bf16, so the combine of quantised rows must equal the bf16 combine of the
+    # decoded rows, bit for bit.
+    r = np.random.default_rng(4)
+    N, K, H = 6, 5, 256
+    x = synth.to_bf16_bits((r.standard_normal((N * K, H)) * 3).astype(np.float32))
+    D, S = oracle.row_bytes(mode, H)
+    data = np.zeros((N, K, D), np.uint8)
+    scale = np.zeros((N, K, S), np.uint8)
+    dec = np.zeros((N, K, H), np.uint16)
+    for i in range(N * K):
+        d, s = oracle.quant_row(mode, x[i])
+        data.reshape(-1, D)[i], scale.reshape(-1, S)[i] = d, s
+        dec.reshape(-1, H)[i] = synth.to_bf16_bits(_table_dequant(mode, d, s, H).astype(np.float32))
+    w = r.random((N, K)).astype(np.float32)
+    valid = (r.random((N, K)) < 0.8).astype(np.uint8)
+    got = oracle.combine_gathered_q(mode, data, scale, w, valid, H)
+    want = oracle.combine_gathered(dec, w, valid)
+    assert np.array_equal(got, want)
+
+
+def test_combine_of_int8_rows_within_one_ulp_of_float64():
+    r = np.random.default_rng(6)
+    N, K, H = 4, 6, 512
+    data = r.integers(0, 256, (N, K, H), dtype=np.uint8)
+    sc = (r.random((N, K)) * 0.05 + 1e-3).astype(np.float32)
+    w = r.random((N, K)).astype(np.float32)
+    valid = np.ones((N, K), np.uint8)
+    got = oracle.combine_gathered_q("int8_token", data, sc.view(np.uint8).reshape(N, K, 4), w, valid, H)
+    q = data.view(np.int8).astype(np.float64)
+    ref = (w.astype(np.float64)[:, :, None] * q * sc.astype(np.float64)[:, :, None]).sum(axis=1)
+    want = synth.to_bf16_bits(ref.astype(np.float32))
+    assert _bf16_ulp_distance(got, want).max() <= 1
+
+
+def test_combine_of_bf16_rows_is_the_plain_combine():
+    r = np.random.default_rng(8)
+    N, K, H = 3, 4, 128
+    y = synth.to_bf16_bits(r.standard_normal((N, K, H)).astype(np.float32))
+    w = r.random((N, K)).astype(np.float32)
+    valid = np.ones((N, K), np.uint8)
+    got = oracle.combine_gathered_q("bf16", y.view(np.uint8).reshape(N, K, 2 * H), np.zeros((N, K, 0), np.uint8), w, valid, H)
+    assert np.array_equal(got, oracle.combine_gathered(y, w, valid))
