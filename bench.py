@@ -59,6 +59,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--flush-mib", type=int, default=512)
     p.add_argument("--cpu-seconds", type=float, default=10.0)
+    p.add_argument("--quantized-combine", action="store_true",
+                   help="combine reads expert outputs stored in the dispatch format")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     return p.parse_args()
@@ -67,17 +69,18 @@ def parse():
 # ---------------------------------------------------------------------------
 # algorithmic bytes (what the method must move; unwritten capacity not counted)
 # ---------------------------------------------------------------------------
-def algorithmic_bytes(w, mode, idx):
+def algorithmic_bytes(w, mode, idx, quantized_combine=False):
     """Bytes per launch of each kernel, from the per-token counts."""
     import oracle
 
     N, K, H, R = w["N"], w["K"], w["H"], w["R"]
     D, S = oracle.row_bytes(mode, H)
     v = int(((idx >= 0) & (idx < w["E"])).sum())
+    y_row = (D + S) if quantized_combine else 2 * H
     out = {
         "layout": N * (8 * K + 4 * K + R),
         "dispatch": N * (2 * H + 8 * K + 4 * K) + v * (D + S + 4),
-        "combine": v * 2 * H + N * (8 * K + 4 * K + 4 * K + 2 * H),
+        "combine": v * y_row + N * (8 * K + 4 * K + 4 * K + 2 * H),
     }
     if w.get("backward"):
         out["combine_bwd"] = N * (2 * H + 4 * K + 4 * K + 8 * K) + v * (H + H // 32)
@@ -303,6 +306,9 @@ def main():
     x = synth.make_x(w, replica)
     cfg = ep.make_config(R, T, M, K, E, H, mode, w["layout"])
     b = ep.Buffers(cfg, device=dev, grad=bool(w.get("backward")))
+    ccfg = cfg  # the combine's configuration
+    if args.quantized_combine:
+        ccfg = ep.make_config(R, T, M, K, E, H, mode, w["layout"], flags=ep.F_COMBINE_QUANTIZED)
     rows = b.sizes["rows"]
     idx_d = torch.from_numpy(idx).to(dev)
     wts_d = torch.from_numpy(wts).to(dev)
@@ -312,6 +318,13 @@ def main():
     torch.index_select(pool_d.as_strided((synth.POOL, H), (1, 1)), 0,
                        torch.from_numpy(yoff).to(dev), out=b.y.view(torch.int16))
     del pool_d
+    if args.quantized_combine:
+        # expert outputs in the dispatch format: the dispatched rows of one
+        # pass, copied to their own buffer (cold after every L2 flush)
+        ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
+                                   b.recv_buf, b.src_info, b.dev_status,
+                                   expert_offset=b.expert_offset)
+        b.y = b.recv_buf.clone()
     g_d = None
     if w.get("backward"):
         gp, go = synth.g_source(w, replica)
@@ -334,7 +347,7 @@ def main():
         ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
                                    b.recv_buf, b.src_info, b.dev_status,
                                    expert_offset=b.expert_offset, stream=stream, bind=True),
-        ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
+        ep.ep_combine(ccfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
                       expert_offset=b.expert_offset, stream=stream, bind=True),
     ]
     calls = [
@@ -342,7 +355,7 @@ def main():
                               expert_offset=b.expert_offset, stream=stream, bind=True),
         ep.ep_dispatch(cfg, x_d, idx_d, b.token_slot, b.recv_buf, b.src_info, b.dev_status,
                        expert_offset=b.expert_offset, stream=stream, bind=True),
-        ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
+        ep.ep_combine(ccfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
                       expert_offset=b.expert_offset, stream=stream, bind=True),
     ]
     if g_d is not None:
@@ -404,7 +417,7 @@ def main():
         for i, k in enumerate(kernels):
             per_kernel[k].append(e[i].elapsed_time(e[i + 1]))
 
-    alg, v = algorithmic_bytes(w, mode, idx)
+    alg, v = algorithmic_bytes(w, mode, idx, quantized_combine=args.quantized_combine)
     peaks = measured_peaks()
     peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else FALLBACK_HBM_GBS
     peak_src = "measured" if peaks and peaks.get("hbm_gbs") else "fallback"
@@ -443,8 +456,8 @@ def main():
     except Exception:
         pass
 
-    e2e = None if args.no_e2e else run_e2e(ep, cfg, b, w, idx, wts, x, g_d, flush, stream, dev,
-                                          args, world)
+    e2e = None if args.no_e2e else run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream,
+                                          dev, args, world)
 
     out = {
         "metric": METRIC,
@@ -460,7 +473,8 @@ def main():
         "dtype": "f32",
         "data": "synthetic",
         "config": {
-            "workload": f"{wname}: R={R} T={T} H={H} K={K} E={E} M={M} {mode} {w['layout']}",
+            "workload": f"{wname}: R={R} T={T} H={H} K={K} E={E} M={M} {mode} {w['layout']}"
+                        + (", combine of quantised expert outputs" if args.quantized_combine else ""),
             "tokens_per_step": N, "valid_entries": v,
             "l2": f"flushed between steps outside the step events ({args.flush_mib} MiB write, "
                   f"then {args.flush_mib} MiB read)",
@@ -485,7 +499,7 @@ def main():
     dist_done(world)
 
 
-def run_e2e(ep, cfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, world):
+def run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, world):
     """The same step through the public API with host buffers: pinned host
     inputs copied in, the combined output and the counts copied back, inside
     the timed region of every step.  Expert outputs (and the gradient) stay on
@@ -506,7 +520,7 @@ def run_e2e(ep, cfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, world):
         ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
                                    b.recv_buf, b.src_info, b.dev_status,
                                    expert_offset=b.expert_offset, stream=stream, bind=True),
-        ep.ep_combine(cfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
+        ep.ep_combine(ccfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
                       expert_offset=b.expert_offset, stream=stream, bind=True),
     ]
     if g_d is not None:

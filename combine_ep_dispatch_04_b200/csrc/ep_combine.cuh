@@ -38,72 +38,10 @@ constexpr int kCombineThreads = 256;
 
 enum { QIN_BF16 = 0, QIN_E4M3_B128 = 1, QIN_INT8 = 2, QIN_MXFP8 = 3, QIN_MXFP4 = 4 };
 
-// Eight expert-output values of granule g of `row`, as fp32: bf16 widened, or
-// quantised codes decoded and multiplied by their scale (one fp32 multiply --
-// "DeepEP FP8 Dispatch and Combine Operations", The FP8 Combine Operation).
-template <int QIN>
-struct Granule {
-    uint4 raw;   // bf16: 16 bytes; e4m3 / int8: 8 bytes in .x .y; e2m1: 4 bytes in .x
-    float scale;
-};
-
-template <int QIN>
-__device__ __forceinline__ Granule<QIN> load_granule(const CombineArgs &a, int64_t row, int g) {
-    Granule<QIN> r;
-    const uint8_t *base = reinterpret_cast<const uint8_t *>(a.y);
-    if constexpr (QIN == QIN_BF16) {
-        r.raw = ld_stream(a.y + row * a.H + (int64_t)g * 8);
-        r.scale = 1.0f;
-    } else {
-        const uint8_t *sc = base + a.scale_off + row * a.S;
-        if constexpr (QIN == QIN_MXFP4) {
-            r.raw.x = __ldcs(reinterpret_cast<const unsigned int *>(base + row * a.D + (int64_t)g * 4));
-            r.raw.y = r.raw.z = r.raw.w = 0u;
-        } else {
-            const uint2 d = __ldcs(reinterpret_cast<const uint2 *>(base + row * a.D + (int64_t)g * 8));
-            r.raw = make_uint4(d.x, d.y, 0u, 0u);
-        }
-        if constexpr (QIN == QIN_INT8) r.scale = __ldg(reinterpret_cast<const float *>(sc));
-        if constexpr (QIN == QIN_E4M3_B128)
-            r.scale = __ldg(reinterpret_cast<const float *>(sc) + (g >> 4));
-        if constexpr (QIN == QIN_MXFP8 || QIN == QIN_MXFP4)
-            r.scale = exp2_neg(127 - (int)__ldg(sc + (g >> 2)));
-    }
-    return r;
-}
-
-template <int QIN>
-__device__ __forceinline__ void decode_granule(const Granule<QIN> &r, float (&v)[8]) {
-    if constexpr (QIN == QIN_BF16) {
-        const uint32_t u[4] = {r.raw.x, r.raw.y, r.raw.z, r.raw.w};
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-            v[2 * q] = bf_lo(u[q]);
-            v[2 * q + 1] = bf_hi(u[q]);
-        }
-    } else if constexpr (QIN == QIN_INT8) {
-        const uint32_t u[2] = {r.raw.x, r.raw.y};
-#pragma unroll
-        for (int q = 0; q < 8; q++)
-            v[q] = __fmul_rn((float)(int8_t)((u[q >> 2] >> (8 * (q & 3))) & 0xFFu), r.scale);
-    } else if constexpr (QIN == QIN_MXFP4) {
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-            const float2 f = e2m1x2_to_f32(r.raw.x >> (8 * q));
-            v[2 * q] = __fmul_rn(f.x, r.scale);
-            v[2 * q + 1] = __fmul_rn(f.y, r.scale);
-        }
-    } else {  // e4m3 codes
-        const uint32_t u[2] = {r.raw.x, r.raw.y};
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-            const float2 f = e4m3x2_to_f32(u[q >> 1] >> (16 * (q & 1)));
-            v[2 * q] = __fmul_rn(f.x, r.scale);
-            v[2 * q + 1] = __fmul_rn(f.y, r.scale);
-        }
-    }
-}
-
+// Quantised expert outputs ("DeepEP FP8 Dispatch and Combine Operations",
+// The FP8 Combine Operation): each code is decoded exactly (e4m3 / e2m1 via
+// the hardware conversions to f16, int8 as an integer) and multiplied by its
+// row / block scale as one fp32 multiply before the FMA.
 template <int TPT, int GMAX, int KB, int QIN>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
     pdl_enter();
@@ -169,12 +107,30 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
                     }
                 }
             } else {
-                Granule<QIN> buf[KB];
+                // quantised rows: the codes of the granule (8 bytes, 4 for e2m1)
+                // and their scale, loaded for all KB entries before any use
+                const uint8_t *ybase = reinterpret_cast<const uint8_t *>(a.y);
+                uint2 raw[KB];
+                float sc[KB];
 #pragma unroll
                 for (int kk = 0; kk < KB; kk++) {
                     const int k = k0 + kk;
                     const int64_t row = k < a.K ? s_row[grp][k] : -1;
-                    if (row >= 0) buf[kk] = load_granule<QIN>(a, row, g);
+                    raw[kk] = make_uint2(0u, 0u);
+                    sc[kk] = 0.0f;
+                    if (row >= 0) {
+                        const uint8_t *d = ybase + row * a.D;
+                        const uint8_t *sp = ybase + a.scale_off + row * a.S;
+                        if constexpr (QIN == QIN_MXFP4)
+                            raw[kk].x = __ldcs(reinterpret_cast<const unsigned int *>(d + (int64_t)g * 4));
+                        else
+                            raw[kk] = __ldcs(reinterpret_cast<const uint2 *>(d + (int64_t)g * 8));
+                        if constexpr (QIN == QIN_INT8) sc[kk] = __ldg(reinterpret_cast<const float *>(sp));
+                        if constexpr (QIN == QIN_E4M3_B128)
+                            sc[kk] = __ldg(reinterpret_cast<const float *>(sp) + (g >> 4));
+                        if constexpr (QIN == QIN_MXFP8 || QIN == QIN_MXFP4)
+                            sc[kk] = exp2_neg(127 - (int)__ldg(sp + (g >> 2)));
+                    }
                 }
 #pragma unroll
                 for (int kk = 0; kk < KB; kk++) {
@@ -182,7 +138,28 @@ __global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a)
                     if (k >= a.K || s_row[grp][k] < 0) continue;
                     const float w = s_w[grp][k];
                     float v[8];
-                    decode_granule<QIN>(buf[kk], v);
+                    if constexpr (QIN == QIN_INT8) {
+#pragma unroll
+                        for (int q = 0; q < 8; q++) {
+                            const uint32_t word = q < 4 ? raw[kk].x : raw[kk].y;
+                            v[q] = __fmul_rn((float)(int8_t)((word >> (8 * (q & 3))) & 0xFFu), sc[kk]);
+                        }
+                    } else if constexpr (QIN == QIN_MXFP4) {
+#pragma unroll
+                        for (int q = 0; q < 4; q++) {
+                            const float2 f = e2m1x2_to_f32(raw[kk].x >> (8 * q));
+                            v[2 * q] = __fmul_rn(f.x, sc[kk]);
+                            v[2 * q + 1] = __fmul_rn(f.y, sc[kk]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; q++) {
+                            const uint32_t word = q < 2 ? raw[kk].x : raw[kk].y;
+                            const float2 f = e4m3x2_to_f32(word >> (16 * (q & 1)));
+                            v[2 * q] = __fmul_rn(f.x, sc[kk]);
+                            v[2 * q + 1] = __fmul_rn(f.y, sc[kk]);
+                        }
+                    }
 #pragma unroll
                     for (int q = 0; q < 8; q++) acc[q] = __fmaf_rn(w, v[q], acc[q]);
                 }
