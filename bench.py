@@ -107,7 +107,7 @@ def ncu_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel sources (else None)."""
     try:
-        with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+        with open(os.path.join(ROOT, "profiles", "decode_dispatch_combine_traffic.json")) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
