@@ -2,7 +2,7 @@
 //
 // "Low-Latency Mode API", low_latency_combine (Return Values: combined_x is
 // the weighted sum across experts) and "DeepEP FP8 Dispatch and Combine
-// Operations" (The FP8 Combine Operation: values are cast through fp32):
+// Operations" (The FP8 Combine Operation: the sum is taken in fp32):
 //   out[n,:] = bf16_rne( fma(w_{K-1}, y_{K-1}, ... fma(w_0, y_0, +0)) )
 // over the valid entries in k order.
 //

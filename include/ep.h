@@ -194,8 +194,8 @@ ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
  *          buffer of ep_sizes_t.recv_bytes in cfg->quant's format (data region
  *          then scale region, as ep_dispatch writes it) and each expert value
  *          is decode(code) * scale as one fp32 multiply before the FMA ([FP8]
- *          The FP8 Combine Operation: FP8 values times scale_inv, cast through
- *          fp32).  An e8m0 scale byte of 255 (NaN) is not a valid input.
+ *          The FP8 Combine Operation: codes times the stored inverse scale,
+ *          in fp32).  An e8m0 scale byte of 255 (NaN) is not a valid input.
  *   out    bf16 [N][H]
  */
 ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t *topk_idx,

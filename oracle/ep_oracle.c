@@ -124,9 +124,9 @@ float orc_e2m1_decode(uint8_t c)
 
 /*
  * e8m0 exponent of an MX block: X = ceil(log2 v) for v > 0, where
- * v = amax / qmax.  Reading of "round scaling factors into powers of 2"
- * ([LL] use_ue8m0 / round_scale) as rounding UP, so that every element of the
- * block fits: |x| * 2^-X <= qmax.  Written with frexp, which splits v into
+ * v = amax / qmax.  [LL] use_ue8m0 / round_scale ask for power-of-two scales
+ * without a rounding rule; the reading here rounds UP, so that every element of
+ * the block fits: |x| * 2^-X <= qmax.  Written with frexp, which splits v into
  * m * 2^e exactly (m in [0.5, 1)); log2 v is an integer only when m == 0.5.
  * The exponent is clamped to the e8m0 range [-127, 127] (byte 255 = NaN is
  * never produced).  amax == 0 gives X = 0 (scale 1.0).
@@ -481,8 +481,8 @@ uint32_t orc_combine_bwd(int R, int T, int K, int E, int M, int H, int layout, i
 
 /*
  * Dequantisation of one row stored in a quantised format ([FP8] The FP8
- * Combine Operation: the FP8 values are multiplied by the stored inverse
- * scale, casting through fp32).  Each element is decode(code) * scale_inv as
+ * Combine Operation: the received codes times the stored inverse scale, in
+ * fp32).  Each element is decode(code) * scale_inv as
  * one fp32 multiply: int8 codes and e4m3 / e2m1 values times the row's or
  * block's fp32 scale_inv, MX codes times 2^(byte-127).  BF16 rows widen
  * exactly.
