@@ -9,8 +9,17 @@ receive layout), on one GPU.
 
 Timing: CUDA events on the stream the kernels run on.  The timed region
 brackets each step with one event pair (the reported value); a second pass
-over the same steps puts an event between consecutive kernels for the
-per-kernel durations behind the roofline figures.  Between steps, outside the step's events, L2 is flushed by writing one
+times every kernel alone, between its own event pair, after its own L2 flush,
+for the per-kernel durations behind the roofline figures (a kernel that
+follows the dispatch in the same step would otherwise also pay the write-back
+of the dispatch's dirty L2 lines, which the step-level value already counts).
+A third pass, for workloads that move under 1 GiB a step, launches each
+kernel 4 times back to back on 4 distinct copies of its buffers between one
+pair of events: the per-launch time with the launch overhead amortised as in
+the step (an isolated launch carries ~6 us of launch and drain that the
+dependent launches of a step overlap); the roofline reports it, with the
+isolated figure beside it.
+Between steps, outside the step's events, L2 is flushed by writing one
 512 MiB buffer and then reading another: the read evicts the write's dirty
 lines, so every step starts from a cold L2 holding only clean lines (a
 write-only flush would leave ~126 MB of dirty lines whose write-back the next
@@ -364,15 +373,16 @@ def main():
                                             stream=stream, bind=True))
         step_calls.append(calls[-1])
 
-    def step(evs=None):
+    def step(evs=None, fl=0):
         if evs is None:
             for c in step_calls:
                 c()
             return
-        evs[0].record(stream)
         for i, c in enumerate(calls):
+            flush(fl)
+            evs[i][0].record(stream)
             c()
-            evs[i + 1].record(stream)
+            evs[i][1].record(stream)
 
     for _ in range(max(args.warmup, 3)):
         flush(1)
@@ -403,21 +413,22 @@ def main():
     ms_per_step = total_ms / args.steps
     value = world * N * args.steps / (total_ms / 1e3)
 
-    # per-kernel durations (for the roofline): the same steps again, with an
-    # event between consecutive kernels
-    nev = len(kernels) + 1
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    # per-kernel durations (for the roofline): the same steps again, each
+    # kernel after its own flush and between its own pair of events
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in kernels] for _ in range(args.steps)]
     torch.cuda.synchronize(dev)
     for s in range(args.steps):
-        flush(s & 0xFF)
-        step(evs[s])
+        step(evs[s], s & 0xFF)
     torch.cuda.synchronize(dev)
     per_kernel = {k: [] for k in kernels}
     for e in evs:
         for i, k in enumerate(kernels):
-            per_kernel[k].append(e[i].elapsed_time(e[i + 1]))
+            per_kernel[k].append(e[i][0].elapsed_time(e[i][1]))
 
     alg, v = algorithmic_bytes(w, mode, idx, quantized_combine=args.quantized_combine)
+    steady, sets = steady_launches(ep, args, cfg, ccfg, b, kernels, calls, x_d, idx_d, wts_d, g_d,
+                                   flush, stream, dev, sum(alg.values()))
     peaks = measured_peaks()
     peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else FALLBACK_HBM_GBS
     peak_src = "measured" if peaks and peaks.get("hbm_gbs") else "fallback"
@@ -430,9 +441,22 @@ def main():
                      "us_p90": round(float(np.percentile(per_kernel[k], 90)) * 1e3, 2),
                      "alg_bytes": alg[k], "gbs": round(gbs, 1),
                      "frac_of_" + peak_src: round(gbs / peak, 4)}
+        if sets > 1:
+            st_ms = statistics.mean(steady[k])
+            kstats[k].update({"us_steady": round(st_ms * 1e3, 2),
+                              "gbs_steady": round(alg[k] / (st_ms * 1e-3) / 1e9, 1),
+                              "frac_steady_of_" + peak_src:
+                                  round(alg[k] / (st_ms * 1e-3) / 1e9 / peak, 4)})
     dom = max(kernels, key=lambda k: alg[k])
-    dmean = statistics.mean(per_kernel[dom]) * 1e-3
-    achieved = alg[dom] / dmean / 1e9
+    iso_achieved = alg[dom] / (statistics.mean(per_kernel[dom]) * 1e-3) / 1e9
+    if sets > 1:
+        achieved = alg[dom] / (statistics.mean(steady[dom]) * 1e-3) / 1e9
+        duration = (f"per launch: {sets} launches back to back on {sets} distinct copies of the "
+                    f"kernel's inputs and outputs between one pair of events, L2 flushed before "
+                    f"each group")
+    else:
+        achieved = iso_achieved
+        duration = "per launch: each launch alone between its own events, after an L2 flush"
     step_bytes = sum(alg.values())
 
     # same-run copy bandwidth (reference for the fractions above)
@@ -477,7 +501,8 @@ def main():
                         + (", combine of quantised expert outputs" if args.quantized_combine else ""),
             "tokens_per_step": N, "valid_entries": v,
             "l2": f"flushed between steps outside the step events ({args.flush_mib} MiB write, "
-                  f"then {args.flush_mib} MiB read)",
+                  f"then {args.flush_mib} MiB read); per-kernel timings: each kernel after its "
+                  f"own flush",
             "parallelism": "replicas" if world > 1 else "single",
         },
         "hbm_gbs": round(step_bytes / (ms_per_step * 1e-3) / 1e9, 1),
@@ -487,7 +512,9 @@ def main():
         "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
                      "peak": peak, "peak_source": peak_src, "unit": "GB/s",
                      "frac": round(achieved / peak, 4),
-                     "traffic": ncu_traffic(dom, wname)},
+                     "traffic": ncu_traffic(dom, wname), "duration": duration,
+                     "isolated_launch": {"achieved": round(iso_achieved, 1),
+                                         "frac": round(iso_achieved / peak, 4)}},
         "kernels": kstats,
         "copy_gbs_same_run": copy_gbs,
         "e2e": e2e,
@@ -497,6 +524,59 @@ def main():
     if rank == 0:
         print(json.dumps(out), flush=True)
     dist_done(world)
+
+
+STEADY_SETS = 4
+STEADY_MAX_BYTES = 1 << 30
+
+
+def steady_launches(ep, args, cfg, ccfg, b, kernels, calls, x_d, idx_d, wts_d, g_d, flush, stream,
+                    dev, step_bytes):
+    """Per-launch durations with the launch overhead amortised as in the step:
+    each kernel is launched STEADY_SETS times back to back, on as many
+    distinct copies of the buffers it reads and writes (each launch's data is
+    cold: the group starts after an L2 flush and no two launches share a
+    buffer of the data path), between one pair of events; the dependent
+    launches overlap the tail of the previous grid, as the kernels of a step
+    do.  Workloads that move more than STEADY_MAX_BYTES a step are not timed
+    this way: there the launch overhead is already a negligible part of an
+    isolated launch.  Returns ({kernel: [ms per launch]}, sets)."""
+    if step_bytes > STEADY_MAX_BYTES:
+        return {}, 1
+    sets = STEADY_SETS
+    eo = b.expert_offset
+    per_set = {k: [calls[i]] for i, k in enumerate(kernels)}
+    keep = []
+    for _ in range(1, sets):
+        xs, rb, si = x_d.clone(), torch.empty_like(b.recv_buf), torch.empty_like(b.src_info)
+        ys, os_ = b.y.clone(), torch.empty_like(b.out)
+        keep += [xs, rb, si, ys, os_]
+        per_set["layout"].append(calls[0])
+        per_set["dispatch"].append(ep.ep_dispatch(cfg, xs, idx_d, b.token_slot, rb, si, b.dev_status,
+                                                  expert_offset=eo, stream=stream, bind=True))
+        per_set["combine"].append(ep.ep_combine(ccfg, ys, idx_d, wts_d, b.token_slot, os_,
+                                                b.dev_status, expert_offset=eo, stream=stream,
+                                                bind=True))
+        if "combine_bwd" in per_set:
+            gs, gb = g_d.clone(), torch.empty_like(b.grad_buf)
+            keep += [gs, gb]
+            per_set["combine_bwd"].append(ep.ep_combine_backward(
+                cfg, gs, idx_d, wts_d, b.token_slot, gb, b.dev_status, expert_offset=eo,
+                stream=stream, bind=True))
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in kernels] for _ in range(args.steps)]
+    for s in range(args.steps):
+        for i, k in enumerate(kernels):
+            flush(s & 0xFF)
+            evs[s][i][0].record(stream)
+            for c in per_set[k]:
+                c()
+            evs[s][i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    out = {k: [e[i][0].elapsed_time(e[i][1]) / sets for e in evs] for i, k in enumerate(kernels)}
+    del keep, per_set
+    torch.cuda.empty_cache()
+    return out, sets
 
 
 def run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, world):

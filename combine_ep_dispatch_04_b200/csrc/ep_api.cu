@@ -412,7 +412,7 @@ int sm_count();
 
 // `kernel_of(tpt, gmax)` returns the kernel instance (nullptr if none).
 template <typename KernelOf>
-Split split_rows(int64_t N, int ngran, int threads, int max_g, KernelOf kernel_of) {
+Split split_rows(int64_t N, int ngran, int max_g, KernelOf kernel_of) {
     const int64_t sms = sm_count();
     for (int tpt = 256; tpt >= 32; tpt >>= 1) {
         if (tpt > 32 && tpt / 2 >= ngran) continue;  // more than a warp of idle threads
@@ -421,6 +421,7 @@ Split split_rows(int64_t N, int ngran, int threads, int max_g, KernelOf kernel_o
         const int gmax = pow2_at_least(g);
         const void *fn = kernel_of(tpt, gmax);
         if (!fn) continue;
+        const int threads = ep::block_threads(tpt);
         const int64_t ctas = (N + threads / tpt - 1) / (threads / tpt);
         if (ctas <= sms * blocks_per_sm(fn, threads)) return {tpt, gmax};
     }
@@ -429,8 +430,8 @@ Split split_rows(int64_t N, int ngran, int threads, int max_g, KernelOf kernel_o
     return {tpt, pow2_at_least((ngran + tpt - 1) / tpt)};
 }
 
-unsigned grid_for(int64_t N, int threads, int tpt) {
-    const int toks = threads / tpt;
+unsigned grid_for(int64_t N, int tpt) {
+    const int toks = ep::block_threads(tpt) / tpt;
     return (unsigned)((N + toks - 1) / toks);
 }
 
@@ -448,11 +449,11 @@ ep_status_t launch_dispatch(const ep::DispatchArgs &a, cudaStream_t s) {
 #undef EP_FN
         return nullptr;
     };
-    const Split sp = split_rows(a.N, a.H / 16, ep::kDispatchThreads, 8, kernel_of);
-    const unsigned grid = grid_for(a.N, ep::kDispatchThreads, sp.tpt);
+    const Split sp = split_rows(a.N, a.H / 16, 8, kernel_of);
+    const unsigned grid = grid_for(a.N, sp.tpt);
 #define EP_CASE(T_, G_)                                                                     \
     if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
-        launch(ep::dispatch_kernel<MODE, T_, G_>, grid, ep::kDispatchThreads, 0, s, a);     \
+        launch(ep::dispatch_kernel<MODE, T_, G_>, grid, ep::block_threads(T_), 0, s, a);     \
         return launched();                                                                  \
     }
     EP_SPLITS(EP_CASE)
@@ -470,11 +471,11 @@ ep_status_t launch_combine_bwd(const ep::DispatchArgs &a, cudaStream_t s) {
 #undef EP_FN
         return nullptr;
     };
-    const Split sp = split_rows(a.N, a.H / 16, ep::kDispatchThreads, 2, kernel_of);
-    const unsigned grid = grid_for(a.N, ep::kDispatchThreads, sp.tpt);
+    const Split sp = split_rows(a.N, a.H / 16, 2, kernel_of);
+    const unsigned grid = grid_for(a.N, sp.tpt);
 #define EP_CASE(T_, G_)                                                                     \
     if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
-        launch(ep::combine_bwd_kernel<T_, G_>, grid, ep::kDispatchThreads, 0, s, a);        \
+        launch(ep::combine_bwd_kernel<T_, G_>, grid, ep::block_threads(T_), 0, s, a);        \
         return launched();                                                                  \
     }
     EP_SPLITS(EP_CASE)
@@ -583,11 +584,11 @@ ep_status_t launch_combine(const ep::CombineArgs &a, cudaStream_t s) {
 #undef EP_FN
         return nullptr;
     };
-    const Split sp = split_rows(a.N, a.H / 8, ep::kCombineThreads, 8, kernel_of);
-    const unsigned grid = grid_for(a.N, ep::kCombineThreads, sp.tpt);
+    const Split sp = split_rows(a.N, a.H / 8, 8, kernel_of);
+    const unsigned grid = grid_for(a.N, sp.tpt);
 #define EP_CASE(T_, G_)                                                                     \
     if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
-        launch(ep::combine_kernel<T_, G_, 8, QIN>, grid, ep::kCombineThreads, 0, s, a);     \
+        launch(ep::combine_kernel<T_, G_, 8, QIN>, grid, ep::block_threads(T_), 0, s, a);     \
         return launched();                                                                  \
     }
     EP_SPLITS(EP_CASE)

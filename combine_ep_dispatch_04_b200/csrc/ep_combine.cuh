@@ -6,9 +6,10 @@
 //   out[n,:] = bf16_rne( fma(w_{K-1}, y_{K-1}, ... fma(w_0, y_0, +0)) )
 // over the valid entries in k order.
 //
-// Work split: a group of TPT = 128 threads owns one token; the row is cut
-// into 8-element granules (16 bytes of bf16), thread lt holds granules
-// g = i*TPT + lt.  For each granule the thread first issues the loads of all
+// Work split: a group of TPT threads owns one token (TPT is chosen per shape
+// so that the grid fits in one wave where it can; a block holds
+// block_threads(TPT) / TPT tokens); the row is cut into 8-element granules
+// (16 bytes of bf16), thread lt holds granules g = i*TPT + lt.  For each granule the thread first issues the loads of all
 // K expert rows (up to KB = 8 independent 16-byte loads in flight), then runs
 // the fused multiply-adds in k order, so that memory latency is paid once per
 // granule rather than once per expert.  Expert rows are read exactly once:
@@ -34,8 +35,6 @@ struct CombineArgs {
     uint32_t *status;
 };
 
-constexpr int kCombineThreads = 256;
-
 enum { QIN_BF16 = 0, QIN_E4M3_B128 = 1, QIN_INT8 = 2, QIN_MXFP8 = 3, QIN_MXFP4 = 4 };
 
 // Quantised expert outputs ("DeepEP FP8 Dispatch and Combine Operations",
@@ -43,9 +42,9 @@ enum { QIN_BF16 = 0, QIN_E4M3_B128 = 1, QIN_INT8 = 2, QIN_MXFP8 = 3, QIN_MXFP4 =
 // the hardware conversions to f16, int8 as an integer) and multiplied by its
 // row / block scale as one fp32 multiply before the FMA.
 template <int TPT, int GMAX, int KB, int QIN>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(CombineArgs a) {
+__global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs a) {
     pdl_enter();
-    constexpr int TOKS = kCombineThreads / TPT;
+    constexpr int TOKS = block_threads(TPT) / TPT;
     __shared__ int64_t s_row[TOKS][16];
     __shared__ float s_w[TOKS][16];
 

@@ -16,6 +16,12 @@
 namespace ep {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
+
+// Threads of a block whose token groups have TPT threads: one token per block
+// from TPT = 128 up, 128 threads otherwise.  Small blocks spread the tokens of
+// a grid that fits in one wave evenly over the SMs (a block of two 128-thread
+// tokens leaves some SMs with one token more than the rest).
+__host__ __device__ constexpr int block_threads(int tpt) { return tpt < 128 ? 128 : tpt; }
 constexpr uint32_t kDevBadIndex = 0x1u;
 constexpr uint32_t kDevCapacity = 0x2u;
 

@@ -8,7 +8,8 @@
 // receive rows (data region) with its scales (scale region), src_info and the
 // optional weight.
 //
-// Work split: a group of TPT threads (1 or 2 warps) owns one token.  The row
+// Work split: a group of TPT threads owns one token (block_threads(TPT) / TPT
+// tokens per block).  The row
 // is cut into 16-element granules (32 bytes of bf16 input); thread lt of the
 // group holds granules g = i*TPT + lt, i < GMAX, as two 16-byte loads.  A
 // quantisation block of 128 elements is 8 consecutive threads and one of 32
@@ -43,8 +44,6 @@ struct DispatchArgs {
     float *recv_w;
     uint32_t *status;
 };
-
-constexpr int kDispatchThreads = 256;
 
 // Row of entry (n, k) in the receive layout, or -1 (masked, or no row).
 __device__ __forceinline__ int64_t entry_row(const DispatchArgs &a, int64_t n, int k,
@@ -102,8 +101,8 @@ __device__ __forceinline__ uint32_t q_i8(float v, float s) {
 // layout grid lets this grid launch only after its own wait for all earlier
 // work returned.  The slots are read after the wait.
 template <int MODE, int TPT, int GMAX>
-__global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs a) {
-    constexpr int TOKS = kDispatchThreads / TPT;
+__global__ void __launch_bounds__(block_threads(TPT)) dispatch_kernel(DispatchArgs a) {
+    constexpr int TOKS = block_threads(TPT) / TPT;
     constexpr int WPG = TPT / 32;  // warps per token group
     constexpr int OB = GranOut<MODE>::bytes;
     __shared__ int64_t s_row[TOKS][16];
@@ -297,9 +296,9 @@ __global__ void __launch_bounds__(kDispatchThreads) dispatch_kernel(DispatchArgs
 // |fl(w*g_h)| equals fl(|w| * max|g_h|) because rounding is monotone and sign
 // symmetric, so it is taken once per token and scaled per entry.
 template <int TPT, int GMAX>
-__global__ void __launch_bounds__(kDispatchThreads) combine_bwd_kernel(DispatchArgs a) {
+__global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(DispatchArgs a) {
     pdl_enter();
-    constexpr int TOKS = kDispatchThreads / TPT;
+    constexpr int TOKS = block_threads(TPT) / TPT;
     __shared__ int64_t s_row[TOKS][16];
     __shared__ float s_w[TOKS][16];
 
