@@ -7,7 +7,9 @@ product.  The arithmetic lives in ``ep_oracle.c``; this module only builds and
 loads it and marshals numpy arrays.
 
 Modes and layouts use the names of the product's enums, mapped here by value:
-bf16=0, e4m3_b128=1, int8_token=2, mxfp8=3, mxfp4=4; padded=0, packed=1.
+bf16=0, e4m3_b128=1, int8_token=2, mxfp8=3, mxfp4=4; padded=0, packed=1.  Two
+more modes are e4m3_b128 with the scale options: e4m3_b128_p2 (round_scale:
+power-of-two fp32 scales) and e4m3_b128_ue8m0 (the same as e8m0 bytes).
 """
 import ctypes as C
 
@@ -15,7 +17,8 @@ import numpy as np
 
 from . import build as _build
 
-MODES = {"bf16": 0, "e4m3_b128": 1, "int8_token": 2, "mxfp8": 3, "mxfp4": 4}
+MODES = {"bf16": 0, "e4m3_b128": 1, "int8_token": 2, "mxfp8": 3, "mxfp4": 4,
+         "e4m3_b128_p2": 5, "e4m3_b128_ue8m0": 6}
 LAYOUTS = {"padded": 0, "packed": 1}
 ST_BAD_INDEX = 0x1
 ST_CAPACITY = 0x2

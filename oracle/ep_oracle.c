@@ -36,7 +36,9 @@
 #include <string.h>
 
 /* ---- modes, layouts and status bits (restated from their meaning) ------- */
-enum { ORC_BF16 = 0, ORC_E4M3_B128 = 1, ORC_INT8_TOKEN = 2, ORC_MXFP8 = 3, ORC_MXFP4 = 4 };
+enum { ORC_BF16 = 0, ORC_E4M3_B128 = 1, ORC_INT8_TOKEN = 2, ORC_MXFP8 = 3, ORC_MXFP4 = 4,
+       ORC_E4M3_B128_P2 = 5,     /* E4M3_B128 with round_scale: fp32 scales, powers of two */
+       ORC_E4M3_B128_UE8M0 = 6 }; /* ... stored as e8m0 bytes, 4 to an int32 (use_ue8m0) */
 enum { ORC_PADDED = 0, ORC_PACKED = 1 };
 #define ORC_ST_BAD_INDEX 0x1u
 #define ORC_ST_CAPACITY 0x2u
@@ -162,6 +164,8 @@ long orc_row_scale_bytes(int mode, int H)
     case ORC_BF16: return 0;
     case ORC_INT8_TOKEN: return 4;
     case ORC_E4M3_B128: return 4L * (H / 128);
+    case ORC_E4M3_B128_P2: return 4L * (H / 128);
+    case ORC_E4M3_B128_UE8M0: return 4L * ((H / 128 + 3) / 4); /* whole int32 words, pad bytes 0 */
     default: return H / 32; /* one e8m0 byte per 32 elements */
     }
 }
@@ -191,6 +195,15 @@ static float absmax(const float *x, int n)
  *               e4m3(x * 2^-X), byte = X + 127.
  *   MXFP4:      as MXFP8 with e2m1 (max 6); two codes per byte, element 2i
  *               in the low nibble ([LL] use_mxfp4: data [rows, H/2]).
+ *   E4M3_B128_P2: E4M3_B128 with round_scale ([LL] round_scale; [FP8]
+ *               Advanced Configuration Options, Round-Scale Mode): the
+ *               block's scale is the power of two of the MX rule, X =
+ *               ceil(log2(amax_b/qmax)), code = e4m3(x * 2^-X), stored
+ *               scale_inv = 2^X (fp32).
+ *   E4M3_B128_UE8M0: the same codes, the scale stored as the e8m0 byte
+ *               X + 127, one per block, four to an int32 ([FP8] Advanced
+ *               Configuration Options, UE8M0 Support: 8-bit scales in a
+ *               packed format); the row's unused pad bytes are 0.
  * amax == 0 uses the scale 1 (stored 1.0f or byte 127).  The int8/e4m3
  * scale s is limited to FLT_MAX so that a tiny amax cannot turn 0*s into NaN.
  */
@@ -234,6 +247,25 @@ void orc_quant_row_f32(int mode, int H, float e4m3_qmax, const float *x, uint8_t
             }
             for (int i = 0; i < 128; i++) data[128L * b + i] = orc_e4m3_encode(xb[i] * s);
             memcpy(scale + 4L * b, &sinv, 4);
+        }
+        return;
+    }
+    if (mode == ORC_E4M3_B128_P2 || mode == ORC_E4M3_B128_UE8M0) {
+        float qmax = e4m3_qmax > 0.0f ? e4m3_qmax : 448.0f;
+        int nb = H / 128;
+        if (mode == ORC_E4M3_B128_UE8M0)
+            memset(scale, 0, (size_t)orc_row_scale_bytes(mode, H));
+        for (int b = 0; b < nb; b++) {
+            const float *xb = x + 128L * b;
+            int X = orc_mx_exponent(absmax(xb, 128), qmax);
+            float mult = ldexpf(1.0f, -X);
+            for (int i = 0; i < 128; i++) data[128L * b + i] = orc_e4m3_encode(xb[i] * mult);
+            if (mode == ORC_E4M3_B128_P2) {
+                float sinv = ldexpf(1.0f, X);
+                memcpy(scale + 4L * b, &sinv, 4);
+            } else {
+                scale[b] = (uint8_t)(X + 127);
+            }
         }
         return;
     }
@@ -383,8 +415,8 @@ uint32_t orc_dispatch(int R, int T, int K, int E, int M, int H, int mode, float 
 
 /*
  * Weighted top-k combine of one token ([LL] low_latency_combine: combined_x
- * is the weighted sum across experts; [FP8] The FP8 Combine Operation: cast
- * through fp32).  acc starts at +0 and, for k = 0..K-1 in order, each valid
+ * is the weighted sum across experts; [FP8] The FP8 Combine Operation: the
+ * sum is taken in fp32).  acc starts at +0 and, for k = 0..K-1 in order, each valid
  * entry adds w_k * y_k with one fused multiply-add; the sum is rounded to
  * bf16 (RNE).  Masked entries add nothing; weights are used as given.
  */
@@ -503,8 +535,13 @@ void orc_dequant_row(int mode, int H, const uint8_t *data, const uint8_t *scale,
             memcpy(&s, scale, 4);
             break;
         case ORC_E4M3_B128:
+        case ORC_E4M3_B128_P2:
             v = orc_e4m3_decode(data[h]);
             memcpy(&s, scale + 4L * (h / 128), 4);
+            break;
+        case ORC_E4M3_B128_UE8M0:
+            v = orc_e4m3_decode(data[h]);
+            s = ldexpf(1.0f, (int)scale[h / 128] - 127);
             break;
         case ORC_MXFP8:
             v = orc_e4m3_decode(data[h]);

@@ -616,3 +616,78 @@ def test_combine_of_bf16_rows_is_the_plain_combine():
     valid = np.ones((N, K), np.uint8)
     got = oracle.combine_gathered_q("bf16", y.view(np.uint8).reshape(N, K, 2 * H), np.zeros((N, K, 0), np.uint8), w, valid, H)
     assert np.array_equal(got, oracle.combine_gathered(y, w, valid))
+
+
+# ---------------------------------------------------------------------------
+# E4M3 per 128 with round_scale (power-of-two fp32 scales) and with UE8M0
+# (the same scales as e8m0 bytes, four to an int32)
+# ---------------------------------------------------------------------------
+
+def _block_max_in_every_32(x_bits):
+    """bf16 row whose four 32-element sub-blocks of each 128-block share the
+    128-block's maximum magnitude (its element 0 carries it, sign kept)."""
+    xf = _f(x_bits).reshape(-1, 128).copy()
+    amax = np.abs(xf).max(axis=1)
+    for j in range(4):
+        xf[:, 32 * j] = np.where(xf[:, 32 * j] < 0, -amax, amax)
+    return synth.to_bf16_bits(xf.reshape(-1).astype(np.float32))
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_round_scale_equals_mxfp8_when_sub_blocks_share_the_maximum(seed):
+    """With qmax 448, a 128-block whose four 32-blocks have the same maximum is
+    quantised by round_scale exactly as MXFP8 quantises each of them (MXFP8 is
+    pinned on its own above): the same codes, and 2^X = 2^(byte - 127)."""
+    H = 1024
+    x = _block_max_in_every_32(_bf16_row(H, scale=10.0 ** (seed - 2), seed=40 + seed))
+    d2, s2 = oracle.quant_row("e4m3_b128_p2", x)
+    dm, sm = oracle.quant_row("mxfp8", x)
+    assert np.array_equal(d2, dm)
+    p2 = s2.view(np.float32).astype(np.float64)
+    assert np.array_equal(np.repeat(p2, 4), np.ldexp(1.0, sm.astype(np.int64) - 127))
+
+
+@pytest.mark.parametrize("qmax", [448.0, 240.0, 127.0])
+@pytest.mark.parametrize("seed", range(3))
+def test_round_scale_is_the_smallest_power_of_two_that_fits(qmax, seed):
+    """By definition: scale_inv = 2^X with amax * 2^-X <= qmax < amax * 2^-(X-1)
+    (checked in float64 on the fp32 quotient), and the codes are e4m3 of x * 2^-X."""
+    H = 2048
+    x = _bf16_row(H, scale=10.0 ** (seed - 1), seed=50 + seed)
+    d, s = oracle.quant_row("e4m3_b128_p2", x, e4m3_qmax=qmax)
+    sinv = s.view(np.float32).astype(np.float64)
+    X = np.log2(sinv)
+    assert np.all(X == np.round(X))
+    xf = _f(x).reshape(-1, 128)
+    amax = np.abs(xf).max(axis=1)
+    v = (amax.astype(np.float32) / np.float32(qmax)).astype(np.float64)
+    assert np.all(v <= sinv) and np.all(v > sinv / 2)
+    want = oracle.e4m3_encode((xf * (1.0 / sinv)[:, None]).astype(np.float32).reshape(-1))
+    assert np.array_equal(d, want)
+
+
+@pytest.mark.parametrize("H", [128, 384, 1024, 7168])
+def test_ue8m0_is_round_scale_with_byte_scales(H):
+    x = _bf16_row(H, seed=H)
+    d2, s2 = oracle.quant_row("e4m3_b128_p2", x)
+    du, su = oracle.quant_row("e4m3_b128_ue8m0", x)
+    nb = H // 128
+    assert oracle.row_bytes("e4m3_b128_ue8m0", H) == (H, 4 * ((nb + 3) // 4))
+    assert np.array_equal(d2, du)
+    X = np.log2(s2.view(np.float32).astype(np.float64)).astype(np.int64)
+    assert np.array_equal(su[:nb].astype(np.int64), X + 127)
+    assert np.all(su[nb:] == 0)
+    # the two scale forms dequantise to the same values
+    y2 = oracle.dequant_row("e4m3_b128_p2", d2, s2, H)
+    yu = oracle.dequant_row("e4m3_b128_ue8m0", du, su, H)
+    assert np.array_equal(y2.view(np.uint32), yu.view(np.uint32))
+
+
+def test_round_scale_zero_block_uses_unit_scale():
+    x = np.zeros(256, np.uint16)
+    x[128:] = synth.to_bf16_bits(np.float32([3.0] * 128))
+    d, s = oracle.quant_row("e4m3_b128_p2", x)
+    assert list(s.view(np.float32)) == [1.0, 2.0 ** -7]     # 3/448 -> X = -7
+    du, su = oracle.quant_row("e4m3_b128_ue8m0", x)
+    assert list(su) == [127, 120, 0, 0]
+    assert np.all(d[:128] == 0) and np.all(d[128:] == oracle.e4m3_encode(np.float32([3.0 * 128]))[0])
