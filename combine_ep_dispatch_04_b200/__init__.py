@@ -4,14 +4,19 @@ The work runs in libep.so (C ABI in include/ep.h, sm_100a CUDA kernels);
 ``ep`` is its thin Python binding.  Importing the package without the built
 library raises ImportError: there is no CPU or library fallback.
 """
-from .ep import (DEV_BAD_INDEX, DEV_CAPACITY_OVERFLOW, STATIC_SCRATCH_BYTES, F_BWD_UNWEIGHTED, F_COMBINE_QUANTIZED, F_LAYOUT_CLUSTER, F_LAYOUT_MULTI_CTA,
-                 F_LAYOUT_SINGLE_CTA, LAYOUT, QUANT, Buffers, EpConfig, EpError, EpSizes,
-                 Bound, ep_buffer_sizes, ep_combine, ep_combine_backward, ep_copy, ep_cvt_sweep,
-                 ep_dispatch, ep_dispatch_layout, ep_dispatch_layout_static, ep_dispatch_with_layout, ep_get_status, ep_kernel_launches, make_config)
+from .ep import (DEV_BAD_INDEX, DEV_CAPACITY_OVERFLOW, STATIC_SCRATCH_BYTES, F_BWD_UNWEIGHTED,
+                 F_COMBINE_QUANTIZED, F_IDX_I32, F_LAYOUT_CLUSTER, F_LAYOUT_MULTI_CTA,
+                 F_LAYOUT_SINGLE_CTA, F_ROUND_SCALE, F_UE8M0, LAYOUT, QUANT, Bound, Buffers,
+                 EpConfig, EpError, EpSizes, ep_buffer_sizes, ep_combine, ep_combine_backward,
+                 ep_copy, ep_cvt_sweep, ep_dispatch, ep_dispatch_layout,
+                 ep_dispatch_layout_static, ep_dispatch_with_layout, ep_get_status,
+                 ep_kernel_launches, idx_dtype, make_config)
 
 __all__ = [
-    "DEV_BAD_INDEX", "DEV_CAPACITY_OVERFLOW", "STATIC_SCRATCH_BYTES", "F_BWD_UNWEIGHTED", "F_COMBINE_QUANTIZED", "F_LAYOUT_CLUSTER", "F_LAYOUT_MULTI_CTA",
-    "F_LAYOUT_SINGLE_CTA", "LAYOUT", "QUANT", "Bound", "Buffers", "EpConfig", "EpError", "EpSizes",
-    "ep_buffer_sizes", "ep_combine", "ep_combine_backward", "ep_copy", "ep_cvt_sweep",
-    "ep_dispatch", "ep_dispatch_layout", "ep_dispatch_layout_static", "ep_dispatch_with_layout", "ep_get_status", "ep_kernel_launches", "make_config",
+    "DEV_BAD_INDEX", "DEV_CAPACITY_OVERFLOW", "STATIC_SCRATCH_BYTES", "F_BWD_UNWEIGHTED",
+    "F_COMBINE_QUANTIZED", "F_IDX_I32", "F_LAYOUT_CLUSTER", "F_LAYOUT_MULTI_CTA",
+    "F_LAYOUT_SINGLE_CTA", "F_ROUND_SCALE", "F_UE8M0", "LAYOUT", "QUANT", "Bound", "Buffers",
+    "EpConfig", "EpError", "EpSizes", "ep_buffer_sizes", "ep_combine", "ep_combine_backward",
+    "ep_copy", "ep_cvt_sweep", "ep_dispatch", "ep_dispatch_layout", "ep_dispatch_layout_static",
+    "ep_dispatch_with_layout", "ep_get_status", "ep_kernel_launches", "idx_dtype", "make_config",
 ]

@@ -69,13 +69,26 @@ struct Plan {
 int64_t data_row_bytes(int quant, int H) {
     return quant == EP_Q_BF16 ? 2LL * H : (quant == EP_Q_MXFP4 ? H / 2 : H);
 }
-int64_t scale_row_bytes(int quant, int H) {
+int64_t scale_row_bytes(int quant, int H, uint32_t flags) {
     switch (quant) {
     case EP_Q_BF16: return 0;
     case EP_Q_INT8_TOKEN: return 4;
-    case EP_Q_E4M3_B128: return 4LL * (H / 128);
+    case EP_Q_E4M3_B128:  // fp32 per 128, or e8m0 bytes in whole int32 words
+        return (flags & EP_F_UE8M0) ? 4LL * ((H / 128 + 3) / 4) : 4LL * (H / 128);
     default: return H / 32;
     }
+}
+
+// E4M3_B128 scale format: 0 = qmax/amax in fp32, 1 = power of two in fp32,
+// 2 = e8m0 bytes.
+int e4m3_scale_format(const ep_config_t *cfg) {
+    if (cfg->quant != EP_Q_E4M3_B128) return 0;
+    if (cfg->flags & EP_F_UE8M0) return 2;
+    return (cfg->flags & EP_F_ROUND_SCALE) ? 1 : 0;
+}
+
+ep::TopkIdx topk_idx_view(const ep_config_t *cfg, const void *topk_idx) {
+    return ep::TopkIdx{topk_idx, (cfg->flags & EP_F_IDX_I32) ? 1 : 0};
 }
 
 // Every check happens before any arithmetic that uses the values.
@@ -94,8 +107,14 @@ ep_status_t make_plan(const ep_config_t *c, Plan &p) {
     if (c->expert_align < 1) return EP_ERR_INVALID_ARG;
     if (!(c->e4m3_qmax >= 0.0f && c->e4m3_qmax <= 448.0f)) return EP_ERR_INVALID_ARG;  // NaN fails
     const uint32_t paths = EP_F_LAYOUT_SINGLE_CTA | EP_F_LAYOUT_MULTI_CTA | EP_F_LAYOUT_CLUSTER;
-    const uint32_t known = EP_F_BWD_UNWEIGHTED | EP_F_COMBINE_QUANTIZED | paths;
+    const uint32_t known = EP_F_BWD_UNWEIGHTED | EP_F_COMBINE_QUANTIZED | EP_F_IDX_I32 |
+                           EP_F_ROUND_SCALE | EP_F_UE8M0 | paths;
     if (c->flags & ~known) return EP_ERR_INVALID_ARG;
+    // power-of-two scales exist for the e4m3 / e2m1 formats only (MX scales
+    // already are); e8m0 storage of the per-128 scales only for E4M3_B128
+    if ((c->flags & EP_F_ROUND_SCALE) && (c->quant == EP_Q_BF16 || c->quant == EP_Q_INT8_TOKEN))
+        return EP_ERR_INVALID_ARG;
+    if ((c->flags & EP_F_UE8M0) && c->quant != EP_Q_E4M3_B128) return EP_ERR_INVALID_ARG;
     const uint32_t forced = c->flags & paths;
     if (forced & (forced - 1)) return EP_ERR_INVALID_ARG;  // at most one path flag
 
@@ -118,7 +137,7 @@ ep_status_t make_plan(const ep_config_t *c, Plan &p) {
         if (p.rows > kIntLimit) return EP_ERR_INVALID_ARG;  // expert_offset scan is int32 per tile
     }
     p.D = data_row_bytes(c->quant, p.H);
-    p.S = scale_row_bytes(c->quant, p.H);
+    p.S = scale_row_bytes(c->quant, p.H, c->flags);
     p.scale_off = round_up(p.rows * p.D, 256);
     p.recv_bytes = p.scale_off + p.rows * p.S;
     p.grad_scale_off = round_up(p.rows * p.H, 256);
@@ -135,9 +154,9 @@ ep_status_t make_plan(const ep_config_t *c, Plan &p) {
 
 
 struct ClusterChoice;
-ep_status_t check_layout_args(const ep_config_t *, const Plan &, const int64_t *, const int32_t *,
+ep_status_t check_layout_args(const ep_config_t *, const Plan &, const void *, const int32_t *,
                               const int64_t *, const int64_t *, const void *, const uint32_t *);
-ep::LayoutArgs layout_args(const ep_config_t *, const Plan &, const int64_t *, int32_t *, int32_t *,
+ep::LayoutArgs layout_args(const ep_config_t *, const Plan &, const void *, int32_t *, int32_t *,
                            uint8_t *, int32_t *, int64_t *, int64_t *, int64_t *, void *,
                            uint32_t *);
 ep_status_t run_layout(const ep_config_t *, const Plan &, const ep::LayoutArgs &, cudaStream_t);
@@ -359,7 +378,7 @@ ep_status_t ep_buffer_sizes(const ep_config_t *cfg, ep_sizes_t *out) {
     return EP_OK;
 }
 
-ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const int64_t *topk_idx,
+ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const void *topk_idx,
                                int32_t *tokens_per_rank, int32_t *tokens_per_expert,
                                uint8_t *is_token_in_rank, int32_t *token_slot,
                                int64_t *recv_count, int64_t *expert_offset,
@@ -491,12 +510,13 @@ ep::DispatchArgs dispatch_args(const ep_config_t *cfg, const Plan &p) {
     a.cap = p.cap;
     a.rows = p.rows;
     a.qmax = cfg->e4m3_qmax > 0.0f ? cfg->e4m3_qmax : 448.0f;
+    a.sfmt = e4m3_scale_format(cfg);
     return a;
 }
 
 
 // ---- argument checks and launch bodies shared by the entry points ----------------
-ep_status_t check_layout_args(const ep_config_t *cfg, const Plan &p, const int64_t *topk_idx,
+ep_status_t check_layout_args(const ep_config_t *cfg, const Plan &p, const void *topk_idx,
                               const int32_t *token_slot, const int64_t *recv_count,
                               const int64_t *expert_offset, const void *workspace,
                               const uint32_t *dev_status) {
@@ -506,7 +526,7 @@ ep_status_t check_layout_args(const ep_config_t *cfg, const Plan &p, const int64
     return EP_OK;
 }
 
-ep::LayoutArgs layout_args(const ep_config_t *cfg, const Plan &p, const int64_t *topk_idx,
+ep::LayoutArgs layout_args(const ep_config_t *cfg, const Plan &p, const void *topk_idx,
                            int32_t *tokens_per_rank, int32_t *tokens_per_expert,
                            uint8_t *is_token_in_rank, int32_t *token_slot, int64_t *recv_count,
                            int64_t *expert_offset, int64_t *cumulative_recv_stats,
@@ -517,7 +537,7 @@ ep::LayoutArgs layout_args(const ep_config_t *cfg, const Plan &p, const int64_t 
     a.packed = cfg->layout == EP_LAYOUT_PACKED;
     a.align = cfg->expert_align;
     a.cap = p.cap;
-    a.idx = topk_idx;
+    a.idx = topk_idx_view(cfg, topk_idx);
     a.tpr = tokens_per_rank;
     a.tpe = tokens_per_expert;
     a.itr = is_token_in_rank;
@@ -549,7 +569,7 @@ ep_status_t run_layout(const ep_config_t *cfg, const Plan &p, const ep::LayoutAr
     return launch_layout_multi(a, p, s);
 }
 
-ep_status_t check_dispatch_args(const ep_config_t *cfg, const uint16_t *x, const int64_t *topk_idx,
+ep_status_t check_dispatch_args(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
                                 const float *topk_weights, const int32_t *token_slot,
                                 const int64_t *expert_offset, const void *recv_buf,
                                 const int32_t *src_info, const float *recv_weights) {
@@ -561,13 +581,14 @@ ep_status_t check_dispatch_args(const ep_config_t *cfg, const uint16_t *x, const
 }
 
 ep::DispatchArgs full_dispatch_args(const ep_config_t *cfg, const Plan &p, const uint16_t *x,
-                                    const int64_t *topk_idx, const float *topk_weights,
+                                    const void *topk_idx, const float *topk_weights,
                                     const int32_t *token_slot, const int64_t *expert_offset,
                                     void *recv_buf, int32_t *src_info, float *recv_weights,
                                     uint32_t *dev_status) {
     ep::DispatchArgs a = dispatch_args(cfg, p);
     a.D = p.D; a.S = p.S; a.scale_off = p.scale_off;
-    a.x = x; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
+    a.x = x; a.idx = topk_idx_view(cfg, topk_idx);
+    a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
     a.out = static_cast<uint8_t *>(recv_buf);
     a.src_info = src_info;
     a.recv_w = recv_weights;
@@ -575,7 +596,7 @@ ep::DispatchArgs full_dispatch_args(const ep_config_t *cfg, const Plan &p, const
     return a;
 }
 
-// 8-element granules: 16 bytes of bf16, 8 of int8 / e4m3, 4 of e2m1.
+// Granules of 16 bytes of expert output (combine_granule elements).
 template <int QIN>
 ep_status_t launch_combine(const ep::CombineArgs &a, cudaStream_t s) {
     auto kernel_of = [](int t, int g) -> const void * {
@@ -584,7 +605,7 @@ ep_status_t launch_combine(const ep::CombineArgs &a, cudaStream_t s) {
 #undef EP_FN
         return nullptr;
     };
-    const Split sp = split_rows(a.N, a.H / 8, 8, kernel_of);
+    const Split sp = split_rows(a.N, a.H / ep::combine_granule(QIN), 8, kernel_of);
     const unsigned grid = grid_for(a.N, sp.tpt);
 #define EP_CASE(T_, G_)                                                                     \
     if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
@@ -610,7 +631,7 @@ ep_status_t run_dispatch(const ep_config_t *cfg, const ep::DispatchArgs &a, cuda
 
 extern "C" {
 
-ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const int64_t *topk_idx,
+ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
                         const float *topk_weights, const int32_t *token_slot,
                         const int64_t *expert_offset, void *recv_buf, int32_t *src_info,
                         float *recv_weights, uint32_t *dev_status, ep_stream_t stream) {
@@ -629,7 +650,7 @@ ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const int64_t
 }
 
 ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
-                                    const int64_t *topk_idx, const float *topk_weights,
+                                    const void *topk_idx, const float *topk_weights,
                                     int32_t *tokens_per_rank, int32_t *tokens_per_expert,
                                     uint8_t *is_token_in_rank, int32_t *token_slot,
                                     int64_t *recv_count, int64_t *expert_offset,
@@ -659,7 +680,7 @@ ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
     return run_dispatch(cfg, a, s);
 }
 
-ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t *topk_idx,
+ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const void *topk_idx,
                        const float *topk_weights, const int32_t *token_slot,
                        const int64_t *expert_offset, uint16_t *out, uint32_t *dev_status,
                        ep_stream_t stream) {
@@ -678,7 +699,9 @@ ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t 
     a.packed = cfg->layout == EP_LAYOUT_PACKED;
     a.cap = p.cap; a.rows = p.rows;
     a.D = p.D; a.S = p.S; a.scale_off = p.scale_off;
-    a.y = y; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
+    a.sfmt = e4m3_scale_format(cfg);
+    a.y = y; a.idx = topk_idx_view(cfg, topk_idx);
+    a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
     a.out = out; a.status = dev_status;
     cudaStream_t s = cs(stream);
     switch (qin) {
@@ -691,7 +714,7 @@ ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t 
 }
 
 ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
-                                const int64_t *topk_idx, const float *topk_weights,
+                                const void *topk_idx, const float *topk_weights,
                                 const int32_t *token_slot, const int64_t *expert_offset,
                                 void *grad_buf, uint32_t *dev_status, ep_stream_t stream) {
     Plan p;
@@ -708,7 +731,8 @@ ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
     ep::DispatchArgs a = dispatch_args(cfg, p);
     a.D = p.H; a.S = p.H / 32; a.scale_off = p.grad_scale_off;
     a.unweighted = unweighted;
-    a.x = g; a.idx = topk_idx; a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
+    a.x = g; a.idx = topk_idx_view(cfg, topk_idx);
+    a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
     a.out = static_cast<uint8_t *>(grad_buf);
     a.status = dev_status;
     return launch_combine_bwd(a, cs(stream));
@@ -823,7 +847,7 @@ ep_status_t static_scratch(void **out) {
 }  // namespace
 
 extern "C" ep_status_t ep_dispatch_layout_static(
-    const ep_config_t *cfg, const int64_t *topk_idx, int32_t *tokens_per_rank,
+    const ep_config_t *cfg, const void *topk_idx, int32_t *tokens_per_rank,
     int32_t *tokens_per_expert, uint8_t *is_token_in_rank, int32_t *token_slot,
     int64_t *recv_count, int64_t *expert_offset, int64_t *cumulative_recv_stats,
     uint32_t *dev_status, ep_stream_t stream) {
@@ -843,7 +867,7 @@ extern "C" ep_status_t ep_dispatch_layout_static(
     a.packed = cfg->layout == EP_LAYOUT_PACKED;
     a.align = cfg->expert_align;
     a.cap = p.cap;
-    a.idx = topk_idx;
+    a.idx = topk_idx_view(cfg, topk_idx);
     a.tpr = tokens_per_rank;
     a.tpe = tokens_per_expert;
     a.itr = is_token_in_rank;

@@ -8,12 +8,13 @@
 //
 // Work split: a group of TPT threads owns one token (TPT is chosen per shape
 // so that the grid fits in one wave where it can; a block holds
-// block_threads(TPT) / TPT tokens); the row is cut into 8-element granules
-// (16 bytes of bf16), thread lt holds granules g = i*TPT + lt.  For each granule the thread first issues the loads of all
-// K expert rows (up to KB = 8 independent 16-byte loads in flight), then runs
-// the fused multiply-adds in k order, so that memory latency is paid once per
-// granule rather than once per expert.  Expert rows are read exactly once:
-// loads are streaming (evict-first).
+// block_threads(TPT) / TPT tokens); the row is cut into granules of 16 bytes
+// of expert output (8 bf16 elements; 16 e4m3 / int8 codes; 32 e2m1 codes),
+// thread lt holds granules g = i*TPT + lt.  For each granule the thread first
+// issues the loads of all K expert rows (up to KB = 8 independent 16-byte
+// loads in flight), then runs the fused multiply-adds in k order, so that
+// memory latency is paid once per granule rather than once per expert.
+// Expert rows are read exactly once: loads are streaming (evict-first).
 #pragma once
 
 #include "ep_device.cuh"
@@ -26,8 +27,9 @@ struct CombineArgs {
     int packed;
     int64_t cap, rows;
     int64_t D, S, scale_off;  // quantised expert outputs: row bytes, scale bytes, scale region
+    int sfmt;                 // e4m3_b128 scales: fp32 (0, 1) or e8m0 bytes (2)
     const uint16_t *y;        // bf16 rows, or the quantised buffer (data then scales)
-    const int64_t *idx;
+    TopkIdx idx;
     const float *wts;
     const int32_t *slot;
     const int64_t *eo;
@@ -37,14 +39,75 @@ struct CombineArgs {
 
 enum { QIN_BF16 = 0, QIN_E4M3_B128 = 1, QIN_INT8 = 2, QIN_MXFP8 = 3, QIN_MXFP4 = 4 };
 
+// Elements of a granule: 16 bytes of bf16 expert output, or of codes.
+__host__ __device__ constexpr int combine_granule(int qin) {
+    return qin == QIN_BF16 ? 8 : (qin == QIN_MXFP4 ? 32 : 16);
+}
+
 // Quantised expert outputs ("DeepEP FP8 Dispatch and Combine Operations",
-// The FP8 Combine Operation): each code is decoded exactly (e4m3 / e2m1 via
-// the hardware conversions to f16, int8 as an integer) and multiplied by its
-// row / block scale as one fp32 multiply before the FMA.
+// The FP8 Combine Operation): every code is decoded exactly and multiplied by
+// its row / block scale as one fp32 multiply, y = fl(decode(c) * s), before
+// the FMA.  The decode is done with integer operations (e4m3_rebiased and
+// the like), its power-of-two factor folded into the scale: fl(c' * (s*2^B))
+// is the same single rounding of the same real product.  Where s*2^B is not
+// finite, or an e4m3 code is NaN, the hardware conversions decode instead.
+template <int QIN>
+__device__ __forceinline__ void dequant_fma(float (&acc)[combine_granule(QIN)], const uint4 &r,
+                                            float s, float w) {
+    constexpr int EPG = combine_granule(QIN);
+    const uint32_t u[4] = {r.x, r.y, r.z, r.w};
+    float v[EPG];
+    if constexpr (QIN == QIN_INT8) {
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            const uint32_t wx = u[q] ^ 0x80808080u;
+#pragma unroll
+            for (int j = 0; j < 4; j++) v[4 * q + j] = __fmul_rn(i8_exact(wx, j), s);
+        }
+    } else if constexpr (QIN == QIN_MXFP4) {
+        const float s1 = __fmul_rn(s, 0x1p126f);
+        if (fabsf(s1) <= FLT_MAX) {
+#pragma unroll
+            for (int q = 0; q < 4; q++)
+#pragma unroll
+                for (int j = 0; j < 8; j++) v[8 * q + j] = __fmul_rn(e2m1_rebiased(u[q], j), s1);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; q++)
+#pragma unroll
+                for (int b = 0; b < 4; b++) {
+                    const float2 f = e2m1x2_to_f32(u[q] >> (8 * b));
+                    v[8 * q + 2 * b] = __fmul_rn(f.x, s);
+                    v[8 * q + 2 * b + 1] = __fmul_rn(f.y, s);
+                }
+        }
+    } else {  // e4m3 codes
+        const float s1 = __fmul_rn(s, 0x1p120f);
+        if (fabsf(s1) <= FLT_MAX && !e4m3_has_nan(u)) {
+#pragma unroll
+            for (int q = 0; q < 4; q++)
+#pragma unroll
+                for (int j = 0; j < 4; j++) v[4 * q + j] = __fmul_rn(e4m3_rebiased(u[q], j), s1);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; q++)
+#pragma unroll
+                for (int h = 0; h < 2; h++) {
+                    const float2 f = e4m3x2_to_f32(u[q] >> (16 * h));
+                    v[4 * q + 2 * h] = __fmul_rn(f.x, s);
+                    v[4 * q + 2 * h + 1] = __fmul_rn(f.y, s);
+                }
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < EPG; j++) acc[j] = __fmaf_rn(w, v[j], acc[j]);
+}
+
 template <int TPT, int GMAX, int KB, int QIN>
 __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs a) {
     pdl_enter();
     constexpr int TOKS = block_threads(TPT) / TPT;
+    constexpr int EPG = combine_granule(QIN);
     __shared__ int64_t s_row[TOKS][16];
     __shared__ float s_w[TOKS][16];
 
@@ -75,14 +138,14 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
     __syncthreads();
     if (!active) return;
 
-    const int ngran = a.H >> 3;
-#pragma unroll
+    const int ngran = a.H / EPG;
+#pragma unroll (QIN == QIN_BF16 ? GMAX : 1)
     for (int i = 0; i < GMAX; i++) {
         const int g = i * TPT + lt;
         if (g >= ngran) break;
-        float acc[8];
+        float acc[EPG];
 #pragma unroll
-        for (int q = 0; q < 8; q++) acc[q] = 0.0f;
+        for (int q = 0; q < EPG; q++) acc[q] = 0.0f;
         for (int k0 = 0; k0 < a.K; k0 += KB) {
             if constexpr (QIN == QIN_BF16) {
                 uint4 buf[KB];
@@ -106,67 +169,43 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
                     }
                 }
             } else {
-                // quantised rows: the codes of the granule (8 bytes, 4 for e2m1)
-                // and their scale, loaded for all KB entries before any use
+                // quantised rows: 16 bytes of codes and their scale per entry,
+                // loaded for all KB entries before any use
                 const uint8_t *ybase = reinterpret_cast<const uint8_t *>(a.y);
-                uint2 raw[KB];
+                uint4 raw[KB];
                 float sc[KB];
 #pragma unroll
                 for (int kk = 0; kk < KB; kk++) {
                     const int k = k0 + kk;
                     const int64_t row = k < a.K ? s_row[grp][k] : -1;
-                    raw[kk] = make_uint2(0u, 0u);
+                    raw[kk] = make_uint4(0u, 0u, 0u, 0u);
                     sc[kk] = 0.0f;
                     if (row >= 0) {
-                        const uint8_t *d = ybase + row * a.D;
                         const uint8_t *sp = ybase + a.scale_off + row * a.S;
-                        if constexpr (QIN == QIN_MXFP4)
-                            raw[kk].x = __ldcs(reinterpret_cast<const unsigned int *>(d + (int64_t)g * 4));
-                        else
-                            raw[kk] = __ldcs(reinterpret_cast<const uint2 *>(d + (int64_t)g * 8));
+                        raw[kk] = ld_stream(ybase + row * a.D + (int64_t)g * 16);
                         if constexpr (QIN == QIN_INT8) sc[kk] = __ldg(reinterpret_cast<const float *>(sp));
-                        if constexpr (QIN == QIN_E4M3_B128)
-                            sc[kk] = __ldg(reinterpret_cast<const float *>(sp) + (g >> 4));
-                        if constexpr (QIN == QIN_MXFP8 || QIN == QIN_MXFP4)
-                            sc[kk] = exp2_neg(127 - (int)__ldg(sp + (g >> 2)));
+                        if constexpr (QIN == QIN_E4M3_B128)  // 128 elements a scale
+                            sc[kk] = a.sfmt == 2 ? exp2_neg(127 - (int)__ldg(sp + (g >> 3)))
+                                                 : __ldg(reinterpret_cast<const float *>(sp) + (g >> 3));
+                        if constexpr (QIN == QIN_MXFP8)  // 32 elements a scale
+                            sc[kk] = exp2_neg(127 - (int)__ldg(sp + (g >> 1)));
+                        if constexpr (QIN == QIN_MXFP4)
+                            sc[kk] = exp2_neg(127 - (int)__ldg(sp + g));
                     }
                 }
 #pragma unroll
                 for (int kk = 0; kk < KB; kk++) {
                     const int k = k0 + kk;
                     if (k >= a.K || s_row[grp][k] < 0) continue;
-                    const float w = s_w[grp][k];
-                    float v[8];
-                    if constexpr (QIN == QIN_INT8) {
-#pragma unroll
-                        for (int q = 0; q < 8; q++) {
-                            const uint32_t word = q < 4 ? raw[kk].x : raw[kk].y;
-                            v[q] = __fmul_rn((float)(int8_t)((word >> (8 * (q & 3))) & 0xFFu), sc[kk]);
-                        }
-                    } else if constexpr (QIN == QIN_MXFP4) {
-#pragma unroll
-                        for (int q = 0; q < 4; q++) {
-                            const float2 f = e2m1x2_to_f32(raw[kk].x >> (8 * q));
-                            v[2 * q] = __fmul_rn(f.x, sc[kk]);
-                            v[2 * q + 1] = __fmul_rn(f.y, sc[kk]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 4; q++) {
-                            const uint32_t word = q < 2 ? raw[kk].x : raw[kk].y;
-                            const float2 f = e4m3x2_to_f32(word >> (16 * (q & 1)));
-                            v[2 * q] = __fmul_rn(f.x, sc[kk]);
-                            v[2 * q + 1] = __fmul_rn(f.y, sc[kk]);
-                        }
-                    }
-#pragma unroll
-                    for (int q = 0; q < 8; q++) acc[q] = __fmaf_rn(w, v[q], acc[q]);
+                    dequant_fma<QIN>(acc, raw[kk], sc[kk], s_w[grp][k]);
                 }
             }
         }
-        st_v4(a.out + n * a.H + (int64_t)g * 8,
-              make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                         pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7])));
+        uint16_t *o = a.out + n * a.H + (int64_t)g * EPG;
+#pragma unroll
+        for (int q = 0; q < EPG; q += 8)
+            st_v4(o + q, make_uint4(pack_bf16x2(acc[q], acc[q + 1]), pack_bf16x2(acc[q + 2], acc[q + 3]),
+                                    pack_bf16x2(acc[q + 4], acc[q + 5]), pack_bf16x2(acc[q + 6], acc[q + 7])));
     }
 }
 

@@ -17,6 +17,17 @@ namespace ep {
 
 constexpr uint32_t kFull = 0xFFFFFFFFu;
 
+// topk_idx as stored by the caller: int64 ("Low-Latency Mode API", topk_idx)
+// or int32 ("DeepEP topk_idx_t Custom Dtype Requirements": the index type
+// built with 32 bits).  One uniform branch per load.
+struct TopkIdx {
+    const void *p;
+    int i32;
+    __device__ __forceinline__ int64_t operator[](int64_t i) const {
+        return i32 ? (int64_t)static_cast<const int32_t *>(p)[i] : static_cast<const int64_t *>(p)[i];
+    }
+};
+
 // Threads of a block whose token groups have TPT threads: one token per block
 // from TPT = 128 up, 128 threads otherwise.  Small blocks spread the tokens of
 // a grid that fits in one wave evenly over the SMs (a block of two 128-thread
@@ -77,6 +88,37 @@ __device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t two_codes) {
         : "=r"(h2)
         : "r"(two_codes & 0xFFu));
     return __half22float2(*reinterpret_cast<__half2 *>(&h2));
+}
+
+// ---- exact decoding with integer operations -------------------------------------
+// The conversions above issue at a fraction of the FMA rate.  These place a
+// code's sign and magnitude bits in an fp32 word whose exponent bias is 127
+// instead of the format's: read back, that word is the code's value times
+// 2^-(127 - bias) exactly (a zero or subnormal code gives an fp32 zero or
+// subnormal), so one exact power-of-two factor restores the value:
+// 2^120 for e4m3 (bias 7), 2^126 for e2m1 (bias 1).  The e4m3 NaN codes
+// (low seven bits all set) do not decode this way; e4m3_has_nan finds them.
+// (j is a constant once the callers' loops are unrolled)
+__device__ __forceinline__ float e4m3_rebiased(uint32_t w, int j) {  // byte j of w
+    const uint32_t top = __byte_perm(w, 0u, (j << 12) | 0x444);  // the code in bits 24..31
+    return __uint_as_float((uint32_t)((int32_t)top >> 4) & 0x87FFFFFFu);
+}
+// nibble j of w: element 2i is the low nibble of byte i
+__device__ __forceinline__ float e2m1_rebiased(uint32_t w, int j) {
+    uint32_t top = __byte_perm(w, 0u, ((j >> 1) << 12) | 0x444);  // byte in bits 24..31
+    if ((j & 1) == 0) top <<= 4;                                    // the nibble in 28..31
+    return __uint_as_float((uint32_t)((int32_t)top >> 6) & 0x81C00000u);
+}
+// Any of the 16 e4m3 codes a NaN code?
+__device__ __forceinline__ bool e4m3_has_nan(const uint32_t (&u)[4]) {
+    uint32_t t = 0u;
+#pragma unroll
+    for (int q = 0; q < 4; q++) t |= (u[q] & 0x7F7F7F7Fu) + 0x01010101u;  // no carry between bytes
+    return (t & 0x80808080u) != 0u;
+}
+// int8 byte j of wx = w ^ 0x80808080: the fp32 2^23 + 128 + b, less 2^23 + 128 (both exact).
+__device__ __forceinline__ float i8_exact(uint32_t wx, int j) {
+    return __uint_as_float(__byte_perm(wx, 0x4B000000u, 0x7440 | j)) - 8388736.0f;
 }
 
 // ---- scales ------------------------------------------------------------------

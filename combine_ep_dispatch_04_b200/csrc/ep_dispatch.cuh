@@ -32,10 +32,11 @@ struct DispatchArgs {
     int64_t cap, rows;       // padded rows per expert, buffer row capacity
     int64_t D, S, scale_off; // row data bytes, row scale bytes, scale region offset
     float qmax;              // e4m3_b128 target max
+    int sfmt;                // e4m3_b128 scales: 0 qmax/amax, 1 power of two, 2 e8m0 bytes
     int unweighted;          // combine backward only
     int early;               // load and quantise x before waiting for the previous grid
     const uint16_t *x;       // [N][H] bf16 (the gradient g for the backward)
-    const int64_t *idx;
+    TopkIdx idx;
     const float *wts;
     const int32_t *slot;
     const int64_t *eo;
@@ -187,9 +188,16 @@ __global__ void __launch_bounds__(block_threads(TPT)) dispatch_kernel(DispatchAr
             m = fmaxf(m, __shfl_xor_sync(kFull, m, 4));
             bs[i] = 1.0f;
             bsinv[i] = 1.0f;
-            if (m != 0.0f) {
-                bs[i] = fminf(__fdiv_rn(a.qmax, m), FLT_MAX);
-                bsinv[i] = __fdiv_rn(m, a.qmax);
+            if (a.sfmt == 0) {
+                if (m != 0.0f) {
+                    bs[i] = fminf(__fdiv_rn(a.qmax, m), FLT_MAX);
+                    bsinv[i] = __fdiv_rn(m, a.qmax);
+                }
+            } else {  // round_scale: the block's power of two by the MX rule
+                const int X = a.qmax == 448.0f ? mx_exponent_fast<448>(m) : mx_exponent(m, a.qmax);
+                bs[i] = exp2_neg(X);
+                bsinv[i] = exp2_neg(-X);
+                bx[i] = (uint32_t)(X + 127);
             }
         }
     }
@@ -278,7 +286,15 @@ __global__ void __launch_bounds__(block_threads(TPT)) dispatch_kernel(DispatchAr
                 st_v2(p, make_uint2(c[i][0], c[i][1]));
             }
             if constexpr (MODE == Q_E4M3_B128) {
-                if ((g & 7) == 0) reinterpret_cast<float *>(sdst)[g >> 3] = bsinv[i];
+                if ((g & 7) == 0) {
+                    if (a.sfmt == 2) {  // e8m0 bytes, the row padded to whole int32 words with 0
+                        sdst[g >> 3] = (uint8_t)bx[i];
+                        if ((g >> 3) == (a.H >> 7) - 1)
+                            for (int j = a.H >> 7; j < a.S; j++) sdst[j] = 0;
+                    } else {
+                        reinterpret_cast<float *>(sdst)[g >> 3] = bsinv[i];
+                    }
+                }
             }
             if constexpr (MODE == Q_MXFP8 || MODE == Q_MXFP4) {
                 if ((g & 1) == 0) sdst[g >> 1] = (uint8_t)bx[i];

@@ -43,7 +43,7 @@ struct LayoutArgs {
     int TC, CR, C;  // tokens per chunk, chunks per rank, chunks
     int packed, align;
     int64_t cap;    // padded rows per expert (R*M)
-    const int64_t *idx;
+    TopkIdx idx;
     int32_t *tpr, *tpe;
     uint8_t *itr;
     int32_t *slot;
@@ -59,9 +59,9 @@ constexpr int kMaxTopk = 16;
 // ---- shared helpers ------------------------------------------------------------
 
 // keys[i] = expert of entry f0+i, or -1 when masked or out of range; returns
-// true if a value outside [-1, E) was seen.  Coalesced int64 loads, 8 in
-// flight per thread.
-__device__ __forceinline__ bool stage_keys(const int64_t *idx, int64_t f0, int nent, int E,
+// true if a value outside [-1, E) was seen.  Coalesced loads, 8 in flight per
+// thread.
+__device__ __forceinline__ bool stage_keys(TopkIdx idx, int64_t f0, int nent, int E,
                                            int *keys) {
     constexpr int U = 8;
     bool bad = false;

@@ -26,6 +26,9 @@ DEV_BAD_INDEX = 0x1
 DEV_CAPACITY_OVERFLOW = 0x2
 F_BWD_UNWEIGHTED = 0x1
 F_COMBINE_QUANTIZED = 0x2
+F_IDX_I32 = 0x4
+F_ROUND_SCALE = 0x8
+F_UE8M0 = 0x10
 F_LAYOUT_SINGLE_CTA = 0x100
 F_LAYOUT_MULTI_CTA = 0x200
 F_LAYOUT_CLUSTER = 0x400
@@ -164,6 +167,11 @@ def _nk(cfg):
     return cfg.num_ranks * cfg.num_tokens, cfg.num_topk
 
 
+def idx_dtype(cfg):
+    """dtype of topk_idx for this configuration: int64, or int32 with F_IDX_I32."""
+    return torch.int32 if cfg.flags & F_IDX_I32 else torch.int64
+
+
 def ep_dispatch_layout(cfg, topk_idx, token_slot, recv_count, workspace, dev_status,
                        tokens_per_rank=None, tokens_per_expert=None, is_token_in_rank=None,
                        expert_offset=None, cumulative_recv_stats=None, stream=None, bind=False):
@@ -171,7 +179,7 @@ def ep_dispatch_layout(cfg, topk_idx, token_slot, recv_count, workspace, dev_sta
     R, E = cfg.num_ranks, cfg.num_experts
     sz = ep_buffer_sizes(cfg)
     args = [
-        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
         _dev(tokens_per_rank, "tokens_per_rank", torch.int32, (R, R), optional=True),
         _dev(tokens_per_expert, "tokens_per_expert", torch.int32, (R, E), optional=True),
         _dev(is_token_in_rank, "is_token_in_rank", torch.uint8, (N, R), optional=True),
@@ -197,7 +205,7 @@ def ep_dispatch_layout_static(cfg, topk_idx, token_slot, recv_count, dev_status,
     N, K = _nk(cfg)
     R, E = cfg.num_ranks, cfg.num_experts
     args = [
-        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
         _dev(tokens_per_rank, "tokens_per_rank", torch.int32, (R, R), optional=True),
         _dev(tokens_per_expert, "tokens_per_expert", torch.int32, (R, E), optional=True),
         _dev(is_token_in_rank, "is_token_in_rank", torch.uint8, (N, R), optional=True),
@@ -218,7 +226,7 @@ def ep_dispatch(cfg, x, topk_idx, token_slot, recv_buf, src_info, dev_status, to
     sz = ep_buffer_sizes(cfg)
     args = [
         _dev(x, "x", torch.bfloat16, (N, cfg.hidden)),
-        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
         _dev(topk_weights, "topk_weights", torch.float32, (N, K), optional=True),
         _dev(token_slot, "token_slot", torch.int32, (N, K)),
         _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
@@ -244,7 +252,7 @@ def ep_dispatch_with_layout(cfg, x, topk_idx, token_slot, recv_count, workspace,
     sz = ep_buffer_sizes(cfg)
     args = [
         _dev(x, "x", torch.bfloat16, (N, cfg.hidden)),
-        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
         _dev(topk_weights, "topk_weights", torch.float32, (N, K), optional=True),
         _dev(tokens_per_rank, "tokens_per_rank", torch.int32, (R, R), optional=True),
         _dev(tokens_per_expert, "tokens_per_expert", torch.int32, (R, E), optional=True),
@@ -273,7 +281,7 @@ def ep_combine(cfg, y, topk_idx, topk_weights, token_slot, out, dev_status, expe
         raise TypeError("y (expert outputs) must be bfloat16 unless F_COMBINE_QUANTIZED")
     args = [
         _bytes(y, "y", sz["recv_bytes"] if quantized else sz["expert_out_bytes"]),
-        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
         _dev(topk_weights, "topk_weights", torch.float32, (N, K)),
         _dev(token_slot, "token_slot", torch.int32, (N, K)),
         _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
@@ -291,7 +299,7 @@ def ep_combine_backward(cfg, g, topk_idx, topk_weights, token_slot, grad_buf, de
     sz = ep_buffer_sizes(cfg)
     args = [
         _dev(g, "g", torch.bfloat16, (N, cfg.hidden)),
-        _dev(topk_idx, "topk_idx", torch.int64, (N, K)),
+        _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
         _dev(topk_weights, "topk_weights", torch.float32, (N, K),
              optional=bool(cfg.flags & F_BWD_UNWEIGHTED)),
         _dev(token_slot, "token_slot", torch.int32, (N, K)),

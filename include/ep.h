@@ -83,10 +83,33 @@ typedef enum {
 /* ep_config_t.flags */
 #define EP_F_BWD_UNWEIGHTED 0x1u    /* combine-backward re-dispatches g without w */
 #define EP_F_COMBINE_QUANTIZED 0x2u /* ep_combine's y is in cfg->quant's format (recv_buf layout) */
+#define EP_F_IDX_I32 0x4u           /* topk_idx is int32 [N][K] instead of int64 ([IDX]) */
+#define EP_F_ROUND_SCALE 0x8u       /* E4M3_B128: power-of-two scales ([LL] round_scale) */
+#define EP_F_UE8M0 0x10u            /* E4M3_B128: the power-of-two scales as e8m0 bytes */
 #define EP_F_LAYOUT_SINGLE_CTA 0x100u /* force the one-block layout path */
 #define EP_F_LAYOUT_MULTI_CTA 0x200u  /* force the multi-block layout path */
 #define EP_F_LAYOUT_CLUSTER 0x400u    /* force the thread-block-cluster layout path */
 
+/*
+ * Flags on the formats:
+ *   EP_F_IDX_I32      every topk_idx argument is int32 [N][K] ([IDX]: the
+ *                     index type may be built with 32 or 64 bits); values
+ *                     have the same meaning.
+ *   EP_F_ROUND_SCALE  E4M3_B128 ([LL] round_scale; [FP8] Advanced Configuration
+ *                     Options, Round-Scale Mode): each 128-block's scale is the
+ *                     smallest power of two 2^X with amax/qmax <= 2^X (amax 0:
+ *                     X = 0; X clamped to [-127, 127]), codes = e4m3(x * 2^-X),
+ *                     stored scale_inv = 2^X (fp32).  The pages ask for
+ *                     power-of-two scales without fixing the rounding; rounding
+ *                     up keeps every element within qmax.  Allowed and without
+ *                     effect for MXFP8 / MXFP4 (their scales are powers of two);
+ *                     invalid for BF16 and INT8_TOKEN.
+ *   EP_F_UE8M0        E4M3_B128 only, implies EP_F_ROUND_SCALE ([FP8] Advanced
+ *                     Configuration Options, UE8M0 Support: 8-bit scales in a
+ *                     packed format): the scale of block j is the e8m0 byte
+ *                     X + 127 at byte j of the row's scales, four to an int32;
+ *                     S = 4 * ceil(H/128 / 4) bytes, pad bytes written as 0.
+ */
 typedef struct {
     int32_t num_ranks;           /* R > 0 */
     int32_t num_tokens;          /* T tokens per rank, 0 <= T <= M */
@@ -107,7 +130,7 @@ typedef struct {
 typedef struct {
     int64_t rows;
     int64_t data_row_bytes;     /* D: 2H bf16, H int8/e4m3, H/2 e2m1 */
-    int64_t scale_row_bytes;    /* S: 0 bf16, 4 int8, 4*H/128 e4m3_b128, H/32 mx */
+    int64_t scale_row_bytes;    /* S: 0 bf16, 4 int8, 4*H/128 e4m3_b128 (UE8M0: above), H/32 mx */
     int64_t recv_scale_offset;  /* recv_buf: data region [rows][D] then, here, scales [rows][S] */
     int64_t recv_bytes;
     int64_t src_info_bytes;     /* int32 [rows] */
@@ -127,7 +150,7 @@ ep_status_t ep_buffer_sizes(const ep_config_t *cfg, ep_sizes_t *out);
  * Routing layout and slot assignment ([LL] low_latency_dispatch: topk_idx
  * [num_tokens, num_topk] int64, -1 = no expert; recv_count [num_local_experts]
  * int64; cumulative_local_expert_recv_stats).
- *   topk_idx            int64 [N][K], N = R*T
+ *   topk_idx            int64 [N][K], N = R*T (int32 with EP_F_IDX_I32)
  *   tokens_per_rank     int32 [R][R]: tokens of src r with >= 1 expert on rank d (nullable)
  *   tokens_per_expert   int32 [R][E]: entries of src r routed to e (nullable)
  *   is_token_in_rank    uint8 [N][R]: 1 if token n has an expert on rank d (nullable)
@@ -140,7 +163,7 @@ ep_status_t ep_buffer_sizes(const ep_config_t *cfg, ep_sizes_t *out);
  *   workspace           ep_sizes_t.workspace_bytes of scratch (contents undefined after)
  * Deterministic: the result never depends on thread timing.
  */
-ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const int64_t *topk_idx,
+ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const void *topk_idx,
                                int32_t *tokens_per_rank, int32_t *tokens_per_expert,
                                uint8_t *is_token_in_rank, int32_t *token_slot,
                                int64_t *recv_count, int64_t *expert_offset,
@@ -152,7 +175,8 @@ ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const int64_t *topk_idx,
  * ([LL] low_latency_dispatch Return Values; [FP8] The Dispatch Stage; [TE]
  * Changes: data region then scale region in one caller buffer).
  *   x              bf16 [N][H]
- *   topk_idx       int64 [N][K]; token_slot/expert_offset from ep_dispatch_layout
+ *   topk_idx       int64 [N][K] (int32 with EP_F_IDX_I32); token_slot /
+ *                  expert_offset from ep_dispatch_layout
  *   topk_weights   float [N][K] (nullable; needed for recv_weights)
  *   recv_buf       ep_sizes_t.recv_bytes: row (e, slot) holds the token's
  *                  quantised row; padded row = e*R*M + slot, packed row =
@@ -160,7 +184,7 @@ ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const int64_t *topk_idx,
  *   src_info       int32 [rows]: r*M + t of the row's source token
  *   recv_weights   float [rows] (nullable): the entry's top-k weight
  */
-ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const int64_t *topk_idx,
+ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
                         const float *topk_weights, const int32_t *token_slot,
                         const int64_t *expert_offset, void *recv_buf, int32_t *src_info,
                         float *recv_weights, uint32_t *dev_status, ep_stream_t stream);
@@ -174,7 +198,7 @@ ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const int64_t
  * before reading token_slot / expert_offset.
  */
 ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
-                                    const int64_t *topk_idx, const float *topk_weights,
+                                    const void *topk_idx, const float *topk_weights,
                                     int32_t *tokens_per_rank, int32_t *tokens_per_expert,
                                     uint8_t *is_token_in_rank, int32_t *token_slot,
                                     int64_t *recv_count, int64_t *expert_offset,
@@ -198,7 +222,7 @@ ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
  *          in fp32).  An e8m0 scale byte of 255 (NaN) is not a valid input.
  *   out    bf16 [N][H]
  */
-ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t *topk_idx,
+ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const void *topk_idx,
                        const float *topk_weights, const int32_t *token_slot,
                        const int64_t *expert_offset, uint16_t *out, uint32_t *dev_status,
                        ep_stream_t stream);
@@ -213,7 +237,7 @@ ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const int64_t 
  *   grad_buf   ep_sizes_t.grad_bytes: e4m3 [rows][H] then e8m0 [rows][H/32]
  */
 ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
-                                const int64_t *topk_idx, const float *topk_weights,
+                                const void *topk_idx, const float *topk_weights,
                                 const int32_t *token_slot, const int64_t *expert_offset,
                                 void *grad_buf, uint32_t *dev_status, ep_stream_t stream);
 
@@ -241,7 +265,7 @@ ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
  */
 #define EP_STATIC_SCRATCH_BYTES (1u << 20)
-ep_status_t ep_dispatch_layout_static(const ep_config_t *cfg, const int64_t *topk_idx,
+ep_status_t ep_dispatch_layout_static(const ep_config_t *cfg, const void *topk_idx,
                                       int32_t *tokens_per_rank, int32_t *tokens_per_expert,
                                       uint8_t *is_token_in_rank, int32_t *token_slot,
                                       int64_t *recv_count, int64_t *expert_offset,

@@ -20,6 +20,15 @@ def to_np_u16(t):
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+def oracle_mode(mode, flags):
+    """The oracle's name for a quantisation mode with its scale flags."""
+    if mode == "e4m3_b128" and flags & ep.F_UE8M0:
+        return "e4m3_b128_ue8m0"
+    if mode == "e4m3_b128" and flags & ep.F_ROUND_SCALE:
+        return "e4m3_b128_p2"
+    return mode
+
+
 class Run:
     """One pass of layout -> dispatch -> combine (-> combine backward) on the GPU."""
 
@@ -33,11 +42,14 @@ class Run:
             idx = i2 if idx is None else idx
             wts = w2 if wts is None else wts
         self.idx = np.ascontiguousarray(idx, np.int64)
+        if flags & ep.F_IDX_I32:  # the values the device sees
+            self.idx = self.idx.astype(np.int32).astype(np.int64)
         self.wts = np.ascontiguousarray(wts, np.float32)
         self.x = synth.make_x(w, replica) if x is None else np.ascontiguousarray(x, np.uint16)
         self.cfg = ep.make_config(R, T, M, K, E, H, mode, layout, align, qmax,
                                   flags | (ep.F_BWD_UNWEIGHTED if bwd_unweighted else 0))
         self.bwd_unweighted = bwd_unweighted
+        self.omode = oracle_mode(mode, flags)
         b = ep.Buffers(self.cfg, recv_weights=with_weights, grad=backward)
         self.b = b
         b.recv_buf.fill_(fill)
@@ -46,7 +58,7 @@ class Run:
         b.src_info.fill_(-7)
         self.sizes = b.sizes
         N = R * T
-        self.idx_d = torch.from_numpy(self.idx).cuda()
+        self.idx_d = torch.from_numpy(self.idx).cuda().to(ep.idx_dtype(self.cfg))
         self.wts_d = torch.from_numpy(self.wts).cuda()
         self.x_d = bf16_dev(self.x)
         self.stats_d = torch.zeros(E, dtype=torch.int64, device="cuda") if stats else None
@@ -117,7 +129,7 @@ class Run:
         expect_cache = {}
         for i, (n, k, row) in enumerate(zip(ns, ks, rows)):
             if n not in expect_cache:
-                expect_cache[n] = oracle.quant_row(self.mode, self.x[n], e4m3_qmax=self.qmax)
+                expect_cache[n] = oracle.quant_row(self.omode, self.x[n], e4m3_qmax=self.qmax)
             d, s = expect_cache[n]
             assert np.array_equal(data[i], d), f"data row {row} (token {n}, k {k})"
             if S:
@@ -187,26 +199,46 @@ def quantized_rows(mode, H, nrows, seed):
     r = np.random.default_rng(seed)
     D, S = oracle.row_bytes(mode, H)
     data = r.integers(0, 256, (nrows, D), dtype=np.uint8)
-    if mode in ("e4m3_b128", "mxfp8"):
+    if mode.startswith("e4m3") or mode == "mxfp8":
         data[(data & 0x7F) == 0x7F] ^= 0x01          # 0x7F / 0xFF are NaN in e4m3
     if mode == "int8_token":
         scale = (r.random((nrows, 1)) * 0.05 + 1e-3).astype(np.float32).view(np.uint8)
     elif mode == "e4m3_b128":
         scale = (r.random((nrows, S // 4)) * 0.02 + 1e-4).astype(np.float32).view(np.uint8)
+    elif mode == "e4m3_b128_p2":
+        scale = np.ldexp(1.0, r.integers(-20, 5, (nrows, S // 4))).astype(np.float32).view(np.uint8)
     else:
         scale = r.integers(112, 140, (nrows, S), dtype=np.uint8)
     return data, scale.reshape(nrows, S)
 
 
-def combine_quantized_check(run, tokens=None, seed=0):
-    """Combine of quantised expert outputs on the GPU against the oracle."""
+def special_quantized_rows(mode, H, nrows, seed):
+    """Quantised rows with the values a decoder can get wrong: every code
+    (NaN codes included), and scales that are zero, subnormal, huge, infinite,
+    NaN or negative (fp32 scales), or every e8m0 byte from 0 to 255."""
+    r = np.random.default_rng(seed)
+    D, S = oracle.row_bytes(mode, H)
+    data = r.integers(0, 256, (nrows, D), dtype=np.uint8)
+    if mode in ("int8_token", "e4m3_b128", "e4m3_b128_p2"):
+        pick = np.array([0.0, 1e-45, 1e-40, 3e-39, 1e-3, 0.5, 1.0, 200.0, 255.9, 256.0, 1e30,
+                         3e38, np.inf, np.nan, -0.75, -np.inf], np.float32)
+        scale = pick[r.integers(0, len(pick), (nrows, S // 4))].view(np.uint8)
+    else:
+        scale = r.integers(0, 256, (nrows, S), dtype=np.uint8)
+        scale[:, 0] = np.arange(nrows) % 256
+    return data, scale.reshape(nrows, S)
+
+
+def combine_quantized_check(run, tokens=None, seed=0, rows_fn=None):
+    """Combine of quantised expert outputs on the GPU against the oracle:
+    within 1 bf16 ulp, and NaN exactly where the oracle gives NaN."""
     w, b = run.w, run.b
     K, H = w["K"], w["H"]
-    mode = run.mode
-    cfg = ep.make_config(w["R"], w["T"], w["M"], K, w["E"], H, mode, run.layout, run.align,
+    mode = run.omode
+    cfg = ep.make_config(w["R"], w["T"], w["M"], K, w["E"], H, run.mode, run.layout, run.align,
                          run.qmax, run.cfg.flags | ep.F_COMBINE_QUANTIZED)
     ns, ks, rows = run.entries(None)
-    data, scale = quantized_rows(mode, H, len(rows), seed)
+    data, scale = (rows_fn or quantized_rows)(mode, H, len(rows), seed)
     sz = run.sizes
     yq = torch.zeros(sz["recv_bytes"], dtype=torch.uint8, device="cuda")
     D, S = sz["data_row_bytes"], sz["scale_row_bytes"]
@@ -231,6 +263,9 @@ def combine_quantized_check(run, tokens=None, seed=0):
             if i is not None:
                 qd[j, k], qs[j, k], valid[j, k] = data[i], scale[i], 1
     want = oracle.combine_gathered_q(mode, qd, qs, run.wts[tokens], valid, H)
-    d = ulp_distance(got, want)
+    nan_g = (got & 0x7FFF) > 0x7F80
+    nan_w = (want & 0x7FFF) > 0x7F80
+    assert np.array_equal(nan_g, nan_w), int((nan_g != nan_w).sum())
+    d = np.where(nan_w, 0, ulp_distance(got, want))
     assert d.max() <= 1, int(d.max())
     return int(d.max())

@@ -68,11 +68,37 @@ def test_sizes_packed_every_mode(quant, D, S):
     dict(flags=ep.F_LAYOUT_CLUSTER | ep.F_LAYOUT_SINGLE_CTA),
     dict(flags=ep.F_LAYOUT_CLUSTER | ep.F_LAYOUT_MULTI_CTA),
     dict(quant="e4m3_b128", H=96),
+    dict(quant="bf16", flags=ep.F_ROUND_SCALE), dict(quant="int8_token", flags=ep.F_ROUND_SCALE),
+    dict(quant="mxfp8", flags=ep.F_UE8M0), dict(quant="int8_token", flags=ep.F_UE8M0),
+    dict(quant="bf16", flags=ep.F_UE8M0 | ep.F_ROUND_SCALE),
 ])
 def test_invalid_configs_rejected(bad):
     with pytest.raises(ep.EpError) as ei:
         ep.ep_buffer_sizes(_cfg(**bad))
     assert ei.value.status == 1
+
+
+@pytest.mark.parametrize("H,flags,S", [
+    (7168, 0, 224), (7168, ep.F_ROUND_SCALE, 224), (7168, ep.F_UE8M0, 56),
+    (7168, ep.F_UE8M0 | ep.F_ROUND_SCALE, 56), (384, ep.F_UE8M0, 4), (640, ep.F_UE8M0, 8),
+])
+def test_sizes_e4m3_scale_options(H, flags, S):
+    s = ep.ep_buffer_sizes(_cfg(H=H, flags=flags))
+    assert s["scale_row_bytes"] == S and s["data_row_bytes"] == H
+    assert s["recv_bytes"] == s["recv_scale_offset"] + s["rows"] * S
+
+
+@pytest.mark.parametrize("quant", ["mxfp8", "mxfp4"])
+def test_round_scale_accepted_for_mx(quant):
+    a = ep.ep_buffer_sizes(_cfg(H=1024, quant=quant))
+    b = ep.ep_buffer_sizes(_cfg(H=1024, quant=quant, flags=ep.F_ROUND_SCALE))
+    assert a == b
+
+
+def test_index_dtype_follows_the_flag():
+    import torch
+    assert ep.idx_dtype(_cfg()) == torch.int64
+    assert ep.idx_dtype(_cfg(flags=ep.F_IDX_I32)) == torch.int32
 
 
 def test_entry_points_reject_before_any_launch():

@@ -325,3 +325,113 @@ def test_combine_of_quantized_expert_outputs(mode, name, override):
     from harness import combine_quantized_check
     r = Run(w, mode, layout=w["layout"])
     combine_quantized_check(r, seed=31 * len(mode) + len(name))
+
+
+@pytest.mark.parametrize("mode", ["int8_token", "e4m3_b128", "mxfp8", "mxfp4"])
+def test_combine_of_quantized_special_values(mode):
+    """NaN codes, zero / subnormal / huge / infinite / NaN / negative scales,
+    and every e8m0 byte: the decoder's exact fast path and its fallback."""
+    from harness import combine_quantized_check, special_quantized_rows
+    w = synth.workload("decode", T=24)
+    r = Run(w, mode, layout="packed")
+    combine_quantized_check(r, seed=7 + len(mode), rows_fn=special_quantized_rows)
+
+
+# ---------------------------------------------------------------------------
+# int32 topk_idx, and the E4M3-per-128 scale options (round_scale, UE8M0)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("mode", ["bf16", "e4m3_b128", "mxfp4"])
+@pytest.mark.parametrize("path", [ep.F_LAYOUT_SINGLE_CTA, ep.F_LAYOUT_MULTI_CTA,
+                                  ep.F_LAYOUT_CLUSTER])
+def test_int32_topk_idx(mode, path):
+    w = _edge(R=4, T=37, M=40, K=5, E=8, H=384)
+    idx, wts = synth.make_routing(w)
+    idx[::3, 1] = idx[::3, 0]          # duplicates
+    idx[5, 2] = w["E"] + 3             # out of range
+    idx[7, 0] = -9
+    idx[9, 1] = -(1 << 31)
+    r = Run(w, mode, layout="packed", align=2, idx=idx, wts=wts, flags=path | ep.F_IDX_I32,
+            backward=True, stats=True)
+    assert r.idx_d.dtype == torch.int32
+    assert r.status & ep.DEV_BAD_INDEX
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+    r.check_backward()
+
+
+def test_int32_topk_idx_decode_and_one_call_dispatch():
+    w = synth.workload("decode")
+    r = Run(w, "e4m3_b128", flags=ep.F_IDX_I32)
+    r.check_layout()
+    r.check_dispatch(check_unwritten=False)
+    r.check_combine()
+    b = ep.Buffers(r.cfg)
+    ep.ep_dispatch_with_layout(r.cfg, r.x_d, r.idx_d, b.token_slot, b.recv_count, b.workspace,
+                               b.recv_buf, b.src_info, b.dev_status)
+    assert torch.equal(b.token_slot, r.b.token_slot)
+    ns, ks, rows = r.entries()
+    rows_d = torch.from_numpy(rows).cuda()
+    assert torch.equal(b.recv_data().index_select(0, rows_d), r.b.recv_data().index_select(0, rows_d))
+    assert torch.equal(b.recv_scale().index_select(0, rows_d), r.b.recv_scale().index_select(0, rows_d))
+
+
+def test_int64_index_rejected_when_int32_expected():
+    w = _edge()
+    cfg = ep.make_config(w["R"], w["T"], w["M"], w["K"], w["E"], w["H"], "bf16",
+                         flags=ep.F_IDX_I32)
+    b = ep.Buffers(cfg)
+    idx64 = torch.zeros((w["N"], w["K"]), dtype=torch.int64, device="cuda")
+    with pytest.raises(TypeError):
+        ep.ep_dispatch_layout(cfg, idx64, b.token_slot, b.recv_count, b.workspace, b.dev_status)
+
+
+@pytest.mark.parametrize("flags", [ep.F_ROUND_SCALE, ep.F_UE8M0, ep.F_ROUND_SCALE | ep.F_UE8M0])
+@pytest.mark.parametrize("qmax", [0.0, 240.0])
+@pytest.mark.parametrize("H", [384, 7168])
+def test_e4m3_round_scale_and_ue8m0(flags, qmax, H):
+    w = _edge(R=3, T=13, M=16, K=4, E=12, H=H)
+    r = Run(w, "e4m3_b128", layout="packed", qmax=qmax, flags=flags)
+    assert r.sizes["scale_row_bytes"] == (4 * ((H // 128 + 3) // 4) if flags & ep.F_UE8M0
+                                          else 4 * (H // 128))
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+
+
+def test_e4m3_round_scale_extreme_magnitudes():
+    w = _edge(H=512)
+    x = synth.make_x(w)
+    f = oracle.bf16_to_f32(x).copy()
+    f[0] *= np.float32(2.0 ** -120)
+    f[1] *= np.float32(2.0 ** -126)
+    f[2] *= np.float32(2.0 ** 100)
+    f[3, ::7] *= 50
+    x = synth.to_bf16_bits(f)
+    x[4] = 0
+    x[5, :128] = 0x8000
+    for flags in (ep.F_ROUND_SCALE, ep.F_UE8M0):
+        for qmax in (0.0, 3.5):
+            r = Run(w, "e4m3_b128", layout="packed", x=x, qmax=qmax, flags=flags)
+            r.check_dispatch()
+
+
+def test_e4m3_ue8m0_decode_workload():
+    r = Run(synth.workload("decode"), "e4m3_b128", flags=ep.F_UE8M0)
+    r.check_dispatch(check_unwritten=False)
+
+
+@pytest.mark.parametrize("mode", ["mxfp8", "mxfp4"])
+def test_round_scale_changes_nothing_for_mx(mode):
+    w = _edge(R=3, T=13, M=16, K=4, E=12, H=640)
+    a = Run(w, mode, layout="packed")
+    b = Run(w, mode, layout="packed", flags=ep.F_ROUND_SCALE)
+    assert torch.equal(a.b.recv_buf, b.b.recv_buf)
+
+
+@pytest.mark.parametrize("flags", [ep.F_ROUND_SCALE, ep.F_UE8M0])
+def test_combine_of_quantized_round_scale_rows(flags):
+    from harness import combine_quantized_check, special_quantized_rows
+    r = Run(synth.workload("decode", T=24), "e4m3_b128", layout="packed", flags=flags)
+    combine_quantized_check(r, seed=3 + flags)
+    combine_quantized_check(r, seed=5 + flags, rows_fn=special_quantized_rows)
