@@ -596,9 +596,36 @@ ep::DispatchArgs full_dispatch_args(const ep_config_t *cfg, const Plan &p, const
     return a;
 }
 
+// Quantised expert outputs with K <= 8 and 4-byte aligned scale rows: the
+// kernel that keeps the next granule's copies in flight (blocks of 128).
+template <int QIN>
+ep_status_t launch_combine_pipelined(const ep::CombineArgs &a, cudaStream_t s) {
+    auto kernel_of = [](int t, int g) -> const void * {
+#define EP_FN(T_, G_)                                                                      \
+    if (T_ <= 128 && t == T_ && g == G_) return (const void *)ep::combine_q_kernel<(T_ <= 128 ? T_ : 128), G_, QIN>;
+        EP_SPLITS(EP_FN)
+#undef EP_FN
+        return nullptr;
+    };
+    const Split sp = split_rows(a.N, a.H / ep::combine_granule(QIN), 8, kernel_of);
+    const unsigned grid = grid_for(a.N, sp.tpt);
+#define EP_CASE(T_, G_)                                                                     \
+    if (T_ <= 128 && sp.tpt == T_ && sp.gmax == G_) {                                       \
+        launch(ep::combine_q_kernel<(T_ <= 128 ? T_ : 128), G_, QIN>, grid, ep::block_threads(T_), 0, s, a); \
+        return launched();                                                                  \
+    }
+    EP_SPLITS(EP_CASE)
+#undef EP_CASE
+    return EP_ERR_UNSUPPORTED;
+}
+
 // Granules of 16 bytes of expert output (combine_granule elements).
 template <int QIN>
 ep_status_t launch_combine(const ep::CombineArgs &a, cudaStream_t s) {
+    if constexpr (QIN != ep::QIN_BF16) {
+        if (a.K <= ep::kPipeRows && a.S % 4 == 0 && a.S <= ep::kPipeScaleBytes)
+            return launch_combine_pipelined<QIN>(a, s);
+    }
     auto kernel_of = [](int t, int g) -> const void * {
 #define EP_FN(T_, G_) if (t == T_ && g == G_) return (const void *)ep::combine_kernel<T_, G_, 8, QIN>;
         EP_SPLITS(EP_FN)

@@ -45,62 +45,75 @@ __host__ __device__ constexpr int combine_granule(int qin) {
 }
 
 // Quantised expert outputs ("DeepEP FP8 Dispatch and Combine Operations",
-// The FP8 Combine Operation): every code is decoded exactly and multiplied by
-// its row / block scale as one fp32 multiply, y = fl(decode(c) * s), before
-// the FMA.  The decode is done with integer operations (e4m3_rebiased and
-// the like), its power-of-two factor folded into the scale: fl(c' * (s*2^B))
-// is the same single rounding of the same real product.  Where s*2^B is not
-// finite, or an e4m3 code is NaN, the hardware conversions decode instead.
+// The FP8 Combine Operation): every code is decoded exactly (e4m3 / e2m1 by
+// the hardware conversions to f16 and then f32, which also turn the e4m3 NaN
+// codes into NaN; int8 through the 2^23 constant of i8_exact) and multiplied
+// by its row / block scale as one fp32 multiply, y = fl(decode(c) * s),
+// before the FMA.
 template <int QIN>
 __device__ __forceinline__ void dequant_fma(float (&acc)[combine_granule(QIN)], const uint4 &r,
                                             float s, float w) {
-    constexpr int EPG = combine_granule(QIN);
     const uint32_t u[4] = {r.x, r.y, r.z, r.w};
-    float v[EPG];
-    if constexpr (QIN == QIN_INT8) {
 #pragma unroll
-        for (int q = 0; q < 4; q++) {
+    for (int q = 0; q < 4; q++) {
+        if constexpr (QIN == QIN_INT8) {
             const uint32_t wx = u[q] ^ 0x80808080u;
 #pragma unroll
-            for (int j = 0; j < 4; j++) v[4 * q + j] = __fmul_rn(i8_exact(wx, j), s);
-        }
-    } else if constexpr (QIN == QIN_MXFP4) {
-        const float s1 = __fmul_rn(s, 0x1p126f);
-        if (fabsf(s1) <= FLT_MAX) {
+            for (int j = 0; j < 4; j++)
+                acc[4 * q + j] = __fmaf_rn(w, __fmul_rn(i8_exact(wx, j), s), acc[4 * q + j]);
+        } else if constexpr (QIN == QIN_MXFP4) {
 #pragma unroll
-            for (int q = 0; q < 4; q++)
-#pragma unroll
-                for (int j = 0; j < 8; j++) v[8 * q + j] = __fmul_rn(e2m1_rebiased(u[q], j), s1);
+            for (int b = 0; b < 4; b++) {
+                const float2 f = e2m1x2_to_f32(u[q] >> (8 * b));
+                acc[8 * q + 2 * b] = __fmaf_rn(w, __fmul_rn(f.x, s), acc[8 * q + 2 * b]);
+                acc[8 * q + 2 * b + 1] = __fmaf_rn(w, __fmul_rn(f.y, s), acc[8 * q + 2 * b + 1]);
+            }
         } else {
 #pragma unroll
-            for (int q = 0; q < 4; q++)
-#pragma unroll
-                for (int b = 0; b < 4; b++) {
-                    const float2 f = e2m1x2_to_f32(u[q] >> (8 * b));
-                    v[8 * q + 2 * b] = __fmul_rn(f.x, s);
-                    v[8 * q + 2 * b + 1] = __fmul_rn(f.y, s);
-                }
-        }
-    } else {  // e4m3 codes
-        const float s1 = __fmul_rn(s, 0x1p120f);
-        if (fabsf(s1) <= FLT_MAX && !e4m3_has_nan(u)) {
-#pragma unroll
-            for (int q = 0; q < 4; q++)
-#pragma unroll
-                for (int j = 0; j < 4; j++) v[4 * q + j] = __fmul_rn(e4m3_rebiased(u[q], j), s1);
-        } else {
-#pragma unroll
-            for (int q = 0; q < 4; q++)
-#pragma unroll
-                for (int h = 0; h < 2; h++) {
-                    const float2 f = e4m3x2_to_f32(u[q] >> (16 * h));
-                    v[4 * q + 2 * h] = __fmul_rn(f.x, s);
-                    v[4 * q + 2 * h + 1] = __fmul_rn(f.y, s);
-                }
+            for (int h = 0; h < 2; h++) {
+                const float2 f = e4m3x2_to_f32(u[q] >> (16 * h));
+                acc[4 * q + 2 * h] = __fmaf_rn(w, __fmul_rn(f.x, s), acc[4 * q + 2 * h]);
+                acc[4 * q + 2 * h + 1] = __fmaf_rn(w, __fmul_rn(f.y, s), acc[4 * q + 2 * h + 1]);
+            }
         }
     }
+}
+
+// Where s is a normal power of two 2^k (every MX scale; E4M3 per 128 with
+// round_scale or UE8M0), y = decode(c) * s is exact (a code has at most four
+// significant bits and k keeps it finite), and so is W = w * s when W is
+// normal (or w is zero); then fma(W, decode(c), acc) equals the oracle's
+// fma(w, y, acc), with one FFMA per element and no multiply.  Returns false,
+// doing nothing, where that does not hold.
+template <int QIN>
+__device__ __forceinline__ bool pow2_fma(float (&acc)[combine_granule(QIN)], const uint4 &r,
+                                         float s, float w) {
+    constexpr int kMaxExp = QIN == QIN_MXFP4 ? 125 : 119;  // largest code * 2^k finite
+    const uint32_t sb = __float_as_uint(s);
+    const int ex = (int)(sb >> 23);  // a set sign bit makes ex > 255
+    if ((sb & 0x007FFFFFu) != 0u || ex < 1 || ex - 127 > kMaxExp) return false;
+    const float W = __fmul_rn(w, s);
+    if (!((fabsf(W) >= FLT_MIN || w == 0.0f) && fabsf(W) <= FLT_MAX)) return false;
+    const uint32_t u[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
-    for (int j = 0; j < EPG; j++) acc[j] = __fmaf_rn(w, v[j], acc[j]);
+    for (int q = 0; q < 4; q++) {
+        if constexpr (QIN == QIN_MXFP4) {
+#pragma unroll
+            for (int b = 0; b < 4; b++) {
+                const float2 f = e2m1x2_to_f32(u[q] >> (8 * b));
+                acc[8 * q + 2 * b] = __fmaf_rn(W, f.x, acc[8 * q + 2 * b]);
+                acc[8 * q + 2 * b + 1] = __fmaf_rn(W, f.y, acc[8 * q + 2 * b + 1]);
+            }
+        } else {
+#pragma unroll
+            for (int h = 0; h < 2; h++) {
+                const float2 f = e4m3x2_to_f32(u[q] >> (16 * h));
+                acc[4 * q + 2 * h] = __fmaf_rn(W, f.x, acc[4 * q + 2 * h]);
+                acc[4 * q + 2 * h + 1] = __fmaf_rn(W, f.y, acc[4 * q + 2 * h + 1]);
+            }
+        }
+    }
+    return true;
 }
 
 template <int TPT, int GMAX, int KB, int QIN>
@@ -197,6 +210,9 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
                 for (int kk = 0; kk < KB; kk++) {
                     const int k = k0 + kk;
                     if (k >= a.K || s_row[grp][k] < 0) continue;
+                    if constexpr (QIN != QIN_INT8) {
+                        if (pow2_fma<QIN>(acc, raw[kk], sc[kk], s_w[grp][k])) continue;
+                    }
                     dequant_fma<QIN>(acc, raw[kk], sc[kk], s_w[grp][k]);
                 }
             }
@@ -204,9 +220,150 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
         uint16_t *o = a.out + n * a.H + (int64_t)g * EPG;
 #pragma unroll
         for (int q = 0; q < EPG; q += 8)
-            st_v4(o + q, make_uint4(pack_bf16x2(acc[q], acc[q + 1]), pack_bf16x2(acc[q + 2], acc[q + 3]),
-                                    pack_bf16x2(acc[q + 4], acc[q + 5]), pack_bf16x2(acc[q + 6], acc[q + 7])));
+            st_v4(o + q, make_uint4(pack_bf16x2(acc[q], acc[q + 1]),
+                                    pack_bf16x2(acc[q + 2], acc[q + 3]),
+                                    pack_bf16x2(acc[q + 4], acc[q + 5]),
+                                    pack_bf16x2(acc[q + 6], acc[q + 7])));
     }
+}
+
+// ---------------------------------------------------------------------------
+// Combine of quantised expert outputs with the next granule's codes in flight
+// while the current one is decoded.  Decoding costs several operations per
+// element, so a thread that loaded, then decoded, would have no load in flight
+// for much of its time: here each thread copies the codes of granule i+1 (16
+// bytes per row) into its own slots of a two-stage shared-memory buffer
+// (cp.async) before it decodes granule i.  The scales of the token's rows are
+// copied once, with granule 0's codes.  Each thread reads only codes it copied
+// itself, so its own cp.async.wait_group orders those copies before the reads;
+// the scales, copied by all threads of the token, are read after a barrier.
+// No spin wait is involved.  Power-of-two scales take pow2_fma (one FFMA per
+// element), others dequant_fma.  Requires K <= 8 and scale rows of a multiple
+// of 4 bytes (S % 4 == 0) and at most kPipeScaleBytes; the launcher takes
+// combine_kernel otherwise.
+constexpr int kPipeRows = 8;          // K bound of combine_q_kernel
+constexpr int kPipeScaleBytes = 256;  // S bound (H <= 8192: 4*H/128 or H/32)
+
+template <int QIN>
+__device__ __forceinline__ float scale_at(const uint8_t *srow, int g, int sfmt) {
+    if constexpr (QIN == QIN_INT8) return *reinterpret_cast<const float *>(srow);
+    if constexpr (QIN == QIN_E4M3_B128) {
+        if (sfmt != 2) return reinterpret_cast<const float *>(srow)[g >> 3];
+        return exp2_neg(127 - (int)srow[g >> 3]);
+    }
+    if constexpr (QIN == QIN_MXFP8) return exp2_neg(127 - (int)srow[g >> 1]);
+    return exp2_neg(127 - (int)srow[g]);  // MXFP4: one byte per granule of 32
+}
+
+template <int TPT, int GMAX, int QIN>
+__global__ void __launch_bounds__(block_threads(TPT)) combine_q_kernel(CombineArgs a) {
+    static_assert(QIN != QIN_BF16 && TPT <= 128, "quantised rows, blocks of 128 threads");
+    pdl_enter();
+    constexpr int NT = block_threads(TPT);
+    constexpr int TOKS = NT / TPT;
+    constexpr int EPG = combine_granule(QIN);
+    constexpr int KB = kPipeRows;
+    __shared__ int64_t s_row[TOKS][16];
+    __shared__ float s_w[TOKS][16];
+    __shared__ __align__(16) uint4 s_code[2][KB][NT];
+    __shared__ __align__(16) uint8_t s_scl[TOKS][KB * kPipeScaleBytes];
+
+    const int tid = threadIdx.x;
+    const int grp = tid / TPT, lt = tid % TPT;
+    const int64_t n = (int64_t)blockIdx.x * TOKS + grp;
+    const bool active = n < a.N;
+
+    if (active && lt < a.K) {
+        uint32_t flags = 0;
+        int64_t row = -1;
+        const int64_t e = a.idx[n * a.K + lt];
+        if (e < -1 || e >= a.E) flags |= kDevBadIndex;
+        const int32_t s = (e >= 0 && e < a.E) ? a.slot[n * a.K + lt] : -1;
+        if (s >= 0) {
+            if (!a.packed) {
+                if (s < a.cap) row = e * a.cap + s;
+                else flags |= kDevCapacity;
+            } else {
+                const int64_t r = a.eo[e] + s;
+                if (r < a.eo[e + 1] && r < a.rows) row = r;
+                else flags |= kDevCapacity;
+            }
+        }
+        if (flags) atomicOr(a.status, flags);
+        s_row[grp][lt] = row;
+        s_w[grp][lt] = a.wts[n * a.K + lt];
+    }
+    __syncthreads();
+
+    const int ngran = a.H / EPG;
+    const uint8_t *ybase = reinterpret_cast<const uint8_t *>(a.y);
+    // the token's scale rows, whole, in 16- or 4-byte pieces
+    if (active) {
+        const uint8_t *sbase = ybase + a.scale_off;
+        const int S = (int)a.S;
+        if (S % 16 == 0) {
+            const int per = S / 16;
+            for (int w = lt; w < a.K * per; w += TPT) {
+                const int kk = w / per, o = (w - kk * per) * 16;
+                const int64_t row = s_row[grp][kk];
+                if (row >= 0) cp_async16(&s_scl[grp][kk * S + o], sbase + row * a.S + o);
+            }
+        } else {
+            const int per = S / 4;
+            for (int w = lt; w < a.K * per; w += TPT) {
+                const int kk = w / per, o = (w - kk * per) * 4;
+                const int64_t row = s_row[grp][kk];
+                if (row >= 0) cp_async4(&s_scl[grp][kk * S + o], sbase + row * a.S + o);
+            }
+        }
+    }
+    // copies of granule i's codes (if it exists) into stage i & 1, as one group
+    auto issue = [&](int i) {
+        const int g = i * TPT + lt;
+        if (active && i < GMAX && g < ngran) {
+#pragma unroll
+            for (int kk = 0; kk < KB; kk++) {
+                const int64_t row = kk < a.K ? s_row[grp][kk] : -1;
+                if (row >= 0)
+                    cp_async16(&s_code[i & 1][kk][tid], ybase + row * a.D + (int64_t)g * 16);
+            }
+        }
+        cp_async_commit();
+    };
+    issue(0);
+    cp_async_wait<0>();  // this thread's scale pieces and granule 0
+    __syncthreads();     // every thread's scale pieces
+    if (!active) return;
+
+#pragma unroll 1
+    for (int i = 0; i < GMAX; i++) {
+        const int g = i * TPT + lt;
+        if (g >= ngran) break;
+        issue(i + 1);
+        cp_async_wait<1>();  // granule i's group has landed
+        float acc[EPG];
+#pragma unroll
+        for (int q = 0; q < EPG; q++) acc[q] = 0.0f;
+#pragma unroll 1  // a rolled loop keeps the body in the instruction cache
+        for (int kk = 0; kk < KB; kk++) {
+            if (kk >= a.K || s_row[grp][kk] < 0) continue;
+            const uint4 r = s_code[i & 1][kk][tid];
+            const float sc = scale_at<QIN>(&s_scl[grp][kk * (int)a.S], g, a.sfmt);
+            const float w = s_w[grp][kk];
+            if constexpr (QIN != QIN_INT8) {
+                if (pow2_fma<QIN>(acc, r, sc, w)) continue;
+            }
+            dequant_fma<QIN>(acc, r, sc, w);
+        }
+        uint16_t *o = a.out + n * a.H + (int64_t)g * EPG;
+#pragma unroll
+        for (int q = 0; q < EPG; q += 8)
+            st_v4(o + q, make_uint4(pack_bf16x2(acc[q], acc[q + 1]),
+                                    pack_bf16x2(acc[q + 2], acc[q + 3]),
+                                    pack_bf16x2(acc[q + 4], acc[q + 5]),
+                                    pack_bf16x2(acc[q + 6], acc[q + 7])));
+    }
+    cp_async_wait<0>();  // nothing in flight when the thread exits
 }
 
 }  // namespace ep

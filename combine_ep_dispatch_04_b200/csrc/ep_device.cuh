@@ -90,32 +90,7 @@ __device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t two_codes) {
     return __half22float2(*reinterpret_cast<__half2 *>(&h2));
 }
 
-// ---- exact decoding with integer operations -------------------------------------
-// The conversions above issue at a fraction of the FMA rate.  These place a
-// code's sign and magnitude bits in an fp32 word whose exponent bias is 127
-// instead of the format's: read back, that word is the code's value times
-// 2^-(127 - bias) exactly (a zero or subnormal code gives an fp32 zero or
-// subnormal), so one exact power-of-two factor restores the value:
-// 2^120 for e4m3 (bias 7), 2^126 for e2m1 (bias 1).  The e4m3 NaN codes
-// (low seven bits all set) do not decode this way; e4m3_has_nan finds them.
-// (j is a constant once the callers' loops are unrolled)
-__device__ __forceinline__ float e4m3_rebiased(uint32_t w, int j) {  // byte j of w
-    const uint32_t top = __byte_perm(w, 0u, (j << 12) | 0x444);  // the code in bits 24..31
-    return __uint_as_float((uint32_t)((int32_t)top >> 4) & 0x87FFFFFFu);
-}
-// nibble j of w: element 2i is the low nibble of byte i
-__device__ __forceinline__ float e2m1_rebiased(uint32_t w, int j) {
-    uint32_t top = __byte_perm(w, 0u, ((j >> 1) << 12) | 0x444);  // byte in bits 24..31
-    if ((j & 1) == 0) top <<= 4;                                    // the nibble in 28..31
-    return __uint_as_float((uint32_t)((int32_t)top >> 6) & 0x81C00000u);
-}
-// Any of the 16 e4m3 codes a NaN code?
-__device__ __forceinline__ bool e4m3_has_nan(const uint32_t (&u)[4]) {
-    uint32_t t = 0u;
-#pragma unroll
-    for (int q = 0; q < 4; q++) t |= (u[q] & 0x7F7F7F7Fu) + 0x01010101u;  // no carry between bytes
-    return (t & 0x80808080u) != 0u;
-}
+// ---- exact int8 decoding without a conversion instruction ----------------------
 // int8 byte j of wx = w ^ 0x80808080: the fp32 2^23 + 128 + b, less 2^23 + 128 (both exact).
 __device__ __forceinline__ float i8_exact(uint32_t wx, int j) {
     return __uint_as_float(__byte_perm(wx, 0x4B000000u, 0x7440 | j)) - 8388736.0f;
@@ -170,6 +145,25 @@ __device__ __forceinline__ int mx_exponent_fast(float amax) {
 __device__ __forceinline__ float exp2_neg(int X) {
     int e = 127 - X;
     return e > 0 ? __uint_as_float((uint32_t)e << 23) : __uint_as_float(0x00400000u);
+}
+
+// ---- asynchronous copies global -> shared (per thread, completion by group) -----
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {  // L2 only
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(smem)), "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr(smem)), "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// Wait until at most N of this thread's committed groups are still in flight.
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // ---- streaming memory access --------------------------------------------------

@@ -435,3 +435,21 @@ def test_combine_of_quantized_round_scale_rows(flags):
     r = Run(synth.workload("decode", T=24), "e4m3_b128", layout="packed", flags=flags)
     combine_quantized_check(r, seed=3 + flags)
     combine_quantized_check(r, seed=5 + flags, rows_fn=special_quantized_rows)
+
+
+@pytest.mark.parametrize("mode,flags", [("mxfp8", 0), ("mxfp4", 0), ("e4m3_b128", ep.F_UE8M0),
+                                        ("e4m3_b128", ep.F_ROUND_SCALE), ("e4m3_b128", 0),
+                                        ("int8_token", 0)])
+def test_combine_of_quantized_special_weights(mode, flags):
+    """Weights that are zero, negative zero, subnormal, huge, infinite or NaN,
+    against scales of every kind: the weight-folded path must hand every case
+    it cannot do exactly to the scale multiply."""
+    from harness import combine_quantized_check, special_quantized_rows
+    w = synth.workload("decode", T=24)
+    idx, wts = synth.make_routing(w)
+    pick = np.float32([0.0, -0.0, 1e-45, 1e-39, 1e-30, 0.5, -2.0, 3e38, np.inf, -np.inf, np.nan,
+                       7.0, 0.125])
+    wts = pick[np.random.default_rng(9).integers(0, len(pick), wts.shape)]
+    r = Run(w, mode, layout="packed", idx=idx, wts=wts, flags=flags)
+    combine_quantized_check(r, seed=11, rows_fn=special_quantized_rows)
+    combine_quantized_check(r, seed=12)
