@@ -72,6 +72,10 @@ def parse():
                    help="combine reads expert outputs stored in the dispatch format")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-steady", action="store_true",
+                   help="skip the steady-state pass and its buffer copies (profiling runs)")
+    p.add_argument("--no-copy", action="store_true",
+                   help="skip the same-run copy-bandwidth measurement (profiling runs)")
     return p.parse_args()
 
 
@@ -462,6 +466,8 @@ def main():
     # same-run copy bandwidth (reference for the fractions above)
     copy_gbs = None
     try:
+        if args.no_copy:
+            raise RuntimeError("skipped")
         src = torch.empty(2 << 30, dtype=torch.uint8, device=dev)
         dst = torch.empty_like(src)
         for _ in range(3):
@@ -541,7 +547,7 @@ def steady_launches(ep, args, cfg, ccfg, b, kernels, calls, x_d, idx_d, wts_d, g
     do.  Workloads that move more than STEADY_MAX_BYTES a step are not timed
     this way: there the launch overhead is already a negligible part of an
     isolated launch.  Returns ({kernel: [ms per launch]}, sets)."""
-    if step_bytes > STEADY_MAX_BYTES:
+    if step_bytes > STEADY_MAX_BYTES or args.no_steady:
         return {}, 1
     sets = STEADY_SETS
     eo = b.expert_offset
