@@ -45,6 +45,18 @@ __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 
 __device__ __forceinline__ uint32_t bf2_absmax(uint32_t acc, uint32_t w) {
     return __vmaxu2(acc, w & 0x7FFF7FFFu);
 }
+// Block maxima leave NaN elements out (as fmaxf does).  Magnitudes compare as
+// unsigned integers and a NaN's is above infinity's (0x7F80), so a running
+// maximum above 0x7F80 says a NaN was seen; the maximum is then taken again
+// over the pairs with their NaN halves zeroed.
+__device__ __forceinline__ bool bf2_any_nan(uint32_t m) {
+    return (m & 0xFFFFu) > 0x7F80u || (m >> 16) > 0x7F80u;
+}
+__device__ __forceinline__ uint32_t bf2_drop_nan(uint32_t w) {
+    const uint32_t m = w & 0x7FFF7FFFu;
+    const uint32_t t = (m + 0x007F007Fu) & 0x80008000u;  // bit 15 of each NaN half
+    return m & ~((t >> 15) * 0xFFFFu);
+}
 __device__ __forceinline__ float bf2_fold(uint32_t m) {  // max of the two halves as fp32
     uint32_t lo = m & 0xFFFFu, hi = m >> 16;
     return __uint_as_float((lo > hi ? lo : hi) << 16);
@@ -108,9 +120,10 @@ __device__ __forceinline__ int ceil_log2_pos(float v) {
 
 // e8m0 exponent X of an MX block: the smallest power of two with
 // amax / qmax <= 2^X, i.e. ceil(log2(amax / qmax)) with one IEEE division,
-// clamped to [-127, 127]; amax == 0 gives 0.
+// clamped to [-127, 127]; amax == 0 gives 0, and so does a NaN amax (a block
+// whose every element is NaN: the maximum of no element).
 __device__ __forceinline__ int mx_exponent(float amax, float qmax) {
-    if (amax == 0.0f) return 0;
+    if (amax == 0.0f || amax != amax) return 0;
     float v = __fdiv_rn(amax, qmax);
     if (v == 0.0f) return -127;
     int X = ceil_log2_pos(v);

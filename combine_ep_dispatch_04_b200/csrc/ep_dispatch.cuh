@@ -90,8 +90,17 @@ template <> struct GranOut<Q_INT8> { static constexpr int bytes = 16; };
 template <> struct GranOut<Q_MXFP8> { static constexpr int bytes = 16; };
 template <> struct GranOut<Q_MXFP4> { static constexpr int bytes = 8; };
 
+// Largest magnitude of 16 bf16 values, NaNs left out, as a bf16 pair word
+// (out of line: taken only for a granule with a NaN).
+__device__ __noinline__ uint32_t nan_free_absmax16(const uint16_t *p) {
+    uint32_t m = 0u;
+    for (int q = 0; q < 8; q++) m = __vmaxu2(m, bf2_drop_nan(reinterpret_cast<const uint32_t *>(p)[q]));
+    return m;
+}
+
 __device__ __forceinline__ uint32_t q_i8(float v, float s) {
-    int q = __float2int_rn(__fmul_rn(v, s));
+    const float p = __fmul_rn(v, s);
+    int q = p != p ? 0 : __float2int_rn(p);  // int8 has no NaN: a NaN product is 0
     q = q > 127 ? 127 : (q < -127 ? -127 : q);
     return (uint32_t)q & 0xFFu;
 }
@@ -147,13 +156,25 @@ __global__ void __launch_bounds__(block_threads(TPT)) dispatch_kernel(DispatchAr
 
     // per-granule block maxima (bf16 magnitudes, exact)
     float gmax[GMAX];
+    uint32_t gm[GMAX];
+    bool nan = false;
 #pragma unroll
     for (int i = 0; i < GMAX; i++) {
         uint32_t m = 0u;
 #pragma unroll
         for (int q = 0; q < 8; q++) m = bf2_absmax(m, v[i][q]);
-        gmax[i] = bf2_fold(m);
+        gm[i] = m;
+        nan = nan || bf2_any_nan(m);
     }
+    if (nan) {  // a NaN element (rare): the maxima again, NaN halves left out
+#pragma unroll
+        for (int i = 0; i < GMAX; i++) {
+            const int g = i * TPT + lt;
+            if (active && g < ngran) gm[i] = nan_free_absmax16(a.x + n * a.H + (int64_t)g * 16);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < GMAX; i++) gmax[i] = bf2_fold(gm[i]);
 
     // scales
     float rs = 1.0f, rsinv = 1.0f;  // int8: per row
@@ -334,6 +355,7 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(Dispatc
     // the token's gradient row, unpacked to fp32 once for all its entries
     float f[GMAX][16];
     float gmax[GMAX];
+    uint32_t gm[GMAX];
 #pragma unroll
     for (int i = 0; i < GMAX; i++) {
         const int g = i * TPT + lt;
@@ -354,7 +376,22 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(Dispatc
             f[i][2 * q] = bf_lo(v[q]);
             f[i][2 * q + 1] = bf_hi(v[q]);
         }
-        const float fm = bf2_fold(m);
+        gm[i] = m;
+    }
+    // a NaN element (rare): the maxima again, NaN halves left out
+    bool nan = false;
+#pragma unroll
+    for (int i = 0; i < GMAX; i++) nan = nan || bf2_any_nan(gm[i]);
+    if (nan) {
+#pragma unroll
+        for (int i = 0; i < GMAX; i++) {
+            const int g = i * TPT + lt;
+            if (active && g < ngran) gm[i] = nan_free_absmax16(a.x + n * a.H + (int64_t)g * 16);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < GMAX; i++) {
+        const float fm = bf2_fold(gm[i]);
         gmax[i] = fmaxf(fm, __shfl_xor_sync(kFull, fm, 1));
     }
     __syncthreads();
@@ -372,6 +409,8 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(Dispatc
         for (int i = 0; i < GMAX; i++) {
             const int g = i * TPT + lt;
             if (g >= ngran) continue;
+            // NaN w (or inf w on a zero row) makes every product NaN: the
+            // maximum of no element, X = 0 (mx_exponent's NaN case)
             const float amax = weighted ? __fmul_rn(aw, gmax[i]) : gmax[i];
             const int X = mx_exponent_fast<448>(amax);
             const float s = exp2_neg(X);

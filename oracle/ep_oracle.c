@@ -101,9 +101,11 @@ uint8_t orc_e4m3_encode(float x)
 }
 
 /* OCP MX FP4 E2M1: bias 1, 1 mantissa bit, values {0,.5,1,1.5,2,3,4,6},
- * sign in bit 3.  Round to nearest even, saturate to 6. */
+ * sign in bit 3.  Round to nearest even, saturate to 6.  The format has no
+ * NaN; a NaN encodes as +6 (code 0x7), whatever its sign. */
 uint8_t orc_e2m1_encode(float x)
 {
+    if (isnan(x)) return 0x7;
     uint8_t sign = signbit(x) ? 0x8 : 0x0;
     float a = fabsf(x);
     return (uint8_t)(sign | small_float_code(a, 1, 1, 6.0f, 0x7));
@@ -131,13 +133,15 @@ float orc_e2m1_decode(uint8_t c)
  * the block fits: |x| * 2^-X <= qmax.  Written with frexp, which splits v into
  * m * 2^e exactly (m in [0.5, 1)); log2 v is an integer only when m == 0.5.
  * The exponent is clamped to the e8m0 range [-127, 127] (byte 255 = NaN is
- * never produced).  amax == 0 gives X = 0 (scale 1.0).
+ * never produced); an infinite quotient gives 127.  amax == 0 gives X = 0
+ * (scale 1.0).
  */
 int orc_mx_exponent(float amax, float qmax)
 {
     if (amax == 0.0f) return 0;
     float v = amax / qmax; /* one IEEE division */
     if (v == 0.0f) return -127; /* underflowed: log2 v is below the e8m0 range */
+    if (isinf(v)) return 127;   /* an infinite maximum: log2 v is above it */
     int e;
     float m = frexpf(v, &e);
     int X = (m == 0.5f) ? e - 1 : e;
@@ -170,6 +174,8 @@ long orc_row_scale_bytes(int mode, int H)
     }
 }
 
+/* Largest magnitude of a block; NaN elements are left out (the comparison
+ * is false for them), as fmaxf does.  A NaN element still encodes as NaN. */
 static float absmax(const float *x, int n)
 {
     float a = 0.0f;
@@ -227,6 +233,7 @@ void orc_quant_row_f32(int mode, int H, float e4m3_qmax, const float *x, uint8_t
         }
         for (int h = 0; h < H; h++) {
             float q = rintf(x[h] * s);
+            if (isnan(q)) q = 0.0f; /* int8 has no NaN: a NaN product (NaN x, or inf * 0) is 0 */
             if (q > 127.0f) q = 127.0f;
             if (q < -127.0f) q = -127.0f;
             data[h] = (uint8_t)(int8_t)q;
@@ -606,7 +613,7 @@ void orc_e2m1_encode_bits(uint32_t start, uint8_t *out, long n)
 {
     for (long i = 0; i < n; i++) {
         float f = bits_to_f32(start + (uint32_t)i);
-        out[i] = isnan(f) ? 0xFF : orc_e2m1_encode(f);
+        out[i] = orc_e2m1_encode(f);
     }
 }
 /* e8m0 byte (X + 127) of a block whose maximum is |value of bit pattern

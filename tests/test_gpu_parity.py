@@ -453,3 +453,52 @@ def test_combine_of_quantized_special_weights(mode, flags):
     r = Run(w, mode, layout="packed", idx=idx, wts=wts, flags=flags)
     combine_quantized_check(r, seed=11, rows_fn=special_quantized_rows)
     combine_quantized_check(r, seed=12)
+
+
+# ---------------------------------------------------------------------------
+# non-finite inputs and weights
+# ---------------------------------------------------------------------------
+def _nonfinite_x(w, with_nan=True):
+    x = synth.make_x(w)
+    f = oracle.bf16_to_f32(x).copy()
+    f[0, 5] = np.inf                      # an infinite block maximum
+    f[1, 130] = -np.inf
+    f[2, ::97] = np.inf
+    if with_nan:
+        f[3, 17] = np.nan                 # NaN elements: left out of the block maximum
+        f[4, ::13] = np.nan
+        f[5, :128] = np.nan               # a block of NaNs only
+    return synth.to_bf16_bits(f)
+
+
+@pytest.mark.parametrize("mode,flags", [("bf16", 0), ("int8_token", 0), ("e4m3_b128", 0),
+                                        ("e4m3_b128", ep.F_UE8M0), ("mxfp8", 0), ("mxfp4", 0)])
+def test_nonfinite_inputs(mode, flags):
+    w = _edge(R=2, T=8, M=8, K=3, E=8, H=512)
+    x = _nonfinite_x(w)
+    r = Run(w, mode, layout="packed", x=x, flags=flags, backward=True)
+    r.check_dispatch()
+    r.check_backward()
+
+
+def test_backward_special_weights():
+    """Weights that are zero, signed zero, subnormal, huge (products overflow),
+    infinite or NaN, on gradients with large and non-finite values: the folded
+    scale multiply must leave every such case to the two-multiply path."""
+    w = _edge(R=2, T=16, M=16, K=4, E=8, H=512)
+    idx, wts = synth.make_routing(w)
+    pick = np.float32([0.0, -0.0, 1e-45, 1e-39, 3e38, -2.0, np.inf, -np.inf, np.nan, 0.25,
+                       1.0, 7.5])
+    wts = pick[np.random.default_rng(5).integers(0, len(pick), wts.shape)]
+    r = Run(w, "mxfp8", layout="packed", idx=idx, wts=wts, backward=True,
+            x=_nonfinite_x(w, with_nan=False))
+    g = oracle.bf16_to_f32(r.g).copy()
+    g[0] *= np.float32(2.0 ** 100)
+    g[1, 3] = np.inf
+    g[2, 9] = np.nan
+    g[3] = 0.0
+    r.g = synth.to_bf16_bits(g)
+    r.g_d = bf16_dev(r.g)
+    ep.ep_combine_backward(r.cfg, r.g_d, r.idx_d, r.wts_d, r.b.token_slot, r.b.grad_buf,
+                           r.b.dev_status, expert_offset=r.b.expert_offset)
+    r.check_backward()

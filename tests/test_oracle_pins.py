@@ -691,3 +691,53 @@ def test_round_scale_zero_block_uses_unit_scale():
     du, su = oracle.quant_row("e4m3_b128_ue8m0", x)
     assert list(su) == [127, 120, 0, 0]
     assert np.all(d[:128] == 0) and np.all(d[128:] == oracle.e4m3_encode(np.float32([3.0 * 128]))[0])
+
+
+# ---------------------------------------------------------------------------
+# non-finite inputs: an infinite block maximum, NaN elements, int8 NaN products
+# ---------------------------------------------------------------------------
+
+def test_infinite_block_maximum_takes_the_largest_exponent():
+    """ceil(log2(inf)) clamped to the e8m0 range is 127: the infinite element
+    saturates, every finite one falls to (signed) zero."""
+    assert oracle.mx_exponent(np.float32([np.inf]), 448.0)[0] == 127
+    assert oracle.mx_exponent(np.float32([np.inf]), 6.0)[0] == 127
+    x = np.zeros(64, np.float32)
+    x[3], x[4], x[5] = np.inf, -np.inf, -3.0
+    x[40] = 1.5
+    d, s = oracle.quant_row("mxfp8", x)
+    assert list(s) == [254, 127 + oracle.mx_exponent(np.float32([1.5]), 448.0)[0]]
+    assert list(d[3:6]) == [0x7E, 0xFE, 0x80] and np.all(d[[0, 1, 2, 6]] == 0)
+    d, s = oracle.quant_row("mxfp4", x)
+    # element 2i is the low nibble: byte 1 = (inf -> 6 | 0), byte 2 = (-inf -> -6 | -3 -> -0)
+    assert s[0] == 254 and d[1] == (0x7 << 4) | 0x0 and d[2] == (0x8 << 4) | 0xF
+    d, s = oracle.quant_row("e4m3_b128_p2", np.concatenate([x, np.zeros(64, np.float32)]))
+    assert s.view(np.float32)[0] == np.float32(2.0 ** 127) and d[3] == 0x7E
+
+
+def test_block_maximum_leaves_nan_out():
+    r = np.random.default_rng(3)
+    x = r.standard_normal(256).astype(np.float32)
+    y = x.copy()
+    y[[7, 100, 200]] = [np.nan, -np.nan, np.nan]
+    z = x.copy()
+    z[[7, 100, 200]] = 0.0
+    for mode in ("mxfp8", "e4m3_b128", "e4m3_b128_p2", "int8_token"):
+        dy, sy = oracle.quant_row(mode, y)
+        dz, sz = oracle.quant_row(mode, z)
+        assert np.array_equal(sy, sz), mode           # the scales ignore the NaNs
+        keep = np.ones(256, bool)
+        keep[[7, 100, 200]] = False
+        assert np.array_equal(dy[keep], dz[keep]), mode
+        want = 0x00 if mode == "int8_token" else 0x7F  # int8 has no NaN
+        assert np.all(dy[[7, 100, 200]] == want), mode
+
+
+def test_e2m1_nan_is_the_largest_positive_code():
+    got = oracle.e2m1_encode(np.float32([np.nan, -np.nan, np.inf, -np.inf]))
+    assert list(got) == [0x7, 0x7, 0x7, 0xF]
+
+
+def test_int8_nan_products_are_zero():
+    d, s = oracle.quant_row("int8_token", np.float32([np.inf, 1.0, -2.0, np.nan]))
+    assert list(d) == [0, 0, 0, 0] and s.view(np.float32)[0] == np.inf
