@@ -62,6 +62,8 @@ _lib.orc_combine.restype = C.c_uint32
 _lib.orc_combine.argtypes = [_i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p]
 _lib.orc_combine_bwd.restype = C.c_uint32
 _lib.orc_combine_bwd.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]
+_lib.orc_combine_wgrad.restype = C.c_uint32
+_lib.orc_combine_wgrad.argtypes = [_i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p]
 _lib.orc_bwd_row.restype = None
 _lib.orc_bwd_row.argtypes = [_i, _f, _i, _p, _p, _p]
 _lib.orc_combine_gathered.restype = None
@@ -299,6 +301,21 @@ def combine_bwd(R, T, K, E, M, H, g, topk_idx, topk_weights, token_slot, expert_
     st = _lib.orc_combine_bwd(R, T, K, E, M, H, _layout(layout), int(bool(unweighted)), _ptr(g),
                               _ptr(idx), _ptr(w), _ptr(slot), _ptr(eo), _ptr(gd), _ptr(gs))
     return dict(grad_data=gd, grad_scale=gs, status=int(st))
+
+
+def combine_wgrad(R, T, K, E, M, H, g, y, topk_idx, token_slot, expert_offset=None,
+                  layout="padded"):
+    """Weight gradient dw [N, K] f32 (dot products of g [N, H] with the entries'
+    expert rows y [rows, H], bf16 bits), and the status bits."""
+    g = _c(g, np.uint16).reshape(R * T, H)
+    y = _c(y, np.uint16)
+    idx = _c(topk_idx, np.int64)
+    slot = _c(token_slot, np.int32)
+    eo = None if expert_offset is None else _c(expert_offset, np.int64)
+    dw = np.zeros((R * T, K), np.float32)
+    st = _lib.orc_combine_wgrad(R, T, K, E, M, H, _layout(layout), _ptr(g), _ptr(y), _ptr(idx),
+                                _ptr(slot), _ptr(eo), _ptr(dw))
+    return dw, int(st)
 
 
 def combine_gathered(yrows, w, valid):

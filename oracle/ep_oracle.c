@@ -519,6 +519,39 @@ uint32_t orc_combine_bwd(int R, int T, int K, int E, int M, int H, int layout, i
 }
 
 /*
+ * Gradient of the combine with respect to the top-k weights (the reading of
+ * the "grad w.r.t. topk_weights" extension of the combine backward: the
+ * combine is out[n] = sum_k w[n,k] * y_k, so d out / d w[n,k] = y_k and the
+ * weight gradient is the dot product of the output gradient g[n,:] with the
+ * entry's expert row).  Every product of two bf16 values is exact in double
+ * and the sum is taken in double in h order, rounded to fp32 once.  Masked
+ * entries get 0.
+ */
+uint32_t orc_combine_wgrad(int R, int T, int K, int E, int M, int H, int layout,
+                           const uint16_t *g, const uint16_t *y, const int64_t *idx,
+                           const int32_t *token_slot, const int64_t *expert_offset, float *dw)
+{
+    uint32_t st = 0;
+    long N = (long)R * T, cap = (long)R * M;
+    for (long n = 0; n < N; n++) {
+        for (int k = 0; k < K; k++) {
+            dw[n * K + k] = 0.0f;
+            int64_t e = idx[n * K + k];
+            if (e < -1 || e >= E) st |= ORC_ST_BAD_INDEX;
+            int32_t slot = token_slot[n * K + k];
+            if (e < 0 || e >= E || slot < 0) continue;
+            long row = row_of(layout, cap, expert_offset, e, slot);
+            if (row < 0) { st |= ORC_ST_CAPACITY; continue; }
+            double acc = 0.0;
+            for (int h = 0; h < H; h++)
+                acc += (double)orc_bf16_to_f32(g[n * H + h]) * (double)orc_bf16_to_f32(y[row * H + h]);
+            dw[n * K + k] = (float)acc;
+        }
+    }
+    return st;
+}
+
+/*
  * Dequantisation of one row stored in a quantised format ([FP8] The FP8
  * Combine Operation: the received codes times the stored inverse scale, in
  * fp32).  Each element is decode(code) * scale_inv as

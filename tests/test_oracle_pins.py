@@ -741,3 +741,63 @@ def test_e2m1_nan_is_the_largest_positive_code():
 def test_int8_nan_products_are_zero():
     d, s = oracle.quant_row("int8_token", np.float32([np.inf, 1.0, -2.0, np.nan]))
     assert list(d) == [0, 0, 0, 0] and s.view(np.float32)[0] == np.inf
+
+
+# ---------------------------------------------------------------------------
+# weight gradient of the combine: dw[n,k] = <g[n,:], y[row(n,k),:]>
+# ---------------------------------------------------------------------------
+
+def _wgrad_case(layout="padded", align=1, H=32, seed=0):
+    w = synth.workload("tiny", R=2, T=5, M=6, K=3, E=4, H=H)
+    idx, _ = synth.make_routing(w, seed)
+    idx[1, 2] = -1
+    lay = _run_layout(w, idx, layout, align)
+    rows = oracle.rows_max(w["R"], w["T"], w["K"], w["E"], w["M"], layout, align)
+    r = np.random.default_rng(seed)
+    # bf16 values with few significant bits: every double sum below is exact
+    y = synth.to_bf16_bits((r.integers(-64, 64, (rows, H)) / 16.0).astype(np.float32))
+    g = synth.to_bf16_bits((r.integers(-64, 64, (w["N"], H)) / 32.0).astype(np.float32))
+    return w, idx, lay, y, g
+
+
+@pytest.mark.parametrize("layout,align", [("padded", 1), ("packed", 1), ("packed", 4)])
+def test_wgrad_equals_exact_rational_dot_products(layout, align):
+    from fractions import Fraction
+    w, idx, lay, y, g = _wgrad_case(layout, align)
+    dw, st = oracle.combine_wgrad(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], g, y, idx,
+                                  lay["token_slot"], lay["expert_offset"], layout=layout)
+    assert st == 0
+    gf, yf = _f(g), _f(y)
+    for n in range(w["N"]):
+        for k in range(w["K"]):
+            if idx[n, k] < 0:
+                assert dw[n, k] == 0.0
+                continue
+            row = int(oracle.row_index(layout, w["R"], w["M"], idx[n, k], lay["token_slot"][n, k],
+                                       lay["expert_offset"]))
+            exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(gf[n], yf[row]))
+            assert dw[n, k] == np.float32(float(exact)), (n, k)
+
+
+def test_wgrad_one_hot_gradient_picks_the_expert_value():
+    w, idx, lay, y, g = _wgrad_case(H=64, seed=3)
+    for j in (0, 17, 63):
+        g1 = np.zeros_like(g)
+        g1[:, j] = synth.to_bf16_bits(np.float32([1.0]))[0]
+        dw, _ = oracle.combine_wgrad(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], g1, y, idx,
+                                     lay["token_slot"], lay["expert_offset"])
+        for n in range(w["N"]):
+            for k in range(w["K"]):
+                if idx[n, k] >= 0:
+                    row = int(oracle.row_index("padded", w["R"], w["M"], idx[n, k],
+                                               lay["token_slot"][n, k]))
+                    assert dw[n, k] == _f(y[row:row + 1, j])[0]
+
+
+def test_wgrad_flags_bad_indices():
+    w, idx, lay, y, g = _wgrad_case()
+    bad = idx.copy()
+    bad[0, 0] = w["E"]
+    dw, st = oracle.combine_wgrad(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], g, y, bad,
+                                  lay["token_slot"], lay["expert_offset"])
+    assert st & oracle.ST_BAD_INDEX and dw[0, 0] == 0.0
