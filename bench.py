@@ -72,6 +72,8 @@ def parse():
                    help="combine reads expert outputs stored in the dispatch format")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--weights-grad", action="store_true",
+                   help="also time the combine's weight gradient (outside the step)")
     p.add_argument("--no-steady", action="store_true",
                    help="skip the steady-state pass and its buffer copies (profiling runs)")
     p.add_argument("--no-copy", action="store_true",
@@ -82,7 +84,7 @@ def parse():
 # ---------------------------------------------------------------------------
 # algorithmic bytes (what the method must move; unwritten capacity not counted)
 # ---------------------------------------------------------------------------
-def algorithmic_bytes(w, mode, idx, quantized_combine=False):
+def algorithmic_bytes(w, mode, idx, quantized_combine=False, weights_grad=False):
     """Bytes per launch of each kernel, from the per-token counts."""
     import oracle
 
@@ -97,6 +99,8 @@ def algorithmic_bytes(w, mode, idx, quantized_combine=False):
     }
     if w.get("backward"):
         out["combine_bwd"] = N * (2 * H + 4 * K + 4 * K + 8 * K) + v * (H + H // 32)
+    if weights_grad:  # g, idx, slots, dw; one expert row per valid entry
+        out["combine_bwd_w"] = N * (2 * H + 8 * K + 4 * K + 4 * K) + v * 2 * H
     return out, v
 
 
@@ -351,6 +355,14 @@ def main():
         flush_r.max()
 
     kernels = ["layout", "dispatch", "combine"] + (["combine_bwd"] if g_d is not None else [])
+    if args.weights_grad and args.quantized_combine:
+        raise SystemExit("--weights-grad reads bf16 expert outputs: not with --quantized-combine")
+    gw_d = dw_d = None
+    if args.weights_grad:
+        gp, go = synth.g_source(w, replica)
+        gw_d = torch.from_numpy(synth.windows(gp, go, H).view(np.int16)).to(dev).view(torch.bfloat16)
+        dw_d = torch.empty((N, K), dtype=torch.float32, device=dev)
+        kernels.append("combine_bwd_w")
 
     # each C-ABI call is checked and marshalled once, then replayed every step.
     # The timed step uses the one-call dispatch (layout + dispatch, the
@@ -376,6 +388,10 @@ def main():
                                             b.dev_status, expert_offset=b.expert_offset,
                                             stream=stream, bind=True))
         step_calls.append(calls[-1])
+    if gw_d is not None:  # timed per kernel only: not a step of the configured path
+        calls.append(ep.ep_combine_backward_weights(cfg, gw_d, b.y, idx_d, b.token_slot, dw_d,
+                                                    b.dev_status, expert_offset=b.expert_offset,
+                                                    stream=stream, bind=True))
 
     def step(evs=None, fl=0):
         if evs is None:
@@ -430,9 +446,10 @@ def main():
         for i, k in enumerate(kernels):
             per_kernel[k].append(e[i][0].elapsed_time(e[i][1]))
 
-    alg, v = algorithmic_bytes(w, mode, idx, quantized_combine=args.quantized_combine)
+    alg, v = algorithmic_bytes(w, mode, idx, quantized_combine=args.quantized_combine,
+                               weights_grad=args.weights_grad)
     steady, sets = steady_launches(ep, args, cfg, ccfg, b, kernels, calls, x_d, idx_d, wts_d, g_d,
-                                   flush, stream, dev, sum(alg.values()))
+                                   flush, stream, dev, sum(alg.values()), gw_d, dw_d)
     peaks = measured_peaks()
     peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else FALLBACK_HBM_GBS
     peak_src = "measured" if peaks and peaks.get("hbm_gbs") else "fallback"
@@ -451,7 +468,7 @@ def main():
                               "gbs_steady": round(alg[k] / (st_ms * 1e-3) / 1e9, 1),
                               "frac_steady_of_" + peak_src:
                                   round(alg[k] / (st_ms * 1e-3) / 1e9 / peak, 4)})
-    dom = max(kernels, key=lambda k: alg[k])
+    dom = max((k for k in kernels if k != "combine_bwd_w"), key=lambda k: alg[k])
     iso_achieved = alg[dom] / (statistics.mean(per_kernel[dom]) * 1e-3) / 1e9
     if sets > 1:
         achieved = alg[dom] / (statistics.mean(steady[dom]) * 1e-3) / 1e9
@@ -461,7 +478,7 @@ def main():
     else:
         achieved = iso_achieved
         duration = "per launch: each launch alone between its own events, after an L2 flush"
-    step_bytes = sum(alg.values())
+    step_bytes = sum(v_ for k_, v_ in alg.items() if k_ != "combine_bwd_w")
 
     # same-run copy bandwidth (reference for the fractions above)
     copy_gbs = None
@@ -537,7 +554,7 @@ STEADY_MAX_BYTES = 1 << 30
 
 
 def steady_launches(ep, args, cfg, ccfg, b, kernels, calls, x_d, idx_d, wts_d, g_d, flush, stream,
-                    dev, step_bytes):
+                    dev, step_bytes, gw_d=None, dw_d=None):
     """Per-launch durations with the launch overhead amortised as in the step:
     each kernel is launched STEADY_SETS times back to back, on as many
     distinct copies of the buffers it reads and writes (each launch's data is
@@ -563,6 +580,12 @@ def steady_launches(ep, args, cfg, ccfg, b, kernels, calls, x_d, idx_d, wts_d, g
         per_set["combine"].append(ep.ep_combine(ccfg, ys, idx_d, wts_d, b.token_slot, os_,
                                                 b.dev_status, expert_offset=eo, stream=stream,
                                                 bind=True))
+        if "combine_bwd_w" in per_set:
+            gws, dws = gw_d.clone(), torch.empty_like(dw_d)
+            keep += [gws, dws]
+            per_set["combine_bwd_w"].append(ep.ep_combine_backward_weights(
+                cfg, gws, ys, idx_d, b.token_slot, dws, b.dev_status, expert_offset=eo,
+                stream=stream, bind=True))
         if "combine_bwd" in per_set:
             gs, gb = g_d.clone(), torch.empty_like(b.grad_buf)
             keep += [gs, gb]

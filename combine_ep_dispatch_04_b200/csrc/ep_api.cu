@@ -765,6 +765,47 @@ ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
     return launch_combine_bwd(a, cs(stream));
 }
 
+ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *g,
+                                        const uint16_t *y, const void *topk_idx,
+                                        const int32_t *token_slot, const int64_t *expert_offset,
+                                        float *topk_weights_grad, uint32_t *dev_status,
+                                        ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (!dev_status) return EP_ERR_INVALID_ARG;
+    if (cfg->flags & EP_F_COMBINE_QUANTIZED) return EP_ERR_UNSUPPORTED;  // bf16 y only
+    if (p.N == 0) return EP_OK;
+    if (!g || !y || !topk_idx || !token_slot || !topk_weights_grad) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    if (!aligned16(g) || !aligned16(y)) return EP_ERR_MISALIGNED;
+
+    ep::WgradArgs a;
+    a.N = p.N; a.K = p.K; a.E = p.E; a.H = p.H;
+    a.packed = cfg->layout == EP_LAYOUT_PACKED;
+    a.cap = p.cap; a.rows = p.rows;
+    a.g = g; a.y = y; a.idx = topk_idx_view(cfg, topk_idx);
+    a.slot = token_slot; a.eo = expert_offset;
+    a.dw = topk_weights_grad; a.status = dev_status;
+    auto kernel_of = [](int t, int gm) -> const void * {
+#define EP_FN(T_, G_) if (t == T_ && gm == G_) return (const void *)ep::combine_wgrad_kernel<T_, G_>;
+        EP_SPLITS(EP_FN)
+#undef EP_FN
+        return nullptr;
+    };
+    const Split sp = split_rows(a.N, a.H / 8, 8, kernel_of);
+    const unsigned grid = grid_for(a.N, sp.tpt);
+    cudaStream_t s = cs(stream);
+#define EP_CASE(T_, G_)                                                                     \
+    if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
+        launch(ep::combine_wgrad_kernel<T_, G_>, grid, ep::block_threads(T_), 0, s, a);     \
+        return launched();                                                                  \
+    }
+    EP_SPLITS(EP_CASE)
+#undef EP_CASE
+    return EP_ERR_UNSUPPORTED;
+}
+
 ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream) {
     if (!dev_status || !host_flags) return EP_ERR_INVALID_ARG;
     cudaStream_t s = cs(stream);

@@ -366,4 +366,117 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_q_kernel(CombineAr
     cp_async_wait<0>();  // nothing in flight when the thread exits
 }
 
+// ---------------------------------------------------------------------------
+// Weight gradient of the combine: dw[n,k] = <g[n,:], y[row(n,k),:]>, the
+// derivative of sum_k w_k y_k with respect to w_k.  Every bf16 x bf16
+// product is exact in fp32 and enters an fp32 FMA chain per thread (its
+// granules in order), then a shuffle / shared-memory tree over the token's
+// threads; masked entries get 0.  Reads g once and each entry's expert row
+// once (the bytes of a combine).
+struct WgradArgs {
+    int64_t N;
+    int K, E, H;
+    int packed;
+    int64_t cap, rows;
+    const uint16_t *g;  // [N][H] bf16
+    const uint16_t *y;  // [rows][H] bf16
+    TopkIdx idx;
+    const int32_t *slot;
+    const int64_t *eo;
+    float *dw;          // [N][K]
+    uint32_t *status;
+};
+
+template <int TPT, int GMAX>
+__global__ void __launch_bounds__(block_threads(TPT)) combine_wgrad_kernel(WgradArgs a) {
+    pdl_enter();
+    constexpr int NT = block_threads(TPT);
+    constexpr int TOKS = NT / TPT;
+    constexpr int WPG = (TPT + 31) / 32;  // warps per token group
+    constexpr int KB = 8;                 // row loads in flight per granule
+    __shared__ int64_t s_row[TOKS][16];
+    __shared__ float s_part[TOKS][WPG][16];
+
+    const int grp = threadIdx.x / TPT, lt = threadIdx.x % TPT;
+    const int64_t n = (int64_t)blockIdx.x * TOKS + grp;
+    const bool active = n < a.N;
+
+    if (active && lt < a.K) {
+        uint32_t flags = 0;
+        int64_t row = -1;
+        const int64_t e = a.idx[n * a.K + lt];
+        if (e < -1 || e >= a.E) flags |= kDevBadIndex;
+        const int32_t s = (e >= 0 && e < a.E) ? a.slot[n * a.K + lt] : -1;
+        if (s >= 0) {
+            if (!a.packed) {
+                if (s < a.cap) row = e * a.cap + s;
+                else flags |= kDevCapacity;
+            } else {
+                const int64_t r = a.eo[e] + s;
+                if (r < a.eo[e + 1] && r < a.rows) row = r;
+                else flags |= kDevCapacity;
+            }
+        }
+        if (flags) atomicOr(a.status, flags);
+        s_row[grp][lt] = row;
+    }
+    __syncthreads();
+
+    float acc[16];
+#pragma unroll
+    for (int k = 0; k < 16; k++) acc[k] = 0.0f;
+    const int ngran = a.H >> 3;
+    if (active) {
+#pragma unroll 1
+        for (int i = 0; i < GMAX; i++) {
+            const int g = i * TPT + lt;
+            if (g >= ngran) break;
+            const uint4 gv = ld_stream(a.g + n * a.H + (int64_t)g * 8);
+            const uint32_t gu[4] = {gv.x, gv.y, gv.z, gv.w};
+#pragma unroll
+            for (int k0 = 0; k0 < 16; k0 += KB) {
+                if (k0 >= a.K) break;
+                uint4 buf[KB];
+#pragma unroll
+                for (int kk = 0; kk < KB; kk++) {
+                    const int k = k0 + kk;
+                    const int64_t row = k < a.K ? s_row[grp][k] : -1;
+                    buf[kk] = row >= 0 ? ld_stream(a.y + row * a.H + (int64_t)g * 8)
+                                       : make_uint4(0u, 0u, 0u, 0u);
+                }
+#pragma unroll
+                for (int kk = 0; kk < KB; kk++) {
+                    const uint32_t u[4] = {buf[kk].x, buf[kk].y, buf[kk].z, buf[kk].w};
+                    float t = acc[k0 + kk];
+#pragma unroll
+                    for (int q = 0; q < 4; q++) {
+                        t = __fmaf_rn(bf_lo(gu[q]), bf_lo(u[q]), t);
+                        t = __fmaf_rn(bf_hi(gu[q]), bf_hi(u[q]), t);
+                    }
+                    acc[k0 + kk] = t;
+                }
+            }
+        }
+    }
+    // the token's threads: warp shuffles, then the warps' partial sums
+#pragma unroll
+    for (int k = 0; k < 16; k++) {
+        float v = acc[k];
+#pragma unroll
+        for (int o = (TPT < 32 ? TPT : 32) / 2; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+        acc[k] = v;
+    }
+    if ((lt & 31) == 0) {
+#pragma unroll
+        for (int k = 0; k < 16; k++) s_part[grp][lt >> 5][k] = acc[k];
+    }
+    __syncthreads();
+    if (active && lt < a.K) {
+        float v = 0.0f;
+#pragma unroll
+        for (int wp = 0; wp < WPG; wp++) v += s_part[grp][wp][lt];
+        a.dw[n * a.K + lt] = s_row[grp][lt] >= 0 ? v : 0.0f;
+    }
+}
+
 }  // namespace ep

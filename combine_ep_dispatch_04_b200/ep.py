@@ -79,6 +79,8 @@ lib.ep_combine.restype = C.c_int
 lib.ep_combine.argtypes = [_CFG] + [_P] * 8
 lib.ep_combine_backward.restype = C.c_int
 lib.ep_combine_backward.argtypes = [_CFG] + [_P] * 8
+lib.ep_combine_backward_weights.restype = C.c_int
+lib.ep_combine_backward_weights.argtypes = [_CFG] + [_P] * 8
 lib.ep_get_status.restype = C.c_int
 lib.ep_get_status.argtypes = [_P, C.POINTER(C.c_uint32), _P]
 lib.ep_copy.restype = C.c_int
@@ -310,6 +312,25 @@ def ep_combine_backward(cfg, g, topk_idx, topk_weights, token_slot, grad_buf, de
         _stream(stream),
     ]
     return _call(lib.ep_combine_backward, cfg, args, "ep_combine_backward", bind)
+
+
+def ep_combine_backward_weights(cfg, g, y, topk_idx, token_slot, topk_weights_grad, dev_status,
+                                expert_offset=None, stream=None, bind=False):
+    """topk_weights_grad[n, k] = <g[n, :], y[row(n, k), :]> (0 for masked entries)."""
+    N, K = _nk(cfg)
+    sz = ep_buffer_sizes(cfg)
+    args = [
+        _dev(g, "g", torch.bfloat16, (N, cfg.hidden)),
+        _dev(y, "y", torch.bfloat16, (sz["rows"], cfg.hidden)),
+        _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
+        _dev(token_slot, "token_slot", torch.int32, (N, K)),
+        _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
+             optional=cfg.layout == LAYOUT["padded"]),
+        _dev(topk_weights_grad, "topk_weights_grad", torch.float32, (N, K)),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    return _call(lib.ep_combine_backward_weights, cfg, args, "ep_combine_backward_weights", bind)
 
 
 def ep_get_status(dev_status, stream=None):

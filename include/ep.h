@@ -242,6 +242,27 @@ ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
                                 void *grad_buf, uint32_t *dev_status, ep_stream_t stream);
 
 /*
+ * Gradient of the combine with respect to the top-k weights (the combine is
+ * out[n] = sum_k w[n,k] * y[row(n,k)], so d out / d w[n,k] is the entry's
+ * expert row; no page defines this call: it completes the combine backward
+ * of [TE] Description, whose other half is ep_combine_backward):
+ *   topk_weights_grad[n,k] = sum_h g[n,h] * y[row(n,k),h]
+ * for each valid entry, 0 for masked ones.  Each bf16 x bf16 product is exact
+ * in fp32; the sum is taken in fp32 (an FMA chain per thread over its part of
+ * the row, then a tree over the token's threads), so its rounding depends on
+ * the order: within 128 * 2^-24 * sum_h |g[n,h] * y[row,h]| of the exact sum.
+ *   g                  bf16 [N][H]: gradient of the combined output
+ *   y                  bf16 [rows][H]: the expert outputs ep_combine read
+ *   topk_weights_grad  float [N][K]
+ * EP_F_COMBINE_QUANTIZED is not supported here (EP_ERR_UNSUPPORTED).
+ */
+ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *g,
+                                        const uint16_t *y, const void *topk_idx,
+                                        const int32_t *token_slot, const int64_t *expert_offset,
+                                        float *topk_weights_grad, uint32_t *dev_status,
+                                        ep_stream_t stream);
+
+/*
  * Allocation-free variant of ep_dispatch_layout.  The pages have no
  * counterpart to this call; it exists for callers that cannot allocate
  * device memory when they route tokens -- for example a serving loop whose

@@ -64,6 +64,8 @@ _lib.orc_combine_bwd.restype = C.c_uint32
 _lib.orc_combine_bwd.argtypes = [_i, _i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p, _p]
 _lib.orc_combine_wgrad.restype = C.c_uint32
 _lib.orc_combine_wgrad.argtypes = [_i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p]
+_lib.orc_combine_wgrad_gathered.restype = None
+_lib.orc_combine_wgrad_gathered.argtypes = [_l, _i, _i, _p, _p, _p, _p, _p]
 _lib.orc_bwd_row.restype = None
 _lib.orc_bwd_row.argtypes = [_i, _f, _i, _p, _p, _p]
 _lib.orc_combine_gathered.restype = None
@@ -316,6 +318,19 @@ def combine_wgrad(R, T, K, E, M, H, g, y, topk_idx, token_slot, expert_offset=No
     st = _lib.orc_combine_wgrad(R, T, K, E, M, H, _layout(layout), _ptr(g), _ptr(y), _ptr(idx),
                                 _ptr(slot), _ptr(eo), _ptr(dw))
     return dw, int(st)
+
+
+def combine_wgrad_gathered(g, yrows, valid):
+    """g [N, H], yrows [N, K, H] bf16 bits, valid [N, K] -> (dw [N, K] f32,
+    sum_h |g * y| [N, K] f64)."""
+    yrows = _c(yrows, np.uint16)
+    N, K, H = yrows.shape
+    g = _c(g, np.uint16).reshape(N, H)
+    v = _c(valid, np.uint8)
+    dw = np.zeros((N, K), np.float32)
+    mag = np.zeros((N, K), np.float64)
+    _lib.orc_combine_wgrad_gathered(N, K, H, _ptr(g), _ptr(yrows), _ptr(v), _ptr(dw), _ptr(mag))
+    return dw, mag
 
 
 def combine_gathered(yrows, w, valid):

@@ -551,6 +551,29 @@ uint32_t orc_combine_wgrad(int R, int T, int K, int E, int M, int H, int layout,
     return st;
 }
 
+/* The same for tokens whose K expert rows are gathered: g [N][H], yrows
+ * [N][K][H], valid [N][K] -> dw [N][K]; also sum_h |g*y| per entry (the
+ * scale of the rounding error of any fp32 summation order) in absdot. */
+void orc_combine_wgrad_gathered(long N, int K, int H, const uint16_t *g, const uint16_t *yrows,
+                                const uint8_t *valid, float *dw, double *absdot)
+{
+    for (long n = 0; n < N; n++) {
+        for (int k = 0; k < K; k++) {
+            double acc = 0.0, mag = 0.0;
+            if (valid[n * K + k]) {
+                const uint16_t *y = yrows + (n * K + k) * (long)H;
+                for (int h = 0; h < H; h++) {
+                    double p = (double)orc_bf16_to_f32(g[n * H + h]) * (double)orc_bf16_to_f32(y[h]);
+                    acc += p;
+                    mag += fabs(p);
+                }
+            }
+            dw[n * K + k] = (float)acc;
+            absdot[n * K + k] = mag;
+        }
+    }
+}
+
 /*
  * Dequantisation of one row stored in a quantised format ([FP8] The FP8
  * Combine Operation: the received codes times the stored inverse scale, in

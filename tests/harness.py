@@ -171,6 +171,42 @@ class Run:
         assert worst <= max_ulp, worst
         return worst
 
+    def check_weights_grad(self, tokens=None, g=None):
+        """Weight gradient on the GPU against the oracle: within 128 * 2^-24 *
+        sum_h |g*y| of the exact dot product (any fp32 summation order of at
+        most ~80 additions per term stays inside it), masked entries 0."""
+        w, b = self.w, self.b
+        K, H = w["K"], w["H"]
+        if g is None:
+            gp, go = synth.g_source(w)
+            g = synth.windows(gp, go, H)
+        g_d = bf16_dev(g)
+        dw = torch.full((w["N"], K), float("nan"), dtype=torch.float32, device="cuda")
+        ep.ep_combine_backward_weights(self.cfg, g_d, b.y, self.idx_d, b.token_slot, dw,
+                                       b.dev_status, expert_offset=b.expert_offset)
+        assert ep.ep_get_status(b.dev_status) == self.status
+        tokens = np.arange(w["N"]) if tokens is None else np.asarray(tokens)
+        got = dw.cpu().numpy()[tokens]
+        worst = 0.0
+        for a in range(0, len(tokens), 256):
+            tk = tokens[a:a + 256]
+            yr = np.zeros((len(tk), K, H), np.uint16)
+            valid = np.zeros((len(tk), K), np.uint8)
+            ns, ks, rows = self.entries(tk)
+            pos = {n: i for i, n in enumerate(tk)}
+            if len(rows):
+                ys = self.y_rows_host(rows)
+                for j, (n, k) in enumerate(zip(ns, ks)):
+                    yr[pos[n], k] = ys[j]
+                    valid[pos[n], k] = 1
+            want, mag = oracle.combine_wgrad_gathered(g[tk], yr, valid)
+            err = np.abs(got[a:a + 256].astype(np.float64) - want.astype(np.float64))
+            bound = 128 * 2.0 ** -24 * mag + np.abs(want.astype(np.float64)) * 2.0 ** -24
+            assert np.all(err <= bound), float((err - bound).max())
+            assert np.all(got[a:a + 256][valid == 0] == 0.0)
+            worst = max(worst, float((err / np.maximum(mag, 1e-300)).max()) if err.size else 0.0)
+        return worst
+
     def check_backward(self, tokens=None):
         w, b = self.w, self.b
         H = w["H"]

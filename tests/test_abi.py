@@ -112,6 +112,9 @@ def test_entry_points_reject_before_any_launch():
     assert lib.ep_dispatch(C.byref(cfg), *([null] * 10)) == 1
     assert lib.ep_combine(C.byref(cfg), *([null] * 8)) == 1
     assert lib.ep_combine_backward(C.byref(cfg), *([null] * 8)) == 1
+    assert lib.ep_combine_backward_weights(C.byref(cfg), *([null] * 8)) == 1
+    qcfg = _cfg(quant="mxfp8", flags=ep.F_COMBINE_QUANTIZED)
+    assert lib.ep_combine_backward_weights(C.byref(qcfg), *([C.c_void_p(0x1000)] * 7), null) == 2
     assert lib.ep_get_status(null, None, null) == 1
     bad = _cfg(E=255)
     fake = C.c_void_p(0x1000)

@@ -502,3 +502,61 @@ def test_backward_special_weights():
     ep.ep_combine_backward(r.cfg, r.g_d, r.idx_d, r.wts_d, r.b.token_slot, r.b.grad_buf,
                            r.b.dev_status, expert_offset=r.b.expert_offset)
     r.check_backward()
+
+
+# ---------------------------------------------------------------------------
+# weight gradient of the combine
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("name,override,layout", [
+    ("decode", {}, "padded"), ("tiny", {}, "padded"), ("skewed", dict(T=64), "padded"),
+    ("prefill", dict(T=40), "packed"), ("large", dict(T=24), "packed")])
+def test_weights_grad(name, override, layout):
+    w = synth.workload(name, **override)
+    r = Run(w, "bf16", layout=layout)
+    r.check_weights_grad()
+
+
+def test_weights_grad_ragged_masked_bad_and_int32():
+    w = _edge(R=3, T=13, M=16, K=5, E=12, H=608)
+    idx, wts = synth.make_routing(w)
+    idx[2, :] = -1
+    idx[4, 1] = w["E"] + 1
+    r = Run(w, "bf16", layout="packed", align=3, idx=idx, wts=wts, flags=ep.F_IDX_I32)
+    assert r.status & ep.DEV_BAD_INDEX
+    r.check_weights_grad()
+
+
+def test_weights_grad_rejects_quantized_outputs():
+    w = _edge()
+    cfg = ep.make_config(w["R"], w["T"], w["M"], w["K"], w["E"], w["H"], "mxfp8",
+                         flags=ep.F_COMBINE_QUANTIZED)
+    b = ep.Buffers(cfg)
+    g = torch.zeros((w["N"], w["H"]), dtype=torch.bfloat16, device="cuda")
+    idx = torch.zeros((w["N"], w["K"]), dtype=torch.int64, device="cuda")
+    dw = torch.zeros((w["N"], w["K"]), dtype=torch.float32, device="cuda")
+    with pytest.raises(ep.EpError) as ei:
+        ep.ep_combine_backward_weights(cfg, g, b.y, idx, b.token_slot, dw, b.dev_status)
+    assert ei.value.status == 2
+
+
+def test_variable_tokens_per_rank_by_masking():
+    """Ranks with different token counts T_r <= M ("Low-Latency Mode API",
+    low_latency_combine: num_combined_tokens is the rank's dispatched token
+    count): the ranks share T = max T_r and the missing tokens' topk_idx rows
+    are -1.  They then take no slot, count nowhere, and combine to +0."""
+    w = _edge(R=3, T=13, M=16, K=4, E=12, H=256)
+    t_r = [13, 5, 0]
+    idx, wts = synth.make_routing(w)
+    for r, tr in enumerate(t_r):
+        idx[r * w["T"] + tr:(r + 1) * w["T"]] = -1
+    r = Run(w, "e4m3_b128", layout="packed", idx=idx, wts=wts, backward=True)
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+    r.check_backward()
+    out = r.b.out.view(torch.int16).cpu().numpy()
+    for rr, tr in enumerate(t_r):
+        assert np.all(out[rr * w["T"] + tr:(rr + 1) * w["T"]] == 0)
+    tpr = r.b.tokens_per_rank.cpu().numpy()
+    assert list(tpr.sum(axis=1) >= 0) and tpr[2].sum() == 0
+    assert r.b.recv_count.sum().item() == int((idx >= 0).sum())

@@ -801,3 +801,18 @@ def test_wgrad_flags_bad_indices():
     dw, st = oracle.combine_wgrad(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], g, y, bad,
                                   lay["token_slot"], lay["expert_offset"])
     assert st & oracle.ST_BAD_INDEX and dw[0, 0] == 0.0
+
+
+def test_wgrad_gathered_equals_the_layout_form():
+    w, idx, lay, y, g = _wgrad_case("packed", 2, seed=7)
+    dw, _ = oracle.combine_wgrad(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], g, y, idx,
+                                 lay["token_slot"], lay["expert_offset"], layout="packed")
+    yr = np.zeros((w["N"], w["K"], w["H"]), np.uint16)
+    valid = idx >= 0
+    for n, k in zip(*np.nonzero(valid)):
+        row = int(oracle.row_index("packed", w["R"], w["M"], idx[n, k], lay["token_slot"][n, k],
+                                   lay["expert_offset"]))
+        yr[n, k] = y[row]
+    dg, mag = oracle.combine_wgrad_gathered(g, yr, valid)
+    assert np.array_equal(dg, dw)
+    assert np.all(mag >= np.abs(dg)) and np.all(mag[~valid] == 0)
