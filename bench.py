@@ -433,6 +433,9 @@ def main():
     ms_per_step = total_ms / args.steps
     value = world * N * args.steps / (total_ms / 1e3)
 
+    graph = graph_steps(ep, args, cfg, ccfg, b, x_d, idx_d, wts_d, g_d, flush, stream, dev, N,
+                        world)
+
     # per-kernel durations (for the roofline): the same steps again, each
     # kernel after its own flush and between its own pair of events
     evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -539,6 +542,7 @@ def main():
                      "isolated_launch": {"achieved": round(iso_achieved, 1),
                                          "frac": round(iso_achieved / peak, 4)}},
         "kernels": kstats,
+        "graph": graph,
         "copy_gbs_same_run": copy_gbs,
         "e2e": e2e,
     }
@@ -547,6 +551,56 @@ def main():
     if rank == 0:
         print(json.dumps(out), flush=True)
     dist_done(world)
+
+
+def graph_steps(ep, args, cfg, ccfg, b, x_d, idx_d, wts_d, g_d, flush, stream, dev, N, world):
+    """The timed step captured once in a CUDA graph and replayed, with the same
+    flush and event protocol: the step without the host's per-launch work (the
+    device-side gaps between the kernels remain).  None if capture fails."""
+    try:
+        gs = torch.cuda.Stream(dev)
+        gcalls = [
+            ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
+                                       b.recv_buf, b.src_info, b.dev_status,
+                                       expert_offset=b.expert_offset, stream=gs, bind=True),
+            ep.ep_combine(ccfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
+                          expert_offset=b.expert_offset, stream=gs, bind=True),
+        ]
+        if g_d is not None:
+            gcalls.append(ep.ep_combine_backward(cfg, g_d, idx_d, wts_d, b.token_slot,
+                                                 b.grad_buf, b.dev_status,
+                                                 expert_offset=b.expert_offset, stream=gs,
+                                                 bind=True))
+        gs.wait_stream(stream)
+        for c in gcalls:  # warm, outside capture
+            c()
+        stream.wait_stream(gs)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=gs):
+            for c in gcalls:
+                c()
+        torch.cuda.synchronize(dev)
+        for _ in range(3):
+            flush(1)
+            graph.replay()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        for s in range(args.steps):
+            flush(s & 0xFF)
+            evs[s][0].record(stream)
+            graph.replay()
+            evs[s][1].record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(world)
+        total = max_over_ranks(sum(a.elapsed_time(c) for a, c in evs), world)
+        del graph
+        return {"ms_per_step": round(total / args.steps, 5),
+                "value": round(world * N * args.steps / (total / 1e3), 1), "unit": "tokens/s"}
+    except Exception as e:  # report, do not fail the bench
+        return {"unavailable": f"{type(e).__name__}: {str(e).splitlines()[0][:120]}"}
 
 
 STEADY_SETS = 4

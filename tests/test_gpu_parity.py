@@ -558,5 +558,5 @@ def test_variable_tokens_per_rank_by_masking():
     for rr, tr in enumerate(t_r):
         assert np.all(out[rr * w["T"] + tr:(rr + 1) * w["T"]] == 0)
     tpr = r.b.tokens_per_rank.cpu().numpy()
-    assert list(tpr.sum(axis=1) >= 0) and tpr[2].sum() == 0
+    assert tpr[1].max() <= t_r[1] and tpr[2].sum() == 0
     assert r.b.recv_count.sum().item() == int((idx >= 0).sum())
