@@ -560,3 +560,39 @@ def test_variable_tokens_per_rank_by_masking():
     tpr = r.b.tokens_per_rank.cpu().numpy()
     assert tpr[1].max() <= t_r[1] and tpr[2].sum() == 0
     assert r.b.recv_count.sum().item() == int((idx >= 0).sum())
+
+
+# ---------------------------------------------------------------------------
+# K = 16 (the largest top-k) and the quantised combine's fallback kernel
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("mode", ["bf16", "int8_token", "e4m3_b128", "mxfp8", "mxfp4"])
+def test_k16_every_mode(mode):
+    w = _edge(R=4, T=21, M=24, K=16, E=32, H=640)
+    r = Run(w, mode, layout="packed", align=2, backward=True)
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
+    r.check_backward()
+    if mode == "bf16":
+        r.check_weights_grad()
+
+
+@pytest.mark.parametrize("mode,flags", [("int8_token", 0), ("e4m3_b128", 0),
+                                        ("e4m3_b128", ep.F_UE8M0), ("mxfp8", 0), ("mxfp4", 0)])
+def test_quantized_combine_k_above_eight(mode, flags):
+    """K > 8 takes the one-stage kernel (the pipelined one holds 8 rows)."""
+    from harness import combine_quantized_check, special_quantized_rows
+    w = _edge(R=4, T=21, M=24, K=12, E=32, H=640)
+    r = Run(w, mode, layout="packed", flags=flags)
+    combine_quantized_check(r, seed=21)
+    combine_quantized_check(r, seed=22, rows_fn=special_quantized_rows)
+
+
+@pytest.mark.parametrize("mode", ["mxfp8", "mxfp4"])
+def test_quantized_combine_unaligned_scale_rows(mode):
+    """H = 96 gives 3-byte MX scale rows: the one-stage kernel."""
+    from harness import combine_quantized_check
+    w = _edge(R=2, T=9, M=12, K=4, E=8, H=96 if mode == "mxfp8" else 224)
+    r = Run(w, mode, layout="packed")
+    assert r.sizes["scale_row_bytes"] % 4 != 0
+    combine_quantized_check(r, seed=23)
