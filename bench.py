@@ -299,6 +299,51 @@ def cpu_baseline(w, mode, idx, wts, x, seconds, replica=0):
             "sample": f"{st.sample}; {reps} steps in {el:.1f} s, single thread"}
 
 
+def _oracle_worker(job, barrier, results):
+    """One independent oracle instance (a spawned process): the seeded inputs
+    rebuilt here and one warm-up step, then, after every instance has reached
+    the barrier, steps for `seconds`."""
+    wname, t_override, mode, replica, sub_t, seconds = job
+    w = synth.workload(wname) if t_override is None else synth.workload(wname, T=t_override)
+    idx, wts = synth.make_routing(w, replica)
+    x = synth.make_x(w, replica)
+    st = OracleStep(w, mode, idx, wts, x, sub_t=sub_t, replica=replica)
+    st.step()
+    barrier.wait(timeout=600)
+    t0 = time.perf_counter()
+    done = 0
+    while True:
+        done += st.step()
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    results.put((done, el))
+
+
+def cpu_baseline_all_cores(wname, t_override, mode, seconds, replica=0):
+    """The oracle on the host's cores (up to 32): as many independent instances as cores
+    (spawned processes, each on a sample of T/8 tokens per rank), released
+    together by a barrier and timed over the same interval; tokens/s summed."""
+    import multiprocessing as mp
+    ctx = mp.get_context("spawn")
+    cores = min(os.cpu_count() or 1, 32)  # each instance is a process with its own imports
+    w = synth.workload(wname) if t_override is None else synth.workload(wname, T=t_override)
+    sub_t = max(1, w["T"] // 8)
+    barrier, results = ctx.Barrier(cores), ctx.Queue()
+    job = (wname, t_override, mode, replica, sub_t, seconds)
+    procs = [ctx.Process(target=_oracle_worker, args=(job, barrier, results)) for _ in range(cores)]
+    for pr in procs:
+        pr.start()
+    res = [results.get(timeout=900) for _ in procs]
+    for pr in procs:
+        pr.join(timeout=60)
+    total = sum(d for d, _ in res)
+    el = max(e for _, e in res)
+    return {"value": total / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{cores} independent instances, each the first {sub_t} of {w['T']} tokens "
+                      f"of each of the {w['R']} ranks, started together; {seconds:.0f} s, summed"}
+
+
 # ---------------------------------------------------------------------------
 def main():
     args = parse()
@@ -548,6 +593,11 @@ def main():
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(w, mode, idx, wts, x, args.cpu_seconds, replica)
+        try:
+            out["cpu_baseline_all_cores"] = cpu_baseline_all_cores(
+                wname, args.tokens_per_rank, mode, args.cpu_seconds, replica)
+        except Exception as e:  # a host without process support: report, do not fail
+            out["cpu_baseline_all_cores"] = {"unavailable": f"{type(e).__name__}: {e}"[:160]}
     if rank == 0:
         print(json.dumps(out), flush=True)
     dist_done(world)
