@@ -12,6 +12,7 @@ more modes are e4m3_b128 with the scale options: e4m3_b128_p2 (round_scale:
 power-of-two fp32 scales) and e4m3_b128_ue8m0 (the same as e8m0 bytes).
 """
 import ctypes as C
+import os
 
 import numpy as np
 
@@ -23,7 +24,9 @@ LAYOUTS = {"padded": 0, "packed": 1}
 ST_BAD_INDEX = 0x1
 ST_CAPACITY = 0x2
 
-_lib = C.CDLL(_build.build())
+# EP_ORACLE_LIB names another build of ep_oracle.c (the mutation tests load
+# copies with planted mistakes through it); normally the library is built here.
+_lib = C.CDLL(os.environ.get("EP_ORACLE_LIB") or _build.build())
 
 _p = C.c_void_p
 _i = C.c_int

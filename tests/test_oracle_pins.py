@@ -119,6 +119,16 @@ def test_decoders_invert_encoders_on_every_code():
         assert oracle.e2m1_encode(np.float32([v]))[0] == c
 
 
+def test_decoders_give_nan_for_the_e4m3_nan_codes():
+    dec = oracle.e4m3_decode(np.uint8([0x7F, 0xFF, 0x7E, 0xFE]))
+    assert np.isnan(dec[0]) and np.isnan(dec[1]) and list(dec[2:]) == [448.0, -448.0]
+    # and the combine of a row holding one turns that element into NaN only
+    d = np.zeros(32, np.uint8)
+    d[[0, 5]] = [0x7F, 0x38]                       # NaN, 1.0
+    y = oracle.dequant_row("mxfp8", d, np.uint8([127]), 32)
+    assert np.isnan(y[0]) and y[5] == 1.0 and np.all(y[[1, 2, 3, 4]] == 0)
+
+
 def test_bf16_rounding_matches_torch():
     x = np.concatenate([_random_f32(1_000_000, -130, 127),
                         # exact ties: low half 0x8000 with even and odd kept bit
@@ -395,8 +405,10 @@ def _run_layout(w, idx, layout, align=1):
 
 
 @pytest.mark.parametrize("layout,align", [("padded", 1), ("packed", 1), ("packed", 8)])
-def test_dispatch_bf16_is_an_exact_scatter(layout, align):
-    w, idx, wt, x = _small("tiny")
+@pytest.mark.parametrize("shape", [{}, dict(R=4, T=5, M=8, K=3, E=8, H=64)],
+                         ids=["one-rank", "four-ranks"])
+def test_dispatch_bf16_is_an_exact_scatter(layout, align, shape):
+    w, idx, wt, x = _small("tiny", **shape)
     lay = _run_layout(w, idx, layout, align)
     out = oracle.dispatch(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], "bf16", x, idx,
                           lay["token_slot"], lay["expert_offset"], topk_weights=wt,
