@@ -336,20 +336,24 @@ template <int TPT, int GMAX>
 __global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(DispatchArgs a) {
     pdl_enter();
     constexpr int TOKS = block_threads(TPT) / TPT;
-    __shared__ int64_t s_row[TOKS][16];
-    __shared__ float s_w[TOKS][16];
+    static_assert(TPT >= 32, "a warp belongs to one token");
 
     const int grp = threadIdx.x / TPT, lt = threadIdx.x % TPT;
     const int64_t n = (int64_t)blockIdx.x * TOKS + grp;
     const bool active = n < a.N;
     const int ngran = a.H >> 4;
+    const int lane = lt & 31;
 
-    if (active && lt < a.K) {
+    // Every warp reads the token's entries itself (lane k holds entry k) and
+    // hands them out by shuffles: no block barrier stands between a warp's
+    // gradient loads and its stores.  The first warp reports the flags.
+    int64_t my_row = -1;
+    float my_w = 0.0f;
+    if (active && lane < a.K) {
         uint32_t flags = 0;
-        const int64_t row = entry_row(a, n, lt, flags);
-        if (flags) atomicOr(a.status, flags);
-        s_row[grp][lt] = row;
-        s_w[grp][lt] = a.unweighted ? 1.0f : a.wts[n * a.K + lt];
+        my_row = entry_row(a, n, lane, flags);
+        if (flags && lt < 32) atomicOr(a.status, flags);
+        my_w = a.unweighted ? 1.0f : a.wts[n * a.K + lane];
     }
 
     // the token's gradient row, unpacked to fp32 once for all its entries
@@ -394,14 +398,13 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(Dispatc
         const float fm = bf2_fold(gm[i]);
         gmax[i] = fmaxf(fm, __shfl_xor_sync(kFull, fm, 1));
     }
-    __syncthreads();
-    if (!active) return;
+    if (!active) return;  // a whole warp: tokens do not share warps
 
     const bool weighted = !a.unweighted;
     for (int k = 0; k < a.K; k++) {
-        const int64_t row = s_row[grp][k];
+        const int64_t row = __shfl_sync(kFull, my_row, k);
+        const float w = __shfl_sync(kFull, my_w, k);
         if (row < 0) continue;
-        const float w = s_w[grp][k];
         const float aw = fabsf(w);
         uint8_t *dst = a.out + row * (int64_t)a.H;
         uint8_t *sdst = a.out + a.scale_off + row * (int64_t)(a.H >> 5);
