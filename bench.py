@@ -606,7 +606,10 @@ def main():
 def graph_steps(ep, args, cfg, ccfg, b, x_d, idx_d, wts_d, g_d, flush, stream, dev, N, world):
     """The timed step captured once in a CUDA graph and replayed, with the same
     flush and event protocol: the step without the host's per-launch work (the
-    device-side gaps between the kernels remain).  None if capture fails."""
+    device-side gaps between the kernels remain).  Every rank takes the same
+    collective steps: the capture's outcome is agreed on first (a failure on
+    any rank reports it on all and times nothing)."""
+    graph, why = None, None
     try:
         gs = torch.cuda.Stream(dev)
         gcalls = [
@@ -631,26 +634,29 @@ def graph_steps(ep, args, cfg, ccfg, b, x_d, idx_d, wts_d, g_d, flush, stream, d
             for c in gcalls:
                 c()
         torch.cuda.synchronize(dev)
-        for _ in range(3):
-            flush(1)
-            graph.replay()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(args.steps)]
-        barrier(world)
-        torch.cuda.synchronize(dev)
-        for s in range(args.steps):
-            flush(s & 0xFF)
-            evs[s][0].record(stream)
-            graph.replay()
-            evs[s][1].record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(world)
-        total = max_over_ranks(sum(a.elapsed_time(c) for a, c in evs), world)
-        del graph
-        return {"ms_per_step": round(total / args.steps, 5),
-                "value": round(world * N * args.steps / (total / 1e3), 1), "unit": "tokens/s"}
     except Exception as e:  # report, do not fail the bench
-        return {"unavailable": f"{type(e).__name__}: {str(e).splitlines()[0][:120]}"}
+        graph, why = None, f"{type(e).__name__}: {str(e).splitlines()[0][:120]}" if str(e) else \
+            type(e).__name__
+    if max_over_ranks(0.0 if graph is not None else 1.0, world) > 0.0:
+        return {"unavailable": why or "capture failed on another rank"}
+    for _ in range(3):
+        flush(1)
+        graph.replay()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    for s in range(args.steps):
+        flush(s & 0xFF)
+        evs[s][0].record(stream)
+        graph.replay()
+        evs[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    total = max_over_ranks(sum(a.elapsed_time(c) for a, c in evs), world)
+    del graph
+    return {"ms_per_step": round(total / args.steps, 5),
+            "value": round(world * N * args.steps / (total / 1e3), 1), "unit": "tokens/s"}
 
 
 STEADY_SETS = 4
