@@ -69,6 +69,8 @@ _lib.orc_combine_wgrad.restype = C.c_uint32
 _lib.orc_combine_wgrad.argtypes = [_i, _i, _i, _i, _i, _i, _i, _p, _p, _p, _p, _p, _p]
 _lib.orc_combine_wgrad_gathered.restype = None
 _lib.orc_combine_wgrad_gathered.argtypes = [_l, _i, _i, _p, _p, _p, _p, _p]
+_lib.orc_expert_gemm.restype = None
+_lib.orc_expert_gemm.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p]
 _lib.orc_bwd_row.restype = None
 _lib.orc_bwd_row.argtypes = [_i, _f, _i, _p, _p, _p]
 _lib.orc_combine_gathered.restype = None
@@ -334,6 +336,22 @@ def combine_wgrad_gathered(g, yrows, valid):
     mag = np.zeros((N, K), np.float64)
     _lib.orc_combine_wgrad_gathered(N, K, H, _ptr(g), _ptr(yrows), _ptr(v), _ptr(dw), _ptr(mag))
     return dw, mag
+
+
+def expert_gemm(x, w, expert_offset, count, n_out, y=None):
+    """Per-expert linear maps on packed rows: x [rows, H] bf16 bits, w [E, n_out, H]
+    bf16 bits; rows expert_offset[e] .. + count[e] -> y [rows, n_out] bf16 bits
+    (other rows of y untouched)."""
+    x = _c(x, np.uint16)
+    rows, H = x.shape
+    w = _c(w, np.uint16)
+    E = w.shape[0]
+    eo = _c(expert_offset, np.int64)
+    cnt = _c(count, np.int64)
+    if y is None:
+        y = np.zeros((rows, n_out), np.uint16)
+    _lib.orc_expert_gemm(E, H, n_out, _ptr(eo), _ptr(cnt), _ptr(x), _ptr(w), _ptr(y))
+    return y
 
 
 def combine_gathered(yrows, w, valid):

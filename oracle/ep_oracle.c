@@ -575,6 +575,33 @@ void orc_combine_wgrad_gathered(long N, int K, int H, const uint16_t *g, const u
 }
 
 /*
+ * The experts between dispatch and combine (SURVEY NEXT-4 stand-in: each
+ * expert a single linear map, as the deep-fused MoE operator of "[feat] A5
+ * deep fused moe supported" runs grouped matrix multiplications between its
+ * dispatch and combine): for every expert e and each of its rows r (rows
+ * expert_offset[e] .. + count[e] of the packed receive layout),
+ *   y[r, j] = bf16_rne( sum_h x[r, h] * w[e, j, h] ),  j < Nout,
+ * the products exact in double, summed in double in h order, rounded to
+ * fp32 and then to bf16.  Rows past count[e] are left untouched.
+ */
+void orc_expert_gemm(int E, int H, int Nout, const int64_t *expert_offset, const int64_t *count,
+                     const uint16_t *x, const uint16_t *w, uint16_t *y)
+{
+    for (int e = 0; e < E; e++) {
+        for (int64_t i = 0; i < count[e]; i++) {
+            int64_t r = expert_offset[e] + i;
+            for (int j = 0; j < Nout; j++) {
+                const uint16_t *wr = w + ((int64_t)e * Nout + j) * H;
+                double acc = 0.0;
+                for (int h = 0; h < H; h++)
+                    acc += (double)orc_bf16_to_f32(x[r * H + h]) * (double)orc_bf16_to_f32(wr[h]);
+                y[r * Nout + j] = orc_f32_to_bf16((float)acc);
+            }
+        }
+    }
+}
+
+/*
  * Dequantisation of one row stored in a quantised format ([FP8] The FP8
  * Combine Operation: the received codes times the stored inverse scale, in
  * fp32).  Each element is decode(code) * scale_inv as

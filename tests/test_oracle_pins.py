@@ -828,3 +828,42 @@ def test_wgrad_gathered_equals_the_layout_form():
     dg, mag = oracle.combine_wgrad_gathered(g, yr, valid)
     assert np.array_equal(dg, dw)
     assert np.all(mag >= np.abs(dg)) and np.all(mag[~valid] == 0)
+
+
+# ---------------------------------------------------------------------------
+# the experts between dispatch and combine: per-expert linear maps
+# ---------------------------------------------------------------------------
+
+def test_expert_gemm_identity_weights_copy_the_rows():
+    r = np.random.default_rng(1)
+    E, H = 3, 64
+    cnt = np.array([5, 0, 7], np.int64)
+    eo = np.array([0, 8, 8, 16], np.int64)
+    x = synth.to_bf16_bits(r.standard_normal((16, H)).astype(np.float32))
+    w = np.zeros((E, H, H), np.uint16)
+    one = synth.to_bf16_bits(np.float32([1.0]))[0]
+    for e in range(E):
+        w[e][np.arange(H), np.arange(H)] = one
+    y = oracle.expert_gemm(x, w, eo[:E], cnt, H, y=np.full((16, H), 0x7777, np.uint16))
+    for e in range(E):
+        assert np.array_equal(y[eo[e]:eo[e] + cnt[e]], x[eo[e]:eo[e] + cnt[e]])
+    assert np.all(y[5:8] == 0x7777) and np.all(y[15] == 0x7777)   # rows past count untouched
+
+
+def test_expert_gemm_equals_exact_rational_products():
+    from fractions import Fraction
+    r = np.random.default_rng(2)
+    E, H, N = 2, 32, 8
+    cnt = np.array([3, 2], np.int64)
+    eo = np.array([0, 4], np.int64)
+    x = synth.to_bf16_bits((r.integers(-64, 64, (6, H)) / 16.0).astype(np.float32))
+    w = synth.to_bf16_bits((r.integers(-64, 64, (E, N, H)) / 64.0).astype(np.float32))
+    y = oracle.expert_gemm(x, w, eo, cnt, N)
+    xf, wf = _f(x), _f(w)
+    for e in range(E):
+        for i in range(cnt[e]):
+            row = eo[e] + i
+            for j in range(N):
+                exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(xf[row], wf[e, j]))
+                want = synth.to_bf16_bits(np.float32([float(exact)]))[0]
+                assert y[row, j] == want, (e, i, j)
