@@ -11,6 +11,7 @@
 #include "ep_combine.cuh"
 #include "ep_device.cuh"
 #include "ep_dispatch.cuh"
+#include "ep_gemm.cuh"
 #include "ep_layout.cuh"
 
 namespace {
@@ -804,6 +805,74 @@ ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *
     EP_SPLITS(EP_CASE)
 #undef EP_CASE
     return EP_ERR_UNSUPPORTED;
+}
+
+// ---- the experts between dispatch and combine -----------------------------------
+namespace {
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                 const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                 const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link to
+// the driver library)
+EncodeTiled encode_tiled() {
+    static EncodeTiled fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiled>(p);
+    });
+    return fn;
+}
+
+// bf16 matrix [outer][inner] (rows of `inner` elements), tiles of 64 x 128,
+// 128-byte swizzle (the layout the kernel's matrix descriptors describe)
+bool bf16_tile_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer) {
+    const EncodeTiled enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner * 2};
+    const cuuint32_t box[2] = {(cuuint32_t)ep::kGemmBK, (cuuint32_t)ep::kGemmBM};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+}  // namespace
+
+ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
+                           const int64_t *expert_offset, const int64_t *recv_count,
+                           const uint16_t *weights, int32_t n_out, uint16_t *y,
+                           uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (cfg->quant != EP_Q_BF16 || cfg->layout != EP_LAYOUT_PACKED) return EP_ERR_UNSUPPORTED;
+    if (p.H % ep::kGemmBK != 0) return EP_ERR_UNSUPPORTED;
+    if (n_out < ep::kGemmBN || n_out % ep::kGemmBN != 0) return EP_ERR_INVALID_ARG;
+    if ((int64_t)n_out * p.E > kIntLimit || p.E > ep::kGemmMaxExperts) return EP_ERR_INVALID_ARG;
+    if (!recv_buf || !expert_offset || !recv_count || !weights || !y || !dev_status)
+        return EP_ERR_INVALID_ARG;
+    if (!aligned16(recv_buf) || !aligned16(weights) || !aligned16(y)) return EP_ERR_MISALIGNED;
+    if (p.N == 0) return EP_OK;
+
+    CUtensorMap ma, mb;
+    if (!bf16_tile_map(&ma, recv_buf, (uint64_t)p.H, (uint64_t)p.rows) ||
+        !bf16_tile_map(&mb, weights, (uint64_t)p.H, (uint64_t)p.E * n_out))
+        return EP_ERR_CUDA;
+    ep::GemmArgs a;
+    a.E = p.E; a.H = p.H; a.N = n_out; a.ntn = n_out / ep::kGemmBN;
+    a.eo = expert_offset; a.cnt = recv_count; a.y = y; a.status = dev_status;
+    const size_t smem = ep::gemm_smem_bytes();
+    if (!allow_smem(ep::expert_gemm_kernel, 5, smem)) return EP_ERR_CUDA;
+    launch(ep::expert_gemm_kernel, (unsigned)sm_count(), ep::kGemmThreads, smem, cs(stream), ma,
+           mb, a);
+    return launched();
 }
 
 ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream) {

@@ -1,0 +1,348 @@
+// ep_gemm.cuh -- the experts between dispatch and combine: a grouped bf16
+// matrix multiplication on the fifth-generation tensor cores.
+//
+// "[feat] A5 deep fused moe supported" runs grouped matrix multiplications of
+// the experts between its dispatch and its combine.  Here each expert e is one
+// linear map W_e [N][H]: for the rows r of expert e in the packed receive
+// layout (expert_offset[e] .. + count[e]),
+//   y[r, :] = bf16_rne( x[r, :] . W_e^T ),  fp32 accumulation.
+//
+// Tiles of 128 rows x 128 columns, 64-element K steps.  A persistent grid
+// (one block per SM) walks the tiles of all experts; in each block
+//   warp 0        loads A and B K-steps with TMA (128-byte swizzle) into a
+//                 ring of kGemmStages shared-memory stages;
+//   warp 1        allocates 2 x 128 TMEM columns (two fp32 accumulators) and
+//                 one lane issues tcgen05.mma (cta_group::1, kind::f16, M=128,
+//                 N=128, K=16 per instruction), committing each stage back to
+//                 the loader and each finished accumulator to the epilogue;
+//   warps 2 - 5   read the accumulator rows (tcgen05.ld, one TMEM lane
+//                 quarter per warp), round to bf16 and store the tile's valid
+//                 rows, then hand the accumulator back.
+// Every wait on an mbarrier gives up after 2 s of %globaltimer: the block then
+// records kDevTimeout in the status word, drains its copies and MMAs in
+// flight (with the same bound), frees its TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+
+#include "ep_device.cuh"
+
+namespace ep {
+
+constexpr int kGemmBM = 128, kGemmBN = 128, kGemmBK = 64, kGemmStages = 4;
+constexpr int kGemmThreads = 192;
+constexpr uint32_t kDevTimeout = 0x4u;
+constexpr int kGemmTileBytesA = kGemmBM * kGemmBK * 2;  // 16 KB
+constexpr int kGemmTileBytesB = kGemmBN * kGemmBK * 2;  // 16 KB
+constexpr int kGemmMaxExperts = 1024;
+
+struct GemmArgs {
+    int E, H, N;
+    int ntn;                 // N / kGemmBN
+    const int64_t *eo;       // [E+1] first row of each expert (packed layout)
+    const int64_t *cnt;      // [E] rows of each expert
+    uint16_t *y;             // [rows][N] bf16
+    uint32_t *status;
+};
+
+// dynamic shared memory: stages (1024-byte aligned for the swizzle), then the
+// barriers, the TMEM base, an abort flag and the per-expert tile prefix
+__host__ __device__ constexpr size_t gemm_smem_bytes() {
+    return 1024 + (size_t)kGemmStages * (kGemmTileBytesA + kGemmTileBytesB) +
+           (2 * kGemmStages + 5) * 8 + 16 + (kGemmMaxExperts + 1) * 4 + 256;
+}
+
+__device__ __forceinline__ uint64_t gtimer() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+// true once the phase of parity `parity` has completed; false after 2 s
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    const uint64_t t0 = gtimer();
+#pragma unroll 1
+    while (true) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (gtimer() - t0 > 2000000000ull) return false;
+    }
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
+                                            uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+// shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
+// 1024 bytes apart (leading offset 1, stride offset 64 in 16-byte units,
+// descriptor version 1, layout type 2)
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1 << 16) | ((uint64_t)64 << 32) |
+           ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+// instruction descriptor: fp32 accumulator, bf16 A and B, both K-major, N, M
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_bf16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+    // the registers are operands of the wait, so no use moves above it
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                   "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                   "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15])
+                 :
+                 : "memory");
+}
+
+// tile t of the walk -> expert, first row and first column (t < prefix[E])
+__device__ __forceinline__ void gemm_tile(const int *prefix, int E, int ntn, int t, int &e,
+                                          int &m0, int &n0) {
+    int lo = 0, hi = E - 1;  // the last e with prefix[e] <= t
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    e = lo;
+    const int local = t - prefix[e];
+    m0 = (local / ntn) * kGemmBM;
+    n0 = (local % ntn) * kGemmBN;
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    expert_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
+                       const __grid_constant__ CUtensorMap tm_b, GemmArgs a) {
+    extern __shared__ uint8_t gsm_raw[];
+    uint8_t *gsm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = gsm;
+    uint8_t *sB = gsm + kGemmStages * kGemmTileBytesA;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + kGemmStages * kGemmTileBytesB);
+    uint64_t *full = bars, *empty = bars + kGemmStages;
+    uint64_t *accfull = bars + 2 * kGemmStages, *accempty = accfull + 2;
+    uint64_t *drain = accempty + 2;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile uint32_t *s_abort = s_tmem + 1;
+    int *prefix = reinterpret_cast<int *>(s_tmem + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = a.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kGemmStages; s++) {
+            mbar_init(smem_addr(&full[s]), 1);
+            mbar_init(smem_addr(&empty[s]), 1);
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(smem_addr(&accfull[b]), 1);
+            mbar_init(smem_addr(&accempty[b]), 128);
+        }
+        mbar_init(smem_addr(drain), 1);
+        *s_abort = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {  // the whole warp: 2 x kGemmBN columns
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(s_tmem)),
+                     "r"(2 * kGemmBN));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    pdl_enter();
+    if (warp == 0) {  // tiles per expert, exclusive prefix (one lane per run of experts)
+        const int per = (E + 31) / 32;
+        int sum = 0;
+        for (int i = 0; i < per; i++) {
+            const int e = lane * per + i;
+            if (e < E) sum += (int)((a.cnt[e] + kGemmBM - 1) / kGemmBM) * a.ntn;
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+        for (int i = 0; i < per; i++) {
+            const int e = lane * per + i;
+            if (e < E) {
+                prefix[e] = run;
+                run += (int)((a.cnt[e] + kGemmBM - 1) / kGemmBM) * a.ntn;
+            }
+        }
+        if (lane == 31) prefix[E] = incl;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const int total = prefix[E];
+    const int kblocks = a.H / kGemmBK;
+
+    if (warp == 0 && lane == 0) {
+        // ---- loader
+        int it = 0;
+        for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
+            int e, m0, n0;
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0);
+            const int arow = (int)a.eo[e] + m0, brow = e * a.N + n0;
+            for (int kb = 0; kb < kblocks; kb++, it++) {
+                const int s = it % kGemmStages, r = it / kGemmStages;
+                if (!mbar_wait(smem_addr(&empty[s]), (r & 1) ^ 1)) {
+                    *s_abort = 1u;
+                    atomicOr(a.status, kDevTimeout);
+                    break;
+                }
+                const uint32_t fb = smem_addr(&full[s]);
+                mbar_expect_tx(fb, kGemmTileBytesA + kGemmTileBytesB);
+                tma_load_2d(smem_addr(sA + s * kGemmTileBytesA), &tm_a, kb * kGemmBK, arow, fb);
+                tma_load_2d(smem_addr(sB + s * kGemmTileBytesB), &tm_b, kb * kGemmBK, brow, fb);
+            }
+        }
+        // copies still in flight land before the block can leave: wait for the
+        // last fill of every stage that was filled (bounded)
+        for (int j = 0; j < kGemmStages && j < it; j++) {
+            const int i2 = it - 1 - j, s = i2 % kGemmStages, r = i2 / kGemmStages;
+            if (!mbar_wait(smem_addr(&full[s]), r & 1)) atomicOr(a.status, kDevTimeout);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---- MMA issue
+        const uint32_t idesc = umma_idesc_bf16(kGemmBM, kGemmBN);
+        int it = 0, tc = 0;
+        for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x, tc++) {
+            const int acc = tc & 1, use = tc >> 1;
+            if (!mbar_wait(smem_addr(&accempty[acc]), (use & 1) ^ 1)) {
+                *s_abort = 1u;
+                atomicOr(a.status, kDevTimeout);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem_base + (uint32_t)(acc * kGemmBN);
+            bool ok = true;
+            for (int kb = 0; kb < kblocks; kb++, it++) {
+                const int s = it % kGemmStages, r = it / kGemmStages;
+                if (!mbar_wait(smem_addr(&full[s]), r & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t ad = umma_desc_sw128(smem_addr(sA + s * kGemmTileBytesA));
+                const uint64_t bd = umma_desc_sw128(smem_addr(sB + s * kGemmTileBytesB));
+#pragma unroll
+                for (int k = 0; k < kGemmBK / 16; k++)  // 16 elements = 32 bytes = 2 units
+                    umma_bf16(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+                umma_commit(smem_addr(&empty[s]));
+            }
+            if (!ok) {
+                *s_abort = 1u;
+                atomicOr(a.status, kDevTimeout);
+                break;
+            }
+            umma_commit(smem_addr(&accfull[acc]));
+        }
+    } else if (warp >= 2) {
+        // ---- epilogue: warp w reads TMEM lanes 32*(w % 4) ..
+        const int sub = warp & 3;
+        int tc = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, tc++) {
+            const int acc = tc & 1, use = tc >> 1;
+            // one decision for the whole warp: tcgen05.ld is warp-collective
+            const bool ok = __all_sync(kFull, !*s_abort && mbar_wait(smem_addr(&accfull[acc]), use & 1));
+            if (!ok) {
+                if (lane == 0) {
+                    *s_abort = 1u;
+                    atomicOr(a.status, kDevTimeout);
+                }
+                break;
+            }
+            tc_fence_after();
+            int e, m0, n0;
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0);
+            const int m = m0 + sub * 32 + lane;
+            const bool valid = m < a.cnt[e];
+            uint16_t *yrow = a.y + (a.eo[e] + m) * (int64_t)a.N + n0;
+            const uint32_t taddr = tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * kGemmBN);
+#pragma unroll 1
+            for (int c = 0; c < kGemmBN / 16; c++) {
+                uint32_t v[16];
+                tmem_ld16(taddr + c * 16, v);
+                if (valid) {
+                    uint4 lo, hi;
+                    lo.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
+                    lo.y = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
+                    lo.z = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
+                    lo.w = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
+                    hi.x = pack_bf16x2(__uint_as_float(v[8]), __uint_as_float(v[9]));
+                    hi.y = pack_bf16x2(__uint_as_float(v[10]), __uint_as_float(v[11]));
+                    hi.z = pack_bf16x2(__uint_as_float(v[12]), __uint_as_float(v[13]));
+                    hi.w = pack_bf16x2(__uint_as_float(v[14]), __uint_as_float(v[15]));
+                    st_v4(yrow + c * 16, lo);
+                    st_v4(yrow + c * 16 + 8, hi);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_addr(&accempty[acc]));
+        }
+    }
+    // every MMA this block issued has finished before the TMEM is freed: a
+    // last commit arrives on `drain` once they have (bounded wait)
+    if (warp == 1 && lane == 0 && total > (int)blockIdx.x) {
+        umma_commit(smem_addr(drain));
+        if (!mbar_wait(smem_addr(drain), 0)) atomicOr(a.status, kDevTimeout);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(2 * kGemmBN));
+    }
+}
+
+}  // namespace ep

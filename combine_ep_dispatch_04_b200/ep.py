@@ -79,6 +79,8 @@ lib.ep_combine.restype = C.c_int
 lib.ep_combine.argtypes = [_CFG] + [_P] * 8
 lib.ep_combine_backward.restype = C.c_int
 lib.ep_combine_backward.argtypes = [_CFG] + [_P] * 8
+lib.ep_expert_gemm.restype = C.c_int
+lib.ep_expert_gemm.argtypes = [_CFG, _P, _P, _P, _P, C.c_int32, _P, _P, _P]
 lib.ep_combine_backward_weights.restype = C.c_int
 lib.ep_combine_backward_weights.argtypes = [_CFG] + [_P] * 8
 lib.ep_get_status.restype = C.c_int
@@ -312,6 +314,28 @@ def ep_combine_backward(cfg, g, topk_idx, topk_weights, token_slot, grad_buf, de
         _stream(stream),
     ]
     return _call(lib.ep_combine_backward, cfg, args, "ep_combine_backward", bind)
+
+
+def ep_expert_gemm(cfg, recv_buf, expert_offset, recv_count, weights, y, dev_status, stream=None,
+                   bind=False):
+    """y[r] = bf16(x[r] . W[e]^T) for the rows of every expert (packed bf16 receive layout);
+    weights bf16 [E, n_out, H], y bf16 [rows, n_out]."""
+    sz = ep_buffer_sizes(cfg)
+    E, H = cfg.num_experts, cfg.hidden
+    if weights is None or weights.dim() != 3:
+        raise ValueError("weights must be a [E, n_out, H] tensor")
+    n_out = int(weights.shape[1])
+    args = [
+        _bytes(recv_buf, "recv_buf", sz["rows"] * sz["data_row_bytes"]),
+        _dev(expert_offset, "expert_offset", torch.int64, (E + 1,)),
+        _dev(recv_count, "recv_count", torch.int64, (E,)),
+        _dev(weights, "weights", torch.bfloat16, (E, n_out, H)),
+        C.c_int32(n_out),
+        _dev(y, "y", torch.bfloat16, (sz["rows"], n_out)),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    return _call(lib.ep_expert_gemm, cfg, args, "ep_expert_gemm", bind)
 
 
 def ep_combine_backward_weights(cfg, g, y, topk_idx, token_slot, topk_weights_grad, dev_status,

@@ -79,6 +79,7 @@ typedef enum {
 /* Bits of *dev_status. */
 #define EP_DEV_BAD_INDEX 0x1u         /* topk_idx value < -1 or >= E (entry skipped) */
 #define EP_DEV_CAPACITY_OVERFLOW 0x2u /* slot >= R*M in the padded layout (row skipped) */
+#define EP_DEV_TIMEOUT 0x4u           /* a bounded wait inside ep_expert_gemm gave up */
 
 /* ep_config_t.flags */
 #define EP_F_BWD_UNWEIGHTED 0x1u    /* combine-backward re-dispatches g without w */
@@ -261,6 +262,32 @@ ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *
                                         const int32_t *token_slot, const int64_t *expert_offset,
                                         float *topk_weights_grad, uint32_t *dev_status,
                                         ep_stream_t stream);
+
+/*
+ * The experts between dispatch and combine, each one linear map ("[feat] A5
+ * deep fused moe supported": grouped matrix multiplications of the experts run
+ * between the operator's dispatch and combine).  For each expert e and each of
+ * its received rows r (expert_offset[e] .. + recv_count[e] of the packed
+ * receive layout):
+ *   y[r, :] = bf16_rne( x[r, :] . W[e]^T )
+ * with fp32 accumulation on the tensor cores (tcgen05, 128 x 128 tiles);
+ * padding rows of y (past recv_count[e]) are not written.  The summation
+ * order of the fp32 accumulation is the hardware's: results are within
+ * 2^-20 * sum_h |x*w| + 1 bf16 ulp of the exact product.
+ *   cfg          quant EP_Q_BF16 and layout EP_LAYOUT_PACKED (the dispatch that
+ *                wrote recv_buf), H % 64 == 0; otherwise EP_ERR_UNSUPPORTED
+ *   recv_buf     the dispatch's receive buffer: bf16 [rows][H]
+ *   expert_offset, recv_count   from ep_dispatch_layout
+ *   weights      bf16 [E][n_out][H] (row j of W[e] is output column j)
+ *   n_out        output columns, a multiple of 128
+ *   y            bf16 [rows][n_out] (n_out = H gives ep_combine's input)
+ * A wait inside the kernel that exceeds 2 s sets EP_DEV_TIMEOUT and the
+ * kernel returns; it never traps.
+ */
+ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
+                           const int64_t *expert_offset, const int64_t *recv_count,
+                           const uint16_t *weights, int32_t n_out, uint16_t *y,
+                           uint32_t *dev_status, ep_stream_t stream);
 
 /*
  * Allocation-free variant of ep_dispatch_layout.  The pages have no

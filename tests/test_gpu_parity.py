@@ -596,3 +596,100 @@ def test_quantized_combine_unaligned_scale_rows(mode):
     r = Run(w, mode, layout="packed")
     assert r.sizes["scale_row_bytes"] % 4 != 0
     combine_quantized_check(r, seed=23)
+
+
+# ---------------------------------------------------------------------------
+# the experts between dispatch and combine: grouped tcgen05 GEMM
+# ---------------------------------------------------------------------------
+def _seeded_weights(E, n_out, H, scale, seed):
+    """Synthetic expert weights, N(0, scale^2) in bf16, from a seeded generator."""
+    gen = torch.Generator(device="cuda").manual_seed(seed)
+    return torch.randn(E, n_out, H, device="cuda", dtype=torch.bfloat16, generator=gen).mul_(scale)
+
+
+def _gemm_check(cfg, b, W, y, sample_rows=None):
+    """y against the oracle on the rows of every expert (or a sample): within
+    1 bf16 ulp of the oracle's result plus 2^-20 * sum_h |x*w| (the fp32
+    accumulation in the hardware's order); padding rows untouched (0x7777).
+    Only the experts of the checked rows are copied to the host."""
+    E, H = cfg.num_experts, cfg.hidden
+    n_out = W.shape[1]
+    eo = b.expert_offset.cpu().numpy()
+    cnt = b.recv_count.cpu().numpy()
+    rows = b.sizes["rows"]
+    xr = b.recv_data().view(torch.int16).cpu().numpy().view(np.uint16).reshape(rows, H)
+    got = y.view(torch.int16).cpu().numpy().view(np.uint16)
+    valid = np.zeros(rows, bool)
+    for e in range(E):
+        valid[eo[e]:eo[e] + cnt[e]] = True
+    assert np.all(got[~valid] == 0x7777)
+    expert_of = np.repeat(np.arange(E), np.diff(eo))
+    pick = np.nonzero(valid)[0]
+    if sample_rows is not None and len(pick) > sample_rows:
+        pick = np.sort(np.random.default_rng(0).choice(pick, sample_rows, replace=False))
+
+    def f(u):
+        return (u.astype(np.uint32) << 16).view(np.float32)
+    same = 0
+    for e in np.unique(expert_of[pick]):
+        rs = pick[expert_of[pick] == e]
+        We = W[e].view(torch.int16).cpu().numpy().view(np.uint16)          # [n_out, H]
+        want = oracle.expert_gemm(xr[rs], We[None], np.zeros(1, np.int64),
+                                  np.array([len(rs)], np.int64), n_out)
+        mag = np.abs(f(xr[rs])).astype(np.float64) @ np.abs(f(We)).astype(np.float64).T
+        wf, gf = f(want).astype(np.float64), f(got[rs]).astype(np.float64)
+        ulp = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(wf), 2.0 ** -126))).astype(np.int64) - 7)
+        assert np.all(np.abs(gf - wf) <= ulp + mag * 2.0 ** -20), int(e)
+        same += int((got[rs] == want).sum())
+    return same / (len(pick) * n_out)
+
+
+@pytest.mark.parametrize("n_out", [128, 384, 640])
+def test_expert_gemm_small(n_out):
+    w = synth.workload("tiny", R=4, T=40, M=48, K=4, E=8, H=640)
+    idx, wts = synth.make_routing(w)
+    idx[idx == 3] = 5                      # expert 3 receives nothing
+    r = Run(w, "bf16", layout="packed", align=8, idx=idx, wts=wts)
+    W = _seeded_weights(w["E"], n_out, w["H"], 0.05, seed=n_out)
+    y = torch.full((r.sizes["rows"], n_out), 0.0, dtype=torch.bfloat16, device="cuda")
+    y.view(torch.int16).fill_(0x7777)
+    ep.ep_expert_gemm(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, W, y, r.b.dev_status)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    assert r.b.recv_count.cpu().numpy()[3] == 0
+    _gemm_check(r.cfg, r.b, W, y)
+
+
+def test_expert_gemm_decode_shape_sampled():
+    w = synth.workload("decode", layout="packed")
+    r = Run(w, "bf16", layout="packed")
+    W = _seeded_weights(w["E"], w["H"], w["H"], 0.02, seed=7)
+    y = torch.empty((r.sizes["rows"], w["H"]), dtype=torch.bfloat16, device="cuda")
+    y.view(torch.int16).fill_(0x7777)
+    ep.ep_expert_gemm(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, W, y, r.b.dev_status)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    _gemm_check(r.cfg, r.b, W, y, sample_rows=12)
+
+
+def test_dispatch_experts_combine_pipeline():
+    """dispatch -> the experts' linear maps -> combine, against the oracle's
+    combine of the oracle's expert outputs (one bf16 ulp for the experts'
+    rounding, one for the combine's)."""
+    w = synth.workload("tiny", R=2, T=32, M=32, K=4, E=8, H=256)
+    r = Run(w, "bf16", layout="packed")
+    n_out = w["H"]
+    W = _seeded_weights(w["E"], n_out, w["H"], 0.06, seed=11)
+    ep.ep_expert_gemm(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, W, r.b.y,
+                      r.b.dev_status)
+    ep.ep_combine(r.cfg, r.b.y, r.idx_d, r.wts_d, r.b.token_slot, r.b.out, r.b.dev_status,
+                  expert_offset=r.b.expert_offset)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    eo = r.b.expert_offset.cpu().numpy()
+    cnt = r.b.recv_count.cpu().numpy()
+    xr = r.b.recv_data().view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1, w["H"])
+    yw = oracle.expert_gemm(xr, W.view(torch.int16).cpu().numpy().view(np.uint16), eo[:w["E"]],
+                            cnt, n_out)
+    want, st = oracle.combine(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], yw, r.idx, r.wts,
+                              r.lay["token_slot"], r.lay["expert_offset"], layout="packed")
+    from harness import ulp_distance, to_np_u16
+    got = to_np_u16(r.b.out)
+    assert st == 0 and ulp_distance(got, want).max() <= 2
