@@ -74,6 +74,9 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--weights-grad", action="store_true",
                    help="also time the combine's weight gradient (outside the step)")
+    p.add_argument("--gemm", action="store_true",
+                   help="also time the experts' grouped GEMM (bf16, packed, N = H) on the "
+                        "dispatched rows, outside the step")
     p.add_argument("--no-steady", action="store_true",
                    help="skip the steady-state pass and its buffer copies (profiling runs)")
     p.add_argument("--no-copy", action="store_true",
@@ -551,6 +554,8 @@ def main():
     except Exception:
         pass
 
+    gemm = run_gemm(ep, w, x_d, idx_d, flush, stream, dev, args) if args.gemm else None
+
     e2e = None if args.no_e2e else run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream,
                                           dev, args, world, step_bytes)
 
@@ -588,6 +593,7 @@ def main():
                                          "frac": round(iso_achieved / peak, 4)}},
         "kernels": kstats,
         "graph": graph,
+        "expert_gemm": gemm,
         "copy_gbs_same_run": copy_gbs,
         "e2e": e2e,
     }
@@ -657,6 +663,60 @@ def graph_steps(ep, args, cfg, ccfg, b, x_d, idx_d, wts_d, g_d, flush, stream, d
     del graph
     return {"ms_per_step": round(total / args.steps, 5),
             "value": round(world * N * args.steps / (total / 1e3), 1), "unit": "tokens/s"}
+
+
+def run_gemm(ep, w, x_d, idx_d, flush, stream, dev, args):
+    """The experts between dispatch and combine (ep_expert_gemm): the workload's
+    tokens dispatched as bf16 into the packed layout, one seeded random linear
+    map of H x H per expert, timed alone between events after an L2 flush.
+    FLOPs = 2 * (valid entries) * H * H."""
+    R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
+    cfg = ep.make_config(R, T, M, K, E, H, "bf16", "packed")
+    b = ep.Buffers(cfg, device=dev, expert_out=False)
+    ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
+                               b.recv_buf, b.src_info, b.dev_status,
+                               expert_offset=b.expert_offset, stream=stream)
+    gen = torch.Generator(device=dev).manual_seed(1234)
+    W = torch.randn(E, H, H, device=dev, dtype=torch.bfloat16, generator=gen).mul_(0.02)
+    y = torch.empty((b.sizes["rows"], H), dtype=torch.bfloat16, device=dev)
+    call = ep.ep_expert_gemm(cfg, b.recv_buf, b.expert_offset, b.recv_count, W, y, b.dev_status,
+                             stream=stream, bind=True)
+    for _ in range(3):
+        flush(1)
+        call()
+    torch.cuda.synchronize(dev)
+    if ep.ep_get_status(b.dev_status) != 0:
+        raise SystemExit("ep_expert_gemm reported a device error")
+    v = int(b.recv_count.sum().item())
+    reps = max(3, min(args.steps, 20))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for s in range(reps):
+        flush(s & 0xFF)
+        evs[s][0].record(stream)
+        call()
+        evs[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = statistics.mean(a.elapsed_time(c) for a, c in evs)
+    flops = 2.0 * v * H * H
+    # bytes that must move at least once: the weights of every expert that
+    # received a row, the received rows, the outputs
+    used = int((b.recv_count > 0).sum().item())
+    nbytes = 2.0 * used * H * H + 2.0 * 2 * v * H
+    peaks = measured_peaks() or {}
+    peak = peaks.get("bf16_tflops") or 1590.0
+    hbm = peaks.get("hbm_gbs") or 6650.0
+    tf = flops / (ms * 1e-3) / 1e12
+    t_tensor, t_hbm = flops / (peak * 1e12), nbytes / (hbm * 1e9)
+    del W, y, b
+    torch.cuda.empty_cache()
+    return {"ms": round(ms, 4), "flops": flops, "bytes": nbytes, "tflops": round(tf, 1),
+            "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+            "bound": "tensor" if t_tensor >= t_hbm else "hbm",
+            "peak_tflops": peak, "peak_gbs": hbm,
+            "peak_source": "measured" if peaks.get("bf16_tflops") else "fallback",
+            "frac": round(max(t_tensor, t_hbm) / (ms * 1e-3), 4),
+            "shape": f"{E} experts, {v} rows, {H} x {H} bf16 each"}
 
 
 STEADY_SETS = 4

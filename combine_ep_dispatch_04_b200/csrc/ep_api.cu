@@ -830,14 +830,15 @@ EncodeTiled encode_tiled() {
     return fn;
 }
 
-// bf16 matrix [outer][inner] (rows of `inner` elements), tiles of 64 x 128,
-// 128-byte swizzle (the layout the kernel's matrix descriptors describe)
-bool bf16_tile_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer) {
+// bf16 matrix [outer][inner] (rows of `inner` elements), tiles of 64 x
+// box_rows, 128-byte swizzle (the layout the kernel's matrix descriptors describe)
+bool bf16_tile_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+                   uint32_t box_rows) {
     const EncodeTiled enc = encode_tiled();
     if (!enc) return false;
     const cuuint64_t dims[2] = {inner, outer};
     const cuuint64_t strides[1] = {inner * 2};
-    const cuuint32_t box[2] = {(cuuint32_t)ep::kGemmBK, (cuuint32_t)ep::kGemmBM};
+    const cuuint32_t box[2] = {(cuuint32_t)ep::kGemmBK, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -862,8 +863,8 @@ ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
     if (p.N == 0) return EP_OK;
 
     CUtensorMap ma, mb;
-    if (!bf16_tile_map(&ma, recv_buf, (uint64_t)p.H, (uint64_t)p.rows) ||
-        !bf16_tile_map(&mb, weights, (uint64_t)p.H, (uint64_t)p.E * n_out))
+    if (!bf16_tile_map(&ma, recv_buf, (uint64_t)p.H, (uint64_t)p.rows, ep::kGemmBM) ||
+        !bf16_tile_map(&mb, weights, (uint64_t)p.H, (uint64_t)p.E * n_out, ep::kGemmBN))
         return EP_ERR_CUDA;
     ep::GemmArgs a;
     a.E = p.E; a.H = p.H; a.N = n_out; a.ntn = n_out / ep::kGemmBN;

@@ -7,13 +7,14 @@
 // layout (expert_offset[e] .. + count[e]),
 //   y[r, :] = bf16_rne( x[r, :] . W_e^T ),  fp32 accumulation.
 //
-// Tiles of 128 rows x 128 columns, 64-element K steps.  A persistent grid
+// Tiles of 128 rows x 256 columns, 64-element K steps.  A persistent grid
 // (one block per SM) walks the tiles of all experts; in each block
 //   warp 0        loads A and B K-steps with TMA (128-byte swizzle) into a
 //                 ring of kGemmStages shared-memory stages;
-//   warp 1        allocates 2 x 128 TMEM columns (two fp32 accumulators) and
-//                 one lane issues tcgen05.mma (cta_group::1, kind::f16, M=128,
-//                 N=128, K=16 per instruction), committing each stage back to
+//   warp 1        allocates 2 x 256 TMEM columns (two fp32 accumulators: all
+//                 of the SM's TMEM) and one lane issues tcgen05.mma
+//                 (cta_group::1, kind::f16, M=128, N=256, K=16 per
+//                 instruction), committing each stage back to
 //                 the loader and each finished accumulator to the epilogue;
 //   warps 2 - 5   read the accumulator rows (tcgen05.ld, one TMEM lane
 //                 quarter per warp), round to bf16 and store the tile's valid
@@ -29,11 +30,11 @@
 
 namespace ep {
 
-constexpr int kGemmBM = 128, kGemmBN = 128, kGemmBK = 64, kGemmStages = 4;
+constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4;
 constexpr int kGemmThreads = 192;
 constexpr uint32_t kDevTimeout = 0x4u;
 constexpr int kGemmTileBytesA = kGemmBM * kGemmBK * 2;  // 16 KB
-constexpr int kGemmTileBytesB = kGemmBN * kGemmBK * 2;  // 16 KB
+constexpr int kGemmTileBytesB = kGemmBN * kGemmBK * 2;  // 32 KB
 constexpr int kGemmMaxExperts = 1024;
 
 struct GemmArgs {

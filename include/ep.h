@@ -270,7 +270,7 @@ ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *
  * its received rows r (expert_offset[e] .. + recv_count[e] of the packed
  * receive layout):
  *   y[r, :] = bf16_rne( x[r, :] . W[e]^T )
- * with fp32 accumulation on the tensor cores (tcgen05, 128 x 128 tiles);
+ * with fp32 accumulation on the tensor cores (tcgen05, 128 x 256 tiles);
  * padding rows of y (past recv_count[e]) are not written.  The summation
  * order of the fp32 accumulation is the hardware's: results are within
  * 2^-20 * sum_h |x*w| + 1 bf16 ulp of the exact product.
@@ -279,7 +279,7 @@ ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *
  *   recv_buf     the dispatch's receive buffer: bf16 [rows][H]
  *   expert_offset, recv_count   from ep_dispatch_layout
  *   weights      bf16 [E][n_out][H] (row j of W[e] is output column j)
- *   n_out        output columns, a multiple of 128
+ *   n_out        output columns, a multiple of 256
  *   y            bf16 [rows][n_out] (n_out = H gives ep_combine's input)
  * A wait inside the kernel that exceeds 2 s sets EP_DEV_TIMEOUT and the
  * kernel returns; it never traps.

@@ -644,7 +644,7 @@ def _gemm_check(cfg, b, W, y, sample_rows=None):
     return same / (len(pick) * n_out)
 
 
-@pytest.mark.parametrize("n_out", [128, 384, 640])
+@pytest.mark.parametrize("n_out", [256, 768, 1280])
 def test_expert_gemm_small(n_out):
     w = synth.workload("tiny", R=4, T=40, M=48, K=4, E=8, H=640)
     idx, wts = synth.make_routing(w)
