@@ -608,10 +608,19 @@ def _seeded_weights(E, n_out, H, scale, seed):
 
 
 def _gemm_check(cfg, b, W, y, sample_rows=None):
-    """y against the oracle on the rows of every expert (or a sample): within
-    1 bf16 ulp of the oracle's result plus 2^-20 * sum_h |x*w| (the fp32
-    accumulation in the hardware's order); padding rows untouched (0x7777).
-    Only the experts of the checked rows are copied to the host."""
+    """y against the oracle on the rows of every expert (or a sample).
+
+    Every bf16 x bf16 product is exact in fp32.  The kernel adds them into an
+    fp32 accumulator in H/16 tensor-core steps of 16 products each; with the
+    sum inside one step taken in at least fp32 and any rounding of at most one
+    fp32 ulp (truncation allowed) per addition, the chain has at most
+    H/16 + 16 additions, so |acc - exact| <= (H/16 + 16) * 2^-23 * sum_h |x*w|,
+    and the bf16 rounding of acc adds at most one bf16 ulp of the result
+    (the oracle rounds the exact sum once).  Besides the bound, at least 90%
+    of the outputs equal the oracle's correctly rounded ones: the accumulation
+    error is far below half a bf16 ulp for almost every output.  Padding rows
+    stay untouched (0x7777).  Only the experts of the checked rows are copied
+    to the host."""
     E, H = cfg.num_experts, cfg.hidden
     n_out = W.shape[1]
     eo = b.expert_offset.cpu().numpy()
@@ -639,9 +648,11 @@ def _gemm_check(cfg, b, W, y, sample_rows=None):
         mag = np.abs(f(xr[rs])).astype(np.float64) @ np.abs(f(We)).astype(np.float64).T
         wf, gf = f(want).astype(np.float64), f(got[rs]).astype(np.float64)
         ulp = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(wf), 2.0 ** -126))).astype(np.int64) - 7)
-        assert np.all(np.abs(gf - wf) <= ulp + mag * 2.0 ** -20), int(e)
+        assert np.all(np.abs(gf - wf) <= ulp + mag * ((H // 16 + 16) * 2.0 ** -23)), int(e)
         same += int((got[rs] == want).sum())
-    return same / (len(pick) * n_out)
+    frac = same / (len(pick) * n_out)
+    assert frac >= 0.9, frac
+    return frac
 
 
 @pytest.mark.parametrize("n_out", [256, 768, 1280])
