@@ -575,9 +575,9 @@ void orc_combine_wgrad_gathered(long N, int K, int H, const uint16_t *g, const u
 }
 
 /*
- * The experts between dispatch and combine (SURVEY NEXT-4 stand-in: each
- * expert a single linear map, as the deep-fused MoE operator of "[feat] A5
- * deep fused moe supported" runs grouped matrix multiplications between its
+ * The experts between dispatch and combine (each expert a single linear
+ * map, standing in for the grouped matrix multiplications that the deep-fused
+ * MoE operator of "[feat] A5 deep fused moe supported" runs between its
  * dispatch and combine): for every expert e and each of its rows r (rows
  * expert_offset[e] .. + count[e] of the packed receive layout),
  *   y[r, j] = bf16_rne( sum_h x[r, h] * w[e, j, h] ),  j < Nout,
@@ -595,6 +595,44 @@ void orc_expert_gemm(int E, int H, int Nout, const int64_t *expert_offset, const
                 double acc = 0.0;
                 for (int h = 0; h < H; h++)
                     acc += (double)orc_bf16_to_f32(x[r * H + h]) * (double)orc_bf16_to_f32(wr[h]);
+                y[r * Nout + j] = orc_f32_to_bf16((float)acc);
+            }
+        }
+    }
+}
+
+/*
+ * The same linear maps on MXFP8 operands ("[feat] A5 deep fused moe
+ * supported": the deep-fused operator's grouped matrix multiplications take
+ * e4m3 codes with one e8m0 scale per 32 elements, as its MX dispatch emits).
+ * Element h of row r is decode_e4m3(xc[r, h]) * 2^(xs[r, h/32] - 127); weight
+ * element (j, h) of expert e is decode_e4m3(wc[e, j, h]) * 2^(ws[e, j, h/32] - 127);
+ *   y[r, j] = bf16_rne( sum_h x[r, h] * w[e, j, h] )
+ * with every product exact in double (3-bit mantissas, power-of-two scales),
+ * summed in double in h order, rounded to fp32 and then to bf16.  A NaN code
+ * or scale byte 255 (NaN in the MX format) gives NaN.  Rows past count[e] are
+ * left untouched.
+ */
+static double orc_e8m0_value(uint8_t b)
+{
+    return b == 255 ? NAN : ldexp(1.0, (int)b - 127);
+}
+void orc_expert_gemm_mx(int E, int H, int Nout, const int64_t *expert_offset, const int64_t *count,
+                        const uint8_t *xc, const uint8_t *xs, const uint8_t *wc,
+                        const uint8_t *ws, uint16_t *y)
+{
+    const int S = H / 32;
+    for (int e = 0; e < E; e++) {
+        for (int64_t i = 0; i < count[e]; i++) {
+            int64_t r = expert_offset[e] + i;
+            for (int j = 0; j < Nout; j++) {
+                const int64_t wrow = (int64_t)e * Nout + j;
+                double acc = 0.0;
+                for (int h = 0; h < H; h++) {
+                    double xv = (double)orc_e4m3_decode(xc[r * H + h]) * orc_e8m0_value(xs[r * S + h / 32]);
+                    double wv = (double)orc_e4m3_decode(wc[wrow * H + h]) * orc_e8m0_value(ws[wrow * S + h / 32]);
+                    acc += xv * wv;
+                }
                 y[r * Nout + j] = orc_f32_to_bf16((float)acc);
             }
         }

@@ -17,6 +17,11 @@ from oracle.build import CFLAGS  # noqa: E402
 
 # name: ([(text in ep_oracle.c, replacement), ...], pins that must catch it)
 MUTANTS = {
+    "MX weight scale read from the expert's first row": (
+        [("orc_e8m0_value(ws[wrow * S + h / 32])", "orc_e8m0_value(ws[(int64_t)e * Nout * S + h / 32])")],
+        "expert_gemm_mx"),
+    "MX scale bias off by one": (
+        [("ldexp(1.0, (int)b - 127)", "ldexp(1.0, (int)b - 126)")], "expert_gemm_mx"),
     "layout ties broken by descending k": (
         [("            for (int k = 0; k < K; k++) {\n                int64_t e = idx[n * K + k];\n"
           "                if (e < -1 || e >= E) st |= ORC_ST_BAD_INDEX;\n"

@@ -867,3 +867,76 @@ def test_expert_gemm_equals_exact_rational_products():
                 exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(xf[row], wf[e, j]))
                 want = synth.to_bf16_bits(np.float32([float(exact)]))[0]
                 assert y[row, j] == want, (e, i, j)
+
+
+# the same maps on MXFP8 operands (e4m3 codes, e8m0 scale per 32)
+def _mx_operands(r, shape, lo=120, hi=134):
+    """Seeded e4m3 codes (NaN codes 0x7F / 0xFF replaced by zero) and e8m0
+    scale bytes in [lo, hi) for a [..., H] operand."""
+    c = r.integers(0, 256, shape).astype(np.uint8)
+    c[(c & 0x7F) == 0x7F] = 0
+    s = r.integers(lo, hi, shape[:-1] + (shape[-1] // 32,)).astype(np.uint8)
+    return c, s
+
+
+def _mx_values(c, s):
+    """Dequantised values, written out here from the e4m3 decoder and 2^(s-127)."""
+    v = oracle.e4m3_decode(c).astype(np.float64)
+    return v * np.ldexp(1.0, np.repeat(s.astype(np.int64) - 127, 32, axis=-1))
+
+
+def test_expert_gemm_mx_identity_weights_give_the_dequantised_rows():
+    r = np.random.default_rng(3)
+    E, H = 2, 64
+    cnt = np.array([3, 4], np.int64)
+    eo = np.array([0, 4, 8], np.int64)
+    xc, xs = _mx_operands(r, (8, H))
+    wc = np.zeros((E, H, H), np.uint8)
+    for e in range(E):
+        wc[e][np.arange(H), np.arange(H)] = 0x38            # e4m3 1.0
+    ws = np.full((E, H, H // 32), 127, np.uint8)            # 2^0
+    y = oracle.expert_gemm_mx(xc, xs, wc, ws, eo[:E], cnt, H, y=np.full((8, H), 0x7777, np.uint16))
+    for e in range(E):
+        for i in range(cnt[e]):
+            row = eo[e] + i
+            want = synth.to_bf16_bits(oracle.dequant_row("mxfp8", xc[row], xs[row], H))
+            want[want == 0x8000] = 0                         # a sum of zero products is +0
+            assert np.array_equal(y[row], want), (e, i)
+    assert np.all(y[3] == 0x7777)                            # past expert 0's count
+
+
+def test_expert_gemm_mx_equals_exact_rational_sums():
+    from fractions import Fraction
+    r = np.random.default_rng(4)
+    E, H, N = 2, 64, 4
+    cnt = np.array([2, 3], np.int64)
+    eo = np.array([0, 2], np.int64)
+    xc, xs = _mx_operands(r, (5, H), 118, 136)
+    wc, ws = _mx_operands(r, (E, N, H), 118, 136)
+    y = oracle.expert_gemm_mx(xc, xs, wc, ws, eo, cnt, N)
+    xv, wv = _mx_values(xc, xs), _mx_values(wc, ws)
+    for e in range(E):
+        for i in range(cnt[e]):
+            row = eo[e] + i
+            for j in range(N):
+                exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(xv[row], wv[e, j]))
+                want = synth.to_bf16_bits(np.float32([float(exact)]))[0]
+                assert y[row, j] == want, (e, i, j)
+
+
+def test_expert_gemm_mx_equals_bf16_maps_on_dequantised_operands():
+    """e4m3 values times powers of two in the normal range are bf16 values, so
+    the MX maps equal the (separately pinned) bf16 maps of the dequantised
+    operands, bit for bit."""
+    r = np.random.default_rng(5)
+    E, H, N = 3, 256, 16
+    cnt = np.array([4, 0, 6], np.int64)
+    eo = np.array([0, 8, 8], np.int64)
+    xc, xs = _mx_operands(r, (16, H))
+    wc, ws = _mx_operands(r, (E, N, H))
+    xb = synth.to_bf16_bits(_mx_values(xc, xs).astype(np.float32))
+    wb = synth.to_bf16_bits(_mx_values(wc, ws).astype(np.float32))
+    assert np.array_equal(oracle.bf16_to_f32(xb).astype(np.float64), _mx_values(xc, xs))
+    want = oracle.expert_gemm(xb, wb, eo, cnt, N)
+    got = oracle.expert_gemm_mx(xc, xs, wc, ws, eo, cnt, N)
+    assert np.array_equal(got, want)
