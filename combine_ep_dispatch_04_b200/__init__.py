@@ -9,7 +9,8 @@ from .ep import (DEV_BAD_INDEX, DEV_CAPACITY_OVERFLOW, STATIC_SCRATCH_BYTES, F_B
                  F_LAYOUT_SINGLE_CTA, F_ROUND_SCALE, F_UE8M0, LAYOUT, QUANT, Bound, Buffers,
                  EpConfig, EpError, EpSizes, ep_buffer_sizes, ep_combine, ep_combine_backward,
                  ep_combine_backward_weights, ep_copy, ep_cvt_sweep, ep_dispatch, ep_dispatch_layout,
-                 ep_dispatch_layout_static, ep_dispatch_with_layout, ep_expert_gemm, ep_get_status,
+                 ep_dispatch_layout_static, ep_dispatch_with_layout, ep_expert_gemm, ep_expert_gemm_mx,
+                 ep_get_status,
                  ep_kernel_launches, idx_dtype, make_config)
 
 __all__ = [
@@ -19,5 +20,5 @@ __all__ = [
     "EpConfig", "EpError", "EpSizes", "ep_buffer_sizes", "ep_combine", "ep_combine_backward",
     "ep_combine_backward_weights",
     "ep_copy", "ep_cvt_sweep", "ep_dispatch", "ep_dispatch_layout", "ep_dispatch_layout_static",
-    "ep_dispatch_with_layout", "ep_expert_gemm", "ep_get_status", "ep_kernel_launches", "idx_dtype", "make_config",
+    "ep_dispatch_with_layout", "ep_expert_gemm", "ep_expert_gemm_mx", "ep_get_status", "ep_kernel_launches", "idx_dtype", "make_config",
 ]

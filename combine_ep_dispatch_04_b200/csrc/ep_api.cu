@@ -28,6 +28,7 @@ constexpr int64_t kSingleMaxEntries = 2048;
 constexpr int64_t kClusterMaxEntries = 131072;
 constexpr size_t kDefaultSmem = 48 * 1024;
 constexpr size_t kMaxSmem = 200 * 1024;
+constexpr size_t kMaxSmemOptin = 227 * 1024;  // the GEMMs' rings
 
 cudaStream_t cs(ep_stream_t s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -206,12 +207,12 @@ std::atomic<uint32_t> g_smem_done[kMaxDevices];
 template <typename Kernel>
 bool allow_smem(Kernel k, int which, size_t bytes) {
     if (bytes <= kDefaultSmem) return true;
-    if (bytes > kMaxSmem) return false;
+    if (bytes > kMaxSmemOptin) return false;
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
     if (g_smem_done[dev].load() & (1u << which)) return true;
-    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kMaxSmem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)std::max(bytes, kMaxSmem)) != cudaSuccess)
         return false;
     g_smem_done[dev].fetch_or(1u << which);
     return true;
@@ -844,6 +845,52 @@ bool bf16_tile_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t ou
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+// u8 matrix [outer][inner], tiles of 128 x box_rows, 128-byte swizzle
+bool u8_tile_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer,
+                 uint32_t box_rows) {
+    const EncodeTiled enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {inner};
+    const cuuint32_t box[2] = {(cuuint32_t)ep::kMxBK, box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// one launch of the MXFP8 kernel with N tiles of BN columns
+extern "C++" template <int BN>
+ep_status_t launch_gemm_mx(const Plan &p, const void *recv_buf, const int64_t *expert_offset,
+                           const int64_t *recv_count, const uint8_t *w_codes,
+                           const uint8_t *w_scales, int n_out, uint16_t *y,
+                           uint32_t *dev_status, cudaStream_t s, int slot) {
+    CUtensorMap ma, mb;
+    if (!u8_tile_map(&ma, recv_buf, (uint64_t)p.H, (uint64_t)p.rows, ep::kGemmBM) ||
+        !u8_tile_map(&mb, w_codes, (uint64_t)p.H, (uint64_t)p.E * n_out, BN))
+        return EP_ERR_CUDA;
+    ep::MxArgs a;
+    a.E = p.E; a.H = p.H; a.N = n_out; a.ntn = n_out / BN; a.rows = p.rows;
+    a.eo = expert_offset; a.cnt = recv_count;
+    a.xs = static_cast<const uint8_t *>(recv_buf) + p.scale_off;
+    a.ws = w_scales; a.y = y; a.status = dev_status;
+    const size_t smem = ep::MxCfg<BN>::smem();
+    if (!allow_smem(ep::expert_gemm_mx_kernel<BN>, slot, smem)) return EP_ERR_CUDA;
+    launch(ep::expert_gemm_mx_kernel<BN>, (unsigned)sm_count(), ep::kMxThreads, smem, s, ma, mb, a);
+    return launched();
+}
+
+// N tile of the MXFP8 kernel: two accumulators of 224 columns where n_out
+// allows, else one of 256, else two of 128
+#ifndef EP_MX_PREFER_BN
+#define EP_MX_PREFER_BN 224
+#endif
+int mx_tile_n(int n_out) {
+    const int pref[3] = {EP_MX_PREFER_BN, EP_MX_PREFER_BN == 224 ? 256 : 224, 128};
+    for (int bn : pref)
+        if (n_out % bn == 0) return bn;
+    return 0;
+}
 }  // namespace
 
 ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
@@ -874,6 +921,32 @@ ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
     launch(ep::expert_gemm_kernel, (unsigned)sm_count(), ep::kGemmThreads, smem, cs(stream), ma,
            mb, a);
     return launched();
+}
+
+ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
+                              const int64_t *expert_offset, const int64_t *recv_count,
+                              const uint8_t *w_codes, const uint8_t *w_scales, int32_t n_out,
+                              uint16_t *y, uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (cfg->quant != EP_Q_MXFP8 || cfg->layout != EP_LAYOUT_PACKED) return EP_ERR_UNSUPPORTED;
+    if (p.H % ep::kMxBK != 0) return EP_ERR_UNSUPPORTED;
+    if (n_out <= 0) return EP_ERR_INVALID_ARG;
+    const int bn = mx_tile_n(n_out);
+    if (bn == 0) return EP_ERR_INVALID_ARG;
+    if ((int64_t)n_out * p.E > kIntLimit || p.E > ep::kGemmMaxExperts) return EP_ERR_INVALID_ARG;
+    if (!recv_buf || !expert_offset || !recv_count || !w_codes || !w_scales || !y || !dev_status)
+        return EP_ERR_INVALID_ARG;
+    if (!aligned16(recv_buf) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y))
+        return EP_ERR_MISALIGNED;
+    if (p.N == 0) return EP_OK;
+    cudaStream_t s = cs(stream);
+    switch (bn) {
+    case 224: return launch_gemm_mx<224>(p, recv_buf, expert_offset, recv_count, w_codes, w_scales, n_out, y, dev_status, s, 6);
+    case 256: return launch_gemm_mx<256>(p, recv_buf, expert_offset, recv_count, w_codes, w_scales, n_out, y, dev_status, s, 7);
+    default:  return launch_gemm_mx<128>(p, recv_buf, expert_offset, recv_count, w_codes, w_scales, n_out, y, dev_status, s, 8);
+    }
 }
 
 ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream) {

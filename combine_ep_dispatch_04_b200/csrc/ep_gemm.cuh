@@ -144,7 +144,7 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 
 // tile t of the walk -> expert, first row and first column (t < prefix[E])
 __device__ __forceinline__ void gemm_tile(const int *prefix, int E, int ntn, int t, int &e,
-                                          int &m0, int &n0) {
+                                          int &m0, int &n0, int bn = kGemmBN) {
     int lo = 0, hi = E - 1;  // the last e with prefix[e] <= t
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -154,7 +154,34 @@ __device__ __forceinline__ void gemm_tile(const int *prefix, int E, int ntn, int
     e = lo;
     const int local = t - prefix[e];
     m0 = (local / ntn) * kGemmBM;
-    n0 = (local % ntn) * kGemmBN;
+    n0 = (local % ntn) * bn;
+}
+
+// tiles per expert, exclusive prefix into prefix[0..E] (one warp; each lane
+// takes a run of experts)
+__device__ __forceinline__ void tile_prefix(int *prefix, int E, const int64_t *cnt, int ntn,
+                                            int lane) {
+    const int per = (E + 31) / 32;
+    int sum = 0;
+    for (int i = 0; i < per; i++) {
+        const int e = lane * per + i;
+        if (e < E) sum += (int)((cnt[e] + kGemmBM - 1) / kGemmBM) * ntn;
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += v;
+    }
+    int run = incl - sum;
+    for (int i = 0; i < per; i++) {
+        const int e = lane * per + i;
+        if (e < E) {
+            prefix[e] = run;
+            run += (int)((cnt[e] + kGemmBM - 1) / kGemmBM) * ntn;
+        }
+    }
+    if (lane == 31) prefix[E] = incl;
 }
 
 __global__ void __launch_bounds__(kGemmThreads, 1)
@@ -196,29 +223,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     pdl_enter();
-    if (warp == 0) {  // tiles per expert, exclusive prefix (one lane per run of experts)
-        const int per = (E + 31) / 32;
-        int sum = 0;
-        for (int i = 0; i < per; i++) {
-            const int e = lane * per + i;
-            if (e < E) sum += (int)((a.cnt[e] + kGemmBM - 1) / kGemmBM) * a.ntn;
-        }
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - sum;
-        for (int i = 0; i < per; i++) {
-            const int e = lane * per + i;
-            if (e < E) {
-                prefix[e] = run;
-                run += (int)((a.cnt[e] + kGemmBM - 1) / kGemmBM) * a.ntn;
-            }
-        }
-        if (lane == 31) prefix[E] = incl;
-    }
+    if (warp == 0) tile_prefix(prefix, E, a.cnt, a.ntn, lane);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -343,6 +348,322 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                      "r"(2 * kGemmBN));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// MXFP8 operands: e4m3 codes with one e8m0 scale per 32 elements on both the
+// received rows and the weights, multiplied by the block-scaled MMA
+// (tcgen05.mma kind::mxf8f6f4.block_scale, K = 32 per instruction: one scale
+// per row of A and per row of B and instruction).
+//
+// A K step is 128 codes (one 128-byte swizzle row): 4 instructions.  The
+// scales of a step are 4 bytes per row, read from the rows' scale region by
+// one gathering warp and written to shared memory in the arrangement that
+// tcgen05.cp .32x128b.warpx4 copies to TMEM: the 16 bytes of lane l hold rows
+// l, l+32, l+64, l+96 (4 bytes each: the step's 4 scale blocks), one 512-byte
+// chunk per 128 rows.  In TMEM row m's scale for block j then sits in lane
+// m % 32 (of every lane quarter), column m / 32, byte j; byte j is selected by
+// the scale-factor id of the instruction (bits 30-31 of the scale address).
+//
+// Warps: 0 loads the code tiles with TMA; 1 allocates TMEM and one lane
+// issues the scale copies and the MMAs; 2 gathers the scales; 3 - 6 run the
+// epilogue.  A stage is full when the TMA bytes have landed and the gathering
+// warp has arrived.  TMEM holds kAcc accumulators of BN columns and the
+// scales behind them: two accumulators (the epilogue of one tile overlaps the
+// next tile's MMAs) where they and the scales fit in 512 columns, else one.
+// ---------------------------------------------------------------------------
+constexpr int kMxBK = 128, kMxStages = 4, kMxThreads = 224;
+
+template <int BN>
+struct MxCfg {
+    static constexpr int kChunksB = (BN + 127) / 128;      // 128-row scale chunks of B
+    static constexpr int kSfCols = 4 + 4 * kChunksB;       // TMEM columns of A's and B's scales
+    static constexpr int kAcc = (2 * BN + kSfCols <= 512) ? 2 : 1;
+    static constexpr int kBytesA = kGemmBM * kMxBK;         // 16 KB
+    static constexpr int kBytesB = BN * kMxBK;
+    static constexpr int kSfBytes = 512 * (1 + kChunksB);   // one stage's scales, A then B
+    static constexpr int kSfCol = kAcc * BN;                // TMEM column of A's scales
+    static constexpr size_t smem() {
+        return 1024 + (size_t)kMxStages * (kBytesA + kBytesB + kSfBytes) +
+               (2 * kMxStages + 5) * 8 + 16 + (kGemmMaxExperts + 1) * 4 + 256;
+    }
+    static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "N tile");
+    static_assert(kAcc * BN + kSfCols <= 512, "TMEM columns");
+};
+
+struct MxArgs {
+    int E, H, N;
+    int ntn;                 // N / BN
+    int64_t rows;            // rows of the receive buffer (scale rows that exist)
+    const int64_t *eo;       // [E+1] first row of each expert (packed layout)
+    const int64_t *cnt;      // [E] rows of each expert
+    const uint8_t *xs;       // [rows][H/32] e8m0 scales of the received rows
+    const uint8_t *ws;       // [E*N][H/32] e8m0 scales of the weights
+    uint16_t *y;             // [rows][N] bf16
+    uint32_t *status;
+};
+
+// instruction descriptor of the block-scaled MMA: e4m3 A and B, both K-major,
+// e8m0 scales, N, M (the scale-factor ids are or-ed in per instruction)
+__host__ __device__ constexpr uint32_t umma_idesc_mxf8(int M, int N) {
+    return ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24);
+}
+__device__ __forceinline__ void umma_mxf8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t tsfa, uint32_t tsfb,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(tsfa), "r"(tsfb), "r"(accumulate)
+        : "memory");
+}
+// shared-memory descriptor of 32 rows x 16 bytes, rows 16 bytes apart (no
+// swizzle, K-major: 8-row core matrices of 128 contiguous bytes, 128 bytes
+// between them)
+__device__ __forceinline__ uint64_t sf_desc(uint32_t saddr) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)8 << 32) | ((uint64_t)1 << 46);
+}
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+                 : "memory");
+}
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                             uint32_t d) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+                 "r"(d)
+                 : "memory");
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kMxThreads, 1)
+    expert_gemm_mx_kernel(const __grid_constant__ CUtensorMap tm_a,
+                          const __grid_constant__ CUtensorMap tm_b, MxArgs a) {
+    using C = MxCfg<BN>;
+    constexpr int S = kMxStages;
+    extern __shared__ uint8_t gsm_raw[];
+    uint8_t *gsm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t *sA = gsm;
+    uint8_t *sB = sA + S * C::kBytesA;
+    uint8_t *sSF = sB + S * C::kBytesB;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sSF + S * C::kSfBytes);
+    uint64_t *full = bars, *empty = bars + S;
+    uint64_t *accfull = bars + 2 * S, *accempty = accfull + 2;
+    uint64_t *drain = accempty + 2;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile uint32_t *s_abort = s_tmem + 1;
+    int *prefix = reinterpret_cast<int *>(s_tmem + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = a.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(smem_addr(&full[s]), 2);  // the TMA bytes' arrival + the scale warp's
+            mbar_init(smem_addr(&empty[s]), 1);
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(smem_addr(&accfull[b]), 1);
+            mbar_init(smem_addr(&accempty[b]), 128);
+        }
+        mbar_init(smem_addr(drain), 1);
+        *s_abort = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {  // the whole warp: all 512 columns (accumulators, then the scales)
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(s_tmem)),
+                     "r"(512));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    pdl_enter();
+    if (warp == 0) tile_prefix(prefix, E, a.cnt, a.ntn, lane);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const int total = prefix[E];
+    const int kblocks = a.H / kMxBK;
+
+    if (warp == 0 && lane == 0) {
+        // ---- code tiles
+        int it = 0;
+        for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
+            int e, m0, n0;
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, BN);
+            const int arow = (int)a.eo[e] + m0, brow = e * a.N + n0;
+            for (int kb = 0; kb < kblocks; kb++, it++) {
+                const int s = it % S, r = it / S;
+                if (!mbar_wait(smem_addr(&empty[s]), (r & 1) ^ 1)) {
+                    *s_abort = 1u;
+                    atomicOr(a.status, kDevTimeout);
+                    break;
+                }
+                const uint32_t fb = smem_addr(&full[s]);
+                mbar_expect_tx(fb, C::kBytesA + C::kBytesB);
+                tma_load_2d(smem_addr(sA + s * C::kBytesA), &tm_a, kb * kMxBK, arow, fb);
+                tma_load_2d(smem_addr(sB + s * C::kBytesB), &tm_b, kb * kMxBK, brow, fb);
+            }
+        }
+        for (int j = 0; j < S && j < it; j++) {  // copies in flight land before leaving
+            const int i2 = it - 1 - j, s = i2 % S, r = i2 / S;
+            if (!mbar_wait(smem_addr(&full[s]), r & 1)) atomicOr(a.status, kDevTimeout);
+        }
+    } else if (warp == 1 && lane == 0) {
+        // ---- scale copies and MMAs
+        const uint32_t idesc = umma_idesc_mxf8(kGemmBM, BN);
+        const uint32_t tsfa = tmem_base + (uint32_t)C::kSfCol, tsfb = tsfa + 4;
+        int it = 0, tc = 0;
+        for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x, tc++) {
+            const int acc = tc % C::kAcc, use = tc / C::kAcc;
+            if (!mbar_wait(smem_addr(&accempty[acc]), (use & 1) ^ 1)) {
+                *s_abort = 1u;
+                atomicOr(a.status, kDevTimeout);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem_base + (uint32_t)(acc * BN);
+            bool ok = true;
+            for (int kb = 0; kb < kblocks; kb++, it++) {
+                const int s = it % S, r = it / S;
+                if (!mbar_wait(smem_addr(&full[s]), r & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t sf = smem_addr(sSF + s * C::kSfBytes);
+                tmem_cp_32x128b_x4(tsfa, sf_desc(sf));
+#pragma unroll
+                for (int c = 0; c < C::kChunksB; c++)
+                    tmem_cp_32x128b_x4(tsfb + 4 * c, sf_desc(sf + 512 * (1 + c)));
+                const uint64_t ad = umma_desc_sw128(smem_addr(sA + s * C::kBytesA));
+                const uint64_t bd = umma_desc_sw128(smem_addr(sB + s * C::kBytesB));
+#pragma unroll
+                for (int k = 0; k < kMxBK / 32; k++)  // 32 codes = 32 bytes = 2 units
+                    umma_mxf8(d, ad + 2 * k, bd + 2 * k,
+                              idesc | ((uint32_t)k << 29) | ((uint32_t)k << 4),
+                              tsfa | ((uint32_t)k << 30), tsfb | ((uint32_t)k << 30),
+                              (kb | k) != 0);
+                umma_commit(smem_addr(&empty[s]));
+            }
+            if (!ok) {
+                *s_abort = 1u;
+                atomicOr(a.status, kDevTimeout);
+                break;
+            }
+            umma_commit(smem_addr(&accfull[acc]));
+        }
+    } else if (warp == 2) {
+        // ---- scales: 4 bytes (one K step) of every row of the A and B tiles
+        const int SB = a.H / 32;
+        int it = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x) {
+            if (__shfl_sync(kFull, (int)*s_abort, 0)) break;
+            int e, m0, n0;
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, BN);
+            const int64_t arow0 = a.eo[e] + m0;
+            const int64_t brow0 = (int64_t)e * a.N + n0;
+            bool ok = true;
+            for (int kb = 0; kb < kblocks; kb++, it++) {
+                const int s = it % S, r = it / S;
+                uint32_t va[4], vb[C::kChunksB][4];
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const int64_t row = arow0 + lane + 32 * j;
+                    va[j] = row < a.rows ? __ldg(reinterpret_cast<const uint32_t *>(
+                                               a.xs + row * SB + kb * 4))
+                                         : 0u;
+                }
+#pragma unroll
+                for (int c = 0; c < C::kChunksB; c++)
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const int n = 128 * c + 32 * j + lane;
+                        vb[c][j] = n < BN ? __ldg(reinterpret_cast<const uint32_t *>(
+                                                a.ws + (brow0 + n) * SB + kb * 4))
+                                          : 0u;
+                    }
+                int got = 1;
+                if (lane == 0) got = mbar_wait(smem_addr(&empty[s]), (r & 1) ^ 1);
+                if (!__shfl_sync(kFull, got, 0)) {
+                    ok = false;
+                    break;
+                }
+                const uint32_t st = smem_addr(sSF + s * C::kSfBytes) + lane * 16;
+                st_shared_v4(st, va[0], va[1], va[2], va[3]);
+#pragma unroll
+                for (int c = 0; c < C::kChunksB; c++)
+                    st_shared_v4(st + 512 * (1 + c), vb[c][0], vb[c][1], vb[c][2], vb[c][3]);
+                // the copies to TMEM read shared memory through the async proxy
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&full[s]));
+            }
+            if (!ok) {
+                if (lane == 0) {
+                    *s_abort = 1u;
+                    atomicOr(a.status, kDevTimeout);
+                }
+                break;
+            }
+        }
+    } else if (warp >= 3) {
+        // ---- epilogue: warp w reads TMEM lanes 32*(w % 4) ..
+        const int sub = warp & 3;
+        int tc = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, tc++) {
+            const int acc = tc % C::kAcc, use = tc / C::kAcc;
+            const bool ok =
+                __all_sync(kFull, !*s_abort && mbar_wait(smem_addr(&accfull[acc]), use & 1));
+            if (!ok) {
+                if (lane == 0) {
+                    *s_abort = 1u;
+                    atomicOr(a.status, kDevTimeout);
+                }
+                break;
+            }
+            tc_fence_after();
+            int e, m0, n0;
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, BN);
+            const int m = m0 + sub * 32 + lane;
+            const bool valid = m < a.cnt[e];
+            uint16_t *yrow = a.y + (a.eo[e] + m) * (int64_t)a.N + n0;
+            const uint32_t taddr =
+                tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 16; c++) {
+                uint32_t v[16];
+                tmem_ld16(taddr + c * 16, v);
+                if (valid) {
+                    uint4 lo, hi;
+                    lo.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
+                    lo.y = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
+                    lo.z = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
+                    lo.w = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
+                    hi.x = pack_bf16x2(__uint_as_float(v[8]), __uint_as_float(v[9]));
+                    hi.y = pack_bf16x2(__uint_as_float(v[10]), __uint_as_float(v[11]));
+                    hi.z = pack_bf16x2(__uint_as_float(v[12]), __uint_as_float(v[13]));
+                    hi.w = pack_bf16x2(__uint_as_float(v[14]), __uint_as_float(v[15]));
+                    st_v4(yrow + c * 16, lo);
+                    st_v4(yrow + c * 16 + 8, hi);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_addr(&accempty[acc]));
+        }
+    }
+    if (warp == 1 && lane == 0 && total > (int)blockIdx.x) {
+        umma_commit(smem_addr(drain));
+        if (!mbar_wait(smem_addr(drain), 0)) atomicOr(a.status, kDevTimeout);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(512));
     }
 }
 

@@ -81,6 +81,8 @@ lib.ep_combine_backward.restype = C.c_int
 lib.ep_combine_backward.argtypes = [_CFG] + [_P] * 8
 lib.ep_expert_gemm.restype = C.c_int
 lib.ep_expert_gemm.argtypes = [_CFG, _P, _P, _P, _P, C.c_int32, _P, _P, _P]
+lib.ep_expert_gemm_mx.restype = C.c_int
+lib.ep_expert_gemm_mx.argtypes = [_CFG, _P, _P, _P, _P, _P, C.c_int32, _P, _P, _P]
 lib.ep_combine_backward_weights.restype = C.c_int
 lib.ep_combine_backward_weights.argtypes = [_CFG] + [_P] * 8
 lib.ep_get_status.restype = C.c_int
@@ -336,6 +338,29 @@ def ep_expert_gemm(cfg, recv_buf, expert_offset, recv_count, weights, y, dev_sta
         _stream(stream),
     ]
     return _call(lib.ep_expert_gemm, cfg, args, "ep_expert_gemm", bind)
+
+
+def ep_expert_gemm_mx(cfg, recv_buf, expert_offset, recv_count, w_codes, w_scales, y, dev_status,
+                      stream=None, bind=False):
+    """The same maps on MXFP8 operands (packed MXFP8 receive layout): w_codes e4m3
+    [E, n_out, H] as uint8, w_scales e8m0 [E, n_out, H/32] as uint8, y bf16 [rows, n_out]."""
+    sz = ep_buffer_sizes(cfg)
+    E, H = cfg.num_experts, cfg.hidden
+    if w_codes is None or w_codes.dim() != 3:
+        raise ValueError("w_codes must be a [E, n_out, H] tensor")
+    n_out = int(w_codes.shape[1])
+    args = [
+        _bytes(recv_buf, "recv_buf", sz["recv_bytes"]),
+        _dev(expert_offset, "expert_offset", torch.int64, (E + 1,)),
+        _dev(recv_count, "recv_count", torch.int64, (E,)),
+        _dev(w_codes, "w_codes", torch.uint8, (E, n_out, H)),
+        _dev(w_scales, "w_scales", torch.uint8, (E, n_out, H // 32)),
+        C.c_int32(n_out),
+        _dev(y, "y", torch.bfloat16, (sz["rows"], n_out)),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    return _call(lib.ep_expert_gemm_mx, cfg, args, "ep_expert_gemm_mx", bind)
 
 
 def ep_combine_backward_weights(cfg, g, y, topk_idx, token_slot, topk_weights_grad, dev_status,

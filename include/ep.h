@@ -79,7 +79,7 @@ typedef enum {
 /* Bits of *dev_status. */
 #define EP_DEV_BAD_INDEX 0x1u         /* topk_idx value < -1 or >= E (entry skipped) */
 #define EP_DEV_CAPACITY_OVERFLOW 0x2u /* slot >= R*M in the padded layout (row skipped) */
-#define EP_DEV_TIMEOUT 0x4u           /* a bounded wait inside ep_expert_gemm gave up */
+#define EP_DEV_TIMEOUT 0x4u           /* a bounded wait inside ep_expert_gemm(_mx) gave up */
 
 /* ep_config_t.flags */
 #define EP_F_BWD_UNWEIGHTED 0x1u    /* combine-backward re-dispatches g without w */
@@ -272,8 +272,9 @@ ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *
  *   y[r, :] = bf16_rne( x[r, :] . W[e]^T )
  * with fp32 accumulation on the tensor cores (tcgen05, 128 x 256 tiles);
  * padding rows of y (past recv_count[e]) are not written.  The summation
- * order of the fp32 accumulation is the hardware's: results are within
- * 2^-20 * sum_h |x*w| + 1 bf16 ulp of the exact product.
+ * order of the fp32 accumulation is the hardware's: every product is exact
+ * and H/16 partial sums are chained through one fp32 accumulator, so results
+ * are within (H/16 + 16) * 2^-23 * sum_h |x*w| + 1 bf16 ulp of the exact sum.
  *   cfg          quant EP_Q_BF16 and layout EP_LAYOUT_PACKED (the dispatch that
  *                wrote recv_buf), H % 64 == 0; otherwise EP_ERR_UNSUPPORTED
  *   recv_buf     the dispatch's receive buffer: bf16 [rows][H]
@@ -288,6 +289,39 @@ ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
                            const int64_t *expert_offset, const int64_t *recv_count,
                            const uint16_t *weights, int32_t n_out, uint16_t *y,
                            uint32_t *dev_status, ep_stream_t stream);
+
+/*
+ * The same linear maps on MXFP8 operands ("[feat] A5 deep fused moe
+ * supported": the deep-fused operator's grouped matrix multiplications take
+ * the e4m3 codes and e8m0 block scales its MX dispatch emits).  Element h of
+ * received row r is e4m3(code) * 2^(scale[r][h/32] - 127), and likewise for
+ * the weights; for each expert e and each of its received rows r
+ *   y[r, j] = bf16_rne( sum_h x[r, h] * W[e][j, h] )
+ * on the block-scaled tensor-core MMA (tcgen05 kind::mxf8f6f4, fp32
+ * accumulation); padding rows of y are not written.  Every product is exact
+ * and H/32 block sums are chained through one fp32 accumulator: results are
+ * within (H/32 + 32) * 2^-23 * sum_h |x*w| + 1 bf16 ulp of the exact sum.
+ * NaN codes, and scale bytes of 255 (NaN in the MX format), give unspecified
+ * values in the rows or columns they touch.
+ *   cfg          quant EP_Q_MXFP8 and layout EP_LAYOUT_PACKED (the dispatch that
+ *                wrote recv_buf), H % 128 == 0; otherwise EP_ERR_UNSUPPORTED
+ *   recv_buf     the dispatch's receive buffer: e4m3 [rows][H], then at
+ *                ep_sizes_t.recv_scale_offset e8m0 [rows][H/32]
+ *   expert_offset, recv_count   from ep_dispatch_layout
+ *   w_codes      e4m3 [E][n_out][H] (row j of W[e] is output column j)
+ *   w_scales     e8m0 [E][n_out][H/32]
+ *   n_out        output columns, a multiple of 224, 256 or 128 (tiles of 224
+ *                columns are taken where they divide n_out, else 256, else
+ *                128)
+ *   y            bf16 [rows][n_out] (n_out = H gives ep_combine's input)
+ * recv_buf, w_codes, w_scales and y 16-byte aligned (EP_ERR_MISALIGNED).
+ * A wait inside the kernel that exceeds 2 s sets EP_DEV_TIMEOUT and the
+ * kernel returns; it never traps.
+ */
+ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
+                              const int64_t *expert_offset, const int64_t *recv_count,
+                              const uint8_t *w_codes, const uint8_t *w_scales, int32_t n_out,
+                              uint16_t *y, uint32_t *dev_status, ep_stream_t stream);
 
 /*
  * Allocation-free variant of ep_dispatch_layout.  The pages have no

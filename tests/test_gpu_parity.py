@@ -16,7 +16,7 @@ import torch
 import combine_ep_dispatch_04_b200 as ep
 import oracle
 import synth
-from harness import Run, bf16_dev
+from harness import Run, bf16_dev, to_np_u16, ulp_distance
 
 pytestmark = pytest.mark.gpu
 
@@ -607,52 +607,94 @@ def _seeded_weights(E, n_out, H, scale, seed):
     return torch.randn(E, n_out, H, device="cuda", dtype=torch.bfloat16, generator=gen).mul_(scale)
 
 
-def _gemm_check(cfg, b, W, y, sample_rows=None):
-    """y against the oracle on the rows of every expert (or a sample).
+def _seeded_mx_weights(E, n_out, H, seed, lo=118, hi=134):
+    """Synthetic MXFP8 weights from a seeded generator: e4m3 codes uniform over
+    the bit patterns (the two NaN codes replaced by zero), e8m0 scales uniform
+    in [lo, hi)."""
+    gen = torch.Generator(device="cuda").manual_seed(seed)
+    c = torch.randint(0, 256, (E, n_out, H), device="cuda", dtype=torch.int16,
+                      generator=gen).to(torch.uint8)
+    c[(c & 0x7F) == 0x7F] = 0
+    sc = torch.randint(lo, hi, (E, n_out, H // 32), device="cuda", dtype=torch.int16,
+                       generator=gen).to(torch.uint8)
+    return c, sc
 
-    Every bf16 x bf16 product is exact in fp32.  The kernel adds them into an
-    fp32 accumulator in H/16 tensor-core steps of 16 products each; with the
-    sum inside one step taken in at least fp32 and any rounding of at most one
-    fp32 ulp (truncation allowed) per addition, the chain has at most
-    H/16 + 16 additions, so |acc - exact| <= (H/16 + 16) * 2^-23 * sum_h |x*w|,
-    and the bf16 rounding of acc adds at most one bf16 ulp of the result
-    (the oracle rounds the exact sum once).  Besides the bound, at least 90%
-    of the outputs equal the oracle's correctly rounded ones: the accumulation
-    error is far below half a bf16 ulp for almost every output.  Padding rows
-    stay untouched (0x7777).  Only the experts of the checked rows are copied
-    to the host."""
-    E, H = cfg.num_experts, cfg.hidden
-    n_out = W.shape[1]
-    eo = b.expert_offset.cpu().numpy()
-    cnt = b.recv_count.cpu().numpy()
-    rows = b.sizes["rows"]
-    xr = b.recv_data().view(torch.int16).cpu().numpy().view(np.uint16).reshape(rows, H)
+
+def _e4m3_table():
+    return oracle.e4m3_decode(np.arange(256, dtype=np.uint8)).astype(np.float64)
+
+
+def _check_expert_gemm(r, y, n_out, W=None, wc=None, ws=None, sample_rows=None):
+    """y from the GPU against the oracle's maps of the oracle's own receive rows
+    (its layout and its quantisation of the seeded x), on every valid row or a
+    sample; rows outside every expert untouched (0x7777).
+
+    Bound, from the arithmetic: every product is exact in fp32 and the kernel
+    chains H/16 (bf16: 16 products per tensor-core step) or H/32 (MXFP8: one
+    32-element scale block per step) partial sums through one fp32
+    accumulator, the sum inside a step taking at most 16 or 32 additions more;
+    with at most one fp32 ulp lost per addition (truncation allowed)
+    |acc - exact| <= chain * 2^-23 * sum_h |x*w|, and the final bf16 rounding
+    adds at most one bf16 ulp.  Besides the bound, at least 90% of the outputs
+    equal the oracle's correctly rounded ones."""
+    r.check_layout()
+    o = r.lay
+    E, H = r.w["E"], r.w["H"]
+    mx = wc is not None
+    eo, cnt = o["expert_offset"], o["recv_count"]
+    rows = r.sizes["rows"]
     got = y.view(torch.int16).cpu().numpy().view(np.uint16)
     valid = np.zeros(rows, bool)
     for e in range(E):
         valid[eo[e]:eo[e] + cnt[e]] = True
     assert np.all(got[~valid] == 0x7777)
-    expert_of = np.repeat(np.arange(E), np.diff(eo))
+    ns, _, rr = r.entries()
+    tok_of_row = np.full(rows, -1, np.int64)
+    tok_of_row[rr] = ns
+    expert_of = np.repeat(np.arange(E), np.diff(eo[:E + 1]))
     pick = np.nonzero(valid)[0]
     if sample_rows is not None and len(pick) > sample_rows:
         pick = np.sort(np.random.default_rng(0).choice(pick, sample_rows, replace=False))
+    lut = _e4m3_table()
 
     def f(u):
-        return (u.astype(np.uint32) << 16).view(np.float32)
+        return (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+    def mxv(c, sc):
+        return lut[c] * np.ldexp(1.0, np.repeat(sc.astype(np.int64) - 127, 32, axis=-1))
     same = 0
     for e in np.unique(expert_of[pick]):
         rs = pick[expert_of[pick] == e]
-        We = W[e].view(torch.int16).cpu().numpy().view(np.uint16)          # [n_out, H]
-        want = oracle.expert_gemm(xr[rs], We[None], np.zeros(1, np.int64),
-                                  np.array([len(rs)], np.int64), n_out)
-        mag = np.abs(f(xr[rs])).astype(np.float64) @ np.abs(f(We)).astype(np.float64).T
-        wf, gf = f(want).astype(np.float64), f(got[rs]).astype(np.float64)
+        q = [oracle.quant_row(r.omode, r.x[n], e4m3_qmax=r.qmax) for n in tok_of_row[rs]]
+        one, cnt1 = np.zeros(1, np.int64), np.array([len(rs)], np.int64)
+        if mx:
+            xc, xs = np.stack([d for d, _ in q]), np.stack([sc for _, sc in q])
+            wce, wse = wc[e].cpu().numpy(), ws[e].cpu().numpy()
+            want = oracle.expert_gemm_mx(xc, xs, wce[None], wse[None], one, cnt1, n_out)
+            xv, wv = mxv(xc, xs), mxv(wce, wse)
+            chain = H // 32 + 32
+        else:
+            xb = np.stack([d.view(np.uint16) for d, _ in q])
+            We = W[e].view(torch.int16).cpu().numpy().view(np.uint16)
+            want = oracle.expert_gemm(xb, We[None], one, cnt1, n_out)
+            xv, wv = f(xb), f(We)
+            chain = H // 16 + 16
+        mag = np.abs(xv).astype(np.float32) @ np.abs(wv).astype(np.float32).T
+        del wv
+        wf, gf = f(want), f(got[rs])
         ulp = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(wf), 2.0 ** -126))).astype(np.int64) - 7)
-        assert np.all(np.abs(gf - wf) <= ulp + mag * ((H // 16 + 16) * 2.0 ** -23)), int(e)
+        tol = ulp + mag.astype(np.float64) * (chain * 2.0 ** -23) * (1 + 2.0 ** -10)
+        assert np.all(np.abs(gf - wf) <= tol), int(e)
         same += int((got[rs] == want).sum())
     frac = same / (len(pick) * n_out)
     assert frac >= 0.9, frac
     return frac
+
+
+def _sentinel_y(r, n_out):
+    y = torch.empty((r.sizes["rows"], n_out), dtype=torch.bfloat16, device="cuda")
+    y.view(torch.int16).fill_(0x7777)
+    return y
 
 
 @pytest.mark.parametrize("n_out", [256, 768, 1280])
@@ -662,29 +704,91 @@ def test_expert_gemm_small(n_out):
     idx[idx == 3] = 5                      # expert 3 receives nothing
     r = Run(w, "bf16", layout="packed", align=8, idx=idx, wts=wts)
     W = _seeded_weights(w["E"], n_out, w["H"], 0.05, seed=n_out)
-    y = torch.full((r.sizes["rows"], n_out), 0.0, dtype=torch.bfloat16, device="cuda")
-    y.view(torch.int16).fill_(0x7777)
+    y = _sentinel_y(r, n_out)
     ep.ep_expert_gemm(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, W, y, r.b.dev_status)
     assert ep.ep_get_status(r.b.dev_status) == 0
-    assert r.b.recv_count.cpu().numpy()[3] == 0
-    _gemm_check(r.cfg, r.b, W, y)
+    assert r.lay["recv_count"][3] == 0
+    _check_expert_gemm(r, y, n_out, W=W)
 
 
 def test_expert_gemm_decode_shape_sampled():
     w = synth.workload("decode", layout="packed")
     r = Run(w, "bf16", layout="packed")
     W = _seeded_weights(w["E"], w["H"], w["H"], 0.02, seed=7)
-    y = torch.empty((r.sizes["rows"], w["H"]), dtype=torch.bfloat16, device="cuda")
-    y.view(torch.int16).fill_(0x7777)
+    y = _sentinel_y(r, w["H"])
     ep.ep_expert_gemm(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, W, y, r.b.dev_status)
     assert ep.ep_get_status(r.b.dev_status) == 0
-    _gemm_check(r.cfg, r.b, W, y, sample_rows=12)
+    _check_expert_gemm(r, y, w["H"], W=W, sample_rows=12)
+
+
+@pytest.mark.parametrize("n_out", [448, 256, 384])   # N tiles of 224, 256 and 128 columns
+def test_expert_gemm_mx_small(n_out):
+    w = synth.workload("tiny", R=4, T=40, M=48, K=4, E=8, H=640)
+    idx, wts = synth.make_routing(w)
+    idx[idx == 3] = 5                      # expert 3 receives nothing
+    r = Run(w, "mxfp8", layout="packed", align=8, idx=idx, wts=wts)
+    wc, ws = _seeded_mx_weights(w["E"], n_out, w["H"], seed=n_out)
+    y = _sentinel_y(r, n_out)
+    ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws, y,
+                         r.b.dev_status)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    _check_expert_gemm(r, y, n_out, wc=wc, ws=ws)
+
+
+def test_expert_gemm_mx_decode_shape_sampled():
+    w = synth.workload("decode", layout="packed")
+    r = Run(w, "mxfp8", layout="packed")
+    wc, ws = _seeded_mx_weights(w["E"], w["H"], w["H"], seed=9)
+    y = _sentinel_y(r, w["H"])
+    ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws, y,
+                         r.b.dev_status)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    _check_expert_gemm(r, y, w["H"], wc=wc, ws=ws, sample_rows=12)
+
+
+def test_expert_gemm_mx_rejects_other_formats():
+    w = synth.workload("tiny", R=2, T=16, M=16, K=2, E=4, H=256)
+    r = Run(w, "bf16", layout="packed")
+    wc, ws = _seeded_mx_weights(w["E"], 256, w["H"], seed=1)
+    y = _sentinel_y(r, 256)
+    with pytest.raises(ep.EpError):
+        ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws, y,
+                             r.b.dev_status)
+    wc2, ws2 = _seeded_mx_weights(w["E"], 96, w["H"], seed=1)    # no N tile divides 96
+    r2 = Run(w, "mxfp8", layout="packed")
+    with pytest.raises(ep.EpError):
+        ep.ep_expert_gemm_mx(r2.cfg, r2.b.recv_buf, r2.b.expert_offset, r2.b.recv_count, wc2, ws2,
+                             _sentinel_y(r2, 96), r2.b.dev_status)
+    assert torch.all(y.view(torch.int16) == 0x7777)
+
+
+def _pipeline_check(r, maps_fn, n_out, max_ulp):
+    """The GPU's combine of its expert outputs against the oracle's combine of
+    the oracle's expert outputs (oracle layout and quantisation of the seeded x)."""
+    w = r.w
+    o = r.lay
+    E, H = w["E"], w["H"]
+    eo, cnt = o["expert_offset"], o["recv_count"]
+    rows = r.sizes["rows"]
+    ns, _, rr = r.entries()
+    tok = {int(a): int(b) for a, b in zip(rr, ns)}
+    yw = np.zeros((rows, n_out), np.uint16)
+    for e in range(E):
+        rs = np.sort(rr[(rr >= eo[e]) & (rr < eo[e] + cnt[e])])
+        if len(rs) == 0:
+            continue
+        q = [oracle.quant_row(r.omode, r.x[tok[int(x)]], e4m3_qmax=r.qmax) for x in rs]
+        yw[rs] = maps_fn(e, q)
+    want, st = oracle.combine(w["R"], w["T"], w["K"], E, w["M"], H, yw, r.idx, r.wts,
+                              o["token_slot"], o["expert_offset"], layout="packed")
+    got = to_np_u16(r.b.out)
+    assert st == 0 and ulp_distance(got, want).max() <= max_ulp
 
 
 def test_dispatch_experts_combine_pipeline():
-    """dispatch -> the experts' linear maps -> combine, against the oracle's
-    combine of the oracle's expert outputs (one bf16 ulp for the experts'
-    rounding, one for the combine's)."""
+    """dispatch -> the experts' linear maps -> combine on the GPU, against the
+    oracle's chain (one bf16 ulp for the experts' rounding, one for the
+    combine's)."""
     w = synth.workload("tiny", R=2, T=32, M=32, K=4, E=8, H=256)
     r = Run(w, "bf16", layout="packed")
     n_out = w["H"]
@@ -694,13 +798,31 @@ def test_dispatch_experts_combine_pipeline():
     ep.ep_combine(r.cfg, r.b.y, r.idx_d, r.wts_d, r.b.token_slot, r.b.out, r.b.dev_status,
                   expert_offset=r.b.expert_offset)
     assert ep.ep_get_status(r.b.dev_status) == 0
-    eo = r.b.expert_offset.cpu().numpy()
-    cnt = r.b.recv_count.cpu().numpy()
-    xr = r.b.recv_data().view(torch.int16).cpu().numpy().view(np.uint16).reshape(-1, w["H"])
-    yw = oracle.expert_gemm(xr, W.view(torch.int16).cpu().numpy().view(np.uint16), eo[:w["E"]],
-                            cnt, n_out)
-    want, st = oracle.combine(w["R"], w["T"], w["K"], w["E"], w["M"], w["H"], yw, r.idx, r.wts,
-                              r.lay["token_slot"], r.lay["expert_offset"], layout="packed")
-    from harness import ulp_distance, to_np_u16
-    got = to_np_u16(r.b.out)
-    assert st == 0 and ulp_distance(got, want).max() <= 2
+    Wh = W.view(torch.int16).cpu().numpy().view(np.uint16)
+
+    def maps(e, q):
+        xb = np.stack([d.view(np.uint16) for d, _ in q])
+        return oracle.expert_gemm(xb, Wh[e][None], np.zeros(1, np.int64),
+                                  np.array([len(q)], np.int64), n_out)
+    _pipeline_check(r, maps, n_out, 2)
+
+
+def test_dispatch_mx_experts_combine_pipeline():
+    """MXFP8 dispatch -> the experts' block-scaled maps -> combine on the GPU,
+    against the oracle's chain."""
+    w = synth.workload("tiny", R=2, T=32, M=32, K=4, E=8, H=256)
+    r = Run(w, "mxfp8", layout="packed")
+    n_out = w["H"]
+    wc, ws = _seeded_mx_weights(w["E"], n_out, w["H"], seed=12, lo=112, hi=124)
+    ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws, r.b.y,
+                         r.b.dev_status)
+    ep.ep_combine(r.cfg, r.b.y, r.idx_d, r.wts_d, r.b.token_slot, r.b.out, r.b.dev_status,
+                  expert_offset=r.b.expert_offset)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    wch, wsh = wc.cpu().numpy(), ws.cpu().numpy()
+
+    def maps(e, q):
+        xc, xs = np.stack([d for d, _ in q]), np.stack([sc for _, sc in q])
+        return oracle.expert_gemm_mx(xc, xs, wch[e][None], wsh[e][None], np.zeros(1, np.int64),
+                                     np.array([len(q)], np.int64), n_out)
+    _pipeline_check(r, maps, n_out, 2)
