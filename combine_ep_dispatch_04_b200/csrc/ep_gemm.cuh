@@ -142,7 +142,9 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
                  : "memory");
 }
 
-// tile t of the walk -> expert, first row and first column (t < prefix[E])
+// tile t of the walk -> expert, first row and first column (t < prefix[E]).
+// Within an expert the row tiles vary fastest: the blocks that read the same
+// weight columns run side by side, so those columns come from DRAM once.
 __device__ __forceinline__ void gemm_tile(const int *prefix, int E, int ntn, int t, int &e,
                                           int &m0, int &n0, int bn = kGemmBN) {
     int lo = 0, hi = E - 1;  // the last e with prefix[e] <= t
@@ -153,8 +155,9 @@ __device__ __forceinline__ void gemm_tile(const int *prefix, int E, int ntn, int
     }
     e = lo;
     const int local = t - prefix[e];
-    m0 = (local / ntn) * kGemmBM;
-    n0 = (local % ntn) * bn;
+    const int mt = (prefix[e + 1] - prefix[e]) / ntn;  // row tiles of expert e
+    m0 = (local % mt) * kGemmBM;
+    n0 = (local / mt) * bn;
 }
 
 // tiles per expert, exclusive prefix into prefix[0..E] (one warp; each lane
@@ -374,6 +377,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // next tile's MMAs) where they and the scales fit in 512 columns, else one.
 // ---------------------------------------------------------------------------
 constexpr int kMxBK = 128, kMxStages = 4, kMxThreads = 224;
+constexpr int kSfGroup = 4;  // K steps whose scale loads the gathering warp issues together
 
 template <int BN>
 struct MxCfg {
@@ -557,6 +561,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
     } else if (warp == 2) {
         // ---- scales: 4 bytes (one K step) of every row of the A and B tiles
+        // The loads of kSfGroup K steps are issued together: one step's
+        // loads would leave a whole L2 latency between consecutive steps.
+        constexpr int G = kSfGroup;
         const int SB = a.H / 32;
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
@@ -566,40 +573,52 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             const int64_t arow0 = a.eo[e] + m0;
             const int64_t brow0 = (int64_t)e * a.N + n0;
             bool ok = true;
-            for (int kb = 0; kb < kblocks; kb++, it++) {
-                const int s = it % S, r = it / S;
-                uint32_t va[4], vb[C::kChunksB][4];
+            for (int kb0 = 0; kb0 < kblocks && ok; kb0 += G) {
+                const int g = min(G, kblocks - kb0);
+                uint32_t va[G][4], vb[G][C::kChunksB][4];
 #pragma unroll
-                for (int j = 0; j < 4; j++) {
-                    const int64_t row = arow0 + lane + 32 * j;
-                    va[j] = row < a.rows ? __ldg(reinterpret_cast<const uint32_t *>(
-                                               a.xs + row * SB + kb * 4))
-                                         : 0u;
-                }
-#pragma unroll
-                for (int c = 0; c < C::kChunksB; c++)
+                for (int q = 0; q < G; q++) {
+                    if (q >= g) break;
+                    const int kb = kb0 + q;
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
-                        const int n = 128 * c + 32 * j + lane;
-                        vb[c][j] = n < BN ? __ldg(reinterpret_cast<const uint32_t *>(
-                                                a.ws + (brow0 + n) * SB + kb * 4))
-                                          : 0u;
+                        const int64_t row = arow0 + lane + 32 * j;
+                        va[q][j] = row < a.rows ? __ldg(reinterpret_cast<const uint32_t *>(
+                                                      a.xs + row * SB + kb * 4))
+                                                : 0u;
                     }
-                int got = 1;
-                if (lane == 0) got = mbar_wait(smem_addr(&empty[s]), (r & 1) ^ 1);
-                if (!__shfl_sync(kFull, got, 0)) {
-                    ok = false;
-                    break;
-                }
-                const uint32_t st = smem_addr(sSF + s * C::kSfBytes) + lane * 16;
-                st_shared_v4(st, va[0], va[1], va[2], va[3]);
 #pragma unroll
-                for (int c = 0; c < C::kChunksB; c++)
-                    st_shared_v4(st + 512 * (1 + c), vb[c][0], vb[c][1], vb[c][2], vb[c][3]);
-                // the copies to TMEM read shared memory through the async proxy
-                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&full[s]));
+                    for (int c = 0; c < C::kChunksB; c++)
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            const int n = 128 * c + 32 * j + lane;
+                            vb[q][c][j] = n < BN ? __ldg(reinterpret_cast<const uint32_t *>(
+                                                       a.ws + (brow0 + n) * SB + kb * 4))
+                                                 : 0u;
+                        }
+                }
+#pragma unroll
+                for (int q = 0; q < G; q++) {
+                    if (q >= g) break;
+                    const int s = it % S, r = it / S;
+                    int got = 1;
+                    if (lane == 0) got = mbar_wait(smem_addr(&empty[s]), (r & 1) ^ 1);
+                    if (!__shfl_sync(kFull, got, 0)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t st = smem_addr(sSF + s * C::kSfBytes) + lane * 16;
+                    st_shared_v4(st, va[q][0], va[q][1], va[q][2], va[q][3]);
+#pragma unroll
+                    for (int c = 0; c < C::kChunksB; c++)
+                        st_shared_v4(st + 512 * (1 + c), vb[q][c][0], vb[q][c][1], vb[q][c][2],
+                                     vb[q][c][3]);
+                    // the copies to TMEM read shared memory through the async proxy
+                    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&full[s]));
+                    it++;
+                }
             }
             if (!ok) {
                 if (lane == 0) {
