@@ -77,6 +77,9 @@ def parse():
     p.add_argument("--gemm", action="store_true",
                    help="also time the experts' grouped GEMM (bf16, packed, N = H) on the "
                         "dispatched rows, outside the step")
+    p.add_argument("--gemm-experts", type=int, default=0,
+                   help="with --gemm: route the tokens onto this many experts (expert id "
+                        "modulo E) for the GEMM legs only, a small case for profilers")
     p.add_argument("--no-steady", action="store_true",
                    help="skip the steady-state pass and its buffer copies (profiling runs)")
     p.add_argument("--no-copy", action="store_true",
@@ -667,12 +670,23 @@ def graph_steps(ep, args, cfg, ccfg, b, x_d, idx_d, wts_d, g_d, flush, stream, d
             "value": round(world * N * args.steps / (total / 1e3), 1), "unit": "tokens/s"}
 
 
+def gemm_routing(E, idx_d, args):
+    """The GEMM legs' experts: the workload's, or --gemm-experts of them (expert
+    id modulo E; a token may then reach one expert twice, which the packed
+    layout receives as two rows)."""
+    if not args.gemm_experts or args.gemm_experts == E:
+        return E, idx_d
+    E2 = args.gemm_experts
+    return E2, torch.where(idx_d >= 0, torch.remainder(idx_d, E2), idx_d)
+
+
 def run_gemm(ep, w, x_d, idx_d, flush, stream, dev, args):
     """The experts between dispatch and combine (ep_expert_gemm): the workload's
     tokens dispatched as bf16 into the packed layout, one seeded random linear
     map of H x H per expert, timed alone between events after an L2 flush.
     FLOPs = 2 * (valid entries) * H * H."""
     R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
+    E, idx_d = gemm_routing(E, idx_d, args)
     cfg = ep.make_config(R, T, M, K, E, H, "bf16", "packed")
     b = ep.Buffers(cfg, device=dev, expert_out=False)
     ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
@@ -729,6 +743,7 @@ def run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args):
     L2 flush.  FLOPs = 2 * (valid entries) * H * H; the tensor peak is the
     measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)."""
     R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
+    E, idx_d = gemm_routing(E, idx_d, args)
     cfg = ep.make_config(R, T, M, K, E, H, "mxfp8", "packed")
     b = ep.Buffers(cfg, device=dev, expert_out=False)
     ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
