@@ -625,7 +625,11 @@ ep_status_t launch_combine_pipelined(const ep::CombineArgs &a, cudaStream_t s) {
 template <int QIN>
 ep_status_t launch_combine(const ep::CombineArgs &a, cudaStream_t s) {
     if constexpr (QIN != ep::QIN_BF16) {
-        if (a.K <= ep::kPipeRows && a.S % 4 == 0 && a.S <= ep::kPipeScaleBytes)
+        // The pipelined kernel's shared-memory stages cap it near 900 threads an
+        // SM; below about a million granules (decode-sized batches) the
+        // register kernel's higher occupancy wins.
+        if (a.K <= ep::kPipeRows && a.S % 4 == 0 && a.S <= ep::kPipeScaleBytes &&
+            a.N * (int64_t)(a.H / ep::combine_granule(QIN)) > ((int64_t)1 << 20))
             return launch_combine_pipelined<QIN>(a, s);
     }
     auto kernel_of = [](int t, int g) -> const void * {

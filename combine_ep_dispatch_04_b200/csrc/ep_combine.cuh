@@ -116,6 +116,16 @@ __device__ __forceinline__ bool pow2_fma(float (&acc)[combine_granule(QIN)], con
     return true;
 }
 
+// Whether pow2_fma is worth trying: int8 scales are never used that way, and
+// fp32 per-128 scales (amax / qmax, E4M3_B128 without round_scale) are almost
+// never powers of two; pow2_fma's result equals dequant_fma's wherever it applies.
+template <int QIN>
+__device__ __forceinline__ bool use_pow2(int sfmt) {
+    if constexpr (QIN == QIN_INT8 || QIN == QIN_BF16) return false;
+    if constexpr (QIN == QIN_E4M3_B128) return sfmt != 0;
+    return true;
+}
+
 template <int TPT, int GMAX, int KB, int QIN>
 __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs a) {
     pdl_enter();
@@ -210,9 +220,8 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
                 for (int kk = 0; kk < KB; kk++) {
                     const int k = k0 + kk;
                     if (k >= a.K || s_row[grp][k] < 0) continue;
-                    if constexpr (QIN != QIN_INT8) {
-                        if (pow2_fma<QIN>(acc, raw[kk], sc[kk], s_w[grp][k])) continue;
-                    }
+                    if (use_pow2<QIN>(a.sfmt) && pow2_fma<QIN>(acc, raw[kk], sc[kk], s_w[grp][k]))
+                        continue;
                     dequant_fma<QIN>(acc, raw[kk], sc[kk], s_w[grp][k]);
                 }
             }
@@ -335,6 +344,17 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_q_kernel(CombineAr
     __syncthreads();     // every thread's scale pieces
     if (!active) return;
 
+    // the token's weights and live rows, once (the unrolled entry loop below
+    // keeps them in registers)
+    float wk[KB];
+    uint32_t live = 0;
+#pragma unroll
+    for (int kk = 0; kk < KB; kk++) {
+        const bool ok = kk < a.K && s_row[grp][kk] >= 0;
+        live |= ok ? (1u << kk) : 0u;
+        wk[kk] = ok ? s_w[grp][kk] : 0.0f;
+    }
+    const bool try_pow2 = use_pow2<QIN>(a.sfmt);
 #pragma unroll 1
     for (int i = 0; i < GMAX; i++) {
         const int g = i * TPT + lt;
@@ -344,16 +364,27 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_q_kernel(CombineAr
         float acc[EPG];
 #pragma unroll
         for (int q = 0; q < EPG; q++) acc[q] = 0.0f;
-#pragma unroll 1  // a rolled loop keeps the body in the instruction cache
-        for (int kk = 0; kk < KB; kk++) {
-            if (kk >= a.K || s_row[grp][kk] < 0) continue;
-            const uint4 r = s_code[i & 1][kk][tid];
-            const float sc = scale_at<QIN>(&s_scl[grp][kk * (int)a.S], g, a.sfmt);
-            const float w = s_w[grp][kk];
-            if constexpr (QIN != QIN_INT8) {
+        if constexpr (QIN == QIN_MXFP4) {
+            // 32 accumulators a granule: the rolled loop is the faster one here
+#pragma unroll 1
+            for (int kk = 0; kk < KB; kk++) {
+                if (kk >= a.K || s_row[grp][kk] < 0) continue;
+                const uint4 r = s_code[i & 1][kk][tid];
+                const float sc = scale_at<QIN>(&s_scl[grp][kk * (int)a.S], g, a.sfmt);
+                const float w = s_w[grp][kk];
                 if (pow2_fma<QIN>(acc, r, sc, w)) continue;
+                dequant_fma<QIN>(acc, r, sc, w);
             }
-            dequant_fma<QIN>(acc, r, sc, w);
+        } else {
+            // the entries' decode chains are independent: unrolled, they overlap
+#pragma unroll
+            for (int kk = 0; kk < KB; kk++) {
+                if (!(live & (1u << kk))) continue;
+                const uint4 r = s_code[i & 1][kk][tid];
+                const float sc = scale_at<QIN>(&s_scl[grp][kk * (int)a.S], g, a.sfmt);
+                if (try_pow2 && pow2_fma<QIN>(acc, r, sc, wk[kk])) continue;
+                dequant_fma<QIN>(acc, r, sc, wk[kk]);
+            }
         }
         uint16_t *o = a.out + n * a.H + (int64_t)g * EPG;
 #pragma unroll
