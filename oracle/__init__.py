@@ -73,6 +73,8 @@ _lib.orc_expert_gemm.restype = None
 _lib.orc_expert_gemm.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p]
 _lib.orc_expert_gemm_mx.restype = None
 _lib.orc_expert_gemm_mx.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p]
+_lib.orc_expert_gemm_mxfp4.restype = None
+_lib.orc_expert_gemm_mxfp4.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p]
 _lib.orc_bwd_row.restype = None
 _lib.orc_bwd_row.argtypes = [_i, _f, _i, _p, _p, _p]
 _lib.orc_combine_gathered.restype = None
@@ -374,6 +376,28 @@ def expert_gemm_mx(xc, xs, wc, ws, expert_offset, count, n_out, y=None):
         y = np.zeros((rows, n_out), np.uint16)
     _lib.orc_expert_gemm_mx(E, H, n_out, _ptr(eo), _ptr(cnt), _ptr(xc), _ptr(xs), _ptr(wc),
                             _ptr(ws), _ptr(y))
+    return y
+
+
+def expert_gemm_mxfp4(xc, xs, wc, ws, expert_offset, count, n_out, y=None):
+    """Per-expert linear maps on MXFP4 operands: xc [rows, H/2] packed e2m1 codes
+    (even element in the low nibble), xs [rows, H/32] e8m0 bytes, wc [E, n_out, H/2],
+    ws [E, n_out, H/32]; rows expert_offset[e] .. + count[e] -> y [rows, n_out] bf16
+    bits (other rows of y untouched)."""
+    xc = _c(xc, np.uint8)
+    rows, D = xc.shape
+    H = 2 * D
+    xs = _c(xs, np.uint8)
+    wc = _c(wc, np.uint8)
+    ws = _c(ws, np.uint8)
+    E = wc.shape[0]
+    assert xs.shape == (rows, H // 32) and wc.shape == (E, n_out, D) and ws.shape == (E, n_out, H // 32)
+    eo = _c(expert_offset, np.int64)
+    cnt = _c(count, np.int64)
+    if y is None:
+        y = np.zeros((rows, n_out), np.uint16)
+    _lib.orc_expert_gemm_mxfp4(E, H, n_out, _ptr(eo), _ptr(cnt), _ptr(xc), _ptr(xs), _ptr(wc),
+                               _ptr(ws), _ptr(y))
     return y
 
 

@@ -640,6 +640,43 @@ void orc_expert_gemm_mx(int E, int H, int Nout, const int64_t *expert_offset, co
 }
 
 /*
+ * The same linear maps on MXFP4 operands (the deep-fused operator's MX
+ * formats include e2m1 with an e8m0 scale per 32 elements, as its MX
+ * dispatch emits): codes are packed two to a byte, element h in the low
+ * nibble of byte h/2 when h is even and in the high nibble when h is odd.
+ * Element h of row r is decode_e2m1(code) * 2^(xs[r, h/32] - 127), likewise
+ * for the weights; y[r, j] = bf16_rne( sum_h x[r, h] * w[e, j, h] ), the
+ * products exact in double, summed in h order, rounded to fp32 then bf16.
+ * A scale byte 255 gives NaN.  Rows past count[e] are left untouched.
+ */
+static double orc_e2m1_at(const uint8_t *row, int h)
+{
+    uint8_t b = row[h / 2];
+    return (double)orc_e2m1_decode((uint8_t)(h % 2 == 0 ? (b & 0xF) : (b >> 4)));
+}
+void orc_expert_gemm_mxfp4(int E, int H, int Nout, const int64_t *expert_offset,
+                           const int64_t *count, const uint8_t *xc, const uint8_t *xs,
+                           const uint8_t *wc, const uint8_t *ws, uint16_t *y)
+{
+    const int S = H / 32, D = H / 2;
+    for (int e = 0; e < E; e++) {
+        for (int64_t i = 0; i < count[e]; i++) {
+            int64_t r = expert_offset[e] + i;
+            for (int j = 0; j < Nout; j++) {
+                const int64_t wrow = (int64_t)e * Nout + j;
+                double acc = 0.0;
+                for (int h = 0; h < H; h++) {
+                    double xv = orc_e2m1_at(xc + r * D, h) * orc_e8m0_value(xs[r * S + h / 32]);
+                    double wv = orc_e2m1_at(wc + wrow * D, h) * orc_e8m0_value(ws[wrow * S + h / 32]);
+                    acc += xv * wv;
+                }
+                y[r * Nout + j] = orc_f32_to_bf16((float)acc);
+            }
+        }
+    }
+}
+
+/*
  * Dequantisation of one row stored in a quantised format ([FP8] The FP8
  * Combine Operation: the received codes times the stored inverse scale, in
  * fp32).  Each element is decode(code) * scale_inv as

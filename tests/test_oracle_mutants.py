@@ -17,8 +17,13 @@ from oracle.build import CFLAGS  # noqa: E402
 
 # name: ([(text in ep_oracle.c, replacement), ...], pins that must catch it)
 MUTANTS = {
+    "MXFP4 maps take a row scale per 32 packed bytes": (
+        [("orc_e2m1_at(xc + r * D, h) * orc_e8m0_value(xs[r * S + h / 32])",
+          "orc_e2m1_at(xc + r * D, h) * orc_e8m0_value(xs[r * S + h / 64])")],
+        "expert_gemm_mxfp4"),
     "MX weight scale read from the expert's first row": (
-        [("orc_e8m0_value(ws[wrow * S + h / 32])", "orc_e8m0_value(ws[(int64_t)e * Nout * S + h / 32])")],
+        [("orc_e4m3_decode(wc[wrow * H + h]) * orc_e8m0_value(ws[wrow * S + h / 32])",
+          "orc_e4m3_decode(wc[wrow * H + h]) * orc_e8m0_value(ws[(int64_t)e * Nout * S + h / 32])")],
         "expert_gemm_mx"),
     "MX scale bias off by one": (
         [("ldexp(1.0, (int)b - 127)", "ldexp(1.0, (int)b - 126)")], "expert_gemm_mx"),

@@ -940,3 +940,75 @@ def test_expert_gemm_mx_equals_bf16_maps_on_dequantised_operands():
     want = oracle.expert_gemm(xb, wb, eo, cnt, N)
     got = oracle.expert_gemm_mx(xc, xs, wc, ws, eo, cnt, N)
     assert np.array_equal(got, want)
+
+
+# the same maps on MXFP4 operands (packed e2m1 codes, e8m0 scale per 32)
+def _fp4_operands(r, shape, lo=120, hi=134):
+    """Seeded packed e2m1 codes (two a byte) and e8m0 scales for a [..., H] operand."""
+    c = r.integers(0, 256, shape[:-1] + (shape[-1] // 2,)).astype(np.uint8)
+    s = r.integers(lo, hi, shape[:-1] + (shape[-1] // 32,)).astype(np.uint8)
+    return c, s
+
+
+def _fp4_values(c, s):
+    """Dequantised values written out here: e2m1 table, even element in the low nibble."""
+    table = oracle.e2m1_decode(np.arange(16, dtype=np.uint8)).astype(np.float64)
+    v = np.empty(c.shape[:-1] + (2 * c.shape[-1],), np.float64)
+    v[..., 0::2] = table[c & 0xF]
+    v[..., 1::2] = table[c >> 4]
+    return v * np.ldexp(1.0, np.repeat(s.astype(np.int64) - 127, 32, axis=-1))
+
+
+def test_expert_gemm_mxfp4_identity_weights_give_the_dequantised_rows():
+    r = np.random.default_rng(6)
+    E, H = 2, 64
+    cnt = np.array([3, 4], np.int64)
+    eo = np.array([0, 4, 8], np.int64)
+    xc, xs = _fp4_operands(r, (8, H))
+    wc = np.zeros((E, H, H // 2), np.uint8)
+    for e in range(E):
+        for j in range(H):
+            wc[e, j, j // 2] = 0x2 if j % 2 == 0 else 0x20        # e2m1 1.0 at element j
+    ws = np.full((E, H, H // 32), 127, np.uint8)
+    y = oracle.expert_gemm_mxfp4(xc, xs, wc, ws, eo[:E], cnt, H, y=np.full((8, H), 0x7777, np.uint16))
+    for e in range(E):
+        for i in range(cnt[e]):
+            row = eo[e] + i
+            want = synth.to_bf16_bits(oracle.dequant_row("mxfp4", xc[row], xs[row], H))
+            want[want == 0x8000] = 0                                 # a sum of zero products is +0
+            assert np.array_equal(y[row], want), (e, i)
+    assert np.all(y[3] == 0x7777)
+
+
+def test_expert_gemm_mxfp4_equals_exact_rational_sums():
+    from fractions import Fraction
+    r = np.random.default_rng(7)
+    E, H, N = 2, 64, 4
+    cnt = np.array([2, 3], np.int64)
+    eo = np.array([0, 2], np.int64)
+    xc, xs = _fp4_operands(r, (5, H), 118, 136)
+    wc, ws = _fp4_operands(r, (E, N, H), 118, 136)
+    y = oracle.expert_gemm_mxfp4(xc, xs, wc, ws, eo, cnt, N)
+    xv, wv = _fp4_values(xc, xs), _fp4_values(wc, ws)
+    for e in range(E):
+        for i in range(cnt[e]):
+            row = eo[e] + i
+            for j in range(N):
+                exact = sum(Fraction(float(a)) * Fraction(float(b)) for a, b in zip(xv[row], wv[e, j]))
+                want = synth.to_bf16_bits(np.float32([float(exact)]))[0]
+                assert y[row, j] == want, (e, i, j)
+
+
+def test_expert_gemm_mxfp4_equals_bf16_maps_on_dequantised_operands():
+    r = np.random.default_rng(8)
+    E, H, N = 3, 256, 16
+    cnt = np.array([4, 0, 6], np.int64)
+    eo = np.array([0, 8, 8], np.int64)
+    xc, xs = _fp4_operands(r, (16, H))
+    wc, ws = _fp4_operands(r, (E, N, H))
+    xb = synth.to_bf16_bits(_fp4_values(xc, xs).astype(np.float32))
+    wb = synth.to_bf16_bits(_fp4_values(wc, ws).astype(np.float32))
+    assert np.array_equal(oracle.bf16_to_f32(xb).astype(np.float64), _fp4_values(xc, xs))
+    want = oracle.expert_gemm(xb, wb, eo, cnt, N)
+    got = oracle.expert_gemm_mxfp4(xc, xs, wc, ws, eo, cnt, N)
+    assert np.array_equal(got, want)
