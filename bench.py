@@ -559,6 +559,8 @@ def main():
 
     gemm = run_gemm(ep, w, x_d, idx_d, flush, stream, dev, args) if args.gemm else None
     gemm_mx = run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args) if args.gemm else None
+    gemm_mx4 = (run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args, "mxfp4")
+                if args.gemm and w["H"] % 256 == 0 else None)
 
     e2e = None if args.no_e2e else run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream,
                                           dev, args, world, step_bytes)
@@ -599,6 +601,7 @@ def main():
         "graph": graph,
         "expert_gemm": gemm,
         "expert_gemm_mx": gemm_mx,
+        "expert_gemm_mxfp4": gemm_mx4,
         "copy_gbs_same_run": copy_gbs,
         "e2e": e2e,
     }
@@ -735,23 +738,27 @@ def run_gemm(ep, w, x_d, idx_d, flush, stream, dev, args):
             "shape": f"{E} experts, {v} rows, {H} x {H} bf16 each"}
 
 
-def run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args):
-    """The experts' maps on MXFP8 operands (ep_expert_gemm_mx): the workload's
-    tokens dispatched as MXFP8 into the packed layout, seeded random MXFP8
-    weights of H x H per expert (e4m3 codes uniform over the finite bit
-    patterns, e8m0 scales in [118, 134)), timed alone between events after an
-    L2 flush.  FLOPs = 2 * (valid entries) * H * H; the tensor peak is the
-    measured bf16 peak times the nominal fp8 / bf16 ratio (4.5 / 2.25)."""
+def run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args, fmt="mxfp8"):
+    """The experts' maps on MX operands (ep_expert_gemm_mx): the workload's
+    tokens dispatched as MXFP8 or MXFP4 into the packed layout, seeded random
+    weights of H x H per expert in the same format (e4m3 codes uniform over
+    the finite bit patterns, or packed e2m1 bytes uniform over all 256; e8m0
+    scales in [118, 134)), timed alone between events after an L2 flush.
+    FLOPs = 2 * (valid entries) * H * H; the tensor peak is the measured bf16
+    peak times the nominal ratio (fp8 4.5 / 2.25, fp4 9 / 2.25)."""
     R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
     E, idx_d = gemm_routing(E, idx_d, args)
-    cfg = ep.make_config(R, T, M, K, E, H, "mxfp8", "packed")
+    fp4 = fmt == "mxfp4"
+    cfg = ep.make_config(R, T, M, K, E, H, fmt, "packed")
     b = ep.Buffers(cfg, device=dev, expert_out=False)
     ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
                                b.recv_buf, b.src_info, b.dev_status,
                                expert_offset=b.expert_offset, stream=stream)
     gen = torch.Generator(device=dev).manual_seed(4321)
-    wc = torch.randint(0, 256, (E, H, H), device=dev, dtype=torch.int16, generator=gen).to(torch.uint8)
-    wc[(wc & 0x7F) == 0x7F] = 0
+    D = H // 2 if fp4 else H
+    wc = torch.randint(0, 256, (E, H, D), device=dev, dtype=torch.int16, generator=gen).to(torch.uint8)
+    if not fp4:
+        wc[(wc & 0x7F) == 0x7F] = 0
     ws = torch.randint(118, 134, (E, H, H // 32), device=dev, dtype=torch.int16,
                        generator=gen).to(torch.uint8)
     y = torch.empty((b.sizes["rows"], H), dtype=torch.bfloat16, device=dev)
@@ -762,7 +769,7 @@ def run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args):
         call()
     torch.cuda.synchronize(dev)
     if ep.ep_get_status(b.dev_status) != 0:
-        raise SystemExit("ep_expert_gemm_mx reported a device error")
+        raise SystemExit(f"ep_expert_gemm_mx ({fmt}) reported a device error")
     v = int(b.recv_count.sum().item())
     reps = max(3, min(args.steps, 20))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -776,10 +783,11 @@ def run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args):
     ms = statistics.mean(a.elapsed_time(c) for a, c in evs)
     flops = 2.0 * v * H * H
     used = int((b.recv_count > 0).sum().item())
-    row = H + H / 32                      # codes and scales of one row
+    row = D + H / 32                      # codes and scales of one row
     nbytes = used * H * row + v * row + 2.0 * v * H
     peaks = measured_peaks() or {}
-    peak = (peaks.get("bf16_tflops") or 1590.0) * 2.0
+    ratio = 4.0 if fp4 else 2.0
+    peak = (peaks.get("bf16_tflops") or 1590.0) * ratio
     hbm = peaks.get("hbm_gbs") or 6650.0
     tf = flops / (ms * 1e-3) / 1e12
     t_tensor, t_hbm = flops / (peak * 1e12), nbytes / (hbm * 1e9)
@@ -789,10 +797,10 @@ def run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args):
             "gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
             "bound": "tensor" if t_tensor >= t_hbm else "hbm",
             "peak_tflops": peak, "peak_gbs": hbm,
-            "peak_source": ("measured bf16 x 2 (nominal fp8 / bf16)" if peaks.get("bf16_tflops")
-                            else "fallback bf16 x 2"),
+            "peak_source": (f"measured bf16 x {ratio:g} (nominal {'fp4' if fp4 else 'fp8'} / bf16)"
+                            if peaks.get("bf16_tflops") else f"fallback bf16 x {ratio:g}"),
             "frac": round(max(t_tensor, t_hbm) / (ms * 1e-3), 4),
-            "shape": f"{E} experts, {v} rows, {H} x {H} MXFP8 each"}
+            "shape": f"{E} experts, {v} rows, {H} x {H} {fmt.upper()} each"}
 
 
 STEADY_SETS = 4

@@ -863,24 +863,26 @@ bool u8_tile_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t oute
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// one launch of the MXFP8 kernel with N tiles of BN columns
-extern "C++" template <int BN>
+// one launch of the MX kernel (e4m3 or packed e2m1 codes) with N tiles of BN columns
+extern "C++" template <int BN, bool FP4>
 ep_status_t launch_gemm_mx(const Plan &p, const void *recv_buf, const int64_t *expert_offset,
                            const int64_t *recv_count, const uint8_t *w_codes,
                            const uint8_t *w_scales, int n_out, uint16_t *y,
                            uint32_t *dev_status, cudaStream_t s, int slot) {
+    const uint64_t D = FP4 ? (uint64_t)p.H / 2 : (uint64_t)p.H;  // code bytes of a row
     CUtensorMap ma, mb;
-    if (!u8_tile_map(&ma, recv_buf, (uint64_t)p.H, (uint64_t)p.rows, ep::kGemmBM) ||
-        !u8_tile_map(&mb, w_codes, (uint64_t)p.H, (uint64_t)p.E * n_out, BN))
+    if (!u8_tile_map(&ma, recv_buf, D, (uint64_t)p.rows, ep::kGemmBM) ||
+        !u8_tile_map(&mb, w_codes, D, (uint64_t)p.E * n_out, BN))
         return EP_ERR_CUDA;
     ep::MxArgs a;
     a.E = p.E; a.H = p.H; a.N = n_out; a.ntn = n_out / BN; a.rows = p.rows;
     a.eo = expert_offset; a.cnt = recv_count;
     a.xs = static_cast<const uint8_t *>(recv_buf) + p.scale_off;
     a.ws = w_scales; a.y = y; a.status = dev_status;
-    const size_t smem = ep::MxCfg<BN>::smem();
-    if (!allow_smem(ep::expert_gemm_mx_kernel<BN>, slot, smem)) return EP_ERR_CUDA;
-    launch(ep::expert_gemm_mx_kernel<BN>, (unsigned)sm_count(), ep::kMxThreads, smem, s, ma, mb, a);
+    const size_t smem = ep::MxCfg<BN, FP4>::smem();
+    if (!allow_smem(ep::expert_gemm_mx_kernel<BN, FP4>, slot, smem)) return EP_ERR_CUDA;
+    launch(ep::expert_gemm_mx_kernel<BN, FP4>, (unsigned)sm_count(), ep::kMxThreads, smem, s, ma,
+           mb, a);
     return launched();
 }
 
@@ -934,8 +936,10 @@ ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
     Plan p;
     ep_status_t st = make_plan(cfg, p);
     if (st != EP_OK) return st;
-    if (cfg->quant != EP_Q_MXFP8 || cfg->layout != EP_LAYOUT_PACKED) return EP_ERR_UNSUPPORTED;
-    if (p.H % ep::kMxBK != 0) return EP_ERR_UNSUPPORTED;
+    const bool fp4 = cfg->quant == EP_Q_MXFP4;
+    if ((cfg->quant != EP_Q_MXFP8 && !fp4) || cfg->layout != EP_LAYOUT_PACKED)
+        return EP_ERR_UNSUPPORTED;
+    if (p.H % (fp4 ? 2 * ep::kMxBK : ep::kMxBK) != 0) return EP_ERR_UNSUPPORTED;
     if (n_out <= 0) return EP_ERR_INVALID_ARG;
     const int bn = mx_tile_n(n_out);
     if (bn == 0) return EP_ERR_INVALID_ARG;
@@ -946,11 +950,18 @@ ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
         return EP_ERR_MISALIGNED;
     if (p.N == 0) return EP_OK;
     cudaStream_t s = cs(stream);
-    switch (bn) {
-    case 224: return launch_gemm_mx<224>(p, recv_buf, expert_offset, recv_count, w_codes, w_scales, n_out, y, dev_status, s, 6);
-    case 256: return launch_gemm_mx<256>(p, recv_buf, expert_offset, recv_count, w_codes, w_scales, n_out, y, dev_status, s, 7);
-    default:  return launch_gemm_mx<128>(p, recv_buf, expert_offset, recv_count, w_codes, w_scales, n_out, y, dev_status, s, 8);
+#define EP_MX(BN_, FP4_, SLOT_)                                                              \
+    return launch_gemm_mx<BN_, FP4_>(p, recv_buf, expert_offset, recv_count, w_codes, w_scales, \
+                                     n_out, y, dev_status, s, SLOT_)
+    if (fp4) {
+        if (bn == 224) EP_MX(224, true, 9);
+        if (bn == 256) EP_MX(256, true, 10);
+        EP_MX(128, true, 11);
     }
+    if (bn == 224) EP_MX(224, false, 6);
+    if (bn == 256) EP_MX(256, false, 7);
+    EP_MX(128, false, 8);
+#undef EP_MX
 }
 
 ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream) {

@@ -355,19 +355,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// MXFP8 operands: e4m3 codes with one e8m0 scale per 32 elements on both the
-// received rows and the weights, multiplied by the block-scaled MMA
-// (tcgen05.mma kind::mxf8f6f4.block_scale, K = 32 per instruction: one scale
-// per row of A and per row of B and instruction).
+// MX operands: e4m3 (MXFP8) or packed e2m1 (MXFP4) codes with one e8m0 scale
+// per 32 elements on both the received rows and the weights, multiplied by
+// the block-scaled MMA: tcgen05.mma kind::mxf8f6f4.block_scale (e4m3, K = 32
+// per instruction, one scale per row of A and of B) or kind::mxf4.block_scale
+// .block32 (e2m1 two a byte, K = 64, two scales per row).
 //
-// A K step is 128 codes (one 128-byte swizzle row): 4 instructions.  The
-// scales of a step are 4 bytes per row, read from the rows' scale region by
-// one gathering warp and written to shared memory in the arrangement that
-// tcgen05.cp .32x128b.warpx4 copies to TMEM: the 16 bytes of lane l hold rows
-// l, l+32, l+64, l+96 (4 bytes each: the step's 4 scale blocks), one 512-byte
-// chunk per 128 rows.  In TMEM row m's scale for block j then sits in lane
-// m % 32 (of every lane quarter), column m / 32, byte j; byte j is selected by
-// the scale-factor id of the instruction (bits 30-31 of the scale address).
+// A K step is 128 bytes of codes per row (one 128-byte swizzle row): 4
+// instructions, 4 (MXFP8) or 8 (MXFP4) scale blocks.  The scales of a step
+// are read from the rows' scale region by one gathering warp and written to
+// shared memory in the arrangement that tcgen05.cp .32x128b.warpx4 copies to
+// TMEM: per 128 rows and group of 4 scale blocks, a 512-byte chunk in which
+// the 16 bytes of lane l hold rows l, l+32, l+64, l+96 (4 bytes each).  In
+// TMEM row m's scale for block j of a group then sits in lane m % 32 (of
+// every lane quarter), column (group's first) + m / 32, byte j; an
+// instruction names the first of its blocks by the scale-factor id (byte j,
+// also bits 30-31 of the scale address).
 //
 // Warps: 0 loads the code tiles with TMA; 1 allocates TMEM and one lane
 // issues the scale copies and the MMAs; 2 gathers the scales; 3 - 6 run the
@@ -375,18 +378,22 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // warp has arrived.  TMEM holds kAcc accumulators of BN columns and the
 // scales behind them: two accumulators (the epilogue of one tile overlaps the
 // next tile's MMAs) where they and the scales fit in 512 columns, else one.
+// TMEM scale columns: A's groups (4 columns each), then B's (group-major,
+// then 128-row block).
 // ---------------------------------------------------------------------------
 constexpr int kMxBK = 128, kMxStages = 4, kMxThreads = 224;
 constexpr int kSfGroup = 4;  // K steps whose scale loads the gathering warp issues together
 
-template <int BN>
+template <int BN, bool FP4>
 struct MxCfg {
-    static constexpr int kChunksB = (BN + 127) / 128;      // 128-row scale chunks of B
-    static constexpr int kSfCols = 4 + 4 * kChunksB;       // TMEM columns of A's and B's scales
+    static constexpr int kNsf = FP4 ? 2 : 1;                // scale blocks per instruction
+    static constexpr int kGroups = kNsf;                    // groups of 4 blocks per K step
+    static constexpr int kChunksB = (BN + 127) / 128;       // 128-row blocks of B
+    static constexpr int kSfCols = 4 * kGroups * (1 + kChunksB);  // TMEM columns of the scales
     static constexpr int kAcc = (2 * BN + kSfCols <= 512) ? 2 : 1;
     static constexpr int kBytesA = kGemmBM * kMxBK;         // 16 KB
     static constexpr int kBytesB = BN * kMxBK;
-    static constexpr int kSfBytes = 512 * (1 + kChunksB);   // one stage's scales, A then B
+    static constexpr int kSfBytes = 512 * kGroups * (1 + kChunksB);  // a stage's scales, A then B
     static constexpr int kSfCol = kAcc * BN;                // TMEM column of A's scales
     static constexpr size_t smem() {
         return 1024 + (size_t)kMxStages * (kBytesA + kBytesB + kSfBytes) +
@@ -408,20 +415,31 @@ struct MxArgs {
     uint32_t *status;
 };
 
-// instruction descriptor of the block-scaled MMA: e4m3 A and B, both K-major,
-// e8m0 scales, N, M (the scale-factor ids are or-ed in per instruction)
-__host__ __device__ constexpr uint32_t umma_idesc_mxf8(int M, int N) {
-    return ((uint32_t)(N >> 3) << 17) | (1u << 23) | ((uint32_t)(M >> 4) << 24);
+// instruction descriptor of the block-scaled MMA: A and B formats (e4m3 = 0
+// for kind::mxf8f6f4, e2m1 = 1 for kind::mxf4), both K-major, e8m0 scales,
+// N, M (the scale-factor ids are or-ed in per instruction)
+__host__ __device__ constexpr uint32_t umma_idesc_mx(int M, int N, bool fp4) {
+    return (fp4 ? (1u << 7) | (1u << 10) : 0u) | ((uint32_t)(N >> 3) << 17) | (1u << 23) |
+           ((uint32_t)(M >> 4) << 24);
 }
-__device__ __forceinline__ void umma_mxf8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
-                                          uint32_t idesc, uint32_t tsfa, uint32_t tsfb,
-                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %6, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
-        ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(tsfa), "r"(tsfb), "r"(accumulate)
-        : "memory");
+template <bool FP4>
+__device__ __forceinline__ void umma_mx(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                        uint32_t idesc, uint32_t tsfa, uint32_t tsfb,
+                                        uint32_t accumulate) {
+    if constexpr (FP4)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(tsfa), "r"(tsfb), "r"(accumulate)
+            : "memory");
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "setp.ne.b32 p, %6, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}"
+            ::"r"(tmem_d), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(tsfa), "r"(tsfb), "r"(accumulate)
+            : "memory");
 }
 // shared-memory descriptor of 32 rows x 16 bytes, rows 16 bytes apart (no
 // swizzle, K-major: 8-row core matrices of 128 contiguous bytes, 128 bytes
@@ -440,11 +458,11 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
-template <int BN>
+template <int BN, bool FP4>
 __global__ void __launch_bounds__(kMxThreads, 1)
     expert_gemm_mx_kernel(const __grid_constant__ CUtensorMap tm_a,
                           const __grid_constant__ CUtensorMap tm_b, MxArgs a) {
-    using C = MxCfg<BN>;
+    using C = MxCfg<BN, FP4>;
     constexpr int S = kMxStages;
     extern __shared__ uint8_t gsm_raw[];
     uint8_t *gsm = reinterpret_cast<uint8_t *>(
@@ -489,7 +507,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
     const int total = prefix[E];
-    const int kblocks = a.H / kMxBK;
+    const int kblocks = (FP4 ? a.H / 2 : a.H) / kMxBK;  // 128-byte K steps
 
     if (warp == 0 && lane == 0) {
         // ---- code tiles
@@ -517,8 +535,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
     } else if (warp == 1 && lane == 0) {
         // ---- scale copies and MMAs
-        const uint32_t idesc = umma_idesc_mxf8(kGemmBM, BN);
-        const uint32_t tsfa = tmem_base + (uint32_t)C::kSfCol, tsfb = tsfa + 4;
+        const uint32_t idesc = umma_idesc_mx(kGemmBM, BN, FP4);
+        const uint32_t tsfa = tmem_base + (uint32_t)C::kSfCol, tsfb = tsfa + 4 * C::kGroups;
         int it = 0, tc = 0;
         for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x, tc++) {
             const int acc = tc % C::kAcc, use = tc / C::kAcc;
@@ -538,18 +556,19 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 }
                 tc_fence_after();
                 const uint32_t sf = smem_addr(sSF + s * C::kSfBytes);
-                tmem_cp_32x128b_x4(tsfa, sf_desc(sf));
 #pragma unroll
-                for (int c = 0; c < C::kChunksB; c++)
-                    tmem_cp_32x128b_x4(tsfb + 4 * c, sf_desc(sf + 512 * (1 + c)));
+                for (int c = 0; c < C::kGroups * (1 + C::kChunksB); c++)  // A's, then B's
+                    tmem_cp_32x128b_x4(tsfa + 4 * c, sf_desc(sf + 512 * c));
                 const uint64_t ad = umma_desc_sw128(smem_addr(sA + s * C::kBytesA));
                 const uint64_t bd = umma_desc_sw128(smem_addr(sB + s * C::kBytesB));
 #pragma unroll
-                for (int k = 0; k < kMxBK / 32; k++)  // 32 codes = 32 bytes = 2 units
-                    umma_mxf8(d, ad + 2 * k, bd + 2 * k,
-                              idesc | ((uint32_t)k << 29) | ((uint32_t)k << 4),
-                              tsfa | ((uint32_t)k << 30), tsfb | ((uint32_t)k << 30),
-                              (kb | k) != 0);
+                for (int k = 0; k < 4; k++) {  // 32 bytes of codes = 2 units each
+                    const int blk = k * C::kNsf, grp = blk / 4;
+                    const uint32_t byte = (uint32_t)(blk % 4);
+                    umma_mx<FP4>(d, ad + 2 * k, bd + 2 * k, idesc | (byte << 29) | (byte << 4),
+                                 (tsfa + 4 * grp) | (byte << 30),
+                                 (tsfb + 4 * C::kChunksB * grp) | (byte << 30), (kb | k) != 0);
+                }
                 umma_commit(smem_addr(&empty[s]));
             }
             if (!ok) {
@@ -575,27 +594,32 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             bool ok = true;
             for (int kb0 = 0; kb0 < kblocks && ok; kb0 += G) {
                 const int g = min(G, kblocks - kb0);
-                uint32_t va[G][4], vb[G][C::kChunksB][4];
+                constexpr int NG = C::kGroups;
+                uint32_t va[G][NG][4], vb[G][NG][C::kChunksB][4];
 #pragma unroll
                 for (int q = 0; q < G; q++) {
                     if (q >= g) break;
                     const int kb = kb0 + q;
 #pragma unroll
-                    for (int j = 0; j < 4; j++) {
-                        const int64_t row = arow0 + lane + 32 * j;
-                        va[q][j] = row < a.rows ? __ldg(reinterpret_cast<const uint32_t *>(
-                                                      a.xs + row * SB + kb * 4))
-                                                : 0u;
-                    }
-#pragma unroll
-                    for (int c = 0; c < C::kChunksB; c++)
+                    for (int gg = 0; gg < NG; gg++) {
+                        const int off = (kb * NG + gg) * 4;  // the group's 4 scale bytes
 #pragma unroll
                         for (int j = 0; j < 4; j++) {
-                            const int n = 128 * c + 32 * j + lane;
-                            vb[q][c][j] = n < BN ? __ldg(reinterpret_cast<const uint32_t *>(
-                                                       a.ws + (brow0 + n) * SB + kb * 4))
-                                                 : 0u;
+                            const int64_t row = arow0 + lane + 32 * j;
+                            va[q][gg][j] = row < a.rows ? __ldg(reinterpret_cast<const uint32_t *>(
+                                                              a.xs + row * SB + off))
+                                                        : 0u;
                         }
+#pragma unroll
+                        for (int c = 0; c < C::kChunksB; c++)
+#pragma unroll
+                            for (int j = 0; j < 4; j++) {
+                                const int n = 128 * c + 32 * j + lane;
+                                vb[q][gg][c][j] = n < BN ? __ldg(reinterpret_cast<const uint32_t *>(
+                                                               a.ws + (brow0 + n) * SB + off))
+                                                         : 0u;
+                            }
+                    }
                 }
 #pragma unroll
                 for (int q = 0; q < G; q++) {
@@ -608,11 +632,15 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                         break;
                     }
                     const uint32_t st = smem_addr(sSF + s * C::kSfBytes) + lane * 16;
-                    st_shared_v4(st, va[q][0], va[q][1], va[q][2], va[q][3]);
 #pragma unroll
-                    for (int c = 0; c < C::kChunksB; c++)
-                        st_shared_v4(st + 512 * (1 + c), vb[q][c][0], vb[q][c][1], vb[q][c][2],
-                                     vb[q][c][3]);
+                    for (int gg = 0; gg < NG; gg++) {
+                        st_shared_v4(st + 512 * gg, va[q][gg][0], va[q][gg][1], va[q][gg][2],
+                                     va[q][gg][3]);
+#pragma unroll
+                        for (int c = 0; c < C::kChunksB; c++)
+                            st_shared_v4(st + 512 * (NG + gg * C::kChunksB + c), vb[q][gg][c][0],
+                                         vb[q][gg][c][1], vb[q][gg][c][2], vb[q][gg][c][3]);
+                    }
                     // the copies to TMEM read shared memory through the async proxy
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
                     __syncwarp();

@@ -342,18 +342,20 @@ def ep_expert_gemm(cfg, recv_buf, expert_offset, recv_count, weights, y, dev_sta
 
 def ep_expert_gemm_mx(cfg, recv_buf, expert_offset, recv_count, w_codes, w_scales, y, dev_status,
                       stream=None, bind=False):
-    """The same maps on MXFP8 operands (packed MXFP8 receive layout): w_codes e4m3
-    [E, n_out, H] as uint8, w_scales e8m0 [E, n_out, H/32] as uint8, y bf16 [rows, n_out]."""
+    """The same maps on MX operands (packed MXFP8 or MXFP4 receive layout): w_codes
+    [E, n_out, D] as uint8 (D = H for e4m3, H/2 for packed e2m1), w_scales e8m0
+    [E, n_out, H/32] as uint8, y bf16 [rows, n_out]."""
     sz = ep_buffer_sizes(cfg)
     E, H = cfg.num_experts, cfg.hidden
+    D = sz["data_row_bytes"]
     if w_codes is None or w_codes.dim() != 3:
-        raise ValueError("w_codes must be a [E, n_out, H] tensor")
+        raise ValueError("w_codes must be a [E, n_out, D] tensor")
     n_out = int(w_codes.shape[1])
     args = [
         _bytes(recv_buf, "recv_buf", sz["recv_bytes"]),
         _dev(expert_offset, "expert_offset", torch.int64, (E + 1,)),
         _dev(recv_count, "recv_count", torch.int64, (E,)),
-        _dev(w_codes, "w_codes", torch.uint8, (E, n_out, H)),
+        _dev(w_codes, "w_codes", torch.uint8, (E, n_out, D)),
         _dev(w_scales, "w_scales", torch.uint8, (E, n_out, H // 32)),
         C.c_int32(n_out),
         _dev(y, "y", torch.bfloat16, (sz["rows"], n_out)),

@@ -291,24 +291,28 @@ ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
                            uint32_t *dev_status, ep_stream_t stream);
 
 /*
- * The same linear maps on MXFP8 operands ("[feat] A5 deep fused moe
- * supported": the deep-fused operator's grouped matrix multiplications take
- * the e4m3 codes and e8m0 block scales its MX dispatch emits).  Element h of
- * received row r is e4m3(code) * 2^(scale[r][h/32] - 127), and likewise for
- * the weights; for each expert e and each of its received rows r
+ * The same linear maps on MX operands ("[feat] A5 deep fused moe supported":
+ * the deep-fused operator's grouped matrix multiplications take the codes and
+ * e8m0 block scales its MX dispatch emits): MXFP8 (e4m3 codes) or MXFP4 (e2m1
+ * codes two a byte, element h in the low nibble of byte h/2 when h is even).
+ * Element h of received row r is code value * 2^(scale[r][h/32] - 127), and
+ * likewise for the weights; for each expert e and each of its received rows r
  *   y[r, j] = bf16_rne( sum_h x[r, h] * W[e][j, h] )
- * on the block-scaled tensor-core MMA (tcgen05 kind::mxf8f6f4, fp32
- * accumulation); padding rows of y are not written.  Every product is exact
- * and H/32 block sums are chained through one fp32 accumulator: results are
- * within (H/32 + 32) * 2^-23 * sum_h |x*w| + 1 bf16 ulp of the exact sum.
+ * on the block-scaled tensor-core MMA (tcgen05 kind::mxf8f6f4 or kind::mxf4,
+ * fp32 accumulation); padding rows of y are not written.  Every product is
+ * exact and H/32 block sums are chained through one fp32 accumulator: results
+ * are within (H/32 + 32) * 2^-23 * sum_h |x*w| + 1 bf16 ulp of the exact sum.
  * NaN codes, and scale bytes of 255 (NaN in the MX format), give unspecified
  * values in the rows or columns they touch.
- *   cfg          quant EP_Q_MXFP8 and layout EP_LAYOUT_PACKED (the dispatch that
- *                wrote recv_buf), H % 128 == 0; otherwise EP_ERR_UNSUPPORTED
- *   recv_buf     the dispatch's receive buffer: e4m3 [rows][H], then at
- *                ep_sizes_t.recv_scale_offset e8m0 [rows][H/32]
+ *   cfg          quant EP_Q_MXFP8 (H % 128 == 0) or EP_Q_MXFP4 (H % 256 == 0) and
+ *                layout EP_LAYOUT_PACKED (the dispatch that wrote recv_buf);
+ *                otherwise EP_ERR_UNSUPPORTED
+ *   recv_buf     the dispatch's receive buffer: codes [rows][D] (D = H, or H/2
+ *                for MXFP4), then at ep_sizes_t.recv_scale_offset e8m0
+ *                [rows][H/32]
  *   expert_offset, recv_count   from ep_dispatch_layout
- *   w_codes      e4m3 [E][n_out][H] (row j of W[e] is output column j)
+ *   w_codes      [E][n_out][D] in cfg's code format (row j of W[e] is output
+ *                column j)
  *   w_scales     e8m0 [E][n_out][H/32]
  *   n_out        output columns, a multiple of 224, 256 or 128 (tiles of 224
  *                columns are taken where they divide n_out, else 256, else

@@ -607,14 +607,15 @@ def _seeded_weights(E, n_out, H, scale, seed):
     return torch.randn(E, n_out, H, device="cuda", dtype=torch.bfloat16, generator=gen).mul_(scale)
 
 
-def _seeded_mx_weights(E, n_out, H, seed, lo=118, hi=134):
-    """Synthetic MXFP8 weights from a seeded generator: e4m3 codes uniform over
-    the bit patterns (the two NaN codes replaced by zero), e8m0 scales uniform
-    in [lo, hi)."""
+def _seeded_mx_weights(E, n_out, H, seed, lo=118, hi=134, fp4=False):
+    """Synthetic MX weights from a seeded generator: e4m3 codes uniform over the
+    bit patterns (the two NaN codes replaced by zero) or packed e2m1 bytes
+    uniform over all 256 (fp4: [E, n_out, H/2]), e8m0 scales uniform in [lo, hi)."""
     gen = torch.Generator(device="cuda").manual_seed(seed)
-    c = torch.randint(0, 256, (E, n_out, H), device="cuda", dtype=torch.int16,
+    c = torch.randint(0, 256, (E, n_out, H // 2 if fp4 else H), device="cuda", dtype=torch.int16,
                       generator=gen).to(torch.uint8)
-    c[(c & 0x7F) == 0x7F] = 0
+    if not fp4:
+        c[(c & 0x7F) == 0x7F] = 0
     sc = torch.randint(lo, hi, (E, n_out, H // 32), device="cuda", dtype=torch.int16,
                        generator=gen).to(torch.uint8)
     return c, sc
@@ -622,6 +623,15 @@ def _seeded_mx_weights(E, n_out, H, seed, lo=118, hi=134):
 
 def _e4m3_table():
     return oracle.e4m3_decode(np.arange(256, dtype=np.uint8)).astype(np.float64)
+
+
+def _e2m1_values(c):
+    """Values of packed e2m1 bytes (even element in the low nibble)."""
+    t = oracle.e2m1_decode(np.arange(16, dtype=np.uint8)).astype(np.float64)
+    v = np.empty(c.shape[:-1] + (2 * c.shape[-1],), np.float64)
+    v[..., 0::2] = t[c & 0xF]
+    v[..., 1::2] = t[c >> 4]
+    return v
 
 
 def _check_expert_gemm(r, y, n_out, W=None, wc=None, ws=None, sample_rows=None):
@@ -641,6 +651,7 @@ def _check_expert_gemm(r, y, n_out, W=None, wc=None, ws=None, sample_rows=None):
     o = r.lay
     E, H = r.w["E"], r.w["H"]
     mx = wc is not None
+    fp4 = r.mode == "mxfp4"
     eo, cnt = o["expert_offset"], o["recv_count"]
     rows = r.sizes["rows"]
     got = y.view(torch.int16).cpu().numpy().view(np.uint16)
@@ -661,7 +672,8 @@ def _check_expert_gemm(r, y, n_out, W=None, wc=None, ws=None, sample_rows=None):
         return (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
     def mxv(c, sc):
-        return lut[c] * np.ldexp(1.0, np.repeat(sc.astype(np.int64) - 127, 32, axis=-1))
+        v = _e2m1_values(c) if fp4 else lut[c]
+        return v * np.ldexp(1.0, np.repeat(sc.astype(np.int64) - 127, 32, axis=-1))
     same = 0
     for e in np.unique(expert_of[pick]):
         rs = pick[expert_of[pick] == e]
@@ -670,7 +682,8 @@ def _check_expert_gemm(r, y, n_out, W=None, wc=None, ws=None, sample_rows=None):
         if mx:
             xc, xs = np.stack([d for d, _ in q]), np.stack([sc for _, sc in q])
             wce, wse = wc[e].cpu().numpy(), ws[e].cpu().numpy()
-            want = oracle.expert_gemm_mx(xc, xs, wce[None], wse[None], one, cnt1, n_out)
+            gemm = oracle.expert_gemm_mxfp4 if fp4 else oracle.expert_gemm_mx
+            want = gemm(xc, xs, wce[None], wse[None], one, cnt1, n_out)
             xv, wv = mxv(xc, xs), mxv(wce, wse)
             chain = H // 32 + 32
         else:
@@ -746,10 +759,37 @@ def test_expert_gemm_mx_decode_shape_sampled():
     _check_expert_gemm(r, y, w["H"], wc=wc, ws=ws, sample_rows=12)
 
 
+@pytest.mark.parametrize("n_out", [448, 256, 384])   # N tiles of 224, 256 and 128 columns
+def test_expert_gemm_mxfp4_small(n_out):
+    w = synth.workload("tiny", R=4, T=40, M=48, K=4, E=8, H=768)
+    idx, wts = synth.make_routing(w)
+    idx[idx == 3] = 5                      # expert 3 receives nothing
+    r = Run(w, "mxfp4", layout="packed", align=8, idx=idx, wts=wts)
+    wc, ws = _seeded_mx_weights(w["E"], n_out, w["H"], seed=n_out + 1, fp4=True)
+    y = _sentinel_y(r, n_out)
+    ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws, y,
+                         r.b.dev_status)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    _check_expert_gemm(r, y, n_out, wc=wc, ws=ws)
+
+
+def test_expert_gemm_mxfp4_large_shape_sampled():
+    w = synth.workload("large")
+    r = Run(w, "mxfp4", layout="packed")
+    wc, ws = _seeded_mx_weights(w["E"], w["H"], w["H"], seed=10, fp4=True)
+    y = _sentinel_y(r, w["H"])
+    ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws, y,
+                         r.b.dev_status)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    _check_expert_gemm(r, y, w["H"], wc=wc, ws=ws, sample_rows=12)
+
+
 def test_expert_gemm_mx_rejects_other_formats():
     w = synth.workload("tiny", R=2, T=16, M=16, K=2, E=4, H=256)
     r = Run(w, "bf16", layout="packed")
-    wc, ws = _seeded_mx_weights(w["E"], 256, w["H"], seed=1)
+    # codes shaped as the binding expects for this format, so that the library rejects it
+    wc = torch.zeros((w["E"], 256, 2 * w["H"]), dtype=torch.uint8, device="cuda")
+    _, ws = _seeded_mx_weights(w["E"], 256, w["H"], seed=1)
     y = _sentinel_y(r, 256)
     with pytest.raises(ep.EpError):
         ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws, y,
@@ -804,6 +844,27 @@ def test_dispatch_experts_combine_pipeline():
         xb = np.stack([d.view(np.uint16) for d, _ in q])
         return oracle.expert_gemm(xb, Wh[e][None], np.zeros(1, np.int64),
                                   np.array([len(q)], np.int64), n_out)
+    _pipeline_check(r, maps, n_out, 2)
+
+
+def test_dispatch_mxfp4_experts_combine_pipeline():
+    """MXFP4 dispatch -> the experts' block-scaled maps -> combine on the GPU,
+    against the oracle's chain."""
+    w = synth.workload("tiny", R=2, T=32, M=32, K=4, E=8, H=512)
+    r = Run(w, "mxfp4", layout="packed")
+    n_out = w["H"]
+    wc, ws = _seeded_mx_weights(w["E"], n_out, w["H"], seed=13, lo=112, hi=124, fp4=True)
+    ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws, r.b.y,
+                         r.b.dev_status)
+    ep.ep_combine(r.cfg, r.b.y, r.idx_d, r.wts_d, r.b.token_slot, r.b.out, r.b.dev_status,
+                  expert_offset=r.b.expert_offset)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    wch, wsh = wc.cpu().numpy(), ws.cpu().numpy()
+
+    def maps(e, q):
+        xc, xs = np.stack([d for d, _ in q]), np.stack([sc for _, sc in q])
+        return oracle.expert_gemm_mxfp4(xc, xs, wch[e][None], wsh[e][None], np.zeros(1, np.int64),
+                                        np.array([len(q)], np.int64), n_out)
     _pipeline_check(r, maps, n_out, 2)
 
 
