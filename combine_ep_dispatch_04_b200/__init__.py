@@ -5,7 +5,7 @@ The work runs in libep.so (C ABI in include/ep.h, sm_100a CUDA kernels);
 library raises ImportError: there is no CPU or library fallback.
 """
 from .ep import (DEV_BAD_INDEX, DEV_CAPACITY_OVERFLOW, STATIC_SCRATCH_BYTES, F_BWD_UNWEIGHTED,
-                 F_COMBINE_QUANTIZED, F_IDX_I32, F_LAYOUT_CLUSTER, F_LAYOUT_MULTI_CTA,
+                 F_COMBINE_QUANTIZED, F_GEMM_CTA_PAIRS, F_IDX_I32, F_LAYOUT_CLUSTER, F_LAYOUT_MULTI_CTA,
                  F_LAYOUT_SINGLE_CTA, F_ROUND_SCALE, F_UE8M0, LAYOUT, QUANT, Bound, Buffers,
                  EpConfig, EpError, EpSizes, ep_buffer_sizes, ep_combine, ep_combine_backward,
                  ep_combine_backward_weights, ep_copy, ep_cvt_sweep, ep_dispatch, ep_dispatch_layout,
@@ -15,7 +15,7 @@ from .ep import (DEV_BAD_INDEX, DEV_CAPACITY_OVERFLOW, STATIC_SCRATCH_BYTES, F_B
 
 __all__ = [
     "DEV_BAD_INDEX", "DEV_CAPACITY_OVERFLOW", "STATIC_SCRATCH_BYTES", "F_BWD_UNWEIGHTED",
-    "F_COMBINE_QUANTIZED", "F_IDX_I32", "F_LAYOUT_CLUSTER", "F_LAYOUT_MULTI_CTA",
+    "F_COMBINE_QUANTIZED", "F_GEMM_CTA_PAIRS", "F_IDX_I32", "F_LAYOUT_CLUSTER", "F_LAYOUT_MULTI_CTA",
     "F_LAYOUT_SINGLE_CTA", "F_ROUND_SCALE", "F_UE8M0", "LAYOUT", "QUANT", "Bound", "Buffers",
     "EpConfig", "EpError", "EpSizes", "ep_buffer_sizes", "ep_combine", "ep_combine_backward",
     "ep_combine_backward_weights",

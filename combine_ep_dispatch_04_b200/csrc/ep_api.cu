@@ -110,7 +110,7 @@ ep_status_t make_plan(const ep_config_t *c, Plan &p) {
     if (!(c->e4m3_qmax >= 0.0f && c->e4m3_qmax <= 448.0f)) return EP_ERR_INVALID_ARG;  // NaN fails
     const uint32_t paths = EP_F_LAYOUT_SINGLE_CTA | EP_F_LAYOUT_MULTI_CTA | EP_F_LAYOUT_CLUSTER;
     const uint32_t known = EP_F_BWD_UNWEIGHTED | EP_F_COMBINE_QUANTIZED | EP_F_IDX_I32 |
-                           EP_F_ROUND_SCALE | EP_F_UE8M0 | paths;
+                           EP_F_ROUND_SCALE | EP_F_UE8M0 | EP_F_GEMM_CTA_PAIRS | paths;
     if (c->flags & ~known) return EP_ERR_INVALID_ARG;
     // power-of-two scales exist for the e4m3 / e2m1 formats only (MX scales
     // already are); e8m0 storage of the per-128 scales only for E4M3_B128
@@ -886,6 +886,37 @@ ep_status_t launch_gemm_mx(const Plan &p, const void *recv_buf, const int64_t *e
     return launched();
 }
 
+// Pairs of CTAs the two-CTA GEMM can hold resident at once (0: none, then
+// the one-CTA kernel runs), asked of the occupancy calculator once per device.
+int gemm_pairs() {
+    static std::atomic<int> pairs[kMaxDevices];
+    static std::atomic<bool> asked[kMaxDevices];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+    if (asked[dev].load()) return pairs[dev].load();
+    int n = 0;
+    const size_t smem = ep::gemm2_smem_bytes();
+    if (allow_smem(ep::expert_gemm2_kernel, 12, smem)) {
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(2 * (unsigned)(sm_count() / 2));
+        lc.blockDim = dim3(ep::kGemmThreads);
+        lc.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 1;
+        if (cudaOccupancyMaxActiveClusters(&n, ep::expert_gemm2_kernel, &lc) != cudaSuccess) n = 0;
+    }
+    cudaGetLastError();  // a refused query leaves no sticky error
+    n = std::max(0, std::min(n, sm_count() / 2));
+    pairs[dev].store(n);
+    asked[dev].store(true);
+    return n;
+}
+
 // N tile of the MXFP8 kernel: two accumulators of 224 columns where n_out
 // allows, else one of 256, else two of 128
 #ifndef EP_MX_PREFER_BN
@@ -915,13 +946,38 @@ ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
     if (!aligned16(recv_buf) || !aligned16(weights) || !aligned16(y)) return EP_ERR_MISALIGNED;
     if (p.N == 0) return EP_OK;
 
+    ep::GemmArgs a;
+    a.E = p.E; a.H = p.H; a.N = n_out; a.ntn = n_out / ep::kGemmBN;
+    a.eo = expert_offset; a.cnt = recv_count; a.y = y; a.status = dev_status;
+    const int pairs = (cfg->flags & EP_F_GEMM_CTA_PAIRS) ? gemm_pairs() : 0;
+    if (pairs > 0) {
+        CUtensorMap ma, mb;  // each CTA's halves: 128-row boxes
+        if (!bf16_tile_map(&ma, recv_buf, (uint64_t)p.H, (uint64_t)p.rows, 128) ||
+            !bf16_tile_map(&mb, weights, (uint64_t)p.H, (uint64_t)p.E * n_out, 128))
+            return EP_ERR_CUDA;
+        const size_t smem2 = ep::gemm2_smem_bytes();
+        if (!allow_smem(ep::expert_gemm2_kernel, 12, smem2)) return EP_ERR_CUDA;
+        cudaLaunchConfig_t lc = {};
+        lc.gridDim = dim3(2 * pairs);
+        lc.blockDim = dim3(ep::kGemmThreads);
+        lc.dynamicSmemBytes = smem2;
+        lc.stream = cs(stream);
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        lc.attrs = attr;
+        lc.numAttrs = 2;
+        cudaLaunchKernelEx(&lc, ep::expert_gemm2_kernel, ma, mb, a);
+        return launched();
+    }
     CUtensorMap ma, mb;
     if (!bf16_tile_map(&ma, recv_buf, (uint64_t)p.H, (uint64_t)p.rows, ep::kGemmBM) ||
         !bf16_tile_map(&mb, weights, (uint64_t)p.H, (uint64_t)p.E * n_out, ep::kGemmBN))
         return EP_ERR_CUDA;
-    ep::GemmArgs a;
-    a.E = p.E; a.H = p.H; a.N = n_out; a.ntn = n_out / ep::kGemmBN;
-    a.eo = expert_offset; a.cnt = recv_count; a.y = y; a.status = dev_status;
     const size_t smem = ep::gemm_smem_bytes();
     if (!allow_smem(ep::expert_gemm_kernel, 5, smem)) return EP_ERR_CUDA;
     launch(ep::expert_gemm_kernel, (unsigned)sm_count(), ep::kGemmThreads, smem, cs(stream), ma,

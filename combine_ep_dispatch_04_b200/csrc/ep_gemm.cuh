@@ -355,6 +355,296 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// bf16 on CTA pairs: the two-CTA MMA (tcgen05.mma.cta_group::2, M = 256).
+// A thread-block cluster of two CTAs on two SMs computes a 256-row x 256-column
+// output tile: CTA r holds rows 128r .. 128r+127 of A and rows 128r .. of the
+// tile's 256 weight rows (half of B), and its TMEM holds its 128 output rows.
+// One instruction multiplies the pair's whole tile, each SM reading its own
+// halves of A and B, so an SM reads half the B bytes per FLOP that a one-CTA
+// 128 x 256 tile reads.
+//
+// Both CTAs load their halves with the pair form of TMA, whose bytes complete
+// on the leader's (rank 0) stage barrier; the leader expects both CTAs' bytes
+// and one thread of it issues the MMAs, committing each stage to both CTAs'
+// empty barriers and each finished tile to both CTAs' accumulator barriers
+// (multicast commit).  Each CTA's epilogue reads its own TMEM rows and
+// arrives on the leader's accumulator-empty barrier (256 arrivals).  Waits
+// are bounded as in the one-CTA kernels; the pair meets at a cluster barrier
+// after its last MMA has completed and before either frees its TMEM.
+// ---------------------------------------------------------------------------
+constexpr int kG2Stages = 6;
+constexpr int kG2Half = 128 * kGemmBK * 2;  // 16 KB: a CTA's half of an A or B K step
+constexpr int kG2BM = 256, kG2BN = 256;
+
+__host__ __device__ constexpr size_t gemm2_smem_bytes() {
+    return 1024 + (size_t)kG2Stages * 2 * kG2Half + (2 * kG2Stages + 5) * 8 + 16 +
+           (kGemmMaxExperts + 1) * 4 + 256;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// shared::cluster address of the same variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t smem_in_rank(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
+// this CTA's half of a K step, completing on the leader's barrier
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap *map, int c0,
+                                                 int c1, uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar_cluster)
+        : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// arrive on the barrier at this shared offset in both CTAs of the pair once
+// the leader's MMAs issued so far have completed
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+        " [%0], %1;" ::"r"(bar),
+        "h"((uint16_t)0x3)
+        : "memory");
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    expert_gemm2_kernel(const __grid_constant__ CUtensorMap tm_a,
+                        const __grid_constant__ CUtensorMap tm_b, GemmArgs a) {
+    extern __shared__ uint8_t gsm_raw[];
+    uint8_t *gsm = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~(uintptr_t)1023);
+    constexpr int S = kG2Stages;
+    uint8_t *sA = gsm;
+    uint8_t *sB = gsm + S * kG2Half;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sB + S * kG2Half);
+    uint64_t *full = bars, *empty = bars + S;
+    uint64_t *accfull = bars + 2 * S, *accempty = accfull + 2;
+    uint64_t *drain = accempty + 2;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(drain + 1);
+    volatile uint32_t *s_abort = s_tmem + 1;
+    int *prefix = reinterpret_cast<int *>(s_tmem + 4);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int E = a.E;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; s++) {
+            mbar_init(smem_addr(&full[s]), 1);   // the leader's expect_tx (bytes of both CTAs)
+            mbar_init(smem_addr(&empty[s]), 1);  // the leader's multicast commit
+        }
+        for (int b = 0; b < 2; b++) {
+            mbar_init(smem_addr(&accfull[b]), 1);
+            mbar_init(smem_addr(&accempty[b]), 2 * 128);  // both CTAs' epilogue threads
+        }
+        mbar_init(smem_addr(drain), 1);
+        *s_abort = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 1) {  // both CTAs, same warp: 2 x 256 columns in each
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(s_tmem)),
+                     "r"(2 * kG2BN));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    }
+    pdl_enter();
+    if (warp == 0) {  // tiles of 256 rows
+        const int per = (E + 31) / 32;
+        int sum = 0;
+        for (int i = 0; i < per; i++) {
+            const int e = lane * per + i;
+            if (e < E) sum += (int)((a.cnt[e] + kG2BM - 1) / kG2BM) * a.ntn;
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(kFull, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+        for (int i = 0; i < per; i++) {
+            const int e = lane * per + i;
+            if (e < E) {
+                prefix[e] = run;
+                run += (int)((a.cnt[e] + kG2BM - 1) / kG2BM) * a.ntn;
+            }
+        }
+        if (lane == 31) prefix[E] = incl;
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // both CTAs' barriers initialised before any remote use
+    tc_fence_after();
+    const uint32_t tmem_base = *s_tmem;
+    const int total = prefix[E];
+    const int kblocks = a.H / kGemmBK;
+
+    // tile t -> expert, first row (of the pair's 256) and first column
+    auto tile = [&](int t, int &e, int &m0, int &n0) {
+        int lo = 0, hi = E - 1;
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (prefix[mid] <= t) lo = mid;
+            else hi = mid - 1;
+        }
+        e = lo;
+        const int local = t - prefix[e];
+        const int mt = (prefix[e + 1] - prefix[e]) / a.ntn;
+        m0 = (local % mt) * kG2BM;
+        n0 = (local / mt) * kG2BN;
+    };
+
+    if (warp == 0 && lane == 0) {
+        // ---- this CTA's halves of A and B
+        int it = 0;
+        for (int t = pair; t < total && !*s_abort; t += npairs) {
+            int e, m0, n0;
+            tile(t, e, m0, n0);
+            const int arow = (int)a.eo[e] + m0 + 128 * (int)rank;
+            const int brow = e * a.N + n0 + 128 * (int)rank;
+            for (int kb = 0; kb < kblocks; kb++, it++) {
+                const int s = it % S, r = it / S;
+                if (!mbar_wait(smem_addr(&empty[s]), (r & 1) ^ 1)) {
+                    *s_abort = 1u;
+                    atomicOr(a.status, kDevTimeout);
+                    break;
+                }
+                const uint32_t fb = smem_addr(&full[s]);
+                if (leader) mbar_expect_tx(fb, 2 * 2 * kG2Half);
+                const uint32_t fl = smem_in_rank(fb, 0);
+                tma_load_2d_pair(smem_addr(sA + s * kG2Half), &tm_a, kb * kGemmBK, arow, fl);
+                tma_load_2d_pair(smem_addr(sB + s * kG2Half), &tm_b, kb * kGemmBK, brow, fl);
+            }
+        }
+        if (leader)  // the pair's copies in flight land before the leader leaves
+            for (int j = 0; j < S && j < it; j++) {
+                const int i2 = it - 1 - j, s = i2 % S, r = i2 / S;
+                if (!mbar_wait(smem_addr(&full[s]), r & 1)) atomicOr(a.status, kDevTimeout);
+            }
+    } else if (warp == 1 && lane == 0 && leader) {
+        // ---- MMAs for the pair
+        const uint32_t idesc = umma_idesc_bf16(kG2BM, kG2BN);
+        int it = 0, tc = 0;
+        for (int t = pair; t < total && !*s_abort; t += npairs, tc++) {
+            const int acc = tc & 1, use = tc >> 1;
+            if (!mbar_wait(smem_addr(&accempty[acc]), (use & 1) ^ 1)) {
+                *s_abort = 1u;
+                atomicOr(a.status, kDevTimeout);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem_base + (uint32_t)(acc * kG2BN);
+            bool ok = true;
+            for (int kb = 0; kb < kblocks; kb++, it++) {
+                const int s = it % S, r = it / S;
+                if (!mbar_wait(smem_addr(&full[s]), r & 1)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint64_t ad = umma_desc_sw128(smem_addr(sA + s * kG2Half));
+                const uint64_t bd = umma_desc_sw128(smem_addr(sB + s * kG2Half));
+#pragma unroll
+                for (int k = 0; k < kGemmBK / 16; k++)
+                    umma_bf16_pair(d, ad + 2 * k, bd + 2 * k, idesc, (kb | k) != 0);
+                umma_commit_pair(smem_addr(&empty[s]));
+            }
+            if (!ok) {
+                *s_abort = 1u;
+                atomicOr(a.status, kDevTimeout);
+                break;
+            }
+            umma_commit_pair(smem_addr(&accfull[acc]));
+        }
+    } else if (warp >= 2) {
+        // ---- epilogue: this CTA's 128 rows of the pair's tile
+        const int sub = warp & 3;
+        const uint32_t empty_leader0 = smem_in_rank(smem_addr(&accempty[0]), 0);
+        const uint32_t empty_leader1 = smem_in_rank(smem_addr(&accempty[1]), 0);
+        int tc = 0;
+        for (int t = pair; t < total; t += npairs, tc++) {
+            const int acc = tc & 1, use = tc >> 1;
+            const bool ok =
+                __all_sync(kFull, !*s_abort && mbar_wait(smem_addr(&accfull[acc]), use & 1));
+            if (!ok) {
+                if (lane == 0) {
+                    *s_abort = 1u;
+                    atomicOr(a.status, kDevTimeout);
+                }
+                break;
+            }
+            tc_fence_after();
+            int e, m0, n0;
+            tile(t, e, m0, n0);
+            const int m = m0 + 128 * (int)rank + sub * 32 + lane;
+            const bool valid = m < a.cnt[e];
+            uint16_t *yrow = a.y + (a.eo[e] + m) * (int64_t)a.N + n0;
+            const uint32_t taddr =
+                tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * kG2BN);
+#pragma unroll 1
+            for (int c = 0; c < kG2BN / 16; c++) {
+                uint32_t v[16];
+                tmem_ld16(taddr + c * 16, v);
+                if (valid) {
+                    uint4 lo, hi;
+                    lo.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
+                    lo.y = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
+                    lo.z = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
+                    lo.w = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
+                    hi.x = pack_bf16x2(__uint_as_float(v[8]), __uint_as_float(v[9]));
+                    hi.y = pack_bf16x2(__uint_as_float(v[10]), __uint_as_float(v[11]));
+                    hi.z = pack_bf16x2(__uint_as_float(v[12]), __uint_as_float(v[13]));
+                    hi.w = pack_bf16x2(__uint_as_float(v[14]), __uint_as_float(v[15]));
+                    st_v4(yrow + c * 16, lo);
+                    st_v4(yrow + c * 16 + 8, hi);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive_remote(acc ? empty_leader1 : empty_leader0);
+        }
+    }
+    // the leader's MMAs have all completed before either CTA frees its TMEM (a
+    // commit to the leader's own barrier only)
+    if (warp == 1 && lane == 0 && leader && total > pair) {
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_addr(drain))
+                     : "memory");
+        if (!mbar_wait(smem_addr(drain), 0)) atomicOr(a.status, kDevTimeout);
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                     "r"(2 * kG2BN));
+    }
+}
+
+// ---------------------------------------------------------------------------
 // MX operands: e4m3 (MXFP8) or packed e2m1 (MXFP4) codes with one e8m0 scale
 // per 32 elements on both the received rows and the weights, multiplied by
 // the block-scaled MMA: tcgen05.mma kind::mxf8f6f4.block_scale (e4m3, K = 32

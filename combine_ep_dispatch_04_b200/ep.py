@@ -32,6 +32,7 @@ F_UE8M0 = 0x10
 F_LAYOUT_SINGLE_CTA = 0x100
 F_LAYOUT_MULTI_CTA = 0x200
 F_LAYOUT_CLUSTER = 0x400
+F_GEMM_CTA_PAIRS = 0x800
 
 STATIC_SCRATCH_BYTES = 1 << 20  # EP_STATIC_SCRATCH_BYTES of include/ep.h
 

@@ -90,6 +90,7 @@ typedef enum {
 #define EP_F_LAYOUT_SINGLE_CTA 0x100u /* force the one-block layout path */
 #define EP_F_LAYOUT_MULTI_CTA 0x200u  /* force the multi-block layout path */
 #define EP_F_LAYOUT_CLUSTER 0x400u    /* force the thread-block-cluster layout path */
+#define EP_F_GEMM_CTA_PAIRS 0x800u    /* ep_expert_gemm: two-CTA MMAs on CTA pairs */
 
 /*
  * Flags on the formats:
@@ -270,7 +271,9 @@ ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *
  * its received rows r (expert_offset[e] .. + recv_count[e] of the packed
  * receive layout):
  *   y[r, :] = bf16_rne( x[r, :] . W[e]^T )
- * with fp32 accumulation on the tensor cores (tcgen05, 128 x 256 tiles);
+ * with fp32 accumulation on the tensor cores (tcgen05: 128 x 256 tiles on
+ * single CTAs; with EP_F_GEMM_CTA_PAIRS in cfg->flags, where pairs of SMs can
+ * be scheduled, 256 x 256 tiles on CTA pairs with the two-CTA MMA);
  * padding rows of y (past recv_count[e]) are not written.  The summation
  * order of the fp32 accumulation is the hardware's: every product is exact
  * and H/16 partial sums are chained through one fp32 accumulator, so results

@@ -134,3 +134,9 @@ def test_status_strings():
     for s in range(7):
         assert lib.ep_status_string(s)
     assert b"unknown" in lib.ep_status_string(99)
+
+
+def test_gemm_pair_flag_is_known():
+    """EP_F_GEMM_CTA_PAIRS is a valid flag of any configuration (no launch)."""
+    cfg = ep.make_config(2, 16, 16, 2, 4, 256, "bf16", "packed", 1, 0.0, ep.F_GEMM_CTA_PAIRS)
+    assert ep.ep_buffer_sizes(cfg)["rows"] > 0

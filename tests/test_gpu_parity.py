@@ -710,18 +710,33 @@ def _sentinel_y(r, n_out):
     return y
 
 
+@pytest.mark.parametrize("pairs", [False, True])   # single CTAs / CTA pairs (two-CTA MMA)
 @pytest.mark.parametrize("n_out", [256, 768, 1280])
-def test_expert_gemm_small(n_out):
+def test_expert_gemm_small(n_out, pairs):
     w = synth.workload("tiny", R=4, T=40, M=48, K=4, E=8, H=640)
     idx, wts = synth.make_routing(w)
     idx[idx == 3] = 5                      # expert 3 receives nothing
-    r = Run(w, "bf16", layout="packed", align=8, idx=idx, wts=wts)
+    r = Run(w, "bf16", layout="packed", align=8, idx=idx, wts=wts,
+            flags=ep.F_GEMM_CTA_PAIRS if pairs else 0)
     W = _seeded_weights(w["E"], n_out, w["H"], 0.05, seed=n_out)
     y = _sentinel_y(r, n_out)
     ep.ep_expert_gemm(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, W, y, r.b.dev_status)
     assert ep.ep_get_status(r.b.dev_status) == 0
     assert r.lay["recv_count"][3] == 0
     _check_expert_gemm(r, y, n_out, W=W)
+
+
+@pytest.mark.parametrize("pairs", [False, True])
+def test_expert_gemm_many_row_tiles(pairs):
+    """Experts of several hundred rows: several row tiles, partial last tiles."""
+    w = synth.workload("tiny", R=2, T=512, M=512, K=4, E=8, H=512)
+    r = Run(w, "bf16", layout="packed", flags=ep.F_GEMM_CTA_PAIRS if pairs else 0)
+    W = _seeded_weights(w["E"], 512, w["H"], 0.05, seed=21)
+    y = _sentinel_y(r, 512)
+    ep.ep_expert_gemm(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, W, y, r.b.dev_status)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    assert r.lay["recv_count"].max() > 256
+    _check_expert_gemm(r, y, 512, W=W, sample_rows=200)
 
 
 def test_expert_gemm_decode_shape_sampled():
