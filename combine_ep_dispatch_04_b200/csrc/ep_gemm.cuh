@@ -142,6 +142,21 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
                  : "memory");
 }
 
+// 16 fp32 accumulator columns of one row -> 16 bf16 (round to nearest even)
+__device__ __forceinline__ void store_bf16x16(uint16_t *dst, const uint32_t (&v)[16]) {
+    uint4 lo, hi;
+    lo.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
+    lo.y = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
+    lo.z = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
+    lo.w = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
+    hi.x = pack_bf16x2(__uint_as_float(v[8]), __uint_as_float(v[9]));
+    hi.y = pack_bf16x2(__uint_as_float(v[10]), __uint_as_float(v[11]));
+    hi.z = pack_bf16x2(__uint_as_float(v[12]), __uint_as_float(v[13]));
+    hi.w = pack_bf16x2(__uint_as_float(v[14]), __uint_as_float(v[15]));
+    st_v4(dst, lo);
+    st_v4(dst + 8, hi);
+}
+
 // tile t of the walk -> expert, first row and first column (t < prefix[E]).
 // Within an expert the row tiles vary fastest: the blocks that read the same
 // weight columns run side by side, so those columns come from DRAM once.
@@ -163,12 +178,12 @@ __device__ __forceinline__ void gemm_tile(const int *prefix, int E, int ntn, int
 // tiles per expert, exclusive prefix into prefix[0..E] (one warp; each lane
 // takes a run of experts)
 __device__ __forceinline__ void tile_prefix(int *prefix, int E, const int64_t *cnt, int ntn,
-                                            int lane) {
+                                            int lane, int bm = kGemmBM) {
     const int per = (E + 31) / 32;
     int sum = 0;
     for (int i = 0; i < per; i++) {
         const int e = lane * per + i;
-        if (e < E) sum += (int)((cnt[e] + kGemmBM - 1) / kGemmBM) * ntn;
+        if (e < E) sum += (int)((cnt[e] + bm - 1) / bm) * ntn;
     }
     int incl = sum;
 #pragma unroll
@@ -181,7 +196,7 @@ __device__ __forceinline__ void tile_prefix(int *prefix, int E, const int64_t *c
         const int e = lane * per + i;
         if (e < E) {
             prefix[e] = run;
-            run += (int)((cnt[e] + kGemmBM - 1) / kGemmBM) * ntn;
+            run += (int)((cnt[e] + bm - 1) / bm) * ntn;
         }
     }
     if (lane == 31) prefix[E] = incl;
@@ -321,19 +336,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int c = 0; c < kGemmBN / 16; c++) {
                 uint32_t v[16];
                 tmem_ld16(taddr + c * 16, v);
-                if (valid) {
-                    uint4 lo, hi;
-                    lo.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
-                    lo.y = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
-                    lo.z = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
-                    lo.w = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
-                    hi.x = pack_bf16x2(__uint_as_float(v[8]), __uint_as_float(v[9]));
-                    hi.y = pack_bf16x2(__uint_as_float(v[10]), __uint_as_float(v[11]));
-                    hi.z = pack_bf16x2(__uint_as_float(v[12]), __uint_as_float(v[13]));
-                    hi.w = pack_bf16x2(__uint_as_float(v[14]), __uint_as_float(v[15]));
-                    st_v4(yrow + c * 16, lo);
-                    st_v4(yrow + c * 16 + 8, hi);
-                }
+                if (valid) store_bf16x16(yrow + c * 16, v);
             }
             tc_fence_before();
             mbar_arrive(smem_addr(&accempty[acc]));
@@ -471,29 +474,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
     }
     pdl_enter();
-    if (warp == 0) {  // tiles of 256 rows
-        const int per = (E + 31) / 32;
-        int sum = 0;
-        for (int i = 0; i < per; i++) {
-            const int e = lane * per + i;
-            if (e < E) sum += (int)((a.cnt[e] + kG2BM - 1) / kG2BM) * a.ntn;
-        }
-        int incl = sum;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int v = __shfl_up_sync(kFull, incl, o);
-            if (lane >= o) incl += v;
-        }
-        int run = incl - sum;
-        for (int i = 0; i < per; i++) {
-            const int e = lane * per + i;
-            if (e < E) {
-                prefix[e] = run;
-                run += (int)((a.cnt[e] + kG2BM - 1) / kG2BM) * a.ntn;
-            }
-        }
-        if (lane == 31) prefix[E] = incl;
-    }
+    if (warp == 0) tile_prefix(prefix, E, a.cnt, a.ntn, lane, kG2BM);  // tiles of 256 rows
     tc_fence_before();
     __syncthreads();
     cluster_sync_all();  // both CTAs' barriers initialised before any remote use
@@ -608,19 +589,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             for (int c = 0; c < kG2BN / 16; c++) {
                 uint32_t v[16];
                 tmem_ld16(taddr + c * 16, v);
-                if (valid) {
-                    uint4 lo, hi;
-                    lo.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
-                    lo.y = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
-                    lo.z = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
-                    lo.w = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
-                    hi.x = pack_bf16x2(__uint_as_float(v[8]), __uint_as_float(v[9]));
-                    hi.y = pack_bf16x2(__uint_as_float(v[10]), __uint_as_float(v[11]));
-                    hi.z = pack_bf16x2(__uint_as_float(v[12]), __uint_as_float(v[13]));
-                    hi.w = pack_bf16x2(__uint_as_float(v[14]), __uint_as_float(v[15]));
-                    st_v4(yrow + c * 16, lo);
-                    st_v4(yrow + c * 16 + 8, hi);
-                }
+                if (valid) store_bf16x16(yrow + c * 16, v);
             }
             tc_fence_before();
             mbar_arrive_remote(acc ? empty_leader1 : empty_leader0);
@@ -973,19 +942,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             for (int c = 0; c < BN / 16; c++) {
                 uint32_t v[16];
                 tmem_ld16(taddr + c * 16, v);
-                if (valid) {
-                    uint4 lo, hi;
-                    lo.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
-                    lo.y = pack_bf16x2(__uint_as_float(v[2]), __uint_as_float(v[3]));
-                    lo.z = pack_bf16x2(__uint_as_float(v[4]), __uint_as_float(v[5]));
-                    lo.w = pack_bf16x2(__uint_as_float(v[6]), __uint_as_float(v[7]));
-                    hi.x = pack_bf16x2(__uint_as_float(v[8]), __uint_as_float(v[9]));
-                    hi.y = pack_bf16x2(__uint_as_float(v[10]), __uint_as_float(v[11]));
-                    hi.z = pack_bf16x2(__uint_as_float(v[12]), __uint_as_float(v[13]));
-                    hi.w = pack_bf16x2(__uint_as_float(v[14]), __uint_as_float(v[15]));
-                    st_v4(yrow + c * 16, lo);
-                    st_v4(yrow + c * 16 + 8, hi);
-                }
+                if (valid) store_bf16x16(yrow + c * 16, v);
             }
             tc_fence_before();
             mbar_arrive(smem_addr(&accempty[acc]));
