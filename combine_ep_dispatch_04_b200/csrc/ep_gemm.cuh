@@ -843,6 +843,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         // loads would leave a whole L2 latency between consecutive steps.
         constexpr int G = kSfGroup;
         const int SB = a.H / 32;
+        // 16-byte loads where every row's scales start on a 16-byte boundary
+        // (the scale regions themselves are 16-byte aligned)
+        const bool vec = SB % 16 == 0;
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             if (__shfl_sync(kFull, (int)*s_abort, 0)) break;
@@ -855,6 +858,40 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 const int g = min(G, kblocks - kb0);
                 constexpr int NG = C::kGroups;
                 uint32_t va[G][NG][4], vb[G][NG][C::kChunksB][4];
+                if (vec && g == G) {
+                    // a row's scales of the G steps are G * NG contiguous words,
+                    // 16-byte aligned: NG 16-byte loads per row
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const int64_t row = arow0 + lane + 32 * j;
+#pragma unroll
+                        for (int h = 0; h < NG; h++) {
+                            const uint4 w4 = row < a.rows
+                                                 ? __ldg(reinterpret_cast<const uint4 *>(
+                                                       a.xs + row * SB + kb0 * NG * 4) + h)
+                                                 : make_uint4(0u, 0u, 0u, 0u);
+                            const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                            for (int u = 0; u < 4; u++) va[(4 * h + u) / NG][(4 * h + u) % NG][j] = wv[u];
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < C::kChunksB; c++)
+#pragma unroll
+                        for (int j = 0; j < 4; j++) {
+                            const int n = 128 * c + 32 * j + lane;
+#pragma unroll
+                            for (int h = 0; h < NG; h++) {
+                                const uint4 w4 = n < BN ? __ldg(reinterpret_cast<const uint4 *>(
+                                                              a.ws + (brow0 + n) * SB + kb0 * NG * 4) + h)
+                                                        : make_uint4(0u, 0u, 0u, 0u);
+                                const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+                                for (int u = 0; u < 4; u++)
+                                    vb[(4 * h + u) / NG][(4 * h + u) % NG][c][j] = wv[u];
+                            }
+                        }
+                } else {
 #pragma unroll
                 for (int q = 0; q < G; q++) {
                     if (q >= g) break;
@@ -879,6 +916,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                                                          : 0u;
                             }
                     }
+                }
                 }
 #pragma unroll
                 for (int q = 0; q < G; q++) {
