@@ -557,9 +557,9 @@ def main():
     except Exception:
         pass
 
-    gemm = run_gemm(ep, w, x_d, idx_d, flush, stream, dev, args) if args.gemm else None
-    gemm_mx = run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args) if args.gemm else None
-    gemm_mx4 = (run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args, "mxfp4")
+    gemm = run_gemm(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args) if args.gemm else None
+    gemm_mx = run_gemm_mx(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args) if args.gemm else None
+    gemm_mx4 = (run_gemm_mx(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args, "mxfp4")
                 if args.gemm and w["H"] % 256 == 0 else None)
 
     e2e = None if args.no_e2e else run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream,
@@ -683,7 +683,37 @@ def gemm_routing(E, idx_d, args):
     return E2, torch.where(idx_d >= 0, torch.remainder(idx_d, E2), idx_d)
 
 
-def run_gemm(ep, w, x_d, idx_d, flush, stream, dev, args):
+def time_moe_forward(ep, cfg, b, x_d, idx_d, wts_d, wc, ws, y, flush, stream, dev, args):
+    """The whole forward path in one call (ep_moe_forward: layout + dispatch ->
+    the experts' maps -> combine) with the GEMM leg's weights, timed alone
+    between events after an L2 flush; tokens/s = N / time."""
+    N, H = cfg.num_ranks * cfg.num_tokens, cfg.hidden
+    out = torch.empty((N, H), dtype=torch.bfloat16, device=dev)
+    call = ep.ep_moe_forward(cfg, x_d, idx_d, wts_d, wc, ws, b.token_slot, b.recv_count,
+                             b.expert_offset, b.workspace, b.recv_buf, b.src_info, y, out,
+                             b.dev_status, stream=stream, bind=True)
+    for _ in range(3):
+        flush(1)
+        call()
+    torch.cuda.synchronize(dev)
+    if ep.ep_get_status(b.dev_status) != 0:
+        raise SystemExit("ep_moe_forward reported a device error")
+    reps = max(3, min(args.steps, 20))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(reps)]
+    for s in range(reps):
+        flush(s & 0xFF)
+        evs[s][0].record(stream)
+        call()
+        evs[s][1].record(stream)
+    torch.cuda.synchronize(dev)
+    ms = statistics.mean(a.elapsed_time(c) for a, c in evs)
+    del out
+    return {"ms": round(ms, 4), "tokens_per_s": round(N / (ms * 1e-3), 1),
+            "launches": 4, "what": "layout + dispatch, the experts' maps (n_out = H), combine"}
+
+
+def run_gemm(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args):
     """The experts between dispatch and combine (ep_expert_gemm): the workload's
     tokens dispatched as bf16 into the packed layout, one seeded random linear
     map of H x H per expert, timed alone between events after an L2 flush.
@@ -727,6 +757,7 @@ def run_gemm(ep, w, x_d, idx_d, flush, stream, dev, args):
     hbm = peaks.get("hbm_gbs") or 6650.0
     tf = flops / (ms * 1e-3) / 1e12
     t_tensor, t_hbm = flops / (peak * 1e12), nbytes / (hbm * 1e9)
+    moe = time_moe_forward(ep, cfg, b, x_d, idx_d, wts_d, W, None, y, flush, stream, dev, args)
     del W, y, b
     torch.cuda.empty_cache()
     return {"ms": round(ms, 4), "flops": flops, "bytes": nbytes, "tflops": round(tf, 1),
@@ -735,10 +766,10 @@ def run_gemm(ep, w, x_d, idx_d, flush, stream, dev, args):
             "peak_tflops": peak, "peak_gbs": hbm,
             "peak_source": "measured" if peaks.get("bf16_tflops") else "fallback",
             "frac": round(max(t_tensor, t_hbm) / (ms * 1e-3), 4),
-            "shape": f"{E} experts, {v} rows, {H} x {H} bf16 each"}
+            "shape": f"{E} experts, {v} rows, {H} x {H} bf16 each", "moe_forward": moe}
 
 
-def run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args, fmt="mxfp8"):
+def run_gemm_mx(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args, fmt="mxfp8"):
     """The experts' maps on MX operands (ep_expert_gemm_mx): the workload's
     tokens dispatched as MXFP8 or MXFP4 into the packed layout, seeded random
     weights of H x H per expert in the same format (e4m3 codes uniform over
@@ -791,6 +822,7 @@ def run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args, fmt="mxfp8"):
     hbm = peaks.get("hbm_gbs") or 6650.0
     tf = flops / (ms * 1e-3) / 1e12
     t_tensor, t_hbm = flops / (peak * 1e12), nbytes / (hbm * 1e9)
+    moe = time_moe_forward(ep, cfg, b, x_d, idx_d, wts_d, wc, ws, y, flush, stream, dev, args)
     del wc, ws, y, b
     torch.cuda.empty_cache()
     return {"ms": round(ms, 4), "flops": flops, "bytes": nbytes, "tflops": round(tf, 1),
@@ -800,7 +832,7 @@ def run_gemm_mx(ep, w, x_d, idx_d, flush, stream, dev, args, fmt="mxfp8"):
             "peak_source": (f"measured bf16 x {ratio:g} (nominal {'fp4' if fp4 else 'fp8'} / bf16)"
                             if peaks.get("bf16_tflops") else f"fallback bf16 x {ratio:g}"),
             "frac": round(max(t_tensor, t_hbm) / (ms * 1e-3), 4),
-            "shape": f"{E} experts, {v} rows, {H} x {H} {fmt.upper()} each"}
+            "shape": f"{E} experts, {v} rows, {H} x {H} {fmt.upper()} each", "moe_forward": moe}
 
 
 STEADY_SETS = 4

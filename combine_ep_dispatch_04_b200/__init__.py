@@ -11,7 +11,7 @@ from .ep import (DEV_BAD_INDEX, DEV_CAPACITY_OVERFLOW, STATIC_SCRATCH_BYTES, F_B
                  ep_combine_backward_weights, ep_copy, ep_cvt_sweep, ep_dispatch, ep_dispatch_layout,
                  ep_dispatch_layout_static, ep_dispatch_with_layout, ep_expert_gemm, ep_expert_gemm_mx,
                  ep_get_status,
-                 ep_kernel_launches, idx_dtype, make_config)
+                 ep_kernel_launches, ep_moe_forward, idx_dtype, make_config)
 
 __all__ = [
     "DEV_BAD_INDEX", "DEV_CAPACITY_OVERFLOW", "STATIC_SCRATCH_BYTES", "F_BWD_UNWEIGHTED",
@@ -20,5 +20,5 @@ __all__ = [
     "EpConfig", "EpError", "EpSizes", "ep_buffer_sizes", "ep_combine", "ep_combine_backward",
     "ep_combine_backward_weights",
     "ep_copy", "ep_cvt_sweep", "ep_dispatch", "ep_dispatch_layout", "ep_dispatch_layout_static",
-    "ep_dispatch_with_layout", "ep_expert_gemm", "ep_expert_gemm_mx", "ep_get_status", "ep_kernel_launches", "idx_dtype", "make_config",
+    "ep_dispatch_with_layout", "ep_expert_gemm", "ep_expert_gemm_mx", "ep_get_status", "ep_kernel_launches", "ep_moe_forward", "idx_dtype", "make_config",
 ]

@@ -928,24 +928,40 @@ int mx_tile_n(int n_out) {
         if (n_out % bn == 0) return bn;
     return 0;
 }
-}  // namespace
 
-ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
-                           const int64_t *expert_offset, const int64_t *recv_count,
-                           const uint16_t *weights, int32_t n_out, uint16_t *y,
-                           uint32_t *dev_status, ep_stream_t stream) {
-    Plan p;
-    ep_status_t st = make_plan(cfg, p);
-    if (st != EP_OK) return st;
-    if (cfg->quant != EP_Q_BF16 || cfg->layout != EP_LAYOUT_PACKED) return EP_ERR_UNSUPPORTED;
-    if (p.H % ep::kGemmBK != 0) return EP_ERR_UNSUPPORTED;
-    if (n_out < ep::kGemmBN || n_out % ep::kGemmBN != 0) return EP_ERR_INVALID_ARG;
+// The experts' maps: argument checks (EP_OK: a launch may follow, or there is
+// nothing to do when p.N == 0), then the launches.  `w_scales` null selects
+// the bf16 maps, else the MX ones (cfg->quant MXFP8 / MXFP4).
+ep_status_t check_gemm_args(const ep_config_t *cfg, const Plan &p, bool mx, int n_out,
+                            const void *recv_buf, const int64_t *expert_offset,
+                            const int64_t *recv_count, const void *w_codes,
+                            const void *w_scales, const void *y, const uint32_t *dev_status) {
+    const bool fp4 = cfg->quant == EP_Q_MXFP4;
+    if (cfg->layout != EP_LAYOUT_PACKED) return EP_ERR_UNSUPPORTED;
+    if (mx) {
+        if (cfg->quant != EP_Q_MXFP8 && !fp4) return EP_ERR_UNSUPPORTED;
+        if (p.H % (fp4 ? 2 * ep::kMxBK : ep::kMxBK) != 0) return EP_ERR_UNSUPPORTED;
+        if (n_out <= 0 || mx_tile_n(n_out) == 0) return EP_ERR_INVALID_ARG;
+    } else {
+        if (cfg->quant != EP_Q_BF16) return EP_ERR_UNSUPPORTED;
+        if (p.H % ep::kGemmBK != 0) return EP_ERR_UNSUPPORTED;
+        if (n_out < ep::kGemmBN || n_out % ep::kGemmBN != 0) return EP_ERR_INVALID_ARG;
+    }
     if ((int64_t)n_out * p.E > kIntLimit || p.E > ep::kGemmMaxExperts) return EP_ERR_INVALID_ARG;
-    if (!recv_buf || !expert_offset || !recv_count || !weights || !y || !dev_status)
+    if (!dev_status) return EP_ERR_INVALID_ARG;
+    if (p.N == 0) return EP_OK;  // nothing to multiply (empty buffers may be null)
+    if (!recv_buf || !expert_offset || !recv_count || !w_codes || !y || (mx && !w_scales))
         return EP_ERR_INVALID_ARG;
-    if (!aligned16(recv_buf) || !aligned16(weights) || !aligned16(y)) return EP_ERR_MISALIGNED;
-    if (p.N == 0) return EP_OK;
+    if (!aligned16(recv_buf) || !aligned16(w_codes) || !aligned16(y) ||
+        (mx && !aligned16(w_scales)))
+        return EP_ERR_MISALIGNED;
+    return EP_OK;
+}
 
+ep_status_t run_gemm_bf16(const ep_config_t *cfg, const Plan &p, const void *recv_buf,
+                          const int64_t *expert_offset, const int64_t *recv_count,
+                          const uint16_t *weights, int n_out, uint16_t *y, uint32_t *dev_status,
+                          cudaStream_t s) {
     ep::GemmArgs a;
     a.E = p.E; a.H = p.H; a.N = n_out; a.ntn = n_out / ep::kGemmBN;
     a.eo = expert_offset; a.cnt = recv_count; a.y = y; a.status = dev_status;
@@ -961,7 +977,7 @@ ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
         lc.gridDim = dim3(2 * pairs);
         lc.blockDim = dim3(ep::kGemmThreads);
         lc.dynamicSmemBytes = smem2;
-        lc.stream = cs(stream);
+        lc.stream = s;
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 2;
@@ -980,32 +996,16 @@ ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
         return EP_ERR_CUDA;
     const size_t smem = ep::gemm_smem_bytes();
     if (!allow_smem(ep::expert_gemm_kernel, 5, smem)) return EP_ERR_CUDA;
-    launch(ep::expert_gemm_kernel, (unsigned)sm_count(), ep::kGemmThreads, smem, cs(stream), ma,
-           mb, a);
+    launch(ep::expert_gemm_kernel, (unsigned)sm_count(), ep::kGemmThreads, smem, s, ma, mb, a);
     return launched();
 }
 
-ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
-                              const int64_t *expert_offset, const int64_t *recv_count,
-                              const uint8_t *w_codes, const uint8_t *w_scales, int32_t n_out,
-                              uint16_t *y, uint32_t *dev_status, ep_stream_t stream) {
-    Plan p;
-    ep_status_t st = make_plan(cfg, p);
-    if (st != EP_OK) return st;
+ep_status_t run_gemm_mx(const ep_config_t *cfg, const Plan &p, const void *recv_buf,
+                        const int64_t *expert_offset, const int64_t *recv_count,
+                        const uint8_t *w_codes, const uint8_t *w_scales, int n_out, uint16_t *y,
+                        uint32_t *dev_status, cudaStream_t s) {
     const bool fp4 = cfg->quant == EP_Q_MXFP4;
-    if ((cfg->quant != EP_Q_MXFP8 && !fp4) || cfg->layout != EP_LAYOUT_PACKED)
-        return EP_ERR_UNSUPPORTED;
-    if (p.H % (fp4 ? 2 * ep::kMxBK : ep::kMxBK) != 0) return EP_ERR_UNSUPPORTED;
-    if (n_out <= 0) return EP_ERR_INVALID_ARG;
     const int bn = mx_tile_n(n_out);
-    if (bn == 0) return EP_ERR_INVALID_ARG;
-    if ((int64_t)n_out * p.E > kIntLimit || p.E > ep::kGemmMaxExperts) return EP_ERR_INVALID_ARG;
-    if (!recv_buf || !expert_offset || !recv_count || !w_codes || !w_scales || !y || !dev_status)
-        return EP_ERR_INVALID_ARG;
-    if (!aligned16(recv_buf) || !aligned16(w_codes) || !aligned16(w_scales) || !aligned16(y))
-        return EP_ERR_MISALIGNED;
-    if (p.N == 0) return EP_OK;
-    cudaStream_t s = cs(stream);
 #define EP_MX(BN_, FP4_, SLOT_)                                                              \
     return launch_gemm_mx<BN_, FP4_>(p, recv_buf, expert_offset, recv_count, w_codes, w_scales, \
                                      n_out, y, dev_status, s, SLOT_)
@@ -1018,6 +1018,75 @@ ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
     if (bn == 256) EP_MX(256, false, 7);
     EP_MX(128, false, 8);
 #undef EP_MX
+}
+}  // namespace
+
+ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
+                           const int64_t *expert_offset, const int64_t *recv_count,
+                           const uint16_t *weights, int32_t n_out, uint16_t *y,
+                           uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if ((st = check_gemm_args(cfg, p, false, n_out, recv_buf, expert_offset, recv_count, weights,
+                              nullptr, y, dev_status)) != EP_OK || p.N == 0)
+        return st;
+    return run_gemm_bf16(cfg, p, recv_buf, expert_offset, recv_count, weights, n_out, y,
+                         dev_status, cs(stream));
+}
+
+ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
+                              const int64_t *expert_offset, const int64_t *recv_count,
+                              const uint8_t *w_codes, const uint8_t *w_scales, int32_t n_out,
+                              uint16_t *y, uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if ((st = check_gemm_args(cfg, p, true, n_out, recv_buf, expert_offset, recv_count, w_codes,
+                              w_scales, y, dev_status)) != EP_OK || p.N == 0)
+        return st;
+    return run_gemm_mx(cfg, p, recv_buf, expert_offset, recv_count, w_codes, w_scales, n_out, y,
+                       dev_status, cs(stream));
+}
+
+ep_status_t ep_moe_forward(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
+                           const float *topk_weights, const void *w_codes,
+                           const uint8_t *w_scales, int32_t *token_slot, int64_t *recv_count,
+                           int64_t *expert_offset, void *workspace, void *recv_buf,
+                           int32_t *src_info, uint16_t *y, uint16_t *out, uint32_t *dev_status,
+                           ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (cfg->flags & EP_F_COMBINE_QUANTIZED) return EP_ERR_UNSUPPORTED;  // y is bf16 here
+    const bool mx = cfg->quant != EP_Q_BF16;
+    // every argument is checked before the first launch
+    if ((st = check_layout_args(cfg, p, topk_idx, token_slot, recv_count, expert_offset, workspace,
+                                dev_status)) != EP_OK)
+        return st;
+    if ((st = check_gemm_args(cfg, p, mx, p.H, recv_buf, expert_offset, recv_count, w_codes,
+                              w_scales, y, dev_status)) != EP_OK)
+        return st;
+    if (p.N > 0) {
+        if ((st = check_dispatch_args(cfg, x, topk_idx, topk_weights, token_slot, expert_offset,
+                                      recv_buf, src_info, nullptr)) != EP_OK)
+            return st;
+        if (!topk_weights || !out) return EP_ERR_INVALID_ARG;
+        if (!aligned16(out)) return EP_ERR_MISALIGNED;
+    }
+    if ((st = ep_dispatch_with_layout(cfg, x, topk_idx, topk_weights, nullptr, nullptr, nullptr,
+                                      token_slot, recv_count, expert_offset, nullptr, workspace,
+                                      recv_buf, src_info, nullptr, dev_status, stream)) != EP_OK ||
+        p.N == 0)
+        return st;
+    const cudaStream_t s = cs(stream);
+    st = mx ? run_gemm_mx(cfg, p, recv_buf, expert_offset, recv_count,
+                          static_cast<const uint8_t *>(w_codes), w_scales, p.H, y, dev_status, s)
+            : run_gemm_bf16(cfg, p, recv_buf, expert_offset, recv_count,
+                            static_cast<const uint16_t *>(w_codes), p.H, y, dev_status, s);
+    if (st != EP_OK) return st;
+    return ep_combine(cfg, y, topk_idx, topk_weights, token_slot, expert_offset, out, dev_status,
+                      stream);
 }
 
 ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream) {

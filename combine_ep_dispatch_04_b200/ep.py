@@ -82,6 +82,8 @@ lib.ep_combine_backward.restype = C.c_int
 lib.ep_combine_backward.argtypes = [_CFG] + [_P] * 8
 lib.ep_expert_gemm.restype = C.c_int
 lib.ep_expert_gemm.argtypes = [_CFG, _P, _P, _P, _P, C.c_int32, _P, _P, _P]
+lib.ep_moe_forward.restype = C.c_int
+lib.ep_moe_forward.argtypes = [_CFG] + [_P] * 14 + [_P]
 lib.ep_expert_gemm_mx.restype = C.c_int
 lib.ep_expert_gemm_mx.argtypes = [_CFG, _P, _P, _P, _P, _P, C.c_int32, _P, _P, _P]
 lib.ep_combine_backward_weights.restype = C.c_int
@@ -364,6 +366,42 @@ def ep_expert_gemm_mx(cfg, recv_buf, expert_offset, recv_count, w_codes, w_scale
         _stream(stream),
     ]
     return _call(lib.ep_expert_gemm_mx, cfg, args, "ep_expert_gemm_mx", bind)
+
+
+def ep_moe_forward(cfg, x, topk_idx, topk_weights, w_codes, w_scales, token_slot, recv_count,
+                   expert_offset, workspace, recv_buf, src_info, y, out, dev_status, stream=None,
+                   bind=False):
+    """Layout + dispatch -> the experts' maps (n_out = H) -> combine in one call:
+    w_codes bf16 [E, H, H] with w_scales None, or MX codes uint8 [E, H, D] with
+    e8m0 w_scales uint8 [E, H, H/32]; y bf16 [rows, H] scratch; out bf16 [N, H]."""
+    N, K = _nk(cfg)
+    sz = ep_buffer_sizes(cfg)
+    E, H = cfg.num_experts, cfg.hidden
+    if cfg.quant == QUANT["bf16"]:
+        if w_scales is not None:
+            raise ValueError("bf16 weights take no scales")
+        wc = _dev(w_codes, "w_codes", torch.bfloat16, (E, H, H))
+        ws = None
+    else:
+        wc = _dev(w_codes, "w_codes", torch.uint8, (E, H, sz["data_row_bytes"]))
+        ws = _dev(w_scales, "w_scales", torch.uint8, (E, H, H // 32))
+    args = [
+        _dev(x, "x", torch.bfloat16, (N, H)),
+        _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
+        _dev(topk_weights, "topk_weights", torch.float32, (N, K)),
+        wc, ws,
+        _dev(token_slot, "token_slot", torch.int32, (N, K)),
+        _dev(recv_count, "recv_count", torch.int64, (E,)),
+        _dev(expert_offset, "expert_offset", torch.int64, (E + 1,)),
+        _bytes(workspace, "workspace", sz["workspace_bytes"]),
+        _bytes(recv_buf, "recv_buf", sz["recv_bytes"]),
+        _bytes(src_info, "src_info", sz["src_info_bytes"]),
+        _dev(y, "y", torch.bfloat16, (sz["rows"], H)),
+        _dev(out, "out", torch.bfloat16, (N, H)),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    return _call(lib.ep_moe_forward, cfg, args, "ep_moe_forward", bind)
 
 
 def ep_combine_backward_weights(cfg, g, y, topk_idx, token_slot, topk_weights_grad, dev_status,

@@ -331,6 +331,35 @@ ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
                               uint16_t *y, uint32_t *dev_status, ep_stream_t stream);
 
 /*
+ * One call for the whole forward path with the experts between dispatch and
+ * combine ("[feat] A5 deep fused moe supported": one operator runs the
+ * dispatch, the experts' grouped matrix multiplications and the combine):
+ * ep_dispatch_with_layout, then the experts' maps (ep_expert_gemm for
+ * cfg->quant EP_Q_BF16, ep_expert_gemm_mx for EP_Q_MXFP8 / EP_Q_MXFP4) with
+ * n_out = H, then ep_combine of their bf16 outputs.  The launches follow one
+ * another on `stream` with programmatic dependent launch: each kernel's
+ * set-up overlaps the previous kernel's tail.  Every argument is checked
+ * before the first launch; the result equals the four calls made one by one.
+ *   cfg          layout EP_LAYOUT_PACKED; quant EP_Q_BF16 (H % 256 == 0),
+ *                EP_Q_MXFP8 (H % 128 == 0) or EP_Q_MXFP4 (H % 256 == 0);
+ *                EP_F_COMBINE_QUANTIZED is not supported (EP_ERR_UNSUPPORTED)
+ *   x, topk_idx, topk_weights    as ep_dispatch / ep_combine
+ *   w_codes      bf16 [E][H][H] (w_scales NULL) or the MX codes [E][H][D]
+ *   w_scales     e8m0 [E][H][H/32] for the MX formats
+ *   token_slot, recv_count, expert_offset, workspace   as ep_dispatch_layout
+ *   recv_buf, src_info           as ep_dispatch
+ *   y            bf16 [rows][H]: the experts' outputs (scratch owned by the caller)
+ *   out          bf16 [N][H]
+ * A wait inside the GEMM kernel that exceeds 2 s sets EP_DEV_TIMEOUT.
+ */
+ep_status_t ep_moe_forward(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
+                           const float *topk_weights, const void *w_codes,
+                           const uint8_t *w_scales, int32_t *token_slot, int64_t *recv_count,
+                           int64_t *expert_offset, void *workspace, void *recv_buf,
+                           int32_t *src_info, uint16_t *y, uint16_t *out, uint32_t *dev_status,
+                           ep_stream_t stream);
+
+/*
  * Allocation-free variant of ep_dispatch_layout.  The pages have no
  * counterpart to this call; it exists for callers that cannot allocate
  * device memory when they route tokens -- for example a serving loop whose

@@ -799,6 +799,59 @@ def test_expert_gemm_mxfp4_large_shape_sampled():
     _check_expert_gemm(r, y, w["H"], wc=wc, ws=ws, sample_rows=12)
 
 
+def test_expert_gemm_empty_batch_launches_nothing():
+    w = synth.workload("tiny", R=2, T=0, M=16, K=2, E=4, H=256)
+    for mode in ("bf16", "mxfp8"):
+        r = Run(w, mode, layout="packed")
+        y = _sentinel_y(r, 256)
+        n0 = ep.ep_kernel_launches()
+        if mode == "bf16":
+            W = _seeded_weights(w["E"], 256, w["H"], 0.05, seed=1)
+            ep.ep_expert_gemm(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, W, y,
+                              r.b.dev_status)
+        else:
+            wc, ws = _seeded_mx_weights(w["E"], 256, w["H"], seed=1)
+            ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws,
+                                 y, r.b.dev_status)
+        assert ep.ep_kernel_launches() == n0
+        assert torch.all(y.view(torch.int16) == 0x7777)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "mxfp8", "mxfp4"])
+def test_expert_gemm_one_expert_takes_every_token(mode):
+    """Every token to expert 2: one expert with many row tiles (a partial last
+    one), every other expert empty."""
+    w = synth.workload("tiny", R=2, T=300, M=300, K=1, E=8, H=512)
+    idx = np.full((w["R"] * w["T"], 1), 2, np.int64)
+    wts = np.ones((w["R"] * w["T"], 1), np.float32)
+    r = Run(w, mode, layout="packed", idx=idx, wts=wts)
+    y = _sentinel_y(r, 256)
+    if mode == "bf16":
+        W = _seeded_weights(w["E"], 256, w["H"], 0.05, seed=3)
+        ep.ep_expert_gemm(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, W, y,
+                          r.b.dev_status)
+        kw = dict(W=W)
+    else:
+        wc, ws = _seeded_mx_weights(w["E"], 256, w["H"], seed=3, fp4=mode == "mxfp4")
+        ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws, y,
+                             r.b.dev_status)
+        kw = dict(wc=wc, ws=ws)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    assert r.lay["recv_count"][2] == 600
+    _check_expert_gemm(r, y, 256, sample_rows=160, **kw)
+
+
+def test_expert_gemm_most_experts():
+    """E = 1024 (the limit): the per-expert tile prefix over 32 experts a lane."""
+    w = synth.workload("tiny", R=4, T=64, M=64, K=4, E=1024, H=256)
+    r = Run(w, "bf16", layout="packed")
+    W = _seeded_weights(w["E"], 256, w["H"], 0.05, seed=4)
+    y = _sentinel_y(r, 256)
+    ep.ep_expert_gemm(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, W, y, r.b.dev_status)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    _check_expert_gemm(r, y, 256, W=W, sample_rows=200)
+
+
 def test_expert_gemm_mx_rejects_other_formats():
     w = synth.workload("tiny", R=2, T=16, M=16, K=2, E=4, H=256)
     r = Run(w, "bf16", layout="packed")
@@ -817,27 +870,56 @@ def test_expert_gemm_mx_rejects_other_formats():
     assert torch.all(y.view(torch.int16) == 0x7777)
 
 
-def _pipeline_check(r, maps_fn, n_out, max_ulp):
+def _bf16_ulp(bits):
+    v = np.abs((bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64))
+    return np.ldexp(1.0, np.floor(np.log2(np.maximum(v, 2.0 ** -126))).astype(np.int64) - 7)
+
+
+def _chain_check(got, want, yw, mag, chain, idx, wts, rows_of):
+    """The GPU's chain against the oracle's, element by element, within a bound
+    derived from the arithmetic: each expert output the GPU combines may differ
+    from the oracle's by its own allowance (one bf16 ulp plus
+    chain * 2^-23 * sum_h |x*w|, the GEMM bound), which the combine scales by
+    |w_k|; the combine's own rounding adds up to two bf16 ulps of the result
+    (its fp32 sum of perturbed terms, then bf16)."""
+    N, K = idx.shape
+    bound = 2.0 * _bf16_ulp(want)
+    for n in range(N):
+        for k in range(K):
+            row = rows_of.get((n, k))
+            if row is None:
+                continue
+            allow = _bf16_ulp(yw[row]) + mag[row] * (chain * 2.0 ** -23)
+            bound[n] += abs(float(wts[n, k])) * allow
+    gf = (got.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    wf = (want.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    assert np.all(np.abs(gf - wf) <= bound)
+
+
+def _pipeline_check(r, maps_fn, n_out, chain):
     """The GPU's combine of its expert outputs against the oracle's combine of
-    the oracle's expert outputs (oracle layout and quantisation of the seeded x)."""
+    the oracle's expert outputs (oracle layout and quantisation of the seeded x),
+    within _chain_check's bound.  maps_fn(e, rows) -> (bf16 outputs, sum_h |x*w|)."""
     w = r.w
     o = r.lay
     E, H = w["E"], w["H"]
     eo, cnt = o["expert_offset"], o["recv_count"]
     rows = r.sizes["rows"]
-    ns, _, rr = r.entries()
+    ns, ks, rr = r.entries()
     tok = {int(a): int(b) for a, b in zip(rr, ns)}
     yw = np.zeros((rows, n_out), np.uint16)
+    mag = np.zeros((rows, n_out), np.float64)
     for e in range(E):
         rs = np.sort(rr[(rr >= eo[e]) & (rr < eo[e] + cnt[e])])
         if len(rs) == 0:
             continue
         q = [oracle.quant_row(r.omode, r.x[tok[int(x)]], e4m3_qmax=r.qmax) for x in rs]
-        yw[rs] = maps_fn(e, q)
+        yw[rs], mag[rs] = maps_fn(e, q)
     want, st = oracle.combine(w["R"], w["T"], w["K"], E, w["M"], H, yw, r.idx, r.wts,
                               o["token_slot"], o["expert_offset"], layout="packed")
-    got = to_np_u16(r.b.out)
-    assert st == 0 and ulp_distance(got, want).max() <= max_ulp
+    assert st == 0
+    _chain_check(to_np_u16(r.b.out), want, yw, mag, chain, r.idx, r.wts,
+                 {(int(n), int(k)): int(x) for n, k, x in zip(ns, ks, rr)})
 
 
 def test_dispatch_experts_combine_pipeline():
@@ -857,9 +939,11 @@ def test_dispatch_experts_combine_pipeline():
 
     def maps(e, q):
         xb = np.stack([d.view(np.uint16) for d, _ in q])
-        return oracle.expert_gemm(xb, Wh[e][None], np.zeros(1, np.int64),
-                                  np.array([len(q)], np.int64), n_out)
-    _pipeline_check(r, maps, n_out, 2)
+        y = oracle.expert_gemm(xb, Wh[e][None], np.zeros(1, np.int64),
+                               np.array([len(q)], np.int64), n_out)
+        f = lambda u: (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        return y, np.abs(f(xb)) @ np.abs(f(Wh[e])).T
+    _pipeline_check(r, maps, n_out, w["H"] // 16 + 16)
 
 
 def test_dispatch_mxfp4_experts_combine_pipeline():
@@ -878,9 +962,11 @@ def test_dispatch_mxfp4_experts_combine_pipeline():
 
     def maps(e, q):
         xc, xs = np.stack([d for d, _ in q]), np.stack([sc for _, sc in q])
-        return oracle.expert_gemm_mxfp4(xc, xs, wch[e][None], wsh[e][None], np.zeros(1, np.int64),
-                                        np.array([len(q)], np.int64), n_out)
-    _pipeline_check(r, maps, n_out, 2)
+        y = oracle.expert_gemm_mxfp4(xc, xs, wch[e][None], wsh[e][None], np.zeros(1, np.int64),
+                                     np.array([len(q)], np.int64), n_out)
+        sv = lambda c, sc: _e2m1_values(c) * np.ldexp(1.0, np.repeat(sc.astype(np.int64) - 127, 32, axis=-1))
+        return y, np.abs(sv(xc, xs)) @ np.abs(sv(wch[e], wsh[e])).T
+    _pipeline_check(r, maps, n_out, w["H"] // 32 + 32)
 
 
 def test_dispatch_mx_experts_combine_pipeline():
@@ -899,6 +985,112 @@ def test_dispatch_mx_experts_combine_pipeline():
 
     def maps(e, q):
         xc, xs = np.stack([d for d, _ in q]), np.stack([sc for _, sc in q])
-        return oracle.expert_gemm_mx(xc, xs, wch[e][None], wsh[e][None], np.zeros(1, np.int64),
-                                     np.array([len(q)], np.int64), n_out)
-    _pipeline_check(r, maps, n_out, 2)
+        y = oracle.expert_gemm_mx(xc, xs, wch[e][None], wsh[e][None], np.zeros(1, np.int64),
+                                  np.array([len(q)], np.int64), n_out)
+        lut = _e4m3_table()
+        sv = lambda c, sc: lut[c] * np.ldexp(1.0, np.repeat(sc.astype(np.int64) - 127, 32, axis=-1))
+        return y, np.abs(sv(xc, xs)) @ np.abs(sv(wch[e], wsh[e])).T
+    _pipeline_check(r, maps, n_out, w["H"] // 32 + 32)
+
+
+# ---------------------------------------------------------------------------
+# the whole forward path in one call
+# ---------------------------------------------------------------------------
+def _moe_case(mode, seed):
+    w = synth.workload("tiny", R=2, T=48, M=48, K=4, E=8, H=512)
+    idx, wts = synth.make_routing(w)
+    x = synth.make_x(w)
+    cfg = ep.make_config(w["R"], w["T"], w["M"], w["K"], w["E"], w["H"], mode, "packed")
+    if mode == "bf16":
+        wc, ws = _seeded_weights(w["E"], w["H"], w["H"], 0.05, seed), None
+    else:
+        wc, ws = _seeded_mx_weights(w["E"], w["H"], w["H"], seed, lo=112, hi=124,
+                                    fp4=mode == "mxfp4")
+    return w, cfg, bf16_dev(x), torch.from_numpy(idx).cuda(), torch.from_numpy(wts).cuda(), wc, ws, idx, wts, x
+
+
+@pytest.mark.parametrize("mode", ["bf16", "mxfp8", "mxfp4"])
+def test_moe_forward_equals_the_calls_one_by_one(mode):
+    w, cfg, x_d, idx_d, wts_d, wc, ws, idx, wts, x = _moe_case(mode, 31)
+    H = w["H"]
+    outs = []
+    for one_call in (True, False):
+        b = ep.Buffers(cfg)
+        b.recv_buf.fill_(0xAB)
+        y = torch.empty((b.sizes["rows"], H), dtype=torch.bfloat16, device="cuda")
+        out = torch.full((w["N"], H), 7.0, dtype=torch.bfloat16, device="cuda")
+        if one_call:
+            n0 = ep.ep_kernel_launches()
+            ep.ep_moe_forward(cfg, x_d, idx_d, wts_d, wc, ws, b.token_slot, b.recv_count,
+                              b.expert_offset, b.workspace, b.recv_buf, b.src_info, y, out,
+                              b.dev_status)
+            assert ep.ep_kernel_launches() - n0 == 4   # layout, dispatch, experts, combine
+        else:
+            ep.ep_dispatch_layout(cfg, idx_d, b.token_slot, b.recv_count, b.workspace,
+                                  b.dev_status, expert_offset=b.expert_offset)
+            ep.ep_dispatch(cfg, x_d, idx_d, b.token_slot, b.recv_buf, b.src_info, b.dev_status,
+                           expert_offset=b.expert_offset)
+            if mode == "bf16":
+                ep.ep_expert_gemm(cfg, b.recv_buf, b.expert_offset, b.recv_count, wc, y,
+                                  b.dev_status)
+            else:
+                ep.ep_expert_gemm_mx(cfg, b.recv_buf, b.expert_offset, b.recv_count, wc, ws, y,
+                                     b.dev_status)
+            ep.ep_combine(cfg, y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
+                          expert_offset=b.expert_offset)
+            out = b.out
+        assert ep.ep_get_status(b.dev_status) == 0
+        outs.append(to_np_u16(out))
+    assert np.array_equal(outs[0], outs[1])
+
+
+def test_moe_forward_against_the_oracle_chain():
+    """bf16: the one call against the oracle's layout, dispatch, maps and combine."""
+    w, cfg, x_d, idx_d, wts_d, W, _, idx, wts, x = _moe_case("bf16", 32)
+    H, E = w["H"], w["E"]
+    b = ep.Buffers(cfg)
+    y = torch.empty((b.sizes["rows"], H), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((w["N"], H), dtype=torch.bfloat16, device="cuda")
+    ep.ep_moe_forward(cfg, x_d, idx_d, wts_d, W, None, b.token_slot, b.recv_count, b.expert_offset,
+                      b.workspace, b.recv_buf, b.src_info, y, out, b.dev_status)
+    assert ep.ep_get_status(b.dev_status) == 0
+    lay = oracle.layout(w["R"], w["T"], w["K"], E, w["M"], idx, layout="packed")
+    eo, cnt = lay["expert_offset"], lay["recv_count"]
+    rows = b.sizes["rows"]
+    xr = np.zeros((rows, H), np.uint16)
+    for n in range(w["N"]):
+        for k in range(w["K"]):
+            e = idx[n, k]
+            if 0 <= e < E:
+                xr[eo[e] + lay["token_slot"][n, k]] = x[n]       # bf16 dispatch is a scatter
+    Wh = W.view(torch.int16).cpu().numpy().view(np.uint16)
+    yw = oracle.expert_gemm(xr, Wh, eo[:E], cnt, H)
+    want, st = oracle.combine(w["R"], w["T"], w["K"], E, w["M"], H, yw, idx, wts,
+                              lay["token_slot"], eo, layout="packed")
+    assert st == 0
+    f = lambda u: (u.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    mag = np.zeros((rows, H))
+    rows_of = {}
+    for e in range(E):
+        rs = np.arange(eo[e], eo[e] + cnt[e])
+        if len(rs):
+            mag[rs] = np.abs(f(xr[rs])) @ np.abs(f(Wh[e])).T
+    for n in range(w["N"]):
+        for k in range(w["K"]):
+            if 0 <= idx[n, k] < E:
+                rows_of[(n, k)] = int(eo[idx[n, k]] + lay["token_slot"][n, k])
+    _chain_check(to_np_u16(out), want, yw, mag, H // 16 + 16, idx, wts, rows_of)
+
+
+def test_moe_forward_checks_before_launching():
+    w, cfg, x_d, idx_d, wts_d, wc, ws, *_ = _moe_case("bf16", 33)
+    b = ep.Buffers(cfg)
+    y = torch.empty((b.sizes["rows"], w["H"]), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((w["N"], w["H"]), dtype=torch.bfloat16, device="cuda")
+    bad = ep.make_config(w["R"], w["T"], w["M"], w["K"], w["E"], w["H"], "bf16", "packed",
+                         flags=ep.F_COMBINE_QUANTIZED)
+    n0 = ep.ep_kernel_launches()
+    with pytest.raises(ep.EpError):
+        ep.ep_moe_forward(bad, x_d, idx_d, wts_d, wc, None, b.token_slot, b.recv_count,
+                          b.expert_offset, b.workspace, b.recv_buf, b.src_info, y, out, b.dev_status)
+    assert ep.ep_kernel_launches() == n0
