@@ -917,14 +917,10 @@ int gemm_pairs() {
     return n;
 }
 
-// N tile of the MXFP8 kernel: two accumulators of 224 columns where n_out
-// allows, else one of 256, else two of 128
-#ifndef EP_MX_PREFER_BN
-#define EP_MX_PREFER_BN 224
-#endif
+// N tile of the MX kernels: two accumulators of 224 columns where n_out
+// allows, else one of 256, else two of 128 (0: none divides n_out)
 int mx_tile_n(int n_out) {
-    const int pref[3] = {EP_MX_PREFER_BN, EP_MX_PREFER_BN == 224 ? 256 : 224, 128};
-    for (int bn : pref)
+    for (int bn : {224, 256, 128})
         if (n_out % bn == 0) return bn;
     return 0;
 }
