@@ -1,13 +1,17 @@
-// ep_gemm.cuh -- the experts between dispatch and combine: a grouped bf16
-// matrix multiplication on the fifth-generation tensor cores.
+// ep_gemm.cuh -- the experts between dispatch and combine: grouped matrix
+// multiplications on the fifth-generation tensor cores.
 //
 // "[feat] A5 deep fused moe supported" runs grouped matrix multiplications of
 // the experts between its dispatch and its combine.  Here each expert e is one
 // linear map W_e [N][H]: for the rows r of expert e in the packed receive
 // layout (expert_offset[e] .. + count[e]),
 //   y[r, :] = bf16_rne( x[r, :] . W_e^T ),  fp32 accumulation.
+// Three kernels: expert_gemm_kernel (bf16, below), expert_gemm2_kernel (bf16
+// on CTA pairs with the two-CTA MMA) and expert_gemm_mx_kernel (MXFP8 / MXFP4
+// codes with e8m0 block scales, the block-scaled MMA), each described where
+// it is defined.
 //
-// Tiles of 128 rows x 256 columns, 64-element K steps.  A persistent grid
+// bf16: tiles of 128 rows x 256 columns, 64-element K steps.  A persistent grid
 // (one block per SM) walks the tiles of all experts; in each block
 //   warp 0        loads A and B K-steps with TMA (128-byte swizzle) into a
 //                 ring of kGemmStages shared-memory stages;
