@@ -75,8 +75,11 @@ def parse():
     p.add_argument("--weights-grad", action="store_true",
                    help="also time the combine's weight gradient (outside the step)")
     p.add_argument("--gemm", action="store_true",
-                   help="also time the experts' grouped GEMM (bf16, packed, N = H) on the "
-                        "dispatched rows, outside the step")
+                   help="time the experts' grouped GEMMs (bf16, MXFP8, MXFP4; packed, N = H) and "
+                        "the one-call forward path outside the step, also when N > 1 (one GPU: "
+                        "the default)")
+    p.add_argument("--no-gemm", action="store_true",
+                   help="skip the experts' GEMM legs on one GPU")
     p.add_argument("--gemm-experts", type=int, default=0,
                    help="with --gemm: route the tokens onto this many experts (expert id "
                         "modulo E) for the GEMM legs only, a small case for profilers")
@@ -557,10 +560,21 @@ def main():
     except Exception:
         pass
 
-    gemm = run_gemm(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args) if args.gemm else None
-    gemm_mx = run_gemm_mx(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args) if args.gemm else None
-    gemm_mx4 = (run_gemm_mx(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args, "mxfp4")
-                if args.gemm and w["H"] % 256 == 0 else None)
+    # the experts between dispatch and combine, outside the step: by default on
+    # one GPU; a leg that fails reports its error instead of ending the bench
+    gemm_on = args.gemm or (world == 1 and not args.no_gemm)
+
+    def leg(fn, *a):
+        if not gemm_on:
+            return None
+        try:
+            return fn(*a)
+        except Exception as ex:  # noqa: BLE001 -- reported in the line
+            return {"error": f"{type(ex).__name__}: {ex}"[:300]}
+    gemm = leg(run_gemm, ep, w, x_d, idx_d, wts_d, flush, stream, dev, args)
+    gemm_mx = leg(run_gemm_mx, ep, w, x_d, idx_d, wts_d, flush, stream, dev, args)
+    gemm_mx4 = (leg(run_gemm_mx, ep, w, x_d, idx_d, wts_d, flush, stream, dev, args, "mxfp4")
+                if w["H"] % 256 == 0 else None)
 
     e2e = None if args.no_e2e else run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream,
                                           dev, args, world, step_bytes)
@@ -697,7 +711,7 @@ def time_moe_forward(ep, cfg, b, x_d, idx_d, wts_d, wc, ws, y, flush, stream, de
         call()
     torch.cuda.synchronize(dev)
     if ep.ep_get_status(b.dev_status) != 0:
-        raise SystemExit("ep_moe_forward reported a device error")
+        raise RuntimeError("ep_moe_forward reported a device error")
     reps = max(3, min(args.steps, 20))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(reps)]
@@ -735,7 +749,7 @@ def run_gemm(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args):
         call()
     torch.cuda.synchronize(dev)
     if ep.ep_get_status(b.dev_status) != 0:
-        raise SystemExit("ep_expert_gemm reported a device error")
+        raise RuntimeError("ep_expert_gemm reported a device error")
     v = int(b.recv_count.sum().item())
     reps = max(3, min(args.steps, 20))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -800,7 +814,7 @@ def run_gemm_mx(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args, fmt="mxfp8")
         call()
     torch.cuda.synchronize(dev)
     if ep.ep_get_status(b.dev_status) != 0:
-        raise SystemExit(f"ep_expert_gemm_mx ({fmt}) reported a device error")
+        raise RuntimeError(f"ep_expert_gemm_mx ({fmt}) reported a device error")
     v = int(b.recv_count.sum().item())
     reps = max(3, min(args.steps, 20))
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
