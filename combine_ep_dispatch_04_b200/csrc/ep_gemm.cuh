@@ -646,6 +646,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // ---------------------------------------------------------------------------
 constexpr int kMxBK = 128, kMxStages = 4, kMxThreads = 224;
 constexpr int kSfGroup = 4;  // K steps whose scale loads the gathering warp issues together
+static_assert(kSfGroup % 4 == 0, "16-byte scale loads cover four steps");
 
 template <int BN, bool FP4>
 struct MxCfg {
@@ -864,12 +865,12 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 uint32_t va[G][NG][4], vb[G][NG][C::kChunksB][4];
                 if (vec && g == G) {
                     // a row's scales of the G steps are G * NG contiguous words,
-                    // 16-byte aligned: NG 16-byte loads per row
+                    // 16-byte aligned: G * NG / 4 16-byte loads per row
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
                         const int64_t row = arow0 + lane + 32 * j;
 #pragma unroll
-                        for (int h = 0; h < NG; h++) {
+                        for (int h = 0; h < G * NG / 4; h++) {
                             const uint4 w4 = row < a.rows
                                                  ? __ldg(reinterpret_cast<const uint4 *>(
                                                        a.xs + row * SB + kb0 * NG * 4) + h)
@@ -885,7 +886,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                         for (int j = 0; j < 4; j++) {
                             const int n = 128 * c + 32 * j + lane;
 #pragma unroll
-                            for (int h = 0; h < NG; h++) {
+                            for (int h = 0; h < G * NG / 4; h++) {
                                 const uint4 w4 = n < BN ? __ldg(reinterpret_cast<const uint4 *>(
                                                               a.ws + (brow0 + n) * SB + kb0 * NG * 4) + h)
                                                         : make_uint4(0u, 0u, 0u, 0u);
