@@ -917,9 +917,14 @@ int gemm_pairs() {
     return n;
 }
 
-// N tile of the MX kernels: two accumulators of 224 columns where n_out
-// allows, else one of 256, else two of 128 (0: none divides n_out)
-int mx_tile_n(int n_out) {
+// N tile of the MX kernels (0: none divides n_out).  Two accumulators of 224
+// columns let a tile's epilogue overlap the next tile's MMAs, which matters
+// where the weights stream past few rows (decode-sized experts); MXFP8 with
+// at least 256 rows an expert on average takes one accumulator of 256
+// columns, the most FLOPs per byte of A (measured faster there, not for
+// MXFP4).  Otherwise 256, then 128, where 224 does not divide n_out.
+int mx_tile_n(int n_out, bool fp4 = false, int64_t rows_per_expert = 0) {
+    if (!fp4 && rows_per_expert >= 256 && n_out % 256 == 0) return 256;
     for (int bn : {224, 256, 128})
         if (n_out % bn == 0) return bn;
     return 0;
@@ -1001,7 +1006,7 @@ ep_status_t run_gemm_mx(const ep_config_t *cfg, const Plan &p, const void *recv_
                         const uint8_t *w_codes, const uint8_t *w_scales, int n_out, uint16_t *y,
                         uint32_t *dev_status, cudaStream_t s) {
     const bool fp4 = cfg->quant == EP_Q_MXFP4;
-    const int bn = mx_tile_n(n_out);
+    const int bn = mx_tile_n(n_out, fp4, p.N * p.K / p.E);
 #define EP_MX(BN_, FP4_, SLOT_)                                                              \
     return launch_gemm_mx<BN_, FP4_>(p, recv_buf, expert_offset, recv_count, w_codes, w_scales, \
                                      n_out, y, dev_status, s, SLOT_)

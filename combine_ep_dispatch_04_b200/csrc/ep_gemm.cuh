@@ -645,8 +645,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // then 128-row block).
 // ---------------------------------------------------------------------------
 constexpr int kMxBK = 128, kMxStages = 4, kMxThreads = 224;
-constexpr int kSfGroup = 4;  // K steps whose scale loads the gathering warp issues together
-static_assert(kSfGroup % 4 == 0, "16-byte scale loads cover four steps");
+// K steps whose scale loads the gathering warp issues together (MXFP4 has
+// twice the scale bytes a step: fewer steps keep its registers unspilled)
+template <bool FP4>
+__host__ __device__ constexpr int sf_group() { return FP4 ? 4 : 8; }
+static_assert(sf_group<false>() % 4 == 0 && sf_group<true>() % 4 == 0,
+              "16-byte scale loads cover four steps");
 
 template <int BN, bool FP4>
 struct MxCfg {
@@ -844,9 +848,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         }
     } else if (warp == 2) {
         // ---- scales: 4 bytes (one K step) of every row of the A and B tiles
-        // The loads of kSfGroup K steps are issued together: one step's
+        // The loads of sf_group() K steps are issued together: one step's
         // loads would leave a whole L2 latency between consecutive steps.
-        constexpr int G = kSfGroup;
+        constexpr int G = sf_group<FP4>();
         const int SB = a.H / 32;
         // 16-byte loads where every row's scales start on a 16-byte boundary
         // (the scale regions themselves are 16-byte aligned)

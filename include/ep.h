@@ -318,8 +318,8 @@ ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
  *                column j)
  *   w_scales     e8m0 [E][n_out][H/32]
  *   n_out        output columns, a multiple of 224, 256 or 128 (tiles of 224
- *                columns are taken where they divide n_out, else 256, else
- *                128)
+ *                columns where they divide n_out, else 256, else 128; MXFP8
+ *                with at least 256 entries an expert on average takes 256)
  *   y            bf16 [rows][n_out] (n_out = H gives ep_combine's input)
  * recv_buf, w_codes, w_scales and y 16-byte aligned (EP_ERR_MISALIGNED).
  * A wait inside the kernel that exceeds 2 s sets EP_DEV_TIMEOUT and the
