@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libep.so")
-SOURCES = [os.path.join(CSRC, "ep_api.cu")]
+SOURCES = [os.path.join(CSRC, "ep_api.cu"), os.path.join(CSRC, "ep_diag.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cuh")] + \
     [os.path.join(ROOT, "include", "ep.h")]
 

@@ -31,12 +31,12 @@
 #include <cuda.h>
 
 #include "ep_device.cuh"
+#include "ep_mbar.cuh"
 
 namespace ep {
 
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64, kGemmStages = 4;
 constexpr int kGemmThreads = 192;
-constexpr uint32_t kDevTimeout = 0x4u;
 constexpr int kGemmTileBytesA = kGemmBM * kGemmBK * 2;  // 16 KB
 constexpr int kGemmTileBytesB = kGemmBN * kGemmBK * 2;  // 32 KB
 constexpr int kGemmMaxExperts = 1024;
@@ -57,38 +57,6 @@ __host__ __device__ constexpr size_t gemm_smem_bytes() {
            (2 * kGemmStages + 5) * 8 + 16 + (kGemmMaxExperts + 1) * 4 + 256;
 }
 
-__device__ __forceinline__ uint64_t gtimer() {
-    uint64_t t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-                 : "memory");
-}
-// true once the phase of parity `parity` has completed; false after 2 s
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    const uint64_t t0 = gtimer();
-#pragma unroll 1
-    while (true) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(bar), "r"(parity)
-            : "memory");
-        if (ok) return true;
-        if (gtimer() - t0 > 2000000000ull) return false;
-    }
-}
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
                                             uint32_t bar) {
     asm volatile(

@@ -24,6 +24,7 @@ QUANT = {"bf16": 0, "e4m3_b128": 1, "int8_token": 2, "mxfp8": 3, "mxfp4": 4}
 LAYOUT = {"padded": 0, "packed": 1}
 DEV_BAD_INDEX = 0x1
 DEV_CAPACITY_OVERFLOW = 0x2
+DEV_TIMEOUT = 0x4
 F_BWD_UNWEIGHTED = 0x1
 F_COMBINE_QUANTIZED = 0x2
 F_IDX_I32 = 0x4
@@ -82,6 +83,8 @@ lib.ep_combine_backward.restype = C.c_int
 lib.ep_combine_backward.argtypes = [_CFG] + [_P] * 8
 lib.ep_expert_gemm.restype = C.c_int
 lib.ep_expert_gemm.argtypes = [_CFG, _P, _P, _P, _P, C.c_int32, _P, _P, _P]
+lib.ep_wait_probe.restype = C.c_int
+lib.ep_wait_probe.argtypes = [_P, _P]
 lib.ep_moe_forward.restype = C.c_int
 lib.ep_moe_forward.argtypes = [_CFG] + [_P] * 14 + [_P]
 lib.ep_expert_gemm_mx.restype = C.c_int
@@ -366,6 +369,14 @@ def ep_expert_gemm_mx(cfg, recv_buf, expert_offset, recv_count, w_codes, w_scale
         _stream(stream),
     ]
     return _call(lib.ep_expert_gemm_mx, cfg, args, "ep_expert_gemm_mx", bind)
+
+
+def ep_wait_probe(dev_status, stream=None):
+    """One block waits on a barrier nothing completes: after 2 s the wait gives
+    up and sets DEV_TIMEOUT in dev_status (read it with ep_get_status)."""
+    st = lib.ep_wait_probe(_dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream))
+    if st != 0:
+        raise EpError(st, "ep_wait_probe")
 
 
 def ep_moe_forward(cfg, x, topk_idx, topk_weights, w_codes, w_scales, token_slot, recv_count,

@@ -360,6 +360,16 @@ ep_status_t ep_moe_forward(const ep_config_t *cfg, const uint16_t *x, const void
                            ep_stream_t stream);
 
 /*
+ * Diagnostic of the bounded waits in the tensor-core kernels (ep_expert_gemm,
+ * ep_expert_gemm_mx, ep_moe_forward): one block waits, with the helper those
+ * kernels use, on a shared-memory barrier that nothing completes.  After 2 s
+ * the wait gives up, EP_DEV_TIMEOUT is set in *dev_status and the kernel
+ * returns; the context stays usable.  Takes about 2 s of one SM.
+ *   dev_status   device uint32, read and cleared by ep_get_status
+ */
+ep_status_t ep_wait_probe(uint32_t *dev_status, ep_stream_t stream);
+
+/*
  * Allocation-free variant of ep_dispatch_layout.  The pages have no
  * counterpart to this call; it exists for callers that cannot allocate
  * device memory when they route tokens -- for example a serving loop whose

@@ -1094,3 +1094,26 @@ def test_moe_forward_checks_before_launching():
         ep.ep_moe_forward(bad, x_d, idx_d, wts_d, wc, None, b.token_slot, b.recv_count,
                           b.expert_offset, b.workspace, b.recv_buf, b.src_info, y, out, b.dev_status)
     assert ep.ep_kernel_launches() == n0
+
+
+# ---------------------------------------------------------------------------
+# the bounded waits of the tensor-core kernels
+# ---------------------------------------------------------------------------
+def test_bounded_wait_gives_up_reports_and_leaves_the_context_usable():
+    """A wait on a barrier that nothing completes (the GEMMs' own wait helper)
+    gives up after about 2 s and sets DEV_TIMEOUT; the kernel returns and the
+    next calls run normally."""
+    import time
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.monotonic()
+    ep.ep_wait_probe(st)
+    flags = ep.ep_get_status(st)
+    dt = time.monotonic() - t0
+    assert flags == ep.DEV_TIMEOUT
+    assert 1.5 < dt < 60, dt
+    assert ep.ep_get_status(st) == 0                   # read and cleared
+    r = Run(synth.workload("tiny"), "bf16")             # the context is still usable
+    r.check_layout()
+    r.check_dispatch()
+    r.check_combine()
