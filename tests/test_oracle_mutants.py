@@ -17,6 +17,10 @@ from oracle.build import CFLAGS  # noqa: E402
 
 # name: ([(text in ep_oracle.c, replacement), ...], pins that must catch it)
 MUTANTS = {
+    "bf16 expert maps all use expert 0's weights": (
+        [("const uint16_t *wr = w + ((int64_t)e * Nout + j) * H;",
+          "const uint16_t *wr = w + ((int64_t)0 * Nout + j) * H;")],
+        "expert_gemm_equals or expert_gemm_identity"),
     "MXFP4 maps take a row scale per 32 packed bytes": (
         [("orc_e2m1_at(xc + r * D, h) * orc_e8m0_value(xs[r * S + h / 32])",
           "orc_e2m1_at(xc + r * D, h) * orc_e8m0_value(xs[r * S + h / 64])")],
