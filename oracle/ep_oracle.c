@@ -17,14 +17,17 @@
  *          Operation; Advanced Configuration Options; Summary.
  *   [TE]   "[Common][PyTorch] EP dispatch with unfused MXFP8 quantization"
  *          (TransformerEngine PR): Description; Changes.
- *   [A5]   "[feat] A5 deep fused moe supported" (sgl-kernel-npu PR): Testing.
+ *   [A5]   "[feat] A5 deep fused moe supported" (sgl-kernel-npu PR): Testing;
+ *          the operator's grouped matrix multiplications between dispatch
+ *          and combine (the expert maps below, bf16 / MXFP8 / MXFP4).
  * The e4m3 / e2m1 / e8m0 encodings are written from the public OCP 8-bit
  * floating point and OCP Microscaling (MX) v1.0 format definitions.
  *
  * Arithmetic rules: every float operation here is a single IEEE-754 binary32
  * operation, round-to-nearest-even (the file is built with
  * -ffp-contract=off -fno-fast-math, so no multiply-add is fused unless
- * fmaf() is called by name).
+ * fmaf() is called by name); the dot products of the weight gradient and
+ * the expert maps are summed in double (exact products) and rounded once.
  *
  * Parity: every function here is pinned by the CPU test suite against
  * brute force, closed forms, library routines or the pages' worked example.
