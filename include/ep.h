@@ -67,7 +67,9 @@ typedef enum {
     EP_Q_E4M3_B128 = 1,  /* e4m3 + one fp32 scale_inv per 128 elements ([FP8] Dispatch Stage) */
     EP_Q_INT8_TOKEN = 2, /* int8 + one fp32 scale per row ([LL] use_fp8, quant_mode 2) */
     EP_Q_MXFP8 = 3,      /* e4m3 + one e8m0 byte per 32 elements ([LL] use_ue8m0; [TE]) */
-    EP_Q_MXFP4 = 4       /* e2m1 x2 per byte + one e8m0 byte per 32 ([LL] use_mxfp4) */
+    EP_Q_MXFP4 = 4       /* e2m1 x2 per byte + one e8m0 byte per 32 ([LL] use_mxfp4);
+                          * e2m1 has no NaN: the nibble a NaN element takes is unspecified
+                          * (the block's scale and its other elements are not affected) */
 } ep_quant_t;
 
 /* Receive-buffer layouts. */

@@ -104,11 +104,15 @@ uint8_t orc_e4m3_encode(float x)
 }
 
 /* OCP MX FP4 E2M1: bias 1, 1 mantissa bit, values {0,.5,1,1.5,2,3,4,6},
- * sign in bit 3.  Round to nearest even, saturate to 6.  The format has no
- * NaN; a NaN encodes as +6 (code 0x7), whatever its sign. */
+ * sign in bit 3.  Round to nearest even, saturate to 6 (infinities
+ * included).  The format has no NaN and neither the OCP definition nor the
+ * pages say which code a NaN input takes: it is unspecified, and this
+ * encoder returns ORC_E2M1_NO_CODE (not a 4-bit code) so that a comparison
+ * that forgets to leave such elements out fails. */
+#define ORC_E2M1_NO_CODE 0xFFu
 uint8_t orc_e2m1_encode(float x)
 {
-    if (isnan(x)) return 0x7;
+    if (isnan(x)) return ORC_E2M1_NO_CODE;
     uint8_t sign = signbit(x) ? 0x8 : 0x0;
     float a = fabsf(x);
     return (uint8_t)(sign | small_float_code(a, 1, 1, 6.0f, 0x7));
@@ -292,6 +296,8 @@ void orc_quant_row_f32(int mode, int H, float e4m3_qmax, const float *x, uint8_t
                 data[32L * b + i] = orc_e4m3_encode(v);
             } else {
                 uint8_t c = orc_e2m1_encode(v);
+                if (c == ORC_E2M1_NO_CODE) c = 0; /* NaN element: unspecified nibble, 0 as a
+                                                     placeholder that comparisons leave out */
                 long byte = (32L * b + i) / 2;
                 if (i % 2 == 0) data[byte] = c;                 /* low nibble */
                 else data[byte] = (uint8_t)(data[byte] | (c << 4)); /* high nibble */
@@ -765,7 +771,8 @@ void orc_e2m1_encode_array(const float *x, uint8_t *out, long n)
     for (long i = 0; i < n; i++) out[i] = orc_e2m1_encode(x[i]);
 }
 /* Encode the fp32 values with bit patterns start .. start+n-1 (a sweep of
- * the whole binary32 space in chunks); NaN patterns give the NaN code. */
+ * the whole binary32 space in chunks); NaN patterns give the e4m3 NaN code,
+ * and ORC_E2M1_NO_CODE for e2m1 (unspecified there). */
 void orc_e4m3_encode_bits(uint32_t start, uint8_t *out, long n)
 {
     for (long i = 0; i < n; i++) out[i] = orc_e4m3_encode(bits_to_f32(start + (uint32_t)i));

@@ -745,9 +745,30 @@ def test_block_maximum_leaves_nan_out():
         assert np.all(dy[[7, 100, 200]] == want), mode
 
 
-def test_e2m1_nan_is_the_largest_positive_code():
-    got = oracle.e2m1_encode(np.float32([np.nan, -np.nan, np.inf, -np.inf]))
-    assert list(got) == [0x7, 0x7, 0x7, 0xF]
+def test_e2m1_infinities_saturate_and_nan_has_no_code():
+    """satfinite clamps every overflow, infinities included, to +-6; the format
+    has no NaN, so a NaN input has no specified code (the encoder's marker)."""
+    got = oracle.e2m1_encode(np.float32([np.inf, -np.inf, 7.0, -1e30, np.nan, -np.nan]))
+    assert list(got) == [0x7, 0xF, 0x7, 0xF, 0xFF, 0xFF]
+
+
+def test_mxfp4_nan_elements_leave_the_rest_of_the_block_alone():
+    """In an MXFP4 row the NaN elements stay out of the block maximum, so the
+    scales and every other element's nibble equal those of the row with the
+    NaNs replaced by zero (the NaN elements' own nibbles are unspecified)."""
+    x = (np.random.default_rng(3).standard_normal(256) * 4).astype(np.float32)
+    y = x.copy()
+    y[[7, 100, 200, 201]] = np.nan
+    z = x.copy()
+    z[[7, 100, 200, 201]] = 0.0
+    dy, sy = oracle.quant_row("mxfp4", y)
+    dz, sz = oracle.quant_row("mxfp4", z)
+    assert np.array_equal(sy, sz)
+    nib_y = np.stack([dy & 0xF, dy >> 4], axis=1).reshape(-1)
+    nib_z = np.stack([dz & 0xF, dz >> 4], axis=1).reshape(-1)
+    keep = np.ones(256, bool)
+    keep[[7, 100, 200, 201]] = False
+    assert np.array_equal(nib_y[keep], nib_z[keep])
 
 
 def test_int8_nan_products_are_zero():
