@@ -3,9 +3,14 @@
 
 One step = the whole hot path over one batch: routing layout, quantise +
 scatter (dispatch), weighted combine (and combine-backward for the prefill
-workload).  Default workload: decode (R=8 logical ranks x T=128 tokens,
-H=7168, top-8 of 256 experts, M=128, per-128-channel e4m3 dispatch, padded
-receive layout), on one GPU.
+workload).  Default workload (the headline): prefill, the largest of the five
+named workloads that fits one GPU (R=32 logical ranks x T=4096 tokens,
+H=7168, top-8 of 256 experts, MXFP8 dispatch into the packed receive layout,
+weighted combine and the MXFP8 combine-backward), on one GPU.  After the
+headline, every other named workload (tiny in both of its modes, decode,
+skewed, large) is run through the same per-kernel protocol and reported in
+the line's "workloads" object, with the combine of quantised expert outputs
+of every quantised mode.
 
 Timing: CUDA events on the stream the kernels run on.  The timed region
 brackets each step with one event pair (the reported value); a second pass
@@ -29,7 +34,7 @@ the reported time is the max over ranks.  With --gpus N > 1 (torchrun), each
 rank runs an independent replica of the workload (different seed): the path
 has no exchange step on one GPU, so no collective is added ("weak" scaling).
 
-  python bench.py [--steps K] [--warmup W] [--workload decode] [--impl reference]
+  python bench.py [--steps K] [--warmup W] [--workload prefill] [--impl reference]
 """
 import argparse
 import datetime
@@ -62,7 +67,7 @@ def parse():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=300)
     p.add_argument("--warmup", type=int, default=10)
-    p.add_argument("--workload", default="decode", choices=sorted(synth.WORKLOADS))
+    p.add_argument("--workload", default="prefill", choices=sorted(synth.WORKLOADS))
     p.add_argument("--tokens-per-rank", type=int, default=None,
                    help="override T (profiling a reduced case; the reported workload says so)")
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -71,6 +76,10 @@ def parse():
     p.add_argument("--quantized-combine", action="store_true",
                    help="combine reads expert outputs stored in the dispatch format")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-workloads", action="store_true",
+                   help="skip the per-kernel pass over the other named workloads")
+    p.add_argument("--gemm-workload", default="decode", choices=sorted(synth.WORKLOADS),
+                   help="the workload whose routing the GEMM legs use")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--weights-grad", action="store_true",
                    help="also time the combine's weight gradient (outside the step)")
@@ -106,6 +115,8 @@ def algorithmic_bytes(w, mode, idx, quantized_combine=False, weights_grad=False)
         "dispatch": N * (2 * H + 8 * K + 4 * K) + v * (D + S + 4),
         "combine": v * y_row + N * (8 * K + 4 * K + 4 * K + 2 * H),
     }
+    if mode != "bf16":  # the combine of expert outputs stored in the dispatch format
+        out["combine_q"] = v * (D + S) + N * (8 * K + 4 * K + 4 * K + 2 * H)
     if w.get("backward"):
         out["combine_bwd"] = N * (2 * H + 4 * K + 4 * K + 8 * K) + v * (H + H // 32)
     if weights_grad:  # g, idx, slots, dw; one expert row per valid entry
@@ -129,11 +140,14 @@ def measured_peaks():
         return None
 
 
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dispatch_combine_traffic.json")
+
+
 def ncu_traffic(kernel, workload):
     """DRAM bytes per launch from a committed ncu summary, if it was taken on
     the current kernel sources (else None)."""
     try:
-        with open(os.path.join(ROOT, "profiles", "decode_dispatch_combine_traffic.json")) as f:
+        with open(TRAFFIC_FILE) as f:
             t = json.load(f)
     except (OSError, ValueError):
         return None
@@ -252,6 +266,14 @@ def dist_done(world):
 # ---------------------------------------------------------------------------
 # the oracle as the CPU baseline / reference arm
 # ---------------------------------------------------------------------------
+SAMPLE_TOKENS = 1024  # tokens of one oracle step (a bounded sample of the workload)
+
+
+def sample_tokens_per_rank(w):
+    """Tokens per source rank in the oracle's sample: about SAMPLE_TOKENS in all."""
+    return max(1, min(w["T"], SAMPLE_TOKENS // w["R"]))
+
+
 class OracleStep:
     """The oracle (plain single-threaded C) running one step of the workload --
     layout, dispatch and combine -- on a bounded sample: the first `sub_t`
@@ -259,14 +281,16 @@ class OracleStep:
     size).  Inputs and output arrays are built before timing; only rows that
     hold entries are ever touched."""
 
-    def __init__(self, w, mode, idx, wts, x, sub_t, replica=0):
+    def __init__(self, w, mode, sub_t, replica=0):
         import oracle
         self.o, self.mode = oracle, mode
         R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
         sub_t = max(1, min(sub_t, T))
         take = (np.arange(R)[:, None] * T + np.arange(sub_t)[None, :]).reshape(-1)
+        idx, wts = synth.make_routing(w, replica)
         self.w = synth.workload(w["name"], T=sub_t)
-        self.idx, self.wts, self.x = idx[take], wts[take], x[take]
+        self.idx, self.wts = idx[take], wts[take]
+        self.x = synth.make_x(w, replica, rows=take)
         self.n = take.size
         lay = oracle.layout(R, sub_t, K, E, M, self.idx, layout=w["layout"])
         rows = oracle.rows_max(R, sub_t, K, E, M, w["layout"])
@@ -293,8 +317,8 @@ class OracleStep:
         return self.n
 
 
-def cpu_baseline(w, mode, idx, wts, x, seconds, replica=0):
-    st = OracleStep(w, mode, idx, wts, x, sub_t=w["T"], replica=replica)
+def cpu_baseline(w, mode, seconds, replica=0):
+    st = OracleStep(w, mode, sample_tokens_per_rank(w), replica=replica)
     st.step()
     t0 = time.perf_counter()
     done, reps = 0, 0
@@ -310,13 +334,11 @@ def cpu_baseline(w, mode, idx, wts, x, seconds, replica=0):
 
 def _oracle_worker(job, barrier, results):
     """One independent oracle instance (a spawned process): the seeded inputs
-    rebuilt here and one warm-up step, then, after every instance has reached
-    the barrier, steps for `seconds`."""
+    of its sample rebuilt here and one warm-up step, then, after every instance
+    has reached the barrier, steps for `seconds`."""
     wname, t_override, mode, replica, sub_t, seconds = job
     w = synth.workload(wname) if t_override is None else synth.workload(wname, T=t_override)
-    idx, wts = synth.make_routing(w, replica)
-    x = synth.make_x(w, replica)
-    st = OracleStep(w, mode, idx, wts, x, sub_t=sub_t, replica=replica)
+    st = OracleStep(w, mode, sub_t, replica=replica)
     st.step()
     barrier.wait(timeout=600)
     t0 = time.perf_counter()
@@ -330,14 +352,14 @@ def _oracle_worker(job, barrier, results):
 
 
 def cpu_baseline_all_cores(wname, t_override, mode, seconds, replica=0):
-    """The oracle on the host's cores (up to 32): as many independent instances as cores
-    (spawned processes, each on a sample of T/8 tokens per rank), released
+    """The oracle on the host's cores (up to 32): as many independent instances as
+    cores (spawned processes, each on the same bounded sample), released
     together by a barrier and timed over the same interval; tokens/s summed."""
     import multiprocessing as mp
     ctx = mp.get_context("spawn")
     cores = min(os.cpu_count() or 1, 32)  # each instance is a process with its own imports
     w = synth.workload(wname) if t_override is None else synth.workload(wname, T=t_override)
-    sub_t = max(1, w["T"] // 8)
+    sub_t = sample_tokens_per_rank(w)
     barrier, results = ctx.Barrier(cores), ctx.Queue()
     job = (wname, t_override, mode, replica, sub_t, seconds)
     procs = [ctx.Process(target=_oracle_worker, args=(job, barrier, results)) for _ in range(cores)]
@@ -351,6 +373,273 @@ def cpu_baseline_all_cores(wname, t_override, mode, seconds, replica=0):
     return {"value": total / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
             "sample": f"{cores} independent instances, each the first {sub_t} of {w['T']} tokens "
                       f"of each of the {w['R']} ranks, started together; {seconds:.0f} s, summed"}
+
+
+# ---------------------------------------------------------------------------
+# one workload on the device: inputs, buffers and the bound C-ABI calls
+# ---------------------------------------------------------------------------
+class WorkloadRun:
+    """Device inputs, caller-owned buffers and bound C-ABI calls of one
+    workload.  Kernels (each a bound call, timed separately):
+      layout, dispatch, combine     the step (layout + dispatch run as the
+                                    one-call dispatch inside a step)
+      combine_bwd                   the step, for workloads with a backward
+      combine_q                     the combine of expert outputs stored in
+                                    the dispatch's quantised format (outside
+                                    the step), quantised modes only
+      combine_bwd_w                 the weight gradient (outside the step,
+                                    with --weights-grad)"""
+
+    def __init__(self, ep, wname, args, dev, stream, replica, mode=None, t_override=None,
+                 with_q=True, quantized_step=False, weights_grad=False):
+        w = synth.workload(wname) if t_override is None else synth.workload(wname, T=t_override)
+        self.ep, self.w, self.dev, self.stream = ep, w, dev, stream
+        self.mode = mode or WORKLOAD_MODE[wname]
+        R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
+        self.idx, self.wts = synth.make_routing(w, replica)
+        self.x = synth.make_x(w, replica)
+        self.cfg = cfg = ep.make_config(R, T, M, K, E, H, self.mode, w["layout"])
+        self.b = b = ep.Buffers(cfg, device=dev, grad=bool(w.get("backward")))
+        self.idx_d = torch.from_numpy(self.idx).to(dev)
+        self.wts_d = torch.from_numpy(self.wts).to(dev)
+        self.x_d = torch.from_numpy(self.x.view(np.int16)).to(dev).view(torch.bfloat16)
+        ypool, yoff = synth.y_source(w, b.sizes["rows"], replica)
+        pool_d = torch.from_numpy(ypool.view(np.int16)).to(dev)
+        torch.index_select(pool_d.as_strided((synth.POOL, H), (1, 1)), 0,
+                           torch.from_numpy(yoff).to(dev), out=b.y.view(torch.int16))
+        del pool_d
+        quantized = self.mode != "bf16"
+        self.qcfg = ep.make_config(R, T, M, K, E, H, self.mode, w["layout"],
+                                   flags=ep.F_COMBINE_QUANTIZED) if quantized else None
+        self.y_q = None
+        if quantized and (with_q or quantized_step):
+            # expert outputs in the dispatch format: the dispatched rows of one
+            # pass, copied to their own buffer (cold after every L2 flush)
+            ep.ep_dispatch_with_layout(cfg, self.x_d, self.idx_d, b.token_slot, b.recv_count,
+                                       b.workspace, b.recv_buf, b.src_info, b.dev_status,
+                                       expert_offset=b.expert_offset, stream=stream)
+            self.y_q = b.recv_buf.clone()
+        self.g_d = None
+        if w.get("backward"):
+            gp, go = synth.g_source(w, replica)
+            self.g_d = torch.from_numpy(synth.windows(gp, go, H).view(np.int16)).to(dev) \
+                .view(torch.bfloat16)
+        self.gw_d = self.dw_d = None
+        if weights_grad:
+            gp, go = synth.g_source(w, replica)
+            self.gw_d = torch.from_numpy(synth.windows(gp, go, H).view(np.int16)).to(dev) \
+                .view(torch.bfloat16)
+            self.dw_d = torch.empty((w["N"], K), dtype=torch.float32, device=dev)
+        eo = b.expert_offset
+        self.step_ccfg, self.step_y = (self.qcfg, self.y_q) if quantized_step and quantized \
+            else (cfg, b.y)
+        self.kernels = ["layout", "dispatch", "combine"]
+        if self.g_d is not None:
+            self.kernels.append("combine_bwd")
+        if quantized and with_q:
+            self.kernels.append("combine_q")
+        if weights_grad:
+            self.kernels.append("combine_bwd_w")
+        self.calls = {k: self.bound(k, 0) for k in self.kernels}
+        self.step_calls = [
+            ep.ep_dispatch_with_layout(cfg, self.x_d, self.idx_d, b.token_slot, b.recv_count,
+                                       b.workspace, b.recv_buf, b.src_info, b.dev_status,
+                                       expert_offset=eo, stream=stream, bind=True),
+            ep.ep_combine(self.step_ccfg, self.step_y, self.idx_d, self.wts_d, b.token_slot,
+                          b.out, b.dev_status, expert_offset=eo, stream=stream, bind=True),
+        ]
+        if self.g_d is not None:
+            self.step_calls.append(self.calls["combine_bwd"])
+        self.keep = []
+
+    def name(self):
+        w = self.w
+        return (f"{w['name']}: R={w['R']} T={w['T']} H={w['H']} K={w['K']} E={w['E']} "
+                f"M={w['M']} {self.mode} {w['layout']}")
+
+    def bound(self, k, copy):
+        """The bound call of kernel k; copy > 0 gives it its own copies of the
+        data-path buffers it reads and writes (for back-to-back launches whose
+        data is all cold)."""
+        ep, b, eo, s = self.ep, self.b, self.b.expert_offset, self.stream
+        cfg = self.cfg
+
+        def fresh(t, clone):
+            if not copy:
+                return t
+            u = t.clone() if clone else torch.empty_like(t)
+            self.keep.append(u)
+            return u
+        if k == "layout":
+            return ep.ep_dispatch_layout(cfg, self.idx_d, b.token_slot, b.recv_count, b.workspace,
+                                         b.dev_status, expert_offset=eo, stream=s, bind=True)
+        if k == "dispatch":
+            return ep.ep_dispatch(cfg, fresh(self.x_d, True), self.idx_d, b.token_slot,
+                                  fresh(b.recv_buf, False), fresh(b.src_info, False), b.dev_status,
+                                  expert_offset=eo, stream=s, bind=True)
+        if k == "combine":
+            return ep.ep_combine(cfg, fresh(b.y, True), self.idx_d, self.wts_d, b.token_slot,
+                                 fresh(b.out, False), b.dev_status, expert_offset=eo, stream=s,
+                                 bind=True)
+        if k == "combine_q":
+            return ep.ep_combine(self.qcfg, fresh(self.y_q, True), self.idx_d, self.wts_d,
+                                 b.token_slot, fresh(b.out, False), b.dev_status,
+                                 expert_offset=eo, stream=s, bind=True)
+        if k == "combine_bwd":
+            return ep.ep_combine_backward(cfg, fresh(self.g_d, True), self.idx_d, self.wts_d,
+                                          b.token_slot, fresh(b.grad_buf, False), b.dev_status,
+                                          expert_offset=eo, stream=s, bind=True)
+        if k == "combine_bwd_w":
+            return ep.ep_combine_backward_weights(cfg, fresh(self.gw_d, True), fresh(b.y, True),
+                                                  self.idx_d, b.token_slot, fresh(self.dw_d, False),
+                                                  b.dev_status, expert_offset=eo, stream=s,
+                                                  bind=True)
+        raise KeyError(k)
+
+    def step(self):
+        for c in self.step_calls:
+            c()
+
+    def release(self):
+        self.keep.clear()
+        self.calls.clear()
+        self.step_calls = []
+        for a in ("b", "x_d", "idx_d", "wts_d", "y_q", "g_d", "gw_d", "dw_d"):
+            setattr(self, a, None)
+        torch.cuda.empty_cache()
+
+
+STEADY_SETS = 4
+STEADY_MAX_BYTES = 1 << 30
+
+
+def isolated_launches(run, steps, flush):
+    """Each kernel alone between its own pair of events, after its own L2 flush,
+    `steps` times: {kernel: [ms]}."""
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in run.kernels] for _ in range(steps)]
+    torch.cuda.synchronize(run.dev)
+    for s in range(steps):
+        for i, k in enumerate(run.kernels):
+            flush(s & 0xFF)
+            evs[s][i][0].record(run.stream)
+            run.calls[k]()
+            evs[s][i][1].record(run.stream)
+    torch.cuda.synchronize(run.dev)
+    return {k: [e[i][0].elapsed_time(e[i][1]) for e in evs] for i, k in enumerate(run.kernels)}
+
+
+def steady_launches(run, steps, flush, step_bytes, skip=False):
+    """Per-launch durations with the launch overhead amortised as in the step:
+    each kernel is launched STEADY_SETS times back to back, on as many
+    distinct copies of the buffers it reads and writes (each launch's data is
+    cold: the group starts after an L2 flush and no two launches share a
+    buffer of the data path), between one pair of events; the dependent
+    launches overlap the tail of the previous grid, as the kernels of a step
+    do.  Workloads that move more than STEADY_MAX_BYTES a step are not timed
+    this way: there the launch overhead is already a negligible part of an
+    isolated launch.  Returns ({kernel: [ms per launch]}, sets)."""
+    if step_bytes > STEADY_MAX_BYTES or skip:
+        return {}, 1
+    sets = STEADY_SETS
+    per_set = {k: [run.calls[k]] + [run.bound(k, j) for j in range(1, sets)] for k in run.kernels}
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in run.kernels] for _ in range(steps)]
+    for s in range(steps):
+        for i, k in enumerate(run.kernels):
+            flush(s & 0xFF)
+            evs[s][i][0].record(run.stream)
+            for c in per_set[k]:
+                c()
+            evs[s][i][1].record(run.stream)
+    torch.cuda.synchronize(run.dev)
+    out = {k: [e[i][0].elapsed_time(e[i][1]) / sets for e in evs]
+           for i, k in enumerate(run.kernels)}
+    del per_set
+    run.keep.clear()
+    torch.cuda.empty_cache()
+    return out, sets
+
+
+def kernel_stats(run, per_kernel, steady, sets, alg, peak, peak_src):
+    ks = {}
+    for k in run.kernels:
+        mean_ms = statistics.mean(per_kernel[k])
+        gbs = alg[k] / (mean_ms * 1e-3) / 1e9
+        ks[k] = {"us_mean": round(mean_ms * 1e3, 2),
+                 "us_p10": round(float(np.percentile(per_kernel[k], 10)) * 1e3, 2),
+                 "us_p90": round(float(np.percentile(per_kernel[k], 90)) * 1e3, 2),
+                 "alg_bytes": alg[k], "gbs": round(gbs, 1),
+                 "frac_of_" + peak_src: round(gbs / peak, 4)}
+        if sets > 1:
+            st_ms = statistics.mean(steady[k])
+            ks[k].update({"us_steady": round(st_ms * 1e3, 2),
+                          "gbs_steady": round(alg[k] / (st_ms * 1e-3) / 1e9, 1),
+                          "frac_steady_of_" + peak_src:
+                              round(alg[k] / (st_ms * 1e-3) / 1e9 / peak, 4)})
+    return ks
+
+
+def step_bytes_of(alg):
+    """Algorithmic bytes of one step: the kernels of the step only."""
+    return sum(v for k, v in alg.items() if k not in ("combine_bwd_w", "combine_q"))
+
+
+def hbm_peak():
+    peaks = measured_peaks()
+    if peaks and peaks.get("hbm_gbs"):
+        return peaks["hbm_gbs"], "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def timed_steps(run, steps, flush):
+    """`steps` steps, one event pair each, L2 flushed before each outside the
+    events: [ms per step]."""
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for s in range(steps):
+        flush(s & 0xFF)
+        evs[s][0].record(run.stream)
+        run.step()
+        evs[s][1].record(run.stream)
+    torch.cuda.synchronize(run.dev)
+    return [a.elapsed_time(c) for a, c in evs]
+
+
+def other_workload(ep, wname, mode, args, dev, stream, flush, local):
+    """One of the other named workloads at full size: warm-up, the step timed
+    `steps` times, then the per-kernel passes; its own clock record."""
+    run = WorkloadRun(ep, wname, args, dev, stream, replica=0, mode=mode)
+    try:
+        for _ in range(max(args.warmup, 3)):
+            flush(1)
+            run.step()
+            for k in run.kernels:
+                run.calls[k]()
+        torch.cuda.synchronize(dev)
+        if ep.ep_get_status(run.b.dev_status) != 0:
+            raise RuntimeError("device status reported errors")
+        alg, v = algorithmic_bytes(run.w, run.mode, run.idx)
+        peak, peak_src = hbm_peak()
+        clocks = ClockSampler(local)
+        with clocks:
+            step_ms = timed_steps(run, args.steps, flush)
+            iso = isolated_launches(run, args.steps, flush)
+            steady, sets = steady_launches(run, args.steps, flush, step_bytes_of(alg),
+                                           skip=args.no_steady)
+        ms = statistics.mean(step_ms)
+        return {"workload": run.name(), "tokens_per_step": run.w["N"], "valid_entries": v,
+                "step_us": round(ms * 1e3, 2),
+                "tokens_per_s": round(run.w["N"] / (ms * 1e-3), 1),
+                "step_frac_of_" + peak_src: round(step_bytes_of(alg) / (ms * 1e-3) / 1e9 / peak, 4),
+                "kernels": kernel_stats(run, iso, steady, sets, alg, peak, peak_src),
+                "clocks": clocks.report()}
+    finally:
+        run.release()
+
+
+OTHER_WORKLOADS = [("tiny", "int8_token"), ("tiny", "bf16"), ("decode", None), ("skewed", None),
+                   ("large", None), ("prefill", None)]
 
 
 # ---------------------------------------------------------------------------
@@ -371,161 +660,53 @@ def main():
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    R, T, M, K, E, H = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"]
-    N = w["N"]
-    idx, wts = synth.make_routing(w, replica)
-    x = synth.make_x(w, replica)
-    cfg = ep.make_config(R, T, M, K, E, H, mode, w["layout"])
-    b = ep.Buffers(cfg, device=dev, grad=bool(w.get("backward")))
-    ccfg = cfg  # the combine's configuration
-    if args.quantized_combine:
-        ccfg = ep.make_config(R, T, M, K, E, H, mode, w["layout"], flags=ep.F_COMBINE_QUANTIZED)
-    rows = b.sizes["rows"]
-    idx_d = torch.from_numpy(idx).to(dev)
-    wts_d = torch.from_numpy(wts).to(dev)
-    x_d = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
-    ypool, yoff = synth.y_source(w, rows, replica)
-    pool_d = torch.from_numpy(ypool.view(np.int16)).to(dev)
-    torch.index_select(pool_d.as_strided((synth.POOL, H), (1, 1)), 0,
-                       torch.from_numpy(yoff).to(dev), out=b.y.view(torch.int16))
-    del pool_d
-    if args.quantized_combine:
-        # expert outputs in the dispatch format: the dispatched rows of one
-        # pass, copied to their own buffer (cold after every L2 flush)
-        ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
-                                   b.recv_buf, b.src_info, b.dev_status,
-                                   expert_offset=b.expert_offset)
-        b.y = b.recv_buf.clone()
-    g_d = None
-    if w.get("backward"):
-        gp, go = synth.g_source(w, replica)
-        g_d = torch.from_numpy(synth.windows(gp, go, H).view(np.int16)).to(dev).view(torch.bfloat16)
+    if args.weights_grad and args.quantized_combine:
+        raise SystemExit("--weights-grad reads bf16 expert outputs: not with --quantized-combine")
+    stream = torch.cuda.current_stream(dev)
     flush_w = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
     flush_r = torch.ones(args.flush_mib << 20, dtype=torch.uint8, device=dev)
-    stream = torch.cuda.current_stream(dev)
 
     def flush(v):
         flush_w.fill_(v)
         flush_r.max()
 
-    kernels = ["layout", "dispatch", "combine"] + (["combine_bwd"] if g_d is not None else [])
-    if args.weights_grad and args.quantized_combine:
-        raise SystemExit("--weights-grad reads bf16 expert outputs: not with --quantized-combine")
-    gw_d = dw_d = None
-    if args.weights_grad:
-        gp, go = synth.g_source(w, replica)
-        gw_d = torch.from_numpy(synth.windows(gp, go, H).view(np.int16)).to(dev).view(torch.bfloat16)
-        dw_d = torch.empty((N, K), dtype=torch.float32, device=dev)
-        kernels.append("combine_bwd_w")
-
-    # each C-ABI call is checked and marshalled once, then replayed every step.
-    # The timed step uses the one-call dispatch (layout + dispatch, the
-    # dispatch kernel overlapping the layout); the per-kernel pass uses the
-    # separate calls so that every kernel gets its own duration.
-    step_calls = [
-        ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
-                                   b.recv_buf, b.src_info, b.dev_status,
-                                   expert_offset=b.expert_offset, stream=stream, bind=True),
-        ep.ep_combine(ccfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
-                      expert_offset=b.expert_offset, stream=stream, bind=True),
-    ]
-    calls = [
-        ep.ep_dispatch_layout(cfg, idx_d, b.token_slot, b.recv_count, b.workspace, b.dev_status,
-                              expert_offset=b.expert_offset, stream=stream, bind=True),
-        ep.ep_dispatch(cfg, x_d, idx_d, b.token_slot, b.recv_buf, b.src_info, b.dev_status,
-                       expert_offset=b.expert_offset, stream=stream, bind=True),
-        ep.ep_combine(ccfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
-                      expert_offset=b.expert_offset, stream=stream, bind=True),
-    ]
-    if g_d is not None:
-        calls.append(ep.ep_combine_backward(cfg, g_d, idx_d, wts_d, b.token_slot, b.grad_buf,
-                                            b.dev_status, expert_offset=b.expert_offset,
-                                            stream=stream, bind=True))
-        step_calls.append(calls[-1])
-    if gw_d is not None:  # timed per kernel only: not a step of the configured path
-        calls.append(ep.ep_combine_backward_weights(cfg, gw_d, b.y, idx_d, b.token_slot, dw_d,
-                                                    b.dev_status, expert_offset=b.expert_offset,
-                                                    stream=stream, bind=True))
-
-    def step(evs=None, fl=0):
-        if evs is None:
-            for c in step_calls:
-                c()
-            return
-        for i, c in enumerate(calls):
-            flush(fl)
-            evs[i][0].record(stream)
-            c()
-            evs[i][1].record(stream)
-
+    run = WorkloadRun(ep, wname, args, dev, stream, replica, t_override=args.tokens_per_rank,
+                      quantized_step=args.quantized_combine, weights_grad=args.weights_grad)
+    N = run.w["N"]
     for _ in range(max(args.warmup, 3)):
         flush(1)
-        step()
+        run.step()
     torch.cuda.synchronize(dev)
-    if ep.ep_get_status(b.dev_status) != 0:
+    if ep.ep_get_status(run.b.dev_status) != 0:
         raise SystemExit("device status reported errors during warm-up")
 
     # timed region: K steps, one event pair per step (events between the
     # kernels would add their own ~2 us each to the step)
-    steps_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps)]
     clocks = ClockSampler(local)
     barrier(world)
     torch.cuda.synchronize(dev)
     launches0 = ep.ep_kernel_launches()
     with clocks:
-        for s in range(args.steps):
-            flush(s & 0xFF)
-            steps_ev[s][0].record(stream)
-            step()
-            steps_ev[s][1].record(stream)
-        torch.cuda.synchronize(dev)
+        step_ms = timed_steps(run, args.steps, flush)
     launches = ep.ep_kernel_launches() - launches0
     barrier(world)
-    step_ms = [a.elapsed_time(c) for a, c in steps_ev]
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
     value = world * N * args.steps / (total_ms / 1e3)
 
-    graph = graph_steps(ep, args, cfg, ccfg, b, x_d, idx_d, wts_d, g_d, flush, stream, dev, N,
-                        world)
+    graph = graph_steps(ep, args, run, flush, world)
 
-    # per-kernel durations (for the roofline): the same steps again, each
-    # kernel after its own flush and between its own pair of events
-    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in kernels] for _ in range(args.steps)]
-    torch.cuda.synchronize(dev)
-    for s in range(args.steps):
-        step(evs[s], s & 0xFF)
-    torch.cuda.synchronize(dev)
-    per_kernel = {k: [] for k in kernels}
-    for e in evs:
-        for i, k in enumerate(kernels):
-            per_kernel[k].append(e[i][0].elapsed_time(e[i][1]))
-
-    alg, v = algorithmic_bytes(w, mode, idx, quantized_combine=args.quantized_combine,
+    # per-kernel durations (for the roofline): each kernel after its own flush
+    # and between its own pair of events, then back to back where the step is small
+    per_kernel = isolated_launches(run, args.steps, flush)
+    alg, v = algorithmic_bytes(run.w, run.mode, run.idx, quantized_combine=args.quantized_combine,
                                weights_grad=args.weights_grad)
-    steady, sets = steady_launches(ep, args, cfg, ccfg, b, kernels, calls, x_d, idx_d, wts_d, g_d,
-                                   flush, stream, dev, sum(alg.values()), gw_d, dw_d)
-    peaks = measured_peaks()
-    peak = peaks["hbm_gbs"] if peaks and peaks.get("hbm_gbs") else FALLBACK_HBM_GBS
-    peak_src = "measured" if peaks and peaks.get("hbm_gbs") else "fallback"
-    kstats = {}
-    for k in kernels:
-        mean_ms = statistics.mean(per_kernel[k])
-        gbs = alg[k] / (mean_ms * 1e-3) / 1e9
-        kstats[k] = {"us_mean": round(mean_ms * 1e3, 2),
-                     "us_p10": round(float(np.percentile(per_kernel[k], 10)) * 1e3, 2),
-                     "us_p90": round(float(np.percentile(per_kernel[k], 90)) * 1e3, 2),
-                     "alg_bytes": alg[k], "gbs": round(gbs, 1),
-                     "frac_of_" + peak_src: round(gbs / peak, 4)}
-        if sets > 1:
-            st_ms = statistics.mean(steady[k])
-            kstats[k].update({"us_steady": round(st_ms * 1e3, 2),
-                              "gbs_steady": round(alg[k] / (st_ms * 1e-3) / 1e9, 1),
-                              "frac_steady_of_" + peak_src:
-                                  round(alg[k] / (st_ms * 1e-3) / 1e9 / peak, 4)})
-    dom = max((k for k in kernels if k != "combine_bwd_w"), key=lambda k: alg[k])
+    step_bytes = step_bytes_of(alg)
+    steady, sets = steady_launches(run, args.steps, flush, step_bytes, skip=args.no_steady)
+    peak, peak_src = hbm_peak()
+    kstats = kernel_stats(run, per_kernel, steady, sets, alg, peak, peak_src)
+    step_kernels = [k for k in run.kernels if k not in ("combine_bwd_w", "combine_q")]
+    dom = max(step_kernels, key=lambda k: alg[k])
     iso_achieved = alg[dom] / (statistics.mean(per_kernel[dom]) * 1e-3) / 1e9
     if sets > 1:
         achieved = alg[dom] / (statistics.mean(steady[dom]) * 1e-3) / 1e9
@@ -535,7 +716,12 @@ def main():
     else:
         achieved = iso_achieved
         duration = "per launch: each launch alone between its own events, after an L2 flush"
-    step_bytes = sum(v_ for k_, v_ in alg.items() if k_ != "combine_bwd_w")
+
+    e2e = None if args.no_e2e else run_e2e(ep, run, flush, args, world, step_bytes)
+    workload_name = run.name() + (", combine of quantised expert outputs"
+                                  if args.quantized_combine else "")
+    run.release()
+    del run
 
     # same-run copy bandwidth (reference for the fractions above)
     copy_gbs = None
@@ -557,27 +743,50 @@ def main():
             best = t if best is None or t < best else best
         copy_gbs = round(2 * src.numel() / (best * 1e-3) / 1e9, 1)
         del src, dst
+        torch.cuda.empty_cache()
     except Exception:
         pass
 
+    # every other named workload through the same per-kernel protocol (one GPU)
+    workloads = None
+    if world == 1 and not args.no_workloads and args.tokens_per_rank is None:
+        workloads = {}
+        for wn, md in OTHER_WORKLOADS:
+            key = wn if md is None or md == WORKLOAD_MODE[wn] else f"{wn}_{md}"
+            if wn == wname and (md is None or md == mode):
+                workloads[key] = {"see": "headline (kernels, roofline)"}
+                continue
+            try:
+                workloads[key] = other_workload(ep, wn, md, args, dev, stream, flush, local)
+            except Exception as ex:  # noqa: BLE001 -- reported in the line
+                workloads[key] = {"error": f"{type(ex).__name__}: {ex}"[:300]}
+                torch.cuda.empty_cache()
+
     # the experts between dispatch and combine, outside the step: by default on
-    # one GPU; a leg that fails reports its error instead of ending the bench
+    # one GPU, on the routing of --gemm-workload; a leg that fails reports its
+    # error instead of ending the bench
     gemm_on = args.gemm or (world == 1 and not args.no_gemm)
+    gemm = gemm_mx = gemm_mx4 = None
+    if gemm_on:
+        gw = synth.workload(args.gemm_workload)
+        gidx, gwts = synth.make_routing(gw, replica)
+        gx = synth.make_x(gw, replica)
+        gidx_d = torch.from_numpy(gidx).to(dev)
+        gwts_d = torch.from_numpy(gwts).to(dev)
+        gx_d = torch.from_numpy(gx.view(np.int16)).to(dev).view(torch.bfloat16)
 
-    def leg(fn, *a):
-        if not gemm_on:
-            return None
-        try:
-            return fn(*a)
-        except Exception as ex:  # noqa: BLE001 -- reported in the line
-            return {"error": f"{type(ex).__name__}: {ex}"[:300]}
-    gemm = leg(run_gemm, ep, w, x_d, idx_d, wts_d, flush, stream, dev, args)
-    gemm_mx = leg(run_gemm_mx, ep, w, x_d, idx_d, wts_d, flush, stream, dev, args)
-    gemm_mx4 = (leg(run_gemm_mx, ep, w, x_d, idx_d, wts_d, flush, stream, dev, args, "mxfp4")
-                if w["H"] % 256 == 0 else None)
-
-    e2e = None if args.no_e2e else run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream,
-                                          dev, args, world, step_bytes)
+        def leg(fn, *a):
+            try:
+                return fn(*a)
+            except Exception as ex:  # noqa: BLE001 -- reported in the line
+                torch.cuda.empty_cache()
+                return {"error": f"{type(ex).__name__}: {ex}"[:300]}
+        gemm = leg(run_gemm, ep, gw, gx_d, gidx_d, gwts_d, flush, stream, dev, args)
+        gemm_mx = leg(run_gemm_mx, ep, gw, gx_d, gidx_d, gwts_d, flush, stream, dev, args)
+        gemm_mx4 = (leg(run_gemm_mx, ep, gw, gx_d, gidx_d, gwts_d, flush, stream, dev, args,
+                        "mxfp4") if gw["H"] % 256 == 0 else None)
+        del gx_d, gidx_d, gwts_d
+        torch.cuda.empty_cache()
 
     out = {
         "metric": METRIC,
@@ -593,8 +802,7 @@ def main():
         "dtype": "f32",
         "data": "synthetic",
         "config": {
-            "workload": f"{wname}: R={R} T={T} H={H} K={K} E={E} M={M} {mode} {w['layout']}"
-                        + (", combine of quantised expert outputs" if args.quantized_combine else ""),
+            "workload": workload_name,
             "tokens_per_step": N, "valid_entries": v,
             "l2": f"flushed between steps outside the step events ({args.flush_mib} MiB write, "
                   f"then {args.flush_mib} MiB read); per-kernel timings: each kernel after its "
@@ -612,6 +820,7 @@ def main():
                      "isolated_launch": {"achieved": round(iso_achieved, 1),
                                          "frac": round(iso_achieved / peak, 4)}},
         "kernels": kstats,
+        "workloads": workloads,
         "graph": graph,
         "expert_gemm": gemm,
         "expert_gemm_mx": gemm_mx,
@@ -620,7 +829,7 @@ def main():
         "e2e": e2e,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(w, mode, idx, wts, x, args.cpu_seconds, replica)
+        out["cpu_baseline"] = cpu_baseline(w, mode, args.cpu_seconds, replica)
         try:
             out["cpu_baseline_all_cores"] = cpu_baseline_all_cores(
                 wname, args.tokens_per_rank, mode, args.cpu_seconds, replica)
@@ -631,25 +840,26 @@ def main():
     dist_done(world)
 
 
-def graph_steps(ep, args, cfg, ccfg, b, x_d, idx_d, wts_d, g_d, flush, stream, dev, N, world):
+def graph_steps(ep, args, run, flush, world):
     """The timed step captured once in a CUDA graph and replayed, with the same
     flush and event protocol: the step without the host's per-launch work (the
     device-side gaps between the kernels remain).  Every rank takes the same
     collective steps: the capture's outcome is agreed on first (a failure on
     any rank reports it on all and times nothing)."""
+    dev, stream, b = run.dev, run.stream, run.b
     graph, why = None, None
     try:
         gs = torch.cuda.Stream(dev)
         gcalls = [
-            ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
-                                       b.recv_buf, b.src_info, b.dev_status,
+            ep.ep_dispatch_with_layout(run.cfg, run.x_d, run.idx_d, b.token_slot, b.recv_count,
+                                       b.workspace, b.recv_buf, b.src_info, b.dev_status,
                                        expert_offset=b.expert_offset, stream=gs, bind=True),
-            ep.ep_combine(ccfg, b.y, idx_d, wts_d, b.token_slot, b.out, b.dev_status,
-                          expert_offset=b.expert_offset, stream=gs, bind=True),
+            ep.ep_combine(run.step_ccfg, run.step_y, run.idx_d, run.wts_d, b.token_slot, b.out,
+                          b.dev_status, expert_offset=b.expert_offset, stream=gs, bind=True),
         ]
-        if g_d is not None:
-            gcalls.append(ep.ep_combine_backward(cfg, g_d, idx_d, wts_d, b.token_slot,
-                                                 b.grad_buf, b.dev_status,
+        if run.g_d is not None:
+            gcalls.append(ep.ep_combine_backward(run.cfg, run.g_d, run.idx_d, run.wts_d,
+                                                 b.token_slot, b.grad_buf, b.dev_status,
                                                  expert_offset=b.expert_offset, stream=gs,
                                                  bind=True))
         gs.wait_stream(stream)
@@ -683,6 +893,7 @@ def graph_steps(ep, args, cfg, ccfg, b, x_d, idx_d, wts_d, g_d, flush, stream, d
     barrier(world)
     total = max_over_ranks(sum(a.elapsed_time(c) for a, c in evs), world)
     del graph
+    N = run.w["N"]
     return {"ms_per_step": round(total / args.steps, 5),
             "value": round(world * N * args.steps / (total / 1e3), 1), "unit": "tokens/s"}
 
@@ -849,69 +1060,10 @@ def run_gemm_mx(ep, w, x_d, idx_d, wts_d, flush, stream, dev, args, fmt="mxfp8")
             "shape": f"{E} experts, {v} rows, {H} x {H} {fmt.upper()} each", "moe_forward": moe}
 
 
-STEADY_SETS = 4
-STEADY_MAX_BYTES = 1 << 30
-
-
-def steady_launches(ep, args, cfg, ccfg, b, kernels, calls, x_d, idx_d, wts_d, g_d, flush, stream,
-                    dev, step_bytes, gw_d=None, dw_d=None):
-    """Per-launch durations with the launch overhead amortised as in the step:
-    each kernel is launched STEADY_SETS times back to back, on as many
-    distinct copies of the buffers it reads and writes (each launch's data is
-    cold: the group starts after an L2 flush and no two launches share a
-    buffer of the data path), between one pair of events; the dependent
-    launches overlap the tail of the previous grid, as the kernels of a step
-    do.  Workloads that move more than STEADY_MAX_BYTES a step are not timed
-    this way: there the launch overhead is already a negligible part of an
-    isolated launch.  Returns ({kernel: [ms per launch]}, sets)."""
-    if step_bytes > STEADY_MAX_BYTES or args.no_steady:
-        return {}, 1
-    sets = STEADY_SETS
-    eo = b.expert_offset
-    per_set = {k: [calls[i]] for i, k in enumerate(kernels)}
-    keep = []
-    for _ in range(1, sets):
-        xs, rb, si = x_d.clone(), torch.empty_like(b.recv_buf), torch.empty_like(b.src_info)
-        ys, os_ = b.y.clone(), torch.empty_like(b.out)
-        keep += [xs, rb, si, ys, os_]
-        per_set["layout"].append(calls[0])
-        per_set["dispatch"].append(ep.ep_dispatch(cfg, xs, idx_d, b.token_slot, rb, si, b.dev_status,
-                                                  expert_offset=eo, stream=stream, bind=True))
-        per_set["combine"].append(ep.ep_combine(ccfg, ys, idx_d, wts_d, b.token_slot, os_,
-                                                b.dev_status, expert_offset=eo, stream=stream,
-                                                bind=True))
-        if "combine_bwd_w" in per_set:
-            gws, dws = gw_d.clone(), torch.empty_like(dw_d)
-            keep += [gws, dws]
-            per_set["combine_bwd_w"].append(ep.ep_combine_backward_weights(
-                cfg, gws, ys, idx_d, b.token_slot, dws, b.dev_status, expert_offset=eo,
-                stream=stream, bind=True))
-        if "combine_bwd" in per_set:
-            gs, gb = g_d.clone(), torch.empty_like(b.grad_buf)
-            keep += [gs, gb]
-            per_set["combine_bwd"].append(ep.ep_combine_backward(
-                cfg, gs, idx_d, wts_d, b.token_slot, gb, b.dev_status, expert_offset=eo,
-                stream=stream, bind=True))
-    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-            for _ in kernels] for _ in range(args.steps)]
-    for s in range(args.steps):
-        for i, k in enumerate(kernels):
-            flush(s & 0xFF)
-            evs[s][i][0].record(stream)
-            for c in per_set[k]:
-                c()
-            evs[s][i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    out = {k: [e[i][0].elapsed_time(e[i][1]) / sets for e in evs] for i, k in enumerate(kernels)}
-    del keep, per_set
-    torch.cuda.empty_cache()
-    return out, sets
-
-
 L2_BYTES = 126 << 20
 
 
-def run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, world, step_bytes):
+def run_e2e(ep, run, flush, args, world, step_bytes):
     """The same step through the public API with host buffers: every step
     copies its inputs in from pinned host memory and its combined output and
     counts back, inside the timed region.  Steps are pipelined as a serving
@@ -922,10 +1074,12 @@ def run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, wor
     alternating sets move more than three L2s of data per pair of steps, so
     no step finds its data in L2; smaller workloads flush L2 before each
     step's kernels instead."""
+    w, b, cfg, ccfg, g_d = run.w, run.b, run.cfg, run.step_ccfg, run.g_d
+    dev, stream = run.dev, run.stream
     N, H = w["N"], w["H"]
-    x_h = torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory()
-    idx_h = torch.from_numpy(idx).to(ep.idx_dtype(cfg)).pin_memory()
-    wts_h = torch.from_numpy(wts).pin_memory()
+    x_h = torch.from_numpy(run.x.view(np.int16)).view(torch.bfloat16).pin_memory()
+    idx_h = torch.from_numpy(run.idx).to(ep.idx_dtype(cfg)).pin_memory()
+    wts_h = torch.from_numpy(run.wts).pin_memory()
     h2d = x_h.numel() * 2 + idx_h.numel() * idx_h.element_size() + wts_h.numel() * 4
     d2h = N * H * 2 + w["E"] * 8
     flush_each = 2 * step_bytes < 3 * L2_BYTES
@@ -934,9 +1088,8 @@ def run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, wor
     for j in range(2):
         bj = b if j == 0 else ep.Buffers(cfg, device=dev, expert_out=False,
                                           grad=g_d is not None)
-        if j == 1:
-            bj.y = b.y.clone()
-        st = {"b": bj,
+        yj = run.step_y if j == 0 else run.step_y.clone()
+        st = {"b": bj, "y": yj,
               "x": torch.empty((N, H), dtype=torch.bfloat16, device=dev),
               "idx": torch.empty_like(idx_h, device=dev),
               "wts": torch.empty_like(wts_h, device=dev),
@@ -948,7 +1101,7 @@ def run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, wor
             ep.ep_dispatch_with_layout(cfg, st["x"], st["idx"], bj.token_slot, bj.recv_count,
                                        bj.workspace, bj.recv_buf, bj.src_info, bj.dev_status,
                                        expert_offset=bj.expert_offset, stream=stream, bind=True),
-            ep.ep_combine(ccfg, bj.y, st["idx"], st["wts"], bj.token_slot, bj.out, bj.dev_status,
+            ep.ep_combine(ccfg, yj, st["idx"], st["wts"], bj.token_slot, bj.out, bj.dev_status,
                           expert_offset=bj.expert_offset, stream=stream, bind=True),
         ]
         if g_d is not None:
@@ -1011,13 +1164,12 @@ def run_e2e(ep, cfg, ccfg, b, w, idx, wts, x, g_d, flush, stream, dev, args, wor
 
 
 def run_reference(args, w, mode, world, rank):
-    """The reference arm: the oracle on the host cores, rank 0 only."""
+    """The reference arm: the oracle on the host cores, rank 0 only, each step
+    a bounded sample of the workload (about SAMPLE_TOKENS tokens)."""
     if rank != 0:
         dist_done(world)
         return
-    idx, wts = synth.make_routing(w, 0)
-    x = synth.make_x(w, 0)
-    st = OracleStep(w, mode, idx, wts, x, sub_t=max(1, w["T"] // 8))
+    st = OracleStep(w, mode, sample_tokens_per_rank(w))
     for _ in range(args.warmup):
         st.step()
     t0 = time.perf_counter()

@@ -4,7 +4,8 @@ The work runs in libep.so (C ABI in include/ep.h, sm_100a CUDA kernels);
 ``ep`` is its thin Python binding.  Importing the package without the built
 library raises ImportError: there is no CPU or library fallback.
 """
-from .ep import (DEV_BAD_INDEX, DEV_CAPACITY_OVERFLOW, DEV_TIMEOUT, STATIC_SCRATCH_BYTES, F_BWD_UNWEIGHTED,
+from .ep import (DEV_BAD_INDEX, DEV_CAPACITY_OVERFLOW, DEV_TIMEOUT, ERR_BUFFER_TOO_SMALL,
+                 STATIC_SCRATCH_BYTES, F_BWD_UNWEIGHTED,
                  F_COMBINE_QUANTIZED, F_GEMM_CTA_PAIRS, F_IDX_I32, F_LAYOUT_CLUSTER, F_LAYOUT_MULTI_CTA,
                  F_LAYOUT_SINGLE_CTA, F_ROUND_SCALE, F_UE8M0, LAYOUT, QUANT, Bound, Buffers,
                  EpConfig, EpError, EpSizes, ep_buffer_sizes, ep_combine, ep_combine_backward,
@@ -15,7 +16,8 @@ from .ep import (DEV_BAD_INDEX, DEV_CAPACITY_OVERFLOW, DEV_TIMEOUT, STATIC_SCRAT
                  make_config)
 
 __all__ = [
-    "DEV_BAD_INDEX", "DEV_CAPACITY_OVERFLOW", "DEV_TIMEOUT", "STATIC_SCRATCH_BYTES", "F_BWD_UNWEIGHTED",
+    "DEV_BAD_INDEX", "DEV_CAPACITY_OVERFLOW", "DEV_TIMEOUT", "ERR_BUFFER_TOO_SMALL",
+    "STATIC_SCRATCH_BYTES", "F_BWD_UNWEIGHTED",
     "F_COMBINE_QUANTIZED", "F_GEMM_CTA_PAIRS", "F_IDX_I32", "F_LAYOUT_CLUSTER", "F_LAYOUT_MULTI_CTA",
     "F_LAYOUT_SINGLE_CTA", "F_ROUND_SCALE", "F_UE8M0", "LAYOUT", "QUANT", "Bound", "Buffers",
     "EpConfig", "EpError", "EpSizes", "ep_buffer_sizes", "ep_combine", "ep_combine_backward",

@@ -55,6 +55,12 @@ cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
     return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// A caller buffer of `have` bytes where `want` are needed ([IDX] Runtime
+// Validation: sizes are checked before any GPU work).
+ep_status_t need(size_t have, int64_t want) {
+    return (int64_t)have >= want ? EP_OK : EP_ERR_BUFFER_TOO_SMALL;
+}
+
 ep_status_t launched() {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError() == cudaSuccess ? EP_OK : EP_ERR_CUDA;
@@ -157,7 +163,8 @@ ep_status_t make_plan(const ep_config_t *c, Plan &p) {
 
 struct ClusterChoice;
 ep_status_t check_layout_args(const ep_config_t *, const Plan &, const void *, const int32_t *,
-                              const int64_t *, const int64_t *, const void *, const uint32_t *);
+                              const int64_t *, const int64_t *, const void *, size_t,
+                              const uint32_t *);
 ep::LayoutArgs layout_args(const ep_config_t *, const Plan &, const void *, int32_t *, int32_t *,
                            uint8_t *, int32_t *, int64_t *, int64_t *, int64_t *, void *,
                            uint32_t *);
@@ -352,6 +359,7 @@ const char *ep_status_string(ep_status_t s) {
     case EP_ERR_CUDA: return "CUDA runtime error";
     case EP_ERR_DEVICE_STATUS: return "device reported bad indices or capacity overflow";
     case EP_ERR_TIMEOUT: return "timed out";
+    case EP_ERR_BUFFER_TOO_SMALL: return "a caller buffer is smaller than the configuration needs";
     }
     return "unknown status";
 }
@@ -385,12 +393,12 @@ ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const void *topk_idx,
                                uint8_t *is_token_in_rank, int32_t *token_slot,
                                int64_t *recv_count, int64_t *expert_offset,
                                int64_t *cumulative_recv_stats, void *workspace,
-                               uint32_t *dev_status, ep_stream_t stream) {
+                               size_t workspace_bytes, uint32_t *dev_status, ep_stream_t stream) {
     Plan p;
     ep_status_t st = make_plan(cfg, p);
     if (st != EP_OK) return st;
     if ((st = check_layout_args(cfg, p, topk_idx, token_slot, recv_count, expert_offset, workspace,
-                                dev_status)) != EP_OK)
+                                workspace_bytes, dev_status)) != EP_OK)
         return st;
     const ep::LayoutArgs a =
         layout_args(cfg, p, topk_idx, tokens_per_rank, tokens_per_expert, is_token_in_rank,
@@ -521,11 +529,11 @@ ep::DispatchArgs dispatch_args(const ep_config_t *cfg, const Plan &p) {
 ep_status_t check_layout_args(const ep_config_t *cfg, const Plan &p, const void *topk_idx,
                               const int32_t *token_slot, const int64_t *recv_count,
                               const int64_t *expert_offset, const void *workspace,
-                              const uint32_t *dev_status) {
+                              size_t workspace_bytes, const uint32_t *dev_status) {
     if (!recv_count || !workspace || !dev_status) return EP_ERR_INVALID_ARG;
     if (p.N > 0 && (!topk_idx || !token_slot)) return EP_ERR_INVALID_ARG;
     if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
-    return EP_OK;
+    return need(workspace_bytes, p.ws_bytes);
 }
 
 ep::LayoutArgs layout_args(const ep_config_t *cfg, const Plan &p, const void *topk_idx,
@@ -571,14 +579,20 @@ ep_status_t run_layout(const ep_config_t *cfg, const Plan &p, const ep::LayoutAr
     return launch_layout_multi(a, p, s);
 }
 
-ep_status_t check_dispatch_args(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
-                                const float *topk_weights, const int32_t *token_slot,
-                                const int64_t *expert_offset, const void *recv_buf,
-                                const int32_t *src_info, const float *recv_weights) {
+ep_status_t check_dispatch_args(const ep_config_t *cfg, const Plan &p, const uint16_t *x,
+                                const void *topk_idx, const float *topk_weights,
+                                const int32_t *token_slot, const int64_t *expert_offset,
+                                const void *recv_buf, size_t recv_bytes, const int32_t *src_info,
+                                size_t src_info_bytes, const float *recv_weights,
+                                size_t recv_weights_bytes) {
     if (!x || !topk_idx || !token_slot || !recv_buf || !src_info) return EP_ERR_INVALID_ARG;
     if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
     if (recv_weights && !topk_weights) return EP_ERR_INVALID_ARG;
     if (!aligned16(x) || !aligned16(recv_buf)) return EP_ERR_MISALIGNED;
+    ep_status_t st;
+    if ((st = need(recv_bytes, p.recv_bytes)) != EP_OK) return st;
+    if ((st = need(src_info_bytes, p.rows * 4)) != EP_OK) return st;
+    if (recv_weights && (st = need(recv_weights_bytes, p.rows * 4)) != EP_OK) return st;
     return EP_OK;
 }
 
@@ -666,15 +680,17 @@ extern "C" {
 
 ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
                         const float *topk_weights, const int32_t *token_slot,
-                        const int64_t *expert_offset, void *recv_buf, int32_t *src_info,
-                        float *recv_weights, uint32_t *dev_status, ep_stream_t stream) {
+                        const int64_t *expert_offset, void *recv_buf, size_t recv_bytes,
+                        int32_t *src_info, size_t src_info_bytes, float *recv_weights,
+                        size_t recv_weights_bytes, uint32_t *dev_status, ep_stream_t stream) {
     Plan p;
     ep_status_t st = make_plan(cfg, p);
     if (st != EP_OK) return st;
     if (!dev_status) return EP_ERR_INVALID_ARG;
     if (p.N == 0) return EP_OK;
-    if ((st = check_dispatch_args(cfg, x, topk_idx, topk_weights, token_slot, expert_offset,
-                                  recv_buf, src_info, recv_weights)) != EP_OK)
+    if ((st = check_dispatch_args(cfg, p, x, topk_idx, topk_weights, token_slot, expert_offset,
+                                  recv_buf, recv_bytes, src_info, src_info_bytes, recv_weights,
+                                  recv_weights_bytes)) != EP_OK)
         return st;
     ep::DispatchArgs a = full_dispatch_args(cfg, p, x, topk_idx, topk_weights, token_slot,
                                             expert_offset, recv_buf, src_info, recv_weights,
@@ -688,17 +704,20 @@ ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
                                     uint8_t *is_token_in_rank, int32_t *token_slot,
                                     int64_t *recv_count, int64_t *expert_offset,
                                     int64_t *cumulative_recv_stats, void *workspace,
-                                    void *recv_buf, int32_t *src_info, float *recv_weights,
-                                    uint32_t *dev_status, ep_stream_t stream) {
+                                    size_t workspace_bytes, void *recv_buf, size_t recv_bytes,
+                                    int32_t *src_info, size_t src_info_bytes, float *recv_weights,
+                                    size_t recv_weights_bytes, uint32_t *dev_status,
+                                    ep_stream_t stream) {
     Plan p;
     ep_status_t st = make_plan(cfg, p);
     if (st != EP_OK) return st;
     if ((st = check_layout_args(cfg, p, topk_idx, token_slot, recv_count, expert_offset, workspace,
-                                dev_status)) != EP_OK)
+                                workspace_bytes, dev_status)) != EP_OK)
         return st;
-    if (p.N > 0 && (st = check_dispatch_args(cfg, x, topk_idx, topk_weights, token_slot,
-                                             expert_offset, recv_buf, src_info, recv_weights)) !=
-                       EP_OK)
+    if (p.N > 0 &&
+        (st = check_dispatch_args(cfg, p, x, topk_idx, topk_weights, token_slot, expert_offset,
+                                  recv_buf, recv_bytes, src_info, src_info_bytes, recv_weights,
+                                  recv_weights_bytes)) != EP_OK)
         return st;
     cudaStream_t s = cs(stream);
     const ep::LayoutArgs la =
@@ -713,8 +732,8 @@ ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
     return run_dispatch(cfg, a, s);
 }
 
-ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const void *topk_idx,
-                       const float *topk_weights, const int32_t *token_slot,
+ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, size_t y_bytes,
+                       const void *topk_idx, const float *topk_weights, const int32_t *token_slot,
                        const int64_t *expert_offset, uint16_t *out, uint32_t *dev_status,
                        ep_stream_t stream) {
     Plan p;
@@ -727,6 +746,8 @@ ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const void *to
     if (!aligned16(y) || !aligned16(out)) return EP_ERR_MISALIGNED;
 
     const int qin = (cfg->flags & EP_F_COMBINE_QUANTIZED) ? cfg->quant : EP_Q_BF16;
+    if ((st = need(y_bytes, qin == EP_Q_BF16 ? p.rows * p.H * 2 : p.recv_bytes)) != EP_OK)
+        return st;
     ep::CombineArgs a;
     a.N = p.N; a.K = p.K; a.E = p.E; a.H = p.H;
     a.packed = cfg->layout == EP_LAYOUT_PACKED;
@@ -749,7 +770,8 @@ ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const void *to
 ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
                                 const void *topk_idx, const float *topk_weights,
                                 const int32_t *token_slot, const int64_t *expert_offset,
-                                void *grad_buf, uint32_t *dev_status, ep_stream_t stream) {
+                                void *grad_buf, size_t grad_bytes, uint32_t *dev_status,
+                                ep_stream_t stream) {
     Plan p;
     ep_status_t st = make_plan(cfg, p);
     if (st != EP_OK) return st;
@@ -760,6 +782,7 @@ ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
     if (!unweighted && !topk_weights) return EP_ERR_INVALID_ARG;
     if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
     if (!aligned16(g) || !aligned16(grad_buf)) return EP_ERR_MISALIGNED;
+    if ((st = need(grad_bytes, p.grad_bytes)) != EP_OK) return st;
 
     ep::DispatchArgs a = dispatch_args(cfg, p);
     a.D = p.H; a.S = p.H / 32; a.scale_off = p.grad_scale_off;
@@ -772,7 +795,7 @@ ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
 }
 
 ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *g,
-                                        const uint16_t *y, const void *topk_idx,
+                                        const uint16_t *y, size_t y_bytes, const void *topk_idx,
                                         const int32_t *token_slot, const int64_t *expert_offset,
                                         float *topk_weights_grad, uint32_t *dev_status,
                                         ep_stream_t stream) {
@@ -785,6 +808,7 @@ ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *
     if (!g || !y || !topk_idx || !token_slot || !topk_weights_grad) return EP_ERR_INVALID_ARG;
     if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
     if (!aligned16(g) || !aligned16(y)) return EP_ERR_MISALIGNED;
+    if ((st = need(y_bytes, p.rows * p.H * 2)) != EP_OK) return st;
 
     ep::WgradArgs a;
     a.N = p.N; a.K = p.K; a.E = p.E; a.H = p.H;
@@ -934,9 +958,10 @@ int mx_tile_n(int n_out, bool fp4 = false, int64_t rows_per_expert = 0) {
 // nothing to do when p.N == 0), then the launches.  `w_scales` null selects
 // the bf16 maps, else the MX ones (cfg->quant MXFP8 / MXFP4).
 ep_status_t check_gemm_args(const ep_config_t *cfg, const Plan &p, bool mx, int n_out,
-                            const void *recv_buf, const int64_t *expert_offset,
-                            const int64_t *recv_count, const void *w_codes,
-                            const void *w_scales, const void *y, const uint32_t *dev_status) {
+                            const void *recv_buf, size_t recv_bytes,
+                            const int64_t *expert_offset, const int64_t *recv_count,
+                            const void *w_codes, const void *w_scales, const void *y,
+                            size_t y_bytes, const uint32_t *dev_status) {
     const bool fp4 = cfg->quant == EP_Q_MXFP4;
     if (cfg->layout != EP_LAYOUT_PACKED) return EP_ERR_UNSUPPORTED;
     if (mx) {
@@ -956,7 +981,10 @@ ep_status_t check_gemm_args(const ep_config_t *cfg, const Plan &p, bool mx, int 
     if (!aligned16(recv_buf) || !aligned16(w_codes) || !aligned16(y) ||
         (mx && !aligned16(w_scales)))
         return EP_ERR_MISALIGNED;
-    return EP_OK;
+    // the bf16 maps read the data region only; the MX maps also the scales after it
+    ep_status_t st = need(recv_bytes, mx ? p.recv_bytes : p.rows * p.D);
+    if (st != EP_OK) return st;
+    return need(y_bytes, p.rows * (int64_t)n_out * 2);
 }
 
 ep_status_t run_gemm_bf16(const ep_config_t *cfg, const Plan &p, const void *recv_buf,
@@ -1022,29 +1050,32 @@ ep_status_t run_gemm_mx(const ep_config_t *cfg, const Plan &p, const void *recv_
 }
 }  // namespace
 
-ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
+ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf, size_t recv_bytes,
                            const int64_t *expert_offset, const int64_t *recv_count,
-                           const uint16_t *weights, int32_t n_out, uint16_t *y,
+                           const uint16_t *weights, int32_t n_out, uint16_t *y, size_t y_bytes,
                            uint32_t *dev_status, ep_stream_t stream) {
     Plan p;
     ep_status_t st = make_plan(cfg, p);
     if (st != EP_OK) return st;
-    if ((st = check_gemm_args(cfg, p, false, n_out, recv_buf, expert_offset, recv_count, weights,
-                              nullptr, y, dev_status)) != EP_OK || p.N == 0)
+    if ((st = check_gemm_args(cfg, p, false, n_out, recv_buf, recv_bytes, expert_offset,
+                              recv_count, weights, nullptr, y, y_bytes, dev_status)) != EP_OK ||
+        p.N == 0)
         return st;
     return run_gemm_bf16(cfg, p, recv_buf, expert_offset, recv_count, weights, n_out, y,
                          dev_status, cs(stream));
 }
 
-ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
+ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf, size_t recv_bytes,
                               const int64_t *expert_offset, const int64_t *recv_count,
                               const uint8_t *w_codes, const uint8_t *w_scales, int32_t n_out,
-                              uint16_t *y, uint32_t *dev_status, ep_stream_t stream) {
+                              uint16_t *y, size_t y_bytes, uint32_t *dev_status,
+                              ep_stream_t stream) {
     Plan p;
     ep_status_t st = make_plan(cfg, p);
     if (st != EP_OK) return st;
-    if ((st = check_gemm_args(cfg, p, true, n_out, recv_buf, expert_offset, recv_count, w_codes,
-                              w_scales, y, dev_status)) != EP_OK || p.N == 0)
+    if ((st = check_gemm_args(cfg, p, true, n_out, recv_buf, recv_bytes, expert_offset,
+                              recv_count, w_codes, w_scales, y, y_bytes, dev_status)) != EP_OK ||
+        p.N == 0)
         return st;
     return run_gemm_mx(cfg, p, recv_buf, expert_offset, recv_count, w_codes, w_scales, n_out, y,
                        dev_status, cs(stream));
@@ -1053,9 +1084,10 @@ ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
 ep_status_t ep_moe_forward(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
                            const float *topk_weights, const void *w_codes,
                            const uint8_t *w_scales, int32_t *token_slot, int64_t *recv_count,
-                           int64_t *expert_offset, void *workspace, void *recv_buf,
-                           int32_t *src_info, uint16_t *y, uint16_t *out, uint32_t *dev_status,
-                           ep_stream_t stream) {
+                           int64_t *expert_offset, void *workspace, size_t workspace_bytes,
+                           void *recv_buf, size_t recv_bytes, int32_t *src_info,
+                           size_t src_info_bytes, uint16_t *y, size_t y_bytes, uint16_t *out,
+                           uint32_t *dev_status, ep_stream_t stream) {
     Plan p;
     ep_status_t st = make_plan(cfg, p);
     if (st != EP_OK) return st;
@@ -1063,21 +1095,23 @@ ep_status_t ep_moe_forward(const ep_config_t *cfg, const uint16_t *x, const void
     const bool mx = cfg->quant != EP_Q_BF16;
     // every argument is checked before the first launch
     if ((st = check_layout_args(cfg, p, topk_idx, token_slot, recv_count, expert_offset, workspace,
-                                dev_status)) != EP_OK)
+                                workspace_bytes, dev_status)) != EP_OK)
         return st;
-    if ((st = check_gemm_args(cfg, p, mx, p.H, recv_buf, expert_offset, recv_count, w_codes,
-                              w_scales, y, dev_status)) != EP_OK)
+    if ((st = check_gemm_args(cfg, p, mx, p.H, recv_buf, recv_bytes, expert_offset, recv_count,
+                              w_codes, w_scales, y, y_bytes, dev_status)) != EP_OK)
         return st;
     if (p.N > 0) {
-        if ((st = check_dispatch_args(cfg, x, topk_idx, topk_weights, token_slot, expert_offset,
-                                      recv_buf, src_info, nullptr)) != EP_OK)
+        if ((st = check_dispatch_args(cfg, p, x, topk_idx, topk_weights, token_slot,
+                                      expert_offset, recv_buf, recv_bytes, src_info,
+                                      src_info_bytes, nullptr, 0)) != EP_OK)
             return st;
         if (!topk_weights || !out) return EP_ERR_INVALID_ARG;
         if (!aligned16(out)) return EP_ERR_MISALIGNED;
     }
     if ((st = ep_dispatch_with_layout(cfg, x, topk_idx, topk_weights, nullptr, nullptr, nullptr,
                                       token_slot, recv_count, expert_offset, nullptr, workspace,
-                                      recv_buf, src_info, nullptr, dev_status, stream)) != EP_OK ||
+                                      workspace_bytes, recv_buf, recv_bytes, src_info,
+                                      src_info_bytes, nullptr, 0, dev_status, stream)) != EP_OK ||
         p.N == 0)
         return st;
     const cudaStream_t s = cs(stream);
@@ -1086,8 +1120,8 @@ ep_status_t ep_moe_forward(const ep_config_t *cfg, const uint16_t *x, const void
             : run_gemm_bf16(cfg, p, recv_buf, expert_offset, recv_count,
                             static_cast<const uint16_t *>(w_codes), p.H, y, dev_status, s);
     if (st != EP_OK) return st;
-    return ep_combine(cfg, y, topk_idx, topk_weights, token_slot, expert_offset, out, dev_status,
-                      stream);
+    return ep_combine(cfg, y, y_bytes, topk_idx, topk_weights, token_slot, expert_offset, out,
+                      dev_status, stream);
 }
 
 ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream) {

@@ -38,7 +38,9 @@ F_GEMM_CTA_PAIRS = 0x800
 STATIC_SCRATCH_BYTES = 1 << 20  # EP_STATIC_SCRATCH_BYTES of include/ep.h
 
 STATUS = {0: "EP_OK", 1: "EP_ERR_INVALID_ARG", 2: "EP_ERR_UNSUPPORTED", 3: "EP_ERR_MISALIGNED",
-          4: "EP_ERR_CUDA", 5: "EP_ERR_DEVICE_STATUS", 6: "EP_ERR_TIMEOUT"}
+          4: "EP_ERR_CUDA", 5: "EP_ERR_DEVICE_STATUS", 6: "EP_ERR_TIMEOUT",
+          7: "EP_ERR_BUFFER_TOO_SMALL"}
+ERR_BUFFER_TOO_SMALL = 7
 
 
 class EpError(RuntimeError):
@@ -64,33 +66,34 @@ class EpSizes(C.Structure):
 
 
 _P = C.c_void_p
+_Z = C.c_size_t
 _CFG = C.POINTER(EpConfig)
 lib.ep_status_string.restype = C.c_char_p
 lib.ep_status_string.argtypes = [C.c_int]
 lib.ep_buffer_sizes.restype = C.c_int
 lib.ep_buffer_sizes.argtypes = [_CFG, C.POINTER(EpSizes)]
 lib.ep_dispatch_layout.restype = C.c_int
-lib.ep_dispatch_layout.argtypes = [_CFG] + [_P] * 11
+lib.ep_dispatch_layout.argtypes = [_CFG] + [_P] * 9 + [_Z, _P, _P]
 lib.ep_dispatch_layout_static.restype = C.c_int
 lib.ep_dispatch_layout_static.argtypes = [_CFG] + [_P] * 10
 lib.ep_dispatch_with_layout.restype = C.c_int
-lib.ep_dispatch_with_layout.argtypes = [_CFG] + [_P] * 16
+lib.ep_dispatch_with_layout.argtypes = [_CFG] + [_P] * 11 + [_Z, _P, _Z, _P, _Z, _P, _Z, _P, _P]
 lib.ep_dispatch.restype = C.c_int
-lib.ep_dispatch.argtypes = [_CFG] + [_P] * 10
+lib.ep_dispatch.argtypes = [_CFG] + [_P] * 6 + [_Z, _P, _Z, _P, _Z, _P, _P]
 lib.ep_combine.restype = C.c_int
-lib.ep_combine.argtypes = [_CFG] + [_P] * 8
+lib.ep_combine.argtypes = [_CFG, _P, _Z] + [_P] * 7
 lib.ep_combine_backward.restype = C.c_int
-lib.ep_combine_backward.argtypes = [_CFG] + [_P] * 8
+lib.ep_combine_backward.argtypes = [_CFG] + [_P] * 6 + [_Z, _P, _P]
 lib.ep_expert_gemm.restype = C.c_int
-lib.ep_expert_gemm.argtypes = [_CFG, _P, _P, _P, _P, C.c_int32, _P, _P, _P]
+lib.ep_expert_gemm.argtypes = [_CFG, _P, _Z, _P, _P, _P, C.c_int32, _P, _Z, _P, _P]
 lib.ep_wait_probe.restype = C.c_int
 lib.ep_wait_probe.argtypes = [_P, _P]
 lib.ep_moe_forward.restype = C.c_int
-lib.ep_moe_forward.argtypes = [_CFG] + [_P] * 14 + [_P]
+lib.ep_moe_forward.argtypes = [_CFG] + [_P] * 9 + [_Z, _P, _Z, _P, _Z, _P, _Z, _P, _P, _P]
 lib.ep_expert_gemm_mx.restype = C.c_int
-lib.ep_expert_gemm_mx.argtypes = [_CFG, _P, _P, _P, _P, _P, C.c_int32, _P, _P, _P]
+lib.ep_expert_gemm_mx.argtypes = [_CFG, _P, _Z, _P, _P, _P, _P, C.c_int32, _P, _Z, _P, _P]
 lib.ep_combine_backward_weights.restype = C.c_int
-lib.ep_combine_backward_weights.argtypes = [_CFG] + [_P] * 8
+lib.ep_combine_backward_weights.argtypes = [_CFG, _P, _P, _Z] + [_P] * 6
 lib.ep_get_status.restype = C.c_int
 lib.ep_get_status.argtypes = [_P, C.POINTER(C.c_uint32), _P]
 lib.ep_copy.restype = C.c_int
@@ -164,15 +167,14 @@ def _dev(t, name, dtype, shape=None, optional=False):
     return C.c_void_p(t.data_ptr())
 
 
-def _bytes(t, name, nbytes, optional=False):
-    """Device pointer of a contiguous CUDA byte buffer of at least nbytes."""
+def _buf(t, name, optional=False):
+    """(device pointer, byte count) of a contiguous CUDA buffer; libep checks the
+    count against what the configuration needs (EP_ERR_BUFFER_TOO_SMALL)."""
     if t is None and optional:
-        return None
-    if t is None or not t.is_cuda or not t.is_contiguous():
+        return [None, C.c_size_t(0)]
+    if t is None or not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA tensor")
-    if t.numel() * t.element_size() < nbytes:
-        raise ValueError(f"{name} holds {t.numel() * t.element_size()} bytes, needs {nbytes}")
-    return C.c_void_p(t.data_ptr())
+    return [C.c_void_p(t.data_ptr()), C.c_size_t(t.numel() * t.element_size())]
 
 
 def _nk(cfg):
@@ -189,7 +191,6 @@ def ep_dispatch_layout(cfg, topk_idx, token_slot, recv_count, workspace, dev_sta
                        expert_offset=None, cumulative_recv_stats=None, stream=None, bind=False):
     N, K = _nk(cfg)
     R, E = cfg.num_ranks, cfg.num_experts
-    sz = ep_buffer_sizes(cfg)
     args = [
         _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
         _dev(tokens_per_rank, "tokens_per_rank", torch.int32, (R, R), optional=True),
@@ -200,7 +201,7 @@ def ep_dispatch_layout(cfg, topk_idx, token_slot, recv_count, workspace, dev_sta
         _dev(expert_offset, "expert_offset", torch.int64, (E + 1,),
              optional=cfg.layout == LAYOUT["padded"]),
         _dev(cumulative_recv_stats, "cumulative_recv_stats", torch.int64, (E,), optional=True),
-        _bytes(workspace, "workspace", sz["workspace_bytes"]),
+        *_buf(workspace, "workspace"),
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
     ]
@@ -235,7 +236,6 @@ def ep_dispatch_layout_static(cfg, topk_idx, token_slot, recv_count, dev_status,
 def ep_dispatch(cfg, x, topk_idx, token_slot, recv_buf, src_info, dev_status, topk_weights=None,
                 expert_offset=None, recv_weights=None, stream=None, bind=False):
     N, K = _nk(cfg)
-    sz = ep_buffer_sizes(cfg)
     args = [
         _dev(x, "x", torch.bfloat16, (N, cfg.hidden)),
         _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
@@ -243,9 +243,9 @@ def ep_dispatch(cfg, x, topk_idx, token_slot, recv_buf, src_info, dev_status, to
         _dev(token_slot, "token_slot", torch.int32, (N, K)),
         _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
              optional=cfg.layout == LAYOUT["padded"]),
-        _bytes(recv_buf, "recv_buf", sz["recv_bytes"]),
-        _bytes(src_info, "src_info", sz["src_info_bytes"]),
-        _bytes(recv_weights, "recv_weights", sz["recv_weights_bytes"], optional=True),
+        *_buf(recv_buf, "recv_buf"),
+        *_buf(src_info, "src_info"),
+        *_buf(recv_weights, "recv_weights", optional=True),
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
     ]
@@ -261,7 +261,6 @@ def ep_dispatch_with_layout(cfg, x, topk_idx, token_slot, recv_count, workspace,
     overlaps the layout; see include/ep.h)."""
     N, K = _nk(cfg)
     R, E = cfg.num_ranks, cfg.num_experts
-    sz = ep_buffer_sizes(cfg)
     args = [
         _dev(x, "x", torch.bfloat16, (N, cfg.hidden)),
         _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
@@ -274,10 +273,10 @@ def ep_dispatch_with_layout(cfg, x, topk_idx, token_slot, recv_count, workspace,
         _dev(expert_offset, "expert_offset", torch.int64, (E + 1,),
              optional=cfg.layout == LAYOUT["padded"]),
         _dev(cumulative_recv_stats, "cumulative_recv_stats", torch.int64, (E,), optional=True),
-        _bytes(workspace, "workspace", sz["workspace_bytes"]),
-        _bytes(recv_buf, "recv_buf", sz["recv_bytes"]),
-        _bytes(src_info, "src_info", sz["src_info_bytes"]),
-        _bytes(recv_weights, "recv_weights", sz["recv_weights_bytes"], optional=True),
+        *_buf(workspace, "workspace"),
+        *_buf(recv_buf, "recv_buf"),
+        *_buf(src_info, "src_info"),
+        *_buf(recv_weights, "recv_weights", optional=True),
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
     ]
@@ -287,12 +286,11 @@ def ep_dispatch_with_layout(cfg, x, topk_idx, token_slot, recv_count, workspace,
 def ep_combine(cfg, y, topk_idx, topk_weights, token_slot, out, dev_status, expert_offset=None,
                stream=None, bind=False):
     N, K = _nk(cfg)
-    sz = ep_buffer_sizes(cfg)
     quantized = bool(cfg.flags & F_COMBINE_QUANTIZED) and cfg.quant != QUANT["bf16"]
     if y is None or (not quantized and y.dtype != torch.bfloat16):
         raise TypeError("y (expert outputs) must be bfloat16 unless F_COMBINE_QUANTIZED")
     args = [
-        _bytes(y, "y", sz["recv_bytes"] if quantized else sz["expert_out_bytes"]),
+        *_buf(y, "y"),
         _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
         _dev(topk_weights, "topk_weights", torch.float32, (N, K)),
         _dev(token_slot, "token_slot", torch.int32, (N, K)),
@@ -308,7 +306,6 @@ def ep_combine(cfg, y, topk_idx, topk_weights, token_slot, out, dev_status, expe
 def ep_combine_backward(cfg, g, topk_idx, topk_weights, token_slot, grad_buf, dev_status,
                         expert_offset=None, stream=None, bind=False):
     N, K = _nk(cfg)
-    sz = ep_buffer_sizes(cfg)
     args = [
         _dev(g, "g", torch.bfloat16, (N, cfg.hidden)),
         _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
@@ -317,7 +314,7 @@ def ep_combine_backward(cfg, g, topk_idx, topk_weights, token_slot, grad_buf, de
         _dev(token_slot, "token_slot", torch.int32, (N, K)),
         _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
              optional=cfg.layout == LAYOUT["padded"]),
-        _bytes(grad_buf, "grad_buf", sz["grad_bytes"]),
+        *_buf(grad_buf, "grad_buf"),
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
     ]
@@ -334,12 +331,12 @@ def ep_expert_gemm(cfg, recv_buf, expert_offset, recv_count, weights, y, dev_sta
         raise ValueError("weights must be a [E, n_out, H] tensor")
     n_out = int(weights.shape[1])
     args = [
-        _bytes(recv_buf, "recv_buf", sz["rows"] * sz["data_row_bytes"]),
+        *_buf(recv_buf, "recv_buf"),
         _dev(expert_offset, "expert_offset", torch.int64, (E + 1,)),
         _dev(recv_count, "recv_count", torch.int64, (E,)),
         _dev(weights, "weights", torch.bfloat16, (E, n_out, H)),
         C.c_int32(n_out),
-        _dev(y, "y", torch.bfloat16, (sz["rows"], n_out)),
+        _dev(y, "y", torch.bfloat16, (sz["rows"], n_out)), C.c_size_t(sz["rows"] * n_out * 2),
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
     ]
@@ -358,13 +355,13 @@ def ep_expert_gemm_mx(cfg, recv_buf, expert_offset, recv_count, w_codes, w_scale
         raise ValueError("w_codes must be a [E, n_out, D] tensor")
     n_out = int(w_codes.shape[1])
     args = [
-        _bytes(recv_buf, "recv_buf", sz["recv_bytes"]),
+        *_buf(recv_buf, "recv_buf"),
         _dev(expert_offset, "expert_offset", torch.int64, (E + 1,)),
         _dev(recv_count, "recv_count", torch.int64, (E,)),
         _dev(w_codes, "w_codes", torch.uint8, (E, n_out, D)),
         _dev(w_scales, "w_scales", torch.uint8, (E, n_out, H // 32)),
         C.c_int32(n_out),
-        _dev(y, "y", torch.bfloat16, (sz["rows"], n_out)),
+        _dev(y, "y", torch.bfloat16, (sz["rows"], n_out)), C.c_size_t(sz["rows"] * n_out * 2),
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
     ]
@@ -404,10 +401,10 @@ def ep_moe_forward(cfg, x, topk_idx, topk_weights, w_codes, w_scales, token_slot
         _dev(token_slot, "token_slot", torch.int32, (N, K)),
         _dev(recv_count, "recv_count", torch.int64, (E,)),
         _dev(expert_offset, "expert_offset", torch.int64, (E + 1,)),
-        _bytes(workspace, "workspace", sz["workspace_bytes"]),
-        _bytes(recv_buf, "recv_buf", sz["recv_bytes"]),
-        _bytes(src_info, "src_info", sz["src_info_bytes"]),
-        _dev(y, "y", torch.bfloat16, (sz["rows"], H)),
+        *_buf(workspace, "workspace"),
+        *_buf(recv_buf, "recv_buf"),
+        *_buf(src_info, "src_info"),
+        _dev(y, "y", torch.bfloat16, (sz["rows"], H)), C.c_size_t(sz["rows"] * H * 2),
         _dev(out, "out", torch.bfloat16, (N, H)),
         _dev(dev_status, "dev_status", torch.int32, (1,)),
         _stream(stream),
@@ -423,6 +420,7 @@ def ep_combine_backward_weights(cfg, g, y, topk_idx, token_slot, topk_weights_gr
     args = [
         _dev(g, "g", torch.bfloat16, (N, cfg.hidden)),
         _dev(y, "y", torch.bfloat16, (sz["rows"], cfg.hidden)),
+        C.c_size_t(sz["rows"] * cfg.hidden * 2),
         _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
         _dev(token_slot, "token_slot", torch.int32, (N, K)),
         _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
@@ -446,8 +444,10 @@ def ep_get_status(dev_status, stream=None):
 
 def ep_copy(dst, src, stream=None):
     n = src.numel() * src.element_size()
-    _check(lib.ep_copy(_bytes(dst, "dst", n), _bytes(src, "src", n), n, _stream(stream)),
-           "ep_copy")
+    (pd, nd), (ps, _) = _buf(dst, "dst"), _buf(src, "src")
+    if nd.value < n:
+        raise ValueError(f"dst holds {nd.value} bytes, needs {n}")
+    _check(lib.ep_copy(pd, ps, n, _stream(stream)), "ep_copy")
 
 
 def ep_cvt_sweep(fmt, start, out, stream=None):

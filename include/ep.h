@@ -29,6 +29,14 @@
  *     caller value ([A5] review: validate before dividing); a failed check
  *     returns an error and launches nothing.  Vector buffers (x, y, out,
  *     recv_buf, grad_buf) must be 16-byte aligned (EP_ERR_MISALIGNED).
+ *   - Every buffer whose size follows from the receive layout (workspace,
+ *     recv_buf, src_info, recv_weights, grad_buf, the expert outputs y) comes
+ *     with the number of bytes the caller allocated for it (a `*_bytes`
+ *     argument after the pointer).  A count below what the configuration
+ *     needs (ep_buffer_sizes) gives EP_ERR_BUFFER_TOO_SMALL before any launch
+ *     ([IDX] Runtime Validation: sizes are checked before GPU work).  Arrays
+ *     sized by the configuration alone (x, out, topk_idx, token_slot, ...:
+ *     [N][H], [N][K], [E] ...) carry no count.
  *   - Conditions found on the device (an expert index outside [-1, E), a
  *     slot beyond the receive capacity) never trap: the offending entry is
  *     skipped and a bit is OR-ed into *dev_status (a caller-owned uint32_t in
@@ -57,7 +65,8 @@ typedef enum {
     EP_ERR_MISALIGNED = 3,    /* a vector buffer is not 16-byte aligned */
     EP_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, copy, sync) */
     EP_ERR_DEVICE_STATUS = 5, /* ep_get_status found device-side error bits */
-    EP_ERR_TIMEOUT = 6        /* reserved for bounded waits (multi-GPU); not produced */
+    EP_ERR_TIMEOUT = 6,       /* reserved for bounded waits (multi-GPU); not produced */
+    EP_ERR_BUFFER_TOO_SMALL = 7 /* a *_bytes argument is below what the configuration needs */
 } ep_status_t;
 
 /* Quantisation of dispatched rows.  Values 2..4 equal the DeepEP-Ascend
@@ -164,7 +173,8 @@ ep_status_t ep_buffer_sizes(const ep_config_t *cfg, ep_sizes_t *out);
  *   expert_offset       int64 [E+1]: exclusive scan of recv_count rounded up to
  *                       expert_align (required for PACKED, nullable for PADDED)
  *   cumulative_recv_stats int64 [E]: += recv_count (nullable; [LL] load-balance stats)
- *   workspace           ep_sizes_t.workspace_bytes of scratch (contents undefined after)
+ *   workspace           scratch (contents undefined after) of workspace_bytes
+ *                       >= ep_sizes_t.workspace_bytes
  * Deterministic: the result never depends on thread timing.
  */
 ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const void *topk_idx,
@@ -172,7 +182,7 @@ ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const void *topk_idx,
                                uint8_t *is_token_in_rank, int32_t *token_slot,
                                int64_t *recv_count, int64_t *expert_offset,
                                int64_t *cumulative_recv_stats, void *workspace,
-                               uint32_t *dev_status, ep_stream_t stream);
+                               size_t workspace_bytes, uint32_t *dev_status, ep_stream_t stream);
 
 /*
  * Quantise each token once and scatter it to its experts' receive rows
@@ -182,16 +192,19 @@ ep_status_t ep_dispatch_layout(const ep_config_t *cfg, const void *topk_idx,
  *   topk_idx       int64 [N][K] (int32 with EP_F_IDX_I32); token_slot /
  *                  expert_offset from ep_dispatch_layout
  *   topk_weights   float [N][K] (nullable; needed for recv_weights)
- *   recv_buf       ep_sizes_t.recv_bytes: row (e, slot) holds the token's
- *                  quantised row; padded row = e*R*M + slot, packed row =
+ *   recv_buf       recv_bytes >= ep_sizes_t.recv_bytes: row (e, slot) holds the
+ *                  token's quantised row; padded row = e*R*M + slot, packed row =
  *                  expert_offset[e] + slot.  Rows without an entry are not written.
- *   src_info       int32 [rows]: r*M + t of the row's source token
- *   recv_weights   float [rows] (nullable): the entry's top-k weight
+ *   src_info       int32 [rows], src_info_bytes >= 4*rows: r*M + t of the
+ *                  row's source token
+ *   recv_weights   float [rows] (nullable; recv_weights_bytes >= 4*rows, ignored
+ *                  when NULL): the entry's top-k weight
  */
 ep_status_t ep_dispatch(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
                         const float *topk_weights, const int32_t *token_slot,
-                        const int64_t *expert_offset, void *recv_buf, int32_t *src_info,
-                        float *recv_weights, uint32_t *dev_status, ep_stream_t stream);
+                        const int64_t *expert_offset, void *recv_buf, size_t recv_bytes,
+                        int32_t *src_info, size_t src_info_bytes, float *recv_weights,
+                        size_t recv_weights_bytes, uint32_t *dev_status, ep_stream_t stream);
 
 /*
  * ep_dispatch_layout followed by ep_dispatch in one call, with the same
@@ -207,8 +220,10 @@ ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
                                     uint8_t *is_token_in_rank, int32_t *token_slot,
                                     int64_t *recv_count, int64_t *expert_offset,
                                     int64_t *cumulative_recv_stats, void *workspace,
-                                    void *recv_buf, int32_t *src_info, float *recv_weights,
-                                    uint32_t *dev_status, ep_stream_t stream);
+                                    size_t workspace_bytes, void *recv_buf, size_t recv_bytes,
+                                    int32_t *src_info, size_t src_info_bytes, float *recv_weights,
+                                    size_t recv_weights_bytes, uint32_t *dev_status,
+                                    ep_stream_t stream);
 
 /*
  * Weighted top-k combine ([LL] low_latency_combine: combined_x [T, H] bf16 is
@@ -217,17 +232,18 @@ ep_status_t ep_dispatch_with_layout(const ep_config_t *cfg, const uint16_t *x,
  *                        w[n,k] * y[row(n,k), :] )
  * accumulated in fp32 with one fused multiply-add per term.  Masked entries
  * add nothing; a token with no valid entry gets +0.  Weights are used as given.
- *   y      bf16 [rows][H] expert outputs in the receive layout; with
- *          EP_F_COMBINE_QUANTIZED (and cfg->quant != EP_Q_BF16) y is instead a
- *          buffer of ep_sizes_t.recv_bytes in cfg->quant's format (data region
+ *   y      bf16 [rows][H] expert outputs in the receive layout (y_bytes >=
+ *          ep_sizes_t.expert_out_bytes); with EP_F_COMBINE_QUANTIZED (and
+ *          cfg->quant != EP_Q_BF16) y is instead a buffer of y_bytes >=
+ *          ep_sizes_t.recv_bytes in cfg->quant's format (data region
  *          then scale region, as ep_dispatch writes it) and each expert value
  *          is decode(code) * scale as one fp32 multiply before the FMA ([FP8]
  *          The FP8 Combine Operation: codes times the stored inverse scale,
  *          in fp32).  An e8m0 scale byte of 255 (NaN) is not a valid input.
  *   out    bf16 [N][H]
  */
-ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const void *topk_idx,
-                       const float *topk_weights, const int32_t *token_slot,
+ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, size_t y_bytes,
+                       const void *topk_idx, const float *topk_weights, const int32_t *token_slot,
                        const int64_t *expert_offset, uint16_t *out, uint32_t *dev_status,
                        ep_stream_t stream);
 
@@ -238,12 +254,14 @@ ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, const void *to
  * (MXFP8(g[n,:]) with EP_F_BWD_UNWEIGHTED).  cfg->quant is ignored: the
  * gradient is always MXFP8.
  *   g          bf16 [N][H]
- *   grad_buf   ep_sizes_t.grad_bytes: e4m3 [rows][H] then e8m0 [rows][H/32]
+ *   grad_buf   grad_bytes >= ep_sizes_t.grad_bytes: e4m3 [rows][H] then e8m0
+ *              [rows][H/32]
  */
 ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
                                 const void *topk_idx, const float *topk_weights,
                                 const int32_t *token_slot, const int64_t *expert_offset,
-                                void *grad_buf, uint32_t *dev_status, ep_stream_t stream);
+                                void *grad_buf, size_t grad_bytes, uint32_t *dev_status,
+                                ep_stream_t stream);
 
 /*
  * Gradient of the combine with respect to the top-k weights (the combine is
@@ -257,11 +275,12 @@ ep_status_t ep_combine_backward(const ep_config_t *cfg, const uint16_t *g,
  * the order: within 128 * 2^-24 * sum_h |g[n,h] * y[row,h]| of the exact sum.
  *   g                  bf16 [N][H]: gradient of the combined output
  *   y                  bf16 [rows][H]: the expert outputs ep_combine read
+ *                      (y_bytes >= ep_sizes_t.expert_out_bytes)
  *   topk_weights_grad  float [N][K]
  * EP_F_COMBINE_QUANTIZED is not supported here (EP_ERR_UNSUPPORTED).
  */
 ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *g,
-                                        const uint16_t *y, const void *topk_idx,
+                                        const uint16_t *y, size_t y_bytes, const void *topk_idx,
                                         const int32_t *token_slot, const int64_t *expert_offset,
                                         float *topk_weights_grad, uint32_t *dev_status,
                                         ep_stream_t stream);
@@ -282,17 +301,19 @@ ep_status_t ep_combine_backward_weights(const ep_config_t *cfg, const uint16_t *
  * are within (H/16 + 16) * 2^-23 * sum_h |x*w| + 1 bf16 ulp of the exact sum.
  *   cfg          quant EP_Q_BF16 and layout EP_LAYOUT_PACKED (the dispatch that
  *                wrote recv_buf), H % 64 == 0; otherwise EP_ERR_UNSUPPORTED
- *   recv_buf     the dispatch's receive buffer: bf16 [rows][H]
+ *   recv_buf     the dispatch's receive buffer: bf16 [rows][H] (recv_bytes >=
+ *                rows * 2H)
  *   expert_offset, recv_count   from ep_dispatch_layout
  *   weights      bf16 [E][n_out][H] (row j of W[e] is output column j)
  *   n_out        output columns, a multiple of 256
- *   y            bf16 [rows][n_out] (n_out = H gives ep_combine's input)
+ *   y            bf16 [rows][n_out] (y_bytes >= rows * n_out * 2; n_out = H
+ *                gives ep_combine's input)
  * A wait inside the kernel that exceeds 2 s sets EP_DEV_TIMEOUT and the
  * kernel returns; it never traps.
  */
-ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
+ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf, size_t recv_bytes,
                            const int64_t *expert_offset, const int64_t *recv_count,
-                           const uint16_t *weights, int32_t n_out, uint16_t *y,
+                           const uint16_t *weights, int32_t n_out, uint16_t *y, size_t y_bytes,
                            uint32_t *dev_status, ep_stream_t stream);
 
 /*
@@ -312,9 +333,9 @@ ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
  *   cfg          quant EP_Q_MXFP8 (H % 128 == 0) or EP_Q_MXFP4 (H % 256 == 0) and
  *                layout EP_LAYOUT_PACKED (the dispatch that wrote recv_buf);
  *                otherwise EP_ERR_UNSUPPORTED
- *   recv_buf     the dispatch's receive buffer: codes [rows][D] (D = H, or H/2
- *                for MXFP4), then at ep_sizes_t.recv_scale_offset e8m0
- *                [rows][H/32]
+ *   recv_buf     the dispatch's receive buffer (recv_bytes >= ep_sizes_t.recv_bytes):
+ *                codes [rows][D] (D = H, or H/2 for MXFP4), then at
+ *                ep_sizes_t.recv_scale_offset e8m0 [rows][H/32]
  *   expert_offset, recv_count   from ep_dispatch_layout
  *   w_codes      [E][n_out][D] in cfg's code format (row j of W[e] is output
  *                column j)
@@ -322,15 +343,17 @@ ep_status_t ep_expert_gemm(const ep_config_t *cfg, const void *recv_buf,
  *   n_out        output columns, a multiple of 224, 256 or 128 (tiles of 224
  *                columns where they divide n_out, else 256, else 128; MXFP8
  *                with at least 256 entries an expert on average takes 256)
- *   y            bf16 [rows][n_out] (n_out = H gives ep_combine's input)
+ *   y            bf16 [rows][n_out] (y_bytes >= rows * n_out * 2; n_out = H
+ *                gives ep_combine's input)
  * recv_buf, w_codes, w_scales and y 16-byte aligned (EP_ERR_MISALIGNED).
  * A wait inside the kernel that exceeds 2 s sets EP_DEV_TIMEOUT and the
  * kernel returns; it never traps.
  */
-ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
+ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf, size_t recv_bytes,
                               const int64_t *expert_offset, const int64_t *recv_count,
                               const uint8_t *w_codes, const uint8_t *w_scales, int32_t n_out,
-                              uint16_t *y, uint32_t *dev_status, ep_stream_t stream);
+                              uint16_t *y, size_t y_bytes, uint32_t *dev_status,
+                              ep_stream_t stream);
 
 /*
  * One call for the whole forward path with the experts between dispatch and
@@ -348,18 +371,20 @@ ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf,
  *   x, topk_idx, topk_weights    as ep_dispatch / ep_combine
  *   w_codes      bf16 [E][H][H] (w_scales NULL) or the MX codes [E][H][D]
  *   w_scales     e8m0 [E][H][H/32] for the MX formats
- *   token_slot, recv_count, expert_offset, workspace   as ep_dispatch_layout
- *   recv_buf, src_info           as ep_dispatch
- *   y            bf16 [rows][H]: the experts' outputs (scratch owned by the caller)
+ *   token_slot, recv_count, expert_offset, workspace(_bytes)   as ep_dispatch_layout
+ *   recv_buf(_bytes), src_info(_bytes)                          as ep_dispatch
+ *   y            bf16 [rows][H]: the experts' outputs (scratch owned by the
+ *                caller; y_bytes >= ep_sizes_t.expert_out_bytes)
  *   out          bf16 [N][H]
  * A wait inside the GEMM kernel that exceeds 2 s sets EP_DEV_TIMEOUT.
  */
 ep_status_t ep_moe_forward(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
                            const float *topk_weights, const void *w_codes,
                            const uint8_t *w_scales, int32_t *token_slot, int64_t *recv_count,
-                           int64_t *expert_offset, void *workspace, void *recv_buf,
-                           int32_t *src_info, uint16_t *y, uint16_t *out, uint32_t *dev_status,
-                           ep_stream_t stream);
+                           int64_t *expert_offset, void *workspace, size_t workspace_bytes,
+                           void *recv_buf, size_t recv_bytes, int32_t *src_info,
+                           size_t src_info_bytes, uint16_t *y, size_t y_bytes, uint16_t *out,
+                           uint32_t *dev_status, ep_stream_t stream);
 
 /*
  * Diagnostic of the bounded waits in the tensor-core kernels (ep_expert_gemm,
@@ -393,6 +418,12 @@ ep_status_t ep_wait_probe(uint32_t *dev_status, ep_stream_t stream);
  *     to start at zero; but calls that overlap on the GPU (different streams,
  *     or several host threads) race on the array: serialise them.
  *   - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ *     The array itself comes into being when CUDA loads this library's
+ *     device code on a device, which under CUDA's default lazy loading is
+ *     the first call into the library there.  A caller that reserves the
+ *     whole device up front should make one call into the library per device
+ *     first (for example this call on a tiny configuration), so that the
+ *     array already exists when memory runs out.
  */
 #define EP_STATIC_SCRATCH_BYTES (1u << 20)
 ep_status_t ep_dispatch_layout_static(const ep_config_t *cfg, const void *topk_idx,

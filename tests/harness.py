@@ -20,6 +20,55 @@ def to_np_u16(t):
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
 
 
+GUARD_BYTES = 4096
+GUARD_FILL = 0x5C
+BUFFER_FIELDS = ("tokens_per_rank", "tokens_per_expert", "is_token_in_rank", "token_slot",
+                 "recv_count", "expert_offset", "workspace", "recv_buf", "src_info",
+                 "recv_weights", "y", "out", "grad_buf", "dev_status")
+
+
+class Guards:
+    """Guard bands around the device buffers a test hands to the library (the
+    stand-in for a memory checker): each buffer is carved out of a larger
+    allocation with GUARD_BYTES of a fill pattern on both sides (plus the
+    rounding up to 16 bytes after it); check() asserts that no kernel wrote
+    into a band.  The byte count each buffer reports is its own, so the
+    library's size checks see the exact size."""
+
+    def __init__(self):
+        self.items = []
+
+    def alloc(self, shape, dtype, name):
+        nbytes = int(np.prod(shape, dtype=np.int64)) * torch.empty((), dtype=dtype).element_size()
+        span = (nbytes + 15) // 16 * 16
+        base = torch.full((2 * GUARD_BYTES + span,), GUARD_FILL, dtype=torch.uint8,
+                          device="cuda")
+        self.items.append((name, base, nbytes))
+        return base[GUARD_BYTES:GUARD_BYTES + nbytes].view(dtype).view(shape)
+
+    def like(self, t, name):
+        g = self.alloc(tuple(t.shape), t.dtype, name)
+        g.copy_(t)
+        return g
+
+    def wrap(self, buffers):
+        """Replace every buffer of an ep.Buffers with a guarded copy."""
+        for f in BUFFER_FIELDS:
+            t = getattr(buffers, f, None)
+            if isinstance(t, torch.Tensor):
+                setattr(buffers, f, self.like(t, f))
+        torch.cuda.empty_cache()
+        return buffers
+
+    def check(self):
+        torch.cuda.synchronize()
+        for name, base, nbytes in self.items:
+            lo = base[:GUARD_BYTES]
+            hi = base[GUARD_BYTES + nbytes:]
+            assert bool((lo == GUARD_FILL).all()), f"write below {name}"
+            assert bool((hi == GUARD_FILL).all()), f"write past the end of {name}"
+
+
 def oracle_mode(mode, flags):
     """The oracle's name for a quantisation mode with its scale flags."""
     if mode == "e4m3_b128" and flags & ep.F_UE8M0:
@@ -50,7 +99,8 @@ class Run:
                                   flags | (ep.F_BWD_UNWEIGHTED if bwd_unweighted else 0))
         self.bwd_unweighted = bwd_unweighted
         self.omode = oracle_mode(mode, flags)
-        b = ep.Buffers(self.cfg, recv_weights=with_weights, grad=backward)
+        self.guards = Guards()
+        b = self.guards.wrap(ep.Buffers(self.cfg, recv_weights=with_weights, grad=backward))
         self.b = b
         b.recv_buf.fill_(fill)
         if b.recv_weights is not None:
@@ -92,6 +142,7 @@ class Run:
 
     # ---- comparisons ----------------------------------------------------------
     def check_layout(self):
+        self.guards.check()
         b, o = self.b, self.lay
         assert np.array_equal(b.token_slot.cpu().numpy(), o["token_slot"])
         assert np.array_equal(b.recv_count.cpu().numpy(), o["recv_count"])
@@ -119,6 +170,7 @@ class Run:
         return ns, ks, rows
 
     def check_dispatch(self, tokens=None, check_unwritten=True):
+        self.guards.check()
         w, b = self.w, self.b
         ns, ks, rows = self.entries(tokens)
         rows_d = torch.from_numpy(rows).cuda()
@@ -156,6 +208,7 @@ class Run:
         return synth.windows(self.y_pool, self.y_off[np.asarray(rows, np.int64)], self.w["H"])
 
     def check_combine(self, tokens=None, max_ulp=1):
+        self.guards.check()
         w, b = self.w, self.b
         K, H = w["K"], w["H"]
         tokens = np.arange(self.idx.shape[0]) if tokens is None else np.asarray(tokens)
@@ -188,10 +241,12 @@ class Run:
             gp, go = synth.g_source(w)
             g = synth.windows(gp, go, H)
         g_d = bf16_dev(g)
-        dw = torch.full((w["N"], K), float("nan"), dtype=torch.float32, device="cuda")
+        dw = self.guards.alloc((w["N"], K), torch.float32, "topk_weights_grad")
+        dw.fill_(float("nan"))
         ep.ep_combine_backward_weights(self.cfg, g_d, b.y, self.idx_d, b.token_slot, dw,
                                        b.dev_status, expert_offset=b.expert_offset)
         assert ep.ep_get_status(b.dev_status) == self.status
+        self.guards.check()
         tokens = np.arange(w["N"]) if tokens is None else np.asarray(tokens)
         got = dw.cpu().numpy()[tokens]
         worst = 0.0
@@ -215,6 +270,7 @@ class Run:
         return worst
 
     def check_backward(self, tokens=None):
+        self.guards.check()
         w, b = self.w, self.b
         H = w["H"]
         ns, ks, rows = self.entries(tokens)
@@ -298,10 +354,12 @@ def combine_quantized_check(run, tokens=None, seed=0, rows_fn=None):
     if S:
         a = sz["recv_scale_offset"]
         yq[a: a + sz["rows"] * S].view(sz["rows"], S).index_copy_(0, rows_d, torch.from_numpy(scale).cuda())
-    out = torch.full((w["N"], H), 1.0, dtype=torch.bfloat16, device="cuda")
+    out = run.guards.alloc((w["N"], H), torch.bfloat16, "out (quantised combine)")
+    out.fill_(1.0)
     ep.ep_combine(cfg, yq, run.idx_d, run.wts_d,
                   b.token_slot, out, b.dev_status, expert_offset=b.expert_offset)
     assert ep.ep_get_status(b.dev_status) == run.status
+    run.guards.check()
     tokens = np.arange(w["N"]) if tokens is None else np.asarray(tokens)
     got = to_np_u16(out)[tokens]
     where = {(int(n), int(k)): i for i, (n, k) in enumerate(zip(ns, ks))}

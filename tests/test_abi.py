@@ -106,23 +106,26 @@ def test_entry_points_reject_before_any_launch():
     these calls reach no CUDA API (there is no device here)."""
     cfg = _cfg()
     null = C.c_void_p(0)
+    z = C.c_size_t(0)
     n0 = ep.ep_kernel_launches()
-    assert lib.ep_dispatch_layout(None, *([null] * 11)) == 1
-    assert lib.ep_dispatch_layout(C.byref(cfg), *([null] * 11)) == 1
-    assert lib.ep_dispatch(C.byref(cfg), *([null] * 10)) == 1
-    assert lib.ep_combine(C.byref(cfg), *([null] * 8)) == 1
-    assert lib.ep_combine_backward(C.byref(cfg), *([null] * 8)) == 1
-    assert lib.ep_combine_backward_weights(C.byref(cfg), *([null] * 8)) == 1
+    assert lib.ep_dispatch_layout(None, *([null] * 9), z, null, null) == 1
+    assert lib.ep_dispatch_layout(C.byref(cfg), *([null] * 9), z, null, null) == 1
+    assert lib.ep_dispatch(C.byref(cfg), *([null] * 6), z, null, z, null, z, null, null) == 1
+    assert lib.ep_combine(C.byref(cfg), null, z, *([null] * 7)) == 1
+    assert lib.ep_combine_backward(C.byref(cfg), *([null] * 6), z, null, null) == 1
+    assert lib.ep_combine_backward_weights(C.byref(cfg), null, null, z, *([null] * 6)) == 1
     qcfg = _cfg(quant="mxfp8", flags=ep.F_COMBINE_QUANTIZED)
-    assert lib.ep_combine_backward_weights(C.byref(qcfg), *([C.c_void_p(0x1000)] * 7), null) == 2
+    fake = C.c_void_p(0x1000)
+    assert lib.ep_combine_backward_weights(C.byref(qcfg), fake, fake, z, *([fake] * 5), null) == 2
     assert lib.ep_get_status(null, None, null) == 1
     bad = _cfg(E=255)
-    fake = C.c_void_p(0x1000)
-    assert lib.ep_dispatch(C.byref(bad), *([fake] * 9), null) == 1
+    big = C.c_size_t(1 << 40)
+    assert lib.ep_dispatch(C.byref(bad), *([fake] * 6), big, fake, big, fake, big, fake,
+                           null) == 1
     # misaligned vector buffers
     odd = C.c_void_p(0x1008)
-    args = [odd, fake, fake, fake, fake, fake, fake, fake, fake, null]
-    assert lib.ep_dispatch(C.byref(cfg), *args) == 3
+    assert lib.ep_dispatch(C.byref(cfg), odd, *([fake] * 5), big, fake, big, fake, big, fake,
+                           null) == 3
     assert lib.ep_copy(fake, fake, 24, null) == 1
     assert lib.ep_copy(odd, fake, 32, null) == 3
     assert lib.ep_cvt_sweep(4, 0, 16, fake, null) == 1
@@ -130,8 +133,88 @@ def test_entry_points_reject_before_any_launch():
     assert ep.ep_kernel_launches() == n0
 
 
+# ---------------------------------------------------------------------------
+# buffer sizes stated by a C caller: one byte short -> EP_ERR_BUFFER_TOO_SMALL
+# before any launch ("DeepEP topk_idx_t Custom Dtype Requirements", Runtime
+# Validation: checks come before GPU work)
+# ---------------------------------------------------------------------------
+_F = C.c_void_p(0x10000)   # a non-null, 16-byte aligned pointer that is never dereferenced
+_N = C.c_void_p(0)
+
+
+def _short_calls():
+    """(name, which buffer, call(sizes) -> status) for every sized buffer of every
+    entry point; `sizes` maps buffer -> byte count."""
+    pad = _cfg(R=4, T=16, M=16, K=4, E=16, H=1024, quant="mxfp8")
+    pk = _cfg(R=4, T=16, M=16, K=4, E=16, H=1024, quant="mxfp8", layout="packed")
+    pkq = _cfg(R=4, T=16, M=16, K=4, E=16, H=1024, quant="mxfp8", layout="packed",
+               flags=ep.F_COMBINE_QUANTIZED)
+    bfp = _cfg(R=4, T=16, M=16, K=4, E=16, H=1024, quant="bf16", layout="packed")
+    Z = C.c_size_t
+    out = []
+
+    def add(name, cfg, need, fn):
+        out.append((name, cfg, need, fn))
+    for cfg in (pad, pk):
+        s = ep.ep_buffer_sizes(cfg)
+        add("ep_dispatch_layout", cfg, {"workspace": s["workspace_bytes"]},
+            lambda c, z: lib.ep_dispatch_layout(C.byref(c), _F, _F, _F, _F, _F, _F, _F, _N, _F,
+                                                Z(z["workspace"]), _F, _N))
+        need = {"recv_buf": s["recv_bytes"], "src_info": s["src_info_bytes"],
+                "recv_weights": s["recv_weights_bytes"]}
+        add("ep_dispatch", cfg, need,
+            lambda c, z: lib.ep_dispatch(C.byref(c), _F, _F, _F, _F, _F, _F, Z(z["recv_buf"]), _F,
+                                         Z(z["src_info"]), _F, Z(z["recv_weights"]), _F, _N))
+        add("ep_dispatch_with_layout", cfg, dict(need, workspace=s["workspace_bytes"]),
+            lambda c, z: lib.ep_dispatch_with_layout(
+                C.byref(c), _F, _F, _F, _F, _F, _F, _F, _F, _F, _N, _F, Z(z["workspace"]), _F,
+                Z(z["recv_buf"]), _F, Z(z["src_info"]), _F, Z(z["recv_weights"]), _F, _N))
+        add("ep_combine", cfg, {"y": s["expert_out_bytes"]},
+            lambda c, z: lib.ep_combine(C.byref(c), _F, Z(z["y"]), _F, _F, _F, _F, _F, _F, _N))
+        add("ep_combine_backward", cfg, {"grad_buf": s["grad_bytes"]},
+            lambda c, z: lib.ep_combine_backward(C.byref(c), _F, _F, _F, _F, _F, _F,
+                                                 Z(z["grad_buf"]), _F, _N))
+        add("ep_combine_backward_weights", cfg, {"y": s["expert_out_bytes"]},
+            lambda c, z: lib.ep_combine_backward_weights(C.byref(c), _F, _F, Z(z["y"]), _F, _F,
+                                                         _F, _F, _F, _N))
+    s = ep.ep_buffer_sizes(pkq)
+    add("ep_combine (quantised y)", pkq, {"y": s["recv_bytes"]},
+        lambda c, z: lib.ep_combine(C.byref(c), _F, Z(z["y"]), _F, _F, _F, _F, _F, _F, _N))
+    s = ep.ep_buffer_sizes(bfp)
+    rows = s["rows"]
+    add("ep_expert_gemm", bfp, {"recv_buf": rows * 2048, "y": rows * 512 * 2},
+        lambda c, z: lib.ep_expert_gemm(C.byref(c), _F, Z(z["recv_buf"]), _F, _F, _F, 512, _F,
+                                        Z(z["y"]), _F, _N))
+    add("ep_moe_forward", bfp, {"workspace": s["workspace_bytes"], "recv_buf": s["recv_bytes"],
+                                "src_info": s["src_info_bytes"], "y": s["expert_out_bytes"]},
+        lambda c, z: lib.ep_moe_forward(C.byref(c), _F, _F, _F, _F, _N, _F, _F, _F, _F,
+                                        Z(z["workspace"]), _F, Z(z["recv_buf"]), _F,
+                                        Z(z["src_info"]), _F, Z(z["y"]), _F, _F, _N))
+    s = ep.ep_buffer_sizes(pk)
+    rows = s["rows"]
+    add("ep_expert_gemm_mx", pk, {"recv_buf": s["recv_bytes"], "y": rows * 224 * 2},
+        lambda c, z: lib.ep_expert_gemm_mx(C.byref(c), _F, Z(z["recv_buf"]), _F, _F, _F, _F, 224,
+                                           _F, Z(z["y"]), _F, _N))
+    return out
+
+
+_CASES = [(name, cfg, need, fn, buf) for name, cfg, need, fn in _short_calls() for buf in need]
+
+
+@pytest.mark.parametrize("case", _CASES,
+                         ids=[f"{c[0]}-{'padded' if c[1].layout == 0 else 'packed'}-{c[4]}"
+                              for c in _CASES])
+def test_one_byte_short_buffer_is_refused_before_any_launch(case):
+    name, cfg, need, fn, buf = case
+    sizes = dict(need)
+    sizes[buf] = need[buf] - 1
+    n0 = ep.ep_kernel_launches()
+    assert fn(cfg, sizes) == ep.ERR_BUFFER_TOO_SMALL, (name, buf)
+    assert ep.ep_kernel_launches() == n0
+
+
 def test_status_strings():
-    for s in range(7):
+    for s in range(8):
         assert lib.ep_status_string(s)
     assert b"unknown" in lib.ep_status_string(99)
 

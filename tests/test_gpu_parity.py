@@ -16,7 +16,7 @@ import torch
 import combine_ep_dispatch_04_b200 as ep
 import oracle
 import synth
-from harness import Run, bf16_dev, to_np_u16, ulp_distance
+from harness import Guards, Run, bf16_dev, to_np_u16, ulp_distance
 
 pytestmark = pytest.mark.gpu
 
@@ -705,7 +705,7 @@ def _check_expert_gemm(r, y, n_out, W=None, wc=None, ws=None, sample_rows=None):
 
 
 def _sentinel_y(r, n_out):
-    y = torch.empty((r.sizes["rows"], n_out), dtype=torch.bfloat16, device="cuda")
+    y = r.guards.alloc((r.sizes["rows"], n_out), torch.bfloat16, "y (expert outputs)")
     y.view(torch.int16).fill_(0x7777)
     return y
 
@@ -1015,10 +1015,12 @@ def test_moe_forward_equals_the_calls_one_by_one(mode):
     H = w["H"]
     outs = []
     for one_call in (True, False):
-        b = ep.Buffers(cfg)
+        guards = Guards()
+        b = guards.wrap(ep.Buffers(cfg))
         b.recv_buf.fill_(0xAB)
-        y = torch.empty((b.sizes["rows"], H), dtype=torch.bfloat16, device="cuda")
-        out = torch.full((w["N"], H), 7.0, dtype=torch.bfloat16, device="cuda")
+        y = guards.alloc((b.sizes["rows"], H), torch.bfloat16, "y")
+        out = guards.alloc((w["N"], H), torch.bfloat16, "out")
+        out.fill_(7.0)
         if one_call:
             n0 = ep.ep_kernel_launches()
             ep.ep_moe_forward(cfg, x_d, idx_d, wts_d, wc, ws, b.token_slot, b.recv_count,
@@ -1040,6 +1042,7 @@ def test_moe_forward_equals_the_calls_one_by_one(mode):
                           expert_offset=b.expert_offset)
             out = b.out
         assert ep.ep_get_status(b.dev_status) == 0
+        guards.check()
         outs.append(to_np_u16(out))
     assert np.array_equal(outs[0], outs[1])
 

@@ -9,7 +9,11 @@ libep.so instead.  The test calls it through the C ABI twice in a row, on two
 different routings so that the second call starts from the first call's
 leftover scratch, and checks every output against the regular
 ep_dispatch_layout (integer outputs: bit-exact).  It runs the same alone in
-a fresh process or after the rest of the suite.
+a fresh process or after the rest of the suite.  The static array comes into
+being when CUDA loads the library's device code on the device (lazily, at
+the first call into the library there); a caller that reserves the whole
+device up front makes one such call first, which is what the first case
+here is in a fresh process.
 """
 import numpy as np
 import pytest
