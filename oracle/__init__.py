@@ -76,6 +76,8 @@ _lib.orc_expert_gemm_mx.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p]
 _lib.orc_expert_gemm_mxfp4.restype = None
 _lib.orc_expert_gemm_mxfp4.argtypes = [_i, _i, _i, _p, _p, _p, _p, _p, _p, _p]
 _lib.orc_bwd_row.restype = None
+_lib.orc_expert_ffn_mx.restype = None
+_lib.orc_expert_ffn_mx.argtypes = [_i, _i, _i] + [_p] * 13
 _lib.orc_bwd_row.argtypes = [_i, _f, _i, _p, _p, _p]
 _lib.orc_combine_gathered.restype = None
 _lib.orc_combine_gathered.argtypes = [_l, _i, _i, _p, _p, _p, _p]
@@ -377,6 +379,30 @@ def expert_gemm_mx(xc, xs, wc, ws, expert_offset, count, n_out, y=None):
     _lib.orc_expert_gemm_mx(E, H, n_out, _ptr(eo), _ptr(cnt), _ptr(xc), _ptr(xs), _ptr(wc),
                             _ptr(ws), _ptr(y))
     return y
+
+
+def expert_ffn_mx(xc, xs, w1c, w1s, w2c, w2s, expert_offset, count):
+    """The experts' gated MLP on MXFP8 operands: GMM1 (h = x . W1^T, fp32),
+    SwiGLU (z = silu(gate) * up, gate = h[:, :I], up = h[:, I:]), MXFP8 requant
+    of z, GMM2 (y = zq . W2^T, bf16).  xc [rows, H] e4m3 codes, xs [rows, H/32];
+    w1c [E, 2I, H], w1s [E, 2I, H/32]; w2c [E, H, I], w2s [E, H, I/32].
+    Returns dict(h [rows, 2I] f32, z [rows, I] f32, zc [rows, I] u8,
+    zs [rows, I/32] u8, y [rows, H] bf16 bits); rows outside every expert stay 0."""
+    xc, xs = _c(xc, np.uint8), _c(xs, np.uint8)
+    w1c, w1s, w2c, w2s = (_c(a, np.uint8) for a in (w1c, w1s, w2c, w2s))
+    rows, H = xc.shape
+    E, N1 = w1c.shape[0], w1c.shape[1]
+    I = N1 // 2
+    assert xs.shape == (rows, H // 32) and w1c.shape == (E, N1, H) and w1s.shape == (E, N1, H // 32)
+    assert w2c.shape == (E, H, I) and w2s.shape == (E, H, I // 32) and I % 32 == 0
+    eo, cnt = _c(expert_offset, np.int64), _c(count, np.int64)
+    out = dict(h=np.zeros((rows, N1), np.float32), z=np.zeros((rows, I), np.float32),
+               zc=np.zeros((rows, I), np.uint8), zs=np.zeros((rows, I // 32), np.uint8),
+               y=np.zeros((rows, H), np.uint16))
+    _lib.orc_expert_ffn_mx(E, H, I, _ptr(eo), _ptr(cnt), _ptr(xc), _ptr(xs), _ptr(w1c), _ptr(w1s),
+                           _ptr(w2c), _ptr(w2s), _ptr(out["h"]), _ptr(out["z"]), _ptr(out["zc"]),
+                           _ptr(out["zs"]), _ptr(out["y"]))
+    return out
 
 
 def expert_gemm_mxfp4(xc, xs, wc, ws, expert_offset, count, n_out, y=None):

@@ -686,6 +686,74 @@ void orc_expert_gemm_mxfp4(int E, int H, int Nout, const int64_t *expert_offset,
 }
 
 /*
+ * The experts' gated two-layer MLP on MXFP8 operands ("[feat] A5 deep fused
+ * moe supported": Testing, the per-stage table -- Dispatch, GMM1, SwiGLU,
+ * Requant, GMM2, Combine; Benchmarking and Profiling -- hidden 7168,
+ * moe-intermediate-size 3072, FP8 quantisation; its review notes that the
+ * GMM1 operands are e4m3 codes with one e8m0 scale per 32 elements).
+ * I is the intermediate size.  For each expert e and each of its rows r
+ * (expert_offset[e] .. + count[e]):
+ *   GMM1     h[j] = fl32( sum_k x[r,k] * W1[e][j,k] ),   j < 2I
+ *            (exact products, summed in double in k order, one rounding)
+ *   SwiGLU   z[j] = fl32( silu(h[j]) * h[I + j] ),        j < I
+ *            silu(a) = a / (1 + exp(-a)), evaluated in double from the fp32
+ *            h; the first I outputs of GMM1 are the gate, the last I the up
+ *            projection
+ *   Requant  the row z[0..I) quantised to MXFP8 exactly as the MX dispatch
+ *            quantises a token (orc_quant_row_f32, one e8m0 scale per 32)
+ *   GMM2     y[r, j] = bf16( fl32( sum_i zq[i] * W2[e][j,i] ) ),  j < H
+ *            (the MXFP8 maps above with the intermediate size as depth)
+ * W1 codes [E][2I][H] with e8m0 scales [E][2I][H/32]; W2 codes [E][H][I]
+ * with scales [E][H][I/32].  Outputs per row: h_out (fp32 [rows][2I],
+ * nullable), z_out (fp32 [rows][I], nullable), zc / zs (the requantised
+ * codes [rows][I] and scales [rows][I/32]) and y (bf16 [rows][H]); rows past
+ * count[e] are left untouched.
+ */
+void orc_expert_ffn_mx(int E, int H, int I, const int64_t *expert_offset, const int64_t *count,
+                       const uint8_t *xc, const uint8_t *xs, const uint8_t *w1c,
+                       const uint8_t *w1s, const uint8_t *w2c, const uint8_t *w2s, float *h_out,
+                       float *z_out, uint8_t *zc, uint8_t *zs, uint16_t *y)
+{
+    const int SH = H / 32, SI = I / 32, N1 = 2 * I;
+    float *h = (float *)malloc(sizeof(float) * (size_t)N1);
+    float *z = (float *)malloc(sizeof(float) * (size_t)I);
+    for (int e = 0; e < E; e++) {
+        for (int64_t i = 0; i < count[e]; i++) {
+            const int64_t r = expert_offset[e] + i;
+            for (int j = 0; j < N1; j++) { /* GMM1 */
+                const int64_t wrow = (int64_t)e * N1 + j;
+                double acc = 0.0;
+                for (int k = 0; k < H; k++) {
+                    double xv = (double)orc_e4m3_decode(xc[r * H + k]) * orc_e8m0_value(xs[r * SH + k / 32]);
+                    double wv = (double)orc_e4m3_decode(w1c[wrow * H + k]) * orc_e8m0_value(w1s[wrow * SH + k / 32]);
+                    acc += xv * wv;
+                }
+                h[j] = (float)acc;
+            }
+            for (int j = 0; j < I; j++) { /* SwiGLU */
+                const double g = (double)h[j], u = (double)h[I + j];
+                z[j] = (float)(g / (1.0 + exp(-g)) * u);
+            }
+            orc_quant_row_f32(ORC_MXFP8, I, 0.0f, z, zc + r * I, zs + r * SI); /* Requant */
+            for (int j = 0; j < H; j++) { /* GMM2 */
+                const int64_t wrow = (int64_t)e * H + j;
+                double acc = 0.0;
+                for (int k = 0; k < I; k++) {
+                    double zv = (double)orc_e4m3_decode(zc[r * I + k]) * orc_e8m0_value(zs[r * SI + k / 32]);
+                    double wv = (double)orc_e4m3_decode(w2c[wrow * I + k]) * orc_e8m0_value(w2s[wrow * SI + k / 32]);
+                    acc += zv * wv;
+                }
+                y[r * H + j] = orc_f32_to_bf16((float)acc);
+            }
+            if (h_out) memcpy(h_out + r * N1, h, sizeof(float) * (size_t)N1);
+            if (z_out) memcpy(z_out + r * I, z, sizeof(float) * (size_t)I);
+        }
+    }
+    free(h);
+    free(z);
+}
+
+/*
  * Dequantisation of one row stored in a quantised format ([FP8] The FP8
  * Combine Operation: the received codes times the stored inverse scale, in
  * fp32).  Each element is decode(code) * scale_inv as

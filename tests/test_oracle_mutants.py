@@ -76,6 +76,19 @@ MUTANTS = {
           "            } else {\n                scale[b] = (uint8_t)(X + 128);")], "ue8m0"),
     "NaN wins the block maximum": (
         [("        if (v > a) a = v;", "        if (!(v <= a)) a = v;")], "nan"),
+    "SwiGLU gate and up halves swapped": (
+        [("const double g = (double)h[j], u = (double)h[I + j];",
+          "const double g = (double)h[I + j], u = (double)h[j];")], "ffn"),
+    "silu with exp of +a": (
+        [("z[j] = (float)(g / (1.0 + exp(-g)) * u);", "z[j] = (float)(g / (1.0 + exp(g)) * u);")],
+        "ffn"),
+    "GMM2 reads the intermediate scale of the first block only": (
+        [("double zv = (double)orc_e4m3_decode(zc[r * I + k]) * orc_e8m0_value(zs[r * SI + k / 32]);",
+          "double zv = (double)orc_e4m3_decode(zc[r * I + k]) * orc_e8m0_value(zs[r * SI]);")],
+        "ffn"),
+    "GMM1 gate rows of expert 0 for every expert": (
+        [("const int64_t wrow = (int64_t)e * N1 + j;", "const int64_t wrow = (int64_t)0 * N1 + j;")],
+        "ffn"),
     "e4m3 NaN code decodes to 480": (
         [("if (e == 15 && m == 7) return NAN;", "if (e == 15 && m == 7) return 480.0f;")],
         "decoders"),

@@ -1033,3 +1033,173 @@ def test_expert_gemm_mxfp4_equals_bf16_maps_on_dequantised_operands():
     want = oracle.expert_gemm(xb, wb, eo, cnt, N)
     got = oracle.expert_gemm_mxfp4(xc, xs, wc, ws, eo, cnt, N)
     assert np.array_equal(got, want)
+
+
+# ---------------------------------------------------------------------------
+# the experts' gated MLP: GMM1 -> SwiGLU -> MXFP8 requant -> GMM2
+# ---------------------------------------------------------------------------
+# e to 60 digits (a textbook constant, so that no value below comes from a
+# library exp routine)
+_E_DIGITS = "2.718281828459045235360287471352662497757247093699959574966967"
+
+
+def _silu_exact(a):
+    """silu(a) = a / (1 + e^-a) for an integer or half-integer a, in 50-digit
+    decimal arithmetic from the digits of e."""
+    from decimal import Decimal, getcontext
+    getcontext().prec = 50
+    e = Decimal(_E_DIGITS)
+    two_a = int(round(2 * a))
+    assert two_a == 2 * a
+    root = e.sqrt()                       # e^(1/2)
+    p = root ** abs(two_a)                # e^|a|
+    ema = (1 / p) if a > 0 else p         # e^-a
+    return Decimal(two_a) / 2 / (1 + ema)
+
+
+def _ffn_case(E, H, I, rows_per_e, gate_vals, up_vals, seed=0):
+    """Operands whose GMM1 outputs are set by hand: every row's codes are 1.0
+    at one position (scale 2^0), W1's gate row j of expert e holds gate_vals
+    at that position and W1's up row j holds up_vals; W2 holds small integers."""
+    enc = oracle.e4m3_encode
+    rows = E * rows_per_e
+    xc = np.zeros((rows, H), np.uint8)
+    xc[:, 0] = enc(np.float32([1.0]))[0]
+    xs = np.full((rows, H // 32), 127, np.uint8)
+    w1c = np.zeros((E, 2 * I, H), np.uint8)
+    w1c[:, :I, 0] = enc(np.asarray(gate_vals, np.float32))
+    w1c[:, I:, 0] = enc(np.asarray(up_vals, np.float32))
+    w1s = np.full((E, 2 * I, H // 32), 127, np.uint8)
+    r = np.random.default_rng(seed)
+    w2c = enc(r.integers(-3, 4, (E, H, I)).astype(np.float32))
+    w2s = np.full((E, H, I // 32), 127, np.uint8)
+    eo = np.arange(E, dtype=np.int64) * rows_per_e
+    cnt = np.full(E, rows_per_e, np.int64)
+    return xc, xs, w1c, w1s, w2c, w2s, eo, cnt
+
+
+def _f32_ulp(v):
+    return np.spacing(np.abs(np.float32(v)))
+
+
+def test_ffn_silu_matches_the_constant_e_and_the_gate_up_order():
+    """z = silu(gate) * up with gate the first I outputs of GMM1: each z is
+    within one fp32 ulp of the 50-digit value; with the halves swapped the
+    values would be silu(up) * gate, which differ."""
+    from decimal import Decimal
+    gates = [1.0, -1.0, 2.0, -2.0, 0.5, -0.5, 3.0, 4.0] * 4
+    ups = [3.0, 3.0, 1.0, 1.0, 1.0, -2.0, 0.5, -1.0] * 4
+    case = _ffn_case(1, 64, 32, 2, gates, ups)
+    o = oracle.expert_ffn_mx(*case)
+    for j in range(32):
+        want = float(_silu_exact(gates[j]) * Decimal(ups[j]))
+        got = float(o["z"][0, j])
+        assert abs(got - want) <= _f32_ulp(want), (j, got, want)
+    swapped = float(_silu_exact(ups[0]) * Decimal(gates[0]))
+    assert abs(float(o["z"][0, 0]) - swapped) > 0.5
+
+
+def test_ffn_silu_identities():
+    """silu(0) = 0; silu(a) - silu(-a) = a; silu(a) = a for a large gate."""
+    gates = [0.0, 5.0, -5.0, 7.0, -7.0, 448.0, 0.0, 1.5] * 4
+    ups = [9.0, 1.0, 1.0, 1.0, 1.0, 3.0, -6.0, 1.0] * 4
+    o = oracle.expert_ffn_mx(*_ffn_case(1, 64, 32, 1, gates, ups))
+    z = o["z"][0].astype(np.float64)
+    assert z[0] == 0.0 and z[6] == 0.0
+    assert abs((z[1] - z[2]) - 5.0) <= 2 * _f32_ulp(5.0)
+    assert abs((z[3] - z[4]) - 7.0) <= 2 * _f32_ulp(7.0)
+    assert z[5] == 448.0 * 3.0                      # e^-448 is far below half an ulp
+
+
+def test_ffn_zero_gate_gives_zero_codes_and_unit_scale():
+    o = oracle.expert_ffn_mx(*_ffn_case(2, 64, 64, 3, [0.0] * 64, [5.0] * 64))
+    assert np.all(o["z"] == 0) and np.all(o["zc"] == 0) and np.all(o["zs"] == 127)
+    assert np.all(o["y"] == 0)
+
+
+def _mxfp8_by_search(z):
+    """MXFP8 of one fp32 row by brute force: per 32 elements the smallest
+    power of two 2^X (X in [-127, 127]) with amax/448 <= 2^X, found by search,
+    and the nearest e4m3 code of z * 2^-X (ties to the even code)."""
+    z = np.asarray(z, np.float32)
+    table = _e4m3_table()
+    codes = np.empty(z.size, np.uint8)
+    scales = np.empty(z.size // 32, np.uint8)
+    for b in range(z.size // 32):
+        blk = z[32 * b: 32 * b + 32]
+        amax = float(np.max(np.abs(blk)))
+        v = float(np.float32(amax) / np.float32(448.0))
+        X = 0 if amax == 0 else next(x for x in range(-127, 128) if 2.0 ** x >= v)
+        scales[b] = X + 127
+        codes[32 * b: 32 * b + 32] = _brute_encode(blk.astype(np.float64) * 2.0 ** -X, table, 0x80)
+    return codes, scales
+
+
+def test_ffn_chain_equals_brute_force_on_small_integers():
+    """Small-integer operands (every GMM1 output an exact integer): the oracle's
+    h, z, requantised codes and scales and y equal a brute-force chain written
+    here -- integer matmul, silu from the digits of e, MXFP8 by search, the
+    second product summed exactly and rounded by torch."""
+    from fractions import Fraction
+    r = np.random.default_rng(7)
+    E, H, I, per = 2, 64, 64, 3
+    rows = E * per
+    enc = oracle.e4m3_encode
+    xi = r.integers(0, 4, (rows, H))
+    w1i = r.integers(-1, 2, (E, 2 * I, H))
+    w2i = r.integers(-2, 3, (E, H, I))
+    xc = enc(xi.astype(np.float32))
+    xs = np.full((rows, H // 32), 127, np.uint8)
+    w1c, w1s = enc(w1i.astype(np.float32)), np.full((E, 2 * I, H // 32), 127, np.uint8)
+    w2c, w2s = enc(w2i.astype(np.float32)), np.full((E, H, I // 32), 127, np.uint8)
+    eo = np.arange(E, dtype=np.int64) * per
+    cnt = np.full(E, per, np.int64)
+    o = oracle.expert_ffn_mx(xc, xs, w1c, w1s, w2c, w2s, eo, cnt)
+    table = _e4m3_table()
+    for e in range(E):
+        for rr in range(e * per, (e + 1) * per):
+            h = w1i[e] @ xi[rr]                                  # exact integers
+            assert np.array_equal(o["h"][rr], h.astype(np.float32))
+            z = np.array([np.float32(float(_silu_exact(int(h[j])) * int(h[I + j])))
+                          for j in range(I)], np.float32)
+            assert np.array_equal(o["z"][rr], z), rr
+            zc, zs = _mxfp8_by_search(z)
+            assert np.array_equal(o["zc"][rr], zc) and np.array_equal(o["zs"][rr], zs), rr
+            zv = [Fraction(float(table[c & 0x7F])) * (-1 if c & 0x80 else 1) *
+                  Fraction(2) ** (int(zs[i // 32]) - 127) for i, c in enumerate(zc)]
+            y = np.empty(H, np.float32)
+            for j in range(H):
+                y[j] = np.float32(float(sum(zv[i] * int(w2i[e, j, i]) for i in range(I))))
+            want = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+            assert np.array_equal(o["y"][rr], want), rr
+    untouched = np.ones(rows, bool)
+    untouched[:E * per] = False
+    assert np.all(o["y"][untouched] == 0)
+
+
+def test_ffn_requant_window_and_power_of_two_scales():
+    """On random MX operands: each requantised block's scale is a power of two
+    with the block maximum in (224, 448] after scaling, and every dequantised
+    element lies within half an e4m3 step of z."""
+    r = np.random.default_rng(11)
+    E, H, I, per = 2, 128, 96, 4
+    rows = E * per
+    xc = r.integers(0, 0x7E, (rows, H)).astype(np.uint8)
+    xs = r.integers(118, 126, (rows, H // 32)).astype(np.uint8)
+    w1c = (r.integers(0, 0x7E, (E, 2 * I, H)) | (r.integers(0, 2, (E, 2 * I, H)) << 7)).astype(np.uint8)
+    w1s = r.integers(116, 124, (E, 2 * I, H // 32)).astype(np.uint8)
+    w2c = r.integers(0, 0x7E, (E, H, I)).astype(np.uint8)
+    w2s = np.full((E, H, I // 32), 120, np.uint8)
+    o = oracle.expert_ffn_mx(xc, xs, w1c, w1s, w2c, w2s, np.array([0, per]), np.array([per, per]))
+    dec = oracle.e4m3_decode(o["zc"]).astype(np.float64)
+    X = o["zs"].astype(np.int64) - 127
+    for rr in range(rows):
+        for b in range(I // 32):
+            z = o["z"][rr, 32 * b: 32 * b + 32].astype(np.float64)
+            q = dec[rr, 32 * b: 32 * b + 32] * 2.0 ** X[rr, b]
+            amax = np.abs(z).max()
+            if amax == 0:
+                continue
+            assert 224 < amax * 2.0 ** -X[rr, b] <= 448
+            step = np.ldexp(1.0, np.floor(np.log2(np.maximum(np.abs(z) * 2.0 ** -X[rr, b], 2 ** -6))).astype(int) - 3)
+            assert np.all(np.abs(q - z) <= 0.5 * step * 2.0 ** X[rr, b] + 2.0 ** (X[rr, b] - 10))
