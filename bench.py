@@ -57,7 +57,7 @@ import synth  # noqa: E402
 METRIC = "dispatch+combine tokens/s and achieved HBM GB/s (% of B200 peak), 1 GPU"
 FALLBACK_HBM_GBS = 6650.0
 WORKLOAD_MODE = {"tiny": "int8_token", "decode": "e4m3_b128", "skewed": "int8_token",
-                 "prefill": "mxfp8", "large": "mxfp4"}
+                 "prefill": "mxfp8", "large": "mxfp4", "a5": "mxfp8"}
 KERNEL_SOURCES = ["combine_ep_dispatch_04_b200/csrc/" + f for f in
                   ("ep_api.cu", "ep_device.cuh", "ep_layout.cuh", "ep_dispatch.cuh", "ep_combine.cuh")]
 
@@ -509,6 +509,92 @@ class WorkloadRun:
         torch.cuda.empty_cache()
 
 
+def run_ffn_leg(ep, flush, stream, dev, args, replica):
+    """The deep fused MoE page's benchmark case on one GPU ("[feat] A5 deep fused
+    moe supported", Benchmarking: EP 8, hidden 7168, moe-intermediate-size 3072,
+    top-6, 6 experts a rank, FP8, uniform routing; 128 tokens a rank): the
+    experts' gated MLP alone (ep_expert_ffn_mx: GMM1 with SwiGLU and the
+    requant in its epilogue, GMM2) and the whole forward path in one call
+    (ep_moe_forward_ffn: layout + MXFP8 dispatch, the MLP, combine), each timed
+    alone between events after an L2 flush.  Seeded random MXFP8 weights.
+    FLOPs = 2 * entries * (H * 2I + I * H); the bytes that must move at least
+    once are the codes and scales of every used expert's weights, the received
+    rows, z (written and read) and y; the tensor peak is the measured bf16 peak
+    times the nominal fp8 / bf16 ratio 2."""
+    w = synth.workload("a5")
+    R, T, M, K, E, H, I = w["R"], w["T"], w["M"], w["K"], w["E"], w["H"], w["inter"]
+    idx, wts = synth.make_routing(w, replica)
+    x = synth.make_x(w, replica)
+    cfg = ep.make_config(R, T, M, K, E, H, "mxfp8", "packed")
+    b = ep.Buffers(cfg, device=dev)
+    x_d = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    idx_d, wts_d = torch.from_numpy(idx).to(dev), torch.from_numpy(wts).to(dev)
+    gen = torch.Generator(device=dev).manual_seed(77)
+
+    def mxw(n, k, lo, hi):
+        c = torch.randint(0, 256, (E, n, k), device=dev, dtype=torch.int16,
+                          generator=gen).to(torch.uint8)
+        c[(c & 0x7F) == 0x7F] = 0
+        sc = torch.randint(lo, hi, (E, n, k // 32), device=dev, dtype=torch.int16,
+                           generator=gen).to(torch.uint8)
+        return c, sc
+    w1c, w1s = mxw(2 * I, H, 112, 116)
+    w2c, w2s = mxw(H, I, 110, 114)
+    zb, _ = ep.ep_ffn_buffer_bytes(cfg, I)
+    z = torch.empty(zb, dtype=torch.uint8, device=dev)
+    ep.ep_dispatch_with_layout(cfg, x_d, idx_d, b.token_slot, b.recv_count, b.workspace,
+                               b.recv_buf, b.src_info, b.dev_status,
+                               expert_offset=b.expert_offset, stream=stream)
+    mlp = ep.ep_expert_ffn_mx(cfg, b.recv_buf, b.expert_offset, b.recv_count, w1c, w1s, w2c, w2s,
+                              z, b.y, b.dev_status, stream=stream, bind=True)
+    fwd = ep.ep_moe_forward_ffn(cfg, x_d, idx_d, wts_d, w1c, w1s, w2c, w2s, b.token_slot,
+                                b.recv_count, b.expert_offset, b.workspace, b.recv_buf,
+                                b.src_info, z, b.y, b.out, b.dev_status, stream=stream,
+                                bind=True)
+
+    def timed(call):
+        for _ in range(3):
+            flush(1)
+            call()
+        torch.cuda.synchronize(dev)
+        if ep.ep_get_status(b.dev_status) != 0:
+            raise RuntimeError("device status reported errors")
+        reps = max(3, min(args.steps, 20))
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        for s_ in range(reps):
+            flush(s_ & 0xFF)
+            evs[s_][0].record(stream)
+            call()
+            evs[s_][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return statistics.mean(a.elapsed_time(c) for a, c in evs)
+    ms_mlp = timed(mlp)
+    ms_fwd = timed(fwd)
+    v = int(b.recv_count.sum().item())
+    used = int((b.recv_count > 0).sum().item())
+    flops = 2.0 * v * (H * 2 * I + I * H)
+    wbytes = used * (2 * I * H + H * I) * (1 + 1 / 32)
+    nbytes = wbytes + v * (H + H / 32) + 2 * v * (I + I / 32) + 2.0 * v * H
+    peaks = measured_peaks() or {}
+    peak = (peaks.get("bf16_tflops") or 1590.0) * 2.0
+    hbm = peaks.get("hbm_gbs") or FALLBACK_HBM_GBS
+    t_tensor, t_hbm = flops / (peak * 1e12), nbytes / (hbm * 1e9)
+    del w1c, w1s, w2c, w2s, z, b
+    torch.cuda.empty_cache()
+    return {"workload": f"a5: R={R} T={T} H={H} K={K} E={E} M={M} mxfp8 packed, intermediate {I}",
+            "mlp_ms": round(ms_mlp, 4), "forward_ms": round(ms_fwd, 4),
+            "tokens_per_s": round(R * T / (ms_fwd * 1e-3), 1),
+            "flops": flops, "bytes": nbytes, "tflops": round(flops / (ms_mlp * 1e-3) / 1e12, 1),
+            "gbs": round(nbytes / (ms_mlp * 1e-3) / 1e9, 1),
+            "bound": "tensor" if t_tensor >= t_hbm else "hbm", "peak_tflops": peak,
+            "peak_gbs": hbm, "peak_source": ("measured bf16 x 2 (nominal fp8 / bf16)"
+                                              if peaks.get("bf16_tflops") else "fallback bf16 x 2"),
+            "frac": round(max(t_tensor, t_hbm) / (ms_mlp * 1e-3), 4),
+            "launches": {"mlp": 2, "forward": 5},
+            "what": "mlp: GMM1 + SwiGLU + requant, GMM2; forward: layout + dispatch, mlp, combine"}
+
+
 STEADY_SETS = 4
 STEADY_MAX_BYTES = 1 << 30
 
@@ -787,6 +873,13 @@ def main():
                         "mxfp4") if gw["H"] % 256 == 0 else None)
         del gx_d, gidx_d, gwts_d
         torch.cuda.empty_cache()
+    ffn = None
+    if gemm_on:
+        try:
+            ffn = run_ffn_leg(ep, flush, stream, dev, args, replica)
+        except Exception as ex:  # noqa: BLE001 -- reported in the line
+            torch.cuda.empty_cache()
+            ffn = {"error": f"{type(ex).__name__}: {ex}"[:300]}
 
     out = {
         "metric": METRIC,
@@ -825,6 +918,7 @@ def main():
         "expert_gemm": gemm,
         "expert_gemm_mx": gemm_mx,
         "expert_gemm_mxfp4": gemm_mx4,
+        "expert_ffn": ffn,
         "copy_gbs_same_run": copy_gbs,
         "e2e": e2e,
     }

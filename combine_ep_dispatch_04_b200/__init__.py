@@ -10,7 +10,8 @@ from .ep import (DEV_BAD_INDEX, DEV_CAPACITY_OVERFLOW, DEV_TIMEOUT, ERR_BUFFER_T
                  F_LAYOUT_SINGLE_CTA, F_ROUND_SCALE, F_UE8M0, LAYOUT, QUANT, Bound, Buffers,
                  EpConfig, EpError, EpSizes, ep_buffer_sizes, ep_combine, ep_combine_backward,
                  ep_combine_backward_weights, ep_copy, ep_cvt_sweep, ep_dispatch, ep_dispatch_layout,
-                 ep_dispatch_layout_static, ep_dispatch_with_layout, ep_expert_gemm, ep_expert_gemm_mx,
+                 ep_dispatch_layout_static, ep_dispatch_with_layout, ep_expert_ffn_mx, ep_expert_gemm, ep_expert_gemm_mx,
+                 ep_ffn_buffer_bytes, ep_moe_forward_ffn,
                  ep_get_status,
                  ep_kernel_launches, ep_moe_forward, ep_wait_probe, idx_dtype,
                  make_config)
@@ -23,5 +24,6 @@ __all__ = [
     "EpConfig", "EpError", "EpSizes", "ep_buffer_sizes", "ep_combine", "ep_combine_backward",
     "ep_combine_backward_weights",
     "ep_copy", "ep_cvt_sweep", "ep_dispatch", "ep_dispatch_layout", "ep_dispatch_layout_static",
-    "ep_dispatch_with_layout", "ep_expert_gemm", "ep_expert_gemm_mx", "ep_get_status", "ep_kernel_launches", "ep_moe_forward", "ep_wait_probe", "idx_dtype", "make_config",
+    "ep_dispatch_with_layout", "ep_expert_ffn_mx", "ep_ffn_buffer_bytes", "ep_moe_forward_ffn",
+    "ep_expert_gemm", "ep_expert_gemm_mx", "ep_get_status", "ep_kernel_launches", "ep_moe_forward", "ep_wait_probe", "idx_dtype", "make_config",
 ]

@@ -887,26 +887,41 @@ bool u8_tile_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t oute
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// one launch of the MX kernel (e4m3 or packed e2m1 codes) with N tiles of BN columns
-extern "C++" template <int BN, bool FP4>
-ep_status_t launch_gemm_mx(const Plan &p, const void *recv_buf, const int64_t *expert_offset,
+// An MX operand of the maps: codes [rows][K bytes or K/2] and the e8m0 scales
+// [rows][K/32] of the same rows.
+struct MxOperand {
+    const void *codes;
+    const uint8_t *scales;
+    int K;  // elements of a row
+};
+
+// one launch of the MX kernel (e4m3 or packed e2m1 codes) with N tiles of BN
+// columns; GLU: the first layer of the gated MLP (n_out = 2I outputs of which
+// the epilogue writes z = silu(gate) * up requantised to zc / zs, BN/2 of each
+// half per tile)
+extern "C++" template <int BN, bool FP4, bool GLU = false>
+ep_status_t launch_gemm_mx(const Plan &p, const MxOperand &x, const int64_t *expert_offset,
                            const int64_t *recv_count, const uint8_t *w_codes,
-                           const uint8_t *w_scales, int n_out, uint16_t *y,
-                           uint32_t *dev_status, cudaStream_t s, int slot) {
-    const uint64_t D = FP4 ? (uint64_t)p.H / 2 : (uint64_t)p.H;  // code bytes of a row
+                           const uint8_t *w_scales, int n_out, uint16_t *y, uint8_t *zc,
+                           uint8_t *zs, uint32_t *dev_status, cudaStream_t s, int slot) {
+    const uint64_t D = FP4 ? (uint64_t)x.K / 2 : (uint64_t)x.K;  // code bytes of a row
+    constexpr int TN = GLU ? BN / 2 : BN;
     CUtensorMap ma, mb;
-    if (!u8_tile_map(&ma, recv_buf, D, (uint64_t)p.rows, ep::kGemmBM) ||
-        !u8_tile_map(&mb, w_codes, D, (uint64_t)p.E * n_out, BN))
+    if (!u8_tile_map(&ma, x.codes, D, (uint64_t)p.rows, ep::kGemmBM) ||
+        !u8_tile_map(&mb, w_codes, D, (uint64_t)p.E * n_out, TN))
         return EP_ERR_CUDA;
     ep::MxArgs a;
-    a.E = p.E; a.H = p.H; a.N = n_out; a.ntn = n_out / BN; a.rows = p.rows;
+    std::memset(&a, 0, sizeof(a));
+    a.E = p.E; a.K = x.K; a.N = n_out; a.rows = p.rows;
+    a.I = GLU ? n_out / 2 : 0;
+    a.ntn = GLU ? a.I / TN : n_out / BN;
     a.eo = expert_offset; a.cnt = recv_count;
-    a.xs = static_cast<const uint8_t *>(recv_buf) + p.scale_off;
-    a.ws = w_scales; a.y = y; a.status = dev_status;
+    a.xs = x.scales;
+    a.ws = w_scales; a.y = y; a.zc = zc; a.zs = zs; a.status = dev_status;
     const size_t smem = ep::MxCfg<BN, FP4>::smem();
-    if (!allow_smem(ep::expert_gemm_mx_kernel<BN, FP4>, slot, smem)) return EP_ERR_CUDA;
-    launch(ep::expert_gemm_mx_kernel<BN, FP4>, (unsigned)sm_count(), ep::kMxThreads, smem, s, ma,
-           mb, a);
+    if (!allow_smem(ep::expert_gemm_mx_kernel<BN, FP4, GLU>, slot, smem)) return EP_ERR_CUDA;
+    launch(ep::expert_gemm_mx_kernel<BN, FP4, GLU>, (unsigned)sm_count(), ep::kMxThreads, smem, s,
+           ma, mb, a);
     return launched();
 }
 
@@ -1032,12 +1047,16 @@ ep_status_t run_gemm_bf16(const ep_config_t *cfg, const Plan &p, const void *rec
 ep_status_t run_gemm_mx(const ep_config_t *cfg, const Plan &p, const void *recv_buf,
                         const int64_t *expert_offset, const int64_t *recv_count,
                         const uint8_t *w_codes, const uint8_t *w_scales, int n_out, uint16_t *y,
-                        uint32_t *dev_status, cudaStream_t s) {
+                        uint32_t *dev_status, cudaStream_t s, const MxOperand *x_in = nullptr) {
     const bool fp4 = cfg->quant == EP_Q_MXFP4;
     const int bn = mx_tile_n(n_out, fp4, p.N * p.K / p.E);
+    const MxOperand x = x_in ? *x_in
+                             : MxOperand{recv_buf,
+                                         static_cast<const uint8_t *>(recv_buf) + p.scale_off,
+                                         p.H};
 #define EP_MX(BN_, FP4_, SLOT_)                                                              \
-    return launch_gemm_mx<BN_, FP4_>(p, recv_buf, expert_offset, recv_count, w_codes, w_scales, \
-                                     n_out, y, dev_status, s, SLOT_)
+    return launch_gemm_mx<BN_, FP4_>(p, x, expert_offset, recv_count, w_codes, w_scales, n_out, \
+                                     y, nullptr, nullptr, dev_status, s, SLOT_)
     if (fp4) {
         if (bn == 224) EP_MX(224, true, 9);
         if (bn == 256) EP_MX(256, true, 10);
@@ -1079,6 +1098,139 @@ ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf, size
         return st;
     return run_gemm_mx(cfg, p, recv_buf, expert_offset, recv_count, w_codes, w_scales, n_out, y,
                        dev_status, cs(stream));
+}
+
+// ---- the experts' gated MLP ----------------------------------------------------
+namespace {
+// z buffer of the gated MLP: e4m3 codes [rows][I], then at a 256-byte aligned
+// offset the e8m0 scales [rows][I/32]
+int64_t ffn_z_scale_offset(const Plan &p, int I) { return round_up(p.rows * I, 256); }
+int64_t ffn_z_bytes(const Plan &p, int I) { return ffn_z_scale_offset(p, I) + p.rows * (I / 32); }
+
+ep_status_t check_ffn_args(const ep_config_t *cfg, const Plan &p, int I, const void *recv_buf,
+                           size_t recv_bytes, const int64_t *expert_offset,
+                           const int64_t *recv_count, const uint8_t *w1c, const uint8_t *w1s,
+                           const uint8_t *w2c, const uint8_t *w2s, const void *z_buf,
+                           size_t z_bytes, const void *y, size_t y_bytes,
+                           const uint32_t *dev_status) {
+    if (cfg->quant != EP_Q_MXFP8 || cfg->layout != EP_LAYOUT_PACKED) return EP_ERR_UNSUPPORTED;
+    if (p.H % ep::kMxBK != 0) return EP_ERR_UNSUPPORTED;
+    if (I <= 0 || I % ep::kMxBK != 0 || I > kMaxHidden) return EP_ERR_INVALID_ARG;
+    if (mx_tile_n(p.H) == 0) return EP_ERR_INVALID_ARG;
+    if ((int64_t)2 * I * p.E > kIntLimit || (int64_t)p.H * p.E > kIntLimit ||
+        p.E > ep::kGemmMaxExperts)
+        return EP_ERR_INVALID_ARG;
+    if (!dev_status) return EP_ERR_INVALID_ARG;
+    if (p.N == 0) return EP_OK;
+    if (!recv_buf || !expert_offset || !recv_count || !w1c || !w1s || !w2c || !w2s || !z_buf ||
+        !y)
+        return EP_ERR_INVALID_ARG;
+    if (!aligned16(recv_buf) || !aligned16(w1c) || !aligned16(w1s) || !aligned16(w2c) ||
+        !aligned16(w2s) || !aligned16(z_buf) || !aligned16(y))
+        return EP_ERR_MISALIGNED;
+    ep_status_t st;
+    if ((st = need(recv_bytes, p.recv_bytes)) != EP_OK) return st;
+    if ((st = need(z_bytes, ffn_z_bytes(p, I))) != EP_OK) return st;
+    return need(y_bytes, p.rows * p.H * 2);
+}
+
+// GMM1 with SwiGLU and the requant in its epilogue (tiles of 128 gate + 128 up
+// columns where the experts average 256 rows or more, else 64 + 64 with two
+// accumulators so that a tile's epilogue overlaps the next tile's MMAs), then
+// GMM2 on the requantised z.
+ep_status_t run_ffn(const Plan &p, int I, const void *recv_buf, const int64_t *expert_offset,
+                    const int64_t *recv_count, const uint8_t *w1c, const uint8_t *w1s,
+                    const uint8_t *w2c, const uint8_t *w2s, void *z_buf, uint16_t *y,
+                    uint32_t *dev_status, cudaStream_t s) {
+    uint8_t *zc = static_cast<uint8_t *>(z_buf);
+    uint8_t *zs = zc + ffn_z_scale_offset(p, I);
+    const MxOperand x{recv_buf, static_cast<const uint8_t *>(recv_buf) + p.scale_off, p.H};
+    const bool wide = p.N * p.K / p.E >= 256 && I % 128 == 0;
+    ep_status_t st = wide ? launch_gemm_mx<256, false, true>(p, x, expert_offset, recv_count, w1c,
+                                                            w1s, 2 * I, nullptr, zc, zs,
+                                                            dev_status, s, 13)
+                          : launch_gemm_mx<128, false, true>(p, x, expert_offset, recv_count, w1c,
+                                                            w1s, 2 * I, nullptr, zc, zs,
+                                                            dev_status, s, 14);
+    if (st != EP_OK) return st;
+    const MxOperand z{zc, zs, I};
+    ep_config_t c2 = {};
+    c2.quant = EP_Q_MXFP8;
+    return run_gemm_mx(&c2, p, nullptr, expert_offset, recv_count, w2c, w2s, p.H, y, dev_status,
+                       s, &z);
+}
+}  // namespace
+
+ep_status_t ep_ffn_buffer_bytes(const ep_config_t *cfg, int32_t inter, int64_t *z_bytes,
+                                int64_t *z_scale_offset) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (inter <= 0 || inter % ep::kMxBK != 0 || inter > kMaxHidden || !z_bytes)
+        return EP_ERR_INVALID_ARG;
+    *z_bytes = ffn_z_bytes(p, inter);
+    if (z_scale_offset) *z_scale_offset = ffn_z_scale_offset(p, inter);
+    return EP_OK;
+}
+
+ep_status_t ep_expert_ffn_mx(const ep_config_t *cfg, const void *recv_buf, size_t recv_bytes,
+                             const int64_t *expert_offset, const int64_t *recv_count,
+                             const uint8_t *w1_codes, const uint8_t *w1_scales,
+                             const uint8_t *w2_codes, const uint8_t *w2_scales, int32_t inter,
+                             void *z_buf, size_t z_bytes, uint16_t *y, size_t y_bytes,
+                             uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if ((st = check_ffn_args(cfg, p, inter, recv_buf, recv_bytes, expert_offset, recv_count,
+                             w1_codes, w1_scales, w2_codes, w2_scales, z_buf, z_bytes, y, y_bytes,
+                             dev_status)) != EP_OK ||
+        p.N == 0)
+        return st;
+    return run_ffn(p, inter, recv_buf, expert_offset, recv_count, w1_codes, w1_scales, w2_codes,
+                   w2_scales, z_buf, y, dev_status, cs(stream));
+}
+
+ep_status_t ep_moe_forward_ffn(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
+                               const float *topk_weights, const uint8_t *w1_codes,
+                               const uint8_t *w1_scales, const uint8_t *w2_codes,
+                               const uint8_t *w2_scales, int32_t inter, int32_t *token_slot,
+                               int64_t *recv_count, int64_t *expert_offset, void *workspace,
+                               size_t workspace_bytes, void *recv_buf, size_t recv_bytes,
+                               int32_t *src_info, size_t src_info_bytes, void *z_buf,
+                               size_t z_bytes, uint16_t *y, size_t y_bytes, uint16_t *out,
+                               uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (cfg->flags & EP_F_COMBINE_QUANTIZED) return EP_ERR_UNSUPPORTED;  // y is bf16 here
+    // every argument is checked before the first launch
+    if ((st = check_layout_args(cfg, p, topk_idx, token_slot, recv_count, expert_offset, workspace,
+                                workspace_bytes, dev_status)) != EP_OK)
+        return st;
+    if ((st = check_ffn_args(cfg, p, inter, recv_buf, recv_bytes, expert_offset, recv_count,
+                             w1_codes, w1_scales, w2_codes, w2_scales, z_buf, z_bytes, y, y_bytes,
+                             dev_status)) != EP_OK)
+        return st;
+    if (p.N > 0) {
+        if ((st = check_dispatch_args(cfg, p, x, topk_idx, topk_weights, token_slot,
+                                      expert_offset, recv_buf, recv_bytes, src_info,
+                                      src_info_bytes, nullptr, 0)) != EP_OK)
+            return st;
+        if (!topk_weights || !out) return EP_ERR_INVALID_ARG;
+        if (!aligned16(out)) return EP_ERR_MISALIGNED;
+    }
+    if ((st = ep_dispatch_with_layout(cfg, x, topk_idx, topk_weights, nullptr, nullptr, nullptr,
+                                      token_slot, recv_count, expert_offset, nullptr, workspace,
+                                      workspace_bytes, recv_buf, recv_bytes, src_info,
+                                      src_info_bytes, nullptr, 0, dev_status, stream)) != EP_OK ||
+        p.N == 0)
+        return st;
+    if ((st = run_ffn(p, inter, recv_buf, expert_offset, recv_count, w1_codes, w1_scales,
+                      w2_codes, w2_scales, z_buf, y, dev_status, cs(stream))) != EP_OK)
+        return st;
+    return ep_combine(cfg, y, y_bytes, topk_idx, topk_weights, token_slot, expert_offset, out,
+                      dev_status, stream);
 }
 
 ep_status_t ep_moe_forward(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,

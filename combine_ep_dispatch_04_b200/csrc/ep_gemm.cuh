@@ -605,7 +605,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 //
 // Warps: 0 loads the code tiles with TMA; 1 allocates TMEM and one lane
 // issues the scale copies and the MMAs; 2 gathers the scales; 3 - 6 run the
-// epilogue.  A stage is full when the TMA bytes have landed and the gathering
+// epilogue.
+//
+// GLU = true (MXFP8 only) is the first layer of the experts' gated MLP
+// ("[feat] A5 deep fused moe supported": GMM1, SwiGLU and Requant): the
+// weights are [E][2I][K] with the gate projection in rows 0 .. I-1 and the up
+// projection in rows I .. 2I-1 of each expert; a tile's B operand is BN/2
+// gate rows j0 .. and the same BN/2 up rows (two TMA boxes), so the
+// accumulator holds gate columns 0 .. BN/2-1 and the matching up columns
+// BN/2 .. BN-1.  The epilogue forms z = silu(gate) * up in fp32 from the
+// accumulator and writes it requantised to MXFP8 (one e8m0 scale per 32
+// outputs, the dispatch's rule): codes [rows][I], scales [rows][I/32].  A stage is full when the TMA bytes have landed and the gathering
 // warp has arrived.  TMEM holds kAcc accumulators of BN columns and the
 // scales behind them: two accumulators (the epilogue of one tile overlaps the
 // next tile's MMAs) where they and the scales fit in 512 columns, else one.
@@ -640,16 +650,26 @@ struct MxCfg {
 };
 
 struct MxArgs {
-    int E, H, N;
-    int ntn;                 // N / BN
+    int E, K, N;             // experts, depth (elements of a row), output columns
+    int ntn;                 // N / BN (GLU: I / (BN/2))
+    int I;                   // GLU: the intermediate size (N = 2I)
     int64_t rows;            // rows of the receive buffer (scale rows that exist)
     const int64_t *eo;       // [E+1] first row of each expert (packed layout)
     const int64_t *cnt;      // [E] rows of each expert
-    const uint8_t *xs;       // [rows][H/32] e8m0 scales of the received rows
-    const uint8_t *ws;       // [E*N][H/32] e8m0 scales of the weights
-    uint16_t *y;             // [rows][N] bf16
+    const uint8_t *xs;       // [rows][K/32] e8m0 scales of the received rows
+    const uint8_t *ws;       // [E*N][K/32] e8m0 scales of the weights
+    uint16_t *y;             // [rows][N] bf16 (not GLU)
+    uint8_t *zc;             // GLU: [rows][I] e4m3 codes of the requantised z
+    uint8_t *zs;             // GLU: [rows][I/32] their e8m0 scales
     uint32_t *status;
 };
+
+// silu(g) * u in fp32: g / (1 + e^-g) with the library's expf and
+// correctly rounded division and multiply (a very negative g gives
+// e^-g = inf and silu = -0)
+__device__ __forceinline__ float swiglu(float g, float u) {
+    return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
 
 // instruction descriptor of the block-scaled MMA: A and B formats (e4m3 = 0
 // for kind::mxf8f6f4, e2m1 = 1 for kind::mxf4), both K-major, e8m0 scales,
@@ -694,11 +714,13 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
-template <int BN, bool FP4>
+template <int BN, bool FP4, bool GLU = false>
 __global__ void __launch_bounds__(kMxThreads, 1)
     expert_gemm_mx_kernel(const __grid_constant__ CUtensorMap tm_a,
                           const __grid_constant__ CUtensorMap tm_b, MxArgs a) {
     using C = MxCfg<BN, FP4>;
+    static_assert(!GLU || (!FP4 && BN % 64 == 0), "GLU: MXFP8, whole 32-blocks per half tile");
+    constexpr int TN = GLU ? BN / 2 : BN;  // output columns a tile advances by
     constexpr int S = kMxStages;
     extern __shared__ uint8_t gsm_raw[];
     uint8_t *gsm = reinterpret_cast<uint8_t *>(
@@ -743,14 +765,14 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     tc_fence_after();
     const uint32_t tmem_base = *s_tmem;
     const int total = prefix[E];
-    const int kblocks = (FP4 ? a.H / 2 : a.H) / kMxBK;  // 128-byte K steps
+    const int kblocks = (FP4 ? a.K / 2 : a.K) / kMxBK;  // 128-byte K steps
 
     if (warp == 0 && lane == 0) {
         // ---- code tiles
         int it = 0;
         for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
             int e, m0, n0;
-            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, BN);
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN);
             const int arow = (int)a.eo[e] + m0, brow = e * a.N + n0;
             for (int kb = 0; kb < kblocks; kb++, it++) {
                 const int s = it % S, r = it / S;
@@ -762,7 +784,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 const uint32_t fb = smem_addr(&full[s]);
                 mbar_expect_tx(fb, C::kBytesA + C::kBytesB);
                 tma_load_2d(smem_addr(sA + s * C::kBytesA), &tm_a, kb * kMxBK, arow, fb);
-                tma_load_2d(smem_addr(sB + s * C::kBytesB), &tm_b, kb * kMxBK, brow, fb);
+                if constexpr (GLU) {  // gate rows, then the same rows of the up projection
+                    tma_load_2d(smem_addr(sB + s * C::kBytesB), &tm_b, kb * kMxBK, brow, fb);
+                    tma_load_2d(smem_addr(sB + s * C::kBytesB + TN * kMxBK), &tm_b, kb * kMxBK,
+                                brow + a.I, fb);
+                } else {
+                    tma_load_2d(smem_addr(sB + s * C::kBytesB), &tm_b, kb * kMxBK, brow, fb);
+                }
             }
         }
         for (int j = 0; j < S && j < it; j++) {  // copies in flight land before leaving
@@ -819,7 +847,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         // The loads of sf_group() K steps are issued together: one step's
         // loads would leave a whole L2 latency between consecutive steps.
         constexpr int G = sf_group<FP4>();
-        const int SB = a.H / 32;
+        const int SB = a.K / 32;
         // 16-byte loads where every row's scales start on a 16-byte boundary
         // (the scale regions themselves are 16-byte aligned)
         const bool vec = SB % 16 == 0;
@@ -827,9 +855,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             if (__shfl_sync(kFull, (int)*s_abort, 0)) break;
             int e, m0, n0;
-            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, BN);
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN);
             const int64_t arow0 = a.eo[e] + m0;
             const int64_t brow0 = (int64_t)e * a.N + n0;
+            // weight row of B-tile row n (GLU: the up rows follow the gate rows)
+            auto brow_of = [&](int n) -> int64_t {
+                return GLU ? brow0 + n + (n >= TN ? (int64_t)a.I - TN : 0) : brow0 + n;
+            };
             bool ok = true;
             for (int kb0 = 0; kb0 < kblocks && ok; kb0 += G) {
                 const int g = min(G, kblocks - kb0);
@@ -860,7 +892,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
 #pragma unroll
                             for (int h = 0; h < G * NG / 4; h++) {
                                 const uint4 w4 = n < BN ? __ldg(reinterpret_cast<const uint4 *>(
-                                                              a.ws + (brow0 + n) * SB + kb0 * NG * 4) + h)
+                                                              a.ws + brow_of(n) * SB + kb0 * NG * 4) + h)
                                                         : make_uint4(0u, 0u, 0u, 0u);
                                 const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
@@ -889,7 +921,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                             for (int j = 0; j < 4; j++) {
                                 const int n = 128 * c + 32 * j + lane;
                                 vb[q][gg][c][j] = n < BN ? __ldg(reinterpret_cast<const uint32_t *>(
-                                                               a.ws + (brow0 + n) * SB + off))
+                                                               a.ws + brow_of(n) * SB + off))
                                                          : 0u;
                             }
                     }
@@ -947,17 +979,53 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             }
             tc_fence_after();
             int e, m0, n0;
-            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, BN);
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN);
             const int m = m0 + sub * 32 + lane;
             const bool valid = m < a.cnt[e];
-            uint16_t *yrow = a.y + (a.eo[e] + m) * (int64_t)a.N + n0;
             const uint32_t taddr =
                 tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
+            if constexpr (GLU) {
+                const int64_t row = a.eo[e] + m;
+                uint8_t *zrow = a.zc + row * (int64_t)a.I + n0;
+                uint8_t *zsrow = a.zs + row * (int64_t)(a.I / 32) + n0 / 32;
 #pragma unroll 1
-            for (int c = 0; c < BN / 16; c++) {
-                uint32_t v[16];
-                tmem_ld16(taddr + c * 16, v);
-                if (valid) store_bf16x16(yrow + c * 16, v);
+                for (int c = 0; c < TN / 32; c++) {  // one MX block of 32 outputs
+                    uint32_t g0[16], g1[16], u0[16], u1[16];
+                    tmem_ld16(taddr + c * 32, g0);
+                    tmem_ld16(taddr + c * 32 + 16, g1);
+                    tmem_ld16(taddr + TN + c * 32, u0);
+                    tmem_ld16(taddr + TN + c * 32 + 16, u1);
+                    float z[32];
+                    float amax = 0.0f;
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        z[i] = swiglu(__uint_as_float(g0[i]), __uint_as_float(u0[i]));
+                        z[16 + i] = swiglu(__uint_as_float(g1[i]), __uint_as_float(u1[i]));
+                        amax = fmaxf(amax, fmaxf(fabsf(z[i]), fabsf(z[16 + i])));
+                    }
+                    const int X = mx_exponent_fast<448>(amax);
+                    const float mult = exp2_neg(X);
+                    uint32_t w[8];
+#pragma unroll
+                    for (int q = 0; q < 8; q++)
+                        w[q] = cvt_e4m3x2(__fmul_rn(z[4 * q], mult), __fmul_rn(z[4 * q + 1], mult)) |
+                               (cvt_e4m3x2(__fmul_rn(z[4 * q + 2], mult),
+                                           __fmul_rn(z[4 * q + 3], mult))
+                                << 16);
+                    if (valid) {
+                        st_v4(zrow + c * 32, make_uint4(w[0], w[1], w[2], w[3]));
+                        st_v4(zrow + c * 32 + 16, make_uint4(w[4], w[5], w[6], w[7]));
+                        zsrow[c] = (uint8_t)(X + 127);
+                    }
+                }
+            } else {
+                uint16_t *yrow = a.y + (a.eo[e] + m) * (int64_t)a.N + n0;
+#pragma unroll 1
+                for (int c = 0; c < BN / 16; c++) {
+                    uint32_t v[16];
+                    tmem_ld16(taddr + c * 16, v);
+                    if (valid) store_bf16x16(yrow + c * 16, v);
+                }
             }
             tc_fence_before();
             mbar_arrive(smem_addr(&accempty[acc]));

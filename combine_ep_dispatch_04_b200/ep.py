@@ -92,6 +92,14 @@ lib.ep_moe_forward.restype = C.c_int
 lib.ep_moe_forward.argtypes = [_CFG] + [_P] * 9 + [_Z, _P, _Z, _P, _Z, _P, _Z, _P, _P, _P]
 lib.ep_expert_gemm_mx.restype = C.c_int
 lib.ep_expert_gemm_mx.argtypes = [_CFG, _P, _Z, _P, _P, _P, _P, C.c_int32, _P, _Z, _P, _P]
+lib.ep_ffn_buffer_bytes.restype = C.c_int
+lib.ep_ffn_buffer_bytes.argtypes = [_CFG, C.c_int32, C.POINTER(C.c_int64), C.POINTER(C.c_int64)]
+lib.ep_expert_ffn_mx.restype = C.c_int
+lib.ep_expert_ffn_mx.argtypes = [_CFG, _P, _Z, _P, _P, _P, _P, _P, _P, C.c_int32, _P, _Z, _P, _Z,
+                                 _P, _P]
+lib.ep_moe_forward_ffn.restype = C.c_int
+lib.ep_moe_forward_ffn.argtypes = [_CFG] + [_P] * 7 + [C.c_int32] + [_P] * 4 + \
+    [_Z, _P, _Z, _P, _Z, _P, _Z, _P, _Z, _P, _P, _P]
 lib.ep_combine_backward_weights.restype = C.c_int
 lib.ep_combine_backward_weights.argtypes = [_CFG, _P, _P, _Z] + [_P] * 6
 lib.ep_get_status.restype = C.c_int
@@ -366,6 +374,79 @@ def ep_expert_gemm_mx(cfg, recv_buf, expert_offset, recv_count, w_codes, w_scale
         _stream(stream),
     ]
     return _call(lib.ep_expert_gemm_mx, cfg, args, "ep_expert_gemm_mx", bind)
+
+
+def ep_ffn_buffer_bytes(cfg, inter):
+    """(z_bytes, z_scale_offset) of the gated MLP's intermediate buffer."""
+    zb, zo = C.c_int64(0), C.c_int64(0)
+    _check(lib.ep_ffn_buffer_bytes(C.byref(cfg), int(inter), C.byref(zb), C.byref(zo)),
+           "ep_ffn_buffer_bytes")
+    return zb.value, zo.value
+
+
+def _ffn_weights(cfg, w1_codes, w1_scales, w2_codes, w2_scales):
+    E, H = cfg.num_experts, cfg.hidden
+    if w1_codes is None or w1_codes.dim() != 3 or w1_codes.shape[1] % 2:
+        raise ValueError("w1_codes must be a [E, 2I, H] tensor")
+    inter = int(w1_codes.shape[1]) // 2
+    return inter, [
+        _dev(w1_codes, "w1_codes", torch.uint8, (E, 2 * inter, H)),
+        _dev(w1_scales, "w1_scales", torch.uint8, (E, 2 * inter, H // 32)),
+        _dev(w2_codes, "w2_codes", torch.uint8, (E, H, inter)),
+        _dev(w2_scales, "w2_scales", torch.uint8, (E, H, inter // 32)),
+        C.c_int32(inter),
+    ]
+
+
+def ep_expert_ffn_mx(cfg, recv_buf, expert_offset, recv_count, w1_codes, w1_scales, w2_codes,
+                     w2_scales, z_buf, y, dev_status, stream=None, bind=False):
+    """The experts' gated MLP on the packed MXFP8 receive rows: GMM1 (w1 [E, 2I, H],
+    gate rows first) with SwiGLU and the MXFP8 requant of z in its epilogue (z_buf:
+    codes [rows, I] then scales, ep_ffn_buffer_bytes), then GMM2 (w2 [E, H, I]) into
+    y bf16 [rows, H]."""
+    sz = ep_buffer_sizes(cfg)
+    E, H = cfg.num_experts, cfg.hidden
+    _, wargs = _ffn_weights(cfg, w1_codes, w1_scales, w2_codes, w2_scales)
+    args = [
+        *_buf(recv_buf, "recv_buf"),
+        _dev(expert_offset, "expert_offset", torch.int64, (E + 1,)),
+        _dev(recv_count, "recv_count", torch.int64, (E,)),
+        *wargs,
+        *_buf(z_buf, "z_buf"),
+        _dev(y, "y", torch.bfloat16, (sz["rows"], H)), C.c_size_t(sz["rows"] * H * 2),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    return _call(lib.ep_expert_ffn_mx, cfg, args, "ep_expert_ffn_mx", bind)
+
+
+def ep_moe_forward_ffn(cfg, x, topk_idx, topk_weights, w1_codes, w1_scales, w2_codes, w2_scales,
+                       token_slot, recv_count, expert_offset, workspace, recv_buf, src_info,
+                       z_buf, y, out, dev_status, stream=None, bind=False):
+    """Layout + MXFP8 dispatch -> the experts' gated MLP (ep_expert_ffn_mx) ->
+    combine in one call; out bf16 [N, H]."""
+    N, K = _nk(cfg)
+    sz = ep_buffer_sizes(cfg)
+    E, H = cfg.num_experts, cfg.hidden
+    _, wargs = _ffn_weights(cfg, w1_codes, w1_scales, w2_codes, w2_scales)
+    args = [
+        _dev(x, "x", torch.bfloat16, (N, H)),
+        _dev(topk_idx, "topk_idx", idx_dtype(cfg), (N, K)),
+        _dev(topk_weights, "topk_weights", torch.float32, (N, K)),
+        *wargs,
+        _dev(token_slot, "token_slot", torch.int32, (N, K)),
+        _dev(recv_count, "recv_count", torch.int64, (E,)),
+        _dev(expert_offset, "expert_offset", torch.int64, (E + 1,)),
+        *_buf(workspace, "workspace"),
+        *_buf(recv_buf, "recv_buf"),
+        *_buf(src_info, "src_info"),
+        *_buf(z_buf, "z_buf"),
+        _dev(y, "y", torch.bfloat16, (sz["rows"], H)), C.c_size_t(sz["rows"] * H * 2),
+        _dev(out, "out", torch.bfloat16, (N, H)),
+        _dev(dev_status, "dev_status", torch.int32, (1,)),
+        _stream(stream),
+    ]
+    return _call(lib.ep_moe_forward_ffn, cfg, args, "ep_moe_forward_ffn", bind)
 
 
 def ep_wait_probe(dev_status, stream=None):

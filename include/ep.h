@@ -356,6 +356,68 @@ ep_status_t ep_expert_gemm_mx(const ep_config_t *cfg, const void *recv_buf, size
                               ep_stream_t stream);
 
 /*
+ * The experts' gated two-layer MLP on MXFP8 operands ("[feat] A5 deep fused
+ * moe supported": the operator's stages GMM1, SwiGLU, Requant and GMM2
+ * between its dispatch and combine, with moe-intermediate-size I; its review:
+ * GMM1 takes e4m3 codes with one e8m0 scale per 32 elements).  For each
+ * expert e and each of its received rows r (packed layout):
+ *   GMM1     h = x[r] . W1[e]^T                       (2I outputs, fp32)
+ *   SwiGLU   z[j] = silu(h[j]) * h[I + j], j < I        silu(a) = a / (1 + e^-a)
+ *   Requant  z to MXFP8 per 32 with the MX dispatch's rule (written to z_buf)
+ *   GMM2     y[r] = bf16( zq . W2[e]^T )               (H outputs)
+ * The first I rows of W1[e] are the gate projection, the last I the up
+ * projection.  SwiGLU and the requant run in GMM1's epilogue on the fp32
+ * accumulator (tcgen05 block-scaled MMA); GMM2 is ep_expert_gemm_mx's kernel
+ * with depth I.  Accuracy: GMM1's sums are chained as in ep_expert_gemm_mx
+ * ((H/32 + 32) * 2^-23 * sum |x*w| of the exact sum, before the fp32
+ * rounding), silu uses the library expf (a few fp32 ulps), so an element of z
+ * may round to a neighbouring e4m3 code (and a block to the neighbouring
+ * scale) where the exact value lies that close to a rounding boundary.
+ *   cfg          quant EP_Q_MXFP8, layout EP_LAYOUT_PACKED, H % 128 == 0 and a
+ *                multiple of 224, 256 or 128 (GMM2's column tiles);
+ *                otherwise EP_ERR_UNSUPPORTED / EP_ERR_INVALID_ARG
+ *   recv_buf     the dispatch's receive buffer (recv_bytes >= ep_sizes_t.recv_bytes)
+ *   expert_offset, recv_count   from ep_dispatch_layout
+ *   w1_codes     e4m3 [E][2I][H], w1_scales e8m0 [E][2I][H/32]
+ *   w2_codes     e4m3 [E][H][I],  w2_scales e8m0 [E][H][I/32]
+ *   inter        I, a multiple of 128, at most 8192
+ *   z_buf        z_bytes >= ep_ffn_buffer_bytes(): the requantised z, e4m3
+ *                [rows][I] then, at z_scale_offset, e8m0 [rows][I/32]
+ *                (rows past recv_count not written)
+ *   y            bf16 [rows][H] (y_bytes >= ep_sizes_t.expert_out_bytes): the
+ *                input of ep_combine
+ * All weight and buffer pointers 16-byte aligned (EP_ERR_MISALIGNED).  A wait
+ * inside the kernels that exceeds 2 s sets EP_DEV_TIMEOUT; they never trap.
+ */
+ep_status_t ep_ffn_buffer_bytes(const ep_config_t *cfg, int32_t inter, int64_t *z_bytes,
+                                int64_t *z_scale_offset);
+ep_status_t ep_expert_ffn_mx(const ep_config_t *cfg, const void *recv_buf, size_t recv_bytes,
+                             const int64_t *expert_offset, const int64_t *recv_count,
+                             const uint8_t *w1_codes, const uint8_t *w1_scales,
+                             const uint8_t *w2_codes, const uint8_t *w2_scales, int32_t inter,
+                             void *z_buf, size_t z_bytes, uint16_t *y, size_t y_bytes,
+                             uint32_t *dev_status, ep_stream_t stream);
+
+/*
+ * The page's whole forward path in one call ("[feat] A5 deep fused moe
+ * supported": Dispatch, GMM1, SwiGLU, Requant, GMM2, Combine in one
+ * operator): ep_dispatch_with_layout (MXFP8), ep_expert_ffn_mx, then
+ * ep_combine of its bf16 outputs, launched back to back on `stream` with
+ * programmatic dependent launch.  Every argument is checked before the first
+ * launch; the result equals the calls made one by one.  Arguments as those
+ * calls; cfg as ep_expert_ffn_mx (EP_F_COMBINE_QUANTIZED unsupported).
+ */
+ep_status_t ep_moe_forward_ffn(const ep_config_t *cfg, const uint16_t *x, const void *topk_idx,
+                               const float *topk_weights, const uint8_t *w1_codes,
+                               const uint8_t *w1_scales, const uint8_t *w2_codes,
+                               const uint8_t *w2_scales, int32_t inter, int32_t *token_slot,
+                               int64_t *recv_count, int64_t *expert_offset, void *workspace,
+                               size_t workspace_bytes, void *recv_buf, size_t recv_bytes,
+                               int32_t *src_info, size_t src_info_bytes, void *z_buf,
+                               size_t z_bytes, uint16_t *y, size_t y_bytes, uint16_t *out,
+                               uint32_t *dev_status, ep_stream_t stream);
+
+/*
  * One call for the whole forward path with the experts between dispatch and
  * combine ("[feat] A5 deep fused moe supported": one operator runs the
  * dispatch, the experts' grouped matrix multiplications and the combine):

@@ -15,13 +15,16 @@ windows of one long iid sequence, which lets a device rebuild a 15 GB
 expert-output buffer from a 32 MB pool while a host rebuilds only the rows it
 samples.
 
-Workloads (the five named MoE dispatch / combine shapes):
+Workloads (the five named MoE dispatch / combine shapes, and the deep fused MoE
+page's benchmark case):
   tiny     R=1  T=128  H=1024 K=2 E=8   M=128  N(0,1) x, uniform top-2, 5% -1
   decode   R=8  T=128  H=7168 K=8 E=256 M=128  N(0,1) x, uniform top-8
   skewed   R=16 T=512  H=4096 K=6 E=64  M=512  N(0,1) x with 1% channels x50,
                                               Zipf(1.2) expert popularity
   prefill  R=32 T=4096 H=7168 K=8 E=256 M=4096 N(0,1) x, uniform, 2% -1
   large    R=64 T=256  H=7168 K=8 E=256 M=256  0.5*Student-t(3) x, Zipf(0.8)
+  a5       R=8  T=128  H=7168 K=6 E=48  M=128  N(0,1) x, uniform top-6; the experts'
+                                              gated MLP has intermediate size 3072
 Routing draws K distinct experts per token without replacement with
 probabilities p_e (uniform, or p_e ~ 1/rank(e)^s with a seeded rank
 permutation) by the Gumbel-top-K construction; the order of the K picks is the
@@ -47,6 +50,11 @@ WORKLOADS = {
                     backward=True),
     "large": dict(wid=5, R=64, T=256, H=7168, K=8, E=256, M=256, routing="zipf", zipf_s=0.8,
                   mask_p=0.0, x="student_t", modes=("mxfp4",), layout="packed"),
+    # the deep fused MoE page's benchmark case on one GPU: EP 8 (logical ranks),
+    # 128 tokens a rank, hidden 7168, top-6 of 48 experts (6 a rank), uniform
+    # routing, FP8 (MXFP8), moe-intermediate-size 3072
+    "a5": dict(wid=6, R=8, T=128, H=7168, K=6, E=48, M=128, routing="uniform", zipf_s=0.0,
+               mask_p=0.0, x="normal", modes=("mxfp8",), layout="packed", inter=3072),
 }
 
 # tensor tags inside one workload's key space

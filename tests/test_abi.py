@@ -191,6 +191,18 @@ def _short_calls():
                                         Z(z["workspace"]), _F, Z(z["recv_buf"]), _F,
                                         Z(z["src_info"]), _F, Z(z["y"]), _F, _F, _N))
     s = ep.ep_buffer_sizes(pk)
+    zb, _ = ep.ep_ffn_buffer_bytes(pk, 256)
+    add("ep_expert_ffn_mx", pk, {"recv_buf": s["recv_bytes"], "z_buf": zb,
+                                 "y": s["expert_out_bytes"]},
+        lambda c, z: lib.ep_expert_ffn_mx(C.byref(c), _F, Z(z["recv_buf"]), _F, _F, _F, _F, _F, _F,
+                                          256, _F, Z(z["z_buf"]), _F, Z(z["y"]), _F, _N))
+    add("ep_moe_forward_ffn", pk, {"workspace": s["workspace_bytes"], "recv_buf": s["recv_bytes"],
+                                   "src_info": s["src_info_bytes"], "z_buf": zb,
+                                   "y": s["expert_out_bytes"]},
+        lambda c, z: lib.ep_moe_forward_ffn(C.byref(c), _F, _F, _F, _F, _F, _F, _F, 256, _F, _F, _F,
+                                            _F, Z(z["workspace"]), _F, Z(z["recv_buf"]), _F,
+                                            Z(z["src_info"]), _F, Z(z["z_buf"]), _F, Z(z["y"]), _F,
+                                            _F, _N))
     rows = s["rows"]
     add("ep_expert_gemm_mx", pk, {"recv_buf": s["recv_bytes"], "y": rows * 224 * 2},
         lambda c, z: lib.ep_expert_gemm_mx(C.byref(c), _F, Z(z["recv_buf"]), _F, _F, _F, _F, 224,
