@@ -12,6 +12,7 @@
 #include "ep_device.cuh"
 #include "ep_dispatch.cuh"
 #include "ep_gemm.cuh"
+#include "ep_group.cuh"
 #include "ep_layout.cuh"
 
 namespace {
@@ -641,8 +642,9 @@ ep_status_t launch_combine(const ep::CombineArgs &a, cudaStream_t s) {
     if constexpr (QIN != ep::QIN_BF16) {
         // The pipelined kernel's shared-memory stages cap it near 900 threads an
         // SM; below about a million granules (decode-sized batches) the
-        // register kernel's higher occupancy wins.
-        if (a.K <= ep::kPipeRows && a.S % 4 == 0 && a.S <= ep::kPipeScaleBytes &&
+        // register kernel's higher occupancy wins.  (Rows in other GPUs'
+        // windows are read by the register kernel.)
+        if (!a.peer_y && a.K <= ep::kPipeRows && a.S % 4 == 0 && a.S <= ep::kPipeScaleBytes &&
             a.N * (int64_t)(a.H / ep::combine_granule(QIN)) > ((int64_t)1 << 20))
             return launch_combine_pipelined<QIN>(a, s);
     }
@@ -749,6 +751,7 @@ ep_status_t ep_combine(const ep_config_t *cfg, const uint16_t *y, size_t y_bytes
     if ((st = need(y_bytes, qin == EP_Q_BF16 ? p.rows * p.H * 2 : p.recv_bytes)) != EP_OK)
         return st;
     ep::CombineArgs a;
+    std::memset(&a, 0, sizeof(a));
     a.N = p.N; a.K = p.K; a.E = p.E; a.H = p.H;
     a.packed = cfg->layout == EP_LAYOUT_PACKED;
     a.cap = p.cap; a.rows = p.rows;
@@ -1276,6 +1279,352 @@ ep_status_t ep_moe_forward(const ep_config_t *cfg, const uint16_t *x, const void
                       dev_status, stream);
 }
 
+// ---- expert parallelism over GPUs (ep_group.cuh) ---------------------------------
+}  // extern "C"
+namespace {
+
+// The group's shape from the global configuration: GPU g holds ranks
+// g*RG .. (g+1)*RG - 1 and owns experts g*EG .. (g+1)*EG - 1.  A window holds
+// every row its experts can receive: EG * R * M (padded) or all N * K entries
+// plus the alignment of its experts (packed).
+ep_status_t make_group(const ep_config_t *cfg, const ep_group_t *grp, Plan &p,
+                       ep::GroupShape &s) {
+    ep_status_t st = make_plan(cfg, p);
+    if (st != EP_OK) return st;
+    if (!grp || grp->world < 1 || grp->world > ep::kGroupMaxGpus || grp->rank < 0 ||
+        grp->rank >= grp->world || p.R % grp->world != 0)
+        return EP_ERR_INVALID_ARG;
+    if (cfg->flags & (EP_F_LAYOUT_SINGLE_CTA | EP_F_LAYOUT_MULTI_CTA | EP_F_LAYOUT_CLUSTER))
+        return EP_ERR_INVALID_ARG;
+    s.R = p.R; s.E = p.E; s.G = grp->world; s.g = grp->rank;
+    s.RG = p.R / s.G; s.EG = p.E / s.G;
+    s.win_rows = cfg->layout == EP_LAYOUT_PACKED
+                     ? p.N * p.K + (int64_t)s.EG * (cfg->expert_align - 1)
+                     : (int64_t)s.EG * p.cap;
+    if ((int64_t)s.G * s.win_rows > kIntLimit) return EP_ERR_INVALID_ARG;  // int32 slots
+    return EP_OK;
+}
+
+// the configuration of this GPU's own tokens: RG ranks, packed (no capacity:
+// the local ranks of the entries are all the layout is run for)
+ep_config_t local_config(const ep_config_t *cfg, const ep::GroupShape &s) {
+    ep_config_t c = *cfg;
+    c.num_ranks = s.RG;
+    c.layout = EP_LAYOUT_PACKED;
+    c.expert_align = 1;
+    return c;
+}
+
+int64_t group_ws_bytes(const ep_config_t *cfg, const ep::GroupShape &s) {
+    const ep_config_t lc = local_config(cfg, s);
+    Plan lp;
+    if (make_plan(&lc, lp) != EP_OK) return -1;
+    // + the local layout's expert_offset and recv_count (scratch)
+    return lp.ws_bytes + round_up((int64_t)(2 * s.E + 1) * 8, 256);
+}
+
+bool peers_ok(const ep_peers_t *pe) { return pe && pe->flags && pe->my_flags && pe->done; }
+
+bool group_ok(const ep_group_t *grp) {
+    return grp && grp->world >= 1 && grp->world <= ep::kGroupMaxGpus && grp->rank >= 0 &&
+           grp->rank < grp->world && grp->epoch > 0;
+}
+
+}  // namespace
+extern "C" {
+
+ep_status_t ep_group_sizes(const ep_config_t *cfg, const ep_group_t *grp, ep_sizes_t *out) {
+    Plan p;
+    ep::GroupShape s;
+    ep_status_t st = make_group(cfg, grp, p, s);
+    if (st != EP_OK) return st;
+    if (!out) return EP_ERR_INVALID_ARG;
+    const int64_t rows = s.win_rows;
+    std::memset(out, 0, sizeof(*out));
+    out->rows = rows;
+    out->data_row_bytes = p.D;
+    out->scale_row_bytes = p.S;
+    out->recv_scale_offset = round_up(rows * p.D, 256);
+    out->recv_bytes = out->recv_scale_offset + rows * p.S;
+    out->src_info_bytes = rows * 4;
+    out->recv_weights_bytes = rows * 4;
+    out->expert_out_bytes = rows * p.H * 2;
+    out->grad_scale_offset = round_up(rows * p.H, 256);
+    out->grad_bytes = out->grad_scale_offset + rows * (p.H / 32);
+    out->workspace_bytes = group_ws_bytes(cfg, s);
+    out->token_slot_bytes = (int64_t)s.RG * p.T * p.K * 4;
+    out->is_token_in_rank_bytes = 0;  // not produced over GPUs
+    return EP_OK;
+}
+
+ep_status_t ep_group_layout(const ep_config_t *cfg, const ep_group_t *grp,
+                            const ep_peers_t *peers, const void *topk_idx, int32_t *token_slot,
+                            void *workspace, size_t workspace_bytes, uint32_t *dev_status,
+                            ep_stream_t stream) {
+    Plan p;
+    ep::GroupShape s;
+    ep_status_t st = make_group(cfg, grp, p, s);
+    if (st != EP_OK) return st;
+    if (!group_ok(grp) || !peers_ok(peers) || !peers->counts || !peers->my_counts || !workspace ||
+        !dev_status)
+        return EP_ERR_INVALID_ARG;
+    // this GPU's rows of the [R][E] counts table, in its own counts window
+    int32_t *tokens_per_expert = peers->my_counts + (int64_t)s.g * s.RG * s.E;
+    if ((st = need(workspace_bytes, group_ws_bytes(cfg, s))) != EP_OK) return st;
+    const ep_config_t lc = local_config(cfg, s);
+    Plan lp;
+    if ((st = make_plan(&lc, lp)) != EP_OK) return st;
+    if (lp.N > 0 && (!topk_idx || !token_slot)) return EP_ERR_INVALID_ARG;
+    // local ranks, per-rank counts and (scratch) local counts and offsets
+    int64_t *eo_loc = reinterpret_cast<int64_t *>(static_cast<uint8_t *>(workspace) + lp.ws_bytes);
+    int64_t *cnt_loc = eo_loc + (s.E + 1);
+    ep::LayoutArgs a = layout_args(&lc, lp, topk_idx, nullptr, tokens_per_expert, nullptr,
+                                   token_slot, cnt_loc, eo_loc, nullptr, workspace, dev_status);
+    cudaStream_t cstr = cs(stream);
+    if ((st = run_layout(&lc, lp, a, cstr)) != EP_OK) return st;
+    // the counts to every GPU, then the counts signal
+    launch(ep::group_push_counts_kernel, 1, 256, 0, cstr, (const int32_t *)peers->my_counts,
+           peers->counts, (int64_t)s.g * s.RG * s.E, (int64_t)s.RG * s.E, peers->flags, s.g, s.G,
+           grp->epoch);
+    return launched();
+}
+
+ep_status_t ep_group_plan_host(const ep_config_t *cfg, const ep_group_t *grp,
+                               const int32_t *tokens_per_expert_all, int64_t *slot_base,
+                               int64_t *recv_count, int64_t *expert_offset) {
+    Plan p;
+    ep::GroupShape s;
+    ep_status_t st = make_group(cfg, grp, p, s);
+    if (st != EP_OK) return st;
+    if (!tokens_per_expert_all || !slot_base || !recv_count) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    for (int e = 0; e < s.E; e++) {
+        slot_base[e] = ep::group_prefix(tokens_per_expert_all, s.E, s.g * s.RG, e);
+        recv_count[e] = ep::group_total(tokens_per_expert_all, s.R, s.E, e);
+    }
+    if (cfg->layout == EP_LAYOUT_PACKED)
+        ep::group_packed_offsets(s, recv_count, cfg->expert_align, expert_offset);
+    return EP_OK;
+}
+
+ep_status_t ep_group_plan(const ep_config_t *cfg, const ep_group_t *grp,
+                          const ep_peers_t *peers, const void *topk_idx, int32_t *token_slot,
+                          int64_t *recv_count, int64_t *expert_offset,
+                          int64_t *cumulative_recv_stats, void *workspace, size_t workspace_bytes,
+                          uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep::GroupShape s;
+    ep_status_t st = make_group(cfg, grp, p, s);
+    if (st != EP_OK) return st;
+    if (!group_ok(grp) || !peers_ok(peers) || !peers->my_counts || !recv_count || !workspace ||
+        !dev_status)
+        return EP_ERR_INVALID_ARG;
+    const int32_t *tokens_per_expert_all = peers->my_counts;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    if (s.E > ep::kPlanThreads) return EP_ERR_UNSUPPORTED;
+    if ((st = need(workspace_bytes, (int64_t)s.E * 8)) != EP_OK) return st;
+    const int64_t n_loc = (int64_t)s.RG * p.T;
+    if (n_loc > 0 && (!topk_idx || !token_slot)) return EP_ERR_INVALID_ARG;
+    ep::GroupPlanArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.s = s;
+    a.packed = cfg->layout == EP_LAYOUT_PACKED;
+    a.align = cfg->expert_align;
+    a.my_flags = peers->my_flags;
+    a.epoch = grp->epoch;
+    a.status = dev_status;
+    a.n_loc = n_loc;
+    a.K = p.K;
+    a.tpe_all = tokens_per_expert_all;
+    a.idx = topk_idx_view(cfg, topk_idx);
+    a.slot = token_slot;
+    a.recv_count = recv_count;
+    a.expert_offset = expert_offset;
+    a.stats = cumulative_recv_stats;
+    a.slot_base = static_cast<int64_t *>(workspace);
+    cudaStream_t cstr = cs(stream);
+    launch(ep::group_plan_kernel, 1, ep::kPlanThreads, 0, cstr, a);
+    if ((st = launched()) != EP_OK || n_loc == 0) return st;
+    const int64_t entries = n_loc * p.K;
+    const unsigned grid = (unsigned)std::min<int64_t>((entries + 255) / 256, 4 * sm_count());
+    launch(ep::group_shift_kernel, grid, 256, 0, cstr, a);
+    return launched();
+}
+
+ep_status_t ep_group_dispatch(const ep_config_t *cfg, const ep_group_t *grp,
+                              const ep_peers_t *peers, const uint16_t *x, const void *topk_idx,
+                              const float *topk_weights, const int32_t *token_slot,
+                              const int64_t *expert_offset, uint32_t *dev_status,
+                              ep_stream_t stream) {
+    Plan p;
+    ep::GroupShape s;
+    ep_status_t st = make_group(cfg, grp, p, s);
+    if (st != EP_OK) return st;
+    if (!group_ok(grp) || !dev_status || !peers_ok(peers) || !peers->recv || !peers->src_info)
+        return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    if (peers->recv_weights && !topk_weights) return EP_ERR_INVALID_ARG;
+    const int64_t n_loc = (int64_t)s.RG * p.T;
+    cudaStream_t cstr = cs(stream);
+    if (n_loc == 0) {  // nothing to send: the others still learn that this GPU is done
+        launch(ep::group_signal_kernel, 1, 32, 0, cstr, peers->flags, (int)ep::kFlagDispatch, s.g,
+               s.G, grp->epoch);
+        return launched();
+    }
+    if (!x || !topk_idx || !token_slot) return EP_ERR_INVALID_ARG;
+    if (!aligned16(x)) return EP_ERR_MISALIGNED;
+    ep::DispatchArgs a = dispatch_args(cfg, p);
+    a.N = n_loc;
+    a.first_rank = s.g * s.RG;
+    a.rows = (int64_t)s.G * s.win_rows;  // virtual rows
+    a.D = p.D; a.S = p.S; a.scale_off = round_up(s.win_rows * p.D, 256);
+    a.x = x; a.idx = topk_idx_view(cfg, topk_idx);
+    a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
+    a.status = dev_status;
+    a.peer_out = reinterpret_cast<uint8_t *const *>(peers->recv);
+    a.peer_src = peers->src_info;
+    a.peer_w = peers->recv_weights;
+    a.win_rows = s.win_rows;
+    a.done = peers->done + ep::kFlagDispatch;
+    a.flags = peers->flags;
+    a.flag_kind = ep::kFlagDispatch;
+    a.grp_g = s.g; a.grp_G = s.G;
+    a.epoch = grp->epoch;
+    return run_dispatch(cfg, a, cstr);
+}
+
+ep_status_t ep_group_combine(const ep_config_t *cfg, const ep_group_t *grp,
+                             const ep_peers_t *peers, const void *topk_idx,
+                             const float *topk_weights, const int32_t *token_slot,
+                             const int64_t *expert_offset, uint16_t *out, uint32_t *dev_status,
+                             ep_stream_t stream) {
+    Plan p;
+    ep::GroupShape s;
+    ep_status_t st = make_group(cfg, grp, p, s);
+    if (st != EP_OK) return st;
+    if (!group_ok(grp) || !dev_status || !peers || !peers->y) return EP_ERR_INVALID_ARG;
+    if (cfg->flags & EP_F_COMBINE_QUANTIZED) return EP_ERR_UNSUPPORTED;
+    const int64_t n_loc = (int64_t)s.RG * p.T;
+    if (n_loc == 0) return EP_OK;
+    if (!topk_idx || !topk_weights || !token_slot || !out) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    if (!aligned16(out)) return EP_ERR_MISALIGNED;
+    ep::CombineArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.N = n_loc; a.K = p.K; a.E = p.E; a.H = p.H;
+    a.packed = cfg->layout == EP_LAYOUT_PACKED;
+    a.cap = p.cap; a.rows = (int64_t)s.G * s.win_rows;
+    a.idx = topk_idx_view(cfg, topk_idx);
+    a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
+    a.out = out; a.status = dev_status;
+    a.peer_y = reinterpret_cast<const uint8_t *const *>(peers->y);
+    a.win_rows = s.win_rows;
+    return launch_combine<ep::QIN_BF16>(a, cs(stream));
+}
+
+ep_status_t ep_group_combine_backward(const ep_config_t *cfg, const ep_group_t *grp,
+                                      const ep_peers_t *peers, const uint16_t *g,
+                                      const void *topk_idx, const float *topk_weights,
+                                      const int32_t *token_slot, const int64_t *expert_offset,
+                                      uint32_t *dev_status, ep_stream_t stream) {
+    Plan p;
+    ep::GroupShape s;
+    ep_status_t st = make_group(cfg, grp, p, s);
+    if (st != EP_OK) return st;
+    if (!group_ok(grp) || !dev_status || !peers_ok(peers) || !peers->grad)
+        return EP_ERR_INVALID_ARG;
+    const bool unweighted = (cfg->flags & EP_F_BWD_UNWEIGHTED) != 0;
+    const int64_t n_loc = (int64_t)s.RG * p.T;
+    cudaStream_t cstr = cs(stream);
+    if (n_loc == 0) {
+        launch(ep::group_signal_kernel, 1, 32, 0, cstr, peers->flags, (int)ep::kFlagBackward, s.g,
+               s.G, grp->epoch);
+        return launched();
+    }
+    if (!g || !topk_idx || !token_slot || (!unweighted && !topk_weights)) return EP_ERR_INVALID_ARG;
+    if (cfg->layout == EP_LAYOUT_PACKED && !expert_offset) return EP_ERR_INVALID_ARG;
+    if (!aligned16(g)) return EP_ERR_MISALIGNED;
+    ep::DispatchArgs a = dispatch_args(cfg, p);
+    a.N = n_loc;
+    a.rows = (int64_t)s.G * s.win_rows;
+    a.D = p.H; a.S = p.H / 32; a.scale_off = round_up(s.win_rows * p.H, 256);
+    a.unweighted = unweighted;
+    a.x = g; a.idx = topk_idx_view(cfg, topk_idx);
+    a.wts = topk_weights; a.slot = token_slot; a.eo = expert_offset;
+    a.status = dev_status;
+    a.peer_out = reinterpret_cast<uint8_t *const *>(peers->grad);
+    a.win_rows = s.win_rows;
+    a.done = peers->done + ep::kFlagBackward;
+    a.flags = peers->flags;
+    a.flag_kind = ep::kFlagBackward;
+    a.grp_g = s.g; a.grp_G = s.G;
+    a.epoch = grp->epoch;
+    return launch_combine_bwd(a, cstr);
+}
+
+ep_status_t ep_group_signal(const ep_group_t *grp, const ep_peers_t *peers, int32_t kind,
+                            ep_stream_t stream) {
+    if (!group_ok(grp) || !peers || !peers->flags) return EP_ERR_INVALID_ARG;
+    if (kind < 0 || kind >= ep::kGroupKinds) return EP_ERR_INVALID_ARG;
+    launch(ep::group_signal_kernel, 1, 32, 0, cs(stream), peers->flags, (int)kind, grp->rank,
+           grp->world, grp->epoch);
+    return launched();
+}
+
+ep_status_t ep_group_wait(const ep_group_t *grp, const ep_peers_t *peers, int32_t kind,
+                          uint64_t timeout_ns, uint32_t *dev_status, ep_stream_t stream) {
+    if (!group_ok(grp) || !peers || !peers->my_flags || !dev_status) return EP_ERR_INVALID_ARG;
+    if (kind < 0 || kind >= ep::kGroupKinds) return EP_ERR_INVALID_ARG;
+    const uint64_t limit = timeout_ns ? std::min<uint64_t>(timeout_ns, ep::kWaitLimitNs * 5)
+                                      : ep::kWaitLimitNs;
+    launch(ep::group_wait_kernel, 1, 64, 0, cs(stream), (const uint64_t *)peers->my_flags,
+           (int)kind, (int)grp->world, grp->epoch, limit, dev_status);
+    return launched();
+}
+
+// CUDA IPC of a window: the handle of the allocation that holds `ptr` and the
+// offset of ptr inside it, and the mapping of a peer's window from them.
+ep_status_t ep_ipc_export(const void *ptr, uint8_t *handle, uint64_t *offset) {
+    if (!ptr || !handle || !offset) return EP_ERR_INVALID_ARG;
+    using GetRange = CUresult (*)(CUdeviceptr *, size_t *, CUdeviceptr);
+    static GetRange get_range = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_range = reinterpret_cast<GetRange>(f);
+    });
+    if (!get_range) return EP_ERR_CUDA;
+    CUdeviceptr base = 0;
+    size_t size = 0;
+    if (get_range(&base, &size, reinterpret_cast<CUdeviceptr>(ptr)) != CUDA_SUCCESS)
+        return EP_ERR_CUDA;
+    cudaIpcMemHandle_t h;
+    if (cudaIpcGetMemHandle(&h, reinterpret_cast<void *>(base)) != cudaSuccess) return EP_ERR_CUDA;
+    std::memcpy(handle, &h, sizeof(h));
+    *offset = (uint64_t)(reinterpret_cast<uintptr_t>(ptr) - (uintptr_t)base);
+    return EP_OK;
+}
+
+ep_status_t ep_ipc_import(const uint8_t *handle, uint64_t offset, void **ptr) {
+    if (!handle || !ptr) return EP_ERR_INVALID_ARG;
+    cudaIpcMemHandle_t h;
+    std::memcpy(&h, handle, sizeof(h));
+    void *base = nullptr;
+    if (cudaIpcOpenMemHandle(&base, h, cudaIpcMemLazyEnablePeerAccess) != cudaSuccess)
+        return EP_ERR_CUDA;
+    *ptr = static_cast<uint8_t *>(base) + offset;
+    return EP_OK;
+}
+
+ep_status_t ep_ipc_close(void *base) {
+    if (!base) return EP_ERR_INVALID_ARG;
+    return cudaIpcCloseMemHandle(base) == cudaSuccess ? EP_OK : EP_ERR_CUDA;
+}
+
 ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream) {
     if (!dev_status || !host_flags) return EP_ERR_INVALID_ARG;
     cudaStream_t s = cs(stream);
@@ -1285,6 +1634,7 @@ ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_
     if (cudaStreamSynchronize(s) != cudaSuccess) return EP_ERR_CUDA;
     if (cudaMemsetAsync(dev_status, 0, sizeof(uint32_t), s) != cudaSuccess) return EP_ERR_CUDA;
     *host_flags = h;
+    if (h & EP_DEV_TIMEOUT) return EP_ERR_TIMEOUT;
     return h ? EP_ERR_DEVICE_STATUS : EP_OK;
 }
 

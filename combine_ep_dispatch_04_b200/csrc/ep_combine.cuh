@@ -35,6 +35,10 @@ struct CombineArgs {
     const int64_t *eo;
     uint16_t *out;
     uint32_t *status;
+    // expert parallelism over GPUs (ep_group.cuh): y is read from the window of
+    // the GPU that owns each virtual row; peer_y == nullptr on one GPU
+    const uint8_t *const *peer_y;  // [G] expert-output windows
+    int64_t win_rows;
 };
 
 enum { QIN_BF16 = 0, QIN_E4M3_B128 = 1, QIN_INT8 = 2, QIN_MXFP8 = 3, QIN_MXFP4 = 4 };
@@ -131,7 +135,8 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
     pdl_enter();
     constexpr int TOKS = block_threads(TPT) / TPT;
     constexpr int EPG = combine_granule(QIN);
-    __shared__ int64_t s_row[TOKS][16];
+    __shared__ int64_t s_row[TOKS][16];          // the row in its window (-1: none)
+    __shared__ const uint8_t *s_ybase[TOKS][16];  // the window: y, or the owner GPU's
     __shared__ float s_w[TOKS][16];
 
     const int grp = threadIdx.x / TPT, lt = threadIdx.x % TPT;
@@ -155,7 +160,14 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
             }
         }
         if (flags) atomicOr(a.status, flags);
+        const uint8_t *yb = reinterpret_cast<const uint8_t *>(a.y);
+        if (a.peer_y && row >= 0) {  // virtual row -> owner's window
+            const int o = (int)(row / a.win_rows);
+            row -= (int64_t)o * a.win_rows;
+            yb = a.peer_y[o];
+        }
         s_row[grp][lt] = row;
+        s_ybase[grp][lt] = yb;
         s_w[grp][lt] = a.wts[n * a.K + lt];
     }
     __syncthreads();
@@ -176,7 +188,9 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
                 for (int kk = 0; kk < KB; kk++) {
                     const int k = k0 + kk;
                     const int64_t row = k < a.K ? s_row[grp][k] : -1;
-                    buf[kk] = row >= 0 ? ld_stream(a.y + row * a.H + (int64_t)g * 8)
+                    buf[kk] = row >= 0 ? ld_stream(reinterpret_cast<const uint16_t *>(
+                                                       s_ybase[grp][k]) +
+                                                   row * a.H + (int64_t)g * 8)
                                        : make_uint4(0u, 0u, 0u, 0u);
                 }
 #pragma unroll
@@ -194,7 +208,6 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
             } else {
                 // quantised rows: 16 bytes of codes and their scale per entry,
                 // loaded for all KB entries before any use
-                const uint8_t *ybase = reinterpret_cast<const uint8_t *>(a.y);
                 uint4 raw[KB];
                 float sc[KB];
 #pragma unroll
@@ -204,6 +217,7 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
                     raw[kk] = make_uint4(0u, 0u, 0u, 0u);
                     sc[kk] = 0.0f;
                     if (row >= 0) {
+                        const uint8_t *ybase = s_ybase[grp][k];
                         const uint8_t *sp = ybase + a.scale_off + row * a.S;
                         raw[kk] = ld_stream(ybase + row * a.D + (int64_t)g * 16);
                         if constexpr (QIN == QIN_INT8) sc[kk] = __ldg(reinterpret_cast<const float *>(sp));

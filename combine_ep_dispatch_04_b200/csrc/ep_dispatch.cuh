@@ -20,6 +20,7 @@
 #pragma once
 
 #include "ep_device.cuh"
+#include "ep_group.cuh"
 
 namespace ep {
 
@@ -28,6 +29,7 @@ enum { Q_BF16 = 0, Q_E4M3_B128 = 1, Q_INT8 = 2, Q_MXFP8 = 3, Q_MXFP4 = 4 };
 struct DispatchArgs {
     int64_t N;
     int T, K, E, M, H;
+    int first_rank;          // logical rank of this GPU's first token (0 on one GPU)
     int packed;
     int64_t cap, rows;       // padded rows per expert, buffer row capacity
     int64_t D, S, scale_off; // row data bytes, row scale bytes, scale region offset
@@ -44,7 +46,36 @@ struct DispatchArgs {
     int32_t *src_info;
     float *recv_w;
     uint32_t *status;
+    // expert parallelism over GPUs (ep_group.cuh); peer_out == nullptr on one GPU
+    uint8_t *const *peer_out;  // [G] window bases (recv_buf / grad_buf of every GPU)
+    int32_t *const *peer_src;  // [G] source-info windows (dispatch)
+    float *const *peer_w;      // [G] weight windows (nullable)
+    int64_t win_rows;          // rows of one window: a virtual row's owner is row / win_rows
+    uint32_t *done;            // this GPU's block counter for the end-of-grid signal
+    uint64_t *const *flags;    // [G] flag words of every GPU
+    int flag_kind, grp_g, grp_G;
+    uint64_t epoch;
 };
+
+// Data and scale destinations of a (virtual) row: in this GPU's buffer, or in
+// the window of the GPU that owns the row.
+__device__ __forceinline__ void row_dest(const DispatchArgs &a, int64_t row, uint8_t *&dst,
+                                         uint8_t *&sdst, int32_t *&src, float *&rw,
+                                         int64_t &lrow) {
+    uint8_t *base = a.out;
+    src = a.src_info;
+    rw = a.recv_w;
+    lrow = row;
+    if (a.peer_out) {
+        const int o = (int)(row / a.win_rows);
+        lrow = row - (int64_t)o * a.win_rows;
+        base = a.peer_out[o];
+        src = a.peer_src ? a.peer_src[o] : nullptr;
+        rw = a.peer_w ? a.peer_w[o] : nullptr;
+    }
+    dst = base + lrow * a.D;
+    sdst = base + a.scale_off + lrow * a.S;
+}
 
 // Row of entry (n, k) in the receive layout, or -1 (masked, or no row).
 __device__ __forceinline__ int64_t entry_row(const DispatchArgs &a, int64_t n, int k,
@@ -111,11 +142,12 @@ __device__ __forceinline__ uint32_t q_i8(float v, float s) {
 // layout grid lets this grid launch only after its own wait for all earlier
 // work returned.  The slots are read after the wait.
 template <int MODE, int TPT, int GMAX>
-__global__ void __launch_bounds__(block_threads(TPT)) dispatch_kernel(DispatchArgs a) {
+__device__ __forceinline__ void dispatch_body(const DispatchArgs &a) {
     constexpr int TOKS = block_threads(TPT) / TPT;
     constexpr int WPG = TPT / 32;  // warps per token group
     constexpr int OB = GranOut<MODE>::bytes;
-    __shared__ int64_t s_row[TOKS][16];
+    __shared__ uint8_t *s_dst[TOKS][16];   // each entry's data row and scale row
+    __shared__ uint8_t *s_sdst[TOKS][16];
     __shared__ float s_red[TOKS][WPG];
 
     const int grp = threadIdx.x / TPT, lt = threadIdx.x % TPT;
@@ -134,7 +166,7 @@ __global__ void __launch_bounds__(block_threads(TPT)) dispatch_kernel(DispatchAr
     if (!a.early) pdl_enter();
     if (router) {
         r_e = a.idx[n * a.K + lt];
-        if (a.recv_w) r_w = a.wts[n * a.K + lt];
+        if (a.recv_w || a.peer_w) r_w = a.wts[n * a.K + lt];
         if (!a.early) r_s = a.slot[n * a.K + lt];
     }
 
@@ -279,20 +311,26 @@ __global__ void __launch_bounds__(block_threads(TPT)) dispatch_kernel(DispatchAr
         uint32_t flags = 0;
         const int64_t row = row_of_entry(a, r_e, r_s, flags);
         if (flags) atomicOr(a.status, flags);
-        s_row[grp][lt] = row;
+        uint8_t *dst = nullptr, *sdst = nullptr;
         if (row >= 0) {
-            a.src_info[row] = (int32_t)((n / a.T) * a.M + n % a.T);
-            if (a.recv_w) a.recv_w[row] = r_w;
+            int32_t *src;
+            float *rw;
+            int64_t lrow;
+            row_dest(a, row, dst, sdst, src, rw, lrow);
+            // source rank and token; a GPU of a group holds ranks first_rank ..
+            src[lrow] = (int32_t)((n / a.T + a.first_rank) * a.M + n % a.T);
+            if (rw) rw[lrow] = r_w;
         }
+        s_dst[grp][lt] = dst;
+        s_sdst[grp][lt] = sdst;
     }
     __syncthreads();
     if (!active) return;
     // scatter to every destination row
     for (int k = 0; k < a.K; k++) {
-        const int64_t row = s_row[grp][k];
-        if (row < 0) continue;
-        uint8_t *dst = a.out + row * a.D;
-        uint8_t *sdst = a.out + a.scale_off + row * a.S;
+        uint8_t *dst = s_dst[grp][k];
+        if (!dst) continue;
+        uint8_t *sdst = s_sdst[grp][k];
 #pragma unroll
         for (int i = 0; i < GMAX; i++) {
             const int g = i * TPT + lt;
@@ -327,13 +365,20 @@ __global__ void __launch_bounds__(block_threads(TPT)) dispatch_kernel(DispatchAr
     }
 }
 
+template <int MODE, int TPT, int GMAX>
+__global__ void __launch_bounds__(block_threads(TPT)) dispatch_kernel(DispatchArgs a) {
+    dispatch_body<MODE, TPT, GMAX>(a);
+    // over GPUs: the grid's last block tells every GPU that the rows are there
+    if (a.done) group_grid_done(a.done, a.flags, a.flag_kind, a.grp_g, a.grp_G, a.epoch);
+}
+
 // ---------------------------------------------------------------------------
 // Combine backward ("EP dispatch with unfused MXFP8 quantization",
 // Description): row(n,k) <- MXFP8(w[n,k] * g[n,:]).  The block maximum of
 // |fl(w*g_h)| equals fl(|w| * max|g_h|) because rounding is monotone and sign
 // symmetric, so it is taken once per token and scaled per entry.
 template <int TPT, int GMAX>
-__global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(DispatchArgs a) {
+__device__ __forceinline__ void combine_bwd_body(const DispatchArgs &a) {
     pdl_enter();
     constexpr int TOKS = block_threads(TPT) / TPT;
     static_assert(TPT >= 32, "a warp belongs to one token");
@@ -347,13 +392,19 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(Dispatc
     // Every warp reads the token's entries itself (lane k holds entry k) and
     // hands them out by shuffles: no block barrier stands between a warp's
     // gradient loads and its stores.  The first warp reports the flags.
-    int64_t my_row = -1;
+    uint8_t *my_dst = nullptr, *my_sdst = nullptr;
     float my_w = 0.0f;
     if (active && lane < a.K) {
         uint32_t flags = 0;
-        my_row = entry_row(a, n, lane, flags);
+        const int64_t row = entry_row(a, n, lane, flags);
         if (flags && lt < 32) atomicOr(a.status, flags);
         my_w = a.unweighted ? 1.0f : a.wts[n * a.K + lane];
+        if (row >= 0) {
+            int32_t *src;
+            float *rw;
+            int64_t lrow;
+            row_dest(a, row, my_dst, my_sdst, src, rw, lrow);
+        }
     }
 
     // the token's gradient row, unpacked to fp32 once for all its entries
@@ -402,12 +453,13 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(Dispatc
 
     const bool weighted = !a.unweighted;
     for (int k = 0; k < a.K; k++) {
-        const int64_t row = __shfl_sync(kFull, my_row, k);
+        uint8_t *dst = reinterpret_cast<uint8_t *>(
+            __shfl_sync(kFull, reinterpret_cast<uintptr_t>(my_dst), k));
+        uint8_t *sdst = reinterpret_cast<uint8_t *>(
+            __shfl_sync(kFull, reinterpret_cast<uintptr_t>(my_sdst), k));
         const float w = __shfl_sync(kFull, my_w, k);
-        if (row < 0) continue;
+        if (!dst) continue;
         const float aw = fabsf(w);
-        uint8_t *dst = a.out + row * (int64_t)a.H;
-        uint8_t *sdst = a.out + a.scale_off + row * (int64_t)(a.H >> 5);
 #pragma unroll
         for (int i = 0; i < GMAX; i++) {
             const int g = i * TPT + lt;
@@ -432,6 +484,12 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(Dispatc
             if ((g & 1) == 0) sdst[g >> 1] = (uint8_t)(X + 127);
         }
     }
+}
+
+template <int TPT, int GMAX>
+__global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(DispatchArgs a) {
+    combine_bwd_body<TPT, GMAX>(a);
+    if (a.done) group_grid_done(a.done, a.flags, a.flag_kind, a.grp_g, a.grp_G, a.epoch);
 }
 
 }  // namespace ep

@@ -65,6 +65,22 @@ class EpSizes(C.Structure):
         "grad_bytes", "workspace_bytes", "token_slot_bytes", "is_token_in_rank_bytes")]
 
 
+class EpGroupT(C.Structure):
+    _fields_ = [("world", C.c_int32), ("rank", C.c_int32), ("epoch", C.c_uint64)]
+
+
+class EpPeers(C.Structure):
+    """ep_peers_t: device arrays of G window pointers and this GPU's flags."""
+    _fields_ = [("recv", C.c_void_p), ("src_info", C.c_void_p), ("recv_weights", C.c_void_p),
+                ("y", C.c_void_p), ("grad", C.c_void_p), ("counts", C.c_void_p),
+                ("flags", C.c_void_p), ("my_counts", C.c_void_p), ("my_flags", C.c_void_p),
+                ("done", C.c_void_p)]
+
+
+GROUP_KIND_COUNTS, GROUP_KIND_DISPATCH, GROUP_KIND_EXPERT_OUT, GROUP_KIND_COMBINED, \
+    GROUP_KIND_BACKWARD = 0, 1, 2, 3, 4
+GROUP_KINDS = 5
+
 _P = C.c_void_p
 _Z = C.c_size_t
 _CFG = C.POINTER(EpConfig)
@@ -102,6 +118,32 @@ lib.ep_moe_forward_ffn.argtypes = [_CFG] + [_P] * 7 + [C.c_int32] + [_P] * 4 + \
     [_Z, _P, _Z, _P, _Z, _P, _Z, _P, _Z, _P, _P, _P]
 lib.ep_combine_backward_weights.restype = C.c_int
 lib.ep_combine_backward_weights.argtypes = [_CFG, _P, _P, _Z] + [_P] * 6
+_G = C.POINTER(EpGroupT)
+_PE = C.POINTER(EpPeers)
+lib.ep_group_sizes.restype = C.c_int
+lib.ep_group_sizes.argtypes = [_CFG, _G, C.POINTER(EpSizes)]
+lib.ep_group_layout.restype = C.c_int
+lib.ep_group_layout.argtypes = [_CFG, _G, _PE, _P, _P, _P, _Z, _P, _P]
+lib.ep_group_plan.restype = C.c_int
+lib.ep_group_plan.argtypes = [_CFG, _G, _PE, _P, _P, _P, _P, _P, _P, _Z, _P, _P]
+lib.ep_group_plan_host.restype = C.c_int
+lib.ep_group_plan_host.argtypes = [_CFG, _G, _P, _P, _P, _P]
+lib.ep_group_dispatch.restype = C.c_int
+lib.ep_group_dispatch.argtypes = [_CFG, _G, _PE, _P, _P, _P, _P, _P, _P, _P]
+lib.ep_group_combine.restype = C.c_int
+lib.ep_group_combine.argtypes = [_CFG, _G, _PE, _P, _P, _P, _P, _P, _P, _P]
+lib.ep_group_combine_backward.restype = C.c_int
+lib.ep_group_combine_backward.argtypes = [_CFG, _G, _PE, _P, _P, _P, _P, _P, _P, _P]
+lib.ep_group_signal.restype = C.c_int
+lib.ep_group_signal.argtypes = [_G, _PE, C.c_int32, _P]
+lib.ep_group_wait.restype = C.c_int
+lib.ep_group_wait.argtypes = [_G, _PE, C.c_int32, C.c_uint64, _P, _P]
+lib.ep_ipc_export.restype = C.c_int
+lib.ep_ipc_export.argtypes = [_P, _P, C.POINTER(C.c_uint64)]
+lib.ep_ipc_import.restype = C.c_int
+lib.ep_ipc_import.argtypes = [_P, C.c_uint64, C.POINTER(C.c_void_p)]
+lib.ep_ipc_close.restype = C.c_int
+lib.ep_ipc_close.argtypes = [_P]
 lib.ep_get_status.restype = C.c_int
 lib.ep_get_status.argtypes = [_P, C.POINTER(C.c_uint32), _P]
 lib.ep_copy.restype = C.c_int
@@ -518,9 +560,177 @@ def ep_get_status(dev_status, stream=None):
     flags = C.c_uint32(0)
     st = lib.ep_get_status(_dev(dev_status, "dev_status", torch.int32, (1,)), C.byref(flags),
                            _stream(stream))
-    if st not in (0, 5):
+    if st not in (0, 5, 6):
         raise EpError(st, "ep_get_status")
     return flags.value
+
+
+# ---- expert parallelism over GPUs (include/ep.h, ep_group_*) ----------------------
+def make_group(world, rank, epoch=1):
+    return EpGroupT(world, rank, epoch)
+
+
+def ep_group_sizes(cfg, grp):
+    s = EpSizes()
+    _check(lib.ep_group_sizes(C.byref(cfg), C.byref(grp), C.byref(s)), "ep_group_sizes")
+    return {n: getattr(s, n) for n, _ in EpSizes._fields_}
+
+
+def _gnk(cfg, grp):
+    return (cfg.num_ranks // grp.world) * cfg.num_tokens, cfg.num_topk
+
+
+def ep_group_layout(cfg, grp, peers, topk_idx, token_slot, workspace, dev_status, stream=None,
+                    bind=False):
+    """Local ranks of this GPU's entries; its per-rank counts to every GPU's
+    counts window (then the COUNTS signal)."""
+    n, K = _gnk(cfg, grp)
+    args = [C.byref(peers),
+            _dev(topk_idx, "topk_idx", idx_dtype(cfg), (n, K)),
+            _dev(token_slot, "token_slot", torch.int32, (n, K)),
+            *_buf(workspace, "workspace"),
+            _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream)]
+    return _gcall(lib.ep_group_layout, cfg, grp, args, "ep_group_layout", bind)
+
+
+def ep_group_plan(cfg, grp, peers, topk_idx, token_slot, recv_count, expert_offset, slot_scratch,
+                  dev_status, cumulative_recv_stats=None, stream=None, bind=False):
+    """After every GPU's counts: global slots, totals and virtual packed offsets."""
+    n, K = _gnk(cfg, grp)
+    E = cfg.num_experts
+    args = [C.byref(peers),
+            _dev(topk_idx, "topk_idx", idx_dtype(cfg), (n, K)),
+            _dev(token_slot, "token_slot", torch.int32, (n, K)),
+            _dev(recv_count, "recv_count", torch.int64, (E,)),
+            _dev(expert_offset, "expert_offset", torch.int64, (E + 1,),
+                 optional=cfg.layout == LAYOUT["padded"]),
+            _dev(cumulative_recv_stats, "cumulative_recv_stats", torch.int64, (E,), optional=True),
+            *_buf(slot_scratch, "slot_scratch"),
+            _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream)]
+    return _gcall(lib.ep_group_plan, cfg, grp, args, "ep_group_plan", bind)
+
+
+def ep_group_plan_host(cfg, grp, tokens_per_expert_all):
+    """The plan on the host (numpy): (slot_base [E], recv_count [E], expert_offset [E+1])."""
+    import numpy as np
+    E = cfg.num_experts
+    tpe = np.ascontiguousarray(tokens_per_expert_all, np.int32)
+    assert tpe.shape == (cfg.num_ranks, E)
+    base, cnt = np.zeros(E, np.int64), np.zeros(E, np.int64)
+    eo = np.zeros(E + 1, np.int64)
+    p = lambda a: a.ctypes.data_as(C.c_void_p)  # noqa: E731
+    _check(lib.ep_group_plan_host(C.byref(cfg), C.byref(grp), p(tpe), p(base), p(cnt), p(eo)),
+           "ep_group_plan_host")
+    return base, cnt, eo
+
+
+def ep_group_dispatch(cfg, grp, peers, x, topk_idx, token_slot, dev_status, topk_weights=None,
+                      expert_offset=None, stream=None, bind=False):
+    n, K = _gnk(cfg, grp)
+    args = [C.byref(peers),
+            _dev(x, "x", torch.bfloat16, (n, cfg.hidden)),
+            _dev(topk_idx, "topk_idx", idx_dtype(cfg), (n, K)),
+            _dev(topk_weights, "topk_weights", torch.float32, (n, K), optional=True),
+            _dev(token_slot, "token_slot", torch.int32, (n, K)),
+            _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
+                 optional=cfg.layout == LAYOUT["padded"]),
+            _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream)]
+    return _gcall(lib.ep_group_dispatch, cfg, grp, args, "ep_group_dispatch", bind)
+
+
+def ep_group_combine(cfg, grp, peers, topk_idx, topk_weights, token_slot, out, dev_status,
+                     expert_offset=None, stream=None, bind=False):
+    n, K = _gnk(cfg, grp)
+    args = [C.byref(peers),
+            _dev(topk_idx, "topk_idx", idx_dtype(cfg), (n, K)),
+            _dev(topk_weights, "topk_weights", torch.float32, (n, K)),
+            _dev(token_slot, "token_slot", torch.int32, (n, K)),
+            _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
+                 optional=cfg.layout == LAYOUT["padded"]),
+            _dev(out, "out", torch.bfloat16, (n, cfg.hidden)),
+            _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream)]
+    return _gcall(lib.ep_group_combine, cfg, grp, args, "ep_group_combine", bind)
+
+
+def ep_group_combine_backward(cfg, grp, peers, g, topk_idx, topk_weights, token_slot, dev_status,
+                              expert_offset=None, stream=None, bind=False):
+    n, K = _gnk(cfg, grp)
+    args = [C.byref(peers),
+            _dev(g, "g", torch.bfloat16, (n, cfg.hidden)),
+            _dev(topk_idx, "topk_idx", idx_dtype(cfg), (n, K)),
+            _dev(topk_weights, "topk_weights", torch.float32, (n, K),
+                 optional=bool(cfg.flags & F_BWD_UNWEIGHTED)),
+            _dev(token_slot, "token_slot", torch.int32, (n, K)),
+            _dev(expert_offset, "expert_offset", torch.int64, (cfg.num_experts + 1,),
+                 optional=cfg.layout == LAYOUT["padded"]),
+            _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream)]
+    return _gcall(lib.ep_group_combine_backward, cfg, grp, args, "ep_group_combine_backward",
+                  bind)
+
+
+def ep_group_signal(grp, peers, kind, stream=None, bind=False):
+    args = [C.byref(peers), C.c_int32(int(kind)), _stream(stream)]
+    if bind:
+        return _Plain(lib.ep_group_signal, [C.byref(grp)] + args, "ep_group_signal")
+    _check(lib.ep_group_signal(C.byref(grp), *args), "ep_group_signal")
+
+
+def ep_group_wait(grp, peers, kind, dev_status, timeout_ns=0, stream=None, bind=False):
+    args = [C.byref(peers), C.c_int32(int(kind)), C.c_uint64(int(timeout_ns)),
+            _dev(dev_status, "dev_status", torch.int32, (1,)), _stream(stream)]
+    if bind:
+        return _Plain(lib.ep_group_wait, [C.byref(grp)] + args, "ep_group_wait")
+    _check(lib.ep_group_wait(C.byref(grp), *args), "ep_group_wait")
+
+
+class _Plain:
+    """A bound call without a configuration argument."""
+
+    def __init__(self, fn, args, where):
+        self._fn, self._args, self._where = fn, tuple(args), where
+
+    def __call__(self):
+        st = self._fn(*self._args)
+        if st != 0:
+            raise EpError(st, self._where)
+
+
+class _GBound(Bound):
+    def __init__(self, fn, cfg, grp, args, where):
+        super().__init__(fn, cfg, args, where)
+        self._grp = C.byref(grp)
+
+    def __call__(self):
+        st = self._fn(self._ref, self._grp, *self._args)
+        if st != 0:
+            raise EpError(st, self._where)
+
+
+def _gcall(fn, cfg, grp, args, where, bind):
+    if bind:
+        return _GBound(fn, cfg, grp, args, where)
+    _check(fn(C.byref(cfg), C.byref(grp), *args), where)
+    return None
+
+
+def ep_ipc_export(t):
+    """(64-byte handle, offset) of a CUDA tensor's memory, for another process."""
+    h = (C.c_uint8 * 64)()
+    off = C.c_uint64(0)
+    _check(lib.ep_ipc_export(C.c_void_p(t.data_ptr()), h, C.byref(off)), "ep_ipc_export")
+    return bytes(h), off.value
+
+
+def ep_ipc_import(handle, offset):
+    """Device address of another process's exported memory, mapped here."""
+    h = (C.c_uint8 * 64).from_buffer_copy(handle)
+    p = C.c_void_p(0)
+    _check(lib.ep_ipc_import(h, int(offset), C.byref(p)), "ep_ipc_import")
+    return p.value
+
+
+def ep_ipc_close(base):
+    _check(lib.ep_ipc_close(C.c_void_p(base)), "ep_ipc_close")
 
 
 def ep_copy(dst, src, stream=None):

@@ -4,6 +4,7 @@
  *
  * On one GPU the R "ranks" of expert parallelism are logical partitions of
  * buffers that all sit in this GPU's memory: no inter-GPU traffic exists.
+ * The ep_group_* calls (near the end) split the same ranks over several GPUs.
  * Token n = r*T + t is token t of source rank r.  Expert e (of E) lives on
  * rank e / L, L = E / R, as local expert e % L.
  *
@@ -65,7 +66,7 @@ typedef enum {
     EP_ERR_MISALIGNED = 3,    /* a vector buffer is not 16-byte aligned */
     EP_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, copy, sync) */
     EP_ERR_DEVICE_STATUS = 5, /* ep_get_status found device-side error bits */
-    EP_ERR_TIMEOUT = 6,       /* reserved for bounded waits (multi-GPU); not produced */
+    EP_ERR_TIMEOUT = 6,       /* ep_get_status: a bounded wait gave up (EP_DEV_TIMEOUT) */
     EP_ERR_BUFFER_TOO_SMALL = 7 /* a *_bytes argument is below what the configuration needs */
 } ep_status_t;
 
@@ -90,7 +91,7 @@ typedef enum {
 /* Bits of *dev_status. */
 #define EP_DEV_BAD_INDEX 0x1u         /* topk_idx value < -1 or >= E (entry skipped) */
 #define EP_DEV_CAPACITY_OVERFLOW 0x2u /* slot >= R*M in the padded layout (row skipped) */
-#define EP_DEV_TIMEOUT 0x4u           /* a bounded wait inside ep_expert_gemm(_mx) gave up */
+#define EP_DEV_TIMEOUT 0x4u           /* a bounded wait (tensor-core kernels, ep_group_wait) gave up */
 
 /* ep_config_t.flags */
 #define EP_F_BWD_UNWEIGHTED 0x1u    /* combine-backward re-dispatches g without w */
@@ -495,8 +496,149 @@ ep_status_t ep_dispatch_layout_static(const ep_config_t *cfg, const void *topk_i
                                       int64_t *cumulative_recv_stats, uint32_t *dev_status,
                                       ep_stream_t stream);
 
+/*
+ * ---- Expert parallelism over G GPUs (one process per GPU, NVLink peer memory)
+ * ("Low-Latency Mode API": each rank dispatches its tokens into the receive
+ * buffers of the ranks that own their experts and combines the experts'
+ * outputs back; "[Common][PyTorch] EP dispatch with unfused MXFP8
+ * quantization", Changes: symmetric-memory windows, combine forward and
+ * backward as the reverse of the dispatch.)
+ *
+ * Partitioning.  `cfg` describes the whole job (R ranks of T tokens, E
+ * experts).  GPU g of G (R % G == 0) holds the tokens of ranks g*RG ..
+ * (g+1)*RG - 1, RG = R/G (its N_loc = RG*T tokens: x, topk_idx, topk_weights,
+ * token_slot and out are [N_loc] arrays), and owns experts g*EG .. (g+1)*EG - 1,
+ * EG = E/G.  Every GPU has one window per buffer kind, all of ep_group_sizes()'s
+ * `rows` rows in the single-GPU row format: receive window (data then scales),
+ * source info, optional weights, expert outputs y, gradient window.  Rows are
+ * numbered virtually: row r of GPU o's window is o*rows + r; expert_offset and
+ * the padded addressing e*R*M + slot are virtual rows.  Slots are global
+ * (ranked over all GPUs' entries of the expert in (source rank, token, k)
+ * order), so every GPU's window holds what one GPU's buffer would hold for
+ * those experts, row for row.
+ *
+ * One step, every GPU (epoch = 1, 2, ... one more each step; flags are never
+ * reset), all of it in this library's kernels over peer memory:
+ *   ep_group_layout      local ranks of this GPU's entries and its per-rank
+ *                        counts, stored into every GPU's counts window
+ *                        (signal COUNTS)
+ *   ep_group_plan        waits for every GPU's counts, then global slots,
+ *                        totals and virtual packed offsets
+ *   ep_group_dispatch    quantise and store rows into the owners' windows;
+ *                        the grid's last block signals every GPU (DISPATCH)
+ *   ep_group_wait(DISPATCH)              every GPU's rows have arrived
+ *   (the experts of this GPU write y in its window)
+ *   ep_group_signal / wait(EXPERT_OUT)   every GPU's expert outputs are there
+ *   ep_group_combine     read the tokens' rows from the owners' y windows
+ *   ep_group_signal / wait(COMBINED)     windows may be reused next step
+ * and for the backward: ep_group_combine_backward (stores into the owners'
+ * gradient windows, signals BACKWARD), ep_group_wait(BACKWARD).
+ * Waits are bounded: one that gives up sets EP_DEV_TIMEOUT, and ep_get_status
+ * then returns EP_ERR_TIMEOUT; kernels never trap.  Windows of other GPUs
+ * are mapped with ep_ipc_export / ep_ipc_import.  No transfer uses TMA
+ * multicast; stores and loads to peers are plain 16-byte accesses.
+ */
+#define EP_GROUP_KIND_COUNTS 0
+#define EP_GROUP_KIND_DISPATCH 1
+#define EP_GROUP_KIND_EXPERT_OUT 2
+#define EP_GROUP_KIND_COMBINED 3
+#define EP_GROUP_KIND_BACKWARD 4
+#define EP_GROUP_KINDS 5
+
+typedef struct {
+    int32_t world;  /* G, 1 .. 64, R % G == 0 */
+    int32_t rank;   /* this GPU, 0 .. G-1 */
+    uint64_t epoch; /* step number, >= 1, the same on every GPU */
+} ep_group_t;
+
+/* Every GPU's windows as this process sees them: device arrays of G device
+ * pointers (entry g: GPU g's window, mapped into this process), written once
+ * at set-up.  Window layouts as ep_group_sizes(). */
+typedef struct {
+    void *const *recv;            /* receive windows (data, then scales at recv_scale_offset) */
+    int32_t *const *src_info;     /* int32 [rows]: global r*M + t of each row's token */
+    float *const *recv_weights;   /* float [rows] or NULL (array pointer NULL: not written) */
+    const void *const *y;         /* bf16 [rows][H] expert outputs */
+    void *const *grad;            /* gradient windows (MXFP8, as ep_combine_backward) or NULL */
+    int32_t *const *counts;       /* int32 [R][E] counts tables of every GPU */
+    uint64_t *const *flags;       /* uint64 [EP_GROUP_KINDS][G] flag words of every GPU */
+    int32_t *my_counts;           /* this GPU's counts table (its entry of `counts`) */
+    uint64_t *my_flags;           /* this GPU's flag words (zero before the first step) */
+    uint32_t *done;               /* uint32 [EP_GROUP_KINDS] block counters, zero before first use */
+} ep_peers_t;
+
+/* Sizes for GPU grp->rank: `rows` and every *_bytes of one window, the
+ * workspace of ep_group_layout, token_slot_bytes of N_loc*K (no
+ * is_token_in_rank over GPUs). */
+ep_status_t ep_group_sizes(const ep_config_t *cfg, const ep_group_t *grp, ep_sizes_t *out);
+/* This GPU's entries ranked within their experts (the single-GPU layout over
+ * its RG ranks: token_slot int32 [N_loc][K] receives local ranks, which
+ * ep_group_plan makes global) and its per-rank counts: rows g*RG .. of the
+ * [R][E] counts table (tokens_per_expert of ep_dispatch_layout), written in
+ * its own counts window and stored into every other GPU's, then the COUNTS
+ * signal. */
+ep_status_t ep_group_layout(const ep_config_t *cfg, const ep_group_t *grp,
+                            const ep_peers_t *peers, const void *topk_idx, int32_t *token_slot,
+                            void *workspace, size_t workspace_bytes, uint32_t *dev_status,
+                            ep_stream_t stream);
+/* Waits (bounded) for every GPU's COUNTS, then from the [R][E] table:
+ * token_slot += the entries the ranks before this GPU's send to the same
+ * expert; recv_count int64 [E] = entries of each expert over all GPUs;
+ * expert_offset int64 [E+1] = virtual packed offsets (each owner's experts in
+ * order, rounded up to expert_align; [E] = G*rows; required when packed);
+ * cumulative_recv_stats [E] += recv_count of this GPU's experts (nullable).
+ * workspace: 8*E bytes of scratch.  E <= 1024. */
+ep_status_t ep_group_plan(const ep_config_t *cfg, const ep_group_t *grp,
+                          const ep_peers_t *peers, const void *topk_idx, int32_t *token_slot,
+                          int64_t *recv_count, int64_t *expert_offset,
+                          int64_t *cumulative_recv_stats, void *workspace, size_t workspace_bytes,
+                          uint32_t *dev_status, ep_stream_t stream);
+/* The same plan on the host (host pointers, no device work): slot_base [E]
+ * (the shift of this GPU's slots), recv_count [E], expert_offset [E+1]. */
+ep_status_t ep_group_plan_host(const ep_config_t *cfg, const ep_group_t *grp,
+                               const int32_t *tokens_per_expert_all, int64_t *slot_base,
+                               int64_t *recv_count, int64_t *expert_offset);
+/* ep_dispatch of this GPU's tokens into the owners' windows (peers->recv,
+ * src_info, recv_weights), then the EP_GROUP_KIND_DISPATCH signal. */
+ep_status_t ep_group_dispatch(const ep_config_t *cfg, const ep_group_t *grp,
+                              const ep_peers_t *peers, const uint16_t *x, const void *topk_idx,
+                              const float *topk_weights, const int32_t *token_slot,
+                              const int64_t *expert_offset, uint32_t *dev_status,
+                              ep_stream_t stream);
+/* ep_combine of this GPU's tokens, reading each entry's bf16 row from its
+ * owner's y window (EP_F_COMBINE_QUANTIZED unsupported). */
+ep_status_t ep_group_combine(const ep_config_t *cfg, const ep_group_t *grp,
+                             const ep_peers_t *peers, const void *topk_idx,
+                             const float *topk_weights, const int32_t *token_slot,
+                             const int64_t *expert_offset, uint16_t *out, uint32_t *dev_status,
+                             ep_stream_t stream);
+/* ep_combine_backward of this GPU's tokens into the owners' gradient
+ * windows, then the EP_GROUP_KIND_BACKWARD signal. */
+ep_status_t ep_group_combine_backward(const ep_config_t *cfg, const ep_group_t *grp,
+                                      const ep_peers_t *peers, const uint16_t *g,
+                                      const void *topk_idx, const float *topk_weights,
+                                      const int32_t *token_slot, const int64_t *expert_offset,
+                                      uint32_t *dev_status, ep_stream_t stream);
+/* Tell every GPU that this GPU's work of `kind` for grp->epoch is done (its
+ * earlier writes in stream order are visible to a GPU that sees the flag). */
+ep_status_t ep_group_signal(const ep_group_t *grp, const ep_peers_t *peers, int32_t kind,
+                            ep_stream_t stream);
+/* Wait (on the device, in stream order) until every GPU has signalled `kind`
+ * for grp->epoch; gives up after timeout_ns (0: 2 s; at most 10 s), sets
+ * EP_DEV_TIMEOUT in *dev_status and returns. */
+ep_status_t ep_group_wait(const ep_group_t *grp, const ep_peers_t *peers, int32_t kind,
+                          uint64_t timeout_ns, uint32_t *dev_status, ep_stream_t stream);
+/* CUDA IPC of windows: export gives the 64-byte handle of the allocation that
+ * holds ptr and ptr's offset in it; import (in another process) maps it and
+ * returns the same address's mapping; close unmaps (pass the mapping's base,
+ * i.e. the imported pointer minus its offset). */
+ep_status_t ep_ipc_export(const void *ptr, uint8_t *handle, uint64_t *offset);
+ep_status_t ep_ipc_import(const uint8_t *handle, uint64_t offset, void **ptr);
+ep_status_t ep_ipc_close(void *base);
+
 /* Synchronise `stream`, read *dev_status into *host_flags (host pointer) and
- * clear it.  Returns EP_ERR_DEVICE_STATUS when any bit was set. */
+ * clear it.  Returns EP_ERR_TIMEOUT when EP_DEV_TIMEOUT was set,
+ * else EP_ERR_DEVICE_STATUS when any bit was set. */
 ep_status_t ep_get_status(uint32_t *dev_status, uint32_t *host_flags, ep_stream_t stream);
 
 /* Static description of a status code. */

@@ -265,6 +265,8 @@ def dispatch(R, T, K, E, M, H, mode, x, topk_idx, token_slot, expert_offset=None
     if out is None:
         out = dispatch_buffers(R, T, K, E, M, H, m, layout, align, weights=w is not None)
     out = dict(out)
+    if eo is not None and layout in ("packed", 1):  # the rows the offsets address must exist
+        assert int(eo[-1]) <= out["recv_data"].shape[0], "expert_offset beyond the buffers' rows"
     st = _lib.orc_dispatch(R, T, K, E, M, H, m, float(e4m3_qmax), _layout(layout), _ptr(x),
                            _ptr(idx), _ptr(w), _ptr(slot), _ptr(eo), _ptr(out["recv_data"]),
                            _ptr(out["recv_scale"]), _ptr(out["src_info"]), _ptr(out["recv_weights"]))
