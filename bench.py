@@ -76,6 +76,11 @@ def parse():
     p.add_argument("--quantized-combine", action="store_true",
                    help="combine reads expert outputs stored in the dispatch format")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--ep-group", action="store_true",
+                   help="run the expert-parallel group path also on one GPU (a group of one)")
+    p.add_argument("--replicas", action="store_true",
+                   help="with --gpus N > 1: N independent single-GPU replicas instead of one "
+                        "expert-parallel job over the N GPUs")
     p.add_argument("--no-workloads", action="store_true",
                    help="skip the per-kernel pass over the other named workloads")
     p.add_argument("--gemm-workload", default="decode", choices=sorted(synth.WORKLOADS),
@@ -509,6 +514,109 @@ class WorkloadRun:
         torch.cuda.empty_cache()
 
 
+def run_group_bench(ep, args, wname, world, rank, local, dev):
+    """One expert-parallel job over the N GPUs (weak scaling): every GPU holds
+    the named workload's R ranks of T tokens (the job has R * N ranks and the
+    workload's E experts, E / N on each GPU), its tokens drawn with its own
+    replica of the routing and activations.  A step is the library's group
+    path: layout with the counts exchange, plan, dispatch into the owners'
+    windows over NVLink, (the expert outputs stand in the windows), combine
+    from the owners' windows, and the combine-backward for the prefill
+    workload; every transfer and wait is in the library's kernels.  Timed with
+    CUDA events on the stream, L2 flushed before each step, max over ranks."""
+    import torch.distributed as dist
+
+    from combine_ep_dispatch_04_b200.group import EpGroup
+    w1 = synth.workload(wname) if args.tokens_per_rank is None else \
+        synth.workload(wname, T=args.tokens_per_rank)
+    mode = WORKLOAD_MODE[wname]
+    R1, T, M, K, E, H = w1["R"], w1["T"], w1["M"], w1["K"], w1["E"], w1["H"]
+    R = R1 * world
+    if E % R:
+        raise SystemExit(f"{wname}: {E} experts cannot be split over {R} ranks")
+    cfg = ep.make_config(R, T, M, K, E, H, mode, w1["layout"])
+    n_loc = R1 * T
+    stream = torch.cuda.current_stream(dev)
+    idx, wts = synth.make_routing(w1, rank)
+    x = synth.make_x(w1, rank)
+    idx_d, wts_d = torch.from_numpy(idx).to(dev), torch.from_numpy(wts).to(dev)
+    x_d = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+    backward = bool(w1.get("backward"))
+    g_d = None
+    if backward:
+        gp, go = synth.g_source(w1, rank)
+        g_d = torch.from_numpy(synth.windows(gp, go, H).view(np.int16)).to(dev).view(torch.bfloat16)
+    # packed windows for the expected load (each owner receives about n_loc * K
+    # rows under uniform routing) with room to spare; padded: fixed by R * M
+    slack = 2.0 if w1["routing"] == "zipf" else 1.5
+    win = int(slack * n_loc * K) + (E // world) * 8 if w1["layout"] == "packed" else 0
+    eg = EpGroup(cfg, device=dev, grad=backward, stream=stream, timeout_ns=5_000_000_000,
+                 window_rows=win)
+    ypool, yoff = synth.y_source(w1, eg.win.sizes["rows"], rank)
+    pool_d = torch.from_numpy(ypool.view(np.int16)).to(dev)
+    torch.index_select(pool_d.as_strided((synth.POOL, H), (1, 1)), 0,
+                       torch.from_numpy(yoff).to(dev), out=eg.win.y.view(torch.int16))
+    del pool_d
+    out = torch.empty((n_loc, H), dtype=torch.bfloat16, device=dev)
+    flush_w = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+    flush_r = torch.ones(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        eg.dispatch(x_d, idx_d, wts_d)
+        eg.combine(idx_d, wts_d, out)
+        if backward:
+            ep.ep_group_combine_backward(cfg, eg.grp, eg.peers, g_d, idx_d, wts_d, eg.token_slot,
+                                         eg.dev_status, expert_offset=eg.expert_offset,
+                                         stream=stream)
+            ep.ep_group_wait(eg.grp, eg.peers, ep.GROUP_KIND_BACKWARD, eg.dev_status,
+                             eg.timeout_ns, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush_w.fill_(1)
+        flush_r.max()
+        step()
+    torch.cuda.synchronize(dev)
+    if eg.status() != 0:
+        raise SystemExit("device status reported errors during warm-up (timeout or capacity)")
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    launches0 = ep.ep_kernel_launches()
+    with clocks:
+        for s_ in range(args.steps):
+            flush_w.fill_(s_ & 0xFF)
+            flush_r.max()
+            evs[s_][0].record(stream)
+            step()
+            evs[s_][1].record(stream)
+        torch.cuda.synchronize(dev)
+    launches = ep.ep_kernel_launches() - launches0
+    barrier(world)
+    total_ms = max_over_ranks(sum(a.elapsed_time(c) for a, c in evs), world)
+    bad = max_over_ranks(float(eg.status() != 0), world)
+    eg.close()
+    ms = total_ms / args.steps
+    if rank == 0:
+        out_line = {
+            "metric": METRIC, "value": round(world * n_loc * args.steps / (total_ms / 1e3), 1),
+            "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": f"{wname}: {R1} ranks x T={T} a GPU ({R} ranks), H={H} K={K} "
+                                   f"E={E} M={M} {mode} {w1['layout']}",
+                       "tokens_per_step": world * n_loc,
+                       "parallelism": f"ep{world}: expert parallel over NVLink peer memory",
+                       "window_rows": eg.win.sizes["rows"],
+                       "l2": "flushed before each step outside the events"},
+            "clocks": clocks.report(), "gpu_launches": launches,
+            "device_status_clean": bad == 0.0,
+        }
+        print(json.dumps(out_line), flush=True)
+    dist_done(world)
+
+
 def run_ffn_leg(ep, flush, stream, dev, args, replica):
     """The deep fused MoE page's benchmark case on one GPU ("[feat] A5 deep fused
     moe supported", Benchmarking: EP 8, hidden 7168, moe-intermediate-size 3072,
@@ -746,6 +854,9 @@ def main():
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if (world > 1 and not args.replicas) or args.ep_group:
+        run_group_bench(ep, args, wname, world, rank, local, dev)
+        return
     if args.weights_grad and args.quantized_combine:
         raise SystemExit("--weights-grad reads bf16 expert outputs: not with --quantized-combine")
     stream = torch.cuda.current_stream(dev)

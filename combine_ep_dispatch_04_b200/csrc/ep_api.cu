@@ -1298,9 +1298,14 @@ ep_status_t make_group(const ep_config_t *cfg, const ep_group_t *grp, Plan &p,
         return EP_ERR_INVALID_ARG;
     s.R = p.R; s.E = p.E; s.G = grp->world; s.g = grp->rank;
     s.RG = p.R / s.G; s.EG = p.E / s.G;
-    s.win_rows = cfg->layout == EP_LAYOUT_PACKED
-                     ? p.N * p.K + (int64_t)s.EG * (cfg->expert_align - 1)
-                     : (int64_t)s.EG * p.cap;
+    if (cfg->layout == EP_LAYOUT_PACKED) {  // every entry, unless the caller sizes it
+        const int64_t all = p.N * p.K + (int64_t)s.EG * (cfg->expert_align - 1);
+        if (grp->window_rows < 0) return EP_ERR_INVALID_ARG;
+        s.win_rows = grp->window_rows > 0 ? std::min(grp->window_rows, all) : all;
+    } else {  // the padded addressing fixes it
+        s.win_rows = (int64_t)s.EG * p.cap;
+        if (grp->window_rows != 0 && grp->window_rows != s.win_rows) return EP_ERR_INVALID_ARG;
+    }
     if ((int64_t)s.G * s.win_rows > kIntLimit) return EP_ERR_INVALID_ARG;  // int32 slots
     return EP_OK;
 }
@@ -1485,6 +1490,7 @@ ep_status_t ep_group_dispatch(const ep_config_t *cfg, const ep_group_t *grp,
     a.peer_src = peers->src_info;
     a.peer_w = peers->recv_weights;
     a.win_rows = s.win_rows;
+    a.experts_per_gpu = s.EG;
     a.done = peers->done + ep::kFlagDispatch;
     a.flags = peers->flags;
     a.flag_kind = ep::kFlagDispatch;
@@ -1519,6 +1525,7 @@ ep_status_t ep_group_combine(const ep_config_t *cfg, const ep_group_t *grp,
     a.out = out; a.status = dev_status;
     a.peer_y = reinterpret_cast<const uint8_t *const *>(peers->y);
     a.win_rows = s.win_rows;
+    a.experts_per_gpu = s.EG;
     return launch_combine<ep::QIN_BF16>(a, cs(stream));
 }
 
@@ -1554,6 +1561,7 @@ ep_status_t ep_group_combine_backward(const ep_config_t *cfg, const ep_group_t *
     a.status = dev_status;
     a.peer_out = reinterpret_cast<uint8_t *const *>(peers->grad);
     a.win_rows = s.win_rows;
+    a.experts_per_gpu = s.EG;
     a.done = peers->done + ep::kFlagBackward;
     a.flags = peers->flags;
     a.flag_kind = ep::kFlagBackward;

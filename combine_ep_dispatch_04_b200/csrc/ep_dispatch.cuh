@@ -50,53 +50,41 @@ struct DispatchArgs {
     uint8_t *const *peer_out;  // [G] window bases (recv_buf / grad_buf of every GPU)
     int32_t *const *peer_src;  // [G] source-info windows (dispatch)
     float *const *peer_w;      // [G] weight windows (nullable)
-    int64_t win_rows;          // rows of one window: a virtual row's owner is row / win_rows
+    int64_t win_rows;          // rows of one window
+    int experts_per_gpu;       // an expert's owner is e / experts_per_gpu
     uint32_t *done;            // this GPU's block counter for the end-of-grid signal
     uint64_t *const *flags;    // [G] flag words of every GPU
     int flag_kind, grp_g, grp_G;
     uint64_t epoch;
 };
 
-// Data and scale destinations of a (virtual) row: in this GPU's buffer, or in
-// the window of the GPU that owns the row.
-__device__ __forceinline__ void row_dest(const DispatchArgs &a, int64_t row, uint8_t *&dst,
-                                         uint8_t *&sdst, int32_t *&src, float *&rw,
-                                         int64_t &lrow) {
+// Data and scale destinations of expert e's (virtual) row: in this GPU's
+// buffer, or in the window of the GPU that owns e.  False (and the capacity
+// bit) when the row lies past the end of the owner's window.
+__device__ __forceinline__ bool row_dest(const DispatchArgs &a, int64_t e, int64_t row,
+                                         uint8_t *&dst, uint8_t *&sdst, int32_t *&src,
+                                         float *&rw, int64_t &lrow, uint32_t &flags) {
     uint8_t *base = a.out;
     src = a.src_info;
     rw = a.recv_w;
     lrow = row;
     if (a.peer_out) {
-        const int o = (int)(row / a.win_rows);
+        const int o = (int)(e / a.experts_per_gpu);
         lrow = row - (int64_t)o * a.win_rows;
+        if (lrow < 0 || lrow >= a.win_rows) {
+            flags |= kDevCapacity;
+            return false;
+        }
         base = a.peer_out[o];
         src = a.peer_src ? a.peer_src[o] : nullptr;
         rw = a.peer_w ? a.peer_w[o] : nullptr;
     }
     dst = base + lrow * a.D;
     sdst = base + a.scale_off + lrow * a.S;
+    return true;
 }
 
-// Row of entry (n, k) in the receive layout, or -1 (masked, or no row).
-__device__ __forceinline__ int64_t entry_row(const DispatchArgs &a, int64_t n, int k,
-                                             uint32_t &flags) {
-    const int64_t e = a.idx[n * a.K + k];
-    if (e < -1 || e >= a.E) flags |= kDevBadIndex;
-    if (e < 0 || e >= a.E) return -1;
-    const int32_t s = a.slot[n * a.K + k];
-    if (s < 0) return -1;
-    int64_t row;
-    if (!a.packed) {
-        if (s >= a.cap) { flags |= kDevCapacity; return -1; }
-        row = e * a.cap + s;
-    } else {
-        row = a.eo[e] + s;
-        if (row >= a.eo[e + 1] || row >= a.rows) { flags |= kDevCapacity; return -1; }
-    }
-    return row;
-}
-
-// The same from an expert index and slot already loaded.
+// Row of entry (expert e, slot s) in the receive layout, or -1 (masked, or no row).
 __device__ __forceinline__ int64_t row_of_entry(const DispatchArgs &a, int64_t e, int32_t s,
                                                 uint32_t &flags) {
     if (e < -1 || e >= a.E) flags |= kDevBadIndex;
@@ -310,17 +298,16 @@ __device__ __forceinline__ void dispatch_body(const DispatchArgs &a) {
     if (router) {
         uint32_t flags = 0;
         const int64_t row = row_of_entry(a, r_e, r_s, flags);
-        if (flags) atomicOr(a.status, flags);
         uint8_t *dst = nullptr, *sdst = nullptr;
-        if (row >= 0) {
-            int32_t *src;
-            float *rw;
-            int64_t lrow;
-            row_dest(a, row, dst, sdst, src, rw, lrow);
+        int32_t *src;
+        float *rw;
+        int64_t lrow;
+        if (row >= 0 && row_dest(a, r_e, row, dst, sdst, src, rw, lrow, flags)) {
             // source rank and token; a GPU of a group holds ranks first_rank ..
             src[lrow] = (int32_t)((n / a.T + a.first_rank) * a.M + n % a.T);
             if (rw) rw[lrow] = r_w;
         }
+        if (flags) atomicOr(a.status, flags);
         s_dst[grp][lt] = dst;
         s_sdst[grp][lt] = sdst;
     }
@@ -396,15 +383,17 @@ __device__ __forceinline__ void combine_bwd_body(const DispatchArgs &a) {
     float my_w = 0.0f;
     if (active && lane < a.K) {
         uint32_t flags = 0;
-        const int64_t row = entry_row(a, n, lane, flags);
-        if (flags && lt < 32) atomicOr(a.status, flags);
+        const int64_t e = a.idx[n * a.K + lane];
+        const int32_t sl = (e >= 0 && e < a.E) ? a.slot[n * a.K + lane] : -1;
+        const int64_t row = row_of_entry(a, e, sl, flags);
         my_w = a.unweighted ? 1.0f : a.wts[n * a.K + lane];
         if (row >= 0) {
             int32_t *src;
             float *rw;
             int64_t lrow;
-            row_dest(a, row, my_dst, my_sdst, src, rw, lrow);
+            if (!row_dest(a, e, row, my_dst, my_sdst, src, rw, lrow, flags)) my_dst = nullptr;
         }
+        if (flags && lt < 32) atomicOr(a.status, flags);
     }
 
     // the token's gradient row, unpacked to fp32 once for all its entries

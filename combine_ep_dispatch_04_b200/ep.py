@@ -66,7 +66,8 @@ class EpSizes(C.Structure):
 
 
 class EpGroupT(C.Structure):
-    _fields_ = [("world", C.c_int32), ("rank", C.c_int32), ("epoch", C.c_uint64)]
+    _fields_ = [("world", C.c_int32), ("rank", C.c_int32), ("epoch", C.c_uint64),
+                ("window_rows", C.c_int64)]
 
 
 class EpPeers(C.Structure):
@@ -566,8 +567,8 @@ def ep_get_status(dev_status, stream=None):
 
 
 # ---- expert parallelism over GPUs (include/ep.h, ep_group_*) ----------------------
-def make_group(world, rank, epoch=1):
-    return EpGroupT(world, rank, epoch)
+def make_group(world, rank, epoch=1, window_rows=0):
+    return EpGroupT(world, rank, epoch, window_rows)
 
 
 def ep_group_sizes(cfg, grp):

@@ -80,9 +80,9 @@ class EmulatedGroup:
     one GPU: each member's calls run one after another in stream order, so no
     kernel waits on work that has not been issued before it."""
 
-    def __init__(self, cfg, world, device, grad=False, weights=False):
+    def __init__(self, cfg, world, device, grad=False, weights=False, window_rows=0):
         self.cfg, self.world = cfg, world
-        self.wins = [Windows(cfg, ep.make_group(world, g), device, grad, weights)
+        self.wins = [Windows(cfg, ep.make_group(world, g, 1, window_rows), device, grad, weights)
                      for g in range(world)]
         ptrs = [w.pointers() for w in self.wins]
         tables = {f: [p[f] for p in ptrs] for f in Windows.FIELDS}
@@ -93,10 +93,20 @@ class EmulatedGroup:
             self._keep.append(keep)
 
 
+def _world(pg):
+    """(size, rank) of the process group; one GPU alone without one."""
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized():
+        return 1, 0
+    return dist.get_world_size(pg), dist.get_rank(pg)
+
+
 def _exchange(obj, pg, what):
     """all_gather_object over the process group; a peer that does not take part
     before the group's timeout turns into EP_ERR_TIMEOUT."""
     import torch.distributed as dist
+    if _world(pg)[0] == 1:
+        return [obj]
     out = [None] * dist.get_world_size(pg)
     try:
         dist.all_gather_object(out, obj, group=pg)
@@ -111,12 +121,11 @@ class EpGroup:
     step of the path as the sequence of libep calls on `stream`."""
 
     def __init__(self, cfg, pg=None, device=None, grad=False, weights=False, stream=None,
-                 timeout_ns=0):
-        import torch.distributed as dist
+                 timeout_ns=0, window_rows=0):
         self.cfg = cfg
-        G, g = dist.get_world_size(pg), dist.get_rank(pg)
+        G, g = _world(pg)
         self.world, self.rank = G, g
-        self.grp = ep.make_group(G, g, 1)
+        self.grp = ep.make_group(G, g, 1, window_rows)
         self.device = device or torch.device("cuda", torch.cuda.current_device())
         self.stream = stream or torch.cuda.current_stream(self.device)
         self.timeout_ns = timeout_ns

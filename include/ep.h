@@ -546,9 +546,13 @@ ep_status_t ep_dispatch_layout_static(const ep_config_t *cfg, const void *topk_i
 #define EP_GROUP_KINDS 5
 
 typedef struct {
-    int32_t world;  /* G, 1 .. 64, R % G == 0 */
-    int32_t rank;   /* this GPU, 0 .. G-1 */
-    uint64_t epoch; /* step number, >= 1, the same on every GPU */
+    int32_t world;       /* G, 1 .. 64, R % G == 0 */
+    int32_t rank;        /* this GPU, 0 .. G-1 */
+    uint64_t epoch;      /* step number, >= 1, the same on every GPU */
+    int64_t window_rows; /* packed layout: rows of every window; 0 = room for every entry
+                          * of the job (R*T*K + EG*(expert_align-1)).  Rows past a window
+                          * are skipped with EP_DEV_CAPACITY_OVERFLOW.  Padded: 0 (the
+                          * window is EG*R*M rows). */
 } ep_group_t;
 
 /* Every GPU's windows as this process sees them: device arrays of G device

@@ -20,6 +20,7 @@ import torch.multiprocessing as mp
 
 import combine_ep_dispatch_04_b200 as ep
 import synth
+from combine_ep_dispatch_04_b200.ep import lib
 from combine_ep_dispatch_04_b200.group import EmulatedGroup
 from harness import Run, to_np_u16
 
@@ -30,14 +31,15 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 class Members:
     """Per emulated GPU: its slice of the inputs and its own layout buffers."""
 
-    def __init__(self, r, G):
+    def __init__(self, r, G, window_rows=0):
         self.r, self.G = r, G
         w, cfg = r.w, r.cfg
         self.cfg = cfg
-        self.eg = EmulatedGroup(cfg, G, "cuda", grad=r.g is not None, weights=False)
+        self.eg = EmulatedGroup(cfg, G, "cuda", grad=r.g is not None, weights=False,
+                                window_rows=window_rows)
         R, T, K, E = w["R"], w["T"], w["K"], w["E"]
         self.RG, self.EG, self.T = R // G, E // G, T
-        self.grps = [ep.make_group(G, g, 1) for g in range(G)]
+        self.grps = [ep.make_group(G, g, 1, window_rows) for g in range(G)]
         self.status = torch.zeros(1, dtype=torch.int32, device="cuda")
         n = self.RG * T
         sl = [slice(g * n, (g + 1) * n) for g in range(G)]
@@ -210,6 +212,27 @@ def test_group_two_steps_reuse_the_windows():
         assert np.array_equal(data.cpu().numpy()[wrow[sel]], sd[srow[sel]])
 
 
+def test_rows_past_a_window_are_skipped_and_flagged():
+    """Windows smaller than their owners' rows: the rows that fit are the
+    single-GPU rows, the others are skipped and the capacity bit is set."""
+    w = synth.workload("tiny", R=4, T=24, M=24, K=4, E=8, H=256)
+    r = Run(w, "mxfp8", layout="packed")
+    need = int(r.lay["recv_count"][:4].sum())
+    small = need // 2
+    m = Members(r, 2, window_rows=small)
+    m.dispatch()
+    assert ep.ep_get_status(m.status) & ep.DEV_CAPACITY_OVERFLOW
+    own, wrow, srow = m.row_maps()
+    sz = m.sizes
+    assert sz["rows"] == small
+    sd = r.b.recv_data().cpu().numpy()
+    for o in range(2):
+        data, _ = _window_rows(m.eg.wins[o].recv, sz["rows"], sz["data_row_bytes"],
+                               sz["scale_row_bytes"], sz["recv_scale_offset"])
+        sel = (own == o) & (wrow < small)
+        assert np.array_equal(data.cpu().numpy()[wrow[sel]], sd[srow[sel]]), o
+
+
 def test_plan_kernel_equals_the_host_plan_on_many_shapes():
     """The plan kernel (one block: warp sums and a block-wide scan) against the
     host plan (the plain loops), for every member of several group sizes, on
@@ -260,11 +283,11 @@ def test_a_member_that_withholds_its_counts_times_out():
                      m.status)
     flags = ep.ep_get_status(m.status)
     assert flags & ep.DEV_TIMEOUT
-    assert ep.lib.ep_get_status(C.c_void_p(m.status.data_ptr()), C.byref(C.c_uint32(0)),
+    assert lib.ep_get_status(C.c_void_p(m.status.data_ptr()), C.byref(C.c_uint32(0)),
                                 C.c_void_p(torch.cuda.current_stream().cuda_stream)) == 0
     ep.ep_group_wait(m.grps[0], pe[0], ep.GROUP_KIND_EXPERT_OUT, m.status, timeout_ns=50_000_000)
     st = C.c_uint32(0)
-    assert ep.lib.ep_get_status(C.c_void_p(m.status.data_ptr()), C.byref(st),
+    assert lib.ep_get_status(C.c_void_p(m.status.data_ptr()), C.byref(st),
                                 C.c_void_p(torch.cuda.current_stream().cuda_stream)) == 6
     assert st.value & ep.DEV_TIMEOUT
     r2 = Run(w, "mxfp8", layout="packed")   # the context is still usable
@@ -287,7 +310,7 @@ def _ipc_reader(q_in, q_out, res):
     h, off = q_in.get(timeout=120)
     addr = ep_.ep_ipc_import(h, off)
     dst = torch.zeros((1 << 20) - 4096, dtype=torch.int32, device="cuda")
-    st = ep_.lib.ep_copy(C.c_void_p(dst.data_ptr()), C.c_void_p(addr), dst.numel() * 4,
+    st = ep_.ep.lib.ep_copy(C.c_void_p(dst.data_ptr()), C.c_void_p(addr), dst.numel() * 4,
                          C.c_void_p(torch.cuda.current_stream().cuda_stream))
     torch.cuda.synchronize()
     ok = st == 0 and bool(torch.equal(dst.cpu(), torch.arange(4096, 1 << 20, dtype=torch.int32)))
