@@ -39,6 +39,7 @@ struct CombineArgs {
     // the GPU that owns each virtual row; peer_y == nullptr on one GPU
     const uint8_t *const *peer_y;  // [G] expert-output windows
     int64_t win_rows;
+    int experts_per_gpu;           // an expert's owner is e / experts_per_gpu
 };
 
 enum { QIN_BF16 = 0, QIN_E4M3_B128 = 1, QIN_INT8 = 2, QIN_MXFP8 = 3, QIN_MXFP4 = 4 };
@@ -54,6 +55,30 @@ __host__ __device__ constexpr int combine_granule(int qin) {
 // codes into NaN; int8 through the 2^23 constant of i8_exact) and multiplied
 // by its row / block scale as one fp32 multiply, y = fl(decode(c) * s),
 // before the FMA.
+//
+// Two elements at a time on the packed fp32 pipe (mul.rn.f32x2 / fma.rn.f32x2,
+// sm_100): each lane is one IEEE multiply or fused multiply-add, rounded to
+// nearest even, exactly the scalar __fmul_rn / __fmaf_rn.
+// (a0, a1) <- fma(w, fl(x * s), a) lane by lane
+__device__ __forceinline__ void dq2(float &a0, float &a1, float w, float x0, float x1, float s) {
+    asm("{\n\t.reg .b64 a, x, s, w, p;\n\t"
+        "mov.b64 a, {%0, %1};\n\tmov.b64 x, {%4, %5};\n\t"
+        "mov.b64 s, {%3, %3};\n\tmov.b64 w, {%2, %2};\n\t"
+        "mul.rn.f32x2 p, x, s;\n\tfma.rn.f32x2 a, w, p, a;\n\t"
+        "mov.b64 {%0, %1}, a;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(w), "f"(s), "f"(x0), "f"(x1));
+}
+// (a0, a1) <- fma(w, x, a) lane by lane
+__device__ __forceinline__ void fma2(float &a0, float &a1, float w, float x0, float x1) {
+    asm("{\n\t.reg .b64 a, x, w;\n\t"
+        "mov.b64 a, {%0, %1};\n\tmov.b64 x, {%3, %4};\n\tmov.b64 w, {%2, %2};\n\t"
+        "fma.rn.f32x2 a, w, x, a;\n\t"
+        "mov.b64 {%0, %1}, a;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(w), "f"(x0), "f"(x1));
+}
+
 template <int QIN>
 __device__ __forceinline__ void dequant_fma(float (&acc)[combine_granule(QIN)], const uint4 &r,
                                             float s, float w) {
@@ -63,21 +88,19 @@ __device__ __forceinline__ void dequant_fma(float (&acc)[combine_granule(QIN)], 
         if constexpr (QIN == QIN_INT8) {
             const uint32_t wx = u[q] ^ 0x80808080u;
 #pragma unroll
-            for (int j = 0; j < 4; j++)
-                acc[4 * q + j] = __fmaf_rn(w, __fmul_rn(i8_exact(wx, j), s), acc[4 * q + j]);
+            for (int j = 0; j < 4; j += 2)
+                dq2(acc[4 * q + j], acc[4 * q + j + 1], w, i8_exact(wx, j), i8_exact(wx, j + 1), s);
         } else if constexpr (QIN == QIN_MXFP4) {
 #pragma unroll
             for (int b = 0; b < 4; b++) {
                 const float2 f = e2m1x2_to_f32(u[q] >> (8 * b));
-                acc[8 * q + 2 * b] = __fmaf_rn(w, __fmul_rn(f.x, s), acc[8 * q + 2 * b]);
-                acc[8 * q + 2 * b + 1] = __fmaf_rn(w, __fmul_rn(f.y, s), acc[8 * q + 2 * b + 1]);
+                dq2(acc[8 * q + 2 * b], acc[8 * q + 2 * b + 1], w, f.x, f.y, s);
             }
         } else {
 #pragma unroll
             for (int h = 0; h < 2; h++) {
                 const float2 f = e4m3x2_to_f32(u[q] >> (16 * h));
-                acc[4 * q + 2 * h] = __fmaf_rn(w, __fmul_rn(f.x, s), acc[4 * q + 2 * h]);
-                acc[4 * q + 2 * h + 1] = __fmaf_rn(w, __fmul_rn(f.y, s), acc[4 * q + 2 * h + 1]);
+                dq2(acc[4 * q + 2 * h], acc[4 * q + 2 * h + 1], w, f.x, f.y, s);
             }
         }
     }
@@ -105,15 +128,13 @@ __device__ __forceinline__ bool pow2_fma(float (&acc)[combine_granule(QIN)], con
 #pragma unroll
             for (int b = 0; b < 4; b++) {
                 const float2 f = e2m1x2_to_f32(u[q] >> (8 * b));
-                acc[8 * q + 2 * b] = __fmaf_rn(W, f.x, acc[8 * q + 2 * b]);
-                acc[8 * q + 2 * b + 1] = __fmaf_rn(W, f.y, acc[8 * q + 2 * b + 1]);
+                fma2(acc[8 * q + 2 * b], acc[8 * q + 2 * b + 1], W, f.x, f.y);
             }
         } else {
 #pragma unroll
             for (int h = 0; h < 2; h++) {
                 const float2 f = e4m3x2_to_f32(u[q] >> (16 * h));
-                acc[4 * q + 2 * h] = __fmaf_rn(W, f.x, acc[4 * q + 2 * h]);
-                acc[4 * q + 2 * h + 1] = __fmaf_rn(W, f.y, acc[4 * q + 2 * h + 1]);
+                fma2(acc[4 * q + 2 * h], acc[4 * q + 2 * h + 1], W, f.x, f.y);
             }
         }
     }
@@ -159,13 +180,17 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_kernel(CombineArgs
                 else flags |= kDevCapacity;
             }
         }
-        if (flags) atomicOr(a.status, flags);
         const uint8_t *yb = reinterpret_cast<const uint8_t *>(a.y);
-        if (a.peer_y && row >= 0) {  // virtual row -> owner's window
-            const int o = (int)(row / a.win_rows);
+        if (a.peer_y && row >= 0) {  // virtual row -> the expert owner's window
+            const int o = (int)(e / a.experts_per_gpu);
             row -= (int64_t)o * a.win_rows;
             yb = a.peer_y[o];
+            if (row >= a.win_rows) {
+                row = -1;
+                flags |= kDevCapacity;
+            }
         }
+        if (flags) atomicOr(a.status, flags);
         s_row[grp][lt] = row;
         s_ybase[grp][lt] = yb;
         s_w[grp][lt] = a.wts[n * a.K + lt];
