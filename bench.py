@@ -59,7 +59,8 @@ FALLBACK_HBM_GBS = 6650.0
 WORKLOAD_MODE = {"tiny": "int8_token", "decode": "e4m3_b128", "skewed": "int8_token",
                  "prefill": "mxfp8", "large": "mxfp4", "a5": "mxfp8"}
 KERNEL_SOURCES = ["combine_ep_dispatch_04_b200/csrc/" + f for f in
-                  ("ep_api.cu", "ep_device.cuh", "ep_layout.cuh", "ep_dispatch.cuh", "ep_combine.cuh")]
+                  ("ep_api.cu", "ep_device.cuh", "ep_layout.cuh", "ep_dispatch.cuh", "ep_combine.cuh",
+                   "ep_group.cuh")]
 
 
 def parse():
@@ -76,6 +77,8 @@ def parse():
     p.add_argument("--quantized-combine", action="store_true",
                    help="combine reads expert outputs stored in the dispatch format")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--only", choices=["ffn"], default=None,
+                   help="run one leg alone and print its object (profiler captures)")
     p.add_argument("--ep-group", action="store_true",
                    help="run the expert-parallel group path also on one GPU (a group of one)")
     p.add_argument("--replicas", action="store_true",
@@ -854,6 +857,19 @@ def main():
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.only == "ffn":
+        stream = torch.cuda.current_stream(dev)
+        flush_w = torch.empty(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+        flush_r = torch.ones(args.flush_mib << 20, dtype=torch.uint8, device=dev)
+
+        def flush_only(v):
+            flush_w.fill_(v)
+            flush_r.max()
+        leg = run_ffn_leg(ep, flush_only, stream, dev, args, replica)
+        if rank == 0:
+            print(json.dumps({"expert_ffn": leg}), flush=True)
+        dist_done(world)
+        return
     if (world > 1 and not args.replicas) or args.ep_group:
         run_group_bench(ep, args, wname, world, rank, local, dev)
         return

@@ -494,23 +494,29 @@ ep_status_t launch_dispatch(const ep::DispatchArgs &a, cudaStream_t s) {
 // The backward quantises every entry separately (K scaled copies of the
 // row), so its per-thread state grows with G: keep G <= 2 (about 60
 // registers) for occupancy.
-ep_status_t launch_combine_bwd(const ep::DispatchArgs &a, cudaStream_t s) {
+template <bool GROUP>
+ep_status_t launch_combine_bwd_as(const ep::DispatchArgs &a, cudaStream_t s) {
     auto kernel_of = [](int t, int g) -> const void * {
-#define EP_FN(T_, G_) if (t == T_ && g == G_) return (const void *)ep::combine_bwd_kernel<T_, G_>;
+#define EP_FN(T_, G_) \
+    if (t == T_ && g == G_) return (const void *)ep::combine_bwd_kernel<T_, G_, GROUP>;
         EP_SPLITS(EP_FN)
 #undef EP_FN
         return nullptr;
     };
     const Split sp = split_rows(a.N, a.H / 16, 2, kernel_of);
     const unsigned grid = grid_for(a.N, sp.tpt);
-#define EP_CASE(T_, G_)                                                                     \
-    if (sp.tpt == T_ && sp.gmax == G_) {                                                    \
-        launch(ep::combine_bwd_kernel<T_, G_>, grid, ep::block_threads(T_), 0, s, a);        \
-        return launched();                                                                  \
+#define EP_CASE(T_, G_)                                                                        \
+    if (sp.tpt == T_ && sp.gmax == G_) {                                                       \
+        launch(ep::combine_bwd_kernel<T_, G_, GROUP>, grid, ep::block_threads(T_), 0, s, a);    \
+        return launched();                                                                     \
     }
     EP_SPLITS(EP_CASE)
 #undef EP_CASE
     return EP_ERR_UNSUPPORTED;
+}
+
+ep_status_t launch_combine_bwd(const ep::DispatchArgs &a, cudaStream_t s) {
+    return a.peer_out ? launch_combine_bwd_as<true>(a, s) : launch_combine_bwd_as<false>(a, s);
 }
 
 ep::DispatchArgs dispatch_args(const ep_config_t *cfg, const Plan &p) {

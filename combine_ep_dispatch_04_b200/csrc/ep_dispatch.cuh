@@ -364,7 +364,7 @@ __global__ void __launch_bounds__(block_threads(TPT)) dispatch_kernel(DispatchAr
 // Description): row(n,k) <- MXFP8(w[n,k] * g[n,:]).  The block maximum of
 // |fl(w*g_h)| equals fl(|w| * max|g_h|) because rounding is monotone and sign
 // symmetric, so it is taken once per token and scaled per entry.
-template <int TPT, int GMAX>
+template <int TPT, int GMAX, bool GROUP>
 __device__ __forceinline__ void combine_bwd_body(const DispatchArgs &a) {
     pdl_enter();
     constexpr int TOKS = block_threads(TPT) / TPT;
@@ -379,19 +379,22 @@ __device__ __forceinline__ void combine_bwd_body(const DispatchArgs &a) {
     // Every warp reads the token's entries itself (lane k holds entry k) and
     // hands them out by shuffles: no block barrier stands between a warp's
     // gradient loads and its stores.  The first warp reports the flags.
+    // On one GPU the row index is handed out; over GPUs (peer_out) the two
+    // destination pointers in the owner's window.
+    int64_t my_row = -1;
     uint8_t *my_dst = nullptr, *my_sdst = nullptr;
     float my_w = 0.0f;
     if (active && lane < a.K) {
         uint32_t flags = 0;
         const int64_t e = a.idx[n * a.K + lane];
         const int32_t sl = (e >= 0 && e < a.E) ? a.slot[n * a.K + lane] : -1;
-        const int64_t row = row_of_entry(a, e, sl, flags);
+        my_row = row_of_entry(a, e, sl, flags);
         my_w = a.unweighted ? 1.0f : a.wts[n * a.K + lane];
-        if (row >= 0) {
+        if (GROUP && my_row >= 0) {
             int32_t *src;
             float *rw;
             int64_t lrow;
-            if (!row_dest(a, e, row, my_dst, my_sdst, src, rw, lrow, flags)) my_dst = nullptr;
+            if (!row_dest(a, e, my_row, my_dst, my_sdst, src, rw, lrow, flags)) my_row = -1;
         }
         if (flags && lt < 32) atomicOr(a.status, flags);
     }
@@ -442,12 +445,19 @@ __device__ __forceinline__ void combine_bwd_body(const DispatchArgs &a) {
 
     const bool weighted = !a.unweighted;
     for (int k = 0; k < a.K; k++) {
-        uint8_t *dst = reinterpret_cast<uint8_t *>(
-            __shfl_sync(kFull, reinterpret_cast<uintptr_t>(my_dst), k));
-        uint8_t *sdst = reinterpret_cast<uint8_t *>(
-            __shfl_sync(kFull, reinterpret_cast<uintptr_t>(my_sdst), k));
+        const int64_t row = __shfl_sync(kFull, my_row, k);
         const float w = __shfl_sync(kFull, my_w, k);
-        if (!dst) continue;
+        if (row < 0) continue;
+        uint8_t *dst, *sdst;
+        if constexpr (GROUP) {
+            dst = reinterpret_cast<uint8_t *>(
+                __shfl_sync(kFull, reinterpret_cast<uintptr_t>(my_dst), k));
+            sdst = reinterpret_cast<uint8_t *>(
+                __shfl_sync(kFull, reinterpret_cast<uintptr_t>(my_sdst), k));
+        } else {
+            dst = a.out + row * (int64_t)a.H;
+            sdst = a.out + a.scale_off + row * (int64_t)(a.H >> 5);
+        }
         const float aw = fabsf(w);
 #pragma unroll
         for (int i = 0; i < GMAX; i++) {
@@ -475,10 +485,12 @@ __device__ __forceinline__ void combine_bwd_body(const DispatchArgs &a) {
     }
 }
 
-template <int TPT, int GMAX>
+// GROUP: the rows go to the owners' windows over GPUs, and the grid ends with
+// the signal (a separate instantiation: the one-GPU kernel carries neither)
+template <int TPT, int GMAX, bool GROUP = false>
 __global__ void __launch_bounds__(block_threads(TPT)) combine_bwd_kernel(DispatchArgs a) {
-    combine_bwd_body<TPT, GMAX>(a);
-    if (a.done) group_grid_done(a.done, a.flags, a.flag_kind, a.grp_g, a.grp_G, a.epoch);
+    combine_bwd_body<TPT, GMAX, GROUP>(a);
+    if constexpr (GROUP) group_grid_done(a.done, a.flags, a.flag_kind, a.grp_g, a.grp_G, a.epoch);
 }
 
 }  // namespace ep

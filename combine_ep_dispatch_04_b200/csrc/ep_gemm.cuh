@@ -622,7 +622,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // TMEM scale columns: A's groups (4 columns each), then B's (group-major,
 // then 128-row block).
 // ---------------------------------------------------------------------------
-constexpr int kMxBK = 128, kMxStages = 4, kMxThreads = 224;
+constexpr int kMxBK = 128, kMxThreads = 224;
 // K steps whose scale loads the gathering warp issues together (MXFP4 has
 // twice the scale bytes a step: fewer steps keep its registers unspilled)
 template <bool FP4>
@@ -641,10 +641,17 @@ struct MxCfg {
     static constexpr int kBytesB = BN * kMxBK;
     static constexpr int kSfBytes = 512 * kGroups * (1 + kChunksB);  // a stage's scales, A then B
     static constexpr int kSfCol = kAcc * BN;                // TMEM column of A's scales
+    // Stages: as many as the shared memory holds (at most 8).  The operands
+    // stream from L2 and DRAM at a latency of about a microsecond, so the
+    // bytes in flight per SM, not the issue rate, set the narrow tiles' pace.
+    static constexpr size_t kFixed = 1024 + 16 + (kGemmMaxExperts + 1) * 4 + 256 + 5 * 8;
+    static constexpr int kStageBytes = kBytesA + kBytesB + kSfBytes;
+    static constexpr int kStagesFit = (int)((227 * 1024 - kFixed) / (kStageBytes + 16));
+    static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
     static constexpr size_t smem() {
-        return 1024 + (size_t)kMxStages * (kBytesA + kBytesB + kSfBytes) +
-               (2 * kMxStages + 5) * 8 + 16 + (kGemmMaxExperts + 1) * 4 + 256;
+        return kFixed + (size_t)kStages * kStageBytes + (size_t)2 * kStages * 8;
     }
+    static_assert(kStages >= 4, "pipeline depth");
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "N tile");
     static_assert(kAcc * BN + kSfCols <= 512, "TMEM columns");
 };
@@ -721,7 +728,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     using C = MxCfg<BN, FP4>;
     static_assert(!GLU || (!FP4 && BN % 64 == 0), "GLU: MXFP8, whole 32-blocks per half tile");
     constexpr int TN = GLU ? BN / 2 : BN;  // output columns a tile advances by
-    constexpr int S = kMxStages;
+    constexpr int S = C::kStages;
     extern __shared__ uint8_t gsm_raw[];
     uint8_t *gsm = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~(uintptr_t)1023);

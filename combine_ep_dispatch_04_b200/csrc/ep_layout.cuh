@@ -625,14 +625,22 @@ __global__ void __launch_bounds__(512, 1) layout_cluster_kernel(LayoutArgs a, Cl
     }
     cluster.sync();
 
-    // phase 2b: bases from the lower blocks' totals (distributed shared memory)
+    // phase 2b: bases from the lower blocks' totals (distributed shared memory);
+    // the remote loads of all blocks are issued together, then summed
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int base = 0;
-        for (int q2 = 0; q2 < q; q2++) base += cluster.map_shared_rank(tot, q2)[e];
+        const int upto = q == 0 ? cp.Q : q;  // block 0 also sums every block
+        int v[16];
+#pragma unroll
+        for (int q2 = 0; q2 < 16; q2++)
+            v[q2] = q2 < upto ? cluster.map_shared_rank(tot, q2)[e] : 0;
+        int base = 0, all = 0;
+#pragma unroll
+        for (int q2 = 0; q2 < 16; q2++) {
+            base += q2 < q ? v[q2] : 0;
+            all += v[q2];
+        }
         for (int lc = 0; lc < nloc; lc++) off[lc * E + e] += base;
         if (q == 0) {
-            int all = 0;
-            for (int q2 = 0; q2 < cp.Q; q2++) all += cluster.map_shared_rank(tot, q2)[e];
             a.recv_count[e] = all;
             if (a.stats) a.stats[e] += all;
         }
