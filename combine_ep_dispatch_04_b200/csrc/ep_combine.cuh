@@ -59,48 +59,76 @@ __host__ __device__ constexpr int combine_granule(int qin) {
 // Two elements at a time on the packed fp32 pipe (mul.rn.f32x2 / fma.rn.f32x2,
 // sm_100): each lane is one IEEE multiply or fused multiply-add, rounded to
 // nearest even, exactly the scalar __fmul_rn / __fmaf_rn.
+// The weight and the scale are splat once per expert row ({w, w}, {s, s}) and
+// the codes unpacked by vector moves (four e2m1 bytes, two e4m3 halves).
+__device__ __forceinline__ uint64_t splat2(float v) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+    return r;
+}
 // (a0, a1) <- fma(w, fl(x * s), a) lane by lane
-__device__ __forceinline__ void dq2(float &a0, float &a1, float w, float x0, float x1, float s) {
-    asm("{\n\t.reg .b64 a, x, s, w, p;\n\t"
-        "mov.b64 a, {%0, %1};\n\tmov.b64 x, {%4, %5};\n\t"
-        "mov.b64 s, {%3, %3};\n\tmov.b64 w, {%2, %2};\n\t"
-        "mul.rn.f32x2 p, x, s;\n\tfma.rn.f32x2 a, w, p, a;\n\t"
-        "mov.b64 {%0, %1}, a;\n\t}"
+__device__ __forceinline__ void dq2(float &a0, float &a1, uint64_t w2, uint64_t s2, float x0,
+                                    float x1) {
+    asm("{\n\t.reg .b64 a, x;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 x, {%4, %5};\n\t"
+        "mul.rn.f32x2 x, x, %3;\n\tfma.rn.f32x2 a, %2, x, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
         : "+f"(a0), "+f"(a1)
-        : "f"(w), "f"(s), "f"(x0), "f"(x1));
+        : "l"(w2), "l"(s2), "f"(x0), "f"(x1));
 }
 // (a0, a1) <- fma(w, x, a) lane by lane
-__device__ __forceinline__ void fma2(float &a0, float &a1, float w, float x0, float x1) {
-    asm("{\n\t.reg .b64 a, x, w;\n\t"
-        "mov.b64 a, {%0, %1};\n\tmov.b64 x, {%3, %4};\n\tmov.b64 w, {%2, %2};\n\t"
-        "fma.rn.f32x2 a, w, x, a;\n\t"
-        "mov.b64 {%0, %1}, a;\n\t}"
+__device__ __forceinline__ void fma2(float &a0, float &a1, uint64_t w2, float x0, float x1) {
+    asm("{\n\t.reg .b64 a, x;\n\tmov.b64 a, {%0, %1};\n\tmov.b64 x, {%3, %4};\n\t"
+        "fma.rn.f32x2 a, %2, x, a;\n\tmov.b64 {%0, %1}, a;\n\t}"
         : "+f"(a0), "+f"(a1)
-        : "f"(w), "f"(x0), "f"(x1));
+        : "l"(w2), "f"(x0), "f"(x1));
+}
+// Codes widen exactly through f16 (every e4m3 and e2m1 value is an f16 value).
+// The eight e2m1 codes of u (code j in nibble j) as four f16 pairs, h[b] from byte b.
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t u, uint32_t (&h)[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+        : "r"(u));
+}
+// The four e4m3 codes of u (code j in byte j) as two f16 pairs, h[b] from half b.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t u, uint32_t (&h)[2]) {
+    asm("{\n\t.reg .b16 c0, c1;\n\tmov.b32 {c0, c1}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, c0;\n\tcvt.rn.f16x2.e4m3x2 %1, c1;\n\t}"
+        : "=r"(h[0]), "=r"(h[1])
+        : "r"(u));
+}
+__device__ __forceinline__ float2 f16x2_to_f32(uint32_t h) {
+    return __half22float2(*reinterpret_cast<const __half2 *>(&h));
 }
 
+// acc <- fma(w, fl(decode(c) * s), acc) over the 16 bytes of codes in r.
 template <int QIN>
 __device__ __forceinline__ void dequant_fma(float (&acc)[combine_granule(QIN)], const uint4 &r,
                                             float s, float w) {
     const uint32_t u[4] = {r.x, r.y, r.z, r.w};
+    const uint64_t w2 = splat2(w), s2 = splat2(s);
 #pragma unroll
     for (int q = 0; q < 4; q++) {
         if constexpr (QIN == QIN_INT8) {
             const uint32_t wx = u[q] ^ 0x80808080u;
 #pragma unroll
             for (int j = 0; j < 4; j += 2)
-                dq2(acc[4 * q + j], acc[4 * q + j + 1], w, i8_exact(wx, j), i8_exact(wx, j + 1), s);
+                dq2(acc[4 * q + j], acc[4 * q + j + 1], w2, s2, i8_exact(wx, j), i8_exact(wx, j + 1));
         } else if constexpr (QIN == QIN_MXFP4) {
+            uint32_t h[4];
+            e2m1x8_to_f16x2(u[q], h);
 #pragma unroll
             for (int b = 0; b < 4; b++) {
-                const float2 f = e2m1x2_to_f32(u[q] >> (8 * b));
-                dq2(acc[8 * q + 2 * b], acc[8 * q + 2 * b + 1], w, f.x, f.y, s);
+                const float2 f = f16x2_to_f32(h[b]);
+                dq2(acc[8 * q + 2 * b], acc[8 * q + 2 * b + 1], w2, s2, f.x, f.y);
             }
         } else {
+            uint32_t h[2];
+            e4m3x4_to_f16x2(u[q], h);
 #pragma unroll
-            for (int h = 0; h < 2; h++) {
-                const float2 f = e4m3x2_to_f32(u[q] >> (16 * h));
-                dq2(acc[4 * q + 2 * h], acc[4 * q + 2 * h + 1], w, f.x, f.y, s);
+            for (int b = 0; b < 2; b++) {
+                const float2 f = f16x2_to_f32(h[b]);
+                dq2(acc[4 * q + 2 * b], acc[4 * q + 2 * b + 1], w2, s2, f.x, f.y);
             }
         }
     }
@@ -122,19 +150,24 @@ __device__ __forceinline__ bool pow2_fma(float (&acc)[combine_granule(QIN)], con
     const float W = __fmul_rn(w, s);
     if (!((fabsf(W) >= FLT_MIN || w == 0.0f) && fabsf(W) <= FLT_MAX)) return false;
     const uint32_t u[4] = {r.x, r.y, r.z, r.w};
+    const uint64_t W2 = splat2(W);
 #pragma unroll
     for (int q = 0; q < 4; q++) {
         if constexpr (QIN == QIN_MXFP4) {
+            uint32_t h[4];
+            e2m1x8_to_f16x2(u[q], h);
 #pragma unroll
             for (int b = 0; b < 4; b++) {
-                const float2 f = e2m1x2_to_f32(u[q] >> (8 * b));
-                fma2(acc[8 * q + 2 * b], acc[8 * q + 2 * b + 1], W, f.x, f.y);
+                const float2 f = f16x2_to_f32(h[b]);
+                fma2(acc[8 * q + 2 * b], acc[8 * q + 2 * b + 1], W2, f.x, f.y);
             }
         } else {
+            uint32_t h[2];
+            e4m3x4_to_f16x2(u[q], h);
 #pragma unroll
-            for (int h = 0; h < 2; h++) {
-                const float2 f = e4m3x2_to_f32(u[q] >> (16 * h));
-                fma2(acc[4 * q + 2 * h], acc[4 * q + 2 * h + 1], W, f.x, f.y);
+            for (int b = 0; b < 2; b++) {
+                const float2 f = f16x2_to_f32(h[b]);
+                fma2(acc[4 * q + 2 * b], acc[4 * q + 2 * b + 1], W2, f.x, f.y);
             }
         }
     }

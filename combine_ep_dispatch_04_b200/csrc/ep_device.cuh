@@ -72,6 +72,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---- native format conversions (sm_100a) ----------------------------------
 // cvt ... e4m3x2 / e2m1x2 put their first source operand in the upper part of
 // the result, so `lo` is passed second to land at the lower address / nibble.
+// (p0, p1) <- (fl(p0 * s), fl(p1 * s)) on the packed fp32 pipe (sm_100): each
+// lane one IEEE multiply rounded to nearest even, exactly __fmul_rn.
+__device__ __forceinline__ void mul2(float &p0, float &p1, float s) {
+    asm("{\n\t.reg .b64 p, s;\n\tmov.b64 p, {%0, %1};\n\tmov.b64 s, {%2, %2};\n\t"
+        "mul.rn.f32x2 p, p, s;\n\tmov.b64 {%0, %1}, p;\n\t}"
+        : "+f"(p0), "+f"(p1)
+        : "f"(s));
+}
+
 __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
@@ -83,23 +92,6 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
         : "=r"(r)
         : "f"(hi), "f"(lo));
     return r;
-}
-
-// Exact widening of two e4m3 / e2m1 codes (the low byte / nibble first) to
-// fp32, through f16 (every e4m3 and e2m1 value is an f16 value).
-__device__ __forceinline__ float2 e4m3x2_to_f32(uint32_t two_codes) {
-    uint32_t h2;
-    asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}"
-        : "=r"(h2)
-        : "r"(two_codes & 0xFFFFu));
-    return __half22float2(*reinterpret_cast<__half2 *>(&h2));
-}
-__device__ __forceinline__ float2 e2m1x2_to_f32(uint32_t two_codes) {
-    uint32_t h2;
-    asm("{\n\t.reg .b8 c;\n\tcvt.u8.u32 c, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
-        : "=r"(h2)
-        : "r"(two_codes & 0xFFu));
-    return __half22float2(*reinterpret_cast<__half2 *>(&h2));
 }
 
 // ---- exact int8 decoding without a conversion instruction ----------------------

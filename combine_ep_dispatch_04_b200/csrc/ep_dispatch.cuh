@@ -272,8 +272,10 @@ __device__ __forceinline__ void dispatch_body(const DispatchArgs &a) {
 #pragma unroll
             for (int q = 0; q < 4; q++) {
                 const uint32_t w0 = v[i][2 * q], w1 = v[i][2 * q + 1];
-                c[i][q] = cvt_e4m3x2(__fmul_rn(bf_lo(w0), s), __fmul_rn(bf_hi(w0), s)) |
-                          (cvt_e4m3x2(__fmul_rn(bf_lo(w1), s), __fmul_rn(bf_hi(w1), s)) << 16);
+                float p0 = bf_lo(w0), p1 = bf_hi(w0), p2 = bf_lo(w1), p3 = bf_hi(w1);
+                mul2(p0, p1, s);
+                mul2(p2, p3, s);
+                c[i][q] = cvt_e4m3x2(p0, p1) | (cvt_e4m3x2(p2, p3) << 16);
             }
         } else {  // MXFP4: element 2i in the low nibble
             const float s = bs[i];
@@ -283,7 +285,9 @@ __device__ __forceinline__ void dispatch_body(const DispatchArgs &a) {
 #pragma unroll
                 for (int h = 0; h < 4; h++) {
                     const uint32_t wv = v[i][4 * q + h];
-                    word |= cvt_e2m1x2(__fmul_rn(bf_lo(wv), s), __fmul_rn(bf_hi(wv), s)) << (8 * h);
+                    float p0 = bf_lo(wv), p1 = bf_hi(wv);
+                    mul2(p0, p1, s);
+                    word |= cvt_e2m1x2(p0, p1) << (8 * h);
                 }
                 c[i][q] = word;
             }
@@ -472,12 +476,13 @@ __device__ __forceinline__ void combine_bwd_body(const DispatchArgs &a) {
 #pragma unroll
             for (int q = 0; q < 4; q++) {
                 float p0 = f[i][4 * q], p1 = f[i][4 * q + 1], p2 = f[i][4 * q + 2], p3 = f[i][4 * q + 3];
-                if (weighted) {
-                    p0 = __fmul_rn(w, p0); p1 = __fmul_rn(w, p1);
-                    p2 = __fmul_rn(w, p2); p3 = __fmul_rn(w, p3);
+                if (weighted) {  // fl(w * g), then fl(. * 2^-X): two multiplies, as defined
+                    mul2(p0, p1, w);
+                    mul2(p2, p3, w);
                 }
-                cw[q] = cvt_e4m3x2(__fmul_rn(p0, s), __fmul_rn(p1, s)) |
-                        (cvt_e4m3x2(__fmul_rn(p2, s), __fmul_rn(p3, s)) << 16);
+                mul2(p0, p1, s);
+                mul2(p2, p3, s);
+                cw[q] = cvt_e4m3x2(p0, p1) | (cvt_e4m3x2(p2, p3) << 16);
             }
             st_v4(dst + (int64_t)g * 16, make_uint4(cw[0], cw[1], cw[2], cw[3]));
             if ((g & 1) == 0) sdst[g >> 1] = (uint8_t)(X + 127);
