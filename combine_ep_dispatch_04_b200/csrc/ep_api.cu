@@ -904,11 +904,11 @@ struct MxOperand {
     int K;  // elements of a row
 };
 
-// one launch of the MX kernel (e4m3 or packed e2m1 codes) with N tiles of BN
-// columns; GLU: the first layer of the gated MLP (n_out = 2I outputs of which
-// the epilogue writes z = silu(gate) * up requantised to zc / zs, BN/2 of each
-// half per tile)
-extern "C++" template <int BN, bool FP4, bool GLU = false>
+// one launch of the MX kernel (e4m3 or packed e2m1 codes) with tiles of BM
+// rows and BN columns; GLU: the first layer of the gated MLP (n_out = 2I
+// outputs of which the epilogue writes z = silu(gate) * up requantised to
+// zc / zs, BN/2 of each half per tile)
+extern "C++" template <int BN, bool FP4, bool GLU = false, int BM = ep::kGemmBM>
 ep_status_t launch_gemm_mx(const Plan &p, const MxOperand &x, const int64_t *expert_offset,
                            const int64_t *recv_count, const uint8_t *w_codes,
                            const uint8_t *w_scales, int n_out, uint16_t *y, uint8_t *zc,
@@ -927,10 +927,10 @@ ep_status_t launch_gemm_mx(const Plan &p, const MxOperand &x, const int64_t *exp
     a.eo = expert_offset; a.cnt = recv_count;
     a.xs = x.scales;
     a.ws = w_scales; a.y = y; a.zc = zc; a.zs = zs; a.status = dev_status;
-    const size_t smem = ep::MxCfg<BN, FP4>::smem();
-    if (!allow_smem(ep::expert_gemm_mx_kernel<BN, FP4, GLU>, slot, smem)) return EP_ERR_CUDA;
-    launch(ep::expert_gemm_mx_kernel<BN, FP4, GLU>, (unsigned)sm_count(), ep::kMxThreads, smem, s,
-           ma, mb, a);
+    const size_t smem = ep::MxCfg<BN, FP4, BM>::smem();
+    if (!allow_smem(ep::expert_gemm_mx_kernel<BN, FP4, GLU, BM>, slot, smem)) return EP_ERR_CUDA;
+    launch(ep::expert_gemm_mx_kernel<BN, FP4, GLU, BM>, (unsigned)sm_count(), ep::kMxThreads, smem,
+           s, ma, mb, a);
     return launched();
 }
 
@@ -971,11 +971,24 @@ int gemm_pairs() {
 // at least 256 rows an expert on average takes one accumulator of 256
 // columns, the most FLOPs per byte of A (measured faster there, not for
 // MXFP4).  Otherwise 256, then 128, where 224 does not divide n_out.
+// Average rows an expert from which 256-row tiles pay (measured on one B200:
+// MXFP4 gains from 256 rows, MXFP8 from about twice that).
+constexpr int64_t mx_tall_rows(bool fp4) { return fp4 ? 256 : 448; }
+
 int mx_tile_n(int n_out, bool fp4 = false, int64_t rows_per_expert = 0) {
+    if (rows_per_expert >= mx_tall_rows(fp4) && n_out % 224 == 0) return 224;
     if (!fp4 && rows_per_expert >= 256 && n_out % 256 == 0) return 256;
     for (int bn : {224, 256, 128})
         if (n_out % bn == 0) return bn;
     return 0;
+}
+// Row tiles of 256 (two M = 128 MMAs sharing each B tile: a third fewer
+// operand bytes per FLOP than 128 x 224; a tile whose upper half holds no row
+// runs as a 128-row tile) where the experts hold at least mx_tall_rows rows
+// on average.  With 224 columns a half, the two halves fill 448 TMEM columns:
+// one accumulator, so the epilogue does not overlap the next tile's MMAs.
+int mx_tile_m(int bn, bool fp4, int64_t rows_per_expert) {
+    return (bn == 224 && rows_per_expert >= mx_tall_rows(fp4)) ? 256 : ep::kGemmBM;
 }
 
 // The experts' maps: argument checks (EP_OK: a launch may follow, or there is
@@ -1059,13 +1072,19 @@ ep_status_t run_gemm_mx(const ep_config_t *cfg, const Plan &p, const void *recv_
                         uint32_t *dev_status, cudaStream_t s, const MxOperand *x_in = nullptr) {
     const bool fp4 = cfg->quant == EP_Q_MXFP4;
     const int bn = mx_tile_n(n_out, fp4, p.N * p.K / p.E);
+    const int bm = mx_tile_m(bn, fp4, p.N * p.K / p.E);
     const MxOperand x = x_in ? *x_in
                              : MxOperand{recv_buf,
                                          static_cast<const uint8_t *>(recv_buf) + p.scale_off,
                                          p.H};
-#define EP_MX(BN_, FP4_, SLOT_)                                                              \
-    return launch_gemm_mx<BN_, FP4_>(p, x, expert_offset, recv_count, w_codes, w_scales, n_out, \
-                                     y, nullptr, nullptr, dev_status, s, SLOT_)
+#define EP_MX(BN_, FP4_, SLOT_, ...)                                                         \
+    return launch_gemm_mx<BN_, FP4_, false, ##__VA_ARGS__>(p, x, expert_offset, recv_count, w_codes, \
+                                                       w_scales, n_out, y, nullptr, nullptr,      \
+                                                       dev_status, s, SLOT_)
+    if (bm == 256) {
+        if (fp4) EP_MX(224, true, 15, 256);
+        EP_MX(224, false, 16, 256);
+    }
     if (fp4) {
         if (bn == 224) EP_MX(224, true, 9);
         if (bn == 256) EP_MX(256, true, 10);

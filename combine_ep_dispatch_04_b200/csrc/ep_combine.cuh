@@ -436,27 +436,14 @@ __global__ void __launch_bounds__(block_threads(TPT)) combine_q_kernel(CombineAr
         float acc[EPG];
 #pragma unroll
         for (int q = 0; q < EPG; q++) acc[q] = 0.0f;
-        if constexpr (QIN == QIN_MXFP4) {
-            // 32 accumulators a granule: the rolled loop is the faster one here
-#pragma unroll 1
-            for (int kk = 0; kk < KB; kk++) {
-                if (kk >= a.K || s_row[grp][kk] < 0) continue;
-                const uint4 r = s_code[i & 1][kk][tid];
-                const float sc = scale_at<QIN>(&s_scl[grp][kk * (int)a.S], g, a.sfmt);
-                const float w = s_w[grp][kk];
-                if (pow2_fma<QIN>(acc, r, sc, w)) continue;
-                dequant_fma<QIN>(acc, r, sc, w);
-            }
-        } else {
-            // the entries' decode chains are independent: unrolled, they overlap
+        // the entries' decode chains are independent: unrolled, they overlap
 #pragma unroll
-            for (int kk = 0; kk < KB; kk++) {
-                if (!(live & (1u << kk))) continue;
-                const uint4 r = s_code[i & 1][kk][tid];
-                const float sc = scale_at<QIN>(&s_scl[grp][kk * (int)a.S], g, a.sfmt);
-                if (try_pow2 && pow2_fma<QIN>(acc, r, sc, wk[kk])) continue;
-                dequant_fma<QIN>(acc, r, sc, wk[kk]);
-            }
+        for (int kk = 0; kk < KB; kk++) {
+            if (!(live & (1u << kk))) continue;
+            const uint4 r = s_code[i & 1][kk][tid];
+            const float sc = scale_at<QIN>(&s_scl[grp][kk * (int)a.S], g, a.sfmt);
+            if (try_pow2 && pow2_fma<QIN>(acc, r, sc, wk[kk])) continue;
+            dequant_fma<QIN>(acc, r, sc, wk[kk]);
         }
         uint16_t *o = a.out + n * a.H + (int64_t)g * EPG;
 #pragma unroll

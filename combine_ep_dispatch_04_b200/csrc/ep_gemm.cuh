@@ -115,6 +115,30 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 }
 
 // 16 fp32 accumulator columns of one row -> 16 bf16 (round to nearest even)
+// 32 consecutive fp32 columns of this warp's 32 TMEM lanes, one wait
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+        "%11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, "
+        "%28, %29, %30, %31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                   "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                   "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]),
+                   "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]),
+                   "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]),
+                   "+r"(v[30]), "+r"(v[31])
+                 :
+                 : "memory");
+}
+
 __device__ __forceinline__ void store_bf16x16(uint16_t *dst, const uint32_t (&v)[16]) {
     uint4 lo, hi;
     lo.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
@@ -133,7 +157,7 @@ __device__ __forceinline__ void store_bf16x16(uint16_t *dst, const uint32_t (&v)
 // Within an expert the row tiles vary fastest: the blocks that read the same
 // weight columns run side by side, so those columns come from DRAM once.
 __device__ __forceinline__ void gemm_tile(const int *prefix, int E, int ntn, int t, int &e,
-                                          int &m0, int &n0, int bn = kGemmBN) {
+                                          int &m0, int &n0, int bn = kGemmBN, int bm = kGemmBM) {
     int lo = 0, hi = E - 1;  // the last e with prefix[e] <= t
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -143,7 +167,7 @@ __device__ __forceinline__ void gemm_tile(const int *prefix, int E, int ntn, int
     e = lo;
     const int local = t - prefix[e];
     const int mt = (prefix[e + 1] - prefix[e]) / ntn;  // row tiles of expert e
-    m0 = (local % mt) * kGemmBM;
+    m0 = (local % mt) * bm;
     n0 = (local / mt) * bn;
 }
 
@@ -630,17 +654,20 @@ __host__ __device__ constexpr int sf_group() { return FP4 ? 4 : 8; }
 static_assert(sf_group<false>() % 4 == 0 && sf_group<true>() % 4 == 0,
               "16-byte scale loads cover four steps");
 
-template <int BN, bool FP4>
+template <int BN, bool FP4, int BM = kGemmBM>
 struct MxCfg {
     static constexpr int kNsf = FP4 ? 2 : 1;                // scale blocks per instruction
     static constexpr int kGroups = kNsf;                    // groups of 4 blocks per K step
+    static constexpr int kChunksA = BM / 128;               // 128-row halves of A (M = 128 MMAs)
     static constexpr int kChunksB = (BN + 127) / 128;       // 128-row blocks of B
-    static constexpr int kSfCols = 4 * kGroups * (1 + kChunksB);  // TMEM columns of the scales
-    static constexpr int kAcc = (2 * BN + kSfCols <= 512) ? 2 : 1;
-    static constexpr int kBytesA = kGemmBM * kMxBK;         // 16 KB
+    static constexpr int kChunks = kChunksA + kChunksB;
+    static constexpr int kSfCols = 4 * kGroups * kChunks;   // TMEM columns of the scales
+    static constexpr int kAccCols = kChunksA * BN;          // one accumulator: BN columns a half
+    static constexpr int kAcc = (2 * kAccCols + kSfCols <= 512) ? 2 : 1;
+    static constexpr int kBytesA = BM * kMxBK;              // 16 KB a half
     static constexpr int kBytesB = BN * kMxBK;
-    static constexpr int kSfBytes = 512 * kGroups * (1 + kChunksB);  // a stage's scales, A then B
-    static constexpr int kSfCol = kAcc * BN;                // TMEM column of A's scales
+    static constexpr int kSfBytes = 512 * kGroups * kChunks;  // a stage's scales, A then B
+    static constexpr int kSfCol = kAcc * kAccCols;          // TMEM column of A's scales
     // Stages: as many as the shared memory holds (at most 8).  The operands
     // stream from L2 and DRAM at a latency of about a microsecond, so the
     // bytes in flight per SM, not the issue rate, set the narrow tiles' pace.
@@ -651,9 +678,10 @@ struct MxCfg {
     static constexpr size_t smem() {
         return kFixed + (size_t)kStages * kStageBytes + (size_t)2 * kStages * 8;
     }
-    static_assert(kStages >= 4, "pipeline depth");
+    static_assert(kStages >= (BM == 128 ? 4 : 3), "pipeline depth");
     static_assert(BN % 32 == 0 && BN >= 64 && BN <= 256, "N tile");
-    static_assert(kAcc * BN + kSfCols <= 512, "TMEM columns");
+    static_assert(BM == 128 || BM == 256, "M tile");
+    static_assert(kAcc * kAccCols + kSfCols <= 512, "TMEM columns");
 };
 
 struct MxArgs {
@@ -721,12 +749,22 @@ __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t
                  : "memory");
 }
 
-template <int BN, bool FP4, bool GLU = false>
+// 128-row halves of a row tile that hold rows of the expert: a 256-row tile
+// whose upper half would hold none is loaded, multiplied and stored as a
+// 128-row tile (no more MMA work than 128-row tiles at the expert's end)
+template <int HA>
+__device__ __forceinline__ int tile_halves(int64_t cnt, int m0) {
+    return (HA > 1 && cnt - m0 > 128) ? 2 : 1;
+}
+
+template <int BN, bool FP4, bool GLU = false, int BM = kGemmBM>
 __global__ void __launch_bounds__(kMxThreads, 1)
     expert_gemm_mx_kernel(const __grid_constant__ CUtensorMap tm_a,
                           const __grid_constant__ CUtensorMap tm_b, MxArgs a) {
-    using C = MxCfg<BN, FP4>;
+    using C = MxCfg<BN, FP4, BM>;
     static_assert(!GLU || (!FP4 && BN % 64 == 0), "GLU: MXFP8, whole 32-blocks per half tile");
+    static_assert(!GLU || BM == 128, "GLU: 128-row tiles");
+    constexpr int HA = C::kChunksA;  // 128-row halves of a row tile (one M = 128 MMA each)
     constexpr int TN = GLU ? BN / 2 : BN;  // output columns a tile advances by
     constexpr int S = C::kStages;
     extern __shared__ uint8_t gsm_raw[];
@@ -766,7 +804,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     pdl_enter();
-    if (warp == 0) tile_prefix(prefix, E, a.cnt, a.ntn, lane);
+    if (warp == 0) tile_prefix(prefix, E, a.cnt, a.ntn, lane, BM);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -779,8 +817,9 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         int it = 0;
         for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x) {
             int e, m0, n0;
-            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN);
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN, BM);
             const int arow = (int)a.eo[e] + m0, brow = e * a.N + n0;
+            const int halves = tile_halves<HA>(a.cnt[e], m0);
             for (int kb = 0; kb < kblocks; kb++, it++) {
                 const int s = it % S, r = it / S;
                 if (!mbar_wait(smem_addr(&empty[s]), (r & 1) ^ 1)) {
@@ -789,8 +828,10 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                     break;
                 }
                 const uint32_t fb = smem_addr(&full[s]);
-                mbar_expect_tx(fb, C::kBytesA + C::kBytesB);
-                tma_load_2d(smem_addr(sA + s * C::kBytesA), &tm_a, kb * kMxBK, arow, fb);
+                mbar_expect_tx(fb, halves * 128 * kMxBK + C::kBytesB);
+                for (int h = 0; h < halves; h++)
+                    tma_load_2d(smem_addr(sA + s * C::kBytesA + h * 128 * kMxBK), &tm_a, kb * kMxBK,
+                                arow + 128 * h, fb);
                 if constexpr (GLU) {  // gate rows, then the same rows of the up projection
                     tma_load_2d(smem_addr(sB + s * C::kBytesB), &tm_b, kb * kMxBK, brow, fb);
                     tma_load_2d(smem_addr(sB + s * C::kBytesB + TN * kMxBK), &tm_b, kb * kMxBK,
@@ -807,7 +848,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
     } else if (warp == 1 && lane == 0) {
         // ---- scale copies and MMAs
         const uint32_t idesc = umma_idesc_mx(kGemmBM, BN, FP4);
-        const uint32_t tsfa = tmem_base + (uint32_t)C::kSfCol, tsfb = tsfa + 4 * C::kGroups;
+        const uint32_t tsfa = tmem_base + (uint32_t)C::kSfCol, tsfb = tsfa + 4 * C::kGroups * HA;
         int it = 0, tc = 0;
         for (int t = blockIdx.x; t < total && !*s_abort; t += gridDim.x, tc++) {
             const int acc = tc % C::kAcc, use = tc / C::kAcc;
@@ -817,7 +858,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 break;
             }
             tc_fence_after();
-            const uint32_t d = tmem_base + (uint32_t)(acc * BN);
+            const uint32_t d = tmem_base + (uint32_t)(acc * C::kAccCols);
+            int halves = 1;
+            if constexpr (HA > 1) {
+                int e, m0, n0;
+                gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN, BM);
+                halves = tile_halves<HA>(a.cnt[e], m0);
+            }
             bool ok = true;
             for (int kb = 0; kb < kblocks; kb++, it++) {
                 const int s = it % S, r = it / S;
@@ -828,17 +875,23 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 tc_fence_after();
                 const uint32_t sf = smem_addr(sSF + s * C::kSfBytes);
 #pragma unroll
-                for (int c = 0; c < C::kGroups * (1 + C::kChunksB); c++)  // A's, then B's
+                for (int c = 0; c < C::kGroups * C::kChunks; c++)  // A's, then B's
                     tmem_cp_32x128b_x4(tsfa + 4 * c, sf_desc(sf + 512 * c));
-                const uint64_t ad = umma_desc_sw128(smem_addr(sA + s * C::kBytesA));
                 const uint64_t bd = umma_desc_sw128(smem_addr(sB + s * C::kBytesB));
 #pragma unroll
                 for (int k = 0; k < 4; k++) {  // 32 bytes of codes = 2 units each
                     const int blk = k * C::kNsf, grp = blk / 4;
                     const uint32_t byte = (uint32_t)(blk % 4);
-                    umma_mx<FP4>(d, ad + 2 * k, bd + 2 * k, idesc | (byte << 29) | (byte << 4),
-                                 (tsfa + 4 * grp) | (byte << 30),
-                                 (tsfb + 4 * C::kChunksB * grp) | (byte << 30), (kb | k) != 0);
+#pragma unroll
+                    for (int h = 0; h < HA; h++) {  // the halves share the stage's B tile
+                        if (h >= halves) break;
+                        const uint64_t ad =
+                            umma_desc_sw128(smem_addr(sA + s * C::kBytesA + h * 128 * kMxBK));
+                        umma_mx<FP4>(d + h * BN, ad + 2 * k, bd + 2 * k,
+                                     idesc | (byte << 29) | (byte << 4),
+                                     (tsfa + 4 * (grp * HA + h)) | (byte << 30),
+                                     (tsfb + 4 * C::kChunksB * grp) | (byte << 30), (kb | k) != 0);
+                    }
                 }
                 umma_commit(smem_addr(&empty[s]));
             }
@@ -862,7 +915,7 @@ __global__ void __launch_bounds__(kMxThreads, 1)
         for (int t = blockIdx.x; t < total; t += gridDim.x) {
             if (__shfl_sync(kFull, (int)*s_abort, 0)) break;
             int e, m0, n0;
-            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN);
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN, BM);
             const int64_t arow0 = a.eo[e] + m0;
             const int64_t brow0 = (int64_t)e * a.N + n0;
             // weight row of B-tile row n (GLU: the up rows follow the gate rows)
@@ -873,13 +926,15 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             for (int kb0 = 0; kb0 < kblocks && ok; kb0 += G) {
                 const int g = min(G, kblocks - kb0);
                 constexpr int NG = C::kGroups;
-                uint32_t va[G][NG][4], vb[G][NG][C::kChunksB][4];
+                uint32_t va[G][NG][HA][4], vb[G][NG][C::kChunksB][4];
                 if (vec && g == G) {
                     // a row's scales of the G steps are G * NG contiguous words,
                     // 16-byte aligned: G * NG / 4 16-byte loads per row
 #pragma unroll
+                    for (int ha = 0; ha < HA; ha++)
+#pragma unroll
                     for (int j = 0; j < 4; j++) {
-                        const int64_t row = arow0 + lane + 32 * j;
+                        const int64_t row = arow0 + 128 * ha + lane + 32 * j;
 #pragma unroll
                         for (int h = 0; h < G * NG / 4; h++) {
                             const uint4 w4 = row < a.rows
@@ -888,7 +943,8 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                                                  : make_uint4(0u, 0u, 0u, 0u);
                             const uint32_t wv[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-                            for (int u = 0; u < 4; u++) va[(4 * h + u) / NG][(4 * h + u) % NG][j] = wv[u];
+                            for (int u = 0; u < 4; u++)
+                                va[(4 * h + u) / NG][(4 * h + u) % NG][ha][j] = wv[u];
                         }
                     }
 #pragma unroll
@@ -916,11 +972,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                     for (int gg = 0; gg < NG; gg++) {
                         const int off = (kb * NG + gg) * 4;  // the group's 4 scale bytes
 #pragma unroll
+                        for (int ha = 0; ha < HA; ha++)
+#pragma unroll
                         for (int j = 0; j < 4; j++) {
-                            const int64_t row = arow0 + lane + 32 * j;
-                            va[q][gg][j] = row < a.rows ? __ldg(reinterpret_cast<const uint32_t *>(
-                                                              a.xs + row * SB + off))
-                                                        : 0u;
+                            const int64_t row = arow0 + 128 * ha + lane + 32 * j;
+                            va[q][gg][ha][j] = row < a.rows ? __ldg(reinterpret_cast<const uint32_t *>(
+                                                                  a.xs + row * SB + off))
+                                                            : 0u;
                         }
 #pragma unroll
                         for (int c = 0; c < C::kChunksB; c++)
@@ -947,12 +1005,15 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                     const uint32_t st = smem_addr(sSF + s * C::kSfBytes) + lane * 16;
 #pragma unroll
                     for (int gg = 0; gg < NG; gg++) {
-                        st_shared_v4(st + 512 * gg, va[q][gg][0], va[q][gg][1], va[q][gg][2],
-                                     va[q][gg][3]);
+#pragma unroll
+                        for (int ha = 0; ha < HA; ha++)
+                            st_shared_v4(st + 512 * (gg * HA + ha), va[q][gg][ha][0],
+                                         va[q][gg][ha][1], va[q][gg][ha][2], va[q][gg][ha][3]);
 #pragma unroll
                         for (int c = 0; c < C::kChunksB; c++)
-                            st_shared_v4(st + 512 * (NG + gg * C::kChunksB + c), vb[q][gg][c][0],
-                                         vb[q][gg][c][1], vb[q][gg][c][2], vb[q][gg][c][3]);
+                            st_shared_v4(st + 512 * (NG * HA + gg * C::kChunksB + c),
+                                         vb[q][gg][c][0], vb[q][gg][c][1], vb[q][gg][c][2],
+                                         vb[q][gg][c][3]);
                     }
                     // the copies to TMEM read shared memory through the async proxy
                     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -986,11 +1047,13 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             }
             tc_fence_after();
             int e, m0, n0;
-            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN);
-            const int m = m0 + sub * 32 + lane;
+            gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN, BM);
+#pragma unroll 1
+            for (int ha = 0; ha < tile_halves<HA>(a.cnt[e], m0); ha++) {  // the tile's row halves
+            const int m = m0 + 128 * ha + sub * 32 + lane;
             const bool valid = m < a.cnt[e];
-            const uint32_t taddr =
-                tmem_base + ((uint32_t)(sub * 32) << 16) + (uint32_t)(acc * BN);
+            const uint32_t taddr = tmem_base + ((uint32_t)(sub * 32) << 16) +
+                                   (uint32_t)(acc * C::kAccCols + ha * BN);
             if constexpr (GLU) {
                 const int64_t row = a.eo[e] + m;
                 uint8_t *zrow = a.zc + row * (int64_t)a.I + n0;
@@ -1027,12 +1090,18 @@ __global__ void __launch_bounds__(kMxThreads, 1)
                 }
             } else {
                 uint16_t *yrow = a.y + (a.eo[e] + m) * (int64_t)a.N + n0;
+                static_assert(BN % 32 == 0, "32-column epilogue steps");
 #pragma unroll 1
-                for (int c = 0; c < BN / 16; c++) {
-                    uint32_t v[16];
-                    tmem_ld16(taddr + c * 16, v);
-                    if (valid) store_bf16x16(yrow + c * 16, v);
+                for (int c = 0; c < BN / 32; c++) {  // 32 columns a TMEM load
+                    uint32_t v[32];
+                    tmem_ld32(taddr + c * 32, v);
+                    if (valid) {
+                        store_bf16x16(yrow + c * 32, *reinterpret_cast<const uint32_t(*)[16]>(v));
+                        store_bf16x16(yrow + c * 32 + 16,
+                                      *reinterpret_cast<const uint32_t(*)[16]>(v + 16));
+                    }
                 }
+            }
             }
             tc_fence_before();
             mbar_arrive(smem_addr(&accempty[acc]));

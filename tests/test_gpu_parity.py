@@ -799,6 +799,31 @@ def test_expert_gemm_mxfp4_large_shape_sampled():
     _check_expert_gemm(r, y, w["H"], wc=wc, ws=ws, sample_rows=12)
 
 
+@pytest.mark.parametrize("mode,H", [("mxfp8", 1024), ("mxfp8", 640), ("mxfp4", 1024),
+                                    ("mxfp4", 768)])
+def test_expert_gemm_mx_tall_tiles(mode, H):
+    """About 490 rows an expert on average and N tiles of 224: 256-row tiles,
+    two M = 128 MMAs sharing each B tile (MXFP8 and MXFP4).  Expert sizes put
+    tile ends on and around the 128-row half (129: one row in the upper half;
+    556, 555: a last tile whose upper half holds nothing; 384, 640: exactly a
+    half tile more), an empty expert, and H with and without whole groups of
+    scale loads."""
+    counts = np.array([1200, 556, 129, 0, 384, 640, 555, 440])
+    w = synth.workload("tiny", R=2, T=int(counts.sum()) // 2, M=int(counts.sum()) // 2, K=1,
+                       E=8, H=H)
+    idx = np.repeat(np.arange(8), counts)[np.random.default_rng(5).permutation(counts.sum())]
+    idx = idx.reshape(-1, 1).astype(np.int64)
+    wts = np.ones_like(idx, dtype=np.float32)
+    r = Run(w, mode, layout="packed", idx=idx, wts=wts)
+    assert np.array_equal(r.lay["recv_count"], counts)
+    wc, ws = _seeded_mx_weights(w["E"], 448, H, seed=H + len(mode), fp4=mode == "mxfp4")
+    y = _sentinel_y(r, 448)
+    ep.ep_expert_gemm_mx(r.cfg, r.b.recv_buf, r.b.expert_offset, r.b.recv_count, wc, ws, y,
+                         r.b.dev_status)
+    assert ep.ep_get_status(r.b.dev_status) == 0
+    _check_expert_gemm(r, y, 448, wc=wc, ws=ws, sample_rows=400)
+
+
 def test_expert_gemm_empty_batch_launches_nothing():
     w = synth.workload("tiny", R=2, T=0, M=16, K=2, E=4, H=256)
     for mode in ("bf16", "mxfp8"):
