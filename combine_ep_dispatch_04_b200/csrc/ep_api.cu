@@ -1173,13 +1173,21 @@ ep_status_t run_ffn(const Plan &p, int I, const void *recv_buf, const int64_t *e
     uint8_t *zc = static_cast<uint8_t *>(z_buf);
     uint8_t *zs = zc + ffn_z_scale_offset(p, I);
     const MxOperand x{recv_buf, static_cast<const uint8_t *>(recv_buf) + p.scale_off, p.H};
+    // GMM1 tiles: 256 columns (128 gate + 128 up, one accumulator) for experts of
+    // 256 rows and more; else 192 (96 + 96) where I allows, which keeps two
+    // accumulators (the SwiGLU epilogue overlaps the next tile's MMAs) with a
+    // quarter fewer operand bytes per FLOP than 128-column tiles
     const bool wide = p.N * p.K / p.E >= 256 && I % 128 == 0;
-    ep_status_t st = wide ? launch_gemm_mx<256, false, true>(p, x, expert_offset, recv_count, w1c,
-                                                            w1s, 2 * I, nullptr, zc, zs,
-                                                            dev_status, s, 13)
-                          : launch_gemm_mx<128, false, true>(p, x, expert_offset, recv_count, w1c,
-                                                            w1s, 2 * I, nullptr, zc, zs,
-                                                            dev_status, s, 14);
+    ep_status_t st;
+    if (wide)
+        st = launch_gemm_mx<256, false, true>(p, x, expert_offset, recv_count, w1c, w1s, 2 * I,
+                                              nullptr, zc, zs, dev_status, s, 13);
+    else if (I % 96 == 0)
+        st = launch_gemm_mx<192, false, true>(p, x, expert_offset, recv_count, w1c, w1s, 2 * I,
+                                              nullptr, zc, zs, dev_status, s, 17);
+    else
+        st = launch_gemm_mx<128, false, true>(p, x, expert_offset, recv_count, w1c, w1s, 2 * I,
+                                              nullptr, zc, zs, dev_status, s, 14);
     if (st != EP_OK) return st;
     const MxOperand z{zc, zs, I};
     ep_config_t c2 = {};

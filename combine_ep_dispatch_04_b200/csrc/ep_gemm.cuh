@@ -114,7 +114,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
                  : "memory");
 }
 
-// 16 fp32 accumulator columns of one row -> 16 bf16 (round to nearest even)
 // 32 consecutive fp32 columns of this warp's 32 TMEM lanes, one wait
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
     asm volatile(
@@ -139,6 +138,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
                  : "memory");
 }
 
+// 16 fp32 accumulator columns of one row -> 16 bf16 (round to nearest even)
 __device__ __forceinline__ void store_bf16x16(uint16_t *dst, const uint32_t (&v)[16]) {
     uint4 lo, hi;
     lo.x = pack_bf16x2(__uint_as_float(v[0]), __uint_as_float(v[1]));
@@ -1050,58 +1050,60 @@ __global__ void __launch_bounds__(kMxThreads, 1)
             gemm_tile(prefix, E, a.ntn, t, e, m0, n0, TN, BM);
 #pragma unroll 1
             for (int ha = 0; ha < tile_halves<HA>(a.cnt[e], m0); ha++) {  // the tile's row halves
-            const int m = m0 + 128 * ha + sub * 32 + lane;
-            const bool valid = m < a.cnt[e];
-            const uint32_t taddr = tmem_base + ((uint32_t)(sub * 32) << 16) +
-                                   (uint32_t)(acc * C::kAccCols + ha * BN);
-            if constexpr (GLU) {
-                const int64_t row = a.eo[e] + m;
-                uint8_t *zrow = a.zc + row * (int64_t)a.I + n0;
-                uint8_t *zsrow = a.zs + row * (int64_t)(a.I / 32) + n0 / 32;
+                const int m = m0 + 128 * ha + sub * 32 + lane;
+                const bool valid = m < a.cnt[e];
+                const uint32_t taddr = tmem_base + ((uint32_t)(sub * 32) << 16) +
+                                       (uint32_t)(acc * C::kAccCols + ha * BN);
+                if constexpr (GLU) {
+                    const int64_t row = a.eo[e] + m;
+                    uint8_t *zrow = a.zc + row * (int64_t)a.I + n0;
+                    uint8_t *zsrow = a.zs + row * (int64_t)(a.I / 32) + n0 / 32;
 #pragma unroll 1
-                for (int c = 0; c < TN / 32; c++) {  // one MX block of 32 outputs
-                    uint32_t g0[16], g1[16], u0[16], u1[16];
-                    tmem_ld16(taddr + c * 32, g0);
-                    tmem_ld16(taddr + c * 32 + 16, g1);
-                    tmem_ld16(taddr + TN + c * 32, u0);
-                    tmem_ld16(taddr + TN + c * 32 + 16, u1);
-                    float z[32];
-                    float amax = 0.0f;
+                    for (int c = 0; c < TN / 32; c++) {  // one MX block of 32 outputs
+                        uint32_t g0[16], g1[16], u0[16], u1[16];
+                        tmem_ld16(taddr + c * 32, g0);
+                        tmem_ld16(taddr + c * 32 + 16, g1);
+                        tmem_ld16(taddr + TN + c * 32, u0);
+                        tmem_ld16(taddr + TN + c * 32 + 16, u1);
+                        float z[32];
+                        float amax = 0.0f;
 #pragma unroll
-                    for (int i = 0; i < 16; i++) {
-                        z[i] = swiglu(__uint_as_float(g0[i]), __uint_as_float(u0[i]));
-                        z[16 + i] = swiglu(__uint_as_float(g1[i]), __uint_as_float(u1[i]));
-                        amax = fmaxf(amax, fmaxf(fabsf(z[i]), fabsf(z[16 + i])));
+                        for (int i = 0; i < 16; i++) {
+                            z[i] = swiglu(__uint_as_float(g0[i]), __uint_as_float(u0[i]));
+                            z[16 + i] = swiglu(__uint_as_float(g1[i]), __uint_as_float(u1[i]));
+                            amax = fmaxf(amax, fmaxf(fabsf(z[i]), fabsf(z[16 + i])));
+                        }
+                        const int X = mx_exponent_fast<448>(amax);
+                        const float mult = exp2_neg(X);
+                        uint32_t w[8];
+#pragma unroll
+                        for (int q = 0; q < 8; q++)
+                            w[q] = cvt_e4m3x2(__fmul_rn(z[4 * q], mult),
+                                              __fmul_rn(z[4 * q + 1], mult)) |
+                                   (cvt_e4m3x2(__fmul_rn(z[4 * q + 2], mult),
+                                               __fmul_rn(z[4 * q + 3], mult))
+                                    << 16);
+                        if (valid) {
+                            st_v4(zrow + c * 32, make_uint4(w[0], w[1], w[2], w[3]));
+                            st_v4(zrow + c * 32 + 16, make_uint4(w[4], w[5], w[6], w[7]));
+                            zsrow[c] = (uint8_t)(X + 127);
+                        }
                     }
-                    const int X = mx_exponent_fast<448>(amax);
-                    const float mult = exp2_neg(X);
-                    uint32_t w[8];
-#pragma unroll
-                    for (int q = 0; q < 8; q++)
-                        w[q] = cvt_e4m3x2(__fmul_rn(z[4 * q], mult), __fmul_rn(z[4 * q + 1], mult)) |
-                               (cvt_e4m3x2(__fmul_rn(z[4 * q + 2], mult),
-                                           __fmul_rn(z[4 * q + 3], mult))
-                                << 16);
-                    if (valid) {
-                        st_v4(zrow + c * 32, make_uint4(w[0], w[1], w[2], w[3]));
-                        st_v4(zrow + c * 32 + 16, make_uint4(w[4], w[5], w[6], w[7]));
-                        zsrow[c] = (uint8_t)(X + 127);
+                } else {
+                    uint16_t *yrow = a.y + (a.eo[e] + m) * (int64_t)a.N + n0;
+                    static_assert(BN % 32 == 0, "32-column epilogue steps");
+#pragma unroll 1
+                    for (int c = 0; c < BN / 32; c++) {  // 32 columns a TMEM load
+                        uint32_t v[32];
+                        tmem_ld32(taddr + c * 32, v);
+                        if (valid) {
+                            store_bf16x16(yrow + c * 32,
+                                          *reinterpret_cast<const uint32_t(*)[16]>(v));
+                            store_bf16x16(yrow + c * 32 + 16,
+                                          *reinterpret_cast<const uint32_t(*)[16]>(v + 16));
+                        }
                     }
                 }
-            } else {
-                uint16_t *yrow = a.y + (a.eo[e] + m) * (int64_t)a.N + n0;
-                static_assert(BN % 32 == 0, "32-column epilogue steps");
-#pragma unroll 1
-                for (int c = 0; c < BN / 32; c++) {  // 32 columns a TMEM load
-                    uint32_t v[32];
-                    tmem_ld32(taddr + c * 32, v);
-                    if (valid) {
-                        store_bf16x16(yrow + c * 32, *reinterpret_cast<const uint32_t(*)[16]>(v));
-                        store_bf16x16(yrow + c * 32 + 16,
-                                      *reinterpret_cast<const uint32_t(*)[16]>(v + 16));
-                    }
-                }
-            }
             }
             tc_fence_before();
             mbar_arrive(smem_addr(&accempty[acc]));
