@@ -327,6 +327,29 @@ def test_combine_of_quantized_expert_outputs(mode, name, override):
     combine_quantized_check(r, seed=31 * len(mode) + len(name))
 
 
+@pytest.mark.parametrize("special_weights", [False, True])
+@pytest.mark.parametrize("mode", ["int8_token", "e4m3_b128", "mxfp8", "mxfp4"])
+def test_combine_of_quantized_pipelined_kernel(mode, special_weights):
+    """More than 2^20 granules a launch: the pipelined kernel (codes copied a
+    granule ahead into shared memory, scale rows staged once) rather than the
+    register kernel the smaller cases take.  Sampled tokens; random and special
+    rows; ordinary and special weights."""
+    from harness import combine_quantized_check, special_quantized_rows
+    T = 80 if mode == "mxfp4" else 40
+    w = synth.workload("large", T=T)
+    gran = 32 if mode == "mxfp4" else 16
+    assert w["R"] * T * (w["H"] // gran) > (1 << 20)
+    idx, wts = synth.make_routing(w)
+    if special_weights:
+        pick = np.float32([0.0, -0.0, 1e-45, 1e-39, 1e-30, 0.5, -2.0, 3e38, np.inf, -np.inf,
+                           np.nan, 7.0, 0.125])
+        wts = pick[np.random.default_rng(13).integers(0, len(pick), wts.shape)]
+    r = Run(w, mode, layout="packed", idx=idx, wts=wts)
+    sample = np.sort(np.random.default_rng(3).choice(w["R"] * T, 400, replace=False))
+    combine_quantized_check(r, tokens=sample, seed=41 + len(mode))
+    combine_quantized_check(r, tokens=sample, seed=43 + len(mode), rows_fn=special_quantized_rows)
+
+
 @pytest.mark.parametrize("mode", ["int8_token", "e4m3_b128", "mxfp8", "mxfp4"])
 def test_combine_of_quantized_special_values(mode):
     """NaN codes, zero / subnormal / huge / infinite / NaN / negative scales,
