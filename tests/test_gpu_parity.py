@@ -289,30 +289,88 @@ def test_layout_paths_bad_indices_and_duplicates(path):
     ("large", dict(T=40), ep.F_LAYOUT_SINGLE_CTA), ("prefill", dict(T=50), 0),
 ])
 def test_dispatch_with_layout_equals_separate_calls(mode, name, override, path):
-    """The one-call dispatch (whose kernel overlaps the layout) gives the
-    bytes of ep_dispatch_layout + ep_dispatch, and so the oracle's."""
+    """The one-call dispatch (whose kernel overlaps the layout) gives the bytes
+    of ep_dispatch_layout + ep_dispatch, and so the oracle's."""
     w = synth.workload(name, **override)
     r = Run(w, mode, layout=w["layout"], flags=path, stats=True)
     r.check_layout()
-    b = ep.Buffers(r.cfg, recv_weights=True, expert_out=False)
+    _check_one_call(r, w)
+
+
+def _check_one_call(r, w, cfg=None):
+    """ep_dispatch_with_layout on r's inputs (r.cfg unless cfg is given) against
+    r's separate calls, every output byte for byte, the device status and a
+    cumulative_recv_stats accumulated twice."""
+    cfg = cfg or r.cfg
+    b = ep.Buffers(cfg, recv_weights=True, expert_out=False)
     b.recv_buf.fill_(0xAB)
     b.src_info.fill_(-7)
     b.recv_weights.fill_(float("nan"))
-    stats = torch.zeros(w["E"], dtype=torch.int64, device="cuda")
-    ep.ep_dispatch_with_layout(r.cfg, r.x_d, r.idx_d, b.token_slot, b.recv_count, b.workspace,
-                               b.recv_buf, b.src_info, b.dev_status, topk_weights=r.wts_d,
-                               tokens_per_rank=b.tokens_per_rank,
-                               tokens_per_expert=b.tokens_per_expert,
-                               is_token_in_rank=b.is_token_in_rank, expert_offset=b.expert_offset,
-                               cumulative_recv_stats=stats, recv_weights=b.recv_weights)
-    assert ep.ep_get_status(b.dev_status) == r.status
+    b.is_token_in_rank.fill_(7)
+    b.tokens_per_rank.fill_(-3)
+    b.tokens_per_expert.fill_(-3)
+    stats = torch.full((w["E"],), 5, dtype=torch.int64, device="cuda")
+    for _ in range(2):
+        b.token_slot.fill_(-5)
+        b.recv_count.fill_(-5)
+        ep.ep_dispatch_with_layout(cfg, r.x_d, r.idx_d, b.token_slot, b.recv_count, b.workspace,
+                                   b.recv_buf, b.src_info, b.dev_status, topk_weights=r.wts_d,
+                                   tokens_per_rank=b.tokens_per_rank,
+                                   tokens_per_expert=b.tokens_per_expert,
+                                   is_token_in_rank=b.is_token_in_rank,
+                                   expert_offset=b.expert_offset, cumulative_recv_stats=stats,
+                                   recv_weights=b.recv_weights)
+        assert ep.ep_get_status(b.dev_status) == r.status
     for name_ in ("token_slot", "recv_count", "tokens_per_rank", "tokens_per_expert",
                   "is_token_in_rank", "recv_buf", "src_info"):
         assert torch.equal(getattr(b, name_), getattr(r.b, name_)), name_
     assert torch.equal(b.recv_weights.nan_to_num(-1), r.b.recv_weights.nan_to_num(-1))
     if b.expert_offset is not None:
         assert torch.equal(b.expert_offset, r.b.expert_offset)
-    assert torch.equal(stats, r.stats_d)
+    if r.stats_d is not None:
+        assert torch.equal(stats, 5 + 2 * r.stats_d)
+
+
+@pytest.mark.parametrize("mode", ["bf16", "int8_token", "e4m3_b128", "mxfp8", "mxfp4"])
+@pytest.mark.parametrize("case", ["dup_bad_masked", "capacity", "idx_i32", "k1_r1", "wide_e"])
+def test_dispatch_with_layout_edges(mode, case):
+    """The one-call layout + dispatch on edge routings, against the separate
+    calls through a forced layout kernel and the oracle: duplicates within a
+    token, out-of-range and negative indices, masked entries; slots past the
+    capacity; int32 topk_idx; K = 1 on one rank; E = 1024 on 2 ranks."""
+    flags, path = 0, ep.F_LAYOUT_SINGLE_CTA
+    if case == "dup_bad_masked":
+        w = _edge(R=4, T=37, M=40, K=5, E=8, H=2048)
+        idx, wts = synth.make_routing(w)
+        idx[::3, 1] = idx[::3, 0]
+        idx[5, 2] = w["E"] + 3
+        idx[7, 0] = -9
+        idx[11, :] = -1
+    elif case == "capacity":
+        w = _edge(R=2, T=64, M=64, K=4, E=4, H=2048)
+        idx = np.zeros((128, 4), np.int64)
+        idx[:, 1:] = np.random.default_rng(2).integers(0, 4, (128, 3))
+        wts = np.ones_like(idx, dtype=np.float32)
+    elif case == "idx_i32":
+        w = _edge(R=8, T=64, M=64, K=8, E=64, H=4096)
+        idx, wts = synth.make_routing(w)
+        flags = ep.F_IDX_I32
+    elif case == "k1_r1":
+        w = _edge(R=1, T=200, M=200, K=1, E=4, H=2048)
+        idx, wts = synth.make_routing(w)
+    else:
+        w = _edge(R=2, T=100, M=100, K=8, E=1024, H=2048)
+        idx, wts = synth.make_routing(w)
+    r = Run(w, mode, layout="padded", idx=idx, wts=wts, flags=flags | path, stats=True)
+    r.check_layout()
+    r.check_dispatch()
+    if case == "dup_bad_masked":
+        assert r.status & ep.DEV_BAD_INDEX
+    if case == "capacity":
+        assert r.status & ep.DEV_CAPACITY_OVERFLOW
+    cfg = ep.make_config(w["R"], w["T"], w["M"], w["K"], w["E"], w["H"], mode, "padded",
+                         flags=flags)
+    _check_one_call(r, w, cfg)
 
 
 @pytest.mark.parametrize("mode", ["int8_token", "e4m3_b128", "mxfp8", "mxfp4"])
