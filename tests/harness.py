@@ -336,6 +336,48 @@ def special_quantized_rows(mode, H, nrows, seed):
     return data, scale.reshape(nrows, S)
 
 
+def combine_dispatched_check(run, tokens):
+    """The combine of the dispatched rows themselves read as quantised expert
+    outputs (the benchmark's quantised-combine launch), on the given tokens:
+    within 1 bf16 ulp of the oracle, NaN exactly where the oracle gives NaN."""
+    w, b = run.w, run.b
+    K, H = w["K"], w["H"]
+    cfg = ep.make_config(w["R"], w["T"], w["M"], K, w["E"], H, run.mode, run.layout, run.align,
+                         run.qmax, run.cfg.flags | ep.F_COMBINE_QUANTIZED)
+    out = run.guards.alloc((w["N"], H), torch.bfloat16, "out (combine of dispatched rows)")
+    out.fill_(1.0)
+    ep.ep_combine(cfg, b.recv_buf, run.idx_d, run.wts_d, b.token_slot, out, b.dev_status,
+                  expert_offset=b.expert_offset)
+    assert ep.ep_get_status(b.dev_status) == run.status
+    run.guards.check()
+    tokens = np.asarray(tokens)
+    ns, ks, rows = run.entries(tokens)
+    sz = run.sizes
+    D, S = sz["data_row_bytes"], sz["scale_row_bytes"]
+    rows_d = torch.from_numpy(np.ascontiguousarray(rows, np.int64)).cuda()
+    data = b.recv_buf[: sz["rows"] * D].view(sz["rows"], D).index_select(0, rows_d).cpu().numpy()
+    a = sz["recv_scale_offset"]
+    scale = b.recv_buf[a: a + sz["rows"] * S].view(sz["rows"], S).index_select(0, rows_d) \
+        .cpu().numpy() if S else np.zeros((len(rows), 0), np.uint8)
+    where = {(int(n), int(k)): i for i, (n, k) in enumerate(zip(ns, ks))}
+    qd = np.zeros((len(tokens), K, D), np.uint8)
+    qs = np.zeros((len(tokens), K, S), np.uint8)
+    valid = np.zeros((len(tokens), K), np.uint8)
+    for j, n in enumerate(tokens):
+        for k in range(K):
+            i = where.get((int(n), k))
+            if i is not None:
+                qd[j, k], qs[j, k], valid[j, k] = data[i], scale[i], 1
+    want = oracle.combine_gathered_q(run.omode, qd, qs, run.wts[tokens], valid, H)
+    got = to_np_u16(out)[tokens]
+    nan_g = (got & 0x7FFF) > 0x7F80
+    nan_w = (want & 0x7FFF) > 0x7F80
+    assert np.array_equal(nan_g, nan_w), int((nan_g != nan_w).sum())
+    d = np.where(nan_w, 0, ulp_distance(got, want))
+    assert d.max() <= 1, int(d.max())
+    return int(d.max())
+
+
 def combine_quantized_check(run, tokens=None, seed=0, rows_fn=None):
     """Combine of quantised expert outputs on the GPU against the oracle:
     within 1 bf16 ulp, and NaN exactly where the oracle gives NaN."""

@@ -66,6 +66,9 @@ def test_large_workload_full_size():
     r.check_dispatch()
     sample = np.random.default_rng(5).choice(w["N"], 2048, replace=False)
     r.check_combine(tokens=np.sort(sample))
+    # the benchmark's quantised combine (pipelined kernel) of the dispatched MXFP4 rows
+    from harness import combine_dispatched_check
+    combine_dispatched_check(r, np.sort(sample[:600]))
 
 
 def test_prefill_workload_full_size_sampled():
@@ -81,6 +84,9 @@ def test_prefill_workload_full_size_sampled():
     r.check_dispatch(tokens=sample)
     r.check_combine(tokens=sample)
     r.check_backward(tokens=sample[:300])
+    # the benchmark's quantised combine (pipelined kernel) of the dispatched MXFP8 rows
+    from harness import combine_dispatched_check
+    combine_dispatched_check(r, sample[::3])
 
 
 # ---------------------------------------------------------------------------
