@@ -336,6 +336,31 @@ def special_quantized_rows(mode, H, nrows, seed):
     return data, scale.reshape(nrows, S)
 
 
+def _quantized_combine_matches(run, out, tokens, ns, ks, data, scale):
+    """The GPU combine `out` of quantised rows (data / scale of entry i = (ns[i],
+    ks[i])) against the oracle on `tokens`: within 1 bf16 ulp, NaN exactly where
+    the oracle gives NaN.  Returns the largest distance."""
+    K, H = run.w["K"], run.w["H"]
+    D, S = data.shape[1], scale.shape[1]
+    where = {(int(n), int(k)): i for i, (n, k) in enumerate(zip(ns, ks))}
+    qd = np.zeros((len(tokens), K, D), np.uint8)
+    qs = np.zeros((len(tokens), K, S), np.uint8)
+    valid = np.zeros((len(tokens), K), np.uint8)
+    for j, n in enumerate(tokens):
+        for k in range(K):
+            i = where.get((int(n), k))
+            if i is not None:
+                qd[j, k], qs[j, k], valid[j, k] = data[i], scale[i], 1
+    want = oracle.combine_gathered_q(run.omode, qd, qs, run.wts[tokens], valid, H)
+    got = to_np_u16(out)[tokens]
+    nan_g = (got & 0x7FFF) > 0x7F80
+    nan_w = (want & 0x7FFF) > 0x7F80
+    assert np.array_equal(nan_g, nan_w), int((nan_g != nan_w).sum())
+    d = np.where(nan_w, 0, ulp_distance(got, want))
+    assert d.max() <= 1, int(d.max())
+    return int(d.max())
+
+
 def combine_dispatched_check(run, tokens):
     """The combine of the dispatched rows themselves read as quantised expert
     outputs (the benchmark's quantised-combine launch), on the given tokens:
@@ -359,23 +384,7 @@ def combine_dispatched_check(run, tokens):
     a = sz["recv_scale_offset"]
     scale = b.recv_buf[a: a + sz["rows"] * S].view(sz["rows"], S).index_select(0, rows_d) \
         .cpu().numpy() if S else np.zeros((len(rows), 0), np.uint8)
-    where = {(int(n), int(k)): i for i, (n, k) in enumerate(zip(ns, ks))}
-    qd = np.zeros((len(tokens), K, D), np.uint8)
-    qs = np.zeros((len(tokens), K, S), np.uint8)
-    valid = np.zeros((len(tokens), K), np.uint8)
-    for j, n in enumerate(tokens):
-        for k in range(K):
-            i = where.get((int(n), k))
-            if i is not None:
-                qd[j, k], qs[j, k], valid[j, k] = data[i], scale[i], 1
-    want = oracle.combine_gathered_q(run.omode, qd, qs, run.wts[tokens], valid, H)
-    got = to_np_u16(out)[tokens]
-    nan_g = (got & 0x7FFF) > 0x7F80
-    nan_w = (want & 0x7FFF) > 0x7F80
-    assert np.array_equal(nan_g, nan_w), int((nan_g != nan_w).sum())
-    d = np.where(nan_w, 0, ulp_distance(got, want))
-    assert d.max() <= 1, int(d.max())
-    return int(d.max())
+    return _quantized_combine_matches(run, out, tokens, ns, ks, data, scale)
 
 
 def combine_quantized_check(run, tokens=None, seed=0, rows_fn=None):
@@ -403,20 +412,4 @@ def combine_quantized_check(run, tokens=None, seed=0, rows_fn=None):
     assert ep.ep_get_status(b.dev_status) == run.status
     run.guards.check()
     tokens = np.arange(w["N"]) if tokens is None else np.asarray(tokens)
-    got = to_np_u16(out)[tokens]
-    where = {(int(n), int(k)): i for i, (n, k) in enumerate(zip(ns, ks))}
-    qd = np.zeros((len(tokens), K, D), np.uint8)
-    qs = np.zeros((len(tokens), K, S), np.uint8)
-    valid = np.zeros((len(tokens), K), np.uint8)
-    for j, n in enumerate(tokens):
-        for k in range(K):
-            i = where.get((int(n), k))
-            if i is not None:
-                qd[j, k], qs[j, k], valid[j, k] = data[i], scale[i], 1
-    want = oracle.combine_gathered_q(mode, qd, qs, run.wts[tokens], valid, H)
-    nan_g = (got & 0x7FFF) > 0x7F80
-    nan_w = (want & 0x7FFF) > 0x7F80
-    assert np.array_equal(nan_g, nan_w), int((nan_g != nan_w).sum())
-    d = np.where(nan_w, 0, ulp_distance(got, want))
-    assert d.max() <= 1, int(d.max())
-    return int(d.max())
+    return _quantized_combine_matches(run, out, tokens, ns, ks, data, scale)
